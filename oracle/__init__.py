@@ -1,0 +1,254 @@
+"""CPU oracle for the SegQuant DualScale / SegLinear quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the benchmark's CPU-baseline leg may import this package.  The product path
+(``post_quantized_linear_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``segquant_oracle.c`` (plain C, compiled with
+``-O2 -ffp-contract=off -fopenmp``); this module compiles it on demand and
+exposes numpy-level wrappers.  Each wrapper follows the function of the same
+name in the C file, whose comments cite the passage of the SegQuant summaries
+("SegQuant: A Semantics-Aware and Generalizable Quantization Framework for
+Diffusion Models", Spanish technical summary sections 2.A SegLinear and 2.B
+DualScale; Korean technical summary section 2) that it restates.
+
+Every function is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` (exact-rational brute force, closed forms and
+invariants); none is marked "parity unpinned" except agreement with the
+paper's own kernel outputs, which the pages do not print.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "segquant_oracle.c")
+_OUT_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_OUT_DIR, "libsegquant_oracle.so")
+_lib = None
+
+OK, ERR_ARG, ERR_RANGE = 0, 1, 4
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle's C source into a shared library (idempotent)."""
+    os.makedirs(_OUT_DIR, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I64, I32, INT = ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+        lib.sqo_calibrate.argtypes = [P, INT, I64, I64, I64, I32, P, P, P]
+        lib.sqo_quantize_activations.argtypes = [P, INT, I64, I64, I64, I32, P, P, P, P, P]
+        lib.sqo_quantize_weights_w8.argtypes = [P, I64, I64, I64, I32, P, P, P]
+        lib.sqo_quantize_weights_w4.argtypes = [P, I64, I64, I64, I32, P, P]
+        lib.sqo_unpack_w4.argtypes = [P, I64, I64, P]
+        lib.sqo_unpack_w4.restype = None
+        lib.sqo_accumulate.argtypes = [P, P, I64, I64, P, I64, I32, P, P]
+        lib.sqo_epilogue.argtypes = [P, I64, I64, I32, P, P, P, P, P, P, INT, I64]
+        lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.sqo_f32_to_bf16.restype = ctypes.c_uint16
+        lib.sqo_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.sqo_f32_to_f16.restype = ctypes.c_uint16
+        lib.sqo_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.sqo_f16_to_f32.restype = ctypes.c_float
+        for f in ("sqo_calibrate", "sqo_quantize_activations", "sqo_quantize_weights_w8",
+                  "sqo_quantize_weights_w4", "sqo_accumulate", "sqo_epilogue"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _x_dtype(x: np.ndarray) -> int:
+    """0 = fp32 values, 1 = bf16 stored as uint16 bit patterns."""
+    if x.dtype == np.float32:
+        return 0
+    if x.dtype == np.uint16:
+        return 1
+    raise TypeError("activations must be float32 or bf16 bit patterns (uint16)")
+
+
+def _bounds(b: Sequence[int]) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(b, dtype=np.int32))
+
+
+class OracleError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned status {code}")
+        self.code = code
+
+
+def _check(fn: str, code: int, allow_range: bool = False):
+    if code != OK and not (allow_range and code == ERR_RANGE):
+        raise OracleError(fn, code)
+    return code
+
+
+def calibrate(x: np.ndarray, kbounds: Sequence[int]):
+    """Static per-segment DualScale scales (s+, s-), each of shape [J]."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    kb = _bounds(kbounds)
+    J = len(kb) - 1
+    sp = np.zeros(J, np.float32)
+    sn = np.zeros(J, np.float32)
+    _check("sqo_calibrate", _load().sqo_calibrate(_ptr(x), _x_dtype(x), rows, K, K, J, _ptr(kb),
+                                                  _ptr(sp), _ptr(sn)))
+    return sp, sn
+
+
+def quantize_activations(x: np.ndarray, kbounds, s_pos, s_neg):
+    """DualScale codes (q+, q-), each int8 [M, K]."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    kb = _bounds(kbounds)
+    J = len(kb) - 1
+    sp = np.ascontiguousarray(np.asarray(s_pos, np.float32))
+    sn = np.ascontiguousarray(np.asarray(s_neg, np.float32))
+    qp = np.zeros((M, K), np.int8)
+    qn = np.zeros((M, K), np.int8)
+    _check("sqo_quantize_activations",
+           _load().sqo_quantize_activations(_ptr(x), _x_dtype(x), M, K, K, J, _ptr(kb), _ptr(sp),
+                                            _ptr(sn), _ptr(qp), _ptr(qn)))
+    return qp, qn
+
+
+def quantize_weights_w8(w: np.ndarray, kbounds):
+    """Per-(channel, K-segment) int8 codes [N, K] and fp32 scales [J, N]."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    kb = _bounds(kbounds)
+    J = len(kb) - 1
+    codes = np.zeros((N, K), np.int8)
+    scales = np.zeros((J, N), np.float32)
+    _check("sqo_quantize_weights_w8",
+           _load().sqo_quantize_weights_w8(_ptr(w), N, K, K, J, _ptr(kb), _ptr(codes), _ptr(scales)))
+    return codes, scales
+
+
+def quantize_weights_w4(w: np.ndarray, group: int = 128):
+    """Packed int4 codes [N, K/2] (low nibble = even k) and fp16 scales [N, K/group]."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    packed = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, K // group), np.uint16)
+    _check("sqo_quantize_weights_w4",
+           _load().sqo_quantize_weights_w4(_ptr(w), N, K, K, group, _ptr(packed), _ptr(scales)))
+    return packed, scales.view(np.float16)
+
+
+def unpack_w4(packed: np.ndarray, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    codes = np.zeros((N, K), np.int8)
+    _load().sqo_unpack_w4(_ptr(packed), N, K, _ptr(codes))
+    return codes
+
+
+def units_of(bits: int, K: int, kbounds: Sequence[int]):
+    """Unit bounds and the K segment of each unit.
+
+    int8 weights: one unit per K segment.  int4 weights: one unit per 128-wide
+    K group (groups never straddle a segment bound, bounds being multiples of
+    128)."""
+    kb = list(kbounds)
+    if bits == 8:
+        ub = kb
+        seg = list(range(len(kb) - 1))
+    else:
+        ub = list(range(0, K + 1, 128))
+        seg = []
+        for u in range(len(ub) - 1):
+            j = max(i for i in range(len(kb) - 1) if kb[i] <= ub[u])
+            seg.append(j)
+    return np.asarray(ub, np.int32), np.asarray(seg, np.int32)
+
+
+def accumulate(q_pos, q_neg, wcodes, ubounds) -> np.ndarray:
+    """Per-unit int32 accumulators acc[u, polarity, m, n] (polarity 0 = +)."""
+    q_pos = np.ascontiguousarray(q_pos, np.int8)
+    q_neg = np.ascontiguousarray(q_neg, np.int8)
+    wcodes = np.ascontiguousarray(wcodes, np.int8)
+    M, K = q_pos.shape
+    N = wcodes.shape[0]
+    ub = _bounds(ubounds)
+    U = len(ub) - 1
+    acc = np.zeros((U, 2, M, N), np.int32)
+    _check("sqo_accumulate", _load().sqo_accumulate(_ptr(q_pos), _ptr(q_neg), M, K, _ptr(wcodes), N,
+                                                    U, _ptr(ub), _ptr(acc)))
+    return acc
+
+
+def epilogue(acc, unit_seg, s_pos, s_neg, unit_scales, bias=None, out: str = "f32") -> np.ndarray:
+    """Fused DualScale epilogue.  unit_scales: [U, N] fp32.  out: 'f32' or 'bf16'
+    (bf16 is returned as uint16 bit patterns)."""
+    acc = np.ascontiguousarray(acc, np.int32)
+    U, _, M, N = acc.shape
+    us = np.ascontiguousarray(np.asarray(unit_seg, np.int32))
+    sp = np.ascontiguousarray(np.asarray(s_pos, np.float32))
+    sn = np.ascontiguousarray(np.asarray(s_neg, np.float32))
+    sw = np.ascontiguousarray(np.asarray(unit_scales, np.float32))
+    b = None if bias is None else np.ascontiguousarray(np.asarray(bias, np.float32))
+    if out == "f32":
+        y = np.zeros((M, N), np.float32)
+        od = 0
+    else:
+        y = np.zeros((M, N), np.uint16)
+        od = 1
+    _check("sqo_epilogue", _load().sqo_epilogue(_ptr(acc), M, N, U, _ptr(us), _ptr(sp), _ptr(sn),
+                                                _ptr(sw), _ptr(b), _ptr(y), od, N))
+    return y
+
+
+def unit_weight_scales(bits: int, scales: np.ndarray) -> np.ndarray:
+    """Weight scale of every unit as fp32 [U, N]: the [J, N] int8 scales as they
+    are, or the transposed, widened [N, G] fp16 group scales."""
+    if bits == 8:
+        return np.ascontiguousarray(scales, np.float32)
+    return np.ascontiguousarray(np.asarray(scales, np.float16).astype(np.float32).T)
+
+
+def linear_forward(x, kbounds, s_pos, s_neg, bits, wcodes, wscales, bias=None, out="f32",
+                   return_acc: bool = False):
+    """The whole forward pass: codes, per-unit accumulators, epilogue.
+
+    wcodes: int8 [N, K] (bits=8) or packed uint8 [N, K/2] (bits=4);
+    wscales: fp32 [J, N] (bits=8) or fp16 [N, K/128] (bits=4)."""
+    M, K = x.shape
+    qp, qn = quantize_activations(x, kbounds, s_pos, s_neg)
+    codes = wcodes if bits == 8 else unpack_w4(wcodes, K)
+    ub, useg = units_of(bits, K, kbounds)
+    acc = accumulate(qp, qn, codes, ub)
+    y = epilogue(acc, useg, s_pos, s_neg, unit_weight_scales(bits, wscales), bias, out)
+    if return_acc:
+        return y, acc, (qp, qn)
+    return y
+
+
+def f32_to_bf16_bits(v: float) -> int:
+    return int(_load().sqo_f32_to_bf16(float(v)))
+
+
+def f32_to_f16_bits(v: float) -> int:
+    return int(_load().sqo_f32_to_f16(float(v)))
