@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the DualScale / SegLinear quantized linear layer on B200.
+
+One step = one pass of the whole path over one batch: static calibration on
+the workload's calibration rows, weight quantization, and the fused forward
+(in-kernel DualScale quantization, two int8 tensor-core GEMMs, fused
+epilogue).  The metric counts the executed int8 work of the forward, 4*M*N*K
+ops (two GEMMs, one per polarity), per second of step time.
+
+Timing: W warm-up steps, then K timed steps on the device with CUDA events on
+the launching stream; a 256 MiB buffer is written between timed steps (outside
+the events) so that every step starts from a cold L2.  Under torchrun each rank
+runs its own batch (independent problems, no collective on the data path), the
+per-rank time is the max over ranks, and the value is the whole-job rate.
+
+`--impl reference` times the CPU oracle (the plain C implementation in
+oracle/) on the host cores, on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantized-linear int8 TOPS and % of B200 int8 tensor peak (GB/s at small M)"
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dit_xl2_fc2_cfg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]) * INT8_PER_BF16, float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS * INT8_PER_BF16, FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", "-i", str(self.gpu),
+               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 4:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        for p in self.rows:
+            try:
+                s = float(p[0]); m = float(p[1]); r = int(p[3], 16)
+            except ValueError:
+                continue
+            mx = m
+            if r & 0x1:  # idle sample
+                continue
+            sm.append(s)
+            for bit, name in REASON_BITS.items():
+                if r & bit:
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def cpu_oracle_step(wl, xn, wn, bn, rows):
+    """One oracle step on a row sample; returns (seconds, seconds scaled to the full batch)."""
+    import numpy as np
+    import oracle as O
+    t0 = time.perf_counter()
+    calib = xn if wl.calib_rows is None else xn[: wl.calib_rows]
+    sp, sn = O.calibrate(calib, wl.kseg)
+    t1 = time.perf_counter()
+    if wl.bits == 8:
+        wc, ws = O.quantize_weights_w8(wn, wl.kseg)
+    else:
+        wc, ws = O.quantize_weights_w4(wn)
+    t2 = time.perf_counter()
+    O.linear_forward(np.ascontiguousarray(xn[:rows]), wl.kseg, sp, sn, wl.bits, wc, ws, bn,
+                     out="f32" if wl.out == "f32" else "bf16")
+    t3 = time.perf_counter()
+    return t3 - t0, (t2 - t0) + (t3 - t2) * (wl.M / rows)
+
+
+def cpu_baseline(wl, x, w, b, target_s=12.0):
+    import numpy as np
+    import oracle as O
+    from synth import workloads as W
+    O.build()
+    xn, wn = W.to_numpy_x(x), w.numpy()
+    bn = None if b is None else b.numpy()
+    probe_rows = 8
+    t_probe, _ = cpu_oracle_step(wl, xn, wn, bn, probe_rows)
+    per_row = max(t_probe / probe_rows, 1e-6)
+    rows = int(max(8, min(wl.M, target_s / per_row)))
+    t, t_full = cpu_oracle_step(wl, xn, wn, bn, rows)
+    cores = len(os.sched_getaffinity(0))
+    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {
+        "value": wl.exec_ops / t_full / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+        "sample": (f"calibration on the full calibration rows, weight quantization of the full "
+                   f"[{wl.N},{wl.K}] weight, forward of {rows}/{wl.M} rows ({t:.1f} s); "
+                   "forward time scaled by M/rows"),
+    }
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from synth import workloads as W
+    import oracle as O
+    O.build()
+    wl = W.WORKLOADS[args.workload]
+    x, w, b = W.generate(wl)
+    xn, wn = W.to_numpy_x(x), w.numpy()
+    bn = None if b is None else b.numpy()
+    steps, warm = args.steps, args.warmup
+    budget_s = 150.0
+    t_probe, _ = cpu_oracle_step(wl, xn, wn, bn, 8)
+    per_row = max(t_probe / 8, 1e-6)
+    rows = int(max(8, min(wl.M, budget_s / (steps + warm) / per_row)))
+    for _ in range(warm):
+        cpu_oracle_step(wl, xn, wn, bn, rows)
+    full = []
+    raw = []
+    for _ in range(steps):
+        t, tf = cpu_oracle_step(wl, xn, wn, bn, rows)
+        raw.append(t)
+        full.append(tf)
+    t_step = sum(full) / len(full)
+    value = wl.exec_ops / t_step / 1e12
+    cores = len(os.sched_getaffinity(0))
+    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    sample = (f"each step: calibration on the calibration rows, full weight quantization, "
+              f"forward of {rows}/{wl.M} rows (mean {sum(raw)/len(raw):.2f} s); forward time "
+              "scaled by M/rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": steps, "warmup": warm, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": config_of(wl, "host cores, no L2 flush"),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, l2):
+    return {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "bits": wl.bits,
+            "x_dtype": wl.x_dtype, "out_dtype": wl.out, "k_segments": list(wl.kseg),
+            "n_segments": list(wl.nseg), "calib_rows": wl.calib_rows or wl.M,
+            "global_batch": wl.M, "l2": l2}
+
+
+# ------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import post_quantized_linear_b200 as pq
+    from synth import workloads as W
+
+    wl = W.WORKLOADS[args.workload]
+    import dataclasses
+    wl_rank = dataclasses.replace(wl, seed=wl.seed + rank)
+    x, w, b = W.generate(wl_rank)
+    dev = torch.device("cuda", local)
+    xd, wd = x.to(dev), w.to(dev)
+    bd = None if b is None else b.to(dev)
+    out_dtype = torch.float32 if wl.out == "f32" else torch.bfloat16
+    J = len(wl.kseg) - 1
+    sp = torch.empty(J, dtype=torch.float32, device=dev)
+    sn = torch.empty(J, dtype=torch.float32, device=dev)
+    qw = pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=wl.bits)
+    y = torch.empty((wl.M, wl.N), dtype=out_dtype, device=dev)
+    calib = xd if wl.calib_rows is None else xd[: wl.calib_rows]
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(xs=xd, ws=wd, ys=y, gemm_events=None):
+        pq.calibrate(calib if xs is xd else (xs if wl.calib_rows is None else xs[: wl.calib_rows]),
+                     wl.kseg, sp, sn)
+        pq.quantize_weights(ws, wl.kseg, wl.nseg, bits=wl.bits, out=qw)
+        if gemm_events:
+            gemm_events[0].record(stream)
+        pq.linear(xs, qw, sp, sn, bd, out=ys)
+        if gemm_events:
+            gemm_events[1].record(stream)
+
+    def events(n):
+        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n)]
+
+    launches_per_step = 3
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pq.stream_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    sampler = None if args.no_clocks else ClockSampler(local)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev, gev = events(args.steps), events(args.steps)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step(gemm_events=gev[i])
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [a.elapsed_time(bv) for a, bv in ev]
+    gemm_ms = [a.elapsed_time(bv) for a, bv in gev]
+    total_ms = sum(step_ms)
+
+    # forward alone, same protocol (cold L2 per call)
+    fev = events(args.steps)
+    for i in range(args.steps):
+        flush.fill_((i + 7) & 0xFF)
+        fev[i][0].record(stream)
+        pq.linear(xd, qw, sp, sn, bd, out=y)
+        fev[i][1].record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = [a.elapsed_time(bv) for a, bv in fev]
+    if pq.stream_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+
+    # end to end through the API: host inputs in, host result out, every step
+    e2e = None
+    if not args.no_e2e:
+        xh = x.pin_memory()
+        wh = w.pin_memory()
+        yh = torch.empty((wl.M, wl.N), dtype=out_dtype).pin_memory()
+        xdd = torch.empty_like(xd)
+        wdd = torch.empty_like(wd)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            xdd.copy_(xh, non_blocking=True)
+            wdd.copy_(wh, non_blocking=True)
+            step(xs=xdd, ws=wdd)
+            yh.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_total = e0.elapsed_time(e1)
+        bi = xh.numel() * xh.element_size() + wh.numel() * wh.element_size()
+        bo = yh.numel() * yh.element_size()
+        e2e = {"ms": e2e_total, "bi": bi, "bo": bo}
+
+    # max over ranks
+    vals = [total_ms, statistics.mean(gemm_ms), statistics.mean(fwd_ms),
+            e2e["ms"] if e2e else 0.0]
+    if world > 1:
+        t = torch.tensor(vals, dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        vals = t.tolist()
+    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms = vals
+
+    if rank == 0:
+        int8_peak_tops, hbm_peak, peak_kind = peaks()
+        ops = wl.exec_ops
+        value = world * args.steps * ops / (total_ms * 1e-3) / 1e12
+        gemm_tops = ops / (gemm_avg_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "config": config_of(wl, "flushed (256 MiB write between steps)"),
+            "roofline": {
+                "bound": "tensor", "kernel": "dualscale_gemm_kernel",
+                "achieved": gemm_tops, "peak": int8_peak_tops, "unit": "TOPS",
+                "frac": gemm_tops / int8_peak_tops, "traffic": None,
+                "peak_source": f"{peak_kind} bf16 burst x {INT8_PER_BF16:g} (nominal int8/bf16)",
+                "algorithmic_ops_per_launch": ops,
+                "algorithmic_bytes_per_launch": wl.alg_bytes(),
+                "achieved_gbs": wl.alg_bytes() / (gemm_avg_ms * 1e-3) / 1e9,
+                "avg_launch_us": gemm_avg_ms * 1e3,
+            },
+            "forward_only": {
+                "us": fwd_avg_ms * 1e3, "exec_tops": ops / (fwd_avg_ms * 1e-3) / 1e12,
+                "linear_equiv_tops": ops / 2 / (fwd_avg_ms * 1e-3) / 1e12,
+                "frac_int8_peak": ops / (fwd_avg_ms * 1e-3) / 1e12 / int8_peak_tops,
+            },
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if e2e:
+            line["e2e"] = {"value": world * args.steps * ops / (e2e_ms * 1e-3) / 1e12,
+                           "unit": "TOPS", "h2d_bytes_per_step": e2e["bi"],
+                           "d2h_bytes_per_step": e2e["bo"]}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, x, w, b)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,182 @@
+/*
+ * segquant.h -- C ABI of the B200 (sm_100a) DualScale / SegLinear quantized
+ * linear layer.
+ *
+ * What the layer computes comes from the SegQuant summaries ("SegQuant: A
+ * Semantics-Aware and Generalizable Quantization Framework for Diffusion
+ * Models", gist.science):
+ *   - DualScale (Spanish technical summary, section 2.B; Korean technical
+ *     summary, section 2 "DualScale"): the activation X is split into its
+ *     non-negative part X+ and its negative part X-, each quantized with its
+ *     own static scale (s+, s-); the two integer products X+^ W^ and X-^ W^ run
+ *     in one kernel and are combined in a fused epilogue.
+ *   - SegLinear (Spanish technical summary, section 2.A; Korean technical
+ *     summary, section 2 "SegLinear"): each input (K) segment of a linear
+ *     layer has its own activation scales and its own weight scales; output (N)
+ *     segments are quantized independently.
+ *   - Static calibration (Spanish technical summary, section 1 "compiler gap";
+ *     section 3 item 4): scales are fixed offline, no runtime-dynamic values.
+ *
+ * Numeric rules (every entry point follows them bit for bit):
+ *   s+_j = max(max(x,0))/127, s-_j = max(max(-x,0))/127 over segment j (fp32
+ *   division); r = 1/s in fp32 (0 when s = 0); a non-negative x (including
+ *   -0.0) takes q+ = clamp(round_half_even(x*r+), 0, 127) and q- = 0; a
+ *   negative x takes q- = clamp(round_half_even(x*r-), -127, 0) and q+ = 0,
+ *   where x*r is the exact product.  int8 weights: s_w[j][n] =
+ *   max_{k in seg j}|W[n,k]|/127, codes clamp(round_half_even(w/s), -127, 127).
+ *   int4 weights: group 128 along K, s = fp16_rne(max|W|/7), codes in [-7, 7],
+ *   two per byte, low nibble = even k.  Epilogue per output, for units u (a K
+ *   segment for int8 weights, a 128-wide group for int4 weights) in ascending
+ *   order: t = fmaf(s-_j, float(acc-_u), s+_j * float(acc+_u));
+ *   y = fmaf(sw_u[n], t, y) starting from y = 0; then y += bias[n]; then the
+ *   output conversion (fp32 as is, bf16 round-half-even).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller unless marked "host".
+ *     The library allocates no device memory and keeps no per-call state.
+ *   - Matrices are row-major.  X is [M, K] (tokens x in-features, the
+ *     nn.Linear input), W is [N, K] (the nn.Linear weight), Y is [M, N].
+ *     Leading dimensions are in elements.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  Arguments are validated on the host before any
+ *     launch; a rejected call enqueues nothing.
+ *   - Device-side conditions (a non-finite calibration maximum, an fp16 group
+ *     scale overflow, a bounded pipeline wait that expired) are recorded in a
+ *     per-device status word and returned by sq_stream_status().
+ *   - Inputs must be finite.  NaN activations, and an infinite activation whose
+ *     polarity has a zero scale, produce unspecified codes.
+ */
+#ifndef SEGQUANT_H_
+#define SEGQUANT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st* sq_stream_t;
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad dtype, inconsistent sizes */
+  SQ_ERR_ALIGNMENT = 2,   /* a pointer not 16-byte aligned or a row stride not a multiple of 16 bytes */
+  SQ_ERR_UNSUPPORTED = 3, /* segment bound not a multiple of 128, N % 16 != 0, bits/group combination */
+  SQ_ERR_RANGE = 4,       /* non-finite calibration maximum or weight, fp16 group scale overflow, size limit */
+  SQ_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
+  SQ_ERR_TIMEOUT = 6      /* a bounded device-side pipeline wait expired (reported by sq_stream_status) */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_BF16 = 1 } sq_dtype;
+
+/* Largest number of K segments per layer, and the largest K. */
+#define SQ_MAX_SEGMENTS 16
+#define SQ_MAX_K 131072
+
+/* Segment bounds, HOST memory: `count` segments, `count + 1` increasing bounds,
+ * bounds[0] = 0 and bounds[count] = the extent (K or N).  K-segment bounds other
+ * than the last must be multiples of 128. */
+typedef struct {
+  int32_t count;
+  const int32_t* bounds;
+} sq_segments;
+
+/* A quantized weight.  The struct itself is host memory; `codes` and
+ * `scales` are device buffers the caller allocates with the sizes returned by
+ * sq_qweight_sizes().
+ *   bits = 8, group = 0  : codes int8 [N][K]; scales fp32 [J][N] (J = kseg.count),
+ *                          one scale per (K segment, output channel).
+ *   bits = 4, group = 128: codes uint8 [N][K/2], low nibble = even k;
+ *                          scales binary16 [N][K/128], one per (channel, group).
+ * nseg (output segments, e.g. q | k | v) is validated and carried as metadata:
+ * per-channel weight scales make an output split a numerical no-op. */
+typedef struct {
+  int32_t bits;
+  int32_t group;
+  int64_t N;
+  int64_t K;
+  sq_segments kseg;
+  sq_segments nseg;
+  void* codes;
+  void* scales;
+} sq_qweight;
+
+/* Host only.  Byte sizes of the code and scale buffers of a quantized weight.
+ * Errors: SQ_ERR_INVALID_ARG for null outputs or non-positive sizes,
+ * SQ_ERR_UNSUPPORTED for a bits/group combination other than (8, 0), (4, 128)
+ * or K % 128 != 0 with bits = 4. */
+sq_status sq_qweight_sizes(int32_t bits, int64_t N, int64_t K, int32_t J, int32_t group,
+                           size_t* code_bytes, size_t* scale_bytes);
+
+/* Static DualScale calibration (SegQuant, Spanish technical summary 2.B and
+ * 1 "compiler gap"; Korean technical summary section 2 "DualScale").
+ * x: [rows, K] fp32 or bf16 with row stride ldx; the calibration rows.
+ * kseg: host K-segment bounds.  s_pos, s_neg: device fp32 [J] outputs,
+ * s+_j = max(x+)/127 and s-_j = max(|x-|)/127 over rows x segment j.
+ * A NaN input or an infinite maximum sets SQ_ERR_RANGE in the status word.
+ * rows = 0 gives zero scales.  Alignment: x 16-byte aligned, ldx*elt % 16 == 0. */
+sq_status sq_calibrate(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
+                       const sq_segments* kseg, float* s_pos, float* s_neg, sq_stream_t stream);
+
+/* Weight quantization (SegQuant SegLinear: Spanish technical summary 2.A,
+ * Korean technical summary section 2 "SegLinear"; int8 per channel and per K
+ * segment, or int4 with group 128 and fp16 scales).
+ * w: [N, K] fp32 or bf16 with row stride ldw.  `out` describes the
+ * destination (bits, group, N, K, kseg, nseg, codes, scales preset by the
+ * caller).  Non-finite weights or an fp16 scale overflow set SQ_ERR_RANGE in
+ * the status word.  Alignment: w 16-byte aligned, ldw*elt % 16 == 0; codes and
+ * scales 16-byte aligned. */
+sq_status sq_quantize_weights(const void* w, sq_dtype wt, int64_t N, int64_t K, int64_t ldw,
+                              const sq_qweight* out, sq_stream_t stream);
+
+/* The fused forward pass: DualScale quantization of X inside the GEMM, the two
+ * int8 tensor-core products per unit, the per-unit fold and the epilogue
+ * (SegQuant, Spanish technical summary 2.B "BatchedGEMM ... fused in the
+ * epilogue"; Korean technical summary section 2 "Fused Epilogue").
+ * x: [M, K] fp32 or bf16, row stride ldx.  w: quantized weight (K must match).
+ * s_pos, s_neg: device fp32 [J] activation scales.  bias: device fp32 [N] or
+ * NULL.  y: [M, N] fp32 or bf16, row stride ldy.  M = 0 is a no-op.
+ * Requirements: N % 16 == 0; K % 16 == 0 (K % 128 == 0 for int4 weights);
+ * K <= SQ_MAX_K; x, y, codes, scales 16-byte aligned; ldx*elt and ldy*elt
+ * multiples of 16 bytes. */
+sq_status sq_linear_forward(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                            const sq_qweight* w, const float* s_pos, const float* s_neg,
+                            const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                            sq_stream_t stream);
+
+/* Test / fallback surface: the DualScale codes alone (same rules as the
+ * forward's in-kernel quantization).  q_pos, q_neg: device int8 [M, K] with row
+ * stride ldq (a multiple of 16). */
+sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                  const sq_segments* kseg, const float* s_pos,
+                                  const float* s_neg, int8_t* q_pos, int8_t* q_neg, int64_t ldq,
+                                  sq_stream_t stream);
+
+/* Test surface: the same kernel as sq_linear_forward, but the epilogue writes
+ * the raw int32 accumulators of every unit instead of Y:
+ * acc[u][p][m][n], p = 0 for the (+) product, 1 for the (-) product; U units
+ * (K segments for int8 weights, K/128 groups for int4 weights); int32
+ * [U, 2, M, N] contiguous.  Intended for small shapes. */
+sq_status sq_linear_accumulators(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                 const sq_qweight* w, const float* s_pos, const float* s_neg,
+                                 int32_t* acc, sq_stream_t stream);
+
+/* Waits for `stream`, then returns and clears the device status word:
+ * SQ_ERR_TIMEOUT, SQ_ERR_RANGE, SQ_ERR_CUDA (a failed synchronize), or SQ_OK.
+ * The status word is per device and shared by all streams of the process. */
+sq_status sq_stream_status(sq_stream_t stream);
+
+/* Static string naming a status code. */
+const char* sq_status_string(sq_status status);
+
+/* Test hook: the device-side wait budget in clock cycles (default about one
+ * second).  0 restores the default.  Host only; affects later launches. */
+void sq_set_wait_budget(int64_t cycles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEGQUANT_H_ */

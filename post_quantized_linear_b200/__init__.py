@@ -1,0 +1,179 @@
+"""B200 (sm_100a) DualScale / SegLinear quantized linear layer.
+
+Python binding of the C ABI in ``include/segquant.h``: PyTorch supplies device
+memory and the current CUDA stream; every step of the layer runs in the
+library's CUDA kernels.  Function names follow the C entry points.
+
+SegQuant ("SegQuant: A Semantics-Aware and Generalizable Quantization
+Framework for Diffusion Models"): DualScale quantizes the non-negative and
+negative parts of each activation with separate static scales and fuses the
+two int8 products in one kernel's epilogue (Spanish technical summary 2.B;
+Korean technical summary section 2); SegLinear gives each input segment its
+own scales (Spanish technical summary 2.A).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import SegQuantError
+
+__all__ = ["QuantizedWeight", "SegQuantError", "calibrate", "quantize_weights", "linear",
+           "quantize_activations", "linear_accumulators", "stream_status", "qweight_sizes"]
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return _lib.SQ_F32
+    if t == torch.bfloat16:
+        return _lib.SQ_BF16
+    raise TypeError(f"unsupported dtype {t}: float32 or bfloat16")
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_2d(x: torch.Tensor, name: str):
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    if not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+@dataclasses.dataclass
+class QuantizedWeight:
+    """Device codes/scales of a quantized [N, K] weight plus its segment bounds."""
+    bits: int
+    N: int
+    K: int
+    kseg: Tuple[int, ...]
+    nseg: Tuple[int, ...]
+    codes: torch.Tensor    # int8 [N, K] or uint8 [N, K/2]
+    scales: torch.Tensor   # float32 [J, N] or float16 [N, K/128]
+
+    @property
+    def group(self) -> int:
+        return 0 if self.bits == 8 else 128
+
+    def c_struct(self):
+        ks, ka = _lib.segments(self.kseg)
+        ns, na = _lib.segments(self.nseg)
+        qw = _lib.SqQWeight(self.bits, self.group, self.N, self.K, ks, ns,
+                            ctypes.c_void_p(self.codes.data_ptr()),
+                            ctypes.c_void_p(self.scales.data_ptr()))
+        return qw, (ka, na)
+
+
+def qweight_sizes(bits: int, N: int, K: int, J: int) -> Tuple[int, int]:
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _lib.check("sq_qweight_sizes", _lib.load().sq_qweight_sizes(
+        bits, N, K, J, 0 if bits == 8 else 128, ctypes.byref(cb), ctypes.byref(sb)))
+    return cb.value, sb.value
+
+
+def calibrate(x: torch.Tensor, kseg: Sequence[int], s_pos: Optional[torch.Tensor] = None,
+              s_neg: Optional[torch.Tensor] = None, stream=None):
+    """Static DualScale scales of the calibration rows ``x`` [rows, K]: (s+, s-) fp32 [J]."""
+    _check_2d(x, "x")
+    J = len(kseg) - 1
+    if s_pos is None:
+        s_pos = torch.empty(J, dtype=torch.float32, device=x.device)
+    if s_neg is None:
+        s_neg = torch.empty(J, dtype=torch.float32, device=x.device)
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_calibrate", _lib.load().sq_calibrate(
+        _ptr(x), _dtype_code(x.dtype), x.shape[0], x.shape[1], x.stride(0), ctypes.byref(seg),
+        _ptr(s_pos), _ptr(s_neg), _stream(stream)))
+    return s_pos, s_neg
+
+
+def quantize_weights(w: torch.Tensor, kseg: Sequence[int], nseg: Optional[Sequence[int]] = None,
+                     bits: int = 8, out: Optional[QuantizedWeight] = None,
+                     stream=None) -> QuantizedWeight:
+    """Quantize an [N, K] weight: int8 per (channel, K segment) or int4 group 128."""
+    _check_2d(w, "w")
+    N, K = w.shape
+    kseg = tuple(int(b) for b in kseg)
+    nseg = tuple(int(b) for b in (nseg if nseg is not None else (0, N)))
+    if out is None:
+        cb, sb = qweight_sizes(bits, N, K, len(kseg) - 1)
+        if bits == 8:
+            codes = torch.empty((N, K), dtype=torch.int8, device=w.device)
+            scales = torch.empty((len(kseg) - 1, N), dtype=torch.float32, device=w.device)
+        else:
+            codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+            scales = torch.empty((N, K // 128), dtype=torch.float16, device=w.device)
+        assert codes.numel() * codes.element_size() == cb
+        assert scales.numel() * scales.element_size() == sb
+        out = QuantizedWeight(bits, N, K, kseg, nseg, codes, scales)
+    qw, keep = out.c_struct()
+    _lib.check("sq_quantize_weights", _lib.load().sq_quantize_weights(
+        _ptr(w), _dtype_code(w.dtype), N, K, w.stride(0), ctypes.byref(qw), _stream(stream)))
+    return out
+
+
+def linear(x: torch.Tensor, qw: QuantizedWeight, s_pos: torch.Tensor, s_neg: torch.Tensor,
+           bias: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
+           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The fused forward pass y = DualScale-quantized x times the quantized weight (+ bias)."""
+    _check_2d(x, "x")
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, qw.N), dtype=out_dtype, device=x.device)
+    _check_2d(out, "out")
+    c, keep = qw.c_struct()
+    _lib.check("sq_linear_forward", _lib.load().sq_linear_forward(
+        _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(c), _ptr(s_pos),
+        _ptr(s_neg), _ptr(bias), _ptr(out), _dtype_code(out.dtype), out.stride(0), _stream(stream)))
+    return out
+
+
+def quantize_activations(x: torch.Tensor, kseg: Sequence[int], s_pos: torch.Tensor,
+                         s_neg: torch.Tensor, stream=None):
+    """DualScale codes (q+, q-), int8 [M, K] each."""
+    _check_2d(x, "x")
+    M, K = x.shape
+    ldq = (K + 15) // 16 * 16
+    qp = torch.empty((M, ldq), dtype=torch.int8, device=x.device)
+    qn = torch.empty((M, ldq), dtype=torch.int8, device=x.device)
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_quantize_activations", _lib.load().sq_quantize_activations(
+        _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(seg), _ptr(s_pos),
+        _ptr(s_neg), _ptr(qp), _ptr(qn), ldq, _stream(stream)))
+    return qp[:, :K], qn[:, :K]
+
+
+def num_units(qw: QuantizedWeight) -> int:
+    return len(qw.kseg) - 1 if qw.bits == 8 else qw.K // 128
+
+
+def linear_accumulators(x: torch.Tensor, qw: QuantizedWeight, s_pos: torch.Tensor,
+                        s_neg: torch.Tensor, stream=None) -> torch.Tensor:
+    """Raw int32 accumulators [U, 2, M, N] of the fused kernel (test surface)."""
+    _check_2d(x, "x")
+    M, K = x.shape
+    acc = torch.empty((num_units(qw), 2, M, qw.N), dtype=torch.int32, device=x.device)
+    c, keep = qw.c_struct()
+    _lib.check("sq_linear_accumulators", _lib.load().sq_linear_accumulators(
+        _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(c), _ptr(s_pos),
+        _ptr(s_neg), _ptr(acc), _stream(stream)))
+    return acc
+
+
+def stream_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status word."""
+    return int(_lib.load().sq_stream_status(_stream(stream)))
+
+
+def set_wait_budget(cycles: int) -> None:
+    _lib.load().sq_set_wait_budget(int(cycles))

@@ -1,0 +1,91 @@
+"""ctypes declarations of the C ABI in ``include/segquant.h``.
+
+Argument marshalling only: no arithmetic of the layer happens here.  Loading
+fails loudly when the compiled library is missing; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libsegquant.so")
+
+SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED = 0, 1, 2, 3
+SQ_ERR_RANGE, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 4, 5, 6
+SQ_F32, SQ_BF16 = 0, 1
+SQ_MAX_SEGMENTS = 16
+SQ_MAX_K = 131072
+
+# Every function declared in include/segquant.h, with (restype, argtypes).
+c_i32, c_i64, c_vp, c_size = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+
+
+class SqSegments(ctypes.Structure):
+    _fields_ = [("count", ctypes.c_int32), ("bounds", ctypes.POINTER(ctypes.c_int32))]
+
+
+class SqQWeight(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group", ctypes.c_int32), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("kseg", SqSegments), ("nseg", SqSegments),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+P_SEG = ctypes.POINTER(SqSegments)
+P_QW = ctypes.POINTER(SqQWeight)
+P_SIZE = ctypes.POINTER(c_size)
+
+SIGNATURES = {
+    "sq_qweight_sizes": (c_i32, [c_i32, c_i64, c_i64, c_i32, c_i32, P_SIZE, P_SIZE]),
+    "sq_calibrate": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp, c_vp, c_vp]),
+    "sq_quantize_weights": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp]),
+    "sq_linear_forward": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp, c_vp,
+                                  c_i32, c_i64, c_vp]),
+    "sq_quantize_activations": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp, c_vp, c_vp,
+                                        c_vp, c_i64, c_vp]),
+    "sq_linear_accumulators": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp,
+                                       c_vp]),
+    "sq_stream_status": (c_i32, [c_vp]),
+    "sq_status_string": (ctypes.c_char_p, [c_i32]),
+    "sq_set_wait_budget": (None, [c_i64]),
+}
+
+_lib = None
+
+
+def load():
+    """Load ``libsegquant.so`` (built by ``post_quantized_linear_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m post_quantized_linear_b200.build`"
+                " (there is no CPU fallback)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load().sq_status_string(int(code)).decode()
+
+
+class SegQuantError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = int(code)
+        super().__init__(f"{fn} failed: {status_string(code)}")
+
+
+def check(fn: str, code: int) -> None:
+    if code != SQ_OK:
+        raise SegQuantError(fn, code)
+
+
+def segments(bounds) -> tuple:
+    """Build an sq_segments struct; returns (struct, keep-alive array)."""
+    arr = (ctypes.c_int32 * len(bounds))(*[int(b) for b in bounds])
+    return SqSegments(len(bounds) - 1, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))), arr

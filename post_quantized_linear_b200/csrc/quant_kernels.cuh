@@ -1,0 +1,276 @@
+// HBM-bound DualScale kernels: static calibration (per-segment polarity
+// maxima), standalone activation quantization, and weight quantization
+// (int8 per channel and K segment, int4 group-128 with fp16 scales).
+//
+// SegQuant ("SegQuant: A Semantics-Aware and Generalizable Quantization
+// Framework for Diffusion Models"): DualScale splits X into non-negative and
+// negative parts with separate static scales (Spanish technical summary 2.B,
+// Korean technical summary section 2 "DualScale"); SegLinear gives each input
+// segment its own scales (Spanish technical summary 2.A).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace sq {
+
+// ----------------------------------------------------------------- loads
+// 16-byte vector of activations widened to fp32: 8 bf16 or 4 fp32 values.
+template <typename XT> struct Vec;
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ __forceinline__ static void load(const void* p, float (&v)[8]) {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <> struct Vec<float> {
+  static constexpr int n = 4;
+  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
+    float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+};
+
+// ------------------------------------------------------------ calibration
+// blockDim = (32, 8).  Lane x of the block owns the 16-byte column vector
+// v = blockIdx.x * 32 + x of every row it visits (rows blockIdx.y*8+y, stepping
+// by gridDim.y*8), so each thread sees one K segment only.  Groups of 16 lanes
+// cover 128 bf16 / 64 fp32 columns, never straddling a segment bound (bounds
+// are multiples of 128), so a 16-lane shuffle reduction is exact.  Block
+// maxima are combined in shared memory, then divided by 127 and merged into
+// the outputs with an integer atomicMax on the fp32 bit patterns: for
+// non-negative floats the bit order is the value order, and rounding the
+// quotient is monotone, so max_c(fl(P_c/127)) = fl(max_c P_c / 127).
+// The outputs must be zeroed before the launch.
+template <typename XT>
+__global__ void __launch_bounds__(256) calibrate_kernel(const XT* __restrict__ x, int64_t rows,
+                                                        int64_t K, int64_t ldx, SegBounds kseg,
+                                                        float* __restrict__ s_pos,
+                                                        float* __restrict__ s_neg) {
+  constexpr int VN = Vec<XT>::n;
+  __shared__ unsigned int sh_p[SQ_MAX_SEG], sh_n[SQ_MAX_SEG];
+  __shared__ int sh_bad;
+  const int tid = threadIdx.y * 32 + threadIdx.x;
+  if (tid < SQ_MAX_SEG) { sh_p[tid] = 0u; sh_n[tid] = 0u; }
+  if (tid == 0) sh_bad = 0;
+  __syncthreads();
+
+  const int64_t nvec = K / VN;
+  const int64_t v = (int64_t)blockIdx.x * 32 + threadIdx.x;
+  const bool active = v < nvec;
+  const int j = active ? kseg.segment_of((int32_t)(v * VN)) : 0;
+  float P = 0.0f, Q = 0.0f;
+  bool bad = false;
+  if (active) {
+    const XT* col = x + v * VN;
+    int64_t m = (int64_t)blockIdx.y * 8 + threadIdx.y;
+    const int64_t step = (int64_t)gridDim.y * 8;
+    for (; m + 3 * step < rows; m += 4 * step) {
+      float a[4][VN];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Vec<XT>::load(col + (m + u * step) * ldx, a[u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < VN; ++i) {
+          const float t = a[u][i];
+          bad |= (t != t) || (fabsf(t) == __int_as_float(0x7f800000));
+          P = fmaxf(P, t);
+          Q = fmaxf(Q, -t);
+        }
+    }
+    for (; m < rows; m += step) {
+      float a[VN];
+      Vec<XT>::load(col + m * ldx, a);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) {
+        bad |= (a[i] != a[i]) || (fabsf(a[i]) == __int_as_float(0x7f800000));
+        P = fmaxf(P, a[i]);
+        Q = fmaxf(Q, -a[i]);
+      }
+    }
+  }
+  // 16-lane max reduction (all 16 lanes share one segment).
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+    P = fmaxf(P, __shfl_xor_sync(0xffffffffu, P, o));
+    Q = fmaxf(Q, __shfl_xor_sync(0xffffffffu, Q, o));
+  }
+  const unsigned any_bad = __ballot_sync(0xffffffffu, bad);
+  if (active && (threadIdx.x & 15) == 0) {
+    atomicMax(&sh_p[j], __float_as_uint(P));
+    atomicMax(&sh_n[j], __float_as_uint(Q));
+  }
+  if (threadIdx.x == 0 && any_bad) sh_bad = 1;
+  __syncthreads();
+  if (tid < kseg.count) {
+    const float p = __uint_as_float(sh_p[tid]) / 127.0f;
+    const float q = __uint_as_float(sh_n[tid]) / 127.0f;
+    if (p > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(s_pos) + tid, __float_as_uint(p));
+    if (q > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(s_neg) + tid, __float_as_uint(q));
+  }
+  if (tid == 0 && sh_bad) raise_status(SQ_STATUS_RANGE);
+}
+
+// ------------------------------------------------------- DualScale codes
+// q+ = clamp(rne(max(x,0) * r+), 0, 127), q- = clamp(rne(min(x,0) * r-), -127, 0).
+// The rounding adds the exact product to 1.5 * 2^23 in one fma: in
+// [2^23, 2^24) the fp32 spacing is 1, so the fma's round-half-even lands on
+// 1.5*2^23 + rne(x*r) (the offset is even, so ties still go to even), and the
+// code is the low byte of the bit pattern.  Out-of-range sums are clamped in
+// the float domain first (fmin/fmax are monotone, so clamping commutes with
+// the rounding).
+__device__ __forceinline__ uint32_t code_pos(float v, float r) {
+  const float t = fminf(fmaf(fmaxf(v, 0.0f), r, kMagic), kMagic + 127.0f);
+  return __float_as_uint(t);
+}
+__device__ __forceinline__ uint32_t code_neg(float v, float r) {
+  const float t = fmaxf(fmaf(fminf(v, 0.0f), r, kMagic), kMagic - 127.0f);
+  return __float_as_uint(t);
+}
+// Low bytes of four fp32 bit patterns into one word (byte i from a_i).
+__device__ __forceinline__ uint32_t pack4_low(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+  const uint32_t lo = __byte_perm(a0, a1, 0x0040);
+  const uint32_t hi = __byte_perm(a2, a3, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+// One thread per 8 consecutive elements of a row (one 16-byte bf16 vector, or
+// two fp32 vectors); 8-byte stores of each code tensor.
+template <typename XT>
+__global__ void __launch_bounds__(256) quantize_activations_kernel(
+    const XT* __restrict__ x, int64_t M, int64_t K, int64_t ldx, SegBounds kseg,
+    const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
+    int8_t* __restrict__ q_neg, int64_t ldq) {
+  const int64_t groups_per_row = K / 8;
+  const int64_t total = M * groups_per_row;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = g / groups_per_row;
+    const int64_t k = (g - m * groups_per_row) * 8;
+    const int j = kseg.segment_of((int32_t)k);
+    const float sp = __ldg(s_pos + j), sn = __ldg(s_neg + j);
+    const float rp = sp > 0.0f ? __frcp_rn(sp) : 0.0f;
+    const float rn = sn > 0.0f ? __frcp_rn(sn) : 0.0f;
+    float v[8];
+    if constexpr (Vec<XT>::n == 8) {
+      Vec<XT>::load(x + m * ldx + k, v);
+    } else {
+      float a[4], b[4];
+      Vec<XT>::load(x + m * ldx + k, a);
+      Vec<XT>::load(x + m * ldx + k + 4, b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { v[i] = a[i]; v[4 + i] = b[i]; }
+    }
+    uint32_t p[8], n[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { p[i] = code_pos(v[i], rp); n[i] = code_neg(v[i], rn); }
+    uint2 up, un;
+    up.x = pack4_low(p[0], p[1], p[2], p[3]); up.y = pack4_low(p[4], p[5], p[6], p[7]);
+    un.x = pack4_low(n[0], n[1], n[2], n[3]); un.y = pack4_low(n[4], n[5], n[6], n[7]);
+    *reinterpret_cast<uint2*>(q_pos + m * ldq + k) = up;
+    *reinterpret_cast<uint2*>(q_neg + m * ldq + k) = un;
+  }
+}
+
+// ------------------------------------------------------ weight quantization
+// int8: one warp per (output channel n, K segment j).  Pass 1: |W| max by
+// warp shuffles; s = max/127; r = 1/s.  Pass 2: codes with the same magic
+// rounding, clamp to +-127.
+template <typename WT>
+__global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
+    const WT* __restrict__ w, int64_t N, int64_t K, int64_t ldw, SegBounds kseg,
+    int8_t* __restrict__ codes, float* __restrict__ scales) {
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = N * kseg.count;
+  if (warp >= total) return;
+  const int64_t n = warp / kseg.count;
+  const int j = (int)(warp - n * kseg.count);
+  const int32_t k0 = kseg.b[j], k1 = kseg.b[j + 1];
+  const WT* row = w + n * ldw;
+  float amax = 0.0f;
+  bool bad = false;
+  for (int32_t k = k0 + lane * 4; k < k1; k += 128) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (k + i < k1) {
+        const float a = fabsf(to_f32(row[k + i]));
+        bad |= !(a <= 3.4028234663852886e38f);
+        amax = fmaxf(amax, a);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(SQ_STATUS_RANGE);
+  const float s = amax / 127.0f;
+  const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+  if (lane == 0) scales[(int64_t)j * N + n] = s;
+  for (int32_t k = k0 + lane * 4; k < k1; k += 128) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (k + i < k1) {
+        const float v = to_f32(row[k + i]);
+        float t = fmaf(v, r, kMagic);
+        t = fminf(fmaxf(t, kMagic - 127.0f), kMagic + 127.0f);
+        codes[n * K + k + i] = (int8_t)(__float_as_uint(t) & 0xFFu);
+      }
+    }
+  }
+}
+
+// int4: one warp per (output channel n, 128-wide group g); lane l owns k =
+// 128g + 4l .. 4l+3.  s16 = fp16_rne(max/7) (fp32 division, then one RNE to
+// binary16); codes use the widened fp16 scale; two codes per byte, low nibble
+// = even k; scales stored [N][K/128].
+template <typename WT>
+__global__ void __launch_bounds__(256) quantize_weights_w4_kernel(
+    const WT* __restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t* __restrict__ packed,
+    __half* __restrict__ scales) {
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t G = K / 128;
+  if (warp >= N * G) return;
+  const int64_t n = warp / G;
+  const int64_t g = warp - n * G;
+  const WT* src = w + n * ldw + g * 128 + lane * 4;
+  float v[4];
+  float amax = 0.0f;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[i] = to_f32(src[i]);
+    const float a = fabsf(v[i]);
+    bad |= !(a <= 3.4028234663852886e38f);
+    amax = fmaxf(amax, a);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const __half s16 = __float2half_rn(amax / 7.0f);
+  const float sf = __half2float(s16);
+  bad |= !(sf <= 65504.0f);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(SQ_STATUS_RANGE);
+  const float r = sf > 0.0f ? __frcp_rn(sf) : 0.0f;
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float t = fmaf(v[i], r, kMagic);
+    t = fminf(fmaxf(t, kMagic - 7.0f), kMagic + 7.0f);
+    q[i] = __float_as_uint(t) & 0xFu;  // two's complement nibble
+  }
+  const uint16_t two = (uint16_t)(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
+  *reinterpret_cast<uint16_t*>(packed + n * (K / 2) + g * 64 + lane * 2) = two;
+  if (lane == 0) scales[n * G + g] = s16;
+}
+
+}  // namespace sq

@@ -1,0 +1,364 @@
+// Host side of the C ABI declared in include/segquant.h: argument validation,
+// TMA descriptor encoding and kernel launches.  One translation unit holds
+// every kernel so that they share the per-device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "segquant.h"
+
+#include "common.cuh"
+#include "gemm_dualscale.cuh"
+#include "ptx.cuh"
+#include "quant_kernels.cuh"
+
+namespace {
+
+using sq::SegBounds;
+
+constexpr long long kDefaultWaitBudget = 2000000000LL;  // ~1 s of SM clock
+long long g_wait_budget = kDefaultWaitBudget;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int elt_size(sq_dtype t) { return t == SQ_F32 ? 4 : 2; }
+bool dtype_ok(sq_dtype t) { return t == SQ_F32 || t == SQ_BF16; }
+
+// Segment bounds: count in [1, max_count], strictly increasing, 0 .. extent;
+// interior bounds multiples of `granule` (when granule > 1).
+sq_status check_segments(const sq_segments* s, int64_t extent, int max_count, int granule,
+                         SegBounds* out) {
+  if (s == nullptr || s->bounds == nullptr) return SQ_ERR_INVALID_ARG;
+  if (s->count < 1) return SQ_ERR_INVALID_ARG;
+  if (s->count > max_count) return SQ_ERR_UNSUPPORTED;
+  if (s->bounds[0] != 0 || (int64_t)s->bounds[s->count] != extent) return SQ_ERR_INVALID_ARG;
+  for (int i = 0; i < s->count; ++i)
+    if (s->bounds[i + 1] <= s->bounds[i]) return SQ_ERR_INVALID_ARG;
+  if (granule > 1)
+    for (int i = 1; i < s->count; ++i)
+      if (s->bounds[i] % granule != 0) return SQ_ERR_UNSUPPORTED;
+  if (out != nullptr) {
+    std::memset(out, 0, sizeof(*out));
+    out->count = s->count;
+    for (int i = 0; i <= s->count; ++i) out->b[i] = s->bounds[i];
+  }
+  return SQ_OK;
+}
+
+sq_status check_nseg(const sq_segments* s, int64_t N) {
+  if (s == nullptr || s->bounds == nullptr || s->count < 1) return SQ_ERR_INVALID_ARG;
+  if (s->bounds[0] != 0 || (int64_t)s->bounds[s->count] != N) return SQ_ERR_INVALID_ARG;
+  for (int i = 0; i < s->count; ++i)
+    if (s->bounds[i + 1] <= s->bounds[i]) return SQ_ERR_INVALID_ARG;
+  return SQ_OK;
+}
+
+sq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D row-major tensor, 128-byte swizzled boxes of box_inner x box_rows.
+sq_status make_tmap(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                    uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return SQ_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SQ_OK : SQ_ERR_CUDA;
+}
+
+sq_status check_qweight(const sq_qweight* w, int64_t K, SegBounds* kseg) {
+  if (w == nullptr) return SQ_ERR_INVALID_ARG;
+  if (w->N <= 0 || w->K <= 0 || w->K != K) return SQ_ERR_INVALID_ARG;
+  if (w->codes == nullptr || w->scales == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!(w->bits == 8 && w->group == 0) && !(w->bits == 4 && w->group == 128))
+    return SQ_ERR_UNSUPPORTED;
+  if (w->N > (int64_t)INT32_MAX - 256) return SQ_ERR_RANGE;
+  if (w->K > SQ_MAX_K) return SQ_ERR_RANGE;
+  if (w->N % 16 != 0 || w->K % 16 != 0) return SQ_ERR_UNSUPPORTED;
+  if (w->bits == 4 && w->K % 128 != 0) return SQ_ERR_UNSUPPORTED;
+  sq_status s = check_segments(&w->kseg, w->K, SQ_MAX_SEGMENTS, 128, kseg);
+  if (s != SQ_OK) return s;
+  s = check_nseg(&w->nseg, w->N);
+  if (s != SQ_OK) return s;
+  if (!aligned16(w->codes) || !aligned16(w->scales)) return SQ_ERR_ALIGNMENT;
+  return SQ_OK;
+}
+
+template <int BN, typename XT, bool ACC, bool YB>
+sq_status launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const sq::GemmArgs& a,
+                      cudaStream_t stream) {
+  using C = sq::GemmCfg<BN, XT>;
+  auto kern = sq::dualscale_gemm_kernel<BN, XT, ACC, YB>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return SQ_ERR_CUDA;
+  dim3 grid((a.N + BN - 1) / BN, (a.M + sq::BM - 1) / sq::BM);
+  kern<<<grid, sq::kThreads, C::SMEM_BYTES, stream>>>(tx, tw, a);
+  return cuda_status(cudaGetLastError());
+}
+
+sq_status gemm_common(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                      const sq_qweight* w, const float* s_pos, const float* s_neg,
+                      const float* bias, void* y, sq_dtype yt, int64_t ldy, int32_t* acc,
+                      cudaStream_t stream) {
+  if (!dtype_ok(xt)) return SQ_ERR_INVALID_ARG;
+  if (acc == nullptr && !dtype_ok(yt)) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  SegBounds kseg;
+  sq_status st = check_qweight(w, K, &kseg);
+  if (st != SQ_OK) return st;
+  const int64_t N = w->N;
+  if (ldx < K) return SQ_ERR_INVALID_ARG;
+  if (acc == nullptr && ldy < N) return SQ_ERR_INVALID_ARG;
+  if (M > (int64_t)65535 * sq::BM) return SQ_ERR_RANGE;
+  if (M == 0) return SQ_OK;
+  if (x == nullptr || s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
+  if (acc == nullptr && y == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || (ldx * elt_size(xt)) % 16 != 0) return SQ_ERR_ALIGNMENT;
+  if (acc == nullptr && (!aligned16(y) || (ldy * elt_size(yt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
+  if (acc != nullptr && !aligned16(acc)) return SQ_ERR_ALIGNMENT;
+  if (bias != nullptr && !aligned16(bias)) return SQ_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(s_pos) & 3u) || (reinterpret_cast<uintptr_t>(s_neg) & 3u))
+    return SQ_ERR_ALIGNMENT;
+  if (w->bits == 4) return SQ_ERR_UNSUPPORTED;  // int4 operand path not built yet
+
+  constexpr int BN = 128;
+  CUtensorMap tx, tw;
+  const int xe = elt_size(xt);
+  st = make_tmap(&tx, xt == SQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                 x, (uint64_t)K, (uint64_t)M, (uint64_t)(ldx * xe), 128 / xe, sq::BM);
+  if (st != SQ_OK) return st;
+  st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K, (uint64_t)N,
+                 (uint64_t)K, 128, BN);
+  if (st != SQ_OK) return st;
+
+  sq::GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int32_t)M;
+  a.N = (int32_t)N;
+  a.K = (int32_t)K;
+  a.num_kb = (int32_t)((K + sq::BK - 1) / sq::BK);
+  a.bits = w->bits;
+  a.kseg = kseg;
+  a.s_pos = s_pos;
+  a.s_neg = s_neg;
+  a.wscales = w->scales;
+  a.bias = bias;
+  a.y = y;
+  a.ldy = ldy;
+  a.acc_out = acc;
+  a.wait_budget = g_wait_budget;
+
+  if (acc != nullptr) {
+    return xt == SQ_BF16 ? launch_gemm<BN, __nv_bfloat16, true, false>(tx, tw, a, stream)
+                         : launch_gemm<BN, float, true, false>(tx, tw, a, stream);
+  }
+  if (xt == SQ_BF16)
+    return yt == SQ_BF16 ? launch_gemm<BN, __nv_bfloat16, false, true>(tx, tw, a, stream)
+                         : launch_gemm<BN, __nv_bfloat16, false, false>(tx, tw, a, stream);
+  return yt == SQ_BF16 ? launch_gemm<BN, float, false, true>(tx, tw, a, stream)
+                       : launch_gemm<BN, float, false, false>(tx, tw, a, stream);
+}
+
+int grid_for(int64_t work_items, int per_block) {
+  int64_t g = (work_items + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > 148 * 32) g = 148 * 32;
+  return (int)g;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sq_status_string(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG";
+    case SQ_ERR_ALIGNMENT: return "SQ_ERR_ALIGNMENT";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED";
+    case SQ_ERR_RANGE: return "SQ_ERR_RANGE";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+  }
+  return "SQ_UNKNOWN_STATUS";
+}
+
+void sq_set_wait_budget(int64_t cycles) { g_wait_budget = cycles > 0 ? cycles : kDefaultWaitBudget; }
+
+sq_status sq_qweight_sizes(int32_t bits, int64_t N, int64_t K, int32_t J, int32_t group,
+                           size_t* code_bytes, size_t* scale_bytes) {
+  if (code_bytes == nullptr || scale_bytes == nullptr) return SQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || J < 1) return SQ_ERR_INVALID_ARG;
+  if (bits == 8 && group == 0) {
+    if (J > SQ_MAX_SEGMENTS) return SQ_ERR_UNSUPPORTED;
+    *code_bytes = (size_t)N * (size_t)K;
+    *scale_bytes = (size_t)J * (size_t)N * sizeof(float);
+    return SQ_OK;
+  }
+  if (bits == 4 && group == 128) {
+    if (K % 128 != 0) return SQ_ERR_UNSUPPORTED;
+    *code_bytes = (size_t)N * (size_t)(K / 2);
+    *scale_bytes = (size_t)N * (size_t)(K / 128) * 2;
+    return SQ_OK;
+  }
+  return SQ_ERR_UNSUPPORTED;
+}
+
+sq_status sq_calibrate(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
+                       const sq_segments* kseg, float* s_pos, float* s_neg, sq_stream_t stream) {
+  if (!dtype_ok(xt) || rows < 0 || K <= 0 || ldx < K) return SQ_ERR_INVALID_ARG;
+  if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
+  if (K > SQ_MAX_K) return SQ_ERR_RANGE;
+  SegBounds sb;
+  sq_status st = check_segments(kseg, K, SQ_MAX_SEGMENTS, 128, &sb);
+  if (st != SQ_OK) return st;
+  const int xe = elt_size(xt);
+  if (K % (16 / xe) != 0) return SQ_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(s_pos) & 3u) || (reinterpret_cast<uintptr_t>(s_neg) & 3u))
+    return SQ_ERR_ALIGNMENT;
+  if (rows > 0) {
+    if (x == nullptr) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || (ldx * xe) % 16 != 0) return SQ_ERR_ALIGNMENT;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(float) * (size_t)sb.count;
+  if (cudaMemsetAsync(s_pos, 0, bytes, s) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemsetAsync(s_neg, 0, bytes, s) != cudaSuccess) return SQ_ERR_CUDA;
+  if (rows == 0) return SQ_OK;
+  const int64_t nvec = K / (16 / xe);
+  const int gx = (int)((nvec + 31) / 32);
+  int64_t gy = (rows + 7) / 8;
+  const int64_t target = (int64_t)148 * 8;
+  int64_t cap = (target + gx - 1) / gx;
+  if (cap < 1) cap = 1;
+  if (gy > cap) gy = cap;
+  if (gy > 65535) gy = 65535;
+  dim3 grid(gx, (unsigned)gy), block(32, 8);
+  if (xt == SQ_BF16)
+    sq::calibrate_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), rows, K, ldx, sb, s_pos, s_neg);
+  else
+    sq::calibrate_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(x), rows, K, ldx,
+                                                       sb, s_pos, s_neg);
+  return cuda_status(cudaGetLastError());
+}
+
+sq_status sq_quantize_weights(const void* w, sq_dtype wt, int64_t N, int64_t K, int64_t ldw,
+                              const sq_qweight* out, sq_stream_t stream) {
+  if (!dtype_ok(wt) || w == nullptr || out == nullptr) return SQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || ldw < K) return SQ_ERR_INVALID_ARG;
+  if (out->N != N) return SQ_ERR_INVALID_ARG;
+  SegBounds kseg;
+  sq_status st = check_qweight(out, K, &kseg);
+  if (st != SQ_OK) return st;
+  if (!aligned16(w) || (ldw * elt_size(wt)) % 16 != 0) return SQ_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (out->bits == 8) {
+    const int64_t warps = N * kseg.count;
+    const int blocks = (int)((warps * 32 + 255) / 256);
+    if (wt == SQ_BF16)
+      sq::quantize_weights_w8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(w), N, K, ldw, kseg, static_cast<int8_t*>(out->codes),
+          static_cast<float*>(out->scales));
+    else
+      sq::quantize_weights_w8_kernel<float><<<blocks, 256, 0, s>>>(
+          static_cast<const float*>(w), N, K, ldw, kseg, static_cast<int8_t*>(out->codes),
+          static_cast<float*>(out->scales));
+  } else {
+    const int64_t warps = N * (K / 128);
+    const int blocks = (int)((warps * 32 + 255) / 256);
+    if (wt == SQ_BF16)
+      sq::quantize_weights_w4_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(w), N, K, ldw, static_cast<uint8_t*>(out->codes),
+          static_cast<__half*>(out->scales));
+    else
+      sq::quantize_weights_w4_kernel<float><<<blocks, 256, 0, s>>>(
+          static_cast<const float*>(w), N, K, ldw, static_cast<uint8_t*>(out->codes),
+          static_cast<__half*>(out->scales));
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                  const sq_segments* kseg, const float* s_pos,
+                                  const float* s_neg, int8_t* q_pos, int8_t* q_neg, int64_t ldq,
+                                  sq_stream_t stream) {
+  if (!dtype_ok(xt) || M < 0 || K <= 0 || ldx < K || ldq < K) return SQ_ERR_INVALID_ARG;
+  if (K > SQ_MAX_K) return SQ_ERR_RANGE;
+  SegBounds sb;
+  sq_status st = check_segments(kseg, K, SQ_MAX_SEGMENTS, 128, &sb);
+  if (st != SQ_OK) return st;
+  if (K % 8 != 0) return SQ_ERR_UNSUPPORTED;
+  if (M == 0) return SQ_OK;
+  if (x == nullptr || s_pos == nullptr || s_neg == nullptr || q_pos == nullptr || q_neg == nullptr)
+    return SQ_ERR_INVALID_ARG;
+  const int xe = elt_size(xt);
+  if (!aligned16(x) || (ldx * xe) % 16 != 0 || !aligned16(q_pos) || !aligned16(q_neg) ||
+      ldq % 16 != 0)
+    return SQ_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int blocks = grid_for(M * (K / 8), 256);
+  if (xt == SQ_BF16)
+    sq::quantize_activations_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), M, K, ldx, sb, s_pos, s_neg, q_pos, q_neg, ldq);
+  else
+    sq::quantize_activations_kernel<float><<<blocks, 256, 0, s>>>(
+        static_cast<const float*>(x), M, K, ldx, sb, s_pos, s_neg, q_pos, q_neg, ldq);
+  return cuda_status(cudaGetLastError());
+}
+
+sq_status sq_linear_forward(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                            const sq_qweight* w, const float* s_pos, const float* s_neg,
+                            const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                            sq_stream_t stream) {
+  return gemm_common(x, xt, M, K, ldx, w, s_pos, s_neg, bias, y, yt, ldy, nullptr,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear_accumulators(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                 const sq_qweight* w, const float* s_pos, const float* s_neg,
+                                 int32_t* acc, sq_stream_t stream) {
+  if (acc == nullptr) return SQ_ERR_INVALID_ARG;
+  return gemm_common(x, xt, M, K, ldx, w, s_pos, s_neg, nullptr, nullptr, SQ_F32, 0, acc,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_stream_status(sq_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, sq::g_status, sizeof(v)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(sq::g_status, &zero, sizeof(zero)) != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  if (v & sq::SQ_STATUS_TIMEOUT) return SQ_ERR_TIMEOUT;
+  if (v & sq::SQ_STATUS_RANGE) return SQ_ERR_RANGE;
+  return SQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,128 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+declared in include/segquant.h, and rejects bad arguments before touching the
+GPU (every call below returns during host validation)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_quantized_linear_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "segquant.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_entry_point():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, n
+
+
+def test_status_strings():
+    assert _lib.status_string(0) == "SQ_OK"
+    assert _lib.status_string(6) == "SQ_ERR_TIMEOUT"
+    assert _lib.status_string(99) == "SQ_UNKNOWN_STATUS"
+
+
+def _sizes(bits, N, K, J, group):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    st = _lib.load().sq_qweight_sizes(bits, N, K, J, group, ctypes.byref(cb), ctypes.byref(sb))
+    return st, cb.value, sb.value
+
+
+def test_qweight_sizes():
+    assert _sizes(8, 1152, 4608, 1, 0) == (0, 1152 * 4608, 4 * 1152)
+    assert _sizes(8, 3456, 2304, 2, 0) == (0, 3456 * 2304, 2 * 4 * 3456)
+    assert _sizes(4, 3072, 3072, 1, 128) == (0, 3072 * 1536, 2 * 3072 * 24)
+    assert _sizes(4, 16, 200, 1, 128)[0] == _lib.SQ_ERR_UNSUPPORTED
+    assert _sizes(4, 16, 256, 1, 64)[0] == _lib.SQ_ERR_UNSUPPORTED
+    assert _sizes(6, 16, 256, 1, 0)[0] == _lib.SQ_ERR_UNSUPPORTED
+    assert _sizes(8, 0, 256, 1, 0)[0] == _lib.SQ_ERR_INVALID_ARG
+    assert _sizes(8, 16, 256, 17, 0)[0] == _lib.SQ_ERR_UNSUPPORTED
+
+
+FAKE = 1 << 20          # a 16-byte aligned, never dereferenced address
+FAKE_ODD = FAKE + 4     # 4-byte aligned only
+
+
+def _qw(bits=8, N=256, K=512, kb=(0, 512), nb=None, codes=FAKE, scales=FAKE):
+    ks, ka = _lib.segments(kb)
+    ns, na = _lib.segments(nb or (0, N))
+    qw = _lib.SqQWeight(bits, 0 if bits == 8 else 128, N, K, ks, ns, codes, scales)
+    return qw, (ka, na)
+
+
+def _fwd(x=FAKE, xt=_lib.SQ_BF16, M=256, K=512, ldx=512, qw=None, sp=FAKE, sn=FAKE, bias=None,
+         y=FAKE, yt=_lib.SQ_BF16, ldy=256):
+    if qw is None:
+        qw, keep = _qw(K=K)
+    return _lib.load().sq_linear_forward(x, xt, M, K, ldx, ctypes.byref(qw), sp, sn, bias, y, yt,
+                                         ldy, None)
+
+
+def test_forward_validation_rejects_before_launch():
+    L = _lib
+    assert _fwd(M=-1) == L.SQ_ERR_INVALID_ARG
+    assert _fwd(xt=7) == L.SQ_ERR_INVALID_ARG
+    assert _fwd(ldx=100) == L.SQ_ERR_INVALID_ARG
+    assert _fwd(x=None) == L.SQ_ERR_INVALID_ARG
+    assert _fwd(x=FAKE + 8) == L.SQ_ERR_ALIGNMENT
+    assert _fwd(y=FAKE + 2) == L.SQ_ERR_ALIGNMENT
+    assert _fwd(ldy=260) == L.SQ_ERR_ALIGNMENT       # 520 bytes: not a multiple of 16
+    assert _fwd(bias=FAKE_ODD) == L.SQ_ERR_ALIGNMENT
+    assert _fwd(sp=FAKE + 2) == L.SQ_ERR_ALIGNMENT
+    qw, k = _qw(kb=(0, 200, 512))                     # interior bound not a multiple of 128
+    assert _fwd(qw=qw) == L.SQ_ERR_UNSUPPORTED
+    qw, k = _qw(kb=(0, 256, 256, 512))                # not increasing
+    assert _fwd(qw=qw) == L.SQ_ERR_INVALID_ARG
+    qw, k = _qw(kb=(0, 384))                          # does not end at K
+    assert _fwd(qw=qw) == L.SQ_ERR_INVALID_ARG
+    qw, k = _qw(N=200)                                # N % 16 != 0
+    assert _fwd(qw=qw, ldy=200) == L.SQ_ERR_UNSUPPORTED
+    qw, k = _qw(nb=(0, 100, 250))                     # output segments must end at N
+    assert _fwd(qw=qw) == L.SQ_ERR_INVALID_ARG
+    qw, k = _qw(K=512, codes=FAKE + 1)
+    assert _fwd(qw=qw) == L.SQ_ERR_ALIGNMENT
+    qw, k = _qw(K=256)                                # weight K differs from x K
+    assert _fwd(qw=qw) == L.SQ_ERR_INVALID_ARG
+    qw, k = _qw(K=262144, kb=(0, 262144))
+    assert _fwd(qw=qw, K=262144, ldx=262144) == L.SQ_ERR_RANGE
+    many = tuple(range(0, 128 * 18, 128))
+    qw, k = _qw(K=128 * 17, kb=many)
+    assert _fwd(qw=qw, K=128 * 17, ldx=128 * 17) == L.SQ_ERR_UNSUPPORTED
+    assert _fwd(M=0) == L.SQ_OK                       # empty input: no launch, no error
+
+
+def test_calibrate_and_quantize_validation():
+    lib = _lib.load()
+    seg, keep = _lib.segments((0, 512))
+    bad, keep2 = _lib.segments((0, 100, 512))
+    assert lib.sq_calibrate(FAKE, 1, 16, 512, 512, ctypes.byref(bad), FAKE, FAKE, None) == _lib.SQ_ERR_UNSUPPORTED
+    assert lib.sq_calibrate(FAKE, 1, -1, 512, 512, ctypes.byref(seg), FAKE, FAKE, None) == _lib.SQ_ERR_INVALID_ARG
+    assert lib.sq_calibrate(FAKE, 1, 16, 512, 512, ctypes.byref(seg), None, FAKE, None) == _lib.SQ_ERR_INVALID_ARG
+    assert lib.sq_calibrate(FAKE + 8, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, None) == _lib.SQ_ERR_ALIGNMENT
+    assert lib.sq_quantize_activations(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE,
+                                       FAKE, 520, None) == _lib.SQ_ERR_ALIGNMENT
+    assert lib.sq_quantize_activations(FAKE, 1, 0, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE,
+                                       FAKE, 512, None) == _lib.SQ_OK
+    qw, k = _qw(bits=4, K=512)
+    qw.N = 128
+    assert lib.sq_quantize_weights(FAKE, 0, 256, 512, 512, ctypes.byref(qw), None) == _lib.SQ_ERR_INVALID_ARG
+    qw, k = _qw(bits=4, K=500, kb=(0, 500))
+    assert lib.sq_quantize_weights(FAKE, 0, 256, 500, 500, ctypes.byref(qw), None) == _lib.SQ_ERR_UNSUPPORTED
+
+
+def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib.load()

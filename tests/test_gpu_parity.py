@@ -1,0 +1,154 @@
+"""GPU-vs-oracle parity of every step of the path, called through the C ABI.
+
+Bit-exact: calibration scales, weight codes and scales, DualScale activation
+codes, int32 accumulators.  Outputs: fp32 within 1e-6 of the magnitude sum,
+bf16 within one ulp (see tests/parity_util.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from synth import workloads as W
+
+from parity_util import (Case, assert_bf16_within_1ulp, assert_f32_within, bf16_bits,
+                         magnitude_sum, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import post_quantized_linear_b200 as pq  # noqa: F401  (fails loudly without the library)
+    O.build()
+    yield
+
+
+# Small shapes that span several tiles in M, N and K with ragged tails.
+SMALL = [
+    dict(M=300, K=640, N=272, kseg=[0, 256, 640], x_sigmas=[1.0, 5.0], x_dtype="bf16", out="bf16"),
+    dict(M=300, K=640, N=272, kseg=[0, 256, 640], x_sigmas=[1.0, 5.0], x_dtype="bf16", out="f32"),
+    dict(M=129, K=384, N=144, kseg=[0, 384], x_dtype="f32", out="f32"),
+    dict(M=64, K=256, N=256, kseg=[0, 256], x_dtype="f32", out="bf16"),
+    dict(M=1, K=16, N=16, kseg=[0, 16], x_dtype="bf16", out="bf16"),
+    dict(M=257, K=1040, N=128, kseg=[0, 128, 512, 1040], x_sigmas=[1.0, 3.0, 0.5], x_dtype="bf16",
+         out="f32"),
+]
+
+
+def _small(i, **over):
+    p = dict(SMALL[i])
+    p.update(over)
+    return W.small_case(p.pop("M"), p.pop("K"), p.pop("N"), seed=10 + i, **p)
+
+
+@pytest.mark.parametrize("i", range(len(SMALL)))
+def test_scales_and_weights_bit_exact(i):
+    c = Case(_small(i))
+    c.check_scales_and_weights()
+
+
+@pytest.mark.parametrize("i", range(len(SMALL)))
+def test_activation_codes_bit_exact(i):
+    import post_quantized_linear_b200 as pq
+    c = Case(_small(i))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    op, on = O.quantize_activations(c.x_np, c.wl.kseg, c.o_sp, c.o_sn)
+    np.testing.assert_array_equal(qp.cpu().numpy(), op)
+    np.testing.assert_array_equal(qn.cpu().numpy(), on)
+
+
+@pytest.mark.parametrize("i", range(len(SMALL)))
+def test_accumulators_bit_exact(i):
+    import post_quantized_linear_b200 as pq
+    c = Case(_small(i))
+    acc = pq.linear_accumulators(c.x, c.qw, c.sp, c.sn)
+    _, o_acc = c.oracle_rows(np.arange(c.wl.M))
+    np.testing.assert_array_equal(acc.cpu().numpy(), o_acc)
+
+
+@pytest.mark.parametrize("i", range(len(SMALL)))
+def test_forward_matches_oracle(i):
+    c = Case(_small(i))
+    c.check_scales_and_weights()
+    y = c.forward()
+    torch.cuda.synchronize()
+    c.compare_rows(y, np.arange(c.wl.M))
+
+
+def test_forward_exact_in_fp32():
+    """With the fp32 epilogue order the kernel reproduces the oracle bit for bit."""
+    c = Case(_small(1))
+    y = c.forward().cpu().numpy()
+    y_ref, _ = c.oracle_rows(np.arange(c.wl.M))
+    np.testing.assert_array_equal(y, y_ref)
+
+
+def test_nonnegative_input_and_zero_rows():
+    import post_quantized_linear_b200 as pq
+    wl = W.small_case(200, 256, 128, seed=3, act="none", bias=True, out="f32")
+    x, w, b = W.generate(wl)
+    x = x.abs().to(torch.float32)
+    x[5] = 0.0
+    xd, wd, bd = x.cuda().to(torch.bfloat16), w.cuda(), b.cuda()
+    sp, sn = pq.calibrate(xd, wl.kseg)
+    assert float(sn[0]) == 0.0
+    qw = pq.quantize_weights(wd, wl.kseg)
+    acc = pq.linear_accumulators(xd, qw, sp, sn)
+    assert int(acc[:, 1].abs().max()) == 0
+    y = pq.linear(xd, qw, sp, sn, bd, out_dtype=torch.float32)
+    np.testing.assert_array_equal(y[5].cpu().numpy(), b.numpy())
+
+
+def test_empty_batch_is_noop():
+    import post_quantized_linear_b200 as pq
+    c = Case(_small(3))
+    x0 = c.x[:0]
+    y = pq.linear(x0, c.qw, c.sp, c.sn, c.b, out_dtype=torch.float32)
+    assert y.shape == (0, c.wl.N)
+
+
+def test_output_segments_are_a_noop():
+    """Quantizing and running q | k | v separately equals the fused N = 3 x 1152 layer."""
+    import post_quantized_linear_b200 as pq
+    wl = W.small_case(256, 512, 384, seed=4, kseg=[0, 256, 512], x_sigmas=[1.0, 5.0], out="bf16")
+    x, w, _ = W.generate(wl)
+    w[128:256] *= 2.5
+    xd, wd = x.cuda(), w.cuda()
+    sp, sn = pq.calibrate(xd, wl.kseg)
+    full = pq.quantize_weights(wd, wl.kseg, (0, 128, 256, 384))
+    y = pq.linear(xd, full, sp, sn)
+    for n0, n1 in [(0, 128), (128, 256), (256, 384)]:
+        part = pq.quantize_weights(wd[n0:n1].contiguous(), wl.kseg)
+        assert torch.equal(part.codes, full.codes[n0:n1])
+        assert torch.equal(part.scales, full.scales[:, n0:n1])
+        assert torch.equal(pq.linear(xd, part, sp, sn), y[:, n0:n1])
+
+
+def test_strided_activations_and_outputs():
+    import post_quantized_linear_b200 as pq
+    c = Case(_small(0))
+    big = torch.zeros((c.wl.M, c.wl.K + 64), dtype=c.x.dtype, device="cuda")
+    big[:, 16:16 + c.wl.K] = c.x
+    xs = big[:, 16:16 + c.wl.K]
+    ybig = torch.zeros((c.wl.M, c.wl.N + 32), dtype=torch.bfloat16, device="cuda")
+    ys = ybig[:, 8:8 + c.wl.N]
+    pq.linear(xs, c.qw, c.sp, c.sn, c.b, out=ys)
+    assert torch.equal(ys, c.forward())
+    assert int(ybig[:, :8].abs().sum()) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny_w8a8", "dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up"])
+def test_workloads_full_size_sampled_rows(name):
+    """Full-size workloads in the bench's launch configuration: bit-exact scales
+    and weights everywhere; outputs of sampled rows against the oracle."""
+    wl = W.WORKLOADS[name]
+    c = Case(wl)
+    c.check_scales_and_weights()
+    y = c.forward()
+    torch.cuda.synchronize()
+    rows = np.arange(wl.M) if wl.M <= 256 else sample_rows(wl.M, 96 if wl.N > 4096 else 160)
+    c.compare_rows(y, rows)
+    import post_quantized_linear_b200 as pq
+    assert pq.stream_status() == 0
