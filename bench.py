@@ -45,6 +45,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_xl2_fc2_cfg")
+    ap.add_argument("--path", choices=["fused", "codes"], default="fused",
+                    help="fused: quantize X inside the GEMM; codes: quantize X once into "
+                         "q+/q- code tensors, then the GEMM loads the codes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -213,8 +216,8 @@ def run_reference(args):
     return 0
 
 
-def config_of(wl, l2):
-    return {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "bits": wl.bits,
+def config_of(wl, l2, path="fused"):
+    return {"workload": wl.name, "path": path, "M": wl.M, "K": wl.K, "N": wl.N, "bits": wl.bits,
             "x_dtype": wl.x_dtype, "out_dtype": wl.out, "k_segments": list(wl.kseg),
             "n_segments": list(wl.nseg), "calib_rows": wl.calib_rows or wl.M,
             "global_batch": wl.M, "l2": l2}
@@ -249,6 +252,11 @@ def run_ours(args):
     qw = pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=wl.bits)
     y = torch.empty((wl.M, wl.N), dtype=out_dtype, device=dev)
     calib = xd if wl.calib_rows is None else xd[: wl.calib_rows]
+    use_codes = args.path == "codes"
+    if use_codes:
+        ldq = (wl.K + 15) // 16 * 16
+        qp_buf = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
+        qn_buf = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -256,9 +264,17 @@ def run_ours(args):
         pq.calibrate(calib if xs is xd else (xs if wl.calib_rows is None else xs[: wl.calib_rows]),
                      wl.kseg, sp, sn)
         pq.quantize_weights(ws, wl.kseg, wl.nseg, bits=wl.bits, out=qw)
+        forward(xs, ys, gemm_events)
+
+    def forward(xs, ys, gemm_events=None):
+        if use_codes:
+            pq.quantize_activations(xs, wl.kseg, sp, sn, out=(qp_buf, qn_buf))
         if gemm_events:
             gemm_events[0].record(stream)
-        pq.linear(xs, qw, sp, sn, bd, out=ys)
+        if use_codes:
+            pq.linear_from_codes(qp_buf, qn_buf, qw, sp, sn, bd, out=ys)
+        else:
+            pq.linear(xs, qw, sp, sn, bd, out=ys)
         if gemm_events:
             gemm_events[1].record(stream)
 
@@ -266,7 +282,7 @@ def run_ours(args):
         return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(n)]
 
-    launches_per_step = 3
+    launches_per_step = 4 if use_codes else 3
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -299,7 +315,7 @@ def run_ours(args):
     for i in range(args.steps):
         flush.fill_((i + 7) & 0xFF)
         fev[i][0].record(stream)
-        pq.linear(xd, qw, sp, sn, bd, out=y)
+        forward(xd, y)
         fev[i][1].record(stream)
     torch.cuda.synchronize()
     fwd_ms = [a.elapsed_time(bv) for a, bv in fev]
@@ -355,7 +371,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-            "data": "synthetic", "config": config_of(wl, "flushed (256 MiB write between steps)"),
+            "data": "synthetic",
+            "config": config_of(wl, "flushed (256 MiB write between steps)", args.path),
             "roofline": {
                 "bound": "tensor", "kernel": "dualscale_gemm_kernel",
                 "achieved": gemm_tops, "peak": int8_peak_tops, "unit": "TOPS",

@@ -146,6 +146,19 @@ sq_status sq_linear_forward(const void* x, sq_dtype xt, int64_t M, int64_t K, in
                             const float* bias, void* y, sq_dtype yt, int64_t ldy,
                             sq_stream_t stream);
 
+/* The forward pass from pre-quantized DualScale codes (the q+ / q- tensors
+ * written by sq_quantize_activations with the same scales): the kernel loads
+ * both int8 code tiles by TMA and runs the two tensor-core products and the
+ * fused epilogue exactly as sq_linear_forward does, so the result is
+ * identical.  Splitting quantization from the GEMM lets one quantization
+ * serve every output tile instead of being redone per tile.
+ * q_pos, q_neg: device int8 [M, K], row stride ldq (a multiple of 16), 16-byte
+ * aligned.  Other arguments and requirements as for sq_linear_forward. */
+sq_status sq_linear_forward_codes(const int8_t* q_pos, const int8_t* q_neg, int64_t ldq,
+                                  int64_t M, int64_t K, const sq_qweight* w, const float* s_pos,
+                                  const float* s_neg, const float* bias, void* y, sq_dtype yt,
+                                  int64_t ldy, sq_stream_t stream);
+
 /* Test / fallback surface: the DualScale codes alone (same rules as the
  * forward's in-kernel quantization).  q_pos, q_neg: device int8 [M, K] with row
  * stride ldq (a multiple of 16). */
@@ -170,6 +183,10 @@ sq_status sq_stream_status(sq_stream_t stream);
 
 /* Static string naming a status code. */
 const char* sq_status_string(sq_status status);
+
+/* Description of the last CUDA error that made a call of this thread return
+ * SQ_ERR_CUDA ("no CUDA error" if none).  Static string; host only. */
+const char* sq_last_cuda_error(void);
 
 /* Test hook: the device-side wait budget in clock cycles (default about one
  * second).  0 restores the default.  Host only; affects later launches. */

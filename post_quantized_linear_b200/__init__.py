@@ -23,7 +23,7 @@ from . import _lib
 from ._lib import SegQuantError
 
 __all__ = ["QuantizedWeight", "SegQuantError", "calibrate", "quantize_weights", "linear",
-           "quantize_activations", "linear_accumulators", "stream_status", "qweight_sizes"]
+           "quantize_activations", "linear_from_codes", "linear_accumulators", "stream_status", "qweight_sizes"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -138,19 +138,44 @@ def linear(x: torch.Tensor, qw: QuantizedWeight, s_pos: torch.Tensor, s_neg: tor
     return out
 
 
+def linear_from_codes(q_pos: torch.Tensor, q_neg: torch.Tensor, qw: QuantizedWeight,
+                      s_pos: torch.Tensor, s_neg: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                      out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """Forward from pre-quantized DualScale codes (same result as ``linear``)."""
+    _check_2d(q_pos, "q_pos")
+    _check_2d(q_neg, "q_neg")
+    M, K = q_pos.shape
+    if q_neg.shape != q_pos.shape or q_neg.stride(0) != q_pos.stride(0):
+        raise ValueError("q_pos and q_neg must have the same shape and row stride")
+    if out is None:
+        out = torch.empty((M, qw.N), dtype=out_dtype, device=q_pos.device)
+    _check_2d(out, "out")
+    c, keep = qw.c_struct()
+    _lib.check("sq_linear_forward_codes", _lib.load().sq_linear_forward_codes(
+        _ptr(q_pos), _ptr(q_neg), q_pos.stride(0), M, K, ctypes.byref(c), _ptr(s_pos), _ptr(s_neg),
+        _ptr(bias), _ptr(out), _dtype_code(out.dtype), out.stride(0), _stream(stream)))
+    return out
+
+
 def quantize_activations(x: torch.Tensor, kseg: Sequence[int], s_pos: torch.Tensor,
-                         s_neg: torch.Tensor, stream=None):
-    """DualScale codes (q+, q-), int8 [M, K] each."""
+                         s_neg: torch.Tensor, out=None, stream=None):
+    """DualScale codes (q+, q-), int8 [M, K] each (row stride a multiple of 16)."""
     _check_2d(x, "x")
     M, K = x.shape
-    ldq = (K + 15) // 16 * 16
-    qp = torch.empty((M, ldq), dtype=torch.int8, device=x.device)
-    qn = torch.empty((M, ldq), dtype=torch.int8, device=x.device)
+    if out is None:
+        ldq = (K + 15) // 16 * 16
+        qp = torch.empty((M, ldq), dtype=torch.int8, device=x.device)[:, :K]
+        qn = torch.empty((M, ldq), dtype=torch.int8, device=x.device)[:, :K]
+    else:
+        qp, qn = out
+        if qp.stride(0) != qn.stride(0):
+            raise ValueError("q_pos and q_neg must share a row stride")
     seg, keep = _lib.segments(kseg)
     _lib.check("sq_quantize_activations", _lib.load().sq_quantize_activations(
         _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(seg), _ptr(s_pos),
-        _ptr(s_neg), _ptr(qp), _ptr(qn), ldq, _stream(stream)))
-    return qp[:, :K], qn[:, :K]
+        _ptr(s_neg), _ptr(qp), _ptr(qn), qp.stride(0), _stream(stream)))
+    return qp, qn
 
 
 def num_units(qw: QuantizedWeight) -> int:

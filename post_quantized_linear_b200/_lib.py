@@ -41,12 +41,15 @@ SIGNATURES = {
     "sq_quantize_weights": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp]),
     "sq_linear_forward": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp, c_vp,
                                   c_i32, c_i64, c_vp]),
+    "sq_linear_forward_codes": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp,
+                                        c_vp, c_i32, c_i64, c_vp]),
     "sq_quantize_activations": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp, c_vp, c_vp,
                                         c_vp, c_i64, c_vp]),
     "sq_linear_accumulators": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp,
                                        c_vp]),
     "sq_stream_status": (c_i32, [c_vp]),
     "sq_status_string": (ctypes.c_char_p, [c_i32]),
+    "sq_last_cuda_error": (ctypes.c_char_p, []),
     "sq_set_wait_budget": (None, [c_i64]),
 }
 
@@ -77,7 +80,10 @@ def status_string(code: int) -> str:
 class SegQuantError(RuntimeError):
     def __init__(self, fn: str, code: int):
         self.code = int(code)
-        super().__init__(f"{fn} failed: {status_string(code)}")
+        msg = f"{fn} failed: {status_string(code)}"
+        if self.code == SQ_ERR_CUDA:
+            msg += f" ({load().sq_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 def check(fn: str, code: int) -> None:

@@ -1,4 +1,4 @@
-// Fused DualScale / SegLinear quantized linear for sm_100a.
+// Fused DualScale / SegLinear quantized linear for sm_100a (W8A8 and W4A8).
 //
 // SegQuant ("SegQuant: A Semantics-Aware and Generalizable Quantization
 // Framework for Diffusion Models"), Spanish technical summary 2.B and Korean
@@ -6,26 +6,32 @@
 // with its own static scale; the products X+^ W^ and X-^ W^ run inside one
 // kernel ("BatchedGEMM") and are combined in a fused epilogue.  Section 2.A /
 // "SegLinear": every input segment carries its own activation and weight
-// scales.
+// scales.  W4A8 (Spanish technical summary 4, results): 4-bit weights.
 //
-// The pages give no kernel; this one is designed for B200:
-//   * warp 0      : TMA producer.  bf16/fp32 activation tiles (128 rows x 128 k,
-//                   128-byte swizzle) and int8 weight tiles (BN rows x 128 k).
-//   * warps 2..5  : quantizer.  Thread t owns tile row t: it reads its row of
-//                   the activation stage, splits by sign, rounds half-to-even
-//                   against each polarity's reciprocal scale and writes the two
-//                   int8 operand tiles (q+ and q-) in the UMMA K-major 128-byte
-//                   swizzled layout.
-//   * warp 1      : TMEM allocator and the single MMA-issuing thread.  Per
-//                   32-wide k step it issues two tcgen05.mma.kind::i8 (q+ W^T
-//                   and q- W^T) sharing the weight descriptor, into two int32
-//                   TMEM accumulators.  A unit (K segment, or 128-wide group
-//                   for int4 weights) ends with a commit; accumulators are
-//                   double-buffered across units (2 polarities x 2 buffers x BN
-//                   columns = 512 TMEM columns for BN = 128).
-//   * warps 6..13 : epilogue.  Per unit: tcgen05.ld of both accumulators,
-//                   t = fmaf(s-, F(acc-), s+ * F(acc+)), y = fmaf(sw[n], t, y);
-//                   after the last unit: + bias, convert, 16-byte stores.
+// The pages give no kernel; this one is designed for B200.  Persistent: one
+// CTA per SM walks output tiles (128 rows x BN columns) in a snake order, and
+// every ring below runs continuously across tiles.
+//   * warp 0       : TMA producer.  Activation tiles (128 rows x 128 k,
+//                    128-byte swizzle) or, for pre-quantized activations, the
+//                    two int8 code tiles; int8 weight tiles (BN x 128 k) or
+//                    packed int4 weight tiles (BN x 64 bytes).
+//   * warps 2..9   : operand producers.  Fused mode: thread t owns tile row
+//                    t % 128 and half of its k range; it splits each activation
+//                    by sign, rounds half-to-even against each polarity's
+//                    reciprocal scale and writes q+ and q- in the UMMA K-major
+//                    128-byte swizzled layout.  int4 weights: the packed tile
+//                    is sign-extended to int8 in the same layout.
+//   * warp 1       : TMEM allocator and the single MMA-issuing thread.  Per
+//                    32-wide k step, two tcgen05.mma.kind::i8 (q+ W^T, q- W^T)
+//                    share the weight descriptor and accumulate into two int32
+//                    TMEM accumulators.  A unit (K segment, or 128-wide group
+//                    for int4 weights) ends with a commit; with BN = 128 the
+//                    accumulators are double-buffered (2 x 2 x 128 = 512 TMEM
+//                    columns), so the epilogue of one unit or tile overlaps the
+//                    MMAs of the next.
+//   * warps 10..17 : epilogue.  tcgen05.ld of both accumulators;
+//                    t = fmaf(s-, F(acc-), s+ * F(acc+)), y = fmaf(sw[n], t, y);
+//                    after the last unit: + bias, convert, 16-byte stores.
 // Every pipeline wait is bounded; on expiry the CTA records SQ_STATUS_TIMEOUT,
 // lets in-flight copies and MMAs land, frees its TMEM and exits.
 #pragma once
@@ -40,17 +46,33 @@
 
 namespace sq {
 
-constexpr int BM = 128;        // token rows per tile (UMMA M)
-constexpr int BK = 128;        // k per pipeline stage (one 128-byte swizzle row of int8)
-constexpr int kWarps = 14;
-constexpr int kThreads = kWarps * 32;
-constexpr int kQuantWarp0 = 2;  // warps 2..5
-constexpr int kEpiWarp0 = 6;    // warps 6..13
+constexpr int BM = 128;  // token rows per tile (UMMA M)
+constexpr int BK = 128;  // k per pipeline stage (one 128-byte swizzle row of int8)
+constexpr int kProdWarp0 = 2;
+constexpr int kProdWarps = 8;
+constexpr int kEpiWarp0 = kProdWarp0 + kProdWarps;  // 10
+
+// Epilogue warps: 8 for one unit per tile (columns streamed from TMEM), 16
+// when partial outputs must stay in registers across units (32 columns per
+// thread).  Registers are granted in 4-warp groups, so 18 warps get at most
+// 96 registers per thread and 26 warps 72.
+__host__ __device__ constexpr int epi_warps(bool multi) { return multi ? 16 : 8; }
+__host__ __device__ constexpr int kernel_threads(bool multi) {
+  return (kEpiWarp0 + epi_warps(multi)) * 32;
+}
+
+// Source of the A operand.
+constexpr int ASRC_X = 0;      // activations, quantized inside the kernel
+constexpr int ASRC_CODES = 1;  // pre-quantized q+ / q- code tensors
 
 struct GemmArgs {
   int32_t M, N, K;
   int32_t num_kb;          // ceil(K / BK)
   int32_t bits;            // 8 or 4
+  int32_t n_full;          // number of full-width N tiles
+  int32_t tail;            // width of the last, narrower N tile (0: none)
+  int32_t m_tiles;         // ceil(M / BM)
+  int32_t num_tiles;
   SegBounds kseg;          // activation (and int8 weight) segments
   const float* s_pos;      // [J]
   const float* s_neg;      // [J]
@@ -62,29 +84,40 @@ struct GemmArgs {
   long long wait_budget;   // clock cycles per wait
 };
 
-template <int BN_, typename XT>
+constexpr int kStageBudget = 229376;  // 224 KiB of pipeline stages
+
+template <int BN_, int ASRC_, typename XT, bool W4_>
 struct GemmCfg {
   static constexpr int BN = BN_;
+  static constexpr int ASRC = ASRC_;
+  static constexpr bool W4 = W4_;
   static constexpr int XE = (int)sizeof(XT);
   static constexpr int X_EPB = 128 / XE;                 // elements per 128-byte box row
   static constexpr int X_BOXES = BK / X_EPB;             // boxes per stage (2 bf16, 4 fp32)
   static constexpr int X_BOX_BYTES = BM * 128;
-  static constexpr int X_STAGE = BM * BK * XE;
+  static constexpr int X_STAGE = (ASRC == ASRC_X) ? BM * BK * XE : 0;
+  static constexpr int WP_STAGE = W4 ? BN * (BK / 2) : 0;  // packed int4 rows of 64 bytes
   static constexpr int W_STAGE = BN * BK;
   static constexpr int Q_TILE = BM * BK;
   static constexpr int Q_STAGE = 2 * Q_TILE;
-  static constexpr int SX = 2;
-  static constexpr int SW = (XE == 2) ? 4 : 2;
-  static constexpr int SQ = (XE == 2) ? 3 : 2;
+  static constexpr bool BIG_X = (ASRC == ASRC_X) && XE == 4;
+  static constexpr int SX = (ASRC == ASRC_X) ? 2 : 0;
+  static constexpr int SWP = W4 ? (BIG_X ? 2 : 4) : 0;
+  static constexpr int SW = W4 ? (BIG_X ? 1 : 2)
+                               : (ASRC == ASRC_CODES ? (BN == 128 ? 4 : 3) : ((BIG_X || BN == 256) ? 2 : 4));
+  static constexpr int SQ = (kStageBudget - SX * X_STAGE - SWP * WP_STAGE - SW * W_STAGE) / Q_STAGE;
+  static constexpr int NBUF = (BN <= 128) ? 2 : 1;       // TMEM accumulator buffers
   static constexpr int OFF_X = 0;
-  static constexpr int OFF_W = OFF_X + SX * X_STAGE;
+  static constexpr int OFF_WP = OFF_X + SX * X_STAGE;
+  static constexpr int OFF_W = OFF_WP + SWP * WP_STAGE;
   static constexpr int OFF_Q = OFF_W + SW * W_STAGE;
   static constexpr int OFF_BAR = OFF_Q + SQ * Q_STAGE;
-  static constexpr int NUM_BARS = 2 * SX + 2 * SW + 2 * SQ + 4 + 1;
+  static constexpr int NUM_BARS = 2 * 2 + 2 * 4 + 2 * 4 + 2 * 8 + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static constexpr int TMEM_COLS = 4 * BN;                 // 2 polarities x 2 buffers
+  static constexpr int TMEM_COLS = 2 * BN * NBUF;
   static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
+  static_assert(SQ >= 2 && SQ <= 8 && SW >= 1 && SW <= 4 && SWP <= 4, "stage counts");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -139,6 +172,49 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, long l
   }
 }
 
+// Waits for the last completion of every stage of a ring that `issued` loads
+// were armed on (stage i % S, phase i / S).
+__device__ __forceinline__ void drain_ring(const uint64_t* full, int S, int issued,
+                                           long long budget) {
+  for (int s = 0; s < S; ++s) {
+    if (issued > s) {
+      const int last = ((issued - 1 - s) / S) * S + s;
+      wait_drain(smem_u32(full + s), (last / S) & 1, budget);
+    }
+  }
+}
+
+// ---------------------------------------------------------- tile schedule
+struct Tile {
+  int m0, n0, width;
+};
+
+// Tiles: full-width tiles first (row-major over (m, n)), then the narrower
+// last-column tiles.  Round `it` of CTA `cta` takes tile it*ncta + pos, with
+// pos reversed on odd rounds (snake) so that CTAs that drew short tiles in one
+// round draw long ones in the next.
+__device__ __forceinline__ bool tile_of(const GemmArgs& a, int it, int bn, Tile& t) {
+  const int ncta = gridDim.x;
+  const int pos = (it & 1) ? (ncta - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int idx = it * ncta + pos;
+  if (idx >= a.num_tiles) return false;
+  const int nfull_tiles = a.m_tiles * a.n_full;
+  if (idx < nfull_tiles) {
+    t.m0 = (idx / a.n_full) * BM;
+    t.n0 = (idx % a.n_full) * bn;
+    t.width = bn;
+  } else {
+    t.m0 = (idx - nfull_tiles) * BM;
+    t.n0 = a.n_full * bn;
+    t.width = a.tail;
+  }
+  return true;
+}
+
+__device__ __forceinline__ int num_rounds(const GemmArgs& a) {
+  return (a.num_tiles + gridDim.x - 1) / gridDim.x;
+}
+
 // ----------------------------------------------------- quantizer helpers
 // Reads 16 consecutive activations (k = 16c .. 16c+15) of tile row `row` from
 // a 128-byte-swizzled activation stage.
@@ -179,9 +255,10 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t a0, uint32_t a1, uint32_
   return __byte_perm(__byte_perm(a0, a1, 0x0040), __byte_perm(a2, a3, 0x0040), 0x5410);
 }
 
-// DualScale rounding (see quant_kernels.cuh for the argument): the fma adds the
-// exact product to 1.5*2^23, whose fp32 spacing is 1, so it rounds half to even
-// to an integer; fmin/fmax clamp to [0,127] / [-127,0] in the float domain.
+// DualScale rounding: the fma adds the exact product to 1.5*2^23, whose fp32
+// spacing is 1, so it rounds half to even to an integer (the offset is even,
+// so ties still go to even); fmin/fmax clamp to [0,127] / [-127,0] in the
+// float domain (monotone, so clamping commutes with the rounding).
 __device__ __forceinline__ void quantize16(const float (&v)[16], float rp, float rn, uint4& qp,
                                            uint4& qn) {
   uint32_t p[16], n[16];
@@ -200,6 +277,17 @@ __device__ __forceinline__ void quantize16(const float (&v)[16], float rp, float
   qn.w = low_bytes4(n[12], n[13], n[14], n[15]);
 }
 
+// Eight int4 codes (two per byte, low nibble = even k) -> eight int8 codes.
+// A nibble n in 0..15 sign-extends to n | 0xF0 when bit 3 is set: the bit,
+// multiplied by 30 (8 * 30 = 0xF0), lands in the high nibble of its own byte.
+__device__ __forceinline__ uint2 unpack8_int4(uint32_t w) {
+  uint32_t lo = w & 0x0F0F0F0Fu;
+  uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
+  lo |= (lo & 0x08080808u) * 30u;
+  hi |= (hi & 0x08080808u) * 30u;
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+
 __device__ __forceinline__ float rcp_or_zero(float s) { return s > 0.0f ? __frcp_rn(s) : 0.0f; }
 
 // Segment of the K block `kb` and whether it closes its unit.
@@ -212,27 +300,138 @@ __device__ __forceinline__ bool kb_closes_unit(const GemmArgs& a, int kb) {
   return (kb + 1) * BK >= a.kseg.b[j + 1];
 }
 
+// ------------------------------------------------------------- epilogue
+// Weight scales of 16 consecutive output channels for unit u.
+__device__ __forceinline__ void load_wscales16(const GemmArgs& a, int u, int j, int n,
+                                               float (&sw)[16]) {
+  if (a.bits == 8) {
+    const float4* s4 =
+        reinterpret_cast<const float4*>(static_cast<const float*>(a.wscales) + (int64_t)j * a.N + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = __ldg(s4 + i);
+      sw[4 * i] = t.x; sw[4 * i + 1] = t.y; sw[4 * i + 2] = t.z; sw[4 * i + 3] = t.w;
+    }
+  } else {
+    const __half* hs = static_cast<const __half*>(a.wscales);
+    const int G = a.K / 128;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sw[i] = __half2float(hs[(int64_t)(n + i) * G + u]);
+  }
+}
+
+// int32 -> fp32, round to nearest even.  With |v| < 2^22 (int4 units) the
+// magic-number form is exact: the pattern 0x4B400000 + v is the float
+// 1.5*2^23 + v, and the subtraction is exact.
+template <bool SMALL>
+__device__ __forceinline__ float acc_to_f32(uint32_t v) {
+  if constexpr (SMALL) return __uint_as_float(v + kMagicBits) - kMagic;
+  else return __int2float_rn((int)v);
+}
+
+// y (+)= sw * (s- F(acc-) + s+ F(acc+)) in the fixed fp32 order.
+template <bool SMALL>
+__device__ __forceinline__ void fold16(const uint32_t (&ap)[16], const uint32_t (&an)[16],
+                                       const float (&sw)[16], float sp, float sn, float* y) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float fp = acc_to_f32<SMALL>(ap[i]);
+    const float fn = acc_to_f32<SMALL>(an[i]);
+    const float t = __fmaf_rn(sn, fn, __fmul_rn(sp, fp));
+    y[i] = __fmaf_rn(sw[i], t, y[i]);
+  }
+}
+
+__device__ __forceinline__ void load_wscales8(const GemmArgs& a, int u, int j, int n,
+                                              float (&sw)[8]) {
+  if (a.bits == 8) {
+    const float4* s4 =
+        reinterpret_cast<const float4*>(static_cast<const float*>(a.wscales) + (int64_t)j * a.N + n);
+    const float4 t0 = __ldg(s4), t1 = __ldg(s4 + 1);
+    sw[0] = t0.x; sw[1] = t0.y; sw[2] = t0.z; sw[3] = t0.w;
+    sw[4] = t1.x; sw[5] = t1.y; sw[6] = t1.z; sw[7] = t1.w;
+  } else {
+    const __half* hs = static_cast<const __half*>(a.wscales);
+    const int G = a.K / 128;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sw[i] = __half2float(hs[(int64_t)(n + i) * G + u]);
+  }
+}
+
+template <bool SMALL>
+__device__ __forceinline__ void fold8(const uint32_t (&ap)[8], const uint32_t (&an)[8],
+                                      const float (&sw)[8], float sp, float sn, float* y) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float fp = acc_to_f32<SMALL>(ap[i]);
+    const float fn = acc_to_f32<SMALL>(an[i]);
+    const float t = __fmaf_rn(sn, fn, __fmul_rn(sp, fp));
+    y[i] = __fmaf_rn(sw[i], t, y[i]);
+  }
+}
+
+// + bias, convert, two (bf16) or four (fp32) 16-byte stores.
+template <bool Y_BF16>
+__device__ __forceinline__ void store16(const GemmArgs& a, int row, int n, float (&o)[16]) {
+  if (a.bias != nullptr) {
+    const float4* b4 = reinterpret_cast<const float4*>(a.bias + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = __ldg(b4 + i);
+      o[4 * i] = __fadd_rn(o[4 * i], t.x);
+      o[4 * i + 1] = __fadd_rn(o[4 * i + 1], t.y);
+      o[4 * i + 2] = __fadd_rn(o[4 * i + 2], t.z);
+      o[4 * i + 3] = __fadd_rn(o[4 * i + 3], t.w);
+    }
+  }
+  if constexpr (Y_BF16) {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.y) + (int64_t)row * a.ldy + n;
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+      pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    float* dst = static_cast<float*>(a.y) + (int64_t)row * a.ldy + n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      reinterpret_cast<float4*>(dst)[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  }
+}
+
 // ------------------------------------------------------------------ kernel
-template <int BN, typename XT, bool ACC_OUT, bool Y_BF16>
-__global__ void __launch_bounds__(kThreads, 1)
-    dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
+// MULTI: more than one unit per tile (several K segments, or int4 groups):
+// partial outputs stay in registers across units (BN = 128 only, 16 epilogue
+// warps).
+template <int BN, int ASRC, typename XT, bool W4, bool ACC_OUT, bool Y_BF16, bool MULTI>
+__global__ void __launch_bounds__(kernel_threads(MULTI), 1)
+    dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                          const __grid_constant__ CUtensorMap tmap_a2,
                           const __grid_constant__ CUtensorMap tmap_w,
                           const __grid_constant__ GemmArgs args) {
-  using C = GemmCfg<BN, XT>;
+  using C = GemmCfg<BN, ASRC, XT, W4>;
+  static_assert(!MULTI || BN == 128, "several units per tile need double-buffered TMEM");
+  static_assert(!W4 || MULTI, "int4 weights fold one unit per 128-wide group");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sm_x = smem + C::OFF_X;
+  uint8_t* sm_wp = smem + C::OFF_WP;
   uint8_t* sm_w = smem + C::OFF_W;
   uint8_t* sm_q = smem + C::OFF_Q;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full_x = bars;
-  uint64_t* empty_x = full_x + C::SX;
-  uint64_t* full_w = empty_x + C::SX;
-  uint64_t* empty_w = full_w + C::SW;
-  uint64_t* full_q = empty_w + C::SW;
-  uint64_t* empty_q = full_q + C::SQ;
-  uint64_t* tmem_full = empty_q + C::SQ;   // [2]
+  uint64_t* full_x = bars;                 // [2]
+  uint64_t* empty_x = full_x + 2;          // [2]
+  uint64_t* full_wp = empty_x + 2;         // [4]
+  uint64_t* empty_wp = full_wp + 4;        // [4]
+  uint64_t* full_w = empty_wp + 4;         // [4]
+  uint64_t* empty_w = full_w + 4;          // [4]
+  uint64_t* full_q = empty_w + 4;          // [8]
+  uint64_t* empty_q = full_q + 8;          // [8]
+  uint64_t* tmem_full = empty_q + 8;       // [2]
   uint64_t* tmem_empty = tmem_full + 2;    // [2]
   uint64_t* drain_bar = tmem_empty + 2;    // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -240,15 +439,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  const int n0 = blockIdx.x * BN;
   const long long budget = args.wait_budget;
+  constexpr bool PROD_Q = (ASRC == ASRC_X);   // producer warps write the Q tiles
+  constexpr bool PROD_W = W4;                 // producer warps write the W tiles
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::SX; ++i) { mbar_init(smem_u32(full_x + i), 1); mbar_init(smem_u32(empty_x + i), 4); }
-    for (int i = 0; i < C::SW; ++i) { mbar_init(smem_u32(full_w + i), 1); mbar_init(smem_u32(empty_w + i), 1); }
-    for (int i = 0; i < C::SQ; ++i) { mbar_init(smem_u32(full_q + i), 4); mbar_init(smem_u32(empty_q + i), 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(tmem_full + i), 1); mbar_init(smem_u32(tmem_empty + i), 8); }
+    for (int i = 0; i < C::SX; ++i) {
+      mbar_init(smem_u32(full_x + i), 1);
+      mbar_init(smem_u32(empty_x + i), kProdWarps);
+    }
+    for (int i = 0; i < C::SWP; ++i) {
+      mbar_init(smem_u32(full_wp + i), 1);
+      mbar_init(smem_u32(empty_wp + i), kProdWarps);
+    }
+    for (int i = 0; i < C::SW; ++i) {
+      mbar_init(smem_u32(full_w + i), PROD_W ? kProdWarps : 1);
+      mbar_init(smem_u32(empty_w + i), 1);
+    }
+    for (int i = 0; i < C::SQ; ++i) {
+      mbar_init(smem_u32(full_q + i), PROD_Q ? kProdWarps : 1);
+      mbar_init(smem_u32(empty_q + i), 1);
+    }
+    for (int i = 0; i < C::NBUF; ++i) {
+      mbar_init(smem_u32(tmem_full + i), 1);
+      mbar_init(smem_u32(tmem_empty + i), epi_warps(MULTI));
+    }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -262,78 +477,99 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = args.num_kb;
+  const int rounds = num_rounds(args);
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_x);
+      tma_prefetch_desc(&tmap_a);
+      if constexpr (ASRC == ASRC_CODES) tma_prefetch_desc(&tmap_a2);
       tma_prefetch_desc(&tmap_w);
-      int issued_x = 0, issued_w = 0;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int sx = issued_x % C::SX;
-        const uint32_t px = (issued_x / C::SX) & 1;
-        if (!wait1(smem_u32(empty_x + sx), px ^ 1, abort_flag, budget)) break;
-        mbar_arrive_expect_tx(smem_u32(full_x + sx), C::X_STAGE);
-        for (int b = 0; b < C::X_BOXES; ++b)
-          tma_load_2d(smem_u32(sm_x + sx * C::X_STAGE + b * C::X_BOX_BYTES), &tmap_x,
-                      smem_u32(full_x + sx), kb * BK + b * C::X_EPB, m0);
-        ++issued_x;
-        const int sw = issued_w % C::SW;
-        const uint32_t pw = (issued_w / C::SW) & 1;
-        if (!wait1(smem_u32(empty_w + sw), pw ^ 1, abort_flag, budget)) break;
-        mbar_arrive_expect_tx(smem_u32(full_w + sw), C::W_STAGE);
-        tma_load_2d(smem_u32(sm_w + sw * C::W_STAGE), &tmap_w, smem_u32(full_w + sw), kb * BK, n0);
-        ++issued_w;
+      int ca = 0, cw = 0;
+      bool ok = true;
+      for (int it = 0; it < rounds && ok; ++it) {
+        Tile t;
+        if (!tile_of(args, it, BN, t)) continue;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if constexpr (ASRC == ASRC_X) {
+            const int s = ca % C::SX;
+            if (!(ok = wait1(smem_u32(empty_x + s), ((ca / C::SX) & 1) ^ 1, abort_flag, budget))) break;
+            mbar_arrive_expect_tx(smem_u32(full_x + s), C::X_STAGE);
+            for (int b = 0; b < C::X_BOXES; ++b)
+              tma_load_2d(smem_u32(sm_x + s * C::X_STAGE + b * C::X_BOX_BYTES), &tmap_a,
+                          smem_u32(full_x + s), kb * BK + b * C::X_EPB, t.m0);
+          } else {
+            const int s = ca % C::SQ;
+            if (!(ok = wait1(smem_u32(empty_q + s), ((ca / C::SQ) & 1) ^ 1, abort_flag, budget))) break;
+            mbar_arrive_expect_tx(smem_u32(full_q + s), C::Q_STAGE);
+            tma_load_2d(smem_u32(sm_q + s * C::Q_STAGE), &tmap_a, smem_u32(full_q + s), kb * BK, t.m0);
+            tma_load_2d(smem_u32(sm_q + s * C::Q_STAGE + C::Q_TILE), &tmap_a2, smem_u32(full_q + s),
+                        kb * BK, t.m0);
+          }
+          ++ca;
+          if constexpr (W4) {
+            const int s = cw % C::SWP;
+            if (!(ok = wait1(smem_u32(empty_wp + s), ((cw / C::SWP) & 1) ^ 1, abort_flag, budget))) break;
+            mbar_arrive_expect_tx(smem_u32(full_wp + s), C::WP_STAGE);
+            tma_load_2d(smem_u32(sm_wp + s * C::WP_STAGE), &tmap_w, smem_u32(full_wp + s),
+                        kb * (BK / 2), t.n0);
+          } else {
+            const int s = cw % C::SW;
+            if (!(ok = wait1(smem_u32(empty_w + s), ((cw / C::SW) & 1) ^ 1, abort_flag, budget))) break;
+            mbar_arrive_expect_tx(smem_u32(full_w + s), C::W_STAGE);
+            tma_load_2d(smem_u32(sm_w + s * C::W_STAGE), &tmap_w, smem_u32(full_w + s), kb * BK, t.n0);
+          }
+          ++cw;
+        }
       }
       // Let every copy this thread started land before the CTA can exit.
-      for (int s = 0; s < C::SX; ++s) {
-        if (issued_x > s) {
-          const int last = ((issued_x - 1 - s) / C::SX) * C::SX + s;
-          wait_drain(smem_u32(full_x + s), (last / C::SX) & 1, budget);
-        }
-      }
-      for (int s = 0; s < C::SW; ++s) {
-        if (issued_w > s) {
-          const int last = ((issued_w - 1 - s) / C::SW) * C::SW + s;
-          wait_drain(smem_u32(full_w + s), (last / C::SW) & 1, budget);
-        }
-      }
+      if constexpr (ASRC == ASRC_X) drain_ring(full_x, C::SX, ca, budget);
+      else drain_ring(full_q, C::SQ, ca, budget);
+      if constexpr (W4) drain_ring(full_wp, C::SWP, cw, budget);
+      else drain_ring(full_w, C::SW, cw, budget);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(BM, BN);
-      int unit = 0;
-      bool unit_open = false;
-      uint32_t d_pos = 0;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!unit_open) {
-          const int b = unit & 1;
-          if (!wait1(smem_u32(tmem_empty + b), ((unit >> 1) & 1) ^ 1, abort_flag, budget)) break;
+      int cq = 0, cw = 0, ug = 0;
+      bool ok = true;
+      for (int it = 0; it < rounds && ok; ++it) {
+        Tile t;
+        if (!tile_of(args, it, BN, t)) continue;
+        const uint32_t idesc = idesc_i8(BM, t.width);
+        bool unit_open = false;
+        uint32_t d_pos = 0;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!unit_open) {
+            const int b = ug % C::NBUF;
+            if (!(ok = wait1(smem_u32(tmem_empty + b), ((ug / C::NBUF) & 1) ^ 1, abort_flag, budget))) break;
+            tc_fence_after();
+            d_pos = tmem_base + (uint32_t)(b * 2 * BN);
+          }
+          const int sw = cw % C::SW, sq = cq % C::SQ;
+          if (!(ok = wait1(smem_u32(full_w + sw), (cw / C::SW) & 1, abort_flag, budget))) break;
+          if (!(ok = wait1(smem_u32(full_q + sq), (cq / C::SQ) & 1, abort_flag, budget))) break;
           tc_fence_after();
-          d_pos = tmem_base + (uint32_t)(b * 2 * BN);
-        }
-        const int sw = kb % C::SW, sq = kb % C::SQ;
-        if (!wait1(smem_u32(full_w + sw), (kb / C::SW) & 1, abort_flag, budget)) break;
-        if (!wait1(smem_u32(full_q + sq), (kb / C::SQ) & 1, abort_flag, budget)) break;
-        tc_fence_after();
-        const uint32_t a_p = smem_u32(sm_q + sq * C::Q_STAGE);
-        const uint32_t a_n = a_p + C::Q_TILE;
-        const uint32_t b_w = smem_u32(sm_w + sw * C::W_STAGE);
+          const uint32_t a_p = smem_u32(sm_q + sq * C::Q_STAGE);
+          const uint32_t a_n = a_p + C::Q_TILE;
+          const uint32_t b_w = smem_u32(sm_w + sw * C::W_STAGE);
 #pragma unroll
-        for (int ks = 0; ks < BK / 32; ++ks) {
-          const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
-          const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
-          umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
-          umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
-        }
-        unit_open = true;
-        umma_commit(smem_u32(empty_w + sw));
-        umma_commit(smem_u32(empty_q + sq));
-        if (kb_closes_unit(args, kb)) {
-          umma_commit(smem_u32(tmem_full + (unit & 1)));
-          ++unit;
-          unit_open = false;
+          for (int ks = 0; ks < BK / 32; ++ks) {
+            const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
+            const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
+            umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
+            umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
+          }
+          unit_open = true;
+          umma_commit(smem_u32(empty_w + sw));
+          umma_commit(smem_u32(empty_q + sq));
+          ++cw;
+          ++cq;
+          if (kb_closes_unit(args, kb)) {
+            umma_commit(smem_u32(tmem_full + (ug % C::NBUF)));
+            ++ug;
+            unit_open = false;
+          }
         }
       }
       // All MMAs this thread issued have landed once the drain barrier flips.
@@ -341,148 +577,175 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(smem_u32(drain_bar), 0, budget);
     }
   } else if (warp < kEpiWarp0) {
-    // -------------------------------------------------------- quantizer
-    const int row = threadIdx.x - kQuantWarp0 * 32;  // 0..127, tile row
-    int cur_seg = -1;
-    float rp = 0.0f, rn = 0.0f;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int j = kb_segment(args, kb);
-      if (j != cur_seg) {
-        cur_seg = j;
-        rp = rcp_or_zero(__ldg(args.s_pos + j));
-        rn = rcp_or_zero(__ldg(args.s_neg + j));
-      }
-      const int sx = kb % C::SX, sq = kb % C::SQ;
-      if (!wait_warp(smem_u32(full_x + sx), (kb / C::SX) & 1, abort_flag, budget)) break;
-      if (!wait_warp(smem_u32(empty_q + sq), ((kb / C::SQ) & 1) ^ 1, abort_flag, budget)) break;
-      const uint8_t* xs = sm_x + sx * C::X_STAGE;
-      uint8_t* qp = sm_q + sq * C::Q_STAGE + row * 128;
-      uint8_t* qn = qp + C::Q_TILE;
+    // ------------------------------------------------- operand producers
+    if constexpr (PROD_Q || PROD_W) {
+      const int t_id = threadIdx.x - kProdWarp0 * 32;  // 0..255
+      const int row = t_id & (BM - 1);                 // tile row (quantizer)
+      const int c0 = (t_id >> 7) * 4;                  // first of its four 16-wide chunks
+      int cx = 0, cq = 0, cwp = 0, cw = 0;
+      int cur_seg = -1;
+      float rp = 0.0f, rn = 0.0f;
+      bool ok = true;
+      for (int it = 0; it < rounds && ok; ++it) {
+        Tile t;
+        if (!tile_of(args, it, BN, t)) continue;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if constexpr (PROD_Q) {
+            const int j = kb_segment(args, kb);
+            if (j != cur_seg) {
+              cur_seg = j;
+              rp = rcp_or_zero(__ldg(args.s_pos + j));
+              rn = rcp_or_zero(__ldg(args.s_neg + j));
+            }
+            const int sx = cx % C::SX, sq = cq % C::SQ;
+            if (!(ok = wait_warp(smem_u32(full_x + sx), (cx / C::SX) & 1, abort_flag, budget))) break;
+            if (!(ok = wait_warp(smem_u32(empty_q + sq), ((cq / C::SQ) & 1) ^ 1, abort_flag, budget))) break;
+            const uint8_t* xs = sm_x + sx * C::X_STAGE;
+            uint8_t* qp = sm_q + sq * C::Q_STAGE + row * 128;
+            uint8_t* qn = qp + C::Q_TILE;
 #pragma unroll 2
-      for (int c = 0; c < 8; ++c) {
-        float v[16];
-        load_row16<XT>(xs, row, c, v);
-        uint4 up, un;
-        quantize16(v, rp, rn, up, un);
-        const int off = (c ^ (row & 7)) << 4;
-        *reinterpret_cast<uint4*>(qp + off) = up;
-        *reinterpret_cast<uint4*>(qn + off) = un;
+            for (int c = c0; c < c0 + 4; ++c) {
+              float v[16];
+              load_row16<XT>(xs, row, c, v);
+              uint4 up, un;
+              quantize16(v, rp, rn, up, un);
+              const int off = (c ^ (row & 7)) << 4;
+              *reinterpret_cast<uint4*>(qp + off) = up;
+              *reinterpret_cast<uint4*>(qn + off) = un;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(empty_x + sx));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(full_q + sq));
+            ++cx;
+            ++cq;
+          }
+          if constexpr (PROD_W) {
+            const int sp_ = cwp % C::SWP, sw = cw % C::SW;
+            if (!(ok = wait_warp(smem_u32(full_wp + sp_), (cwp / C::SWP) & 1, abort_flag, budget))) break;
+            if (!(ok = wait_warp(smem_u32(empty_w + sw), ((cw / C::SW) & 1) ^ 1, abort_flag, budget))) break;
+            const uint8_t* src = sm_wp + sp_ * C::WP_STAGE;
+            uint8_t* dst = sm_w + sw * C::W_STAGE;
+#pragma unroll
+            for (int i = 0; i < (BN * 4) / (kProdWarps * 32); ++i) {
+              const int task = i * (kProdWarps * 32) + t_id;
+              const int n = task >> 2, q = task & 3;   // row, 16-byte quarter of the packed row
+              const uint4 pk = *reinterpret_cast<const uint4*>(src + n * 64 + q * 16);
+              const uint2 e0 = unpack8_int4(pk.x), e1 = unpack8_int4(pk.y);
+              const uint2 e2 = unpack8_int4(pk.z), e3 = unpack8_int4(pk.w);
+              uint8_t* drow = dst + n * 128;
+              *reinterpret_cast<uint4*>(drow + (((2 * q) ^ (n & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+              *reinterpret_cast<uint4*>(drow + (((2 * q + 1) ^ (n & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(empty_wp + sp_));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(full_w + sw));
+            ++cwp;
+            ++cw;
+          }
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(empty_x + sx));
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(full_q + sq));
     }
   } else {
     // --------------------------------------------------------- epilogue
-    constexpr int HALF = BN / 2;
+    constexpr int HALF = BN / (epi_warps(MULTI) / 4);   // columns per epilogue thread
     const int quad = warp & 3;
     const int half = (warp - kEpiWarp0) >> 2;
-    const int row = m0 + quad * 32 + lane;
-    const int col0 = n0 + half * HALF;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    float y[HALF];
-#pragma unroll
-    for (int i = 0; i < HALF; ++i) y[i] = 0.0f;
-    const int num_units = (args.bits == 4) ? num_kb : args.kseg.count;
-    const int G = args.K / 128;
+    const int units = (args.bits == 4) ? num_kb : args.kseg.count;
+    int ug = 0;
     bool ok = true;
-    for (int u = 0; u < num_units; ++u) {
-      const int b = u & 1;
-      if (!wait_warp(smem_u32(tmem_full + b), (u >> 1) & 1, abort_flag, budget)) { ok = false; break; }
-      tc_fence_after();
-      const int j = (args.bits == 4) ? args.kseg.segment_of(u * 128) : u;
-      const float sp = __ldg(args.s_pos + j), sn = __ldg(args.s_neg + j);
+    for (int it = 0; it < rounds && ok; ++it) {
+      Tile t;
+      if (!tile_of(args, it, BN, t)) continue;
+      const int row = t.m0 + quad * 32 + lane;
+      const int c_lo = half * HALF;                 // first tile column of this warp
+      if constexpr (MULTI || ACC_OUT) {
+        float y[MULTI && !ACC_OUT ? HALF : 1];
 #pragma unroll
-      for (int c = 0; c < HALF / 16; ++c) {
-        uint32_t ap[16], an[16];
-        const uint32_t col = (uint32_t)(b * 2 * BN + half * HALF + c * 16);
-        tmem_ld16(t_lane + col, ap);
-        tmem_ld16(t_lane + col + BN, an);
-        tmem_wait_ld();
-        const int n = col0 + c * 16;
-        if constexpr (ACC_OUT) {
-          if (row < args.M && n < args.N) {
-            int32_t* dp = args.acc_out + (((int64_t)u * 2 + 0) * args.M + row) * args.N + n;
-            int32_t* dn = args.acc_out + (((int64_t)u * 2 + 1) * args.M + row) * args.N + n;
+        for (int i = 0; i < (MULTI && !ACC_OUT ? HALF : 1); ++i) y[i] = 0.0f;
+        for (int u = 0; u < units; ++u) {
+          const int b = ug % C::NBUF;
+          if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / C::NBUF) & 1, abort_flag, budget))) break;
+          tc_fence_after();
+          const int j = (args.bits == 4) ? args.kseg.segment_of(u * 128) : u;
+          const float sp = __ldg(args.s_pos + j), sn = __ldg(args.s_neg + j);
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              *reinterpret_cast<uint4*>(dp + i) = make_uint4(ap[i], ap[i + 1], ap[i + 2], ap[i + 3]);
-              *reinterpret_cast<uint4*>(dn + i) = make_uint4(an[i], an[i + 1], an[i + 2], an[i + 3]);
-            }
-          }
-        } else {
-          float sw[16];
-          if (n < args.N) {
-            if (args.bits == 8) {
-              const float4* s4 = reinterpret_cast<const float4*>(
-                  static_cast<const float*>(args.wscales) + (int64_t)j * args.N + n);
+          for (int c = 0; c < HALF / 8; ++c) {
+            if (c_lo + c * 8 < t.width) {
+              uint32_t ap[8], an[8];
+              const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 8);
+              tmem_ld8(t_lane + col, ap);
+              tmem_ld8(t_lane + col + BN, an);
+              tmem_wait_ld();
+              const int n = t.n0 + c_lo + c * 8;
+              if constexpr (ACC_OUT) {
+                if (row < args.M) {
+                  int32_t* dp = args.acc_out + (((int64_t)u * 2 + 0) * args.M + row) * args.N + n;
+                  int32_t* dn = args.acc_out + (((int64_t)u * 2 + 1) * args.M + row) * args.N + n;
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 t = __ldg(s4 + i);
-                sw[4 * i] = t.x; sw[4 * i + 1] = t.y; sw[4 * i + 2] = t.z; sw[4 * i + 3] = t.w;
+                  for (int i = 0; i < 8; i += 4) {
+                    *reinterpret_cast<uint4*>(dp + i) = make_uint4(ap[i], ap[i + 1], ap[i + 2], ap[i + 3]);
+                    *reinterpret_cast<uint4*>(dn + i) = make_uint4(an[i], an[i + 1], an[i + 2], an[i + 3]);
+                  }
+                }
+              } else {
+                float sw[8];
+                load_wscales8(args, u, j, n, sw);
+                fold8<W4>(ap, an, sw, sp, sn, y + c * 8);
               }
-            } else {
-              const __half* hs = static_cast<const __half*>(args.wscales);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) sw[i] = __half2float(hs[(int64_t)(n + i) * G + u]);
             }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sw[i] = 0.0f;
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(tmem_empty + b));
+          ++ug;
+        }
+        if constexpr (!ACC_OUT) {
+          if (ok && row < args.M) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float fp = __int2float_rn((int)ap[i]);
-            const float fn = __int2float_rn((int)an[i]);
-            const float t = __fmaf_rn(sn, fn, __fmul_rn(sp, fp));
-            y[c * 16 + i] = __fmaf_rn(sw[i], t, y[c * 16 + i]);
+            for (int c = 0; c < HALF / 16; ++c) {
+              if (c_lo + c * 16 < t.width) {
+                float o[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = y[c * 16 + i];
+                store16<Y_BF16>(args, row, t.n0 + c_lo + c * 16, o);
+              }
+            }
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(tmem_empty + b));
-    }
-    if constexpr (!ACC_OUT) {
-      if (ok && row < args.M) {
-#pragma unroll
+      } else {
+        // One unit per tile: stream column chunks from TMEM straight to memory.
+        const int b = ug % C::NBUF;
+        if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / C::NBUF) & 1, abort_flag, budget))) break;
+        tc_fence_after();
+        const float sp = __ldg(args.s_pos), sn = __ldg(args.s_neg);
+#pragma unroll 1
         for (int c = 0; c < HALF / 16; ++c) {
-          const int n = col0 + c * 16;
-          if (n < args.N) {
-            float o[16];
+          if (c_lo + c * 16 < t.width) {
+            uint32_t ap[16], an[16];
+            const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 16);
+            tmem_ld16(t_lane + col, ap);
+            tmem_ld16(t_lane + col + BN, an);
+            tmem_wait_ld();
+            if (row < args.M) {
+              const int n = t.n0 + c_lo + c * 16;
+              float sw[16], o[16];
+              load_wscales16(args, 0, 0, n, sw);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = y[c * 16 + i];
-            if (args.bias != nullptr) {
-              const float4* b4 = reinterpret_cast<const float4*>(args.bias + n);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 t = __ldg(b4 + i);
-                o[4 * i] = __fadd_rn(o[4 * i], t.x);
-                o[4 * i + 1] = __fadd_rn(o[4 * i + 1], t.y);
-                o[4 * i + 2] = __fadd_rn(o[4 * i + 2], t.z);
-                o[4 * i + 3] = __fadd_rn(o[4 * i + 3], t.w);
-              }
-            }
-            if constexpr (Y_BF16) {
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.y) + (int64_t)row * args.ldy + n;
-              uint32_t pk[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
-                pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
-              }
-              reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            } else {
-              float* dst = static_cast<float*>(args.y) + (int64_t)row * args.ldy + n;
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                reinterpret_cast<float4*>(dst)[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+              for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+              fold16<false>(ap, an, sw, sp, sn, o);
+              store16<Y_BF16>(args, row, n, o);
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(tmem_empty + b));
+        ++ug;
       }
     }
   }

@@ -144,48 +144,63 @@ __device__ __forceinline__ uint32_t pack4_low(uint32_t a0, uint32_t a1, uint32_t
   return __byte_perm(lo, hi, 0x5410);
 }
 
-// One thread per 8 consecutive elements of a row (one 16-byte bf16 vector, or
-// two fp32 vectors); 8-byte stores of each code tensor.
+// Loads 16 consecutive activations widened to fp32 (two bf16 or four fp32
+// 16-byte vectors).
+template <typename XT>
+__device__ __forceinline__ void load16(const XT* p, float (&v)[16]) {
+  if constexpr (Vec<XT>::n == 8) {
+    float a[8], b[8];
+    Vec<XT>::load(p, a);
+    Vec<XT>::load(p + 8, b);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { v[i] = a[i]; v[8 + i] = b[i]; }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float a[4];
+      Vec<XT>::load(p + 4 * h, a);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[4 * h + i] = a[i];
+    }
+  }
+}
+
+// blockDim = (32, 8): lane x owns the 16-element group blockIdx.x*32 + x of
+// every row it visits (rows blockIdx.y*8 + y, stepping by gridDim.y*8), so its
+// segment and reciprocal scales are fixed; a warp reads 1 KiB (bf16) and
+// writes 512 bytes of each code tensor per row.
 template <typename XT>
 __global__ void __launch_bounds__(256) quantize_activations_kernel(
-    const XT* __restrict__ x, int64_t M, int64_t K, int64_t ldx, SegBounds kseg,
+    const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
     int8_t* __restrict__ q_neg, int64_t ldq) {
-  const int64_t groups_per_row = K / 8;
-  const int64_t total = M * groups_per_row;
-  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
-       g += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t m = g / groups_per_row;
-    const int64_t k = (g - m * groups_per_row) * 8;
-    const int j = kseg.segment_of((int32_t)k);
-    const float sp = __ldg(s_pos + j), sn = __ldg(s_neg + j);
-    const float rp = sp > 0.0f ? __frcp_rn(sp) : 0.0f;
-    const float rn = sn > 0.0f ? __frcp_rn(sn) : 0.0f;
-    float v[8];
-    if constexpr (Vec<XT>::n == 8) {
-      Vec<XT>::load(x + m * ldx + k, v);
-    } else {
-      float a[4], b[4];
-      Vec<XT>::load(x + m * ldx + k, a);
-      Vec<XT>::load(x + m * ldx + k + 4, b);
+  const int32_t k = (blockIdx.x * 32 + threadIdx.x) * 16;
+  if (k >= K) return;
+  const int j = kseg.segment_of(k);
+  const float rp = s_pos[j] > 0.0f ? __frcp_rn(s_pos[j]) : 0.0f;
+  const float rn = s_neg[j] > 0.0f ? __frcp_rn(s_neg[j]) : 0.0f;
+  const int32_t step = gridDim.y * 8;
+  for (int32_t m = blockIdx.y * 8 + threadIdx.y; m < M; m += step) {
+    float v[16];
+    load16<XT>(x + (int64_t)m * ldx + k, v);
+    uint32_t p[16], n[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) { v[i] = a[i]; v[4 + i] = b[i]; }
-    }
-    uint32_t p[8], n[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { p[i] = code_pos(v[i], rp); n[i] = code_neg(v[i], rn); }
-    uint2 up, un;
-    up.x = pack4_low(p[0], p[1], p[2], p[3]); up.y = pack4_low(p[4], p[5], p[6], p[7]);
-    un.x = pack4_low(n[0], n[1], n[2], n[3]); un.y = pack4_low(n[4], n[5], n[6], n[7]);
-    *reinterpret_cast<uint2*>(q_pos + m * ldq + k) = up;
-    *reinterpret_cast<uint2*>(q_neg + m * ldq + k) = un;
+    for (int i = 0; i < 16; ++i) { p[i] = code_pos(v[i], rp); n[i] = code_neg(v[i], rn); }
+    uint4 up, un;
+    up.x = pack4_low(p[0], p[1], p[2], p[3]);   up.y = pack4_low(p[4], p[5], p[6], p[7]);
+    up.z = pack4_low(p[8], p[9], p[10], p[11]); up.w = pack4_low(p[12], p[13], p[14], p[15]);
+    un.x = pack4_low(n[0], n[1], n[2], n[3]);   un.y = pack4_low(n[4], n[5], n[6], n[7]);
+    un.z = pack4_low(n[8], n[9], n[10], n[11]); un.w = pack4_low(n[12], n[13], n[14], n[15]);
+    *reinterpret_cast<uint4*>(q_pos + (int64_t)m * ldq + k) = up;
+    *reinterpret_cast<uint4*>(q_neg + (int64_t)m * ldq + k) = un;
   }
 }
 
 // ------------------------------------------------------ weight quantization
 // int8: one warp per (output channel n, K segment j).  Pass 1: |W| max by
 // warp shuffles; s = max/127; r = 1/s.  Pass 2: codes with the same magic
-// rounding, clamp to +-127.
+// rounding, clamp to +-127, sixteen codes per 16-byte store (segment bounds
+// are multiples of 128 and K of 16).
 template <typename WT>
 __global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
     const WT* __restrict__ w, int64_t N, int64_t K, int64_t ldw, SegBounds kseg,
@@ -200,14 +215,14 @@ __global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
   const WT* row = w + n * ldw;
   float amax = 0.0f;
   bool bad = false;
-  for (int32_t k = k0 + lane * 4; k < k1; k += 128) {
+  for (int32_t k = k0 + lane * 16; k < k1; k += 512) {
+    float v[16];
+    load16<WT>(row + k, v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (k + i < k1) {
-        const float a = fabsf(to_f32(row[k + i]));
-        bad |= !(a <= 3.4028234663852886e38f);
-        amax = fmaxf(amax, a);
-      }
+    for (int i = 0; i < 16; ++i) {
+      const float a = fabsf(v[i]);
+      bad |= !(a <= 3.4028234663852886e38f);
+      amax = fmaxf(amax, a);
     }
   }
 #pragma unroll
@@ -216,16 +231,17 @@ __global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
   const float s = amax / 127.0f;
   const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
   if (lane == 0) scales[(int64_t)j * N + n] = s;
-  for (int32_t k = k0 + lane * 4; k < k1; k += 128) {
+  for (int32_t k = k0 + lane * 16; k < k1; k += 512) {
+    float v[16];
+    load16<WT>(row + k, v);
+    uint32_t c[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (k + i < k1) {
-        const float v = to_f32(row[k + i]);
-        float t = fmaf(v, r, kMagic);
-        t = fminf(fmaxf(t, kMagic - 127.0f), kMagic + 127.0f);
-        codes[n * K + k + i] = (int8_t)(__float_as_uint(t) & 0xFFu);
-      }
-    }
+    for (int i = 0; i < 16; ++i)
+      c[i] = __float_as_uint(fminf(fmaxf(fmaf(v[i], r, kMagic), kMagic - 127.0f), kMagic + 127.0f));
+    uint4 out;
+    out.x = pack4_low(c[0], c[1], c[2], c[3]);   out.y = pack4_low(c[4], c[5], c[6], c[7]);
+    out.z = pack4_low(c[8], c[9], c[10], c[11]); out.w = pack4_low(c[12], c[13], c[14], c[15]);
+    *reinterpret_cast<uint4*>(codes + n * K + k) = out;
   }
 }
 

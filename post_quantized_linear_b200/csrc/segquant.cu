@@ -5,9 +5,12 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "segquant.h"
 
@@ -56,7 +59,13 @@ sq_status check_nseg(const sq_segments* s, int64_t N) {
   return SQ_OK;
 }
 
-sq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+sq_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SQ_OK;
+  g_last_cuda_error = e;
+  return SQ_ERR_CUDA;
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -76,7 +85,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2D row-major tensor, 128-byte swizzled boxes of box_inner x box_rows.
 sq_status make_tmap(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
                     uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
-                    uint32_t box_rows) {
+                    uint32_t box_rows,
+                    CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (fn == nullptr) return SQ_ERR_CUDA;
   cuuint64_t dims[2] = {inner, rows};
@@ -84,7 +94,7 @@ sq_status make_tmap(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SQ_OK : SQ_ERR_CUDA;
 }
@@ -107,52 +117,132 @@ sq_status check_qweight(const sq_qweight* w, int64_t K, SegBounds* kseg) {
   return SQ_OK;
 }
 
-template <int BN, typename XT, bool ACC, bool YB>
-sq_status launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const sq::GemmArgs& a,
-                      cudaStream_t stream) {
-  using C = sq::GemmCfg<BN, XT>;
-  auto kern = sq::dualscale_gemm_kernel<BN, XT, ACC, YB>;
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+template <int BN, int ASRC, typename XT, bool W4, bool ACC, bool YB, bool MULTI>
+sq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tw,
+                      sq::GemmArgs a, cudaStream_t stream) {
+  using C = sq::GemmCfg<BN, ASRC, XT, W4>;
+  auto kern = sq::dualscale_gemm_kernel<BN, ASRC, XT, W4, ACC, YB, MULTI>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e != cudaSuccess) return SQ_ERR_CUDA;
-  dim3 grid((a.N + BN - 1) / BN, (a.M + sq::BM - 1) / sq::BM);
-  kern<<<grid, sq::kThreads, C::SMEM_BYTES, stream>>>(tx, tw, a);
+  if (e != cudaSuccess) return cuda_status(e);
+  a.n_full = a.N / BN;
+  a.tail = a.N % BN;
+  a.m_tiles = (a.M + sq::BM - 1) / sq::BM;
+  a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
+  int grid = num_sms();
+  if (grid > a.num_tiles) grid = a.num_tiles;
+  kern<<<grid, sq::kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(ta, ta2, tw, a);
   return cuda_status(cudaGetLastError());
 }
 
-sq_status gemm_common(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+// Picks the output variant: raw accumulators (test surface) or fp32 / bf16 Y.
+template <int BN, int ASRC, typename XT, bool W4, bool MULTI>
+sq_status launch_out(bool acc, bool y_bf16, const CUtensorMap& ta, const CUtensorMap& ta2,
+                     const CUtensorMap& tw, const sq::GemmArgs& a, cudaStream_t stream) {
+  if constexpr (MULTI) {
+    if (acc) return launch_gemm<BN, ASRC, XT, W4, true, false, true>(ta, ta2, tw, a, stream);
+  }
+  if (acc) return SQ_ERR_UNSUPPORTED;
+  return y_bf16 ? launch_gemm<BN, ASRC, XT, W4, false, true, MULTI>(ta, ta2, tw, a, stream)
+                : launch_gemm<BN, ASRC, XT, W4, false, false, MULTI>(ta, ta2, tw, a, stream);
+}
+
+// Output-tile width.  Several units per tile need double-buffered TMEM, which
+// caps BN at 128; fp32 activation stages leave room for BN = 128 only.
+// Otherwise a makespan model (columns per CTA plus a per-tile overhead) picks
+// between 128 and 256; SEGQUANT_BN=128|256 overrides it (a tuning knob).
+int choose_bn(int64_t M, int64_t N, bool multi, bool f32x) {
+  if (multi || f32x) return 128;
+  if (const char* e = std::getenv("SEGQUANT_BN")) {
+    const int v = std::atoi(e);
+    if (v == 128 || v == 256) return v;
+  }
+  const int sms = num_sms();
+  const int64_t m_tiles = (M + sq::BM - 1) / sq::BM;
+  // Makespan of the kernel's snake schedule: the busiest CTA's columns plus a
+  // per-tile cost (an epilogue that BN = 256, with one TMEM buffer, cannot
+  // overlap with the next tile's MMAs).
+  std::vector<int64_t> load(sms);
+  auto cost = [&](int64_t bn, int64_t per_tile) {
+    std::fill(load.begin(), load.end(), 0);
+    const int64_t full = N / bn, tail = N % bn;
+    const int64_t tiles = m_tiles * (full + (tail ? 1 : 0));
+    const int64_t nfull = m_tiles * full;
+    for (int64_t idx = 0; idx < tiles; ++idx) {
+      const int64_t it = idx / sms, pos = idx % sms;
+      const int64_t cta = (it & 1) ? sms - 1 - pos : pos;
+      load[cta] += (idx < nfull ? bn : tail) + per_tile;
+    }
+    return *std::max_element(load.begin(), load.end());
+  };
+  return cost(256, 48) <= cost(128, 8) ? 256 : 128;
+}
+
+enum class ASource { X, Codes };
+
+sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_pos,
+                      const int8_t* q_neg, int64_t ldq, int64_t M, int64_t K, int64_t ldx,
                       const sq_qweight* w, const float* s_pos, const float* s_neg,
                       const float* bias, void* y, sq_dtype yt, int64_t ldy, int32_t* acc,
                       cudaStream_t stream) {
-  if (!dtype_ok(xt)) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::X && !dtype_ok(xt)) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && !dtype_ok(yt)) return SQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
   SegBounds kseg;
   sq_status st = check_qweight(w, K, &kseg);
   if (st != SQ_OK) return st;
   const int64_t N = w->N;
-  if (ldx < K) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::X && ldx < K) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::Codes && ldq < K) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && ldy < N) return SQ_ERR_INVALID_ARG;
-  if (M > (int64_t)65535 * sq::BM) return SQ_ERR_RANGE;
+  if (M > (int64_t)INT32_MAX - 2 * sq::BM) return SQ_ERR_RANGE;
   if (M == 0) return SQ_OK;
-  if (x == nullptr || s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
+  if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::X && x == nullptr) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::Codes && (q_pos == nullptr || q_neg == nullptr)) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && y == nullptr) return SQ_ERR_INVALID_ARG;
-  if (!aligned16(x) || (ldx * elt_size(xt)) % 16 != 0) return SQ_ERR_ALIGNMENT;
+  if (src == ASource::X && (!aligned16(x) || (ldx * elt_size(xt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
+  if (src == ASource::Codes && (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0))
+    return SQ_ERR_ALIGNMENT;
   if (acc == nullptr && (!aligned16(y) || (ldy * elt_size(yt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (acc != nullptr && !aligned16(acc)) return SQ_ERR_ALIGNMENT;
   if (bias != nullptr && !aligned16(bias)) return SQ_ERR_ALIGNMENT;
   if ((reinterpret_cast<uintptr_t>(s_pos) & 3u) || (reinterpret_cast<uintptr_t>(s_neg) & 3u))
     return SQ_ERR_ALIGNMENT;
-  if (w->bits == 4) return SQ_ERR_UNSUPPORTED;  // int4 operand path not built yet
 
-  constexpr int BN = 128;
-  CUtensorMap tx, tw;
-  const int xe = elt_size(xt);
-  st = make_tmap(&tx, xt == SQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                 x, (uint64_t)K, (uint64_t)M, (uint64_t)(ldx * xe), 128 / xe, sq::BM);
-  if (st != SQ_OK) return st;
-  st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K, (uint64_t)N,
-                 (uint64_t)K, 128, BN);
+  const bool w4 = (w->bits == 4);
+  const bool multi = w4 || kseg.count > 1;
+  const bool f32x = (src == ASource::X && xt == SQ_F32);
+  const int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x);
+  CUtensorMap ta, ta2, tw;
+  if (src == ASource::X) {
+    const int xe = elt_size(xt);
+    st = make_tmap(&ta, xt == SQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   x, (uint64_t)K, (uint64_t)M, (uint64_t)(ldx * xe), 128 / xe, sq::BM);
+    if (st != SQ_OK) return st;
+    ta2 = ta;
+  } else {
+    st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
+                   (uint64_t)ldq, 128, sq::BM);
+    if (st != SQ_OK) return st;
+    st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
+                   (uint64_t)ldq, 128, sq::BM);
+    if (st != SQ_OK) return st;
+  }
+  if (w4)
+    st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)(K / 2), (uint64_t)N,
+                   (uint64_t)(K / 2), 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K, (uint64_t)N,
+                   (uint64_t)K, 128, (uint32_t)BN);
   if (st != SQ_OK) return st;
 
   sq::GemmArgs a;
@@ -172,27 +262,34 @@ sq_status gemm_common(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t 
   a.acc_out = acc;
   a.wait_budget = g_wait_budget;
 
-  if (acc != nullptr) {
-    return xt == SQ_BF16 ? launch_gemm<BN, __nv_bfloat16, true, false>(tx, tw, a, stream)
-                         : launch_gemm<BN, float, true, false>(tx, tw, a, stream);
+  using bf = __nv_bfloat16;
+  constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
+  const bool yb = (yt == SQ_BF16);
+  const bool ac = (acc != nullptr);
+  if (src == ASource::Codes) {
+    if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
+    if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
+    if (BN == 256) return launch_out<256, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+    return launch_out<128, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
   }
-  if (xt == SQ_BF16)
-    return yt == SQ_BF16 ? launch_gemm<BN, __nv_bfloat16, false, true>(tx, tw, a, stream)
-                         : launch_gemm<BN, __nv_bfloat16, false, false>(tx, tw, a, stream);
-  return yt == SQ_BF16 ? launch_gemm<BN, float, false, true>(tx, tw, a, stream)
-                       : launch_gemm<BN, float, false, false>(tx, tw, a, stream);
-}
-
-int grid_for(int64_t work_items, int per_block) {
-  int64_t g = (work_items + per_block - 1) / per_block;
-  if (g < 1) g = 1;
-  if (g > 148 * 32) g = 148 * 32;
-  return (int)g;
+  if (f32x) {
+    if (w4) return launch_out<128, AX, float, true, true>(ac, yb, ta, ta2, tw, a, stream);
+    if (multi || ac) return launch_out<128, AX, float, false, true>(ac, yb, ta, ta2, tw, a, stream);
+    return launch_out<128, AX, float, false, false>(ac, yb, ta, ta2, tw, a, stream);
+  }
+  if (w4) return launch_out<128, AX, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
+  if (multi || ac) return launch_out<128, AX, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
+  if (BN == 256) return launch_out<256, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+  return launch_out<128, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
 }
 
 }  // namespace
 
 extern "C" {
+
+const char* sq_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char* sq_status_string(sq_status s) {
   switch (s) {
@@ -246,8 +343,10 @@ sq_status sq_calibrate(const void* x, sq_dtype xt, int64_t rows, int64_t K, int6
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bytes = sizeof(float) * (size_t)sb.count;
-  if (cudaMemsetAsync(s_pos, 0, bytes, s) != cudaSuccess) return SQ_ERR_CUDA;
-  if (cudaMemsetAsync(s_neg, 0, bytes, s) != cudaSuccess) return SQ_ERR_CUDA;
+  sq_status ms = cuda_status(cudaMemsetAsync(s_pos, 0, bytes, s));
+  if (ms != SQ_OK) return ms;
+  ms = cuda_status(cudaMemsetAsync(s_neg, 0, bytes, s));
+  if (ms != SQ_OK) return ms;
   if (rows == 0) return SQ_OK;
   const int64_t nvec = K / (16 / xe);
   const int gx = (int)((nvec + 31) / 32);
@@ -312,7 +411,8 @@ sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t
   SegBounds sb;
   sq_status st = check_segments(kseg, K, SQ_MAX_SEGMENTS, 128, &sb);
   if (st != SQ_OK) return st;
-  if (K % 8 != 0) return SQ_ERR_UNSUPPORTED;
+  if (K % 16 != 0) return SQ_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX) return SQ_ERR_RANGE;
   if (M == 0) return SQ_OK;
   if (x == nullptr || s_pos == nullptr || s_neg == nullptr || q_pos == nullptr || q_neg == nullptr)
     return SQ_ERR_INVALID_ARG;
@@ -321,13 +421,22 @@ sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t
       ldq % 16 != 0)
     return SQ_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int blocks = grid_for(M * (K / 8), 256);
+  const int64_t groups = K / 16;
+  const int gx = (int)((groups + 31) / 32);
+  int64_t gy = (M + 7) / 8;
+  const int64_t cap = ((int64_t)num_sms() * 16 + gx - 1) / gx;  // ~16 blocks of 256 per SM
+  if (gy > cap) gy = cap;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  dim3 grid(gx, (unsigned)gy), block(32, 8);
   if (xt == SQ_BF16)
-    sq::quantize_activations_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), M, K, ldx, sb, s_pos, s_neg, q_pos, q_neg, ldq);
+    sq::quantize_activations_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos,
+        q_neg, ldq);
   else
-    sq::quantize_activations_kernel<float><<<blocks, 256, 0, s>>>(
-        static_cast<const float*>(x), M, K, ldx, sb, s_pos, s_neg, q_pos, q_neg, ldq);
+    sq::quantize_activations_kernel<float><<<grid, block, 0, s>>>(
+        static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, q_neg,
+        ldq);
   return cuda_status(cudaGetLastError());
 }
 
@@ -335,26 +444,34 @@ sq_status sq_linear_forward(const void* x, sq_dtype xt, int64_t M, int64_t K, in
                             const sq_qweight* w, const float* s_pos, const float* s_neg,
                             const float* bias, void* y, sq_dtype yt, int64_t ldy,
                             sq_stream_t stream) {
-  return gemm_common(x, xt, M, K, ldx, w, s_pos, s_neg, bias, y, yt, ldy, nullptr,
-                     reinterpret_cast<cudaStream_t>(stream));
+  return gemm_common(ASource::X, x, xt, nullptr, nullptr, 0, M, K, ldx, w, s_pos, s_neg, bias, y,
+                     yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear_forward_codes(const int8_t* q_pos, const int8_t* q_neg, int64_t ldq,
+                                  int64_t M, int64_t K, const sq_qweight* w, const float* s_pos,
+                                  const float* s_neg, const float* bias, void* y, sq_dtype yt,
+                                  int64_t ldy, sq_stream_t stream) {
+  return gemm_common(ASource::Codes, nullptr, SQ_BF16, q_pos, q_neg, ldq, M, K, 0, w, s_pos,
+                     s_neg, bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_linear_accumulators(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
                                  const sq_qweight* w, const float* s_pos, const float* s_neg,
                                  int32_t* acc, sq_stream_t stream) {
   if (acc == nullptr) return SQ_ERR_INVALID_ARG;
-  return gemm_common(x, xt, M, K, ldx, w, s_pos, s_neg, nullptr, nullptr, SQ_F32, 0, acc,
-                     reinterpret_cast<cudaStream_t>(stream));
+  return gemm_common(ASource::X, x, xt, nullptr, nullptr, 0, M, K, ldx, w, s_pos, s_neg, nullptr,
+                     nullptr, SQ_F32, 0, acc, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_stream_status(sq_stream_t stream) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (cuda_status(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream))) != SQ_OK)
     return SQ_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, sq::g_status, sizeof(v)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_status(cudaMemcpyFromSymbol(&v, sq::g_status, sizeof(v))) != SQ_OK) return SQ_ERR_CUDA;
   if (v != 0) {
     const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(sq::g_status, &zero, sizeof(zero)) != cudaSuccess) return SQ_ERR_CUDA;
+    if (cuda_status(cudaMemcpyToSymbol(sq::g_status, &zero, sizeof(zero))) != SQ_OK) return SQ_ERR_CUDA;
   }
   if (v & sq::SQ_STATUS_TIMEOUT) return SQ_ERR_TIMEOUT;
   if (v & sq::SQ_STATUS_RANGE) return SQ_ERR_RANGE;

@@ -34,6 +34,11 @@ SMALL = [
     dict(M=1, K=16, N=16, kseg=[0, 16], x_dtype="bf16", out="bf16"),
     dict(M=257, K=1040, N=128, kseg=[0, 128, 512, 1040], x_sigmas=[1.0, 3.0, 0.5], x_dtype="bf16",
          out="f32"),
+    # int4 weights (group 128): several groups, K segments, ragged M and N
+    dict(M=300, K=640, N=272, kseg=[0, 256, 640], x_sigmas=[1.0, 5.0], x_dtype="bf16", out="bf16",
+         bits=4),
+    dict(M=129, K=384, N=144, kseg=[0, 384], x_dtype="f32", out="f32", bits=4),
+    dict(M=200, K=1024, N=400, kseg=[0, 1024], x_dtype="bf16", out="f32", bits=4),
 ]
 
 
@@ -75,6 +80,36 @@ def test_forward_matches_oracle(i):
     y = c.forward()
     torch.cuda.synchronize()
     c.compare_rows(y, np.arange(c.wl.M))
+
+
+@pytest.mark.parametrize("i", range(len(SMALL)))
+def test_forward_from_codes_equals_fused(i):
+    """Pre-quantized codes through TMA give the same bits as the fused quantizer."""
+    import post_quantized_linear_b200 as pq
+    c = Case(_small(i))
+    y = c.forward()
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    y2 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32),
+                       y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2.view(torch.int32))
+
+
+@pytest.mark.parametrize("bn", ["128", "256"])
+@pytest.mark.parametrize("codes", [False, True])
+def test_tile_width_variants_match_oracle(bn, codes, monkeypatch):
+    """Both output-tile widths (BN = 128 double-buffered TMEM, BN = 256 single
+    buffer with the streaming epilogue), fused and from codes, on ragged shapes."""
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_BN", bn)
+    wl = W.small_case(390, 768, 656, seed=21, out="bf16")
+    c = Case(wl)
+    if codes:
+        qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
+        y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b)
+    else:
+        y = c.forward()
+    torch.cuda.synchronize()
+    c.compare_rows(y, np.arange(wl.M))
 
 
 def test_forward_exact_in_fp32():
@@ -139,7 +174,8 @@ def test_strided_activations_and_outputs():
     assert int(ybig[:, :8].abs().sum()) == 0
 
 
-@pytest.mark.parametrize("name", ["tiny_w8a8", "dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up"])
+@pytest.mark.parametrize("name", ["tiny_w8a8", "dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up",
+                                  "w4a8"])
 def test_workloads_full_size_sampled_rows(name):
     """Full-size workloads in the bench's launch configuration: bit-exact scales
     and weights everywhere; outputs of sampled rows against the oracle."""
@@ -152,3 +188,8 @@ def test_workloads_full_size_sampled_rows(name):
     c.compare_rows(y, rows)
     import post_quantized_linear_b200 as pq
     assert pq.stream_status() == 0
+    # the two-pass path (codes, then the GEMM from codes) gives the same bits
+    qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
+    y2 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32),
+                       y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2.view(torch.int32))
