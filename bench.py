@@ -37,6 +37,13 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
 
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu
+# capture of the current kernel build (profiles/dualscale_gemm_codes_*.md);
+# keyed by (workload, path).  Absent: no capture of the current build.
+NCU_TRAFFIC_BYTES = {
+    ("dit_xl2_fc2_cfg", "codes"): 80838656 + 4266752,
+}
+
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -45,7 +52,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_xl2_fc2_cfg")
-    ap.add_argument("--path", choices=["fused", "codes"], default="fused",
+    ap.add_argument("--path", choices=["fused", "codes"], default="codes",
                     help="fused: quantize X inside the GEMM; codes: quantize X once into "
                          "q+/q- code tensors, then the GEMM loads the codes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -207,7 +214,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": steps, "warmup": warm, "ms_per_step": t_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": config_of(wl, "host cores, no L2 flush"),
+        "config": config_of(wl, "host cores, no L2 flush", "oracle"),
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -289,6 +296,44 @@ def run_ours(args):
     if pq.stream_status() != 0:
         raise RuntimeError("device status word set during warm-up")
 
+    # The step, the forward and the GEMM alone are each captured once into a
+    # CUDA graph and replayed: one launch per step, no host gaps between the
+    # step's kernels.
+    def capture(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        torch.cuda.synchronize()
+        return graph
+
+    def gemm_only():
+        if use_codes:
+            pq.linear_from_codes(qp_buf, qn_buf, qw, sp, sn, bd, out=y)
+        else:
+            pq.linear(xd, qw, sp, sn, bd, out=y)
+
+    step_graph = capture(step)
+    fwd_graph = capture(lambda: forward(xd, y))
+    gemm_graph = capture(gemm_only)
+    fused_graph = capture(lambda: pq.linear(xd, qw, sp, sn, bd, out=y)) if use_codes else None
+
+    def timed(graph, n, salt):
+        evs = events(n)
+        for i in range(n):
+            flush.fill_((i + salt) & 0xFF)
+            evs[i][0].record(stream)
+            graph.replay()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    timed(step_graph, 2, 0)
     sampler = None if args.no_clocks else ClockSampler(local)
     if sampler:
         sampler.start()
@@ -296,31 +341,18 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ev, gev = events(args.steps), events(args.steps)
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        step(gemm_events=gev[i])
-        ev[i][1].record(stream)
+    step_ms = timed(step_graph, args.steps, 1)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    step_ms = [a.elapsed_time(bv) for a, bv in ev]
-    gemm_ms = [a.elapsed_time(bv) for a, bv in gev]
     total_ms = sum(step_ms)
-
-    # forward alone, same protocol (cold L2 per call)
-    fev = events(args.steps)
-    for i in range(args.steps):
-        flush.fill_((i + 7) & 0xFF)
-        fev[i][0].record(stream)
-        forward(xd, y)
-        fev[i][1].record(stream)
-    torch.cuda.synchronize()
-    fwd_ms = [a.elapsed_time(bv) for a, bv in fev]
+    gemm_ms = timed(gemm_graph, args.steps, 3)
+    fwd_ms = timed(fwd_graph, args.steps, 5)
+    fused_ms = timed(fused_graph, args.steps, 7) if fused_graph is not None else None
     if pq.stream_status() != 0:
         raise RuntimeError("device status word set during the timed region")
+    del step_graph, fwd_graph, gemm_graph, fused_graph
 
     # end to end through the API: host inputs in, host result out, every step
     e2e = None
@@ -355,12 +387,12 @@ def run_ours(args):
 
     # max over ranks
     vals = [total_ms, statistics.mean(gemm_ms), statistics.mean(fwd_ms),
-            e2e["ms"] if e2e else 0.0]
+            e2e["ms"] if e2e else 0.0, statistics.mean(fused_ms) if fused_ms else 0.0]
     if world > 1:
         t = torch.tensor(vals, dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         vals = t.tolist()
-    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms = vals
+    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms, fused_avg_ms = vals
 
     if rank == 0:
         int8_peak_tops, hbm_peak, peak_kind = peaks()
@@ -376,7 +408,8 @@ def run_ours(args):
             "roofline": {
                 "bound": "tensor", "kernel": "dualscale_gemm_kernel",
                 "achieved": gemm_tops, "peak": int8_peak_tops, "unit": "TOPS",
-                "frac": gemm_tops / int8_peak_tops, "traffic": None,
+                "frac": gemm_tops / int8_peak_tops,
+                "traffic": NCU_TRAFFIC_BYTES.get((wl.name, args.path)),
                 "peak_source": f"{peak_kind} bf16 burst x {INT8_PER_BF16:g} (nominal int8/bf16)",
                 "algorithmic_ops_per_launch": ops,
                 "algorithmic_bytes_per_launch": wl.alg_bytes(),
@@ -389,8 +422,14 @@ def run_ours(args):
                 "frac_int8_peak": ops / (fwd_avg_ms * 1e-3) / 1e12 / int8_peak_tops,
             },
             "gpu_launches": launches_per_step * args.steps,
+            "timing": "each step one CUDA-graph replay, CUDA events on the launching stream",
             "clocks": clocks,
         }
+        if fused_ms:
+            line["fused_forward"] = {
+                "us": fused_avg_ms * 1e3, "exec_tops": ops / (fused_avg_ms * 1e-3) / 1e12,
+                "frac_int8_peak": ops / (fused_avg_ms * 1e-3) / 1e12 / int8_peak_tops,
+                "note": "sq_linear_forward: activations quantized inside the GEMM"}
         if e2e:
             line["e2e"] = {"value": world * args.steps * ops / (e2e_ms * 1e-3) / 1e12,
                            "unit": "TOPS", "h2d_bytes_per_step": e2e["bi"],

@@ -89,7 +89,8 @@ typedef struct {
  *   bits = 8, group = 0  : codes int8 [N][K]; scales fp32 [J][N] (J = kseg.count),
  *                          one scale per (K segment, output channel).
  *   bits = 4, group = 128: codes uint8 [N][K/2], low nibble = even k;
- *                          scales binary16 [N][K/128], one per (channel, group).
+ *                          scales binary16 [K/128][N] (group-major), one per
+ *                          (group, channel).
  * nseg (output segments, e.g. q | k | v) is validated and carried as metadata:
  * per-channel weight scales make an output split a numerical no-op. */
 typedef struct {

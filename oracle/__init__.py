@@ -148,11 +148,11 @@ def quantize_weights_w8(w: np.ndarray, kbounds):
 
 
 def quantize_weights_w4(w: np.ndarray, group: int = 128):
-    """Packed int4 codes [N, K/2] (low nibble = even k) and fp16 scales [N, K/group]."""
+    """Packed int4 codes [N, K/2] (low nibble = even k) and fp16 scales [K/group, N]."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     N, K = w.shape
     packed = np.zeros((N, K // 2), np.uint8)
-    scales = np.zeros((N, K // group), np.uint16)
+    scales = np.zeros((K // group, N), np.uint16)
     _check("sqo_quantize_weights_w4",
            _load().sqo_quantize_weights_w4(_ptr(w), N, K, K, group, _ptr(packed), _ptr(scales)))
     return packed, scales.view(np.float16)
@@ -222,11 +222,11 @@ def epilogue(acc, unit_seg, s_pos, s_neg, unit_scales, bias=None, out: str = "f3
 
 
 def unit_weight_scales(bits: int, scales: np.ndarray) -> np.ndarray:
-    """Weight scale of every unit as fp32 [U, N]: the [J, N] int8 scales as they
-    are, or the transposed, widened [N, G] fp16 group scales."""
+    """Weight scale of every unit as fp32 [U, N]: the [J, N] int8 scales, or the
+    widened [G, N] fp16 group scales."""
     if bits == 8:
         return np.ascontiguousarray(scales, np.float32)
-    return np.ascontiguousarray(np.asarray(scales, np.float16).astype(np.float32).T)
+    return np.ascontiguousarray(np.asarray(scales, np.float16).astype(np.float32))
 
 
 def linear_forward(x, kbounds, s_pos, s_neg, bits, wcodes, wscales, bias=None, out="f32",
@@ -234,7 +234,7 @@ def linear_forward(x, kbounds, s_pos, s_neg, bits, wcodes, wscales, bias=None, o
     """The whole forward pass: codes, per-unit accumulators, epilogue.
 
     wcodes: int8 [N, K] (bits=8) or packed uint8 [N, K/2] (bits=4);
-    wscales: fp32 [J, N] (bits=8) or fp16 [N, K/128] (bits=4)."""
+    wscales: fp32 [J, N] (bits=8) or fp16 [K/128, N] (bits=4)."""
     M, K = x.shape
     qp, qn = quantize_activations(x, kbounds, s_pos, s_neg)
     codes = wcodes if bits == 8 else unpack_w4(wcodes, K)

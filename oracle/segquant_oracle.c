@@ -209,7 +209,7 @@ int sqo_quantize_weights_w8(const float* w, int64_t N, int64_t K, int64_t ldw, i
  * two values per byte, one fp16 scale per group.  Readings: the group scale is
  * fp16_RNE(max|W|/7) with the division in fp32; codes use the fp16 scale
  * widened back to fp32; in each byte the low nibble holds the even k.
- * packed: [N][K/2] bytes; scales: [N][K/128] binary16 patterns. */
+ * packed: [N][K/2] bytes; scales: [K/128][N] binary16 patterns (group-major). */
 int sqo_quantize_weights_w4(const float* w, int64_t N, int64_t K, int64_t ldw, int32_t group,
                             uint8_t* packed, uint16_t* scales) {
   if (group != 128 || K % group != 0) return SQO_ERR_ARG;
@@ -225,7 +225,7 @@ int sqo_quantize_weights_w4(const float* w, int64_t N, int64_t K, int64_t ldw, i
       }
       uint16_t h = sqo_f32_to_f16(amax / 7.0f);
       if ((h & 0x7c00u) == 0x7c00u) bad = 1;
-      scales[n * G + g] = h;
+      scales[g * N + n] = h;
       float r = recip(sqo_f16_to_f32(h));
       for (int64_t k = g * group; k < (g + 1) * group; k += 2) {
         int32_t q0 = round_clamp(w[n * ldw + k], r, -7, 7);

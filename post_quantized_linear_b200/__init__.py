@@ -59,7 +59,7 @@ class QuantizedWeight:
     kseg: Tuple[int, ...]
     nseg: Tuple[int, ...]
     codes: torch.Tensor    # int8 [N, K] or uint8 [N, K/2]
-    scales: torch.Tensor   # float32 [J, N] or float16 [N, K/128]
+    scales: torch.Tensor   # float32 [J, N] or float16 [K/128, N]
 
     @property
     def group(self) -> int:
@@ -112,7 +112,7 @@ def quantize_weights(w: torch.Tensor, kseg: Sequence[int], nseg: Optional[Sequen
             scales = torch.empty((len(kseg) - 1, N), dtype=torch.float32, device=w.device)
         else:
             codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
-            scales = torch.empty((N, K // 128), dtype=torch.float16, device=w.device)
+            scales = torch.empty((K // 128, N), dtype=torch.float16, device=w.device)
         assert codes.numel() * codes.element_size() == cb
         assert scales.numel() * scales.element_size() == sb
         out = QuantizedWeight(bits, N, K, kseg, nseg, codes, scales)

@@ -76,7 +76,7 @@ struct GemmArgs {
   SegBounds kseg;          // activation (and int8 weight) segments
   const float* s_pos;      // [J]
   const float* s_neg;      // [J]
-  const void* wscales;     // fp32 [J][N] (bits 8) or binary16 [N][K/128] (bits 4)
+  const void* wscales;     // fp32 [J][N] (bits 8) or binary16 [K/128][N] (bits 4)
   const float* bias;       // [N] or null
   void* y;                 // [M][ldy]
   int64_t ldy;
@@ -104,7 +104,7 @@ struct GemmCfg {
   static constexpr int SX = (ASRC == ASRC_X) ? 2 : 0;
   static constexpr int SWP = W4 ? (BIG_X ? 2 : 4) : 0;
   static constexpr int SW = W4 ? (BIG_X ? 1 : 2)
-                               : (ASRC == ASRC_CODES ? (BN == 128 ? 4 : 3) : ((BIG_X || BN == 256) ? 2 : 4));
+                               : (ASRC == ASRC_CODES ? (BN == 128 ? 4 : 3) : ((BIG_X || BN >= 192) ? 2 : 4));
   static constexpr int SQ = (kStageBudget - SX * X_STAGE - SWP * WP_STAGE - SW * W_STAGE) / Q_STAGE;
   static constexpr int NBUF = (BN <= 128) ? 2 : 1;       // TMEM accumulator buffers
   static constexpr int OFF_X = 0;
@@ -116,7 +116,9 @@ struct GemmCfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 2 * BN * NBUF;
+  static constexpr int TMEM_ALLOC = TMEM_COLS <= 256 ? 256 : 512;  // a power of two
   static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
+  static_assert(BN % 16 == 0 && BN <= 256, "UMMA N for M = 128");
   static_assert(SQ >= 2 && SQ <= 8 && SW >= 1 && SW <= 4 && SWP <= 4, "stage counts");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -313,10 +315,19 @@ __device__ __forceinline__ void load_wscales16(const GemmArgs& a, int u, int j, 
       sw[4 * i] = t.x; sw[4 * i + 1] = t.y; sw[4 * i + 2] = t.z; sw[4 * i + 3] = t.w;
     }
   } else {
-    const __half* hs = static_cast<const __half*>(a.wscales);
-    const int G = a.K / 128;
+    const uint4* h8 = reinterpret_cast<const uint4*>(static_cast<const __half*>(a.wscales) +
+                                                     (int64_t)u * a.N + n);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) sw[i] = __half2float(hs[(int64_t)(n + i) * G + u]);
+    for (int i = 0; i < 2; ++i) {
+      const uint4 t = __ldg(h8 + i);
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        sw[8 * i + 2 * k] = f.x;
+        sw[8 * i + 2 * k + 1] = f.y;
+      }
+    }
   }
 }
 
@@ -351,10 +362,15 @@ __device__ __forceinline__ void load_wscales8(const GemmArgs& a, int u, int j, i
     sw[0] = t0.x; sw[1] = t0.y; sw[2] = t0.z; sw[3] = t0.w;
     sw[4] = t1.x; sw[5] = t1.y; sw[6] = t1.z; sw[7] = t1.w;
   } else {
-    const __half* hs = static_cast<const __half*>(a.wscales);
-    const int G = a.K / 128;
+    const uint4 t = __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(a.wscales) +
+                                                         (int64_t)u * a.N + n));
+    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sw[i] = __half2float(hs[(int64_t)(n + i) * G + u]);
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      sw[2 * k] = f.x;
+      sw[2 * k + 1] = f.y;
+    }
   }
 }
 
@@ -367,6 +383,24 @@ __device__ __forceinline__ void fold8(const uint32_t (&ap)[8], const uint32_t (&
     const float fn = acc_to_f32<SMALL>(an[i]);
     const float t = __fmaf_rn(sn, fn, __fmul_rn(sp, fp));
     y[i] = __fmaf_rn(sw[i], t, y[i]);
+  }
+}
+
+// int4 units: the accumulators were seeded with the bit pattern of 1.5*2^23
+// (kMagicBits), so each holds kMagicBits + acc; as a float that is exactly
+// 1.5*2^23 + acc (|acc| < 2^22), and one subtraction gives F(acc) exactly.
+// Same fp32 operations as fold8, two outputs per packed f32x2 instruction.
+__device__ __forceinline__ void fold8_seeded(const uint32_t (&ap)[8], const uint32_t (&an)[8],
+                                             const float (&sw)[8], float sp, float sn, float* y) {
+  const uint64_t m2 = f2_pack(-kMagic, -kMagic);
+  const uint64_t sp2 = f2_pack(sp, sp), sn2 = f2_pack(sn, sn);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const uint64_t fp = f2_add(f2_pack(__uint_as_float(ap[i]), __uint_as_float(ap[i + 1])), m2);
+    const uint64_t fn = f2_add(f2_pack(__uint_as_float(an[i]), __uint_as_float(an[i + 1])), m2);
+    const uint64_t t = f2_fma(sn2, fn, f2_mul(sp2, fp));
+    const uint64_t yy = f2_fma(f2_pack(sw[i], sw[i + 1]), t, f2_pack(y[i], y[i + 1]));
+    f2_unpack(yy, y[i], y[i + 1]);
   }
 }
 
@@ -442,6 +476,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
   const long long budget = args.wait_budget;
   constexpr bool PROD_Q = (ASRC == ASRC_X);   // producer warps write the Q tiles
   constexpr bool PROD_W = W4;                 // producer warps write the W tiles
+  constexpr bool SEEDED = W4;                 // accumulators seeded with kMagicBits
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::SX; ++i) {
@@ -469,7 +504,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -542,7 +577,11 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!unit_open) {
             const int b = ug % C::NBUF;
-            if (!(ok = wait1(smem_u32(tmem_empty + b), ((ug / C::NBUF) & 1) ^ 1, abort_flag, budget))) break;
+            // Seeded (int4) accumulators: the epilogue's seeding of a buffer
+            // completes phase 0, so use n waits for phase n; otherwise a fresh
+            // buffer is free at once.
+            const uint32_t par = SEEDED ? ((ug / C::NBUF) & 1) : (((ug / C::NBUF) & 1) ^ 1);
+            if (!(ok = wait1(smem_u32(tmem_empty + b), par, abort_flag, budget))) break;
             tc_fence_after();
             d_pos = tmem_base + (uint32_t)(b * 2 * BN);
           }
@@ -555,7 +594,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
           const uint32_t b_w = smem_u32(sm_w + sw * C::W_STAGE);
 #pragma unroll
           for (int ks = 0; ks < BK / 32; ++ks) {
-            const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
+            const uint32_t acc = (SEEDED || unit_open || ks > 0) ? 1u : 0u;
             const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
             umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
             umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
@@ -658,6 +697,23 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
     const int units = (args.bits == 4) ? num_kb : args.kseg.count;
     int ug = 0;
     bool ok = true;
+    if constexpr (SEEDED) {
+      // Seed both accumulator buffers, then hand them to the MMA warp.
+      const int c_lo = half * HALF;
+      for (int b = 0; b < C::NBUF; ++b) {
+#pragma unroll
+        for (int c = 0; c < HALF / 8; ++c) {
+          const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 8);
+          tmem_st8(t_lane + col, kMagicBits);
+          tmem_st8(t_lane + col + BN, kMagicBits);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        for (int b = 0; b < C::NBUF; ++b) mbar_arrive(smem_u32(tmem_empty + b));
+    }
     for (int it = 0; it < rounds && ok; ++it) {
       Tile t;
       if (!tile_of(args, it, BN, t)) continue;
@@ -681,8 +737,16 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
               tmem_ld8(t_lane + col, ap);
               tmem_ld8(t_lane + col + BN, an);
               tmem_wait_ld();
+              if constexpr (SEEDED) {
+                tmem_st8(t_lane + col, kMagicBits);
+                tmem_st8(t_lane + col + BN, kMagicBits);
+              }
               const int n = t.n0 + c_lo + c * 8;
               if constexpr (ACC_OUT) {
+                if constexpr (SEEDED) {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) { ap[i] -= kMagicBits; an[i] -= kMagicBits; }
+                }
                 if (row < args.M) {
                   int32_t* dp = args.acc_out + (((int64_t)u * 2 + 0) * args.M + row) * args.N + n;
                   int32_t* dn = args.acc_out + (((int64_t)u * 2 + 1) * args.M + row) * args.N + n;
@@ -695,10 +759,12 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
               } else {
                 float sw[8];
                 load_wscales8(args, u, j, n, sw);
-                fold8<W4>(ap, an, sw, sp, sn, y + c * 8);
+                if constexpr (SEEDED) fold8_seeded(ap, an, sw, sp, sn, y + c * 8);
+                else fold8<false>(ap, an, sw, sp, sn, y + c * 8);
               }
             }
           }
+          if constexpr (SEEDED) tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(tmem_empty + b));
@@ -755,7 +821,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    tmem_dealloc(tmem_base, C::TMEM_ALLOC);
   }
 }
 

@@ -197,25 +197,26 @@ __global__ void __launch_bounds__(256) quantize_activations_kernel(
 }
 
 // ------------------------------------------------------ weight quantization
-// int8: one warp per (output channel n, K segment j).  Pass 1: |W| max by
-// warp shuffles; s = max/127; r = 1/s.  Pass 2: codes with the same magic
-// rounding, clamp to +-127, sixteen codes per 16-byte store (segment bounds
-// are multiples of 128 and K of 16).
+// int8: one 128-thread block per (output channel n, K segment j).  Pass 1:
+// |W| max (warp shuffles, then shared memory); s = max/127; r = 1/s.  Pass 2
+// (the segment row is now in L1): codes with the same magic rounding, clamp
+// to +-127, sixteen codes per 16-byte store (segment bounds are multiples of
+// 128 and K of 16).
 template <typename WT>
-__global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
+__global__ void __launch_bounds__(128) quantize_weights_w8_kernel(
     const WT* __restrict__ w, int64_t N, int64_t K, int64_t ldw, SegBounds kseg,
     int8_t* __restrict__ codes, float* __restrict__ scales) {
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int64_t total = N * kseg.count;
-  if (warp >= total) return;
-  const int64_t n = warp / kseg.count;
-  const int j = (int)(warp - n * kseg.count);
+  __shared__ float sh_max[4];
+  __shared__ int sh_bad;
+  const int64_t n = blockIdx.x / kseg.count;
+  const int j = (int)(blockIdx.x - n * kseg.count);
   const int32_t k0 = kseg.b[j], k1 = kseg.b[j + 1];
   const WT* row = w + n * ldw;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid == 0) sh_bad = 0;
   float amax = 0.0f;
   bool bad = false;
-  for (int32_t k = k0 + lane * 16; k < k1; k += 512) {
+  for (int32_t k = k0 + tid * 16; k < k1; k += 128 * 16) {
     float v[16];
     load16<WT>(row + k, v);
 #pragma unroll
@@ -227,11 +228,19 @@ __global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(SQ_STATUS_RANGE);
+  const bool wbad = __any_sync(0xffffffffu, bad);
+  __syncthreads();
+  if (lane == 0) {
+    sh_max[tid >> 5] = amax;
+    if (wbad) sh_bad = 1;
+  }
+  __syncthreads();
+  amax = fmaxf(fmaxf(sh_max[0], sh_max[1]), fmaxf(sh_max[2], sh_max[3]));
+  if (tid == 0 && sh_bad) raise_status(SQ_STATUS_RANGE);
   const float s = amax / 127.0f;
   const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
-  if (lane == 0) scales[(int64_t)j * N + n] = s;
-  for (int32_t k = k0 + lane * 16; k < k1; k += 512) {
+  if (tid == 0) scales[(int64_t)j * N + n] = s;
+  for (int32_t k = k0 + tid * 16; k < k1; k += 128 * 16) {
     float v[16];
     load16<WT>(row + k, v);
     uint32_t c[16];
@@ -248,7 +257,7 @@ __global__ void __launch_bounds__(256) quantize_weights_w8_kernel(
 // int4: one warp per (output channel n, 128-wide group g); lane l owns k =
 // 128g + 4l .. 4l+3.  s16 = fp16_rne(max/7) (fp32 division, then one RNE to
 // binary16); codes use the widened fp16 scale; two codes per byte, low nibble
-// = even k; scales stored [N][K/128].
+// = even k; scales stored group-major [K/128][N].
 template <typename WT>
 __global__ void __launch_bounds__(256) quantize_weights_w4_kernel(
     const WT* __restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t* __restrict__ packed,
@@ -286,7 +295,7 @@ __global__ void __launch_bounds__(256) quantize_weights_w4_kernel(
   }
   const uint16_t two = (uint16_t)(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
   *reinterpret_cast<uint16_t*>(packed + n * (K / 2) + g * 64 + lane * 2) = two;
-  if (lane == 0) scales[n * G + g] = s16;
+  if (lane == 0) scales[g * N + n] = s16;
 }
 
 }  // namespace sq

@@ -157,33 +157,33 @@ sq_status launch_out(bool acc, bool y_bf16, const CUtensorMap& ta, const CUtenso
 
 // Output-tile width.  Several units per tile need double-buffered TMEM, which
 // caps BN at 128; fp32 activation stages leave room for BN = 128 only.
-// Otherwise a makespan model (columns per CTA plus a per-tile overhead) picks
-// between 128 and 256; SEGQUANT_BN=128|256 overrides it (a tuning knob).
+// Otherwise BN in {128, 192, 256} minimises a makespan model of the snake
+// schedule: the busiest CTA's tile columns divided by the measured per-column
+// efficiency of that width (narrow tiles keep less work in flight per byte of
+// pipeline), with the last, narrower tile costing a full one.
+// SEGQUANT_BN=128|192|256 overrides the choice (a tuning knob).
 int choose_bn(int64_t M, int64_t N, bool multi, bool f32x) {
   if (multi || f32x) return 128;
   if (const char* e = std::getenv("SEGQUANT_BN")) {
     const int v = std::atoi(e);
-    if (v == 128 || v == 256) return v;
+    if (v == 128 || v == 192 || v == 256) return v;
   }
   const int sms = num_sms();
   const int64_t m_tiles = (M + sq::BM - 1) / sq::BM;
-  // Makespan of the kernel's snake schedule: the busiest CTA's columns plus a
-  // per-tile cost (an epilogue that BN = 256, with one TMEM buffer, cannot
-  // overlap with the next tile's MMAs).
-  std::vector<int64_t> load(sms);
-  auto cost = [&](int64_t bn, int64_t per_tile) {
-    std::fill(load.begin(), load.end(), 0);
-    const int64_t full = N / bn, tail = N % bn;
-    const int64_t tiles = m_tiles * (full + (tail ? 1 : 0));
-    const int64_t nfull = m_tiles * full;
+  std::vector<double> load(sms);
+  auto cost = [&](int64_t bn, double eff) {
+    std::fill(load.begin(), load.end(), 0.0);
+    const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
     for (int64_t idx = 0; idx < tiles; ++idx) {
       const int64_t it = idx / sms, pos = idx % sms;
       const int64_t cta = (it & 1) ? sms - 1 - pos : pos;
-      load[cta] += (idx < nfull ? bn : tail) + per_tile;
+      load[cta] += (double)bn / eff;
     }
     return *std::max_element(load.begin(), load.end());
   };
-  return cost(256, 48) <= cost(128, 8) ? 256 : 128;
+  const double c128 = cost(128, 0.55), c192 = cost(192, 0.70), c256 = cost(256, 0.81);
+  if (c256 <= c192 && c256 <= c128) return 256;
+  return c192 <= c128 ? 192 : 128;
 }
 
 enum class ASource { X, Codes };
@@ -270,6 +270,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
     if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
     if (BN == 256) return launch_out<256, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+    if (BN == 192) return launch_out<192, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
     return launch_out<128, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
   }
   if (f32x) {
@@ -280,6 +281,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   if (w4) return launch_out<128, AX, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
   if (multi || ac) return launch_out<128, AX, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
   if (BN == 256) return launch_out<256, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+  if (BN == 192) return launch_out<192, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
   return launch_out<128, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
 }
 
@@ -377,14 +379,14 @@ sq_status sq_quantize_weights(const void* w, sq_dtype wt, int64_t N, int64_t K, 
   if (!aligned16(w) || (ldw * elt_size(wt)) % 16 != 0) return SQ_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (out->bits == 8) {
-    const int64_t warps = N * kseg.count;
-    const int blocks = (int)((warps * 32 + 255) / 256);
+    const int64_t blocks = N * kseg.count;
+    if (blocks > INT32_MAX) return SQ_ERR_RANGE;
     if (wt == SQ_BF16)
-      sq::quantize_weights_w8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+      sq::quantize_weights_w8_kernel<__nv_bfloat16><<<(unsigned)blocks, 128, 0, s>>>(
           static_cast<const __nv_bfloat16*>(w), N, K, ldw, kseg, static_cast<int8_t*>(out->codes),
           static_cast<float*>(out->scales));
     else
-      sq::quantize_weights_w8_kernel<float><<<blocks, 256, 0, s>>>(
+      sq::quantize_weights_w8_kernel<float><<<(unsigned)blocks, 128, 0, s>>>(
           static_cast<const float*>(w), N, K, ldw, kseg, static_cast<int8_t*>(out->codes),
           static_cast<float*>(out->scales));
   } else {

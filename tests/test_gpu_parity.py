@@ -94,7 +94,7 @@ def test_forward_from_codes_equals_fused(i):
                        y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2.view(torch.int32))
 
 
-@pytest.mark.parametrize("bn", ["128", "256"])
+@pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("codes", [False, True])
 def test_tile_width_variants_match_oracle(bn, codes, monkeypatch):
     """Both output-tile widths (BN = 128 double-buffered TMEM, BN = 256 single

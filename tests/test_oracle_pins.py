@@ -200,7 +200,7 @@ def test_bruteforce_w4_exact(seed):
     np.testing.assert_array_equal(o["codes"], ex["wq"])
     G = K // 128
     for g in range(G):
-        assert [Fr(float(v)) for v in o["ws"][:, g]] == ex["wsc"][g]
+        assert [Fr(float(v)) for v in o["ws"][g]] == ex["wsc"][g]
     np.testing.assert_array_equal(o["qp"], ex["qp"])
     np.testing.assert_array_equal(o["qn"], ex["qn"])
     np.testing.assert_array_equal(o["acc"], ex["acc"])
@@ -323,11 +323,11 @@ def test_I4_weight_error_within_half_step():
     packed, s16 = O.quantize_weights_w4(w)
     codes = O.unpack_w4(packed, 512)
     assert codes.min() >= -7 and codes.max() <= 7
-    sf = s16.astype(np.float64)
+    sf = s16.astype(np.float64)  # [G, N]
     for g in range(4):
         blk = slice(g * 128, (g + 1) * 128)
-        err = np.abs(w[:, blk].astype(np.float64) - sf[:, g:g + 1] * codes[:, blk])
-        assert np.all(err <= sf[:, g:g + 1] / 2 * (1 + 2.0 ** -10))
+        err = np.abs(w[:, blk].astype(np.float64) - sf[g][:, None] * codes[:, blk])
+        assert np.all(err <= sf[g][:, None] / 2 * (1 + 2.0 ** -10))
 
 
 def test_I5_sign_symmetry():
@@ -458,7 +458,7 @@ def test_int4_packing_layout_and_roundtrip():
     k = np.arange(128)
     w = np.array([((k % 15) - 7).astype(np.float32)], dtype=np.float32)
     packed, s16 = O.quantize_weights_w4(w)
-    assert float(s16[0, 0]) == 1.0
+    assert s16.shape == (1, 1) and float(s16[0, 0]) == 1.0
     codes = ((k % 15) - 7)
     expect = [(int(codes[2 * i]) & 0xF) | ((int(codes[2 * i + 1]) & 0xF) << 4) for i in range(64)]
     assert list(packed[0]) == expect
