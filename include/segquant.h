@@ -193,6 +193,11 @@ const char* sq_last_cuda_error(void);
  * second).  0 restores the default.  Host only; affects later launches. */
 void sq_set_wait_budget(int64_t cycles);
 
+/* Test hook: while enabled, the GEMM kernels' TMA producer issues no copy, so
+ * every consumer's bounded wait expires; the launch still returns SQ_OK and
+ * sq_stream_status() then reports SQ_ERR_TIMEOUT.  Host only. */
+void sq_debug_starve_pipeline(int32_t enable);
+
 #ifdef __cplusplus
 }
 #endif

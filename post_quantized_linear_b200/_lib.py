@@ -51,6 +51,7 @@ SIGNATURES = {
     "sq_status_string": (ctypes.c_char_p, [c_i32]),
     "sq_last_cuda_error": (ctypes.c_char_p, []),
     "sq_set_wait_budget": (None, [c_i64]),
+    "sq_debug_starve_pipeline": (None, [c_i32]),
 }
 
 _lib = None

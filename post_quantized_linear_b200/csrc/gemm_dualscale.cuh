@@ -81,8 +81,13 @@ struct GemmArgs {
   void* y;                 // [M][ldy]
   int64_t ldy;
   int32_t* acc_out;        // [U][2][M][N] (accumulator mode)
-  long long wait_budget;   // clock cycles per wait
+  long long wait_budget;   // clock cycles per pipeline wait
+  int32_t starve;          // test hook: the TMA producer issues nothing
 };
+
+// Teardown waits (copies and MMAs that were issued always complete) get a
+// fixed budget of about two seconds, independent of the pipeline-wait budget.
+constexpr long long kDrainBudget = 4000000000LL;
 
 constexpr int kStageBudget = 229376;  // 224 KiB of pipeline stages
 
@@ -103,7 +108,7 @@ struct GemmCfg {
   static constexpr bool BIG_X = (ASRC == ASRC_X) && XE == 4;
   static constexpr int SX = (ASRC == ASRC_X) ? 2 : 0;
   static constexpr int SWP = W4 ? (BIG_X ? 2 : 4) : 0;
-  static constexpr int SW = W4 ? (BIG_X ? 1 : 2)
+  static constexpr int SW = W4 ? (BIG_X ? 1 : (ASRC == ASRC_CODES ? 3 : 2))
                                : (ASRC == ASRC_CODES ? (BN == 128 ? 4 : 3) : ((BIG_X || BN >= 192) ? 2 : 4));
   static constexpr int SQ = (kStageBudget - SX * X_STAGE - SWP * WP_STAGE - SW * W_STAGE) / Q_STAGE;
   static constexpr int NBUF = (BN <= 128) ? 2 : 1;       // TMEM accumulator buffers
@@ -141,13 +146,39 @@ __device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile in
   }
 }
 
+// Phase test with acquire at CTA scope, or at cluster scope for barriers that
+// receive arrivals from the other CTA of a pair.
+template <bool CLUSTER>
+__device__ __forceinline__ bool try_wait_scoped(uint32_t bar, uint32_t parity) {
+  if constexpr (CLUSTER) return mbar_try_wait_cluster(bar, parity);
+  else return mbar_try_wait(bar, parity);
+}
+
+// Single-thread bounded wait with a selectable acquire scope.
+template <bool CLUSTER>
+__device__ __forceinline__ bool wait1s(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       long long budget) {
+  if (try_wait_scoped<CLUSTER>(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (try_wait_scoped<CLUSTER>(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > budget) {
+      *abort_flag = 1;
+      raise_status(SQ_STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform bounded wait: every lane observes the barrier itself (acquire),
 // the loop exits together.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           long long budget) {
   const long long t0 = clock64();
   while (true) {
-    const bool ok = mbar_try_wait(bar, parity);
+    const bool ok = try_wait_scoped<CLUSTER>(bar, parity);
     if (__all_sync(0xffffffffu, ok)) return true;
     int stop = 0;
     if ((threadIdx.x & 31) == 0) {
@@ -292,6 +323,83 @@ __device__ __forceinline__ uint2 unpack8_int4(uint32_t w) {
 
 __device__ __forceinline__ float rcp_or_zero(float s) { return s > 0.0f ? __frcp_rn(s) : 0.0f; }
 
+// Per-segment constants of the fused quantizer.
+struct QuantParams {
+  float lo;       // inputs below lo behave as lo: the -127 clamp, applied on the input
+  uint32_t rp;    // bit pattern of r+ = 1/s+
+  uint32_t dr;    // r- bits minus r+ bits (mod 2^32): rp + sign * dr selects r-
+};
+
+// The smallest fp32 L with L * r- > -127.5 (exact real product).  Every
+// x >= L rounds to a code >= -127 and every x < L to one <= -128, which the
+// clamp turns into -127 = rne(L * r-); so clamping x at L first is exact.
+// fmaf(L, r, 127.5) rounds L*r + 127.5 once, and rounding keeps the sign, so
+// each test below is exact.
+__device__ __forceinline__ float neg_input_limit(float rn) {
+  if (!(rn > 0.0f)) return -__int_as_float(0x7f800000);  // no negative branch: all codes 0
+  float L = -127.5f / rn;
+  for (int i = 0; i < 4 && !(fmaf(L, rn, 127.5f) > 0.0f); ++i) L = nextafterf(L, 0.0f);
+  for (int i = 0; i < 4; ++i) {
+    const float d = nextafterf(L, -__int_as_float(0x7f800000));
+    if (fmaf(d, rn, 127.5f) > 0.0f) L = d;
+    else break;
+  }
+  return L;
+}
+
+__device__ __forceinline__ QuantParams quant_params(float sp, float sn) {
+  const float rp = rcp_or_zero(sp), rn = rcp_or_zero(sn);
+  QuantParams q;
+  q.lo = neg_input_limit(rn);
+  q.rp = __float_as_uint(rp);
+  q.dr = __float_as_uint(rn) - q.rp;
+  return q;
+}
+
+// One DualScale code for an input already clamped below at QuantParams::lo:
+// the sign bit (IMAD.HI) selects r- or r+ (IMAD), the fma rounds the exact
+// product half-to-even against 1.5*2^23, and the bit difference is the signed
+// code (large positive values saturate in the pack below).
+__device__ __forceinline__ int32_t signed_code(float xc, const QuantParams& p) {
+  const uint32_t sgn = __umulhi(__float_as_uint(xc), 2u);
+  const float r = __uint_as_float(p.rp + sgn * p.dr);
+  return (int32_t)(__float_as_uint(fmaf(xc, r, kMagic)) - kMagicBits);
+}
+
+// Four signed codes -> four bytes, each saturated to [-128, 127]; byte i from c_i.
+__device__ __forceinline__ uint32_t pack_sat4(int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+  uint32_t hi, out;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(c3), "r"(c2));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(out) : "r"(c1), "r"(c0), "r"(hi));
+  return out;
+}
+
+// Splits four signed codes into their non-negative and negative parts (the
+// other part's byte is 0): a byte's sign, replicated, selects it.
+__device__ __forceinline__ void split4(uint32_t c, uint32_t& qp, uint32_t& qn) {
+  uint32_t m;  // prmt with selector nibbles 8..11: each byte's sign bit, replicated
+  asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(m) : "r"(c));
+  qp = c & ~m;
+  qn = c & m;
+}
+
+// 16 activations of one row -> 16 q+ and 16 q- codes.
+__device__ __forceinline__ void quantize16_fast(const float (&v)[16], const QuantParams& p,
+                                                uint4& qp, uint4& qn) {
+  uint32_t w[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    int32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = signed_code(fmaxf(v[4 * g + i], p.lo), p);
+    w[g] = pack_sat4(c[0], c[1], c[2], c[3]);
+  }
+  split4(w[0], qp.x, qn.x);
+  split4(w[1], qp.y, qn.y);
+  split4(w[2], qp.z, qn.z);
+  split4(w[3], qp.w, qn.w);
+}
+
 // Segment of the K block `kb` and whether it closes its unit.
 __device__ __forceinline__ int kb_segment(const GemmArgs& a, int kb) {
   return a.kseg.segment_of(kb * BK);
@@ -386,6 +494,18 @@ __device__ __forceinline__ void fold8(const uint32_t (&ap)[8], const uint32_t (&
   }
 }
 
+// Prefetches into L1 the weight scales this thread will read for unit u:
+// `cols` consecutive columns from tile column n (fp32 [J][N] or fp16 [G][N]).
+__device__ __forceinline__ void prefetch_wscales(const GemmArgs& a, int u, int j, int n, int cols) {
+  if (a.bits == 8) {
+    const float* p = static_cast<const float*>(a.wscales) + (int64_t)j * a.N + n;
+    for (int c = 0; c < cols; c += 32) prefetch_l1(p + c);
+  } else {
+    const __half* p = static_cast<const __half*>(a.wscales) + (int64_t)u * a.N + n;
+    for (int c = 0; c < cols; c += 64) prefetch_l1(p + c);
+  }
+}
+
 // int4 units: the accumulators were seeded with the bit pattern of 1.5*2^23
 // (kMagicBits), so each holds kMagicBits + acc; as a float that is exactly
 // 1.5*2^23 + acc (|acc| < 2^22), and one subtraction gives F(acc) exactly.
@@ -401,6 +521,50 @@ __device__ __forceinline__ void fold8_seeded(const uint32_t (&ap)[8], const uint
     const uint64_t t = f2_fma(sn2, fn, f2_mul(sp2, fp));
     const uint64_t yy = f2_fma(f2_pack(sw[i], sw[i + 1]), t, f2_pack(y[i], y[i + 1]));
     f2_unpack(yy, y[i], y[i + 1]);
+  }
+}
+
+// Weight scales of 8 consecutive output channels for unit u, as four fp32 pairs.
+__device__ __forceinline__ void load_wscales8_pairs(const GemmArgs& a, int u, int j, int n,
+                                                    uint64_t (&sw2)[4]) {
+  if (a.bits == 8) {
+    const float4* s4 =
+        reinterpret_cast<const float4*>(static_cast<const float*>(a.wscales) + (int64_t)j * a.N + n);
+    const float4 t0 = __ldg(s4), t1 = __ldg(s4 + 1);
+    sw2[0] = f2_pack(t0.x, t0.y); sw2[1] = f2_pack(t0.z, t0.w);
+    sw2[2] = f2_pack(t1.x, t1.y); sw2[3] = f2_pack(t1.z, t1.w);
+  } else {
+    const uint4 t = __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(a.wscales) +
+                                                         (int64_t)u * a.N + n));
+    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      sw2[k] = f2_pack(f.x, f.y);
+    }
+  }
+}
+
+// y2 (+)= sw * (s- F(acc-) + s+ F(acc+)) for 8 outputs held as four fp32 pairs,
+// the same fp32 operations as fold8 (R9 order), two outputs per instruction.
+// SEEDED: accumulators hold kMagicBits + acc (int4 units); F is one exact
+// subtraction.  Otherwise F is the round-to-nearest int32 -> fp32 conversion.
+template <bool SEEDED>
+__device__ __forceinline__ void fold8_pairs(const uint32_t (&ap)[8], const uint32_t (&an)[8],
+                                            const uint64_t (&sw2)[4], uint64_t sp2, uint64_t sn2,
+                                            uint64_t* y2) {
+  const uint64_t m2 = f2_pack(-kMagic, -kMagic);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint64_t fp, fn;
+    if constexpr (SEEDED) {
+      fp = f2_add(f2_pack(__uint_as_float(ap[2 * i]), __uint_as_float(ap[2 * i + 1])), m2);
+      fn = f2_add(f2_pack(__uint_as_float(an[2 * i]), __uint_as_float(an[2 * i + 1])), m2);
+    } else {
+      fp = f2_pack(__int2float_rn((int)ap[2 * i]), __int2float_rn((int)ap[2 * i + 1]));
+      fn = f2_pack(__int2float_rn((int)an[2 * i]), __int2float_rn((int)an[2 * i + 1]));
+    }
+    y2[i] = f2_fma(sw2[i], f2_fma(sn2, fn, f2_mul(sp2, fp)), y2[i]);
   }
 }
 
@@ -433,6 +597,176 @@ __device__ __forceinline__ void store16(const GemmArgs& a, int row, int n, float
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       reinterpret_cast<float4*>(dst)[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  }
+}
+
+// --------------------------------------------------------- epilogue role
+// Arrive on an mbarrier of another CTA of the cluster (release, cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// The epilogue of one CTA: for every tile it owns, wait for each unit's
+// accumulators in TMEM, fold them (or write them raw), release the buffer,
+// and after the tile's last unit store its rows.  The thread owns TMEM lane
+// quad*32 + lane (tile row row_shift + quad*32 + lane) and the columns
+// [part*HALF, (part+1)*HALF).  `empty_base` is the address of tmem_empty[0]
+// (a cluster-window address of another CTA when empty_remote).
+template <int BN, int NBUF, bool MULTI, bool ACC_OUT, bool Y_BF16, bool SEEDED, class TileFn,
+          bool CLUSTER = false>
+__device__ __forceinline__ void epilogue_role(const GemmArgs& args, int quad, int part, int lane,
+                                              uint32_t t_lane, uint64_t* tmem_full,
+                                              uint32_t empty_base, bool empty_remote,
+                                              int row_shift, int rounds, TileFn tile_fn,
+                                              volatile int* abort_flag, long long budget) {
+  constexpr int HALF = BN / (epi_warps(MULTI) / 4);   // columns per epilogue thread
+  const int half = part;
+  const int num_kb = args.num_kb;
+  const int units = (args.bits == 4) ? num_kb : args.kseg.count;
+  auto release = [&](int b) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      if (empty_remote) mbar_arrive_remote(empty_base + 8u * (uint32_t)b);
+      else mbar_arrive(empty_base + 8u * (uint32_t)b);
+    }
+  };
+  int ug = 0;
+  bool ok = true;
+  if constexpr (SEEDED) {
+    // Seed both accumulator buffers, then hand them to the MMA warp.
+    const int c_lo = half * HALF;
+    for (int b = 0; b < NBUF; ++b) {
+#pragma unroll
+      for (int c = 0; c < HALF / 8; ++c) {
+        const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 8);
+        tmem_st8(t_lane + col, kMagicBits);
+        tmem_st8(t_lane + col + BN, kMagicBits);
+      }
+    }
+    tmem_wait_st();
+    for (int b = 0; b < NBUF; ++b) release(b);
+  }
+  for (int it = 0; it < rounds && ok; ++it) {
+    Tile t;
+    if (!tile_fn(it, t)) continue;
+    const int row = t.m0 + row_shift + quad * 32 + lane;
+    const int c_lo = half * HALF;                 // first tile column of this warp
+      if constexpr (MULTI || ACC_OUT) {
+        constexpr int NY2 = (MULTI && !ACC_OUT) ? HALF / 2 : 1;
+        uint64_t y2[NY2];  // partial outputs, fp32 pairs
+#pragma unroll
+        for (int i = 0; i < NY2; ++i) y2[i] = 0ull;
+        // Scales are read two units ahead of use, so their L2 latency hides
+        // behind the current unit's MMAs.
+        constexpr int kAhead = 2;
+        if constexpr (!ACC_OUT) {
+          if (lane == 0 && c_lo < t.width)
+            for (int u = 0; u < kAhead && u < units; ++u)
+              prefetch_wscales(args, u, (args.bits == 4) ? args.kseg.segment_of(u * 128) : u,
+                               t.n0 + c_lo, min(HALF, t.width - c_lo));
+        }
+        for (int u = 0; u < units; ++u) {
+          if constexpr (!ACC_OUT) {
+            const int uf = u + kAhead;
+            if (lane == 0 && uf < units && c_lo < t.width)
+              prefetch_wscales(args, uf, (args.bits == 4) ? args.kseg.segment_of(uf * 128) : uf,
+                               t.n0 + c_lo, min(HALF, t.width - c_lo));
+          }
+          const int b = ug % NBUF;
+          if (!(ok = wait_warp<CLUSTER>(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+          tc_fence_after();
+          const int j = (args.bits == 4) ? args.kseg.segment_of(u * 128) : u;
+          const float sp = __ldg(args.s_pos + j), sn = __ldg(args.s_neg + j);
+          const uint64_t sp2 = f2_pack(sp, sp), sn2 = f2_pack(sn, sn);
+#pragma unroll
+          for (int c = 0; c < HALF / 8; ++c) {
+            if (c_lo + c * 8 < t.width) {
+              uint32_t ap[8], an[8];
+              const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 8);
+              tmem_ld8(t_lane + col, ap);
+              tmem_ld8(t_lane + col + BN, an);
+              tmem_wait_ld();
+              if constexpr (SEEDED) {
+                tmem_st8(t_lane + col, kMagicBits);
+                tmem_st8(t_lane + col + BN, kMagicBits);
+              }
+              const int n = t.n0 + c_lo + c * 8;
+              if constexpr (ACC_OUT) {
+                if constexpr (SEEDED) {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) { ap[i] -= kMagicBits; an[i] -= kMagicBits; }
+                }
+                if (row < args.M) {
+                  int32_t* dp = args.acc_out + (((int64_t)u * 2 + 0) * args.M + row) * args.N + n;
+                  int32_t* dn = args.acc_out + (((int64_t)u * 2 + 1) * args.M + row) * args.N + n;
+#pragma unroll
+                  for (int i = 0; i < 8; i += 4) {
+                    *reinterpret_cast<uint4*>(dp + i) = make_uint4(ap[i], ap[i + 1], ap[i + 2], ap[i + 3]);
+                    *reinterpret_cast<uint4*>(dn + i) = make_uint4(an[i], an[i + 1], an[i + 2], an[i + 3]);
+                  }
+                }
+              } else {
+                uint64_t sw2[4];
+                load_wscales8_pairs(args, u, j, n, sw2);
+                fold8_pairs<SEEDED>(ap, an, sw2, sp2, sn2, y2 + c * 4);
+              }
+            }
+          }
+          if constexpr (SEEDED) tmem_wait_st();
+          release(b);
+          ++ug;
+        }
+        if constexpr (!ACC_OUT) {
+          if (ok && row < args.M) {
+#pragma unroll
+            for (int c = 0; c < HALF / 16; ++c) {
+              if (c_lo + c * 16 < t.width) {
+                float o[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f2_unpack(y2[c * 8 + i], o[2 * i], o[2 * i + 1]);
+                store16<Y_BF16>(args, row, t.n0 + c_lo + c * 16, o);
+              }
+            }
+          }
+        }
+      } else {
+        // One unit per tile: stream column chunks from TMEM straight to memory.
+        // The tile's scales and bias are fetched into L1 while its MMAs run.
+        if (c_lo < t.width) {
+          const int cols = min(HALF, t.width - c_lo);
+          const float* sw_row = static_cast<const float*>(args.wscales) + t.n0 + c_lo;
+          for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
+          if (args.bias != nullptr)
+            for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(args.bias + t.n0 + c_lo + c);
+        }
+        const int b = ug % NBUF;
+        if (!(ok = wait_warp<CLUSTER>(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+        tc_fence_after();
+        const float sp = __ldg(args.s_pos), sn = __ldg(args.s_neg);
+#pragma unroll 1
+        for (int c = 0; c < HALF / 16; ++c) {
+          if (c_lo + c * 16 < t.width) {
+            uint32_t ap[16], an[16];
+            const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 16);
+            tmem_ld16(t_lane + col, ap);
+            tmem_ld16(t_lane + col + BN, an);
+            tmem_wait_ld();
+            if (row < args.M) {
+              const int n = t.n0 + c_lo + c * 16;
+              float sw[16], o[16];
+              load_wscales16(args, 0, 0, n, sw);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+              fold16<false>(ap, an, sw, sp, sn, o);
+              store16<Y_BF16>(args, row, n, o);
+            }
+          }
+        }
+        release(b);
+        ++ug;
+      }
   }
 }
 
@@ -521,7 +855,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
       if constexpr (ASRC == ASRC_CODES) tma_prefetch_desc(&tmap_a2);
       tma_prefetch_desc(&tmap_w);
       int ca = 0, cw = 0;
-      bool ok = true;
+      bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
         Tile t;
         if (!tile_of(args, it, BN, t)) continue;
@@ -558,10 +892,10 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
         }
       }
       // Let every copy this thread started land before the CTA can exit.
-      if constexpr (ASRC == ASRC_X) drain_ring(full_x, C::SX, ca, budget);
-      else drain_ring(full_q, C::SQ, ca, budget);
-      if constexpr (W4) drain_ring(full_wp, C::SWP, cw, budget);
-      else drain_ring(full_w, C::SW, cw, budget);
+      if constexpr (ASRC == ASRC_X) drain_ring(full_x, C::SX, ca, kDrainBudget);
+      else drain_ring(full_q, C::SQ, ca, kDrainBudget);
+      if constexpr (W4) drain_ring(full_wp, C::SWP, cw, kDrainBudget);
+      else drain_ring(full_w, C::SW, cw, kDrainBudget);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
@@ -613,7 +947,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
       }
       // All MMAs this thread issued have landed once the drain barrier flips.
       umma_commit(smem_u32(drain_bar));
-      wait_drain(smem_u32(drain_bar), 0, budget);
+      wait_drain(smem_u32(drain_bar), 0, kDrainBudget);
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------- operand producers
@@ -623,7 +957,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
       const int c0 = (t_id >> 7) * 4;                  // first of its four 16-wide chunks
       int cx = 0, cq = 0, cwp = 0, cw = 0;
       int cur_seg = -1;
-      float rp = 0.0f, rn = 0.0f;
+      QuantParams qpar{0.0f, 0u, 0u};
       bool ok = true;
       for (int it = 0; it < rounds && ok; ++it) {
         Tile t;
@@ -633,8 +967,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
             const int j = kb_segment(args, kb);
             if (j != cur_seg) {
               cur_seg = j;
-              rp = rcp_or_zero(__ldg(args.s_pos + j));
-              rn = rcp_or_zero(__ldg(args.s_neg + j));
+              qpar = quant_params(__ldg(args.s_pos + j), __ldg(args.s_neg + j));
             }
             const int sx = cx % C::SX, sq = cq % C::SQ;
             if (!(ok = wait_warp(smem_u32(full_x + sx), (cx / C::SX) & 1, abort_flag, budget))) break;
@@ -647,7 +980,7 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
               float v[16];
               load_row16<XT>(xs, row, c, v);
               uint4 up, un;
-              quantize16(v, rp, rn, up, un);
+              quantize16_fast(v, qpar, up, un);
               const int off = (c ^ (row & 7)) << 4;
               *reinterpret_cast<uint4*>(qp + off) = up;
               *reinterpret_cast<uint4*>(qn + off) = un;
@@ -690,130 +1023,12 @@ __global__ void __launch_bounds__(kernel_threads(MULTI), 1)
     }
   } else {
     // --------------------------------------------------------- epilogue
-    constexpr int HALF = BN / (epi_warps(MULTI) / 4);   // columns per epilogue thread
     const int quad = warp & 3;
-    const int half = (warp - kEpiWarp0) >> 2;
-    const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    const int units = (args.bits == 4) ? num_kb : args.kseg.count;
-    int ug = 0;
-    bool ok = true;
-    if constexpr (SEEDED) {
-      // Seed both accumulator buffers, then hand them to the MMA warp.
-      const int c_lo = half * HALF;
-      for (int b = 0; b < C::NBUF; ++b) {
-#pragma unroll
-        for (int c = 0; c < HALF / 8; ++c) {
-          const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 8);
-          tmem_st8(t_lane + col, kMagicBits);
-          tmem_st8(t_lane + col + BN, kMagicBits);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0)
-        for (int b = 0; b < C::NBUF; ++b) mbar_arrive(smem_u32(tmem_empty + b));
-    }
-    for (int it = 0; it < rounds && ok; ++it) {
-      Tile t;
-      if (!tile_of(args, it, BN, t)) continue;
-      const int row = t.m0 + quad * 32 + lane;
-      const int c_lo = half * HALF;                 // first tile column of this warp
-      if constexpr (MULTI || ACC_OUT) {
-        float y[MULTI && !ACC_OUT ? HALF : 1];
-#pragma unroll
-        for (int i = 0; i < (MULTI && !ACC_OUT ? HALF : 1); ++i) y[i] = 0.0f;
-        for (int u = 0; u < units; ++u) {
-          const int b = ug % C::NBUF;
-          if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / C::NBUF) & 1, abort_flag, budget))) break;
-          tc_fence_after();
-          const int j = (args.bits == 4) ? args.kseg.segment_of(u * 128) : u;
-          const float sp = __ldg(args.s_pos + j), sn = __ldg(args.s_neg + j);
-#pragma unroll
-          for (int c = 0; c < HALF / 8; ++c) {
-            if (c_lo + c * 8 < t.width) {
-              uint32_t ap[8], an[8];
-              const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 8);
-              tmem_ld8(t_lane + col, ap);
-              tmem_ld8(t_lane + col + BN, an);
-              tmem_wait_ld();
-              if constexpr (SEEDED) {
-                tmem_st8(t_lane + col, kMagicBits);
-                tmem_st8(t_lane + col + BN, kMagicBits);
-              }
-              const int n = t.n0 + c_lo + c * 8;
-              if constexpr (ACC_OUT) {
-                if constexpr (SEEDED) {
-#pragma unroll
-                  for (int i = 0; i < 8; ++i) { ap[i] -= kMagicBits; an[i] -= kMagicBits; }
-                }
-                if (row < args.M) {
-                  int32_t* dp = args.acc_out + (((int64_t)u * 2 + 0) * args.M + row) * args.N + n;
-                  int32_t* dn = args.acc_out + (((int64_t)u * 2 + 1) * args.M + row) * args.N + n;
-#pragma unroll
-                  for (int i = 0; i < 8; i += 4) {
-                    *reinterpret_cast<uint4*>(dp + i) = make_uint4(ap[i], ap[i + 1], ap[i + 2], ap[i + 3]);
-                    *reinterpret_cast<uint4*>(dn + i) = make_uint4(an[i], an[i + 1], an[i + 2], an[i + 3]);
-                  }
-                }
-              } else {
-                float sw[8];
-                load_wscales8(args, u, j, n, sw);
-                if constexpr (SEEDED) fold8_seeded(ap, an, sw, sp, sn, y + c * 8);
-                else fold8<false>(ap, an, sw, sp, sn, y + c * 8);
-              }
-            }
-          }
-          if constexpr (SEEDED) tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(tmem_empty + b));
-          ++ug;
-        }
-        if constexpr (!ACC_OUT) {
-          if (ok && row < args.M) {
-#pragma unroll
-            for (int c = 0; c < HALF / 16; ++c) {
-              if (c_lo + c * 16 < t.width) {
-                float o[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = y[c * 16 + i];
-                store16<Y_BF16>(args, row, t.n0 + c_lo + c * 16, o);
-              }
-            }
-          }
-        }
-      } else {
-        // One unit per tile: stream column chunks from TMEM straight to memory.
-        const int b = ug % C::NBUF;
-        if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / C::NBUF) & 1, abort_flag, budget))) break;
-        tc_fence_after();
-        const float sp = __ldg(args.s_pos), sn = __ldg(args.s_neg);
-#pragma unroll 1
-        for (int c = 0; c < HALF / 16; ++c) {
-          if (c_lo + c * 16 < t.width) {
-            uint32_t ap[16], an[16];
-            const uint32_t col = (uint32_t)(b * 2 * BN + c_lo + c * 16);
-            tmem_ld16(t_lane + col, ap);
-            tmem_ld16(t_lane + col + BN, an);
-            tmem_wait_ld();
-            if (row < args.M) {
-              const int n = t.n0 + c_lo + c * 16;
-              float sw[16], o[16];
-              load_wscales16(args, 0, 0, n, sw);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) o[i] = 0.0f;
-              fold16<false>(ap, an, sw, sp, sn, o);
-              store16<Y_BF16>(args, row, n, o);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(tmem_empty + b));
-        ++ug;
-      }
-    }
+    const int part = (warp - kEpiWarp0) >> 2;
+    epilogue_role<BN, C::NBUF, MULTI, ACC_OUT, Y_BF16, SEEDED>(
+        args, quad, part, lane, tmem_base + ((uint32_t)(quad * 32) << 16), tmem_full,
+        smem_u32(tmem_empty), /*empty_remote=*/false, /*row_shift=*/0, rounds,
+        [&](int it, Tile& t) { return tile_of(args, it, BN, t); }, abort_flag, budget);
   }
 
   // ---------------------------------------------------------------- teardown

@@ -16,6 +16,8 @@
 
 #include "common.cuh"
 #include "gemm_dualscale.cuh"
+#include "gemm_dualscale_inplace.cuh"
+#include "gemm_dualscale_pair.cuh"
 #include "ptx.cuh"
 #include "quant_kernels.cuh"
 
@@ -25,6 +27,7 @@ using sq::SegBounds;
 
 constexpr long long kDefaultWaitBudget = 2000000000LL;  // ~1 s of SM clock
 long long g_wait_budget = kDefaultWaitBudget;
+int g_debug_starve = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int elt_size(sq_dtype t) { return t == SQ_F32 ? 4 : 2; }
@@ -155,6 +158,81 @@ sq_status launch_out(bool acc, bool y_bf16, const CUtensorMap& ta, const CUtenso
                 : launch_gemm<BN, ASRC, XT, W4, false, false, MULTI>(ta, ta2, tw, a, stream);
 }
 
+template <int BN, bool ACC, bool YB, bool MULTI>
+sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tw,
+                      sq::GemmArgs a, cudaStream_t stream) {
+  using C = sq::PairCfg<BN>;
+  auto kern = sq::dualscale_gemm_pair_kernel<BN, ACC, YB, MULTI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_status(e);
+  a.n_full = a.N / BN;
+  a.tail = a.N % BN;
+  a.m_tiles = (a.M + sq::BM_PAIR - 1) / sq::BM_PAIR;
+  a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
+  int pairs = num_sms() / 2;
+  if (pairs > a.num_tiles) pairs = a.num_tiles;
+  kern<<<2 * pairs, sq::kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(ta, ta2, tw, a);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int BN, bool MULTI>
+sq_status launch_pair_out(bool acc, bool y_bf16, const CUtensorMap& ta, const CUtensorMap& ta2,
+                          const CUtensorMap& tw, const sq::GemmArgs& a, cudaStream_t stream) {
+  if constexpr (MULTI) {
+    if (acc) return launch_pair<BN, true, false, true>(ta, ta2, tw, a, stream);
+  }
+  if (acc) return SQ_ERR_UNSUPPORTED;
+  return y_bf16 ? launch_pair<BN, false, true, MULTI>(ta, ta2, tw, a, stream)
+                : launch_pair<BN, false, false, MULTI>(ta, ta2, tw, a, stream);
+}
+
+template <int BN, bool ACC, bool YB, bool MULTI>
+sq_status launch_inplace(const CUtensorMap& tx, const CUtensorMap& tw, sq::GemmArgs a,
+                         cudaStream_t stream) {
+  using C = sq::InplaceCfg<BN>;
+  auto kern = sq::dualscale_gemm_inplace_kernel<BN, ACC, YB, MULTI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_status(e);
+  a.n_full = a.N / BN;
+  a.tail = a.N % BN;
+  a.m_tiles = (a.M + sq::BM - 1) / sq::BM;
+  a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
+  int grid = num_sms();
+  if (grid > a.num_tiles) grid = a.num_tiles;
+  kern<<<grid, sq::kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(tx, tw, a);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int BN, bool MULTI>
+sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const CUtensorMap& tw,
+                             const sq::GemmArgs& a, cudaStream_t stream) {
+  if constexpr (MULTI) {
+    if (acc) return launch_inplace<BN, true, false, true>(tx, tw, a, stream);
+  }
+  if (acc) return SQ_ERR_UNSUPPORTED;
+  return y_bf16 ? launch_inplace<BN, false, true, MULTI>(tx, tw, a, stream)
+                : launch_inplace<BN, false, false, MULTI>(tx, tw, a, stream);
+}
+
+// Whether the fused path quantizes bf16 activations in place (one ring of
+// stages): int8 weights; SEGQUANT_INPLACE=0 selects the separate-ring kernel.
+bool use_inplace(bool w4) {
+  if (w4) return false;
+  if (const char* e = std::getenv("SEGQUANT_INPLACE")) return std::atoi(e) != 0;
+  return true;
+}
+
+// Whether the GEMM from codes runs on CTA pairs (2-SM UMMA): int8 weights and a
+// last tile width that is a multiple of 32 (pair MMA N granularity).
+// SEGQUANT_PAIR=0|1 overrides the default.
+bool use_pair(int64_t N, bool w4) {
+  if (w4 || N % 32 != 0) return false;
+  if (const char* e = std::getenv("SEGQUANT_PAIR")) return std::atoi(e) != 0;
+  return false;
+}
+
 // Output-tile width.  Several units per tile need double-buffered TMEM, which
 // caps BN at 128; fp32 activation stages leave room for BN = 128 only.
 // Otherwise BN in {128, 192, 256} minimises a makespan model of the snake
@@ -221,7 +299,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const bool w4 = (w->bits == 4);
   const bool multi = w4 || kseg.count > 1;
   const bool f32x = (src == ASource::X && xt == SQ_F32);
-  const int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x);
+  const bool pair = (src == ASource::Codes) && use_pair(N, w4);
+  int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x);
+  if (pair && !multi && acc == nullptr) {
+    BN = 256;
+    if (const char* e = std::getenv("SEGQUANT_BN")) BN = std::atoi(e) == 128 ? 128 : 256;
+  }
   CUtensorMap ta, ta2, tw;
   if (src == ASource::X) {
     const int xe = elt_size(xt);
@@ -242,7 +325,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
                    (uint64_t)(K / 2), 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   else
     st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K, (uint64_t)N,
-                   (uint64_t)K, 128, (uint32_t)BN);
+                   (uint64_t)K, 128, (uint32_t)(pair ? BN / 2 : BN));
   if (st != SQ_OK) return st;
 
   sq::GemmArgs a;
@@ -261,11 +344,17 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   a.ldy = ldy;
   a.acc_out = acc;
   a.wait_budget = g_wait_budget;
+  a.starve = g_debug_starve;
 
   using bf = __nv_bfloat16;
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
   const bool yb = (yt == SQ_BF16);
   const bool ac = (acc != nullptr);
+  if (pair) {
+    if (multi || ac) return launch_pair_out<128, true>(ac, yb, ta, ta2, tw, a, stream);
+    if (BN == 256) return launch_pair_out<256, false>(ac, yb, ta, ta2, tw, a, stream);
+    return launch_pair_out<128, false>(ac, yb, ta, ta2, tw, a, stream);
+  }
   if (src == ASource::Codes) {
     if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
     if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
@@ -279,6 +368,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     return launch_out<128, AX, float, false, false>(ac, yb, ta, ta2, tw, a, stream);
   }
   if (w4) return launch_out<128, AX, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
+  if (use_inplace(w4)) {
+    if (multi || ac) return launch_inplace_out<128, true>(ac, yb, ta, tw, a, stream);
+    if (BN == 256) return launch_inplace_out<256, false>(ac, yb, ta, tw, a, stream);
+    if (BN == 192) return launch_inplace_out<192, false>(ac, yb, ta, tw, a, stream);
+    return launch_inplace_out<128, false>(ac, yb, ta, tw, a, stream);
+  }
   if (multi || ac) return launch_out<128, AX, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
   if (BN == 256) return launch_out<256, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
   if (BN == 192) return launch_out<192, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
@@ -307,6 +402,8 @@ const char* sq_status_string(sq_status s) {
 }
 
 void sq_set_wait_budget(int64_t cycles) { g_wait_budget = cycles > 0 ? cycles : kDefaultWaitBudget; }
+
+void sq_debug_starve_pipeline(int32_t enable) { g_debug_starve = enable != 0; }
 
 sq_status sq_qweight_sizes(int32_t bits, int64_t N, int64_t K, int32_t J, int32_t group,
                            size_t* code_bytes, size_t* scale_bytes) {

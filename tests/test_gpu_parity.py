@@ -193,3 +193,122 @@ def test_workloads_full_size_sampled_rows(name):
     y2 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
     assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32),
                        y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2.view(torch.int32))
+
+
+# ------------------------------------------------------------- status word
+def test_calibration_non_finite_sets_range_status():
+    import post_quantized_linear_b200 as pq
+    from post_quantized_linear_b200 import _lib
+    x = torch.randn(64, 256, device="cuda", dtype=torch.bfloat16)
+    x[3, 17] = float("inf")
+    pq.calibrate(x, [0, 256])
+    assert pq.stream_status() == _lib.SQ_ERR_RANGE
+    assert pq.stream_status() == _lib.SQ_OK          # the word is cleared by reading it
+    x[3, 17] = float("nan")
+    pq.calibrate(x, [0, 128, 256])
+    assert pq.stream_status() == _lib.SQ_ERR_RANGE
+
+
+def test_weight_quantization_range_status():
+    import post_quantized_linear_b200 as pq
+    from post_quantized_linear_b200 import _lib
+    w = torch.randn(32, 256, device="cuda") * 0.02
+    w[5, 9] = float("nan")
+    pq.quantize_weights(w, [0, 256], bits=8)
+    assert pq.stream_status() == _lib.SQ_ERR_RANGE
+    w[5, 9] = 1.0e6                                  # 1e6 / 7 overflows binary16
+    pq.quantize_weights(w, [0, 256], bits=4)
+    assert pq.stream_status() == _lib.SQ_ERR_RANGE
+    w[5, 9] = 0.01
+    pq.quantize_weights(w, [0, 256], bits=4)
+    assert pq.stream_status() == _lib.SQ_OK
+
+
+@pytest.mark.parametrize("codes", [False, True])
+def test_starved_pipeline_times_out_and_context_recovers(codes):
+    """Bounded waits: with the producer starved every wait expires; the kernel
+    records SQ_ERR_TIMEOUT, frees its TMEM and exits, and the next launch on the
+    same context is correct again."""
+    import post_quantized_linear_b200 as pq
+    from post_quantized_linear_b200 import _lib
+    c = Case(_small(0))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    assert pq.stream_status() == _lib.SQ_OK
+    pq.set_wait_budget(2_000_000)                   # about a millisecond
+    pq.debug_starve_pipeline(True)
+    try:
+        if codes:
+            pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+        else:
+            c.forward()
+        assert pq.stream_status() == _lib.SQ_ERR_TIMEOUT
+    finally:
+        pq.debug_starve_pipeline(False)
+        pq.set_wait_budget(0)
+    y = c.forward()
+    torch.cuda.synchronize()
+    assert pq.stream_status() == _lib.SQ_OK
+    c.compare_rows(y, np.arange(c.wl.M))
+
+
+# ---------------------------------------------------- 2-SM (CTA pair) GEMM
+PAIR_CASES = [
+    dict(M=300, K=640, N=288, kseg=[0, 640]),                       # ragged M, tail N = 32
+    dict(M=513, K=1152, N=1152, kseg=[0, 1152]),                    # 3 pair rows, N = 4.5 x 256
+    dict(M=256, K=384, N=64, kseg=[0, 384]),                        # one pair tile, narrow N
+    dict(M=390, K=768, N=416, kseg=[0, 256, 768], x_sigmas=[1.0, 4.0]),  # two segments
+    dict(M=100, K=256, N=256, kseg=[0, 256]),                       # the peer CTA's rows are all padding
+]
+
+
+@pytest.mark.parametrize("bn", ["128", "256"])
+@pytest.mark.parametrize("i", range(len(PAIR_CASES)))
+def test_pair_gemm_matches_oracle(i, bn, monkeypatch):
+    """The GEMM from codes on CTA pairs (tcgen05.mma.cta_group::2) gives the
+    oracle's result; several K segments use the double-buffered BN = 128 path."""
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_PAIR", "1")
+    monkeypatch.setenv("SEGQUANT_BN", bn)
+    p = dict(PAIR_CASES[i])
+    wl = W.small_case(p.pop("M"), p.pop("K"), p.pop("N"), seed=40 + i, out="bf16", **p)
+    c = Case(wl)
+    qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(y, np.arange(wl.M))
+    # bit-identical to the one-CTA kernel
+    monkeypatch.setenv("SEGQUANT_PAIR", "0")
+    y1 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b)
+    assert torch.equal(y.view(torch.int16), y1.view(torch.int16))
+
+
+def test_pair_gemm_fp32_bit_exact(monkeypatch):
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_PAIR", "1")
+    wl = W.small_case(300, 640, 288, seed=50, kseg=[0, 256, 640], x_sigmas=[1.0, 3.0], out="bf16")
+    c = Case(wl)
+    qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
+    # with fp32 output the fixed epilogue order makes the result bit-exact
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(y.cpu().numpy(), O.epilogue(*_epi_args(c, wl)))
+
+
+def _epi_args(c, wl):
+    _, acc = c.oracle_rows(np.arange(wl.M))
+    ub, useg = O.units_of(wl.bits, wl.K, wl.kseg)
+    return (acc, useg, c.o_sp, c.o_sn, O.unit_weight_scales(wl.bits, c.o_ws), c.b_np, "f32")
+
+
+@pytest.mark.parametrize("name", ["dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up"])
+def test_pair_gemm_full_size_sampled_rows(name, monkeypatch):
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_PAIR", "1")
+    wl = W.WORKLOADS[name]
+    c = Case(wl)
+    qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(y, sample_rows(wl.M, 96 if wl.N > 4096 else 160))
