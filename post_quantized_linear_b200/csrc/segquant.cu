@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "gemm_dualscale.cuh"
+#include "gemm_dualscale_codes.cuh"
 #include "gemm_dualscale_inplace.cuh"
 #include "gemm_dualscale_pair.cuh"
 #include "ptx.cuh"
@@ -216,6 +217,39 @@ sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const
                 : launch_inplace<BN, false, false, MULTI>(tx, tw, a, stream);
 }
 
+template <int BN, bool YB, bool MULTI>
+sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
+                       sq::GemmArgs a, cudaStream_t stream) {
+  using C = sq::CodesCfg<BN>;
+  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_status(e);
+  a.n_full = a.N / BN;
+  a.tail = a.N % BN;
+  a.m_tiles = (a.M + sq::BM - 1) / sq::BM;
+  a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
+  int grid = num_sms();
+  if (grid > a.num_tiles) grid = a.num_tiles;
+  kern<<<grid, sq::codes_kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, a);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int BN, bool MULTI>
+sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+                           const CUtensorMap& tw, const sq::GemmArgs& a, cudaStream_t stream) {
+  return y_bf16 ? launch_codes<BN, true, MULTI>(tqp, tqn, tw, a, stream)
+                : launch_codes<BN, false, MULTI>(tqp, tqn, tw, a, stream);
+}
+
+// Whether the GEMM from int8 codes runs the one-ring kernel (codes and weight
+// tile in one stage); SEGQUANT_CODES_RING=0 selects the kernel with separate
+// operand rings.
+bool use_codes_ring() {
+  if (const char* e = std::getenv("SEGQUANT_CODES_RING")) return std::atoi(e) != 0;
+  return true;
+}
+
 // Whether the fused path quantizes bf16 activations in place (one ring of
 // stages): int8 weights; SEGQUANT_INPLACE=0 selects the separate-ring kernel.
 bool use_inplace(bool w4) {
@@ -357,6 +391,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   }
   if (src == ASource::Codes) {
     if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
+    if (!ac && use_codes_ring()) {
+      if (multi) return launch_codes_out<128, true>(yb, ta, ta2, tw, a, stream);
+      if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, a, stream);
+      if (BN == 192) return launch_codes_out<192, false>(yb, ta, ta2, tw, a, stream);
+      return launch_codes_out<128, false>(yb, ta, ta2, tw, a, stream);
+    }
     if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
     if (BN == 256) return launch_out<256, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
     if (BN == 192) return launch_out<192, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);

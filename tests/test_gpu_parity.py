@@ -112,6 +112,27 @@ def test_tile_width_variants_match_oracle(bn, codes, monkeypatch):
     c.compare_rows(y, np.arange(wl.M))
 
 
+@pytest.mark.parametrize("bn", ["128", "192", "256"])
+@pytest.mark.parametrize("i", [0, 1, 2, 5])
+def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch):
+    """The GEMM from codes with one ring of stages (codes and weights in one
+    stage) and with separate operand rings: the oracle's result, bit-identical
+    to each other, on one and several K segments, bf16 and fp32 outputs."""
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_BN", bn)
+    c = Case(_small(i))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    monkeypatch.setenv("SEGQUANT_CODES_RING", "1")
+    y1 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    monkeypatch.setenv("SEGQUANT_CODES_RING", "0")
+    y0 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(y1, np.arange(c.wl.M))
+    iv = torch.int16 if y1.dtype == torch.bfloat16 else torch.int32
+    assert torch.equal(y1.view(iv), y0.view(iv))
+
+
 def test_forward_exact_in_fp32():
     """With the fp32 epilogue order the kernel reproduces the oracle bit for bit."""
     c = Case(_small(1))
