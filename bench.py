@@ -38,11 +38,20 @@ FALLBACK_HBM_GBS = 6650.0
 INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu
-# capture of the current kernel build (profiles/dualscale_gemm_codes_*.md);
-# keyed by (workload, path).  Absent: no capture of the current build.
-NCU_TRAFFIC_BYTES = {
-    ("dit_xl2_fc2_cfg", "codes"): 80838656 + 4266752,
-}
+# capture of the current kernel build (profiles/*.md); keyed by (workload,
+# path).  Absent: no capture of the current build.
+NCU_TRAFFIC_BYTES = {}
+
+
+def gemm_kernel_name(path: str, bits: int, x_dtype: str) -> str:
+    """The GEMM kernel a forward of this path launches."""
+    if bits == 4:
+        return "dualscale_gemm_kernel"
+    if path == "codes":
+        return "dualscale_gemm_codes_kernel"
+    if path == "combined":
+        return "dualscale_gemm_combined_kernel"
+    return "dualscale_gemm_inplace_kernel" if x_dtype == "bf16" else "dualscale_gemm_kernel"
 
 
 def parse_args():
@@ -52,9 +61,11 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_xl2_fc2_cfg")
-    ap.add_argument("--path", choices=["fused", "codes"], default="codes",
+    ap.add_argument("--path", choices=["fused", "codes", "combined"], default="codes",
                     help="fused: quantize X inside the GEMM; codes: quantize X once into "
-                         "q+/q- code tensors, then the GEMM loads the codes")
+                         "q+/q- code tensors, then the GEMM loads the codes; combined: quantize "
+                         "X once into c = q+ + q- (one byte per activation), then the GEMM "
+                         "loads c and splits it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -259,11 +270,12 @@ def run_ours(args):
     qw = pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=wl.bits)
     y = torch.empty((wl.M, wl.N), dtype=out_dtype, device=dev)
     calib = xd if wl.calib_rows is None else xd[: wl.calib_rows]
-    use_codes = args.path == "codes"
+    use_codes = args.path in ("codes", "combined")
+    combined = args.path == "combined"
     if use_codes:
         ldq = (wl.K + 15) // 16 * 16
         qp_buf = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
-        qn_buf = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
+        qn_buf = None if combined else torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -273,15 +285,22 @@ def run_ours(args):
         pq.quantize_weights(ws, wl.kseg, wl.nseg, bits=wl.bits, out=qw)
         forward(xs, ys, gemm_events)
 
-    def forward(xs, ys, gemm_events=None):
-        if use_codes:
-            pq.quantize_activations(xs, wl.kseg, sp, sn, out=(qp_buf, qn_buf))
-        if gemm_events:
-            gemm_events[0].record(stream)
-        if use_codes:
+    def gemm(xs, ys):
+        if combined:
+            pq.linear_from_combined(qp_buf, qw, sp, sn, bd, out=ys)
+        elif use_codes:
             pq.linear_from_codes(qp_buf, qn_buf, qw, sp, sn, bd, out=ys)
         else:
             pq.linear(xs, qw, sp, sn, bd, out=ys)
+
+    def forward(xs, ys, gemm_events=None):
+        if combined:
+            pq.quantize_activations_combined(xs, wl.kseg, sp, sn, out=qp_buf)
+        elif use_codes:
+            pq.quantize_activations(xs, wl.kseg, sp, sn, out=(qp_buf, qn_buf))
+        if gemm_events:
+            gemm_events[0].record(stream)
+        gemm(xs, ys)
         if gemm_events:
             gemm_events[1].record(stream)
 
@@ -313,10 +332,7 @@ def run_ours(args):
         return graph
 
     def gemm_only():
-        if use_codes:
-            pq.linear_from_codes(qp_buf, qn_buf, qw, sp, sn, bd, out=y)
-        else:
-            pq.linear(xd, qw, sp, sn, bd, out=y)
+        gemm(xd, y)
 
     step_graph = capture(step)
     fwd_graph = capture(lambda: forward(xd, y))
@@ -406,7 +422,7 @@ def run_ours(args):
             "data": "synthetic",
             "config": config_of(wl, "flushed (256 MiB write between steps)", args.path),
             "roofline": {
-                "bound": "tensor", "kernel": "dualscale_gemm_kernel",
+                "bound": "tensor", "kernel": gemm_kernel_name(args.path, wl.bits, wl.x_dtype),
                 "achieved": gemm_tops, "peak": int8_peak_tops, "unit": "TOPS",
                 "frac": gemm_tops / int8_peak_tops,
                 "traffic": NCU_TRAFFIC_BYTES.get((wl.name, args.path)),

@@ -168,6 +168,32 @@ sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t
                                   const float* s_neg, int8_t* q_pos, int8_t* q_neg, int64_t ldq,
                                   sq_stream_t stream);
 
+/* DualScale codes in one byte per activation: c = q+ + q- (SegQuant DualScale,
+ * Spanish technical summary 2.B: X = X+ + X-, the two parts have disjoint
+ * support, so at most one of q+, q- is non-zero and c in [-127, 127] carries
+ * both: q+ = max(c, 0), q- = min(c, 0)).  Same rules and scales as
+ * sq_quantize_activations.  c: device int8 [M, K], row stride ldc (a multiple
+ * of 16), 16-byte aligned; written by the call.  Requirements and errors as for
+ * sq_quantize_activations. */
+sq_status sq_quantize_activations_combined(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                           int64_t ldx, const sq_segments* kseg,
+                                           const float* s_pos, const float* s_neg, int8_t* c,
+                                           int64_t ldc, sq_stream_t stream);
+
+/* The forward pass from combined codes (written by
+ * sq_quantize_activations_combined with the same scales): the kernel loads one
+ * int8 code tile per k block by TMA, splits it into q+ and q- in shared memory
+ * and runs the two tensor-core products and the fused epilogue of
+ * sq_linear_forward, so the result is identical to sq_linear_forward and
+ * sq_linear_forward_codes.  c: device int8 [M, K], row stride ldc (a multiple
+ * of 16), 16-byte aligned.  int8 weights only (bits = 4 returns
+ * SQ_ERR_UNSUPPORTED).  Other arguments and requirements as for
+ * sq_linear_forward. */
+sq_status sq_linear_forward_combined(const int8_t* c, int64_t ldc, int64_t M, int64_t K,
+                                     const sq_qweight* w, const float* s_pos, const float* s_neg,
+                                     const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                                     sq_stream_t stream);
+
 /* Test surface: the same kernel as sq_linear_forward, but the epilogue writes
  * the raw int32 accumulators of every unit instead of Y:
  * acc[u][p][m][n], p = 0 for the (+) product, 1 for the (-) product; U units

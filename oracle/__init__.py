@@ -134,6 +134,13 @@ def quantize_activations(x: np.ndarray, kbounds, s_pos, s_neg):
     return qp, qn
 
 
+def quantize_activations_combined(x: np.ndarray, kbounds, s_pos, s_neg):
+    """Combined DualScale codes c = q+ + q-, int8 [M, K] (SegQuant DualScale:
+    X = X+ + X- with disjoint support, so at most one of q+, q- is non-zero)."""
+    qp, qn = quantize_activations(x, kbounds, s_pos, s_neg)
+    return (qp.astype(np.int16) + qn.astype(np.int16)).astype(np.int8)
+
+
 def quantize_weights_w8(w: np.ndarray, kbounds):
     """Per-(channel, K-segment) int8 codes [N, K] and fp32 scales [J, N]."""
     w = np.ascontiguousarray(w, dtype=np.float32)

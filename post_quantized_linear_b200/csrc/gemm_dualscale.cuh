@@ -770,6 +770,129 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, int quad, in
   }
 }
 
+// ------------------------------------------------- epilogue through TMA stores
+// One unit per tile, output written by TMA tensor stores from a per-warp
+// staging tile of 32 rows x 32 columns in shared memory.  Storing through TMA
+// writes whole 128-byte lines instead of one 16-byte piece per row per lane,
+// and the warp does not wait for the writes; the accumulators are released as
+// soon as the warp's last TMEM columns are in registers.
+//
+// Staging layout: row r (the warp's TMEM lane r) of the 32-column tile at
+// r * ROWB, 16-byte chunk j of the row at position j ^ f(r) -- the TMA
+// 64-byte swizzle for bf16 rows of 64 bytes (f(r) = (r >> 1) & 3) and the
+// 128-byte swizzle for fp32 rows of 128 bytes (f(r) = r & 7) -- so a warp's
+// 16-byte stores touch every bank evenly.  The buffer is 1024-byte aligned.
+constexpr int kStageYBytes = 32 * 128;   // per epilogue warp (fp32 worst case)
+
+template <bool Y_BF16>
+__device__ __forceinline__ void stage16(const GemmArgs& a, int n, float (&o)[16], uint8_t* srow,
+                                        int r, int half) {
+  if (a.bias != nullptr) {
+    const float4* b4 = reinterpret_cast<const float4*>(a.bias + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = __ldg(b4 + i);
+      o[4 * i] = __fadd_rn(o[4 * i], t.x);
+      o[4 * i + 1] = __fadd_rn(o[4 * i + 1], t.y);
+      o[4 * i + 2] = __fadd_rn(o[4 * i + 2], t.z);
+      o[4 * i + 3] = __fadd_rn(o[4 * i + 3], t.w);
+    }
+  }
+  if constexpr (Y_BF16) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+      pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    const int f = (r >> 1) & 3;
+    *reinterpret_cast<uint4*>(srow + (((2 * half) ^ f) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4*>(srow + (((2 * half + 1) ^ f) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    const int f = r & 7;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(srow + (((4 * half + i) ^ f) << 4)) =
+          make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  }
+}
+
+// Epilogue warps: EPW of them, warp (quad, part) owns TMEM lanes quad*32..+31
+// (tile rows) and columns [part*HALF, (part+1)*HALF).
+template <int BN, int NBUF, int EPW, bool Y_BF16, class TileFn>
+__device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
+                                                   uint8_t* stage_y, int quad, int part, int lane,
+                                                   uint32_t t_lane, uint64_t* tmem_full,
+                                                   uint32_t empty_base, int rounds, TileFn tile_fn,
+                                                   volatile int* abort_flag, long long budget) {
+  constexpr int HALF = BN / (EPW / 4);
+  constexpr int ROWB = Y_BF16 ? 64 : 128;
+  static_assert(HALF % 32 == 0, "32-column store passes");
+  uint8_t* srow = stage_y + lane * ROWB;
+  const uint32_t sbase = smem_u32(stage_y);
+  auto release = [&](int b) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
+  };
+  int ug = 0;
+  bool ok = true, pending = false;
+  for (int it = 0; it < rounds && ok; ++it) {
+    Tile t;
+    if (!tile_fn(it, t)) continue;
+    const int c_lo = part * HALF;
+    const int cols = min(HALF, t.width - c_lo);   // may be <= 0 on a narrow tail tile
+    if (cols > 0) {
+      const float* sw_row = static_cast<const float*>(args.wscales) + t.n0 + c_lo;
+      for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
+      if (args.bias != nullptr)
+        for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(args.bias + t.n0 + c_lo + c);
+    }
+    const int b = ug % NBUF;
+    if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+    tc_fence_after();
+    const float sp = __ldg(args.s_pos), sn = __ldg(args.s_neg);
+    const int npass = cols > 0 ? (cols + 31) / 32 : 0;
+    for (int p = 0; p < npass; ++p) {
+      const int col = c_lo + p * 32;
+      if (pending) {   // the previous store has read the staging tile
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cc = col + 16 * h;
+        if (cc < t.width) {
+          uint32_t ap[16], an[16];
+          const uint32_t tcol = (uint32_t)(b * 2 * BN + cc);
+          tmem_ld16(t_lane + tcol, ap);
+          tmem_ld16(t_lane + tcol + BN, an);
+          tmem_wait_ld();
+          float sw[16], o[16];
+          load_wscales16(args, 0, 0, t.n0 + cc, sw);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+          fold16<false>(ap, an, sw, sp, sn, o);
+          stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+        }
+      }
+      if (p == npass - 1) release(b);   // this warp's accumulator columns are all read
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+        bulk_commit_group();
+      }
+      pending = true;
+    }
+    if (npass == 0) release(b);
+    ++ug;
+  }
+  // Every store has completed before the CTA (and its shared memory) exits.
+  if (lane == 0) bulk_wait_all();
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ kernel
 // MULTI: more than one unit per tile (several K segments, or int4 groups):
 // partial outputs stay in registers across units (BN = 128 only, 16 epilogue

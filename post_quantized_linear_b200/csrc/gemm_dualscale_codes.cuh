@@ -12,8 +12,10 @@
 //   * no operand-producer warps: warp 0 issues TMA, warp 1 owns TMEM and
 //     issues the MMAs, warps 2.. run the epilogue (8 warps, or 16 when a tile
 //     folds several units).
-// Stage sizes: 32 KiB of codes + BN x 128 bytes of weights; four stages for
-// BN = 128 and 192, three for BN = 256.
+// Stage sizes: 32 KiB of codes + BN x 128 bytes of weights.  With one unit per
+// tile the output leaves through TMA stores from 32 KiB of staging tiles
+// (epilogue_tma_store), leaving room for four stages at BN = 128 and three at
+// BN = 192 and 256.
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -26,15 +28,18 @@ __host__ __device__ constexpr int codes_kernel_threads(bool multi) {
   return (kCodesEpiWarp0 + epi_warps(multi)) * 32;
 }
 
-template <int BN_>
+template <int BN_, bool MULTI>
 struct CodesCfg {
   static constexpr int BN = BN_;
   static constexpr int A_BYTES = 2 * BM * BK;   // q+ tile, q- tile
   static constexpr int W_BYTES = BN * BK;
   static constexpr int STAGE = A_BYTES + W_BYTES;
-  static constexpr int S = (kStageBudget / STAGE) < 8 ? (kStageBudget / STAGE) : 8;
+  // One unit per tile: Y leaves through per-warp staging tiles and TMA stores.
+  static constexpr int Y_BYTES = MULTI ? 0 : epi_warps(false) * kStageYBytes;
+  static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
   static constexpr int NBUF = (BN <= 128) ? 2 : 1;
-  static constexpr int OFF_BAR = S * STAGE;
+  static constexpr int OFF_Y = S * STAGE;
+  static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
   static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1;  // full, empty; tmem full/empty; drain
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -49,8 +54,9 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
+                                const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN>;
+  using C = CodesCfg<BN, MULTI>;
   static_assert(!MULTI || BN == 128, "several units per tile need double-buffered TMEM");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -99,6 +105,7 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
       tma_prefetch_desc(&tmap_qp);
       tma_prefetch_desc(&tmap_qn);
       tma_prefetch_desc(&tmap_w);
+      if constexpr (!MULTI) tma_prefetch_desc(&tmap_y);
       int c = 0;
       bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
@@ -168,10 +175,17 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
     // lane quarter once per column part.
     const int quad = warp & 3;
     const int part = (warp - kCodesEpiWarp0) >> 2;
-    epilogue_role<BN, C::NBUF, MULTI, false, Y_BF16, false>(
-        args, quad, part, lane, tmem_base + ((uint32_t)(quad * 32) << 16), tmem_full,
-        smem_u32(tmem_empty), /*empty_remote=*/false, /*row_shift=*/0, rounds, tiles, abort_flag,
-        budget);
+    const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
+    if constexpr (MULTI) {
+      epilogue_role<BN, C::NBUF, MULTI, false, Y_BF16, false>(
+          args, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), /*empty_remote=*/false,
+          /*row_shift=*/0, rounds, tiles, abort_flag, budget);
+    } else {
+      uint8_t* stage_y = smem + C::OFF_Y + (warp - kCodesEpiWarp0) * kStageYBytes;
+      epilogue_tma_store<BN, C::NBUF, epi_warps(false), Y_BF16>(
+          args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty),
+          rounds, tiles, abort_flag, budget);
+    }
   }
 
   // ---------------------------------------------------------------- teardown

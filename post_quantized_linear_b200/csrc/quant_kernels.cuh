@@ -169,8 +169,8 @@ __device__ __forceinline__ void load16(const XT* p, float (&v)[16]) {
 // every row it visits (rows blockIdx.y*8 + y, stepping by gridDim.y*8), so its
 // segment and reciprocal scales are fixed; a warp reads 1 KiB (bf16) and
 // writes 512 bytes of each code tensor per row.
-template <typename XT>
-__global__ void __launch_bounds__(256) quantize_activations_kernel(
+template <typename XT, bool COMBINED>
+__device__ __forceinline__ void quantize_activations_body(
     const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
     int8_t* __restrict__ q_neg, int64_t ldq) {
@@ -186,14 +186,41 @@ __global__ void __launch_bounds__(256) quantize_activations_kernel(
     uint32_t p[16], n[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) { p[i] = code_pos(v[i], rp); n[i] = code_neg(v[i], rn); }
-    uint4 up, un;
+    if constexpr (COMBINED) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) p[i] += n[i];
+    }
+    uint4 up;
     up.x = pack4_low(p[0], p[1], p[2], p[3]);   up.y = pack4_low(p[4], p[5], p[6], p[7]);
     up.z = pack4_low(p[8], p[9], p[10], p[11]); up.w = pack4_low(p[12], p[13], p[14], p[15]);
-    un.x = pack4_low(n[0], n[1], n[2], n[3]);   un.y = pack4_low(n[4], n[5], n[6], n[7]);
-    un.z = pack4_low(n[8], n[9], n[10], n[11]); un.w = pack4_low(n[12], n[13], n[14], n[15]);
     *reinterpret_cast<uint4*>(q_pos + (int64_t)m * ldq + k) = up;
-    *reinterpret_cast<uint4*>(q_neg + (int64_t)m * ldq + k) = un;
+    if constexpr (!COMBINED) {
+      uint4 un;
+      un.x = pack4_low(n[0], n[1], n[2], n[3]);   un.y = pack4_low(n[4], n[5], n[6], n[7]);
+      un.z = pack4_low(n[8], n[9], n[10], n[11]); un.w = pack4_low(n[12], n[13], n[14], n[15]);
+      *reinterpret_cast<uint4*>(q_neg + (int64_t)m * ldq + k) = un;
+    }
   }
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(256) quantize_activations_kernel(
+    const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
+    const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
+    int8_t* __restrict__ q_neg, int64_t ldq) {
+  quantize_activations_body<XT, false>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
+}
+
+// Combined codes c = q+ + q- (one signed byte per activation): an element
+// falls in exactly one branch, so the two magic-rounded words carry its code
+// in their low bytes and the other branch's low byte is 0; their sum's low
+// byte is c.
+template <typename XT>
+__global__ void __launch_bounds__(256) quantize_activations_combined_kernel(
+    const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
+    const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ c,
+    int64_t ldc) {
+  quantize_activations_body<XT, true>(x, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc);
 }
 
 // ------------------------------------------------------ weight quantization

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "gemm_dualscale.cuh"
 #include "gemm_dualscale_codes.cuh"
+#include "gemm_dualscale_combined.cuh"
 #include "gemm_dualscale_inplace.cuh"
 #include "gemm_dualscale_pair.cuh"
 #include "ptx.cuh"
@@ -219,8 +220,8 @@ sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const
 
 template <int BN, bool YB, bool MULTI>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
-                       sq::GemmArgs a, cudaStream_t stream) {
-  using C = sq::CodesCfg<BN>;
+                       const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
+  using C = sq::CodesCfg<BN, MULTI>;
   auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -231,15 +232,51 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int grid = num_sms();
   if (grid > a.num_tiles) grid = a.num_tiles;
-  kern<<<grid, sq::codes_kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, a);
+  kern<<<grid, sq::codes_kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
   return cuda_status(cudaGetLastError());
 }
 
 template <int BN, bool MULTI>
 sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
-                           const CUtensorMap& tw, const sq::GemmArgs& a, cudaStream_t stream) {
-  return y_bf16 ? launch_codes<BN, true, MULTI>(tqp, tqn, tw, a, stream)
-                : launch_codes<BN, false, MULTI>(tqp, tqn, tw, a, stream);
+                           const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                           cudaStream_t stream) {
+  return y_bf16 ? launch_codes<BN, true, MULTI>(tqp, tqn, tw, ty, a, stream)
+                : launch_codes<BN, false, MULTI>(tqp, tqn, tw, ty, a, stream);
+}
+
+// Tensor map of Y for the TMA-store epilogue: boxes of 32 rows x 32 columns,
+// bf16 rows of 64 bytes in the 64-byte swizzle, fp32 rows of 128 bytes in the
+// 128-byte swizzle (the staging layout of epilogue_tma_store).
+sq_status make_tmap_y(CUtensorMap* map, void* y, sq_dtype yt, int64_t M, int64_t N, int64_t ldy) {
+  const bool bf = (yt == SQ_BF16);
+  return make_tmap(map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y,
+                   (uint64_t)N, (uint64_t)M, (uint64_t)(ldy * (bf ? 2 : 4)), 32, 32,
+                   bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BN, bool YB, bool MULTI>
+sq_status launch_combined(const CUtensorMap& tc, const CUtensorMap& tw, sq::GemmArgs a,
+                          cudaStream_t stream) {
+  using C = sq::CombinedCfg<BN>;
+  auto kern = sq::dualscale_gemm_combined_kernel<BN, YB, MULTI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_status(e);
+  a.n_full = a.N / BN;
+  a.tail = a.N % BN;
+  a.m_tiles = (a.M + sq::BM - 1) / sq::BM;
+  a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
+  int grid = num_sms();
+  if (grid > a.num_tiles) grid = a.num_tiles;
+  kern<<<grid, sq::combined_kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(tc, tw, a);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int BN, bool MULTI>
+sq_status launch_combined_out(bool y_bf16, const CUtensorMap& tc, const CUtensorMap& tw,
+                              const sq::GemmArgs& a, cudaStream_t stream) {
+  return y_bf16 ? launch_combined<BN, true, MULTI>(tc, tw, a, stream)
+                : launch_combined<BN, false, MULTI>(tc, tw, a, stream);
 }
 
 // Whether the GEMM from int8 codes runs the one-ring kernel (codes and weight
@@ -298,7 +335,57 @@ int choose_bn(int64_t M, int64_t N, bool multi, bool f32x) {
   return c192 <= c128 ? 192 : 128;
 }
 
-enum class ASource { X, Codes };
+// DualScale codes of X: q+ and q-, or (combined) the code c = q+ + q-
+// written to q_pos.
+sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                         const sq_segments* kseg, const float* s_pos, const float* s_neg,
+                         int8_t* q_pos, int8_t* q_neg, int64_t ldq, bool combined,
+                         cudaStream_t s) {
+  if (!dtype_ok(xt) || M < 0 || K <= 0 || ldx < K || ldq < K) return SQ_ERR_INVALID_ARG;
+  if (K > SQ_MAX_K) return SQ_ERR_RANGE;
+  SegBounds sb;
+  sq_status st = check_segments(kseg, K, SQ_MAX_SEGMENTS, 128, &sb);
+  if (st != SQ_OK) return st;
+  if (K % 16 != 0) return SQ_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX) return SQ_ERR_RANGE;
+  if (M == 0) return SQ_OK;
+  if (x == nullptr || s_pos == nullptr || s_neg == nullptr || q_pos == nullptr ||
+      (!combined && q_neg == nullptr))
+    return SQ_ERR_INVALID_ARG;
+  const int xe = elt_size(xt);
+  if (!aligned16(x) || (ldx * xe) % 16 != 0 || !aligned16(q_pos) ||
+      (!combined && !aligned16(q_neg)) || ldq % 16 != 0)
+    return SQ_ERR_ALIGNMENT;
+  const int64_t groups = K / 16;
+  const int gx = (int)((groups + 31) / 32);
+  int64_t gy = (M + 7) / 8;
+  const int64_t cap = ((int64_t)num_sms() * 16 + gx - 1) / gx;  // ~16 blocks of 256 per SM
+  if (gy > cap) gy = cap;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  dim3 grid(gx, (unsigned)gy), block(32, 8);
+  using bf = __nv_bfloat16;
+  if (combined) {
+    if (xt == SQ_BF16)
+      sq::quantize_activations_combined_kernel<bf><<<grid, block, 0, s>>>(
+          static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+    else
+      sq::quantize_activations_combined_kernel<float><<<grid, block, 0, s>>>(
+          static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+  } else {
+    if (xt == SQ_BF16)
+      sq::quantize_activations_kernel<bf><<<grid, block, 0, s>>>(
+          static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, q_neg,
+          ldq);
+    else
+      sq::quantize_activations_kernel<float><<<grid, block, 0, s>>>(
+          static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, q_neg,
+          ldq);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+enum class ASource { X, Codes, Combined };
 
 sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_pos,
                       const int8_t* q_neg, int64_t ldq, int64_t M, int64_t K, int64_t ldx,
@@ -313,17 +400,20 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   if (st != SQ_OK) return st;
   const int64_t N = w->N;
   if (src == ASource::X && ldx < K) return SQ_ERR_INVALID_ARG;
-  if (src == ASource::Codes && ldq < K) return SQ_ERR_INVALID_ARG;
+  if (src != ASource::X && ldq < K) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::Combined && w->bits != 8) return SQ_ERR_UNSUPPORTED;
   if (acc == nullptr && ldy < N) return SQ_ERR_INVALID_ARG;
   if (M > (int64_t)INT32_MAX - 2 * sq::BM) return SQ_ERR_RANGE;
   if (M == 0) return SQ_OK;
   if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::X && x == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::Codes && (q_pos == nullptr || q_neg == nullptr)) return SQ_ERR_INVALID_ARG;
+  if (src == ASource::Combined && q_pos == nullptr) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && y == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::X && (!aligned16(x) || (ldx * elt_size(xt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (src == ASource::Codes && (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0))
     return SQ_ERR_ALIGNMENT;
+  if (src == ASource::Combined && (!aligned16(q_pos) || ldq % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (acc == nullptr && (!aligned16(y) || (ldy * elt_size(yt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (acc != nullptr && !aligned16(acc)) return SQ_ERR_ALIGNMENT;
   if (bias != nullptr && !aligned16(bias)) return SQ_ERR_ALIGNMENT;
@@ -350,9 +440,13 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
                    (uint64_t)ldq, 128, sq::BM);
     if (st != SQ_OK) return st;
-    st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
-                   (uint64_t)ldq, 128, sq::BM);
-    if (st != SQ_OK) return st;
+    if (src == ASource::Codes) {
+      st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
+                     (uint64_t)ldq, 128, sq::BM);
+      if (st != SQ_OK) return st;
+    } else {
+      ta2 = ta;
+    }
   }
   if (w4)
     st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)(K / 2), (uint64_t)N,
@@ -384,6 +478,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
   const bool yb = (yt == SQ_BF16);
   const bool ac = (acc != nullptr);
+  if (src == ASource::Combined) {
+    if (multi) return launch_combined_out<128, true>(yb, ta, tw, a, stream);
+    if (BN == 256) return launch_combined_out<256, false>(yb, ta, tw, a, stream);
+    if (BN == 192) return launch_combined_out<192, false>(yb, ta, tw, a, stream);
+    return launch_combined_out<128, false>(yb, ta, tw, a, stream);
+  }
   if (pair) {
     if (multi || ac) return launch_pair_out<128, true>(ac, yb, ta, ta2, tw, a, stream);
     if (BN == 256) return launch_pair_out<256, false>(ac, yb, ta, ta2, tw, a, stream);
@@ -392,10 +492,13 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   if (src == ASource::Codes) {
     if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
     if (!ac && use_codes_ring()) {
-      if (multi) return launch_codes_out<128, true>(yb, ta, ta2, tw, a, stream);
-      if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, a, stream);
-      if (BN == 192) return launch_codes_out<192, false>(yb, ta, ta2, tw, a, stream);
-      return launch_codes_out<128, false>(yb, ta, ta2, tw, a, stream);
+      CUtensorMap ty;
+      st = make_tmap_y(&ty, y, yt, M, N, ldy);
+      if (st != SQ_OK) return st;
+      if (multi) return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
+      if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, ty, a, stream);
+      if (BN == 192) return launch_codes_out<192, false>(yb, ta, ta2, tw, ty, a, stream);
+      return launch_codes_out<128, false>(yb, ta, ta2, tw, ty, a, stream);
     }
     if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
     if (BN == 256) return launch_out<256, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
@@ -545,38 +648,16 @@ sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t
                                   const sq_segments* kseg, const float* s_pos,
                                   const float* s_neg, int8_t* q_pos, int8_t* q_neg, int64_t ldq,
                                   sq_stream_t stream) {
-  if (!dtype_ok(xt) || M < 0 || K <= 0 || ldx < K || ldq < K) return SQ_ERR_INVALID_ARG;
-  if (K > SQ_MAX_K) return SQ_ERR_RANGE;
-  SegBounds sb;
-  sq_status st = check_segments(kseg, K, SQ_MAX_SEGMENTS, 128, &sb);
-  if (st != SQ_OK) return st;
-  if (K % 16 != 0) return SQ_ERR_UNSUPPORTED;
-  if (M > (int64_t)INT32_MAX) return SQ_ERR_RANGE;
-  if (M == 0) return SQ_OK;
-  if (x == nullptr || s_pos == nullptr || s_neg == nullptr || q_pos == nullptr || q_neg == nullptr)
-    return SQ_ERR_INVALID_ARG;
-  const int xe = elt_size(xt);
-  if (!aligned16(x) || (ldx * xe) % 16 != 0 || !aligned16(q_pos) || !aligned16(q_neg) ||
-      ldq % 16 != 0)
-    return SQ_ERR_ALIGNMENT;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t groups = K / 16;
-  const int gx = (int)((groups + 31) / 32);
-  int64_t gy = (M + 7) / 8;
-  const int64_t cap = ((int64_t)num_sms() * 16 + gx - 1) / gx;  // ~16 blocks of 256 per SM
-  if (gy > cap) gy = cap;
-  if (gy > 65535) gy = 65535;
-  if (gy < 1) gy = 1;
-  dim3 grid(gx, (unsigned)gy), block(32, 8);
-  if (xt == SQ_BF16)
-    sq::quantize_activations_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos,
-        q_neg, ldq);
-  else
-    sq::quantize_activations_kernel<float><<<grid, block, 0, s>>>(
-        static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, q_neg,
-        ldq);
-  return cuda_status(cudaGetLastError());
+  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq, false,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quantize_activations_combined(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                           int64_t ldx, const sq_segments* kseg,
+                                           const float* s_pos, const float* s_neg, int8_t* c,
+                                           int64_t ldc, sq_stream_t stream) {
+  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc, true,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_linear_forward(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
@@ -592,6 +673,14 @@ sq_status sq_linear_forward_codes(const int8_t* q_pos, const int8_t* q_neg, int6
                                   const float* s_neg, const float* bias, void* y, sq_dtype yt,
                                   int64_t ldy, sq_stream_t stream) {
   return gemm_common(ASource::Codes, nullptr, SQ_BF16, q_pos, q_neg, ldq, M, K, 0, w, s_pos,
+                     s_neg, bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear_forward_combined(const int8_t* c, int64_t ldc, int64_t M, int64_t K,
+                                     const sq_qweight* w, const float* s_pos, const float* s_neg,
+                                     const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                                     sq_stream_t stream) {
+  return gemm_common(ASource::Combined, nullptr, SQ_BF16, c, nullptr, ldc, M, K, 0, w, s_pos,
                      s_neg, bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 

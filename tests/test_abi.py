@@ -121,6 +121,34 @@ def test_calibrate_and_quantize_validation():
     assert lib.sq_quantize_weights(FAKE, 0, 256, 500, 500, ctypes.byref(qw), None) == _lib.SQ_ERR_UNSUPPORTED
 
 
+def test_combined_code_entry_points_validate_before_launch():
+    lib = _lib.load()
+    L = _lib
+    seg, keep = _lib.segments((0, 512))
+    qc = lib.sq_quantize_activations_combined
+    assert qc(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, 520, None) == L.SQ_ERR_ALIGNMENT
+    assert qc(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, None, 512, None) == L.SQ_ERR_INVALID_ARG
+    assert qc(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, 256, None) == L.SQ_ERR_INVALID_ARG
+    assert qc(FAKE, 1, 0, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, 512, None) == L.SQ_OK
+    bad, keep2 = _lib.segments((0, 100, 512))
+    assert qc(FAKE, 1, 16, 512, 512, ctypes.byref(bad), FAKE, FAKE, FAKE, 512, None) == L.SQ_ERR_UNSUPPORTED
+
+    def fwd(c=FAKE, ldc=512, M=256, K=512, qw=None, y=FAKE, yt=L.SQ_BF16, ldy=256):
+        if qw is None:
+            qw, k = _qw(K=K)
+            return lib.sq_linear_forward_combined(c, ldc, M, K, ctypes.byref(qw), FAKE, FAKE, None,
+                                                  y, yt, ldy, None)
+        return lib.sq_linear_forward_combined(c, ldc, M, K, ctypes.byref(qw), FAKE, FAKE, None, y,
+                                              yt, ldy, None)
+    assert fwd(c=None) == L.SQ_ERR_INVALID_ARG
+    assert fwd(c=FAKE + 8) == L.SQ_ERR_ALIGNMENT
+    assert fwd(ldc=520) == L.SQ_ERR_ALIGNMENT
+    assert fwd(ldc=256) == L.SQ_ERR_INVALID_ARG
+    qw4, k4 = _qw(bits=4, K=512)
+    assert fwd(qw=qw4) == L.SQ_ERR_UNSUPPORTED        # int8 weights only
+    assert fwd(M=0) == L.SQ_OK
+
+
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -257,6 +257,9 @@ def test_hand_worked_example():
     expect = np.array([[14097 / 2048 + 0.25, 238 / 256 - 0.5],
                        [-7.96875 / 128 + 0.25, 14.875 / 256 - 0.5]], dtype=np.float64)
     np.testing.assert_array_equal(o["y"].astype(np.float64), expect)
+    # combined code c = q+ + q- of the same example, from the hand-derived codes
+    c = O.quantize_activations_combined(x, [0, 4], o["sp"], o["sn"])
+    np.testing.assert_array_equal(c, [[127, 16, -127, -32], [0, 2, 0, -2]])
 
 
 # ------------------------------------------------------------------ invariants
@@ -275,6 +278,9 @@ def test_I1_equal_scales_is_single_scale():
     r = np.float32(1) / s
     single = np.clip(np.rint(x.astype(np.float64) * np.float64(r)), -127, 127).astype(np.int64)
     np.testing.assert_array_equal(qp.astype(np.int64) + qn, single)
+    # with one scale the combined code is the textbook symmetric code
+    c = O.quantize_activations_combined(x, kb, [s], [s])
+    np.testing.assert_array_equal(c.astype(np.int64), single)
     w = _rand_f32(rng, (24, 384), 0.02)
     wc, ws = O.quantize_weights_w8(w, kb)
     acc = O.accumulate(qp, qn, wc, [0, 384])
@@ -392,6 +398,11 @@ def test_I8_code_ranges_and_disjoint_support():
     assert qp.min() >= 0 and qp.max() <= 127 and qn.min() >= -127 and qn.max() <= 0
     assert not (qp.astype(np.int32) * qn).any()
     assert list(qp[0, :4]) == [127, 0, 127, 0] and list(qn[0, :4]) == [0, -127, 0, -127]
+    # disjoint support: the combined code splits back losslessly
+    c = O.quantize_activations_combined(x, kb, sp, sn)
+    assert c.min() >= -127 and c.max() <= 127
+    np.testing.assert_array_equal(np.maximum(c, 0), qp)
+    np.testing.assert_array_equal(np.minimum(c, 0), qn)
 
 
 def test_I9_power_of_two_rescaling():
