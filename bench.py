@@ -338,6 +338,17 @@ def run_ours(args):
     fwd_graph = capture(lambda: forward(xd, y))
     gemm_graph = capture(gemm_only)
     fused_graph = capture(lambda: pq.linear(xd, qw, sp, sn, bd, out=y)) if use_codes else None
+    # The single-scale baseline (one symmetric scale per K segment) of the same
+    # forward: its codes, then one int8 product per unit.
+    single_graph = None
+    if wl.bits == 8:
+        ldc = (wl.K + 15) // 16 * 16
+        c1_buf = torch.empty((wl.M, ldc), dtype=torch.int8, device=dev)[:, : wl.K]
+
+        def single_forward():
+            pq.quantize_activations_single(xd, wl.kseg, sp, sn, out=c1_buf)
+            pq.linear_from_single(c1_buf, qw, sp, sn, bd, out=y)
+        single_graph = capture(single_forward)
 
     def timed(graph, n, salt):
         evs = events(n)
@@ -366,9 +377,10 @@ def run_ours(args):
     gemm_ms = timed(gemm_graph, args.steps, 3)
     fwd_ms = timed(fwd_graph, args.steps, 5)
     fused_ms = timed(fused_graph, args.steps, 7) if fused_graph is not None else None
+    single_ms = timed(single_graph, args.steps, 9) if single_graph is not None else None
     if pq.stream_status() != 0:
         raise RuntimeError("device status word set during the timed region")
-    del step_graph, fwd_graph, gemm_graph, fused_graph
+    del step_graph, fwd_graph, gemm_graph, fused_graph, single_graph
 
     # end to end through the API: host inputs in, host result out, every step
     e2e = None
@@ -403,12 +415,13 @@ def run_ours(args):
 
     # max over ranks
     vals = [total_ms, statistics.mean(gemm_ms), statistics.mean(fwd_ms),
-            e2e["ms"] if e2e else 0.0, statistics.mean(fused_ms) if fused_ms else 0.0]
+            e2e["ms"] if e2e else 0.0, statistics.mean(fused_ms) if fused_ms else 0.0,
+            statistics.mean(single_ms) if single_ms else 0.0]
     if world > 1:
         t = torch.tensor(vals, dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         vals = t.tolist()
-    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms, fused_avg_ms = vals
+    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms, fused_avg_ms, single_avg_ms = vals
 
     if rank == 0:
         int8_peak_tops, hbm_peak, peak_kind = peaks()
@@ -441,6 +454,14 @@ def run_ours(args):
             "timing": "each step one CUDA-graph replay, CUDA events on the launching stream",
             "clocks": clocks,
         }
+        if single_ms:
+            line["single_scale_forward"] = {
+                "us": single_avg_ms * 1e3,
+                "exec_tops": ops / 2 / (single_avg_ms * 1e-3) / 1e12,
+                "dualscale_over_single": fwd_avg_ms / single_avg_ms,
+                "note": "naive baseline: one symmetric scale per K segment, its codes, then one "
+                        "int8 product (half the MMA work of DualScale)",
+            }
         if fused_ms:
             line["fused_forward"] = {
                 "us": fused_avg_ms * 1e3, "exec_tops": ops / (fused_avg_ms * 1e-3) / 1e12,

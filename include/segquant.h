@@ -194,6 +194,31 @@ sq_status sq_linear_forward_combined(const int8_t* c, int64_t ldc, int64_t M, in
                                      const float* bias, void* y, sq_dtype yt, int64_t ldy,
                                      sq_stream_t stream);
 
+/* Single-scale ("naive") baseline of the same layer, for the latency
+ * comparison the SegQuant summaries make against naive quantization (Spanish
+ * technical summary section 4, "Eficiencia y Despliegue"; the standard
+ * single-scale quantization DualScale replaces, section 2.B).  Reading: one
+ * symmetric scale per K segment, s_j = max|x| / 127 over the calibration rows,
+ * which equals max(s_pos[j], s_neg[j]) from sq_calibrate (fp32 division by 127
+ * is monotone); codes c = clamp(round_half_even(x * fl(1/s_j)), -127, 127),
+ * NaN -> 0.  c: device int8 [M, K], row stride ldc (a multiple of 16),
+ * 16-byte aligned.  Requirements and errors as for sq_quantize_activations. */
+sq_status sq_quantize_activations_single(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                         int64_t ldx, const sq_segments* kseg, const float* s_pos,
+                                         const float* s_neg, int8_t* c, int64_t ldc,
+                                         sq_stream_t stream);
+
+/* The single-scale forward from codes written by sq_quantize_activations_single
+ * with the same scales: one int8 tensor-core product per unit, epilogue (fixed
+ * fp32 order) t = s_j * F(acc), y = fma(s_w[j][n], t, y) over the units from
+ * y = 0, then + bias, then the output rounding.  int8 weights only (bits = 4
+ * returns SQ_ERR_UNSUPPORTED).  Other arguments and requirements as for
+ * sq_linear_forward_combined. */
+sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int64_t K,
+                                   const sq_qweight* w, const float* s_pos, const float* s_neg,
+                                   const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                                   sq_stream_t stream);
+
 /* Test surface: the same kernel as sq_linear_forward, but the epilogue writes
  * the raw int32 accumulators of every unit instead of Y:
  * acc[u][p][m][n], p = 0 for the (+) product, 1 for the (-) product; U units

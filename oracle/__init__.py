@@ -63,6 +63,8 @@ def _load():
         lib.sqo_unpack_w4.restype = None
         lib.sqo_accumulate.argtypes = [P, P, I64, I64, P, I64, I32, P, P]
         lib.sqo_epilogue.argtypes = [P, I64, I64, I32, P, P, P, P, P, P, INT, I64]
+        lib.sqo_quantize_activations_single.argtypes = [P, INT, I64, I64, I64, I32, P, P, P, P]
+        lib.sqo_epilogue_single.argtypes = [P, I64, I64, I32, P, P, P, P, P, P, INT, I64]
         lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.sqo_f32_to_bf16.restype = ctypes.c_uint16
         lib.sqo_f32_to_f16.argtypes = [ctypes.c_float]
@@ -70,7 +72,8 @@ def _load():
         lib.sqo_f16_to_f32.argtypes = [ctypes.c_uint16]
         lib.sqo_f16_to_f32.restype = ctypes.c_float
         for f in ("sqo_calibrate", "sqo_quantize_activations", "sqo_quantize_weights_w8",
-                  "sqo_quantize_weights_w4", "sqo_accumulate", "sqo_epilogue"):
+                  "sqo_quantize_weights_w4", "sqo_accumulate", "sqo_epilogue",
+                  "sqo_quantize_activations_single", "sqo_epilogue_single"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -250,6 +253,56 @@ def linear_forward(x, kbounds, s_pos, s_neg, bits, wcodes, wscales, bias=None, o
     y = epilogue(acc, useg, s_pos, s_neg, unit_weight_scales(bits, wscales), bias, out)
     if return_acc:
         return y, acc, (qp, qn)
+    return y
+
+
+def quantize_activations_single(x: np.ndarray, kbounds, s_pos, s_neg):
+    """Single-scale baseline codes, int8 [M, K]: s_j = max(s+_j, s-_j)."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    kb = _bounds(kbounds)
+    J = len(kb) - 1
+    sp = np.ascontiguousarray(np.asarray(s_pos, np.float32))
+    sn = np.ascontiguousarray(np.asarray(s_neg, np.float32))
+    c = np.zeros((M, K), np.int8)
+    _check("sqo_quantize_activations_single",
+           _load().sqo_quantize_activations_single(_ptr(x), _x_dtype(x), M, K, K, J, _ptr(kb),
+                                                   _ptr(sp), _ptr(sn), _ptr(c)))
+    return c
+
+
+def accumulate_single(c, wcodes, ubounds) -> np.ndarray:
+    """Per-unit int32 accumulators acc[u, m, n] of single-scale codes."""
+    c = np.ascontiguousarray(c, np.int8)
+    return accumulate(c, np.zeros_like(c), wcodes, ubounds)[:, 0].copy()
+
+
+def epilogue_single(acc, unit_seg, s_pos, s_neg, unit_scales, bias=None, out: str = "f32"):
+    """Single-scale epilogue; acc int32 [U, M, N]; out 'f32' or 'bf16' (uint16 bits)."""
+    acc = np.ascontiguousarray(acc, np.int32)
+    U, M, N = acc.shape
+    us = np.ascontiguousarray(np.asarray(unit_seg, np.int32))
+    sp = np.ascontiguousarray(np.asarray(s_pos, np.float32))
+    sn = np.ascontiguousarray(np.asarray(s_neg, np.float32))
+    sw = np.ascontiguousarray(np.asarray(unit_scales, np.float32))
+    b = None if bias is None else np.ascontiguousarray(np.asarray(bias, np.float32))
+    y = np.zeros((M, N), np.float32 if out == "f32" else np.uint16)
+    _check("sqo_epilogue_single",
+           _load().sqo_epilogue_single(_ptr(acc), M, N, U, _ptr(us), _ptr(sp), _ptr(sn), _ptr(sw),
+                                       _ptr(b), _ptr(y), 0 if out == "f32" else 1, N))
+    return y
+
+
+def linear_forward_single(x, kbounds, s_pos, s_neg, wcodes, wscales, bias=None, out="f32",
+                          return_acc: bool = False):
+    """The single-scale baseline forward (int8 weights): codes, accumulators, epilogue."""
+    M, K = x.shape
+    c = quantize_activations_single(x, kbounds, s_pos, s_neg)
+    ub, useg = units_of(8, K, kbounds)
+    acc = accumulate_single(c, wcodes, ub)
+    y = epilogue_single(acc, useg, s_pos, s_neg, unit_weight_scales(8, wscales), bias, out)
+    if return_acc:
+        return y, acc, c
     return y
 
 

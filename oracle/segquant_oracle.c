@@ -308,6 +308,59 @@ int sqo_epilogue(const int32_t* acc, int64_t M, int64_t N, int32_t U, const int3
   return SQO_OK;
 }
 
+/* ---- Single-scale baseline --------------------------------------------------
+ * The summaries compare DualScale's latency with naive quantization [ES 4,
+ * "Eficiencia y Despliegue"]; the naive scheme is the standard single-scale
+ * quantization DualScale replaces [ES 2.B].  Reading: one symmetric scale per K
+ * segment, s_j = max|x| / 127 over the calibration rows, which is
+ * max(s+_j, s-_j) (fp32 division by 127 is monotone);
+ * c = clamp(RNE(x * fl(1/s_j)), -127, 127); NaN -> 0 (as in the DualScale
+ * codes, where NaN falls in neither branch). */
+int sqo_quantize_activations_single(const void* x, int dtype, int64_t M, int64_t K, int64_t ldx,
+                                    int32_t J, const int32_t* kb, const float* s_pos,
+                                    const float* s_neg, int8_t* c) {
+  if (J < 1 || kb[0] != 0 || kb[J] != K) return SQO_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int32_t j = 0; j < J; ++j) {
+      float s = s_pos[j] > s_neg[j] ? s_pos[j] : s_neg[j];
+      float r = recip(s);
+      for (int64_t k = kb[j]; k < kb[j + 1]; ++k) {
+        float v = load_elem(x, dtype, m * ldx + k);
+        int32_t q = 0;
+        if (v == v) q = round_clamp(v, r, -127, 127);
+        c[m * K + k] = (int8_t)q;
+      }
+    }
+  }
+  return SQO_OK;
+}
+
+/* Single-scale epilogue (fixed fp32 order, the same shape as R9):
+ *   t_u = s_j * F(acc_u); y = 0; for u ascending: y = fmaf(sw_u[n], t_u, y);
+ *   if bias: y = y + b[n].
+ * acc: int32 [U][M][N]. */
+int sqo_epilogue_single(const int32_t* acc, int64_t M, int64_t N, int32_t U,
+                        const int32_t* unit_seg, const float* s_pos, const float* s_neg,
+                        const float* sw, const float* bias, void* y, int out_dtype, int64_t ldy) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t n = 0; n < N; ++n) {
+      float acc_y = 0.0f;
+      for (int32_t u = 0; u < U; ++u) {
+        int32_t j = unit_seg[u];
+        float s = s_pos[j] > s_neg[j] ? s_pos[j] : s_neg[j];
+        float t = s * (float)acc[((int64_t)u * M + m) * N + n];
+        acc_y = fmaf(sw[(int64_t)u * N + n], t, acc_y);
+      }
+      if (bias) acc_y = acc_y + bias[n];
+      if (out_dtype == 0) ((float*)y)[m * ldy + n] = acc_y;
+      else ((uint16_t*)y)[m * ldy + n] = sqo_f32_to_bf16(acc_y);
+    }
+  }
+  return SQO_OK;
+}
+
 /* Keeps the fp32 value of the epilogue before any output rounding, for tests
  * that need the unrounded fp32 result (same order as sqo_epilogue). */
 int sqo_epilogue_f32(const int32_t* acc, int64_t M, int64_t N, int32_t U,

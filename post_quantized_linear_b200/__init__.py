@@ -24,7 +24,8 @@ from ._lib import SegQuantError
 
 __all__ = ["QuantizedWeight", "SegQuantError", "calibrate", "quantize_weights", "linear",
            "quantize_activations", "linear_from_codes", "quantize_activations_combined",
-           "linear_from_combined", "linear_accumulators", "stream_status", "qweight_sizes"]
+           "linear_from_combined", "quantize_activations_single", "linear_from_single",
+           "linear_accumulators", "stream_status", "qweight_sizes"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -208,6 +209,40 @@ def linear_from_combined(c: torch.Tensor, qw: QuantizedWeight, s_pos: torch.Tens
     _check_2d(out, "out")
     cw, keep = qw.c_struct()
     _lib.check("sq_linear_forward_combined", _lib.load().sq_linear_forward_combined(
+        _ptr(c), c.stride(0), M, K, ctypes.byref(cw), _ptr(s_pos), _ptr(s_neg), _ptr(bias),
+        _ptr(out), _dtype_code(out.dtype), out.stride(0), _stream(stream)))
+    return out
+
+
+def quantize_activations_single(x: torch.Tensor, kseg: Sequence[int], s_pos: torch.Tensor,
+                                s_neg: torch.Tensor, out: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """Single-scale baseline codes, int8 [M, K]: one symmetric scale per K
+    segment, s = max(s_pos, s_neg) (= max|x| / 127 of the calibration rows)."""
+    _check_2d(x, "x")
+    M, K = x.shape
+    if out is None:
+        ldc = (K + 15) // 16 * 16
+        out = torch.empty((M, ldc), dtype=torch.int8, device=x.device)[:, :K]
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_quantize_activations_single", _lib.load().sq_quantize_activations_single(
+        _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(seg), _ptr(s_pos),
+        _ptr(s_neg), _ptr(out), out.stride(0), _stream(stream)))
+    return out
+
+
+def linear_from_single(c: torch.Tensor, qw: QuantizedWeight, s_pos: torch.Tensor,
+                       s_neg: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                       out_dtype: torch.dtype = torch.bfloat16,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Single-scale baseline forward from ``quantize_activations_single`` codes (int8 weights)."""
+    _check_2d(c, "c")
+    M, K = c.shape
+    if out is None:
+        out = torch.empty((M, qw.N), dtype=out_dtype, device=c.device)
+    _check_2d(out, "out")
+    cw, keep = qw.c_struct()
+    _lib.check("sq_linear_forward_single", _lib.load().sq_linear_forward_single(
         _ptr(c), c.stride(0), M, K, ctypes.byref(cw), _ptr(s_pos), _ptr(s_neg), _ptr(bias),
         _ptr(out), _dtype_code(out.dtype), out.stride(0), _stream(stream)))
     return out

@@ -49,6 +49,10 @@ SIGNATURES = {
                                                  c_vp, c_vp, c_i64, c_vp]),
     "sq_linear_forward_combined": (c_i32, [c_vp, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp, c_vp,
                                            c_i32, c_i64, c_vp]),
+    "sq_quantize_activations_single": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp,
+                                               c_vp, c_vp, c_i64, c_vp]),
+    "sq_linear_forward_single": (c_i32, [c_vp, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp, c_vp,
+                                         c_i32, c_i64, c_vp]),
     "sq_linear_accumulators": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp,
                                        c_vp]),
     "sq_stream_status": (c_i32, [c_vp]),

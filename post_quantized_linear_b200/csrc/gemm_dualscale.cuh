@@ -771,18 +771,17 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, int quad, in
 }
 
 // ------------------------------------------------- epilogue through TMA stores
-// One unit per tile, output written by TMA tensor stores from a per-warp
-// staging tile of 32 rows x 32 columns in shared memory.  Storing through TMA
-// writes whole 128-byte lines instead of one 16-byte piece per row per lane,
-// and the warp does not wait for the writes; the accumulators are released as
-// soon as the warp's last TMEM columns are in registers.
+// Output written by TMA tensor stores from a per-warp staging tile of 32 rows x
+// 32 columns in shared memory.  Storing through TMA writes whole 128-byte lines
+// instead of one 16-byte piece per row per lane, and the warp does not wait
+// for the writes.
 //
 // Staging layout: row r (the warp's TMEM lane r) of the 32-column tile at
 // r * ROWB, 16-byte chunk j of the row at position j ^ f(r) -- the TMA
 // 64-byte swizzle for bf16 rows of 64 bytes (f(r) = (r >> 1) & 3) and the
 // 128-byte swizzle for fp32 rows of 128 bytes (f(r) = r & 7) -- so a warp's
 // 16-byte stores touch every bank evenly.  The buffer is 1024-byte aligned.
-constexpr int kStageYBytes = 32 * 128;   // per epilogue warp (fp32 worst case)
+__host__ __device__ constexpr int stage_y_bytes(bool y_bf16) { return 32 * (y_bf16 ? 64 : 128); }
 
 template <bool Y_BF16>
 __device__ __forceinline__ void stage16(const GemmArgs& a, int n, float (&o)[16], uint8_t* srow,
@@ -817,9 +816,30 @@ __device__ __forceinline__ void stage16(const GemmArgs& a, int n, float (&o)[16]
   }
 }
 
-// Epilogue warps: EPW of them, warp (quad, part) owns TMEM lanes quad*32..+31
-// (tile rows) and columns [part*HALF, (part+1)*HALF).
-template <int BN, int NBUF, int EPW, bool Y_BF16, class TileFn>
+// Single-scale fold of 16 columns: t = s * F(acc); y = fma(sw, t, y).
+__device__ __forceinline__ void fold16_single(const uint32_t (&a)[16], const float (&sw)[16],
+                                              float s, float* y) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float t = __fmul_rn(s, acc_to_f32<false>(a[i]));
+    y[i] = __fmaf_rn(sw[i], t, y[i]);
+  }
+}
+
+// Scale of unit u: the DualScale pair (s+, s-), or the single-scale s = max(s+, s-).
+__device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float& sp, float& sn) {
+  sp = __ldg(a.s_pos + j);
+  sn = __ldg(a.s_neg + j);
+}
+
+// Epilogue warps: EPW of them; warp (quad, part) owns TMEM lanes quad*32..+31
+// (tile rows) and columns [part*HALF, (part+1)*HALF).  NACC accumulators per
+// unit (2: DualScale (+)/(-) products at columns c and c + BN of the buffer;
+// 1: single scale).  MULTI: several units (K segments) per tile, folded into
+// registers (HALF == 32), stored once per tile; otherwise one unit per tile,
+// streamed out in 32-column passes with the accumulators released after the
+// warp's last TMEM load.
+template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
@@ -827,13 +847,37 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
                                                    volatile int* abort_flag, long long budget) {
   constexpr int HALF = BN / (EPW / 4);
   constexpr int ROWB = Y_BF16 ? 64 : 128;
+  constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
   static_assert(HALF % 32 == 0, "32-column store passes");
+  static_assert(!MULTI || HALF == 32, "several units: one 32-column pass per warp");
   uint8_t* srow = stage_y + lane * ROWB;
   const uint32_t sbase = smem_u32(stage_y);
+  const int units = args.kseg.count;
   auto release = [&](int b) {
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
+  };
+  // fold of 16 columns at tile column cc of buffer b, unit / segment j, into o
+  auto fold = [&](int b, int cc, int j, const Tile& t, float* o) {
+    const uint32_t tcol = (uint32_t)b * BUF_COLS + (uint32_t)cc;
+    float sw[16];
+    float sp, sn;
+    unit_act_scales(args, j, sp, sn);
+    if constexpr (NACC == 2) {
+      uint32_t ap[16], an[16];
+      tmem_ld16(t_lane + tcol, ap);
+      tmem_ld16(t_lane + tcol + BN, an);
+      tmem_wait_ld();
+      load_wscales16(args, j, j, t.n0 + cc, sw);
+      fold16<false>(ap, an, sw, sp, sn, o);
+    } else {
+      uint32_t ac[16];
+      tmem_ld16(t_lane + tcol, ac);
+      tmem_wait_ld();
+      load_wscales16(args, j, j, t.n0 + cc, sw);
+      fold16_single(ac, sw, fmaxf(sp, sn), o);
+    }
   };
   int ug = 0;
   bool ok = true, pending = false;
@@ -843,50 +887,79 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
     const int c_lo = part * HALF;
     const int cols = min(HALF, t.width - c_lo);   // may be <= 0 on a narrow tail tile
     if (cols > 0) {
-      const float* sw_row = static_cast<const float*>(args.wscales) + t.n0 + c_lo;
-      for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
+      for (int u = 0; u < units; ++u) {
+        const float* sw_row = static_cast<const float*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo;
+        for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
+      }
       if (args.bias != nullptr)
         for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(args.bias + t.n0 + c_lo + c);
     }
-    const int b = ug % NBUF;
-    if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
-    tc_fence_after();
-    const float sp = __ldg(args.s_pos), sn = __ldg(args.s_neg);
     const int npass = cols > 0 ? (cols + 31) / 32 : 0;
-    for (int p = 0; p < npass; ++p) {
-      const int col = c_lo + p * 32;
-      if (pending) {   // the previous store has read the staging tile
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
-      }
+    if constexpr (MULTI) {
+      float y[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int cc = col + 16 * h;
-        if (cc < t.width) {
-          uint32_t ap[16], an[16];
-          const uint32_t tcol = (uint32_t)(b * 2 * BN + cc);
-          tmem_ld16(t_lane + tcol, ap);
-          tmem_ld16(t_lane + tcol + BN, an);
-          tmem_wait_ld();
-          float sw[16], o[16];
-          load_wscales16(args, 0, 0, t.n0 + cc, sw);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = 0.0f;
-          fold16<false>(ap, an, sw, sp, sn, o);
-          stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+      for (int i = 0; i < 32; ++i) y[i] = 0.0f;
+      for (int u = 0; u < units; ++u) {
+        const int b = ug % NBUF;
+        if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+        tc_fence_after();
+        if (npass > 0) {
+          fold(b, c_lo, u, t, y);
+          if (c_lo + 16 < t.width) fold(b, c_lo + 16, u, t, y + 16);
         }
+        release(b);
+        ++ug;
       }
-      if (p == npass - 1) release(b);   // this warp's accumulator columns are all read
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
-        bulk_commit_group();
+      if (!ok) break;
+      if (npass > 0) {
+        if (pending) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+        }
+        stage16<Y_BF16>(args, t.n0 + c_lo, *reinterpret_cast<float(*)[16]>(y), srow, lane, 0);
+        if (c_lo + 16 < t.width)
+          stage16<Y_BF16>(args, t.n0 + c_lo + 16, *reinterpret_cast<float(*)[16]>(y + 16), srow, lane, 1);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tmap_y, sbase, t.n0 + c_lo, t.m0 + quad * 32);
+          bulk_commit_group();
+        }
+        pending = true;
       }
-      pending = true;
+    } else {
+      const int b = ug % NBUF;
+      if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+      tc_fence_after();
+      for (int p = 0; p < npass; ++p) {
+        const int col = c_lo + p * 32;
+        if (pending) {   // the previous store has read the staging tile
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int cc = col + 16 * h;
+          if (cc < t.width) {
+            float o[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+            fold(b, cc, 0, t, o);
+            stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+          }
+        }
+        if (p == npass - 1) release(b);   // this warp's accumulator columns are all read
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+          bulk_commit_group();
+        }
+        pending = true;
+      }
+      if (npass == 0) release(b);
+      ++ug;
     }
-    if (npass == 0) release(b);
-    ++ug;
   }
   // Every store has completed before the CTA (and its shared memory) exits.
   if (lane == 0) bulk_wait_all();

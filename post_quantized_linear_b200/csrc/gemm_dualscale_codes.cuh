@@ -11,11 +11,15 @@
 //     instead of one per operand ring;
 //   * no operand-producer warps: warp 0 issues TMA, warp 1 owns TMEM and
 //     issues the MMAs, warps 2.. run the epilogue (8 warps, or 16 when a tile
-//     folds several units).
-// Stage sizes: 32 KiB of codes + BN x 128 bytes of weights.  With one unit per
-// tile the output leaves through TMA stores from 32 KiB of staging tiles
-// (epilogue_tma_store), leaving room for four stages at BN = 128 and three at
-// BN = 192 and 256.
+//     folds several units), which leaves through TMA stores
+//     (epilogue_tma_store).
+// SINGLE: the single-scale baseline of the same layer (one symmetric scale
+// per K segment, s = max|x| / 127 = max(s+, s-)): one code tile per stage,
+// one product per k step, one accumulator -- which leaves room for two TMEM
+// buffers at every tile width.
+// Stage sizes: (2 or 1) x 16 KiB of codes + BN x 128 bytes of weights, as many
+// as fit in 224 KiB next to the epilogue's staging tiles (2 or 4 KiB per
+// epilogue warp for bf16 or fp32 Y).
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -28,36 +32,38 @@ __host__ __device__ constexpr int codes_kernel_threads(bool multi) {
   return (kCodesEpiWarp0 + epi_warps(multi)) * 32;
 }
 
-template <int BN_, bool MULTI>
+template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE>
 struct CodesCfg {
   static constexpr int BN = BN_;
-  static constexpr int A_BYTES = 2 * BM * BK;   // q+ tile, q- tile
+  static constexpr int NACC = SINGLE ? 1 : 2;          // accumulators (code tiles) per unit
+  static constexpr int A_BYTES = NACC * BM * BK;      // q+ and q- tiles, or the single code tile
   static constexpr int W_BYTES = BN * BK;
   static constexpr int STAGE = A_BYTES + W_BYTES;
-  // One unit per tile: Y leaves through per-warp staging tiles and TMA stores.
-  static constexpr int Y_BYTES = MULTI ? 0 : epi_warps(false) * kStageYBytes;
+  static constexpr int EPW = epi_warps(MULTI);
+  static constexpr int Y_BYTES = EPW * stage_y_bytes(Y_BF16);
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
-  static constexpr int NBUF = (BN <= 128) ? 2 : 1;
+  static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
   static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1;  // full, empty; tmem full/empty; drain
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int TMEM_COLS = 2 * BN * NBUF;
+  static constexpr int TMEM_COLS = NACC * BN * NBUF;
   static constexpr int TMEM_ALLOC = TMEM_COLS <= 256 ? 256 : 512;
   static_assert(S >= 2 && TMEM_COLS <= 512 && SMEM_BYTES <= 232448, "budgets");
   static_assert(BN % 16 == 0 && BN <= 256, "UMMA N for M = 128");
+  static_assert(OFF_Y % 1024 == 0 && stage_y_bytes(Y_BF16) % 1024 == 0, "staging alignment");
 };
 
-template <int BN, bool Y_BF16, bool MULTI>
+template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false>
 __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI>;
-  static_assert(!MULTI || BN == 128, "several units per tile need double-buffered TMEM");
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE>;
+  static_assert(!MULTI || (BN == 128 && C::NBUF == 2), "several units per tile: BN = 128, two buffers");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -103,9 +109,9 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_qp);
-      tma_prefetch_desc(&tmap_qn);
+      if constexpr (!SINGLE) tma_prefetch_desc(&tmap_qn);
       tma_prefetch_desc(&tmap_w);
-      if constexpr (!MULTI) tma_prefetch_desc(&tmap_y);
+      tma_prefetch_desc(&tmap_y);
       int c = 0;
       bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
@@ -117,7 +123,8 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
           uint8_t* st = smem + s * C::STAGE;
           mbar_arrive_expect_tx(smem_u32(full + s), C::STAGE);
           tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
-          tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
+          if constexpr (!SINGLE)
+            tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
           tma_load_2d(smem_u32(st + C::A_BYTES), &tmap_w, smem_u32(full + s), kb * BK, t.n0);
           ++c;
         }
@@ -141,7 +148,7 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
             const int b = ug % C::NBUF;
             if (!(ok = wait1(smem_u32(tmem_empty + b), ((ug / C::NBUF) & 1) ^ 1, abort_flag, budget))) break;
             tc_fence_after();
-            d_pos = tmem_base + (uint32_t)(b * 2 * BN);
+            d_pos = tmem_base + (uint32_t)(b * C::NACC * BN);
           }
           const int s = c % C::S;
           if (!(ok = wait1(smem_u32(full + s), (c / C::S) & 1, abort_flag, budget))) break;
@@ -153,7 +160,8 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
             const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
             const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
             umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
-            umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
+            if constexpr (!SINGLE)
+              umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
           }
           unit_open = true;
           umma_commit(smem_u32(empty + s));
@@ -176,16 +184,10 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
     const int quad = warp & 3;
     const int part = (warp - kCodesEpiWarp0) >> 2;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    if constexpr (MULTI) {
-      epilogue_role<BN, C::NBUF, MULTI, false, Y_BF16, false>(
-          args, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), /*empty_remote=*/false,
-          /*row_shift=*/0, rounds, tiles, abort_flag, budget);
-    } else {
-      uint8_t* stage_y = smem + C::OFF_Y + (warp - kCodesEpiWarp0) * kStageYBytes;
-      epilogue_tma_store<BN, C::NBUF, epi_warps(false), Y_BF16>(
-          args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty),
-          rounds, tiles, abort_flag, budget);
-    }
+    uint8_t* stage_y = smem + C::OFF_Y + (warp - kCodesEpiWarp0) * stage_y_bytes(Y_BF16);
+    epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
+        args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
+        tiles, abort_flag, budget);
   }
 
   // ---------------------------------------------------------------- teardown

@@ -169,7 +169,11 @@ __device__ __forceinline__ void load16(const XT* p, float (&v)[16]) {
 // every row it visits (rows blockIdx.y*8 + y, stepping by gridDim.y*8), so its
 // segment and reciprocal scales are fixed; a warp reads 1 KiB (bf16) and
 // writes 512 bytes of each code tensor per row.
-template <typename XT, bool COMBINED>
+// MODE: CODES_DUAL (q+ and q-), CODES_COMBINED (c = q+ + q-), CODES_SINGLE
+// (the single-scale code: both branches with s = max(s+, s-)).
+constexpr int CODES_DUAL = 0, CODES_COMBINED = 1, CODES_SINGLE = 2;
+
+template <typename XT, int MODE>
 __device__ __forceinline__ void quantize_activations_body(
     const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
@@ -177,8 +181,11 @@ __device__ __forceinline__ void quantize_activations_body(
   const int32_t k = (blockIdx.x * 32 + threadIdx.x) * 16;
   if (k >= K) return;
   const int j = kseg.segment_of(k);
-  const float rp = s_pos[j] > 0.0f ? __frcp_rn(s_pos[j]) : 0.0f;
-  const float rn = s_neg[j] > 0.0f ? __frcp_rn(s_neg[j]) : 0.0f;
+  constexpr bool COMBINED = (MODE != CODES_DUAL);
+  const float sj_p = (MODE == CODES_SINGLE) ? fmaxf(s_pos[j], s_neg[j]) : s_pos[j];
+  const float sj_n = (MODE == CODES_SINGLE) ? sj_p : s_neg[j];
+  const float rp = sj_p > 0.0f ? __frcp_rn(sj_p) : 0.0f;
+  const float rn = sj_n > 0.0f ? __frcp_rn(sj_n) : 0.0f;
   const int32_t step = gridDim.y * 8;
   for (int32_t m = blockIdx.y * 8 + threadIdx.y; m < M; m += step) {
     float v[16];
@@ -208,19 +215,20 @@ __global__ void __launch_bounds__(256) quantize_activations_kernel(
     const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
     int8_t* __restrict__ q_neg, int64_t ldq) {
-  quantize_activations_body<XT, false>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
+  quantize_activations_body<XT, CODES_DUAL>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
 }
 
 // Combined codes c = q+ + q- (one signed byte per activation): an element
 // falls in exactly one branch, so the two magic-rounded words carry its code
 // in their low bytes and the other branch's low byte is 0; their sum's low
-// byte is c.
-template <typename XT>
+// byte is c.  With MODE == CODES_SINGLE both branches use s = max(s+, s-), and
+// c is the single-scale symmetric code.
+template <typename XT, int MODE>
 __global__ void __launch_bounds__(256) quantize_activations_combined_kernel(
     const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ c,
     int64_t ldc) {
-  quantize_activations_body<XT, true>(x, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc);
+  quantize_activations_body<XT, MODE>(x, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc);
 }
 
 // ------------------------------------------------------ weight quantization

@@ -218,11 +218,11 @@ sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const
                 : launch_inplace<BN, false, false, MULTI>(tx, tw, a, stream);
 }
 
-template <int BN, bool YB, bool MULTI>
+template <int BN, bool YB, bool MULTI, bool SINGLE>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  using C = sq::CodesCfg<BN, MULTI>;
-  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI>;
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE>;
+  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
@@ -236,12 +236,12 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   return cuda_status(cudaGetLastError());
 }
 
-template <int BN, bool MULTI>
+template <int BN, bool MULTI, bool SINGLE = false>
 sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                            const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                            cudaStream_t stream) {
-  return y_bf16 ? launch_codes<BN, true, MULTI>(tqp, tqn, tw, ty, a, stream)
-                : launch_codes<BN, false, MULTI>(tqp, tqn, tw, ty, a, stream);
+  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE>(tqp, tqn, tw, ty, a, stream)
+                : launch_codes<BN, false, MULTI, SINGLE>(tqp, tqn, tw, ty, a, stream);
 }
 
 // Tensor map of Y for the TMA-store epilogue: boxes of 32 rows x 32 columns,
@@ -335,12 +335,13 @@ int choose_bn(int64_t M, int64_t N, bool multi, bool f32x) {
   return c192 <= c128 ? 192 : 128;
 }
 
-// DualScale codes of X: q+ and q-, or (combined) the code c = q+ + q-
+// Codes of X: q+ and q- (CODES_DUAL), the combined code c = q+ + q-
+// (CODES_COMBINED) or the single-scale code (CODES_SINGLE), the last two
 // written to q_pos.
 sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
                          const sq_segments* kseg, const float* s_pos, const float* s_neg,
-                         int8_t* q_pos, int8_t* q_neg, int64_t ldq, bool combined,
-                         cudaStream_t s) {
+                         int8_t* q_pos, int8_t* q_neg, int64_t ldq, int mode, cudaStream_t s) {
+  const bool combined = (mode != sq::CODES_DUAL);
   if (!dtype_ok(xt) || M < 0 || K <= 0 || ldx < K || ldq < K) return SQ_ERR_INVALID_ARG;
   if (K > SQ_MAX_K) return SQ_ERR_RANGE;
   SegBounds sb;
@@ -365,12 +366,19 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
   if (gy < 1) gy = 1;
   dim3 grid(gx, (unsigned)gy), block(32, 8);
   using bf = __nv_bfloat16;
-  if (combined) {
+  if (mode == sq::CODES_COMBINED) {
     if (xt == SQ_BF16)
-      sq::quantize_activations_combined_kernel<bf><<<grid, block, 0, s>>>(
+      sq::quantize_activations_combined_kernel<bf, sq::CODES_COMBINED><<<grid, block, 0, s>>>(
           static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
     else
-      sq::quantize_activations_combined_kernel<float><<<grid, block, 0, s>>>(
+      sq::quantize_activations_combined_kernel<float, sq::CODES_COMBINED><<<grid, block, 0, s>>>(
+          static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+  } else if (mode == sq::CODES_SINGLE) {
+    if (xt == SQ_BF16)
+      sq::quantize_activations_combined_kernel<bf, sq::CODES_SINGLE><<<grid, block, 0, s>>>(
+          static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+    else
+      sq::quantize_activations_combined_kernel<float, sq::CODES_SINGLE><<<grid, block, 0, s>>>(
           static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
   } else {
     if (xt == SQ_BF16)
@@ -385,7 +393,7 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
   return cuda_status(cudaGetLastError());
 }
 
-enum class ASource { X, Codes, Combined };
+enum class ASource { X, Codes, Combined, Single };
 
 sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_pos,
                       const int8_t* q_neg, int64_t ldq, int64_t M, int64_t K, int64_t ldx,
@@ -401,19 +409,20 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const int64_t N = w->N;
   if (src == ASource::X && ldx < K) return SQ_ERR_INVALID_ARG;
   if (src != ASource::X && ldq < K) return SQ_ERR_INVALID_ARG;
-  if (src == ASource::Combined && w->bits != 8) return SQ_ERR_UNSUPPORTED;
+  if ((src == ASource::Combined || src == ASource::Single) && w->bits != 8) return SQ_ERR_UNSUPPORTED;
   if (acc == nullptr && ldy < N) return SQ_ERR_INVALID_ARG;
   if (M > (int64_t)INT32_MAX - 2 * sq::BM) return SQ_ERR_RANGE;
   if (M == 0) return SQ_OK;
   if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::X && x == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::Codes && (q_pos == nullptr || q_neg == nullptr)) return SQ_ERR_INVALID_ARG;
-  if (src == ASource::Combined && q_pos == nullptr) return SQ_ERR_INVALID_ARG;
+  if ((src == ASource::Combined || src == ASource::Single) && q_pos == nullptr) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && y == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::X && (!aligned16(x) || (ldx * elt_size(xt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (src == ASource::Codes && (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0))
     return SQ_ERR_ALIGNMENT;
-  if (src == ASource::Combined && (!aligned16(q_pos) || ldq % 16 != 0)) return SQ_ERR_ALIGNMENT;
+  if ((src == ASource::Combined || src == ASource::Single) && (!aligned16(q_pos) || ldq % 16 != 0))
+    return SQ_ERR_ALIGNMENT;
   if (acc == nullptr && (!aligned16(y) || (ldy * elt_size(yt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (acc != nullptr && !aligned16(acc)) return SQ_ERR_ALIGNMENT;
   if (bias != nullptr && !aligned16(bias)) return SQ_ERR_ALIGNMENT;
@@ -478,6 +487,15 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
   const bool yb = (yt == SQ_BF16);
   const bool ac = (acc != nullptr);
+  if (src == ASource::Single) {
+    CUtensorMap ty;
+    st = make_tmap_y(&ty, y, yt, M, N, ldy);
+    if (st != SQ_OK) return st;
+    if (multi) return launch_codes_out<128, true, true>(yb, ta, ta, tw, ty, a, stream);
+    if (BN == 256) return launch_codes_out<256, false, true>(yb, ta, ta, tw, ty, a, stream);
+    if (BN == 192) return launch_codes_out<192, false, true>(yb, ta, ta, tw, ty, a, stream);
+    return launch_codes_out<128, false, true>(yb, ta, ta, tw, ty, a, stream);
+  }
   if (src == ASource::Combined) {
     if (multi) return launch_combined_out<128, true>(yb, ta, tw, a, stream);
     if (BN == 256) return launch_combined_out<256, false>(yb, ta, tw, a, stream);
@@ -648,7 +666,7 @@ sq_status sq_quantize_activations(const void* x, sq_dtype xt, int64_t M, int64_t
                                   const sq_segments* kseg, const float* s_pos,
                                   const float* s_neg, int8_t* q_pos, int8_t* q_neg, int64_t ldq,
                                   sq_stream_t stream) {
-  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq, false,
+  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq, sq::CODES_DUAL,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -656,7 +674,15 @@ sq_status sq_quantize_activations_combined(const void* x, sq_dtype xt, int64_t M
                                            int64_t ldx, const sq_segments* kseg,
                                            const float* s_pos, const float* s_neg, int8_t* c,
                                            int64_t ldc, sq_stream_t stream) {
-  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc, true,
+  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc,
+                        sq::CODES_COMBINED, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quantize_activations_single(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                         int64_t ldx, const sq_segments* kseg, const float* s_pos,
+                                         const float* s_neg, int8_t* c, int64_t ldc,
+                                         sq_stream_t stream) {
+  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, c, nullptr, ldc, sq::CODES_SINGLE,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -682,6 +708,14 @@ sq_status sq_linear_forward_combined(const int8_t* c, int64_t ldc, int64_t M, in
                                      sq_stream_t stream) {
   return gemm_common(ASource::Combined, nullptr, SQ_BF16, c, nullptr, ldc, M, K, 0, w, s_pos,
                      s_neg, bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int64_t K,
+                                   const sq_qweight* w, const float* s_pos, const float* s_neg,
+                                   const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                                   sq_stream_t stream) {
+  return gemm_common(ASource::Single, nullptr, SQ_BF16, c, nullptr, ldc, M, K, 0, w, s_pos, s_neg,
+                     bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_linear_accumulators(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,

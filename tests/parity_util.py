@@ -129,6 +129,25 @@ class Case:
         return y_ref, acc
 
 
+def compare_rows_single(case: "Case", y_gpu: torch.Tensor, rows: np.ndarray):
+    """The single-scale baseline's rows against the oracle (same tolerances)."""
+    wl = case.wl
+    xr = np.ascontiguousarray(case.x_np[rows])
+    out = "f32" if wl.out == "f32" else "bf16"
+    y_ref, acc, _ = O.linear_forward_single(xr, wl.kseg, case.o_sp, case.o_sn, case.o_wc,
+                                            case.o_ws, case.b_np, out=out, return_acc=True)
+    g = y_gpu[torch.as_tensor(rows, device=y_gpu.device)]
+    if wl.out == "f32":
+        ub, useg = O.units_of(8, wl.K, wl.kseg)
+        s = np.maximum(case.o_sp, case.o_sn)
+        acc2 = np.stack([acc, np.zeros_like(acc)], axis=1)
+        D = magnitude_sum(acc2, useg, s, s, O.unit_weight_scales(8, case.o_ws), case.b_np)
+        assert_f32_within(g.cpu().numpy(), y_ref, D)
+    else:
+        assert_bf16_within_1ulp(bf16_bits(g), y_ref)
+    return y_ref, acc
+
+
 def sample_rows(M: int, n: int, seed: int = 0) -> np.ndarray:
     """First and last tile rows, tile edges and a random spread."""
     fixed = [0, 1, 31, 32, 63, 64, 127, 128, M - 1, M - 2, M - 128, M - 129]

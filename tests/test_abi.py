@@ -149,6 +149,25 @@ def test_combined_code_entry_points_validate_before_launch():
     assert fwd(M=0) == L.SQ_OK
 
 
+def test_single_scale_entry_points_validate_before_launch():
+    lib = _lib.load()
+    L = _lib
+    seg, keep = _lib.segments((0, 512))
+    qs = lib.sq_quantize_activations_single
+    assert qs(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, 520, None) == L.SQ_ERR_ALIGNMENT
+    assert qs(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, None, 512, None) == L.SQ_ERR_INVALID_ARG
+    assert qs(FAKE, 9, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, 512, None) == L.SQ_ERR_INVALID_ARG
+    assert qs(FAKE, 1, 0, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, 512, None) == L.SQ_OK
+    qw, k = _qw(K=512)
+    fs = lib.sq_linear_forward_single
+    assert fs(None, 512, 256, 512, ctypes.byref(qw), FAKE, FAKE, None, FAKE, L.SQ_BF16, 256, None) == L.SQ_ERR_INVALID_ARG
+    assert fs(FAKE + 8, 512, 256, 512, ctypes.byref(qw), FAKE, FAKE, None, FAKE, L.SQ_BF16, 256, None) == L.SQ_ERR_ALIGNMENT
+    assert fs(FAKE, 512, 256, 512, ctypes.byref(qw), None, FAKE, None, FAKE, L.SQ_BF16, 256, None) == L.SQ_ERR_INVALID_ARG
+    qw4, k4 = _qw(bits=4, K=512)
+    assert fs(FAKE, 512, 256, 512, ctypes.byref(qw4), FAKE, FAKE, None, FAKE, L.SQ_BF16, 256, None) == L.SQ_ERR_UNSUPPORTED
+    assert fs(FAKE, 512, 0, 512, ctypes.byref(qw), FAKE, FAKE, None, FAKE, L.SQ_BF16, 256, None) == L.SQ_OK
+
+
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
