@@ -69,6 +69,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-small-m", action="store_true",
+                    help="skip the small-M (M <= 128, HBM-bound) measurements")
     return ap.parse_args()
 
 
@@ -80,6 +82,74 @@ def peaks():
         return float(p["bf16_tflops"]) * INT8_PER_BF16, float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_BF16_TFLOPS * INT8_PER_BF16, FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ L2 flush
+class L2Flush:
+    """Evicts the step's inputs from the 126 MB L2 before every timed launch:
+    writes a 256 MiB buffer, then reads a second 256 MiB buffer, so the dirty
+    lines of the write are written back inside the flush and the L2 is left
+    holding clean lines (a write-only flush would leave the next launch to pay
+    for writing ~126 MB back to HBM)."""
+
+    def __init__(self, dev):
+        import torch
+        self.a = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.b = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self, i: int):
+        self.a.fill_(i & 0xFF)
+        self.b.max()
+
+
+# ------------------------------------------------------------------ small M
+SMALL_M_SHAPES = ((3072, 12288), (4608, 1152))
+SMALL_M_ROWS = (16, 64, 128)
+
+
+def small_m_measure(dev, flush, steps: int, hbm_peak: float):
+    """HBM-bound small-M forwards (one K segment, int8 weights, bf16 out): the
+    split-K GEMM from codes and the one-pass GEMM from codes, each replayed
+    from a CUDA graph with the L2 flushed before every launch.  Bytes = weight
+    codes + weight scales + q+/q- codes + Y (the algorithmic traffic)."""
+    import torch
+    import post_quantized_linear_b200 as pq
+    from synth import workloads as W
+    out = []
+    for (K, N) in SMALL_M_SHAPES:
+        for M in SMALL_M_ROWS:
+            wl = W.small_case(M, K, N, seed=7, act="silu", bias=False, out="bf16")
+            x, w, _ = W.generate(wl)
+            xd, wd = x.to(dev), w.to(dev)
+            sp, sn = pq.calibrate(xd, wl.kseg)
+            qw = pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=8)
+            qp, qn = pq.quantize_activations(xd, wl.kseg, sp, sn)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = pq.splitk_workspace(M, N, K, device=dev)
+            res = {"M": M, "K": K, "N": N}
+            for name, fn in (("splitk", lambda: pq.linear_from_codes_splitk(qp, qn, qw, sp, sn, ws, out=y)),
+                             ("one_pass", lambda: pq.linear_from_codes(qp, qn, qw, sp, sn, out=y))):
+                fn()
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    fn()
+                ts = []
+                for i in range(max(steps, 5)):
+                    flush(i)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    g.replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ts.append(e0.elapsed_time(e1))
+                us = statistics.median(ts) * 1e3
+                byts = N * K + 4 * N + 2 * M * K + 2 * M * N
+                res[name] = {"us": us, "gbs": byts / (us * 1e-6) / 1e9,
+                             "frac_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
+                del g
+            out.append(res)
+    return out
 
 
 # ------------------------------------------------------------------ clocks
@@ -277,7 +347,7 @@ def run_ours(args):
         qp_buf = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
         qn_buf = None if combined else torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step(xs=xd, ws=wd, ys=y, gemm_events=None):
         pq.calibrate(calib if xs is xd else (xs if wl.calib_rows is None else xs[: wl.calib_rows]),
@@ -353,7 +423,7 @@ def run_ours(args):
     def timed(graph, n, salt):
         evs = events(n)
         for i in range(n):
-            flush.fill_((i + salt) & 0xFF)
+            flush(i + salt)
             evs[i][0].record(stream)
             graph.replay()
             evs[i][1].record(stream)
@@ -433,7 +503,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
             "data": "synthetic",
-            "config": config_of(wl, "flushed (256 MiB write between steps)", args.path),
+            "config": config_of(wl, "flushed (256 MiB write + 256 MiB read between steps)", args.path),
             "roofline": {
                 "bound": "tensor", "kernel": gemm_kernel_name(args.path, wl.bits, wl.x_dtype),
                 "achieved": gemm_tops, "peak": int8_peak_tops, "unit": "TOPS",
@@ -471,6 +541,12 @@ def run_ours(args):
             line["e2e"] = {"value": world * args.steps * ops / (e2e_ms * 1e-3) / 1e12,
                            "unit": "TOPS", "h2d_bytes_per_step": e2e["bi"],
                            "d2h_bytes_per_step": e2e["bo"]}
+        if world == 1 and not args.no_small_m:
+            line["small_m"] = {
+                "note": "HBM-bound forwards at M <= 128 (median of L2-flushed graph replays); "
+                        "bytes = weight codes + scales + q+/q- codes + Y; peak = measured HBM copy",
+                "peak_gbs": hbm_peak,
+                "cases": small_m_measure(dev, flush, args.steps, hbm_peak)}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, x, w, b)
         print(json.dumps(line), flush=True)

@@ -219,6 +219,34 @@ sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int6
                                    const float* bias, void* y, sq_dtype yt, int64_t ldy,
                                    sq_stream_t stream);
 
+/* Small-M forward from DualScale codes (1 <= M <= 128 tokens): the same result
+ * as sq_linear_forward_codes, bit for bit (SegQuant DualScale, Spanish
+ * technical summary 2.B; the two int8 products and the fused epilogue), with
+ * the weight stream spread over the whole GPU: the K dimension is split, each
+ * (N tile, K split) unit computes int32 partial accumulators, and the last
+ * unit of each output region adds them (integer sums are exact in any order)
+ * and runs the epilogue.  Requirements beyond sq_linear_forward_codes: int8
+ * weights with one K segment (else SQ_ERR_UNSUPPORTED); M <= 128 (else
+ * SQ_ERR_UNSUPPORTED).
+ * workspace: device memory, 256-byte aligned, at least the size returned by
+ * sq_splitk_workspace_size(M, N, K) on the same device; owned by the caller,
+ * used as scratch during the call.  Its first 256-byte-rounded block holds
+ * arrival counters that must be zero before the first call (cudaMemset); a
+ * call that completes leaves them zero again.  After a call that reported
+ * SQ_ERR_TIMEOUT, zero the workspace before reusing it.  Calls that share a
+ * workspace must not overlap on the GPU. */
+sq_status sq_linear_forward_codes_splitk(const int8_t* q_pos, const int8_t* q_neg, int64_t ldq,
+                                         int64_t M, int64_t K, const sq_qweight* w,
+                                         const float* s_pos, const float* s_neg,
+                                         const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                                         void* workspace, size_t workspace_bytes,
+                                         sq_stream_t stream);
+
+/* Host only: workspace bytes sq_linear_forward_codes_splitk needs for an
+ * [M, K] x [N, K]^T problem on the current device (the split count depends on
+ * the device's SM count).  1 <= M <= 128, N, K > 0, else SQ_ERR_INVALID_ARG. */
+sq_status sq_splitk_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes);
+
 /* Test surface: the same kernel as sq_linear_forward, but the epilogue writes
  * the raw int32 accumulators of every unit instead of Y:
  * acc[u][p][m][n], p = 0 for the (+) product, 1 for the (-) product; U units

@@ -25,6 +25,7 @@ from ._lib import SegQuantError
 __all__ = ["QuantizedWeight", "SegQuantError", "calibrate", "quantize_weights", "linear",
            "quantize_activations", "linear_from_codes", "quantize_activations_combined",
            "linear_from_combined", "quantize_activations_single", "linear_from_single",
+           "splitk_workspace_size", "splitk_workspace", "linear_from_codes_splitk",
            "linear_accumulators", "stream_status", "qweight_sizes"]
 
 
@@ -245,6 +246,43 @@ def linear_from_single(c: torch.Tensor, qw: QuantizedWeight, s_pos: torch.Tensor
     _lib.check("sq_linear_forward_single", _lib.load().sq_linear_forward_single(
         _ptr(c), c.stride(0), M, K, ctypes.byref(cw), _ptr(s_pos), _ptr(s_neg), _ptr(bias),
         _ptr(out), _dtype_code(out.dtype), out.stride(0), _stream(stream)))
+    return out
+
+
+def splitk_workspace_size(M: int, N: int, K: int) -> int:
+    """Bytes of workspace ``linear_from_codes_splitk`` needs on the current device."""
+    n = ctypes.c_size_t()
+    _lib.check("sq_splitk_workspace_size",
+               _lib.load().sq_splitk_workspace_size(M, N, K, ctypes.byref(n)))
+    return n.value
+
+
+def splitk_workspace(M: int, N: int, K: int, device=None) -> torch.Tensor:
+    """A zeroed workspace for ``linear_from_codes_splitk`` (uint8, 256-byte aligned)."""
+    return torch.zeros(splitk_workspace_size(M, N, K), dtype=torch.uint8, device=device)
+
+
+def linear_from_codes_splitk(q_pos: torch.Tensor, q_neg: torch.Tensor, qw: QuantizedWeight,
+                             s_pos: torch.Tensor, s_neg: torch.Tensor, workspace: torch.Tensor,
+                             bias: Optional[torch.Tensor] = None,
+                             out_dtype: torch.dtype = torch.bfloat16,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Small-M (M <= 128) forward from DualScale codes, K split across the GPU;
+    bit-identical to ``linear_from_codes``.  ``workspace`` from ``splitk_workspace``
+    (its counters return to zero after every completed call)."""
+    _check_2d(q_pos, "q_pos")
+    _check_2d(q_neg, "q_neg")
+    M, K = q_pos.shape
+    if q_neg.shape != q_pos.shape or q_neg.stride(0) != q_pos.stride(0):
+        raise ValueError("q_pos and q_neg must have the same shape and row stride")
+    if out is None:
+        out = torch.empty((M, qw.N), dtype=out_dtype, device=q_pos.device)
+    _check_2d(out, "out")
+    c, keep = qw.c_struct()
+    _lib.check("sq_linear_forward_codes_splitk", _lib.load().sq_linear_forward_codes_splitk(
+        _ptr(q_pos), _ptr(q_neg), q_pos.stride(0), M, K, ctypes.byref(c), _ptr(s_pos), _ptr(s_neg),
+        _ptr(bias), _ptr(out), _dtype_code(out.dtype), out.stride(0), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 
 

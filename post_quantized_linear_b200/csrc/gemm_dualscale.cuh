@@ -83,6 +83,15 @@ struct GemmArgs {
   int32_t* acc_out;        // [U][2][M][N] (accumulator mode)
   long long wait_budget;   // clock cycles per pipeline wait
   int32_t starve;          // test hook: the TMA producer issues nothing
+  // split-K (small M): K splits per N tile, k blocks per split, workspace
+  int32_t splits;
+  int32_t kb_per_split;
+  int32_t* ws_count;       // [num_tiles][8] arrival counters (zero between calls)
+  int32_t* ws_part;        // [splits][2][M][N] partial accumulators
+  // activation codes read by cp.async loader warps (GEMM from codes)
+  const int8_t* a_pos;     // q+ (or the single code) [M][lda]
+  const int8_t* a_neg;     // q- [M][lda]
+  int64_t lda;
 };
 
 // Teardown waits (copies and MMAs that were issued always complete) get a

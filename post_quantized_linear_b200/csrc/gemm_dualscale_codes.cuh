@@ -31,15 +31,37 @@ constexpr int kCodesEpiWarp0 = 2;
 __host__ __device__ constexpr int codes_kernel_threads(bool multi) {
   return (kCodesEpiWarp0 + epi_warps(multi)) * 32;
 }
+__host__ __device__ constexpr int codes_threads_epw(int epw) { return (kCodesEpiWarp0 + epw) * 32; }
 
-template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE>
+// LDA: the activation code tiles are copied by four loader warps with cp.async
+// (16 bytes per thread, eight lanes per 128-byte row, zero-filled past M and
+// K) instead of TMA; TMA then carries only the weight tile.  An option (the
+// SM's TMA engine moves about 50 bytes per clock in 128-row boxes, less than
+// two code tiles plus a weight tile per k block need at the int8 MMA rate),
+// measured slower than all-TMA loads on the DiT and MMDiT shapes.
+constexpr int kLoaderWarps = 4;
+__host__ __device__ constexpr int codes_epi_warp0(bool lda) {
+  return lda ? kCodesEpiWarp0 + kLoaderWarps : kCodesEpiWarp0;
+}
+__host__ __device__ constexpr int codes_threads(int epw, bool lda) {
+  return (codes_epi_warp0(lda) + epw) * 32;
+}
+
+// EPW_: epilogue warps (4, 8 or 16; a multiple of 4, each lane quarter of TMEM
+// read by EPW/4 warps splitting the tile's columns).  Four warps let narrow
+// tiles (BN = 32, 64, 96) store whole 32-column passes -- the small-M shapes.
+template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
+          bool LDA_ = false>
 struct CodesCfg {
+  static constexpr bool LDA = LDA_;
+  // full barrier: the TMA thread's arrival (+ bytes), plus one per loader thread
+  static constexpr int FULL_COUNT = 1 + (LDA_ ? kLoaderWarps * 32 : 0);
   static constexpr int BN = BN_;
   static constexpr int NACC = SINGLE ? 1 : 2;          // accumulators (code tiles) per unit
   static constexpr int A_BYTES = NACC * BM * BK;      // q+ and q- tiles, or the single code tile
   static constexpr int W_BYTES = BN * BK;
   static constexpr int STAGE = A_BYTES + W_BYTES;
-  static constexpr int EPW = epi_warps(MULTI);
+  static constexpr int EPW = EPW_;
   static constexpr int Y_BYTES = EPW * stage_y_bytes(Y_BF16);
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
   static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
@@ -55,14 +77,17 @@ struct CodesCfg {
   static_assert(OFF_Y % 1024 == 0 && stage_y_bytes(Y_BF16) % 1024 == 0, "staging alignment");
 };
 
-template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false>
-__global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
+template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false, int EPW = epi_warps(MULTI),
+          bool LDA = false>
+__global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE>;
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA>;
+  constexpr int EPI0 = codes_epi_warp0(LDA);
+  static_assert(EPW % 4 == 0 && (BN / (EPW / 4)) % 32 == 0, "32-column store passes per warp");
   static_assert(!MULTI || (BN == 128 && C::NBUF == 2), "several units per tile: BN = 128, two buffers");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -82,12 +107,12 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::S; ++i) {
-      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(full + i), C::FULL_COUNT);
       mbar_init(smem_u32(empty + i), 1);
     }
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(smem_u32(tmem_full + i), 1);
-      mbar_init(smem_u32(tmem_empty + i), epi_warps(MULTI));
+      mbar_init(smem_u32(tmem_empty + i), C::EPW);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
@@ -121,10 +146,14 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
           const int s = c % C::S;
           if (!(ok = wait1(smem_u32(empty + s), ((c / C::S) & 1) ^ 1, abort_flag, budget))) break;
           uint8_t* st = smem + s * C::STAGE;
-          mbar_arrive_expect_tx(smem_u32(full + s), C::STAGE);
-          tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
-          if constexpr (!SINGLE)
-            tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
+          if constexpr (LDA) {
+            mbar_arrive_expect_tx(smem_u32(full + s), C::W_BYTES);
+          } else {
+            mbar_arrive_expect_tx(smem_u32(full + s), C::STAGE);
+            tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
+            if constexpr (!SINGLE)
+              tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
+          }
           tma_load_2d(smem_u32(st + C::A_BYTES), &tmap_w, smem_u32(full + s), kb * BK, t.n0);
           ++c;
         }
@@ -152,6 +181,8 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
           }
           const int s = c % C::S;
           if (!(ok = wait1(smem_u32(full + s), (c / C::S) & 1, abort_flag, budget))) break;
+          // code tiles written by cp.async (generic proxy) before the tensor core reads them
+          if constexpr (LDA) fence_proxy_async_smem();
           const uint32_t a_p = smem_u32(smem + s * C::STAGE);
           const uint32_t a_n = a_p + BM * BK;
           const uint32_t b_w = a_p + C::A_BYTES;
@@ -177,14 +208,51 @@ __global__ void __launch_bounds__(codes_kernel_threads(MULTI), 1)
       umma_commit(smem_u32(drain_bar));
       wait_drain(smem_u32(drain_bar), 0, kDrainBudget);
     }
+  } else if (warp < EPI0) {
+    // --------------------------------------------- code-tile loader warps (LDA)
+    // Thread t: rows (t >> 5) * 32 + 4 * i + ((t & 31) >> 3), i = 0..7, 16-byte
+    // chunk t & 7 of the row's 128-byte k block, stored at the 128-byte-swizzle
+    // position (chunk ^ (row & 7)) of the row -- the layout TMA would write.
+    if constexpr (LDA) {
+      const int t_id = threadIdx.x - kCodesEpiWarp0 * 32;   // 0..127
+      const int chunk = t_id & 7;
+      const int r0 = (t_id >> 5) * 32 + ((t_id & 31) >> 3);
+      int c = 0;
+      bool ok = (args.starve == 0);
+      for (int it = 0; it < rounds && ok; ++it) {
+        Tile t;
+        if (!tiles(it, t)) continue;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          const int s = c % C::S;
+          if (!(ok = wait_warp(smem_u32(empty + s), ((c / C::S) & 1) ^ 1, abort_flag, budget))) break;
+          const uint32_t st = smem_u32(smem + s * C::STAGE);
+          const int k = kb * BK + chunk * 16;
+          const bool k_in = k < args.K;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = r0 + 4 * i;
+            const int grow = t.m0 + r;
+            const bool in = k_in && grow < args.M;
+            const int64_t off = in ? (int64_t)grow * args.lda + k : 0;
+            const uint32_t dst = st + (uint32_t)(r * 128 + ((chunk ^ (r & 7)) << 4));
+            cp_async16(dst, args.a_pos + off, in ? 16u : 0u);
+            if constexpr (!SINGLE) cp_async16(dst + BM * BK, args.a_neg + off, in ? 16u : 0u);
+          }
+          cp_async_arrive_noinc(smem_u32(full + s));
+          ++c;
+        }
+      }
+      // every copy of this thread has landed before the CTA can exit
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
   } else {
     // --------------------------------------------------------- epilogue
-    // Warp w reads TMEM lanes 32*(w % 4) .. +31; warps 2..(2+E-1) cover each
-    // lane quarter once per column part.
+    // Warp w reads TMEM lanes 32*(w % 4) .. +31; the EPW epilogue warps cover
+    // each lane quarter once per column part.
     const int quad = warp & 3;
-    const int part = (warp - kCodesEpiWarp0) >> 2;
+    const int part = (warp - EPI0) >> 2;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    uint8_t* stage_y = smem + C::OFF_Y + (warp - kCodesEpiWarp0) * stage_y_bytes(Y_BF16);
+    uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
     epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
         args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
         tiles, abort_flag, budget);

@@ -18,6 +18,7 @@
 #include "gemm_dualscale.cuh"
 #include "gemm_dualscale_codes.cuh"
 #include "gemm_dualscale_combined.cuh"
+#include "gemm_dualscale_splitk.cuh"
 #include "gemm_dualscale_inplace.cuh"
 #include "gemm_dualscale_pair.cuh"
 #include "ptx.cuh"
@@ -218,11 +219,23 @@ sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const
                 : launch_inplace<BN, false, false, MULTI>(tx, tw, a, stream);
 }
 
-template <int BN, bool YB, bool MULTI, bool SINGLE>
+// Whether the GEMM from codes copies the code tiles with cp.async loader warps
+// (TMA then carries only the weight tile); SEGQUANT_CODES_LDA=0 loads every
+// operand by TMA.  One unit per tile only.
+bool use_codes_lda() {
+  if (const char* e = std::getenv("SEGQUANT_CODES_LDA")) return std::atoi(e) != 0;
+  return false;
+}
+
+
+template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE>;
-  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE>;
+  if constexpr (!MULTI && !LDA) {
+    if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
+  }
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA>;
+  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
@@ -232,16 +245,55 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int grid = num_sms();
   if (grid > a.num_tiles) grid = a.num_tiles;
-  kern<<<grid, sq::codes_kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
+  kern<<<grid, sq::codes_threads(EPW, LDA), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
   return cuda_status(cudaGetLastError());
 }
 
-template <int BN, bool MULTI, bool SINGLE = false>
+template <int BN, bool MULTI, bool SINGLE = false, int EPW = sq::epi_warps(MULTI)>
 sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                            const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                            cudaStream_t stream) {
-  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE>(tqp, tqn, tw, ty, a, stream)
-                : launch_codes<BN, false, MULTI, SINGLE>(tqp, tqn, tw, ty, a, stream);
+  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE, EPW>(tqp, tqn, tw, ty, a, stream)
+                : launch_codes<BN, false, MULTI, SINGLE, EPW>(tqp, tqn, tw, ty, a, stream);
+}
+
+// Small M (one row tile): the work is streaming the weight codes, so the tile
+// width spreads N over as many SMs as possible.  Candidates 32..256 (multiples
+// of 32, four epilogue warps); cost = waves x cycles per MMA, where an M = 128
+// MMA takes about BN/2 cycles but no less than 48 (narrow products lose rate);
+// ties go to the narrower tile (more SMs share the stream).  0 = not small.
+int choose_bn_small(int64_t M, int64_t N) {
+  if (M > sq::BM) return 0;
+  if (const char* e = std::getenv("SEGQUANT_BN_SMALL")) {
+    const int v = std::atoi(e);
+    if (v == 32 || v == 64 || v == 96 || v == 128) return v;
+    if (v == -1) return 0;   // the regular tile choice
+  }
+  const int sms = num_sms();
+  int best = 0;
+  double best_cost = 0.0;
+  for (int bn : {32, 64, 96, 128}) {
+    const int64_t tiles = (N + bn - 1) / bn;
+    const double waves = (double)((tiles + sms - 1) / sms);
+    const double cost = waves * std::max(bn, 96);
+    if (best == 0 || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+template <bool SINGLE>
+sq_status launch_codes_small(int bn, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+                             const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                             cudaStream_t stream) {
+  switch (bn) {
+    case 32: return launch_codes_out<32, false, SINGLE, 4>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 64: return launch_codes_out<64, false, SINGLE, 4>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 96: return launch_codes_out<96, false, SINGLE, 4>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    default: return launch_codes_out<128, false, SINGLE, 4>(y_bf16, tqp, tqn, tw, ty, a, stream);
+  }
 }
 
 // Tensor map of Y for the TMA-store epilogue: boxes of 32 rows x 32 columns,
@@ -277,6 +329,43 @@ sq_status launch_combined_out(bool y_bf16, const CUtensorMap& tc, const CUtensor
                               const sq::GemmArgs& a, cudaStream_t stream) {
   return y_bf16 ? launch_combined<BN, true, MULTI>(tc, tw, a, stream)
                 : launch_combined<BN, false, MULTI>(tc, tw, a, stream);
+}
+
+// Split-K plan for M <= 128: tile width, K splits and workspace layout.  Units
+// (N tile, K split) are sized to fill the SMs once; every split gets at least
+// one k block.
+struct SplitPlan {
+  int bn, splits, kb_per_split, n_tiles;
+  size_t count_bytes, part_bytes;
+};
+
+SplitPlan plan_splitk(int64_t M, int64_t N, int64_t K) {
+  SplitPlan p;
+  p.bn = (N >= 2048) ? 256 : 128;
+  p.n_tiles = (int)((N + p.bn - 1) / p.bn);
+  const int num_kb = (int)((K + sq::BK - 1) / sq::BK);
+  int splits = num_sms() / p.n_tiles;
+  splits = std::max(1, std::min(splits, std::min(num_kb, 16)));
+  p.kb_per_split = (num_kb + splits - 1) / splits;
+  p.splits = (num_kb + p.kb_per_split - 1) / p.kb_per_split;
+  p.count_bytes = ((size_t)p.n_tiles * 8 * sizeof(int32_t) + 255) / 256 * 256;
+  p.part_bytes = (size_t)p.splits * 2 * (size_t)M * (size_t)N * sizeof(int32_t);
+  return p;
+}
+
+template <int BN, bool YB>
+sq_status launch_splitk(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
+                        sq::GemmArgs a, cudaStream_t stream) {
+  using C = sq::SplitKCfg<BN>;
+  auto kern = sq::dualscale_gemm_splitk_kernel<BN, YB>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_status(e);
+  int grid = num_sms();
+  const int units = a.num_tiles * a.splits;
+  if (grid > units) grid = units;
+  kern<<<grid, sq::codes_kernel_threads(false), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, a);
+  return cuda_status(cudaGetLastError());
 }
 
 // Whether the GEMM from int8 codes runs the one-ring kernel (codes and weight
@@ -434,6 +523,11 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const bool f32x = (src == ASource::X && xt == SQ_F32);
   const bool pair = (src == ASource::Codes) && use_pair(N, w4);
   int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x);
+  // one row tile, one unit per tile, GEMM from codes: narrow tiles over all SMs
+  const int bn_small = (!multi && acc == nullptr && (src == ASource::Codes || src == ASource::Single) &&
+                        !(src == ASource::Codes && use_pair(N, w4)) && use_codes_ring())
+                           ? choose_bn_small(M, N) : 0;
+  if (bn_small) BN = bn_small;
   if (pair && !multi && acc == nullptr) {
     BN = 256;
     if (const char* e = std::getenv("SEGQUANT_BN")) BN = std::atoi(e) == 128 ? 128 : 256;
@@ -482,6 +576,9 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   a.acc_out = acc;
   a.wait_budget = g_wait_budget;
   a.starve = g_debug_starve;
+  a.a_pos = q_pos;
+  a.a_neg = q_neg;
+  a.lda = ldq;
 
   using bf = __nv_bfloat16;
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
@@ -492,6 +589,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     st = make_tmap_y(&ty, y, yt, M, N, ldy);
     if (st != SQ_OK) return st;
     if (multi) return launch_codes_out<128, true, true>(yb, ta, ta, tw, ty, a, stream);
+    if (bn_small) return launch_codes_small<true>(bn_small, yb, ta, ta, tw, ty, a, stream);
     if (BN == 256) return launch_codes_out<256, false, true>(yb, ta, ta, tw, ty, a, stream);
     if (BN == 192) return launch_codes_out<192, false, true>(yb, ta, ta, tw, ty, a, stream);
     return launch_codes_out<128, false, true>(yb, ta, ta, tw, ty, a, stream);
@@ -514,6 +612,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       st = make_tmap_y(&ty, y, yt, M, N, ldy);
       if (st != SQ_OK) return st;
       if (multi) return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
+      if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, ty, a, stream);
       if (BN == 192) return launch_codes_out<192, false>(yb, ta, ta2, tw, ty, a, stream);
       return launch_codes_out<128, false>(yb, ta, ta2, tw, ty, a, stream);
@@ -716,6 +815,77 @@ sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int6
                                    sq_stream_t stream) {
   return gemm_common(ASource::Single, nullptr, SQ_BF16, c, nullptr, ldc, M, K, 0, w, s_pos, s_neg,
                      bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_splitk_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {
+  if (bytes == nullptr || M < 1 || M > 128 || N <= 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  const SplitPlan p = plan_splitk(M, N, K);
+  *bytes = p.count_bytes + p.part_bytes;
+  return SQ_OK;
+}
+
+sq_status sq_linear_forward_codes_splitk(const int8_t* q_pos, const int8_t* q_neg, int64_t ldq,
+                                         int64_t M, int64_t K, const sq_qweight* w,
+                                         const float* s_pos, const float* s_neg,
+                                         const float* bias, void* y, sq_dtype yt, int64_t ldy,
+                                         void* workspace, size_t workspace_bytes,
+                                         sq_stream_t stream) {
+  if (!dtype_ok(yt) || M < 0 || K <= 0 || ldq < K) return SQ_ERR_INVALID_ARG;
+  SegBounds kseg;
+  sq_status st = check_qweight(w, K, &kseg);
+  if (st != SQ_OK) return st;
+  const int64_t N = w->N;
+  if (w->bits != 8 || kseg.count != 1 || M > 128) return SQ_ERR_UNSUPPORTED;
+  if (ldy < N) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;
+  if (q_pos == nullptr || q_neg == nullptr || s_pos == nullptr || s_neg == nullptr ||
+      y == nullptr || workspace == nullptr)
+    return SQ_ERR_INVALID_ARG;
+  if (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0 || !aligned16(y) ||
+      (ldy * elt_size(yt)) % 16 != 0 || (bias != nullptr && !aligned16(bias)) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(s_pos) & 3u) || (reinterpret_cast<uintptr_t>(s_neg) & 3u))
+    return SQ_ERR_ALIGNMENT;
+  const SplitPlan p = plan_splitk(M, N, K);
+  if (workspace_bytes < p.count_bytes + p.part_bytes) return SQ_ERR_INVALID_ARG;
+  CUtensorMap ta, ta2, tw;
+  st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
+                 (uint64_t)ldq, 128, sq::BM);
+  if (st != SQ_OK) return st;
+  st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
+                 (uint64_t)ldq, 128, sq::BM);
+  if (st != SQ_OK) return st;
+  st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K, (uint64_t)N,
+                 (uint64_t)K, 128, (uint32_t)p.bn);
+  if (st != SQ_OK) return st;
+  sq::GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int32_t)M;
+  a.N = (int32_t)N;
+  a.K = (int32_t)K;
+  a.num_kb = (int32_t)((K + sq::BK - 1) / sq::BK);
+  a.bits = 8;
+  a.kseg = kseg;
+  a.m_tiles = 1;
+  a.n_full = (int32_t)(N / p.bn);
+  a.tail = (int32_t)(N % p.bn);
+  a.num_tiles = p.n_tiles;
+  a.s_pos = s_pos;
+  a.s_neg = s_neg;
+  a.wscales = w->scales;
+  a.bias = bias;
+  a.y = y;
+  a.ldy = ldy;
+  a.wait_budget = g_wait_budget;
+  a.starve = g_debug_starve;
+  a.splits = p.splits;
+  a.kb_per_split = p.kb_per_split;
+  a.ws_count = static_cast<int32_t*>(workspace);
+  a.ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + p.count_bytes);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool yb = (yt == SQ_BF16);
+  if (p.bn == 256) return yb ? launch_splitk<256, true>(ta, ta2, tw, a, s) : launch_splitk<256, false>(ta, ta2, tw, a, s);
+  return yb ? launch_splitk<128, true>(ta, ta2, tw, a, s) : launch_splitk<128, false>(ta, ta2, tw, a, s);
 }
 
 sq_status sq_linear_accumulators(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,

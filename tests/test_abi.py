@@ -168,6 +168,31 @@ def test_single_scale_entry_points_validate_before_launch():
     assert fs(FAKE, 512, 0, 512, ctypes.byref(qw), FAKE, FAKE, None, FAKE, L.SQ_BF16, 256, None) == L.SQ_OK
 
 
+def test_splitk_entry_points_validate_before_launch():
+    lib = _lib.load()
+    L = _lib
+    n = ctypes.c_size_t()
+    assert lib.sq_splitk_workspace_size(129, 1024, 1024, ctypes.byref(n)) == L.SQ_ERR_INVALID_ARG
+    assert lib.sq_splitk_workspace_size(0, 1024, 1024, ctypes.byref(n)) == L.SQ_ERR_INVALID_ARG
+    assert lib.sq_splitk_workspace_size(64, 1024, 1024, None) == L.SQ_ERR_INVALID_ARG
+    qw, k = _qw(K=512)
+    f = lib.sq_linear_forward_codes_splitk
+
+    def call(M=64, q=FAKE, ws=FAKE, wsb=1 << 30, qw_=qw, y=FAKE):
+        return f(q, q, 512, M, 512, ctypes.byref(qw_), FAKE, FAKE, None, y, L.SQ_BF16, 256, ws,
+                 wsb, None)
+    assert call(M=200) == L.SQ_ERR_UNSUPPORTED
+    qws, ks = _qw(kb=(0, 256, 512))
+    assert call(qw_=qws) == L.SQ_ERR_UNSUPPORTED
+    qw4, k4 = _qw(bits=4, K=512)
+    assert call(qw_=qw4) == L.SQ_ERR_UNSUPPORTED
+    assert call(ws=None) == L.SQ_ERR_INVALID_ARG
+    assert call(ws=FAKE + 16) == L.SQ_ERR_ALIGNMENT          # 256-byte alignment
+    assert call(wsb=16) == L.SQ_ERR_INVALID_ARG
+    assert call(q=FAKE + 8) == L.SQ_ERR_ALIGNMENT
+    assert call(M=0) == L.SQ_OK
+
+
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -133,6 +133,32 @@ def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch):
     assert torch.equal(y1.view(iv), y0.view(iv))
 
 
+@pytest.mark.parametrize("bn", ["128", "192", "256"])
+@pytest.mark.parametrize("MKN", [(390, 768, 656), (300, 640, 272), (64, 1024, 512), (1, 256, 96)])
+def test_code_tiles_by_cp_async_or_tma_agree(MKN, bn, monkeypatch):
+    """The GEMM from codes with the code tiles copied by cp.async loader warps
+    and with every operand loaded by TMA: the oracle's result, identical bits,
+    DualScale and single-scale, ragged M, N and K tails."""
+    import post_quantized_linear_b200 as pq
+    from parity_util import compare_rows_single
+    monkeypatch.setenv("SEGQUANT_BN", bn)
+    M, K, N = MKN
+    c = Case(W.small_case(M, K, N, seed=90 + M, out="bf16"))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    c1 = pq.quantize_activations_single(c.x, c.wl.kseg, c.sp, c.sn)
+    ys = {}
+    for lda in ("1", "0"):
+        monkeypatch.setenv("SEGQUANT_CODES_LDA", lda)
+        ys[lda] = (pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b),
+                   pq.linear_from_single(c1, c.qw, c.sp, c.sn, c.b))
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(ys["1"][0], np.arange(M))
+    compare_rows_single(c, ys["1"][1], np.arange(M))
+    for i in range(2):
+        assert torch.equal(ys["1"][i].view(torch.int16), ys["0"][i].view(torch.int16))
+
+
 def test_forward_exact_in_fp32():
     """With the fp32 epilogue order the kernel reproduces the oracle bit for bit."""
     c = Case(_small(1))
