@@ -247,6 +247,31 @@ sq_status sq_linear_forward_codes_splitk(const int8_t* q_pos, const int8_t* q_ne
  * the device's SM count).  1 <= M <= 128, N, K > 0, else SQ_ERR_INVALID_ARG. */
 sq_status sq_splitk_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes);
 
+/* No counterpart in the SegQuant pages: an interface for callers that cannot
+ * allocate device memory at call time.  The same computation and result as
+ * sq_linear_forward_codes_splitk, with its workspace in a library-owned
+ * file-scope device array of SQ_SPLITK_STATIC_SCRATCH_BYTES (16 MiB) per
+ * device instead of a caller buffer.  The call allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine).
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.
+ * Zeroing: every call clears the array's arrival counters itself
+ * (cudaMemsetAsync on `stream`) before its kernel; the partial sums need no
+ * clearing.
+ * Sharing: all calls on a device share the one array, so calls that overlap
+ * on the GPU (on different streams without ordering between them) race; order
+ * them on one stream.
+ * Limit: if the split-K workspace for (M, N, K) exceeds the array even with a
+ * single K split (8 * M * N bytes plus the counters), SQ_ERR_RANGE.  Other
+ * requirements and errors as for sq_linear_forward_codes_splitk. */
+#define SQ_SPLITK_STATIC_SCRATCH_BYTES (16u << 20)
+sq_status sq_linear_forward_codes_splitk_static(const int8_t* q_pos, const int8_t* q_neg,
+                                                int64_t ldq, int64_t M, int64_t K,
+                                                const sq_qweight* w, const float* s_pos,
+                                                const float* s_neg, const float* bias, void* y,
+                                                sq_dtype yt, int64_t ldy, sq_stream_t stream);
+
 /* Test surface: the same kernel as sq_linear_forward, but the epilogue writes
  * the raw int32 accumulators of every unit instead of Y:
  * acc[u][p][m][n], p = 0 for the (+) product, 1 for the (-) product; U units

@@ -57,6 +57,8 @@ SIGNATURES = {
                                                c_vp, c_vp, c_i32, c_i64, c_vp, ctypes.c_size_t,
                                                c_vp]),
     "sq_splitk_workspace_size": (c_i32, [c_i64, c_i64, c_i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "sq_linear_forward_codes_splitk_static": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i64, P_QW, c_vp,
+                                                      c_vp, c_vp, c_vp, c_i32, c_i64, c_vp]),
     "sq_linear_accumulators": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp,
                                        c_vp]),
     "sq_stream_status": (c_i32, [c_vp]),

@@ -24,6 +24,11 @@
 #include "ptx.cuh"
 #include "quant_kernels.cuh"
 
+// Scratch of sq_linear_forward_codes_splitk_static: a file-scope device array,
+// one per device (zero at module load), located with cudaGetSymbolAddress
+// once per device on the first call with that device current.
+static __device__ __align__(256) uint8_t g_splitk_scratch[SQ_SPLITK_STATIC_SCRATCH_BYTES];
+
 namespace {
 
 using sq::SegBounds;
@@ -351,6 +356,43 @@ SplitPlan plan_splitk(int64_t M, int64_t N, int64_t K) {
   p.count_bytes = ((size_t)p.n_tiles * 8 * sizeof(int32_t) + 255) / 256 * 256;
   p.part_bytes = (size_t)p.splits * 2 * (size_t)M * (size_t)N * sizeof(int32_t);
   return p;
+}
+
+// The split-K plan with its workspace capped at `cap` bytes: fewer K splits
+// until it fits; false if even one split does not.
+bool plan_splitk_capped(int64_t M, int64_t N, int64_t K, size_t cap, SplitPlan* out) {
+  SplitPlan p = plan_splitk(M, N, K);
+  const int num_kb = (int)((K + sq::BK - 1) / sq::BK);
+  for (int want = p.splits; want >= 1; --want) {
+    p.kb_per_split = (num_kb + want - 1) / want;
+    p.splits = (num_kb + p.kb_per_split - 1) / p.kb_per_split;
+    p.part_bytes = (size_t)p.splits * 2 * (size_t)M * (size_t)N * sizeof(int32_t);
+    if (p.count_bytes + p.part_bytes <= cap) {
+      *out = p;
+      return true;
+    }
+  }
+  return false;
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+sq_status static_scratch(void** out) {
+  int dev = 0;
+  sq_status st = cuda_status(cudaGetDevice(&dev));
+  if (st != SQ_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return SQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    st = cuda_status(cudaGetSymbolAddress(&p, g_splitk_scratch));
+    if (st != SQ_OK) return st;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SQ_OK;
 }
 
 template <int BN, bool YB>
@@ -883,6 +925,73 @@ sq_status sq_linear_forward_codes_splitk(const int8_t* q_pos, const int8_t* q_ne
   a.ws_count = static_cast<int32_t*>(workspace);
   a.ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + p.count_bytes);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool yb = (yt == SQ_BF16);
+  if (p.bn == 256) return yb ? launch_splitk<256, true>(ta, ta2, tw, a, s) : launch_splitk<256, false>(ta, ta2, tw, a, s);
+  return yb ? launch_splitk<128, true>(ta, ta2, tw, a, s) : launch_splitk<128, false>(ta, ta2, tw, a, s);
+}
+
+sq_status sq_linear_forward_codes_splitk_static(const int8_t* q_pos, const int8_t* q_neg,
+                                                int64_t ldq, int64_t M, int64_t K,
+                                                const sq_qweight* w, const float* s_pos,
+                                                const float* s_neg, const float* bias, void* y,
+                                                sq_dtype yt, int64_t ldy, sq_stream_t stream) {
+  if (!dtype_ok(yt) || M < 0 || K <= 0 || ldq < K) return SQ_ERR_INVALID_ARG;
+  SegBounds kseg;
+  sq_status st = check_qweight(w, K, &kseg);
+  if (st != SQ_OK) return st;
+  const int64_t N = w->N;
+  if (w->bits != 8 || kseg.count != 1 || M > 128) return SQ_ERR_UNSUPPORTED;
+  if (ldy < N) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;
+  if (q_pos == nullptr || q_neg == nullptr || s_pos == nullptr || s_neg == nullptr || y == nullptr)
+    return SQ_ERR_INVALID_ARG;
+  if (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0 || !aligned16(y) ||
+      (ldy * elt_size(yt)) % 16 != 0 || (bias != nullptr && !aligned16(bias)) ||
+      (reinterpret_cast<uintptr_t>(s_pos) & 3u) || (reinterpret_cast<uintptr_t>(s_neg) & 3u))
+    return SQ_ERR_ALIGNMENT;
+  SplitPlan p;
+  if (!plan_splitk_capped(M, N, K, SQ_SPLITK_STATIC_SCRATCH_BYTES, &p)) return SQ_ERR_RANGE;
+  void* scratch = nullptr;
+  st = static_scratch(&scratch);
+  if (st != SQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the arrival counters start every call at zero
+  st = cuda_status(cudaMemsetAsync(scratch, 0, p.count_bytes, s));
+  if (st != SQ_OK) return st;
+  CUtensorMap ta, ta2, tw;
+  st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
+                 (uint64_t)ldq, 128, sq::BM);
+  if (st != SQ_OK) return st;
+  st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
+                 (uint64_t)ldq, 128, sq::BM);
+  if (st != SQ_OK) return st;
+  st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K, (uint64_t)N,
+                 (uint64_t)K, 128, (uint32_t)p.bn);
+  if (st != SQ_OK) return st;
+  sq::GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int32_t)M;
+  a.N = (int32_t)N;
+  a.K = (int32_t)K;
+  a.num_kb = (int32_t)((K + sq::BK - 1) / sq::BK);
+  a.bits = 8;
+  a.kseg = kseg;
+  a.m_tiles = 1;
+  a.n_full = (int32_t)(N / p.bn);
+  a.tail = (int32_t)(N % p.bn);
+  a.num_tiles = p.n_tiles;
+  a.s_pos = s_pos;
+  a.s_neg = s_neg;
+  a.wscales = w->scales;
+  a.bias = bias;
+  a.y = y;
+  a.ldy = ldy;
+  a.wait_budget = g_wait_budget;
+  a.starve = g_debug_starve;
+  a.splits = p.splits;
+  a.kb_per_split = p.kb_per_split;
+  a.ws_count = static_cast<int32_t*>(scratch);
+  a.ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + p.count_bytes);
   const bool yb = (yt == SQ_BF16);
   if (p.bn == 256) return yb ? launch_splitk<256, true>(ta, ta2, tw, a, s) : launch_splitk<256, false>(ta, ta2, tw, a, s);
   return yb ? launch_splitk<128, true>(ta, ta2, tw, a, s) : launch_splitk<128, false>(ta, ta2, tw, a, s);
