@@ -225,8 +225,8 @@ sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const
 }
 
 // Whether the GEMM from codes copies the code tiles with cp.async loader warps
-// (TMA then carries only the weight tile); SEGQUANT_CODES_LDA=0 loads every
-// operand by TMA.  One unit per tile only.
+// (TMA then carries only the weight tile); off unless SEGQUANT_CODES_LDA=1
+// (measured slower than all-TMA loads on the DiT, MMDiT and SegLinear shapes).
 bool use_codes_lda() {
   if (const char* e = std::getenv("SEGQUANT_CODES_LDA")) return std::atoi(e) != 0;
   return false;
@@ -236,7 +236,7 @@ bool use_codes_lda() {
 template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (!MULTI && !LDA) {
+  if constexpr (!LDA) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
   using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA>;

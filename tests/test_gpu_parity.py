@@ -134,16 +134,19 @@ def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch):
 
 
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
-@pytest.mark.parametrize("MKN", [(390, 768, 656), (300, 640, 272), (64, 1024, 512), (1, 256, 96)])
+@pytest.mark.parametrize("MKN", [(390, 768, 656), (300, 640, 272), (64, 1024, 512), (1, 256, 96),
+                                 (300, 640, 272, (0, 256, 640))])
 def test_code_tiles_by_cp_async_or_tma_agree(MKN, bn, monkeypatch):
     """The GEMM from codes with the code tiles copied by cp.async loader warps
     and with every operand loaded by TMA: the oracle's result, identical bits,
-    DualScale and single-scale, ragged M, N and K tails."""
+    DualScale and single-scale, ragged M, N and K tails, one and two K segments."""
     import post_quantized_linear_b200 as pq
     from parity_util import compare_rows_single
     monkeypatch.setenv("SEGQUANT_BN", bn)
-    M, K, N = MKN
-    c = Case(W.small_case(M, K, N, seed=90 + M, out="bf16"))
+    M, K, N = MKN[:3]
+    kseg = list(MKN[3]) if len(MKN) > 3 else None
+    c = Case(W.small_case(M, K, N, seed=90 + M, out="bf16", kseg=kseg,
+                          x_sigmas=[1.0, 4.0] if kseg else None))
     qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
     c1 = pq.quantize_activations_single(c.x, c.wl.kseg, c.sp, c.sn)
     ys = {}
