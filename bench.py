@@ -40,7 +40,9 @@ INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
 # DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
-NCU_TRAFFIC_BYTES = {}
+NCU_TRAFFIC_BYTES = {
+    ("dit_xl2_fc2_cfg", "codes"): 80845568 + 5145856,   # dualscale_gemm_codes_kernel
+}
 
 
 def gemm_kernel_name(path: str, bits: int, x_dtype: str) -> str:
