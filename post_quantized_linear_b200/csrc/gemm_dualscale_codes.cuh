@@ -50,20 +50,41 @@ __host__ __device__ constexpr int codes_threads(int epw, bool lda) {
 // EPW_: epilogue warps (4, 8 or 16; a multiple of 4, each lane quarter of TMEM
 // read by EPW/4 warps splitting the tile's columns).  Four warps let narrow
 // tiles (BN = 32, 64, 96) store whole 32-column passes -- the small-M shapes.
+// KPS_: k blocks per pipeline stage (1 or 2).  With 2, one full barrier and
+// one tcgen05.commit serve two k blocks: the per-stage commit into the ring
+// costs the MMA issue stream a few hundred cycles when it comes every k block
+// (measured at BN = 128 and 192), much less every second one.  A unit (K
+// segment) may begin or end inside a stage.
+// Whether two stages of two k blocks fit (with the staging tiles the
+// configuration needs): the condition for KPS = 2.
+__host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf16, bool single,
+                                                   int epw) {
+  const int stage = 2 * ((single ? 1 : 2) * BM * BK + bn * BK);
+  const bool tma_y_forced = single || multi || epw != epi_warps(multi);
+  const int y_bytes = epw * stage_y_bytes(y_bf16);
+  return (kStageBudget - y_bytes) / stage >= 2 || (!tma_y_forced && kStageBudget / stage >= 2);
+}
+
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
-          bool LDA_ = false>
+          bool LDA_ = false, int KPS_ = 1>
 struct CodesCfg {
   static constexpr bool LDA = LDA_;
+  static constexpr int KPS = KPS_;
   // full barrier: the TMA thread's arrival (+ bytes), plus one per loader thread
   static constexpr int FULL_COUNT = 1 + (LDA_ ? kLoaderWarps * 32 : 0);
   static constexpr int BN = BN_;
   static constexpr int NACC = SINGLE ? 1 : 2;          // accumulators (code tiles) per unit
   static constexpr int A_BYTES = NACC * BM * BK;      // q+ and q- tiles, or the single code tile
   static constexpr int W_BYTES = BN * BK;
-  static constexpr int STAGE = A_BYTES + W_BYTES;
+  static constexpr int KB_BYTES = A_BYTES + W_BYTES;  // one k block of operands
+  static constexpr int STAGE = KPS * KB_BYTES;
   static constexpr int EPW = EPW_;
-  static constexpr int Y_BYTES = EPW * stage_y_bytes(Y_BF16);
+  // Y through TMA stores when two stages still fit beside the staging tiles
+  static constexpr bool TMA_Y = SINGLE || MULTI || EPW != epi_warps(MULTI) ||
+                                (kStageBudget - EPW * stage_y_bytes(Y_BF16)) / STAGE >= 2;
+  static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
+  static_assert(KPS == 1 || !LDA_, "two k blocks per stage: TMA loads");
   static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
@@ -78,14 +99,14 @@ struct CodesCfg {
 };
 
 template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false, int EPW = epi_warps(MULTI),
-          bool LDA = false>
+          bool LDA = false, int KPS = 1>
 __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA>;
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS>;
   constexpr int EPI0 = codes_epi_warp0(LDA);
   static_assert(EPW % 4 == 0 && (BN / (EPW / 4)) % 32 == 0, "32-column store passes per warp");
   static_assert(!MULTI || (BN == 128 && C::NBUF == 2), "several units per tile: BN = 128, two buffers");
@@ -142,19 +163,25 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
       for (int it = 0; it < rounds && ok; ++it) {
         Tile t;
         if (!tiles(it, t)) continue;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < num_kb; kb0 += KPS) {
           const int s = c % C::S;
           if (!(ok = wait1(smem_u32(empty + s), ((c / C::S) & 1) ^ 1, abort_flag, budget))) break;
-          uint8_t* st = smem + s * C::STAGE;
+          const int nk = min(KPS, num_kb - kb0);           // k blocks in this stage
           if constexpr (LDA) {
             mbar_arrive_expect_tx(smem_u32(full + s), C::W_BYTES);
           } else {
-            mbar_arrive_expect_tx(smem_u32(full + s), C::STAGE);
-            tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
-            if constexpr (!SINGLE)
-              tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
+            mbar_arrive_expect_tx(smem_u32(full + s), nk * C::KB_BYTES);
           }
-          tma_load_2d(smem_u32(st + C::A_BYTES), &tmap_w, smem_u32(full + s), kb * BK, t.n0);
+          for (int j = 0; j < nk; ++j) {
+            const int kb = kb0 + j;
+            uint8_t* st = smem + s * C::STAGE + j * C::KB_BYTES;
+            if constexpr (!LDA) {
+              tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
+              if constexpr (!SINGLE)
+                tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
+            }
+            tma_load_2d(smem_u32(st + C::A_BYTES), &tmap_w, smem_u32(full + s), kb * BK, t.n0);
+          }
           ++c;
         }
       }
@@ -172,36 +199,41 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
         const uint32_t idesc = idesc_i8(BM, t.width);
         bool unit_open = false;
         uint32_t d_pos = 0;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!unit_open) {
-            const int b = ug % C::NBUF;
-            if (!(ok = wait1(smem_u32(tmem_empty + b), ((ug / C::NBUF) & 1) ^ 1, abort_flag, budget))) break;
-            tc_fence_after();
-            d_pos = tmem_base + (uint32_t)(b * C::NACC * BN);
-          }
+        for (int kb0 = 0; kb0 < num_kb && ok; kb0 += KPS) {
           const int s = c % C::S;
           if (!(ok = wait1(smem_u32(full + s), (c / C::S) & 1, abort_flag, budget))) break;
           // code tiles written by cp.async (generic proxy) before the tensor core reads them
           if constexpr (LDA) fence_proxy_async_smem();
-          const uint32_t a_p = smem_u32(smem + s * C::STAGE);
-          const uint32_t a_n = a_p + BM * BK;
-          const uint32_t b_w = a_p + C::A_BYTES;
+          const int nk = min(KPS, num_kb - kb0);
+          for (int j = 0; j < nk; ++j) {
+            const int kb = kb0 + j;
+            if (!unit_open) {   // a unit (K segment) may start inside a stage
+              const int b = ug % C::NBUF;
+              if (!(ok = wait1(smem_u32(tmem_empty + b), ((ug / C::NBUF) & 1) ^ 1, abort_flag, budget))) break;
+              tc_fence_after();
+              d_pos = tmem_base + (uint32_t)(b * C::NACC * BN);
+            }
+            const uint32_t a_p = smem_u32(smem + s * C::STAGE + j * C::KB_BYTES);
+            const uint32_t a_n = a_p + BM * BK;
+            const uint32_t b_w = a_p + C::A_BYTES;
 #pragma unroll
-          for (int ks = 0; ks < BK / 32; ++ks) {
-            const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
-            const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
-            umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
-            if constexpr (!SINGLE)
-              umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
+            for (int ks = 0; ks < BK / 32; ++ks) {
+              const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
+              const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
+              umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
+              if constexpr (!SINGLE)
+                umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
+            }
+            unit_open = true;
+            if (kb_closes_unit(args, kb)) {
+              umma_commit(smem_u32(tmem_full + (ug % C::NBUF)));
+              ++ug;
+              unit_open = false;
+            }
           }
-          unit_open = true;
+          if (!ok) break;
           umma_commit(smem_u32(empty + s));
           ++c;
-          if (kb_closes_unit(args, kb)) {
-            umma_commit(smem_u32(tmem_full + (ug % C::NBUF)));
-            ++ug;
-            unit_open = false;
-          }
         }
       }
       // All MMAs this thread issued have landed once the drain barrier flips.
@@ -252,10 +284,17 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
     const int quad = warp & 3;
     const int part = (warp - EPI0) >> 2;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-    epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
-        args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
-        tiles, abort_flag, budget);
+    if constexpr (C::TMA_Y) {
+      uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
+      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
+          args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
+          tiles, abort_flag, budget);
+    } else {
+      // no room for staging tiles: 16-byte stores straight from registers (DualScale, one unit)
+      epilogue_role<BN, C::NBUF, false, false, Y_BF16, false>(
+          args, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), /*empty_remote=*/false,
+          /*row_shift=*/0, rounds, tiles, abort_flag, budget);
+    }
   }
 
   // ---------------------------------------------------------------- teardown

@@ -233,14 +233,25 @@ bool use_codes_lda() {
 }
 
 
-template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false>
+// k blocks per pipeline stage of the GEMM from codes (2 for TMA loads at
+// BN <= 192, where two such stages fit; 1 otherwise); SEGQUANT_KPS=1 forces one.
+int codes_kps() {
+  if (const char* e = std::getenv("SEGQUANT_KPS")) return std::atoi(e) == 2 ? 2 : 1;
+  return 2;
+}
+
+template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false,
+          int KPS = 1>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (!LDA) {
+  if constexpr (!LDA && KPS == 1) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
-  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA>;
-  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA>;
+  if constexpr (!LDA && KPS == 1 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
+    if (codes_kps() == 2) return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
+  }
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS>;
+  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);

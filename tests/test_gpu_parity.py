@@ -162,6 +162,37 @@ def test_code_tiles_by_cp_async_or_tma_agree(MKN, bn, monkeypatch):
         assert torch.equal(ys["1"][i].view(torch.int16), ys["0"][i].view(torch.int16))
 
 
+@pytest.mark.parametrize("bn", ["128", "192"])
+@pytest.mark.parametrize("MKN", [(390, 640, 656), (300, 1040, 272), (129, 768, 400), (64, 3072, 1024),
+                                 (300, 640, 272, (0, 256, 640)),
+                                 (257, 1040, 256, (0, 128, 512, 1040))])
+def test_two_k_blocks_per_stage_agree(MKN, bn, monkeypatch):
+    """The GEMM from codes with two k blocks per pipeline stage (one commit per
+    stage; odd k-block counts end in a half stage; K tails; K segments that
+    begin or end inside a stage) against the oracle and bit-identical to one k
+    block per stage, DualScale and single-scale."""
+    import post_quantized_linear_b200 as pq
+    from parity_util import compare_rows_single
+    monkeypatch.setenv("SEGQUANT_BN", bn)
+    M, K, N = MKN[:3]
+    kseg = list(MKN[3]) if len(MKN) > 3 else None
+    sig = [1.0 + 2.0 * j for j in range(len(kseg) - 1)] if kseg else None
+    c = Case(W.small_case(M, K, N, seed=110 + M, out="bf16", kseg=kseg, x_sigmas=sig))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    c1 = pq.quantize_activations_single(c.x, c.wl.kseg, c.sp, c.sn)
+    ys = {}
+    for kps in ("2", "1"):
+        monkeypatch.setenv("SEGQUANT_KPS", kps)
+        ys[kps] = (pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b),
+                   pq.linear_from_single(c1, c.qw, c.sp, c.sn, c.b))
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(ys["2"][0], np.arange(M))
+    compare_rows_single(c, ys["2"][1], np.arange(M))
+    for i in range(2):
+        assert torch.equal(ys["2"][i].view(torch.int16), ys["1"][i].view(torch.int16))
+
+
 def test_forward_exact_in_fp32():
     """With the fp32 epilogue order the kernel reproduces the oracle bit for bit."""
     c = Case(_small(1))
