@@ -41,7 +41,7 @@ INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
-    ("dit_xl2_fc2_cfg", "codes"): 80845568 + 5145856,   # dualscale_gemm_codes_kernel
+    ("dit_xl2_fc2_cfg", "codes"): 80836352 + 7128320,   # dualscale_gemm_codes_kernel
 }
 
 
