@@ -41,7 +41,7 @@ INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
-    ("dit_xl2_fc2_cfg", "codes"): 80836352 + 7128320,   # dualscale_gemm_codes_kernel
+    ("dit_xl2_fc2_cfg", "codes"): 93068032 + 11148288,   # dualscale_gemm_codes_kernel
 }
 
 
@@ -73,6 +73,9 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-small-m", action="store_true",
                     help="skip the small-M (M <= 128, HBM-bound) measurements")
+    ap.add_argument("--small-m-only", action="store_true",
+                    help="run only the small-M measurements (one GPU) and print them as one "
+                         "JSON line; not a bench line")
     return ap.parse_args()
 
 
@@ -107,13 +110,21 @@ class L2Flush:
 # ------------------------------------------------------------------ small M
 SMALL_M_SHAPES = ((3072, 12288), (4608, 1152))
 SMALL_M_ROWS = (16, 64, 128)
+SMALL_M_LAYERS = 8     # distinct weight copies of the layer-stream measurement
 
 
 def small_m_measure(dev, flush, steps: int, hbm_peak: float):
     """HBM-bound small-M forwards (one K segment, int8 weights, bf16 out): the
     split-K GEMM from codes and the one-pass GEMM from codes, each replayed
     from a CUDA graph with the L2 flushed before every launch.  Bytes = weight
-    codes + weight scales + q+/q- codes + Y (the algorithmic traffic)."""
+    codes + weight scales + q+/q- codes + Y (the algorithmic traffic).
+
+    `one_pass_layers`: the one-pass GEMM over SMALL_M_LAYERS distinct copies
+    of the weight, back to back in one graph (a stack of layers, each reading
+    its own cold weight: 8 x 37.7 MB exceeds the L2), the L2 flushed before
+    every replay; time per layer = replay time / layers.  This spreads the
+    replay's fixed launch cost (several microseconds, and the event clock here
+    advances in 2.048-microsecond steps) over the layers, as in a model."""
     import torch
     import post_quantized_linear_b200 as pq
     from synth import workloads as W
@@ -150,6 +161,32 @@ def small_m_measure(dev, flush, steps: int, hbm_peak: float):
                 res[name] = {"us": us, "gbs": byts / (us * 1e-6) / 1e9,
                              "frac_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
                 del g
+            qws = [qw] + [pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=8)
+                          for _ in range(SMALL_M_LAYERS - 1)]
+            ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in qws]
+
+            def layers():
+                for q_l, y_l in zip(qws, ys):
+                    pq.linear_from_codes(qp, qn, q_l, sp, sn, out=y_l)
+            layers()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                layers()
+            ts = []
+            for i in range(max(steps, 5)):
+                flush(i)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            us = statistics.median(ts) * 1e3 / len(qws)
+            res["one_pass_layers"] = {"layers": len(qws), "us_per_layer": us,
+                                      "gbs": byts / (us * 1e-6) / 1e9,
+                                      "frac_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
+            del g, qws, ys
             out.append(res)
     return out
 
@@ -327,6 +364,13 @@ def run_ours(args):
 
     import post_quantized_linear_b200 as pq
     from synth import workloads as W
+
+    if args.small_m_only:
+        dev = torch.device("cuda", local)
+        hbm_peak = peaks()[1]
+        print(json.dumps({"small_m": {"peak_gbs": hbm_peak, "cases": small_m_measure(
+            dev, L2Flush(dev), args.steps, hbm_peak)}}), flush=True)
+        return 0
 
     wl = W.WORKLOADS[args.workload]
     import dataclasses
@@ -545,8 +589,10 @@ def run_ours(args):
                            "d2h_bytes_per_step": e2e["bo"]}
         if world == 1 and not args.no_small_m:
             line["small_m"] = {
-                "note": "HBM-bound forwards at M <= 128 (median of L2-flushed graph replays); "
-                        "bytes = weight codes + scales + q+/q- codes + Y; peak = measured HBM copy",
+                "note": "HBM-bound forwards at M <= 128 (median of L2-flushed graph replays; "
+                        "one_pass_layers: per layer of 8 back-to-back layers with distinct "
+                        "weights); bytes = weight codes + scales + q+/q- codes + Y; peak = "
+                        "measured HBM copy",
                 "peak_gbs": hbm_peak,
                 "cases": small_m_measure(dev, flush, args.steps, hbm_peak)}
         if world == 1 and not args.no_cpu_baseline:

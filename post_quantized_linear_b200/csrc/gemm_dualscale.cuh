@@ -92,6 +92,11 @@ struct GemmArgs {
   const int8_t* a_pos;     // q+ (or the single code) [M][lda]
   const int8_t* a_neg;     // q- [M][lda]
   int64_t lda;
+  // Rows of one code-tile TMA box (GEMM from codes): BM, or M rounded up to 16
+  // when a single row tile holds fewer than BM rows (0 means BM).  The rows
+  // past the box keep stale shared memory; their accumulator lanes are never
+  // stored.
+  int32_t a_rows;
 };
 
 // Teardown waits (copies and MMAs that were issued always complete) get a

@@ -158,6 +158,9 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
       if constexpr (!SINGLE) tma_prefetch_desc(&tmap_qn);
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_y);
+      // bytes one k block brings: the code boxes (a_rows rows each) + the weight box
+      const uint32_t kb_tx =
+          (uint32_t)(C::NACC * (args.a_rows > 0 ? args.a_rows : BM) * BK + C::W_BYTES);
       int c = 0;
       bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
           if constexpr (LDA) {
             mbar_arrive_expect_tx(smem_u32(full + s), C::W_BYTES);
           } else {
-            mbar_arrive_expect_tx(smem_u32(full + s), nk * C::KB_BYTES);
+            mbar_arrive_expect_tx(smem_u32(full + s), (uint32_t)nk * kb_tx);
           }
           for (int j = 0; j < nk; ++j) {
             const int kb = kb0 + j;

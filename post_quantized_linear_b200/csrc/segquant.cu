@@ -273,6 +273,14 @@ sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMa
                 : launch_codes<BN, false, MULTI, SINGLE, EPW>(tqp, tqn, tw, ty, a, stream);
 }
 
+// Whether 256-wide tiles of the GEMM from codes drain TMEM with 16 epilogue
+// warps instead of 8 (one TMEM buffer at that width: the MMA waits for the
+// drain); SEGQUANT_EPW16=0|1 overrides the default.
+bool codes_wide_epilogue() {
+  if (const char* e = std::getenv("SEGQUANT_EPW16")) return std::atoi(e) != 0;
+  return true;
+}
+
 // Small M (one row tile): the work is streaming the weight codes, so the tile
 // width spreads N over as many SMs as possible.  Candidates 32..256 (multiples
 // of 32, four epilogue warps); cost = waves x cycles per MMA, where an M = 128
@@ -450,10 +458,13 @@ bool use_pair(int64_t N, bool w4) {
 // caps BN at 128; fp32 activation stages leave room for BN = 128 only.
 // Otherwise BN in {128, 192, 256} minimises a makespan model of the snake
 // schedule: the busiest CTA's tile columns divided by the measured per-column
-// efficiency of that width (narrow tiles keep less work in flight per byte of
-// pipeline), with the last, narrower tile costing a full one.
+// efficiency of that width.  Two calibrations, each measured on B200:
+//  * the GEMM from codes (one stage ring, two k blocks per stage, 16 epilogue
+//    warps at BN = 256): 0.70, 0.79, 0.90, and the last, narrower tile column
+//    costs its own width (full tiles are scheduled first);
+//  * the other kernels: 0.55, 0.70, 0.81, and the last tile costs a full one.
 // SEGQUANT_BN=128|192|256 overrides the choice (a tuning knob).
-int choose_bn(int64_t M, int64_t N, bool multi, bool f32x) {
+int choose_bn(int64_t M, int64_t N, bool multi, bool f32x, bool codes_ring) {
   if (multi || f32x) return 128;
   if (const char* e = std::getenv("SEGQUANT_BN")) {
     const int v = std::atoi(e);
@@ -464,15 +475,19 @@ int choose_bn(int64_t M, int64_t N, bool multi, bool f32x) {
   std::vector<double> load(sms);
   auto cost = [&](int64_t bn, double eff) {
     std::fill(load.begin(), load.end(), 0.0);
-    const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
+    const int64_t n_full = N / bn, tail = N % bn;
+    const int64_t full_tiles = m_tiles * n_full;
+    const int64_t tiles = full_tiles + (tail ? m_tiles : 0);
     for (int64_t idx = 0; idx < tiles; ++idx) {
       const int64_t it = idx / sms, pos = idx % sms;
       const int64_t cta = (it & 1) ? sms - 1 - pos : pos;
-      load[cta] += (double)bn / eff;
+      load[cta] += (double)(idx < full_tiles || !codes_ring ? bn : tail) / eff;
     }
     return *std::max_element(load.begin(), load.end());
   };
-  const double c128 = cost(128, 0.55), c192 = cost(192, 0.70), c256 = cost(256, 0.81);
+  const double c128 = cost(128, codes_ring ? 0.70 : 0.55);
+  const double c192 = cost(192, codes_ring ? 0.79 : 0.70);
+  const double c256 = cost(256, codes_ring ? 0.90 : 0.81);
   if (c256 <= c192 && c256 <= c128) return 256;
   return c192 <= c128 ? 192 : 128;
 }
@@ -575,7 +590,8 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const bool multi = w4 || kseg.count > 1;
   const bool f32x = (src == ASource::X && xt == SQ_F32);
   const bool pair = (src == ASource::Codes) && use_pair(N, w4);
-  int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x);
+  const bool codes_ring = (src == ASource::Codes) && !w4 && !pair && acc == nullptr && use_codes_ring();
+  int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x, codes_ring);
   // one row tile, one unit per tile, GEMM from codes: narrow tiles over all SMs
   const int bn_small = (!multi && acc == nullptr && (src == ASource::Codes || src == ASource::Single) &&
                         !(src == ASource::Codes && use_pair(N, w4)) && use_codes_ring())
@@ -585,6 +601,10 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     BN = 256;
     if (const char* e = std::getenv("SEGQUANT_BN")) BN = std::atoi(e) == 128 ? 128 : 256;
   }
+  // One row tile of fewer than BM rows, read by the GEMM from codes: code boxes
+  // of M rows rounded up to 16 instead of mostly out-of-bounds 128-row boxes.
+  const bool codes_kernel = (src == ASource::Single) || (codes_ring && !w4);
+  const int a_rows = (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
   CUtensorMap ta, ta2, tw;
   if (src == ASource::X) {
     const int xe = elt_size(xt);
@@ -594,11 +614,11 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     ta2 = ta;
   } else {
     st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
-                   (uint64_t)ldq, 128, sq::BM);
+                   (uint64_t)ldq, 128, (uint32_t)a_rows);
     if (st != SQ_OK) return st;
     if (src == ASource::Codes) {
       st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
-                     (uint64_t)ldq, 128, sq::BM);
+                     (uint64_t)ldq, 128, (uint32_t)a_rows);
       if (st != SQ_OK) return st;
     } else {
       ta2 = ta;
@@ -632,6 +652,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   a.a_pos = q_pos;
   a.a_neg = q_neg;
   a.lda = ldq;
+  a.a_rows = a_rows;
 
   using bf = __nv_bfloat16;
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
@@ -666,6 +687,8 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       if (st != SQ_OK) return st;
       if (multi) return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
       if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
+      if (BN == 256 && codes_wide_epilogue())
+        return launch_codes_out<256, false, false, 16>(yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, ty, a, stream);
       if (BN == 192) return launch_codes_out<192, false>(yb, ta, ta2, tw, ty, a, stream);
       return launch_codes_out<128, false>(yb, ta, ta2, tw, ty, a, stream);

@@ -193,6 +193,57 @@ def test_two_k_blocks_per_stage_agree(MKN, bn, monkeypatch):
         assert torch.equal(ys["2"][i].view(torch.int16), ys["1"][i].view(torch.int16))
 
 
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_wide_tiles_with_sixteen_epilogue_warps_agree(out, monkeypatch):
+    """256-wide tiles drained by 16 epilogue warps: the oracle's result and the
+    same bits as with 8 warps (ragged M, N tail)."""
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_BN", "256")
+    c = Case(W.small_case(390, 768, 656, seed=77, out=out))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    ys = {}
+    for e in ("1", "0"):
+        monkeypatch.setenv("SEGQUANT_EPW16", e)
+        ys[e] = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(ys["1"], np.arange(c.wl.M))
+    iv = torch.int16 if out == "bf16" else torch.int32
+    assert torch.equal(ys["1"].view(iv), ys["0"].view(iv))
+
+
+@pytest.mark.parametrize("kseg", [None, (0, 256, 640)])
+@pytest.mark.parametrize("M", [1, 17, 48, 100, 127])
+def test_code_boxes_sized_to_a_short_row_tile(M, kseg, monkeypatch):
+    """Fewer than 128 rows: the GEMM from codes loads code boxes of M rows
+    rounded up to 16 and the MMA's other rows read stale shared memory.  Every
+    row against the oracle (DualScale and single-scale, one and two K
+    segments), and the same bits as the fused forward (which quantizes from X)
+    at every narrow tile width."""
+    import post_quantized_linear_b200 as pq
+    from parity_util import compare_rows_single
+    K = 640 if kseg else 1024
+    c = Case(W.small_case(M, K, 272, seed=170 + M, out="bf16", kseg=list(kseg) if kseg else None,
+                          x_sigmas=[1.0, 4.0] if kseg else None))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    c1 = pq.quantize_activations_single(c.x, c.wl.kseg, c.sp, c.sn)
+    yf = c.forward()
+    res = {}
+    for bn in ("32", "96", "-1"):
+        monkeypatch.setenv("SEGQUANT_BN_SMALL", bn)
+        res[bn] = (pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b),
+                   pq.linear_from_single(c1, c.qw, c.sp, c.sn, c.b))
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    y, ys = res["-1"]
+    c.compare_rows(y, np.arange(M))
+    compare_rows_single(c, ys, np.arange(M))
+    assert torch.equal(y.view(torch.int16), yf.view(torch.int16))
+    for (yd, yds) in res.values():
+        assert torch.equal(yd.view(torch.int16), y.view(torch.int16))
+        assert torch.equal(yds.view(torch.int16), ys.view(torch.int16))
+
+
 def test_forward_exact_in_fp32():
     """With the fp32 epilogue order the kernel reproduces the oracle bit for bit."""
     c = Case(_small(1))
