@@ -42,6 +42,7 @@ INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
     ("dit_xl2_fc2_cfg", "codes"): 93068032 + 11148288,   # dualscale_gemm_codes_kernel
+    ("w4a8", "codes"): 105879296 + 71072768,             # dualscale_gemm_codes_kernel (W4)
 }
 
 

@@ -13,6 +13,14 @@ constexpr int SQ_MAX_SEG = 16;
 constexpr float kMagic = 12582912.0f;
 constexpr uint32_t kMagicBits = 0x4B400000u;
 
+// 1.5 * 2^19, whose fp32 unit in the last place is 2^-4: an int32 accumulator
+// seeded with these bits and fed weights scaled by 16 (int4 codes unpacked
+// into the high nibble of each byte) holds the bits of 1.5 * 2^19 + acc, exact
+// while |acc| < 2^18 (a 128-wide group of int8 x int4 products: |acc| <=
+// 128 * 127 * 8).
+constexpr float kMagicW4 = 786432.0f;
+constexpr uint32_t kMagicW4Bits = 0x49400000u;
+
 // Bits of the per-device status word.
 constexpr unsigned int SQ_STATUS_TIMEOUT = 1u;
 constexpr unsigned int SQ_STATUS_RANGE = 2u;

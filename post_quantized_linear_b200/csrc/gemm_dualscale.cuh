@@ -335,6 +335,15 @@ __device__ __forceinline__ uint2 unpack8_int4(uint32_t w) {
   return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
+// Eight int4 codes (two per byte, low nibble = even k) -> eight int8 bytes
+// holding 16 x the code: each nibble moved to the high half of its byte, whose
+// sign bit it then carries (used with the 1.5 * 2^19 accumulator seed).
+__device__ __forceinline__ uint2 unpack8_int4_x16(uint32_t w) {
+  const uint32_t even = (w << 4) & 0xF0F0F0F0u;
+  const uint32_t odd = w & 0xF0F0F0F0u;
+  return make_uint2(__byte_perm(even, odd, 0x5140), __byte_perm(even, odd, 0x7362));
+}
+
 __device__ __forceinline__ float rcp_or_zero(float s) { return s > 0.0f ? __frcp_rn(s) : 0.0f; }
 
 // Per-segment constants of the fused quantizer.
@@ -525,8 +534,9 @@ __device__ __forceinline__ void prefetch_wscales(const GemmArgs& a, int u, int j
 // 1.5*2^23 + acc (|acc| < 2^22), and one subtraction gives F(acc) exactly.
 // Same fp32 operations as fold8, two outputs per packed f32x2 instruction.
 __device__ __forceinline__ void fold8_seeded(const uint32_t (&ap)[8], const uint32_t (&an)[8],
-                                             const float (&sw)[8], float sp, float sn, float* y) {
-  const uint64_t m2 = f2_pack(-kMagic, -kMagic);
+                                             const float (&sw)[8], float sp, float sn, float* y,
+                                             float magic = kMagic) {
+  const uint64_t m2 = f2_pack(-magic, -magic);
   const uint64_t sp2 = f2_pack(sp, sp), sn2 = f2_pack(sn, sn);
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
@@ -853,7 +863,13 @@ __device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float&
 // registers (HALF == 32), stored once per tile; otherwise one unit per tile,
 // streamed out in 32-column passes with the accumulators released after the
 // warp's last TMEM load.
-template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn>
+// SEEDED (int4 weights unpacked as 16 x the code, one unit per 128-wide
+// group): the accumulators hold the bits of 1.5 * 2^19 + acc (kMagicW4Bits
+// plus 16 * acc).  The warps seed their columns of both buffers before the
+// first unit and again right after reading them, so F(acc) is one exact
+// subtraction; the group's fp16 weight scales and its segment's s+/s- enter
+// the same fp32 order as the other units.
+template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, bool SEEDED, class TileFn>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
@@ -864,9 +880,10 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
   constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
   static_assert(HALF % 32 == 0, "32-column store passes");
   static_assert(!MULTI || HALF == 32, "several units: one 32-column pass per warp");
+  static_assert(!SEEDED || (MULTI && NACC == 2), "seeded accumulators: int4 groups, DualScale");
   uint8_t* srow = stage_y + lane * ROWB;
   const uint32_t sbase = smem_u32(stage_y);
-  const int units = args.kseg.count;
+  const int units = SEEDED ? args.num_kb : args.kseg.count;
   auto release = [&](int b) {
     tc_fence_before();
     __syncwarp();
@@ -893,17 +910,61 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       fold16_single(ac, sw, fmaxf(sp, sn), o);
     }
   };
+  // Seeded (int4) unit: 16 columns at tile column cc of buffer b folded into
+  // y (fp32 pairs per eight columns), the columns re-seeded as soon as they
+  // are read.
+  auto fold_seeded = [&](int b, int cc, int u, int j, const Tile& t, float* y) {
+    const uint32_t tcol = (uint32_t)b * BUF_COLS + (uint32_t)cc;
+    float sp, sn;
+    unit_act_scales(args, j, sp, sn);
+    uint32_t ap[16], an[16];
+    tmem_ld16(t_lane + tcol, ap);
+    tmem_ld16(t_lane + tcol + BN, an);
+    tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 16; h += 8) {
+      tmem_st8(t_lane + tcol + h, kMagicW4Bits);
+      tmem_st8(t_lane + tcol + BN + h, kMagicW4Bits);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {   // scales eight columns at a time (registers)
+      float sw8[8];
+      load_wscales8(args, u, j, t.n0 + cc + 8 * h, sw8);
+      fold8_seeded(*reinterpret_cast<const uint32_t(*)[8]>(ap + 8 * h),
+                   *reinterpret_cast<const uint32_t(*)[8]>(an + 8 * h), sw8, sp, sn, y + 8 * h,
+                   kMagicW4);
+    }
+  };
   int ug = 0;
   bool ok = true, pending = false;
+  if constexpr (SEEDED) {
+    // Seed this warp's columns of both buffers, then hand the buffers to the MMA.
+#pragma unroll
+    for (int b = 0; b < NBUF; ++b) {
+#pragma unroll
+      for (int c = 0; c < HALF; c += 8) {
+        const uint32_t col = (uint32_t)b * BUF_COLS + (uint32_t)(part * HALF + c);
+        tmem_st8(t_lane + col, kMagicW4Bits);
+        tmem_st8(t_lane + col + BN, kMagicW4Bits);
+      }
+    }
+    tmem_wait_st();
+    for (int b = 0; b < NBUF; ++b) release(b);
+  }
   for (int it = 0; it < rounds && ok; ++it) {
     Tile t;
     if (!tile_fn(it, t)) continue;
     const int c_lo = part * HALF;
     const int cols = min(HALF, t.width - c_lo);   // may be <= 0 on a narrow tail tile
     if (cols > 0) {
-      for (int u = 0; u < units; ++u) {
-        const float* sw_row = static_cast<const float*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo;
-        for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
+      if constexpr (SEEDED) {   // fp16 scales [G][N]: 64 bytes per group for 32 columns
+        for (int u = lane; u < units; u += 32)
+          prefetch_l1(static_cast<const __half*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo);
+      } else {
+        for (int u = 0; u < units; ++u) {
+          const float* sw_row = static_cast<const float*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo;
+          for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
+        }
       }
       if (args.bias != nullptr)
         for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(args.bias + t.n0 + c_lo + c);
@@ -913,16 +974,32 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       float y[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) y[i] = 0.0f;
-      for (int u = 0; u < units; ++u) {
-        const int b = ug % NBUF;
-        if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
-        tc_fence_after();
-        if (npass > 0) {
-          fold(b, c_lo, u, t, y);
-          if (c_lo + 16 < t.width) fold(b, c_lo + 16, u, t, y + 16);
+      if constexpr (SEEDED) {
+        for (int u = 0; u < units; ++u) {
+          const int b = ug % NBUF;
+          if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+          tc_fence_after();
+          if (npass > 0) {
+            const int j = args.kseg.segment_of(u * BK);
+            fold_seeded(b, c_lo, u, j, t, y);
+            if (c_lo + 16 < t.width) fold_seeded(b, c_lo + 16, u, j, t, y + 16);
+          }
+          tmem_wait_st();
+          release(b);
+          ++ug;
         }
-        release(b);
-        ++ug;
+      } else {
+        for (int u = 0; u < units; ++u) {
+          const int b = ug % NBUF;
+          if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+          tc_fence_after();
+          if (npass > 0) {
+            fold(b, c_lo, u, t, y);
+            if (c_lo + 16 < t.width) fold(b, c_lo + 16, u, t, y + 16);
+          }
+          release(b);
+          ++ug;
+        }
       }
       if (!ok) break;
       if (npass > 0) {

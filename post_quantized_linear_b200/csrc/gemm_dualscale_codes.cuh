@@ -20,6 +20,12 @@
 // Stage sizes: (2 or 1) x 16 KiB of codes + BN x 128 bytes of weights, as many
 // as fit in 224 KiB next to the epilogue's staging tiles (2 or 4 KiB per
 // epilogue warp for bf16 or fp32 Y).
+// W4: int4 weights with one scale per 128-wide group along K (the SegQuant
+// paper's W4A8 setting): TMA brings the packed tile (BN rows of 64 bytes) into
+// the stage, two unpack warps widen it to int8 in the 128-byte-swizzled
+// layout beside it and signal a per-stage ready barrier that the MMA waits
+// on; every k block is its own unit, folded by the epilogue from seeded
+// accumulators (epilogue_tma_store, SEEDED).
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -40,11 +46,14 @@ __host__ __device__ constexpr int codes_threads_epw(int epw) { return (kCodesEpi
 // two code tiles plus a weight tile per k block need at the int8 MMA rate),
 // measured slower than all-TMA loads on the DiT and MMDiT shapes.
 constexpr int kLoaderWarps = 4;
-__host__ __device__ constexpr int codes_epi_warp0(bool lda) {
-  return lda ? kCodesEpiWarp0 + kLoaderWarps : kCodesEpiWarp0;
+// W4: two int4 unpack warps in the slots after warp 1 (two, not four: with 16
+// epilogue warps a block of 20 warps leaves each thread about 96 registers).
+constexpr int kUnpackWarps = 2;
+__host__ __device__ constexpr int codes_epi_warp0(bool lda, bool w4 = false) {
+  return kCodesEpiWarp0 + (lda ? kLoaderWarps : 0) + (w4 ? kUnpackWarps : 0);
 }
-__host__ __device__ constexpr int codes_threads(int epw, bool lda) {
-  return (codes_epi_warp0(lda) + epw) * 32;
+__host__ __device__ constexpr int codes_threads(int epw, bool lda, bool w4 = false) {
+  return (codes_epi_warp0(lda, w4) + epw) * 32;
 }
 
 // EPW_: epilogue warps (4, 8 or 16; a multiple of 4, each lane quarter of TMEM
@@ -66,7 +75,7 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 }
 
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
-          bool LDA_ = false, int KPS_ = 1>
+          bool LDA_ = false, int KPS_ = 1, bool W4_ = false>
 struct CodesCfg {
   static constexpr bool LDA = LDA_;
   static constexpr int KPS = KPS_;
@@ -76,7 +85,8 @@ struct CodesCfg {
   static constexpr int NACC = SINGLE ? 1 : 2;          // accumulators (code tiles) per unit
   static constexpr int A_BYTES = NACC * BM * BK;      // q+ and q- tiles, or the single code tile
   static constexpr int W_BYTES = BN * BK;
-  static constexpr int KB_BYTES = A_BYTES + W_BYTES;  // one k block of operands
+  static constexpr int WP_BYTES = W4_ ? BN * (BK / 2) : 0;   // packed int4 rows of 64 bytes
+  static constexpr int KB_BYTES = A_BYTES + W_BYTES + WP_BYTES;  // one k block of operands
   static constexpr int STAGE = KPS * KB_BYTES;
   static constexpr int EPW = EPW_;
   // Y through TMA stores when two stages still fit beside the staging tiles
@@ -85,10 +95,13 @@ struct CodesCfg {
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
   static_assert(KPS == 1 || !LDA_, "two k blocks per stage: TMA loads");
+  static_assert(!W4_ || (MULTI && !SINGLE && !LDA_ && KPS_ == 1 && BN_ == 128),
+                "int4 weights: DualScale, one k block per stage, BN = 128");
   static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
-  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1;  // full, empty; tmem full/empty; drain
+  // full, empty; tmem full/empty; drain; (W4) unpacked
+  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = NACC * BN * NBUF;
@@ -99,15 +112,15 @@ struct CodesCfg {
 };
 
 template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false, int EPW = epi_warps(MULTI),
-          bool LDA = false, int KPS = 1>
-__global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
+          bool LDA = false, int KPS = 1, bool W4 = false>
+__global__ void __launch_bounds__(codes_threads(EPW, LDA, W4), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS>;
-  constexpr int EPI0 = codes_epi_warp0(LDA);
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, W4>;
+  constexpr int EPI0 = codes_epi_warp0(LDA, W4);
   static_assert(EPW % 4 == 0 && (BN / (EPW / 4)) % 32 == 0, "32-column store passes per warp");
   static_assert(!MULTI || (BN == 128 && C::NBUF == 2), "several units per tile: BN = 128, two buffers");
   extern __shared__ uint8_t smem_raw[];
@@ -119,6 +132,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
   uint64_t* tmem_full = empty + 8;        // [2]
   uint64_t* tmem_empty = tmem_full + 2;   // [2]
   uint64_t* drain_bar = tmem_empty + 2;
+  uint64_t* ready = drain_bar + 1;        // [8] (W4) int4 tile unpacked
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -136,6 +150,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
       mbar_init(smem_u32(tmem_empty + i), C::EPW);
     }
     mbar_init(smem_u32(drain_bar), 1);
+    if constexpr (W4)
+      for (int i = 0; i < C::S; ++i) mbar_init(smem_u32(ready + i), kUnpackWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -159,8 +175,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_y);
       // bytes one k block brings: the code boxes (a_rows rows each) + the weight box
-      const uint32_t kb_tx =
-          (uint32_t)(C::NACC * (args.a_rows > 0 ? args.a_rows : BM) * BK + C::W_BYTES);
+      const uint32_t kb_tx = (uint32_t)(C::NACC * (args.a_rows > 0 ? args.a_rows : BM) * BK +
+                                        (W4 ? C::WP_BYTES : C::W_BYTES));
       int c = 0;
       bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
@@ -183,7 +199,11 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
               if constexpr (!SINGLE)
                 tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
             }
-            tma_load_2d(smem_u32(st + C::A_BYTES), &tmap_w, smem_u32(full + s), kb * BK, t.n0);
+            if constexpr (W4)   // packed rows land after the unpacked tile's place
+              tma_load_2d(smem_u32(st + C::A_BYTES + C::W_BYTES), &tmap_w, smem_u32(full + s),
+                          kb * (BK / 2), t.n0);
+            else
+              tma_load_2d(smem_u32(st + C::A_BYTES), &tmap_w, smem_u32(full + s), kb * BK, t.n0);
           }
           ++c;
         }
@@ -204,15 +224,20 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
         uint32_t d_pos = 0;
         for (int kb0 = 0; kb0 < num_kb && ok; kb0 += KPS) {
           const int s = c % C::S;
-          if (!(ok = wait1(smem_u32(full + s), (c / C::S) & 1, abort_flag, budget))) break;
-          // code tiles written by cp.async (generic proxy) before the tensor core reads them
-          if constexpr (LDA) fence_proxy_async_smem();
+          // W4: the unpack warps' ready barrier (it follows the stage's full barrier)
+          if (!(ok = wait1(smem_u32((W4 ? ready : full) + s), (c / C::S) & 1, abort_flag, budget))) break;
+          // tiles written by cp.async or by the unpack warps (generic proxy)
+          // before the tensor core reads them
+          if constexpr (LDA || W4) fence_proxy_async_smem();
           const int nk = min(KPS, num_kb - kb0);
           for (int j = 0; j < nk; ++j) {
             const int kb = kb0 + j;
             if (!unit_open) {   // a unit (K segment) may start inside a stage
               const int b = ug % C::NBUF;
-              if (!(ok = wait1(smem_u32(tmem_empty + b), ((ug / C::NBUF) & 1) ^ 1, abort_flag, budget))) break;
+              // seeded (W4) buffers: the epilogue's first release (after seeding)
+              // completes phase 0, so every use waits one phase later
+              const uint32_t par = W4 ? ((ug / C::NBUF) & 1) : (((ug / C::NBUF) & 1) ^ 1);
+              if (!(ok = wait1(smem_u32(tmem_empty + b), par, abort_flag, budget))) break;
               tc_fence_after();
               d_pos = tmem_base + (uint32_t)(b * C::NACC * BN);
             }
@@ -221,7 +246,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
             const uint32_t b_w = a_p + C::A_BYTES;
 #pragma unroll
             for (int ks = 0; ks < BK / 32; ++ks) {
-              const uint32_t acc = (unit_open || ks > 0) ? 1u : 0u;
+              const uint32_t acc = (W4 || unit_open || ks > 0) ? 1u : 0u;
               const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
               umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
               if constexpr (!SINGLE)
@@ -279,6 +304,41 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
       }
       // every copy of this thread has landed before the CTA can exit
       asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if constexpr (W4) {
+      // int4 unpack: thread t widens 16-byte pieces task = i*64 + t of the
+      // packed tile (row n = task / 4, quarter q = task % 4: 32 codes, low
+      // nibble first) into two 16-byte chunks of the int8 row at their
+      // 128-byte-swizzle positions, each byte 16 x its code (the epilogue's
+      // accumulator seed accounts for the factor).
+      const int t_id = threadIdx.x - kCodesEpiWarp0 * 32;   // 0..63
+      int c = 0;
+      bool ok = (args.starve == 0);
+      for (int it = 0; it < rounds && ok; ++it) {
+        Tile t;
+        if (!tiles(it, t)) continue;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          const int s = c % C::S;
+          if (!(ok = wait_warp(smem_u32(full + s), (c / C::S) & 1, abort_flag, budget))) break;
+          uint8_t* st = smem + s * C::STAGE;
+          const uint8_t* src = st + C::A_BYTES + C::W_BYTES;
+          uint8_t* dst = st + C::A_BYTES;
+#pragma unroll
+          for (int i = 0; i < (BN * 4) / (kUnpackWarps * 32); ++i) {
+            const int task = i * (kUnpackWarps * 32) + t_id;
+            const int n = task >> 2, q = task & 3;
+            const uint4 pk = *reinterpret_cast<const uint4*>(src + n * 64 + q * 16);
+            const uint2 e0 = unpack8_int4_x16(pk.x), e1 = unpack8_int4_x16(pk.y);
+            const uint2 e2 = unpack8_int4_x16(pk.z), e3 = unpack8_int4_x16(pk.w);
+            uint8_t* drow = dst + n * 128;
+            *reinterpret_cast<uint4*>(drow + (((2 * q) ^ (n & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+            *reinterpret_cast<uint4*>(drow + (((2 * q + 1) ^ (n & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(ready + s));
+          ++c;
+        }
+      }
     }
   } else {
     // --------------------------------------------------------- epilogue
@@ -289,7 +349,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA), 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
     if constexpr (C::TMA_Y) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
+      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, W4>(
           args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
           tiles, abort_flag, budget);
     } else {

@@ -241,17 +241,17 @@ int codes_kps() {
 }
 
 template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false,
-          int KPS = 1>
+          int KPS = 1, bool W4 = false>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (!LDA && KPS == 1) {
+  if constexpr (!LDA && KPS == 1 && !W4) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
-  if constexpr (!LDA && KPS == 1 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
+  if constexpr (!LDA && KPS == 1 && !W4 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
     if (codes_kps() == 2) return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
   }
-  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS>;
-  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS>;
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, W4>;
+  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, W4>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
@@ -261,16 +261,24 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int grid = num_sms();
   if (grid > a.num_tiles) grid = a.num_tiles;
-  kern<<<grid, sq::codes_threads(EPW, LDA), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
+  kern<<<grid, sq::codes_threads(EPW, LDA, W4), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
   return cuda_status(cudaGetLastError());
 }
 
-template <int BN, bool MULTI, bool SINGLE = false, int EPW = sq::epi_warps(MULTI)>
+template <int BN, bool MULTI, bool SINGLE = false, int EPW = sq::epi_warps(MULTI), bool W4 = false>
 sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                            const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                            cudaStream_t stream) {
-  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE, EPW>(tqp, tqn, tw, ty, a, stream)
-                : launch_codes<BN, false, MULTI, SINGLE, EPW>(tqp, tqn, tw, ty, a, stream);
+  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE, EPW, false, 1, W4>(tqp, tqn, tw, ty, a, stream)
+                : launch_codes<BN, false, MULTI, SINGLE, EPW, false, 1, W4>(tqp, tqn, tw, ty, a, stream);
+}
+
+// Whether int4 weights run through the GEMM from codes (unpack warps, one
+// ring of stages, seeded accumulators); SEGQUANT_W4_CODES=0 selects the
+// operand-ring kernel with producer warps.
+bool use_codes_w4() {
+  if (const char* e = std::getenv("SEGQUANT_W4_CODES")) return std::atoi(e) != 0;
+  return true;
 }
 
 // Whether 256-wide tiles of the GEMM from codes drain TMEM with 16 epilogue
@@ -603,7 +611,8 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   }
   // One row tile of fewer than BM rows, read by the GEMM from codes: code boxes
   // of M rows rounded up to 16 instead of mostly out-of-bounds 128-row boxes.
-  const bool codes_kernel = (src == ASource::Single) || (codes_ring && !w4);
+  const bool codes_w4 = (src == ASource::Codes) && w4 && !pair && acc == nullptr && use_codes_w4();
+  const bool codes_kernel = (src == ASource::Single) || codes_ring || codes_w4;
   const int a_rows = (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
   CUtensorMap ta, ta2, tw;
   if (src == ASource::X) {
@@ -680,6 +689,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     return launch_pair_out<128, false>(ac, yb, ta, ta2, tw, a, stream);
   }
   if (src == ASource::Codes) {
+    if (codes_w4) {
+      CUtensorMap ty;
+      st = make_tmap_y(&ty, y, yt, M, N, ldy);
+      if (st != SQ_OK) return st;
+      return launch_codes_out<128, true, false, sq::epi_warps(true), true>(yb, ta, ta2, tw, ty, a, stream);
+    }
     if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
     if (!ac && use_codes_ring()) {
       CUtensorMap ty;

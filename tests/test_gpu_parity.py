@@ -212,6 +212,32 @@ def test_wide_tiles_with_sixteen_epilogue_warps_agree(out, monkeypatch):
     assert torch.equal(ys["1"].view(iv), ys["0"].view(iv))
 
 
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+@pytest.mark.parametrize("MKN", [(300, 640, 272, (0, 256, 640)), (129, 384, 144), (200, 1024, 400),
+                                 (64, 3072, 1024), (1, 256, 96), (16, 1024, 272, (0, 512, 1024)),
+                                 (257, 1152, 128, (0, 128, 640, 1152))])
+def test_int4_codes_kernel_and_operand_ring_kernel_agree(MKN, out, monkeypatch):
+    """int4 weights (group 128) through the GEMM from codes (unpack warps, one
+    ring of stages, seeded accumulators) and through the operand-ring kernel:
+    the oracle's result on every row and identical bits; ragged M and N tails,
+    one to three K segments, short row tiles."""
+    import post_quantized_linear_b200 as pq
+    M, K, N = MKN[:3]
+    kseg = list(MKN[3]) if len(MKN) > 3 else None
+    sig = [1.0, 4.0, 0.5][: len(kseg) - 1] if kseg else None
+    c = Case(W.small_case(M, K, N, seed=200 + M, bits=4, out=out, kseg=kseg, x_sigmas=sig))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    ys = {}
+    for v in ("1", "0"):
+        monkeypatch.setenv("SEGQUANT_W4_CODES", v)
+        ys[v] = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(ys["1"], np.arange(M))
+    iv = torch.int16 if out == "bf16" else torch.int32
+    assert torch.equal(ys["1"].view(iv), ys["0"].view(iv))
+
+
 @pytest.mark.parametrize("kseg", [None, (0, 256, 640)])
 @pytest.mark.parametrize("M", [1, 17, 48, 100, 127])
 def test_code_boxes_sized_to_a_short_row_tile(M, kseg, monkeypatch):
@@ -356,14 +382,14 @@ def test_weight_quantization_range_status():
     assert pq.stream_status() == _lib.SQ_OK
 
 
-@pytest.mark.parametrize("codes", [False, True])
-def test_starved_pipeline_times_out_and_context_recovers(codes):
+@pytest.mark.parametrize("codes,i", [(False, 0), (True, 0), (True, 6)])
+def test_starved_pipeline_times_out_and_context_recovers(codes, i):
     """Bounded waits: with the producer starved every wait expires; the kernel
     records SQ_ERR_TIMEOUT, frees its TMEM and exits, and the next launch on the
-    same context is correct again."""
+    same context is correct again (int8 and int4 weights)."""
     import post_quantized_linear_b200 as pq
     from post_quantized_linear_b200 import _lib
-    c = Case(_small(0))
+    c = Case(_small(i))
     qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
     assert pq.stream_status() == _lib.SQ_OK
     pq.set_wait_budget(2_000_000)                   # about a millisecond
