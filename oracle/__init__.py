@@ -312,3 +312,112 @@ def f32_to_bf16_bits(v: float) -> int:
 
 def f32_to_f16_bits(v: float) -> int:
     return int(_load().sqo_f32_to_f16(float(v)))
+
+
+# ----------------------------------------------------------------------------
+# Block-diagonal Hadamard transform of the activations ("HQ-DM: Single
+# Hadamard Transformation-Based Quantization-Aware Training for Low-Bit
+# Diffusion Models", Spanish technical summary section 2.1: the activation
+# matrix X is multiplied by a block-diagonal matrix H built from standard
+# Hadamard matrices and XH is quantized; the weights are left untransformed;
+# because H is orthogonal and symmetric the activation is recovered as
+# X^ = S * (XH)_int * H; the normalization 2^(-k/2) of a 2^k-point block is
+# carried by the floating-point scales so the core stays integer).
+#
+# Readings (the page states the recovery step only as that formula):
+# * blocks of b = 16 (k = 4) along K, so 2^(-k/2) = 1/4 is a power of two and
+#   every scaling by it is exact; blocks never straddle a K-segment bound
+#   (bounds are multiples of 128);
+# * the transform is computed in fp32 by the radix-2 butterfly in Sylvester
+#   order (one rounding per addition), then multiplied by 1/4;
+# * the linear layer Y = X^ W^T with X^ = S (XH)_int H and the untransformed
+#   int4 weight W^ = s_w W_int is evaluated exactly as the integer product of
+#   the codes with the weight codes rotated into the same basis,
+#   (XH)_int (W_int H16)^T with H16 the +-1 Sylvester matrix (H = H16 / 4):
+#   Y = s_w * (S / 4) * (XH)_int (W_int H16)^T.  For int4 codes in [-7, 7] the
+#   rotated codes lie in [-112, 112], so the product stays int8 x int8;
+# * the factor 1/4 is applied to the activation scales (s+/4, s-/4) in the
+#   DualScale epilogue, whose fixed fp32 order is otherwise unchanged.
+HADAMARD_BLOCK = 16
+HADAMARD_NORM = np.float32(0.25)      # 2^(-k/2) for b = 2^k = 16
+
+
+def hadamard_matrix(b: int = HADAMARD_BLOCK) -> np.ndarray:
+    """The b x b Sylvester Hadamard matrix (entries +-1, int64), b a power of 2:
+    H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]."""
+    if b < 1 or b & (b - 1):
+        raise ValueError("b must be a power of two")
+    h = np.ones((1, 1), np.int64)
+    while h.shape[0] < b:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def hadamard_transform(x: np.ndarray, b: int = HADAMARD_BLOCK) -> np.ndarray:
+    """X H in fp32: each row split into blocks of b along K, each block
+    replaced by its Sylvester-ordered butterfly (stage h = 1, 2, 4, ...: the
+    pair (v[j], v[j+h]) becomes (v[j] + v[j+h], v[j] - v[j+h]), each rounded
+    to fp32), then multiplied by 1/sqrt(b) (b = 16: 1/4, exact).  x: fp32
+    values or bf16 stored as uint16 bit patterns, shape [M, K], K % b == 0."""
+    if b != HADAMARD_BLOCK:
+        raise ValueError("the transform uses blocks of 16")
+    if x.dtype == np.uint16:
+        x32 = (x.astype(np.uint32) << 16).view(np.float32)
+    else:
+        x32 = np.asarray(x, np.float32)
+    M, K = x32.shape
+    if K % b:
+        raise ValueError("K must be a multiple of the block size")
+    v = x32.reshape(M, K // b, b).copy()
+    h = 1
+    while h < b:
+        for i in range(0, b, 2 * h):
+            for j in range(i, i + h):
+                a = v[..., j].copy()
+                c = v[..., j + h].copy()
+                v[..., j] = a + c
+                v[..., j + h] = a - c
+        h *= 2
+    v *= HADAMARD_NORM
+    return v.reshape(M, K)
+
+
+def calibrate_hadamard(x: np.ndarray, kbounds, b: int = HADAMARD_BLOCK):
+    """Static per-segment DualScale scales of the transformed activations XH."""
+    return calibrate(hadamard_transform(x, b), kbounds)
+
+
+def quantize_activations_hadamard(x: np.ndarray, kbounds, s_pos, s_neg, b: int = HADAMARD_BLOCK):
+    """DualScale codes (q+, q-) of XH, each int8 [M, K]."""
+    return quantize_activations(hadamard_transform(x, b), kbounds, s_pos, s_neg)
+
+
+def rotate_weight_codes(codes: np.ndarray, b: int = HADAMARD_BLOCK) -> np.ndarray:
+    """W_int H_b blockwise along K (exact integers), int8 [N, K]; raises if a
+    rotated code leaves [-127, 127] (int4 codes in [-7, 7] stay within 112)."""
+    c = np.asarray(codes, np.int64)
+    N, K = c.shape
+    r = (c.reshape(N, K // b, b) @ hadamard_matrix(b)).reshape(N, K)
+    if np.abs(r).max(initial=0) > 127:
+        raise ValueError("rotated weight codes exceed int8")
+    return r.astype(np.int8)
+
+
+def linear_forward_hadamard(x, kbounds, s_pos, s_neg, packed, scales, bias=None, out="f32",
+                            b: int = HADAMARD_BLOCK, return_acc: bool = False):
+    """The forward with Hadamard-transformed activations and untransformed int4
+    weights (packed uint8 [N, K/2], fp16 group scales [K/128, N]): codes of XH,
+    per-group int32 accumulators against the rotated weight codes, and the
+    DualScale epilogue with the activation scales times 1/4.  s_pos/s_neg are
+    the scales of XH (calibrate_hadamard)."""
+    M, K = x.shape
+    qp, qn = quantize_activations_hadamard(x, kbounds, s_pos, s_neg, b)
+    rot = rotate_weight_codes(unpack_w4(packed, K), b)
+    ub, useg = units_of(4, K, kbounds)
+    acc = accumulate(qp, qn, rot, ub)
+    sp = np.asarray(s_pos, np.float32) * HADAMARD_NORM
+    sn = np.asarray(s_neg, np.float32) * HADAMARD_NORM
+    y = epilogue(acc, useg, sp, sn, unit_weight_scales(4, scales), bias, out)
+    if return_acc:
+        return y, acc, (qp, qn), rot
+    return y
