@@ -466,6 +466,23 @@ def run_ours(args):
             pq.quantize_activations_single(xd, wl.kseg, sp, sn, out=c1_buf)
             pq.linear_from_single(c1_buf, qw, sp, sn, bd, out=y)
         single_graph = capture(single_forward)
+    # int4 weights: the block-Hadamard variant (HQ-DM) of the same forward --
+    # codes of XH, then the product with the rotated int4 codes.  Its scales
+    # and the weight rotation are offline steps, made once here.
+    had_graph = None
+    if wl.bits == 4:
+        hsp = torch.empty(J, dtype=torch.float32, device=dev)
+        hsn = torch.empty(J, dtype=torch.float32, device=dev)
+        pq.calibrate_hadamard(calib, wl.kseg, hsp, hsn)
+        w_rot = pq.rotate_weights_hadamard(qw)
+        ldh = (wl.K + 15) // 16 * 16
+        hq_p = torch.empty((wl.M, ldh), dtype=torch.int8, device=dev)[:, : wl.K]
+        hq_n = torch.empty((wl.M, ldh), dtype=torch.int8, device=dev)[:, : wl.K]
+
+        def hadamard_forward():
+            pq.quantize_activations_hadamard(xd, wl.kseg, hsp, hsn, out=(hq_p, hq_n))
+            pq.linear_from_codes_hadamard(hq_p, hq_n, qw, w_rot, hsp, hsn, bd, out=y)
+        had_graph = capture(hadamard_forward)
 
     def timed(graph, n, salt):
         evs = events(n)
@@ -495,9 +512,10 @@ def run_ours(args):
     fwd_ms = timed(fwd_graph, args.steps, 5)
     fused_ms = timed(fused_graph, args.steps, 7) if fused_graph is not None else None
     single_ms = timed(single_graph, args.steps, 9) if single_graph is not None else None
+    had_ms = timed(had_graph, args.steps, 11) if had_graph is not None else None
     if pq.stream_status() != 0:
         raise RuntimeError("device status word set during the timed region")
-    del step_graph, fwd_graph, gemm_graph, fused_graph, single_graph
+    del step_graph, fwd_graph, gemm_graph, fused_graph, single_graph, had_graph
 
     # end to end through the API: host inputs in, host result out, every step
     e2e = None
@@ -533,12 +551,13 @@ def run_ours(args):
     # max over ranks
     vals = [total_ms, statistics.mean(gemm_ms), statistics.mean(fwd_ms),
             e2e["ms"] if e2e else 0.0, statistics.mean(fused_ms) if fused_ms else 0.0,
-            statistics.mean(single_ms) if single_ms else 0.0]
+            statistics.mean(single_ms) if single_ms else 0.0,
+            statistics.mean(had_ms) if had_ms else 0.0]
     if world > 1:
         t = torch.tensor(vals, dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         vals = t.tolist()
-    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms, fused_avg_ms, single_avg_ms = vals
+    total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms, fused_avg_ms, single_avg_ms, had_avg_ms = vals
 
     if rank == 0:
         int8_peak_tops, hbm_peak, peak_kind = peaks()
@@ -571,6 +590,13 @@ def run_ours(args):
             "timing": "each step one CUDA-graph replay, CUDA events on the launching stream",
             "clocks": clocks,
         }
+        if had_ms:
+            line["hadamard_forward"] = {
+                "us": had_avg_ms * 1e3,
+                "exec_tops": ops / (had_avg_ms * 1e-3) / 1e12,
+                "over_dualscale_forward": had_avg_ms / fwd_avg_ms,
+                "note": "block-Hadamard activations (blocks of 16): codes of XH, then the product "
+                        "with the Hadamard-rotated int4 codes (rotation and its scales offline)"}
         if single_ms:
             line["single_scale_forward"] = {
                 "us": single_avg_ms * 1e3,

@@ -219,6 +219,60 @@ sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int6
                                    const float* bias, void* y, sq_dtype yt, int64_t ldy,
                                    sq_stream_t stream);
 
+/* ---- Block-Hadamard activations (HQ-DM, "HQ-DM: Single Hadamard
+ * Transformation-Based Quantization-Aware Training for Low-Bit Diffusion
+ * Models", Spanish technical summary section 2.1): the activation matrix is
+ * multiplied by a block-diagonal Hadamard matrix H before quantization, the
+ * weights are quantized untransformed, and the activation is recovered as
+ * X^ = S (XH)_int H (H orthogonal and symmetric), the block normalization
+ * 2^(-k/2) carried by the floating-point scales.  Readings: blocks of 16 along
+ * K (normalization 1/4); the transform in fp32 by the Sylvester-ordered
+ * butterfly (stage h = 1, 2, 4, 8: (v[j], v[j+h]) -> (v[j] + v[j+h],
+ * v[j] - v[j+h]), each rounded), then times 1/4; Y = X^ W^T evaluated exactly
+ * as the integer product of the XH codes with the int4 weight codes rotated by
+ * the +-1 Sylvester matrix, with the activation scales times 1/4 in the
+ * DualScale epilogue.  int4 weights (group 128) only: their rotated codes lie
+ * in [-112, 112] and stay int8. */
+
+/* Per-segment DualScale scales of XH: s_pos[j] = max(XH+)/127, s_neg[j] =
+ * max(-XH-)/127 over the rows (as sq_calibrate, on the transformed values).
+ * K % 16 == 0; other arguments, requirements and errors as for sq_calibrate. */
+sq_status sq_calibrate_hadamard(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
+                                const sq_segments* kseg, float* s_pos, float* s_neg,
+                                sq_stream_t stream);
+
+/* DualScale codes of XH with the scales of sq_calibrate_hadamard (the codes of
+ * sq_quantize_activations applied to the transformed row blocks).  Arguments,
+ * requirements and errors as for sq_quantize_activations. */
+sq_status sq_quantize_activations_hadamard(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                           int64_t ldx, const sq_segments* kseg,
+                                           const float* s_pos, const float* s_neg, int8_t* q_pos,
+                                           int8_t* q_neg, int64_t ldq, sq_stream_t stream);
+
+/* The int4 weight codes of w (bits = 4, group 128, as written by
+ * sq_quantize_weights) rotated into the transform's basis: every 16-wide block
+ * of a row times the +-1 Sylvester matrix, exact, written as int8.
+ * w_rot: device int8 [N, K], row stride ldr (>= K, a multiple of 16), 16-byte
+ * aligned, owned by the caller.  Errors: SQ_ERR_UNSUPPORTED for bits = 8;
+ * SQ_ERR_INVALID_ARG / SQ_ERR_ALIGNMENT as for the other weight calls. */
+sq_status sq_rotate_weights_hadamard(const sq_qweight* w, int8_t* w_rot, int64_t ldr,
+                                     sq_stream_t stream);
+
+/* The forward from the codes of sq_quantize_activations_hadamard: per 128-wide
+ * group g, acc+- = q+- . w_rot^T (int32), then the DualScale epilogue with the
+ * group's fp16 weight scale and the activation scales times 1/4:
+ * t = fma(s-/4, F(acc-), (s+/4) * F(acc+)), y = fma(s_w[g][n], t, y), + bias,
+ * output rounding.  w: the int4 weight the rotation was made from (its N, K,
+ * K segments and group scales are used; its packed codes are not read);
+ * w_rot, ldr: as written by sq_rotate_weights_hadamard.  s_pos/s_neg: the
+ * scales of XH.  Other arguments and requirements as for
+ * sq_linear_forward_codes; SQ_ERR_UNSUPPORTED for bits = 8. */
+sq_status sq_linear_forward_codes_hadamard(const int8_t* q_pos, const int8_t* q_neg, int64_t ldq,
+                                           int64_t M, int64_t K, const sq_qweight* w,
+                                           const int8_t* w_rot, int64_t ldr, const float* s_pos,
+                                           const float* s_neg, const float* bias, void* y,
+                                           sq_dtype yt, int64_t ldy, sq_stream_t stream);
+
 /* Small-M forward from DualScale codes (1 <= M <= 128 tokens): the same result
  * as sq_linear_forward_codes, bit for bit (SegQuant DualScale, Spanish
  * technical summary 2.B; the two int8 products and the fused epilogue), with

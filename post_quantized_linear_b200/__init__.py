@@ -26,7 +26,9 @@ __all__ = ["QuantizedWeight", "SegQuantError", "calibrate", "quantize_weights", 
            "quantize_activations", "linear_from_codes", "quantize_activations_combined",
            "linear_from_combined", "quantize_activations_single", "linear_from_single",
            "splitk_workspace_size", "splitk_workspace", "linear_from_codes_splitk",
-           "linear_accumulators", "stream_status", "qweight_sizes"]
+           "linear_accumulators", "stream_status", "qweight_sizes", "calibrate_hadamard",
+           "quantize_activations_hadamard", "rotate_weights_hadamard",
+           "linear_from_codes_hadamard"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -316,3 +318,84 @@ def set_wait_budget(cycles: int) -> None:
 def debug_starve_pipeline(enable: bool) -> None:
     """Test hook: GEMM launches issue no TMA copies, so their waits expire."""
     _lib.load().sq_debug_starve_pipeline(1 if enable else 0)
+
+
+# ------------------------------------------------- block-Hadamard activations
+# HQ-DM ("HQ-DM: Single Hadamard Transformation-Based Quantization-Aware
+# Training for Low-Bit Diffusion Models", Spanish technical summary 2.1):
+# activations times a block-diagonal Hadamard matrix (blocks of 16 along K)
+# before quantization; int4 weights quantized untransformed; the forward is the
+# integer product of the XH codes with the int4 codes rotated into the same
+# basis, the block normalization 1/4 carried by the activation scales.
+
+def calibrate_hadamard(x: torch.Tensor, kseg: Sequence[int], s_pos: Optional[torch.Tensor] = None,
+                       s_neg: Optional[torch.Tensor] = None, stream=None):
+    """DualScale scales (s+, s-) fp32 [J] of the transformed calibration rows XH."""
+    _check_2d(x, "x")
+    J = len(kseg) - 1
+    if s_pos is None:
+        s_pos = torch.empty(J, dtype=torch.float32, device=x.device)
+    if s_neg is None:
+        s_neg = torch.empty(J, dtype=torch.float32, device=x.device)
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_calibrate_hadamard", _lib.load().sq_calibrate_hadamard(
+        _ptr(x), _dtype_code(x.dtype), x.shape[0], x.shape[1], x.stride(0), ctypes.byref(seg),
+        _ptr(s_pos), _ptr(s_neg), _stream(stream)))
+    return s_pos, s_neg
+
+
+def quantize_activations_hadamard(x: torch.Tensor, kseg: Sequence[int], s_pos: torch.Tensor,
+                                  s_neg: torch.Tensor, out=None, stream=None):
+    """DualScale codes (q+, q-) of XH, int8 [M, K] each (row stride a multiple of 16)."""
+    _check_2d(x, "x")
+    M, K = x.shape
+    if out is None:
+        ldq = (K + 15) // 16 * 16
+        qp = torch.empty((M, ldq), dtype=torch.int8, device=x.device)[:, :K]
+        qn = torch.empty((M, ldq), dtype=torch.int8, device=x.device)[:, :K]
+    else:
+        qp, qn = out
+        if qp.stride(0) != qn.stride(0):
+            raise ValueError("q_pos and q_neg must share a row stride")
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_quantize_activations_hadamard", _lib.load().sq_quantize_activations_hadamard(
+        _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(seg), _ptr(s_pos),
+        _ptr(s_neg), _ptr(qp), _ptr(qn), qp.stride(0), _stream(stream)))
+    return qp, qn
+
+
+def rotate_weights_hadamard(qw: QuantizedWeight, out: Optional[torch.Tensor] = None,
+                            stream=None) -> torch.Tensor:
+    """The int4 codes of ``qw`` rotated into the transform's basis, int8 [N, K]."""
+    if qw.bits != 4:
+        raise ValueError("the Hadamard forward takes int4 weights")
+    if out is None:
+        out = torch.empty((qw.N, qw.K), dtype=torch.int8, device=qw.codes.device)
+    _check_2d(out, "out")
+    c, keep = qw.c_struct()
+    _lib.check("sq_rotate_weights_hadamard", _lib.load().sq_rotate_weights_hadamard(
+        ctypes.byref(c), _ptr(out), out.stride(0), _stream(stream)))
+    return out
+
+
+def linear_from_codes_hadamard(q_pos: torch.Tensor, q_neg: torch.Tensor, qw: QuantizedWeight,
+                               w_rot: torch.Tensor, s_pos: torch.Tensor, s_neg: torch.Tensor,
+                               bias: Optional[torch.Tensor] = None,
+                               out_dtype: torch.dtype = torch.bfloat16,
+                               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Forward from the XH codes and the rotated int4 weight codes."""
+    _check_2d(q_pos, "q_pos")
+    _check_2d(q_neg, "q_neg")
+    _check_2d(w_rot, "w_rot")
+    M, K = q_pos.shape
+    if q_neg.shape != q_pos.shape or q_neg.stride(0) != q_pos.stride(0):
+        raise ValueError("q_pos and q_neg must have the same shape and row stride")
+    if out is None:
+        out = torch.empty((M, qw.N), dtype=out_dtype, device=q_pos.device)
+    _check_2d(out, "out")
+    c, keep = qw.c_struct()
+    _lib.check("sq_linear_forward_codes_hadamard", _lib.load().sq_linear_forward_codes_hadamard(
+        _ptr(q_pos), _ptr(q_neg), q_pos.stride(0), M, K, ctypes.byref(c), _ptr(w_rot),
+        w_rot.stride(0), _ptr(s_pos), _ptr(s_neg), _ptr(bias), _ptr(out), _dtype_code(out.dtype),
+        out.stride(0), _stream(stream)))
+    return out

@@ -61,6 +61,13 @@ SIGNATURES = {
                                                       c_vp, c_vp, c_vp, c_i32, c_i64, c_vp]),
     "sq_linear_accumulators": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp,
                                        c_vp]),
+    "sq_calibrate_hadamard": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp, c_vp, c_vp]),
+    "sq_quantize_activations_hadamard": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp,
+                                                 c_vp, c_vp, c_vp, c_i64, c_vp]),
+    "sq_rotate_weights_hadamard": (c_i32, [P_QW, c_vp, c_i64, c_vp]),
+    "sq_linear_forward_codes_hadamard": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i64, P_QW, c_vp,
+                                                 c_i64, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64,
+                                                 c_vp]),
     "sq_stream_status": (c_i32, [c_vp]),
     "sq_status_string": (ctypes.c_char_p, [c_i32]),
     "sq_last_cuda_error": (ctypes.c_char_p, []),

@@ -863,13 +863,16 @@ __device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float&
 // registers (HALF == 32), stored once per tile; otherwise one unit per tile,
 // streamed out in 32-column passes with the accumulators released after the
 // warp's last TMEM load.
-// SEEDED (int4 weights unpacked as 16 x the code, one unit per 128-wide
-// group): the accumulators hold the bits of 1.5 * 2^19 + acc (kMagicW4Bits
-// plus 16 * acc).  The warps seed their columns of both buffers before the
-// first unit and again right after reading them, so F(acc) is one exact
-// subtraction; the group's fp16 weight scales and its segment's s+/s- enter
-// the same fp32 order as the other units.
-template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, bool SEEDED, class TileFn>
+// SEED (one unit per 128-wide group, the accumulators seeded): 1 -- int4
+// weights unpacked as 16 x the code, the accumulators hold the bits of
+// 1.5 * 2^19 + acc (kMagicW4Bits plus 16 * acc); 2 -- int8 weight codes (the
+// Hadamard-rotated int4 codes, |acc| < 2^22), the accumulators hold the bits
+// of 1.5 * 2^23 + acc, and the activation scales are multiplied by the block
+// normalization 1/4 (exact).  The warps seed their columns of both buffers
+// before the first unit and again right after reading them, so F(acc) is one
+// exact subtraction; the group's fp16 weight scales and its segment's s+/s-
+// enter the same fp32 order as the other units.
+template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, int SEED, class TileFn>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
@@ -880,7 +883,11 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
   constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
   static_assert(HALF % 32 == 0, "32-column store passes");
   static_assert(!MULTI || HALF == 32, "several units: one 32-column pass per warp");
+  constexpr bool SEEDED = (SEED != 0);
   static_assert(!SEEDED || (MULTI && NACC == 2), "seeded accumulators: int4 groups, DualScale");
+  constexpr uint32_t seed_bits = (SEED == 1) ? kMagicW4Bits : kMagicBits;
+  constexpr float seed_value = (SEED == 1) ? kMagicW4 : kMagic;
+  constexpr float act_mult = (SEED == 2) ? 0.25f : 1.0f;   // Hadamard block normalization
   uint8_t* srow = stage_y + lane * ROWB;
   const uint32_t sbase = smem_u32(stage_y);
   const int units = SEEDED ? args.num_kb : args.kseg.count;
@@ -917,14 +924,16 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
     const uint32_t tcol = (uint32_t)b * BUF_COLS + (uint32_t)cc;
     float sp, sn;
     unit_act_scales(args, j, sp, sn);
+    sp = __fmul_rn(sp, act_mult);
+    sn = __fmul_rn(sn, act_mult);
     uint32_t ap[16], an[16];
     tmem_ld16(t_lane + tcol, ap);
     tmem_ld16(t_lane + tcol + BN, an);
     tmem_wait_ld();
 #pragma unroll
     for (int h = 0; h < 16; h += 8) {
-      tmem_st8(t_lane + tcol + h, kMagicW4Bits);
-      tmem_st8(t_lane + tcol + BN + h, kMagicW4Bits);
+      tmem_st8(t_lane + tcol + h, seed_bits);
+      tmem_st8(t_lane + tcol + BN + h, seed_bits);
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {   // scales eight columns at a time (registers)
@@ -932,7 +941,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       load_wscales8(args, u, j, t.n0 + cc + 8 * h, sw8);
       fold8_seeded(*reinterpret_cast<const uint32_t(*)[8]>(ap + 8 * h),
                    *reinterpret_cast<const uint32_t(*)[8]>(an + 8 * h), sw8, sp, sn, y + 8 * h,
-                   kMagicW4);
+                   seed_value);
     }
   };
   int ug = 0;
@@ -944,8 +953,8 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 #pragma unroll
       for (int c = 0; c < HALF; c += 8) {
         const uint32_t col = (uint32_t)b * BUF_COLS + (uint32_t)(part * HALF + c);
-        tmem_st8(t_lane + col, kMagicW4Bits);
-        tmem_st8(t_lane + col + BN, kMagicW4Bits);
+        tmem_st8(t_lane + col, seed_bits);
+        tmem_st8(t_lane + col + BN, seed_bits);
       }
     }
     tmem_wait_st();

@@ -20,12 +20,18 @@
 // Stage sizes: (2 or 1) x 16 KiB of codes + BN x 128 bytes of weights, as many
 // as fit in 224 KiB next to the epilogue's staging tiles (2 or 4 KiB per
 // epilogue warp for bf16 or fp32 Y).
-// W4: int4 weights with one scale per 128-wide group along K (the SegQuant
+// WM (weight mode) 0: int8 weights, one unit per K segment.
+// WM 1 (W4): int4 weights with one scale per 128-wide group along K (the SegQuant
 // paper's W4A8 setting): TMA brings the packed tile (BN rows of 64 bytes) into
 // the stage, two unpack warps widen it to int8 in the 128-byte-swizzled
 // layout beside it and signal a per-stage ready barrier that the MMA waits
 // on; every k block is its own unit, folded by the epilogue from seeded
-// accumulators (epilogue_tma_store, SEEDED).
+// accumulators (epilogue_tma_store, SEED 1).
+// WM 2: int8 weight tiles with the units and fp16 scales of int4 groups -- the
+// int4 codes rotated by the block Hadamard matrix (HQ-DM, "Single Hadamard
+// Transformation", Spanish technical summary 2.1) -- folded from seeded
+// accumulators with the activation scales times the block normalization 1/4
+// (epilogue_tma_store, SEED 2).
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -75,8 +81,9 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 }
 
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
-          bool LDA_ = false, int KPS_ = 1, bool W4_ = false>
+          bool LDA_ = false, int KPS_ = 1, int WM_ = 0>
 struct CodesCfg {
+  static constexpr bool W4_ = (WM_ == 1);
   static constexpr bool LDA = LDA_;
   static constexpr int KPS = KPS_;
   // full barrier: the TMA thread's arrival (+ bytes), plus one per loader thread
@@ -95,8 +102,8 @@ struct CodesCfg {
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
   static_assert(KPS == 1 || !LDA_, "two k blocks per stage: TMA loads");
-  static_assert(!W4_ || (MULTI && !SINGLE && !LDA_ && KPS_ == 1 && BN_ == 128),
-                "int4 weights: DualScale, one k block per stage, BN = 128");
+  static_assert(WM_ == 0 || (MULTI && !SINGLE && !LDA_ && KPS_ == 1 && BN_ == 128),
+                "group units: DualScale, one k block per stage, BN = 128");
   static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
@@ -112,14 +119,16 @@ struct CodesCfg {
 };
 
 template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false, int EPW = epi_warps(MULTI),
-          bool LDA = false, int KPS = 1, bool W4 = false>
-__global__ void __launch_bounds__(codes_threads(EPW, LDA, W4), 1)
+          bool LDA = false, int KPS = 1, int WM = 0>
+__global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, W4>;
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, WM>;
+  constexpr bool W4 = (WM == 1);        // packed int4 tiles, unpack warps
+  constexpr bool SEEDED = (WM != 0);    // one unit per k block, seeded accumulators
   constexpr int EPI0 = codes_epi_warp0(LDA, W4);
   static_assert(EPW % 4 == 0 && (BN / (EPW / 4)) % 32 == 0, "32-column store passes per warp");
   static_assert(!MULTI || (BN == 128 && C::NBUF == 2), "several units per tile: BN = 128, two buffers");
@@ -234,9 +243,9 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, W4), 1)
             const int kb = kb0 + j;
             if (!unit_open) {   // a unit (K segment) may start inside a stage
               const int b = ug % C::NBUF;
-              // seeded (W4) buffers: the epilogue's first release (after seeding)
+              // seeded buffers: the epilogue's first release (after seeding)
               // completes phase 0, so every use waits one phase later
-              const uint32_t par = W4 ? ((ug / C::NBUF) & 1) : (((ug / C::NBUF) & 1) ^ 1);
+              const uint32_t par = SEEDED ? ((ug / C::NBUF) & 1) : (((ug / C::NBUF) & 1) ^ 1);
               if (!(ok = wait1(smem_u32(tmem_empty + b), par, abort_flag, budget))) break;
               tc_fence_after();
               d_pos = tmem_base + (uint32_t)(b * C::NACC * BN);
@@ -246,7 +255,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, W4), 1)
             const uint32_t b_w = a_p + C::A_BYTES;
 #pragma unroll
             for (int ks = 0; ks < BK / 32; ++ks) {
-              const uint32_t acc = (W4 || unit_open || ks > 0) ? 1u : 0u;
+              const uint32_t acc = (SEEDED || unit_open || ks > 0) ? 1u : 0u;
               const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
               umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
               if constexpr (!SINGLE)
@@ -349,7 +358,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, W4), 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
     if constexpr (C::TMA_Y) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, W4>(
+      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, WM>(
           args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
           tiles, abort_flag, budget);
     } else {

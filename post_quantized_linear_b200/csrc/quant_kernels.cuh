@@ -165,13 +165,38 @@ __device__ __forceinline__ void load16(const XT* p, float (&v)[16]) {
   }
 }
 
+// ------------------------------------------------ block Hadamard transform
+// HQ-DM ("HQ-DM: Single Hadamard Transformation-Based Quantization-Aware
+// Training for Low-Bit Diffusion Models", Spanish technical summary 2.1): the
+// activations are multiplied by a block-diagonal Hadamard matrix before they
+// are quantized.  Blocks of 16 along K: the Sylvester-ordered butterfly (stage
+// h = 1, 2, 4, 8: (v[j], v[j+h]) -> (v[j] + v[j+h], v[j] - v[j+h]), each
+// rounded to fp32), then the normalization 1/sqrt(16) = 1/4 (exact).
+constexpr float kHadamardNorm = 0.25f;
+
+__device__ __forceinline__ void hadamard16(float (&v)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 16; i += 2 * h)
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float a = v[j], b = v[j + h];
+        v[j] = __fadd_rn(a, b);
+        v[j + h] = __fsub_rn(a, b);
+      }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], kHadamardNorm);
+}
+
 // blockDim = (32, 8): lane x owns the 16-element group blockIdx.x*32 + x of
 // every row it visits (rows blockIdx.y*8 + y, stepping by gridDim.y*8), so its
 // segment and reciprocal scales are fixed; a warp reads 1 KiB (bf16) and
 // writes 512 bytes of each code tensor per row.
 // MODE: CODES_DUAL (q+ and q-), CODES_COMBINED (c = q+ + q-), CODES_SINGLE
-// (the single-scale code: both branches with s = max(s+, s-)).
-constexpr int CODES_DUAL = 0, CODES_COMBINED = 1, CODES_SINGLE = 2;
+// (the single-scale code: both branches with s = max(s+, s-)), CODES_HADAMARD
+// (q+ and q- of the block-Hadamard-transformed activations).
+constexpr int CODES_DUAL = 0, CODES_COMBINED = 1, CODES_SINGLE = 2, CODES_HADAMARD = 3;
 
 template <typename XT, int MODE>
 __device__ __forceinline__ void quantize_activations_body(
@@ -181,7 +206,7 @@ __device__ __forceinline__ void quantize_activations_body(
   const int32_t k = (blockIdx.x * 32 + threadIdx.x) * 16;
   if (k >= K) return;
   const int j = kseg.segment_of(k);
-  constexpr bool COMBINED = (MODE != CODES_DUAL);
+  constexpr bool COMBINED = (MODE == CODES_COMBINED || MODE == CODES_SINGLE);
   const float sj_p = (MODE == CODES_SINGLE) ? fmaxf(s_pos[j], s_neg[j]) : s_pos[j];
   const float sj_n = (MODE == CODES_SINGLE) ? sj_p : s_neg[j];
   const float rp = sj_p > 0.0f ? __frcp_rn(sj_p) : 0.0f;
@@ -190,6 +215,7 @@ __device__ __forceinline__ void quantize_activations_body(
   for (int32_t m = blockIdx.y * 8 + threadIdx.y; m < M; m += step) {
     float v[16];
     load16<XT>(x + (int64_t)m * ldx + k, v);
+    if constexpr (MODE == CODES_HADAMARD) hadamard16(v);
     uint32_t p[16], n[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) { p[i] = code_pos(v[i], rp); n[i] = code_neg(v[i], rn); }
@@ -216,6 +242,110 @@ __global__ void __launch_bounds__(256) quantize_activations_kernel(
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
     int8_t* __restrict__ q_neg, int64_t ldq) {
   quantize_activations_body<XT, CODES_DUAL>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(256) quantize_activations_hadamard_kernel(
+    const XT* __restrict__ x, int32_t M, int32_t K, int64_t ldx, SegBounds kseg,
+    const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
+    int8_t* __restrict__ q_neg, int64_t ldq) {
+  quantize_activations_body<XT, CODES_HADAMARD>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
+}
+
+// Calibration of the transformed activations: per K segment max(XH+) / 127
+// and max(-XH-) / 127.  blockDim = (32, 8) with the quantizer's layout (lane x
+// owns the 16-element group blockIdx.x*32 + x of every row it visits); eight
+// lanes cover 128 columns, which never straddle a segment bound, so an
+// eight-lane shuffle reduction is exact; then shared and global atomicMax on
+// the fp32 bit patterns as in calibrate_kernel.  The outputs must be zeroed
+// before the launch.
+template <typename XT>
+__global__ void __launch_bounds__(256) calibrate_hadamard_kernel(const XT* __restrict__ x,
+                                                                 int64_t rows, int32_t K,
+                                                                 int64_t ldx, SegBounds kseg,
+                                                                 float* __restrict__ s_pos,
+                                                                 float* __restrict__ s_neg) {
+  __shared__ unsigned int sh_p[SQ_MAX_SEG], sh_n[SQ_MAX_SEG];
+  __shared__ int sh_bad;
+  const int tid = threadIdx.y * 32 + threadIdx.x;
+  if (tid < SQ_MAX_SEG) { sh_p[tid] = 0u; sh_n[tid] = 0u; }
+  if (tid == 0) sh_bad = 0;
+  __syncthreads();
+  const int32_t k = (blockIdx.x * 32 + threadIdx.x) * 16;
+  const bool active = k < K;
+  const int j = active ? kseg.segment_of(k) : 0;
+  float P = 0.0f, Q = 0.0f;
+  bool bad = false;
+  if (active) {
+    const int64_t step = (int64_t)gridDim.y * 8;
+    for (int64_t m = (int64_t)blockIdx.y * 8 + threadIdx.y; m < rows; m += step) {
+      float v[16];
+      load16<XT>(x + m * ldx + k, v);
+      hadamard16(v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        bad |= (v[i] != v[i]) || (fabsf(v[i]) == __int_as_float(0x7f800000));
+        P = fmaxf(P, v[i]);
+        Q = fmaxf(Q, -v[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) {
+    P = fmaxf(P, __shfl_xor_sync(0xffffffffu, P, o));
+    Q = fmaxf(Q, __shfl_xor_sync(0xffffffffu, Q, o));
+  }
+  const unsigned any_bad = __ballot_sync(0xffffffffu, bad);
+  if (active && (threadIdx.x & 7) == 0) {
+    atomicMax(&sh_p[j], __float_as_uint(P));
+    atomicMax(&sh_n[j], __float_as_uint(Q));
+  }
+  if (threadIdx.x == 0 && any_bad) sh_bad = 1;
+  __syncthreads();
+  if (tid < kseg.count) {
+    const float p = __uint_as_float(sh_p[tid]) / 127.0f;
+    const float q = __uint_as_float(sh_n[tid]) / 127.0f;
+    if (p > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(s_pos) + tid, __float_as_uint(p));
+    if (q > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(s_neg) + tid, __float_as_uint(q));
+  }
+  if (tid == 0 && sh_bad) raise_status(SQ_STATUS_RANGE);
+}
+
+// Untransformed int4 weight codes rotated into the transform's basis: each
+// 16-wide block of a row times the +-1 Sylvester matrix (exact integers; codes
+// in [-7, 7] give values in [-112, 112]), written as int8.  One thread per
+// (row, block): 8 packed bytes in (low nibble = even k), 16 bytes out.
+__global__ void __launch_bounds__(256) rotate_weights_hadamard_kernel(
+    const uint8_t* __restrict__ packed, int64_t N, int64_t K, int8_t* __restrict__ out,
+    int64_t ldo) {
+  const int64_t blocks = K / 16;
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= N * blocks) return;
+  const int64_t n = t / blocks, b = t % blocks;
+  const uint2 pk = __ldg(reinterpret_cast<const uint2*>(packed + n * (K / 2) + b * 8));
+  const uint32_t w[2] = {pk.x, pk.y};
+  int v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int nib = (int)((w[i >> 3] >> (4 * (i & 7))) & 0xFu);
+    v[i] = (nib ^ 8) - 8;
+  }
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 16; i += 2 * h)
+#pragma unroll
+      for (int jj = i; jj < i + h; ++jj) {
+        const int a = v[jj], c = v[jj + h];
+        v[jj] = a + c;
+        v[jj + h] = a - c;
+      }
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    o[q] = (uint32_t)(v[4 * q] & 0xFF) | ((uint32_t)(v[4 * q + 1] & 0xFF) << 8) |
+           ((uint32_t)(v[4 * q + 2] & 0xFF) << 16) | ((uint32_t)(v[4 * q + 3] & 0xFF) << 24);
+  *reinterpret_cast<uint4*>(out + n * ldo + b * 16) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Combined codes c = q+ + q- (one signed byte per activation): an element

@@ -241,17 +241,17 @@ int codes_kps() {
 }
 
 template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false,
-          int KPS = 1, bool W4 = false>
+          int KPS = 1, int WM = 0>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (!LDA && KPS == 1 && !W4) {
+  if constexpr (!LDA && KPS == 1 && WM == 0) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
-  if constexpr (!LDA && KPS == 1 && !W4 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
+  if constexpr (!LDA && KPS == 1 && WM == 0 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
     if (codes_kps() == 2) return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
   }
-  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, W4>;
-  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, W4>;
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, WM>;
+  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
@@ -261,16 +261,16 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int grid = num_sms();
   if (grid > a.num_tiles) grid = a.num_tiles;
-  kern<<<grid, sq::codes_threads(EPW, LDA, W4), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
+  kern<<<grid, sq::codes_threads(EPW, LDA, WM == 1), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
   return cuda_status(cudaGetLastError());
 }
 
-template <int BN, bool MULTI, bool SINGLE = false, int EPW = sq::epi_warps(MULTI), bool W4 = false>
+template <int BN, bool MULTI, bool SINGLE = false, int EPW = sq::epi_warps(MULTI), int WM = 0>
 sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                            const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                            cudaStream_t stream) {
-  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE, EPW, false, 1, W4>(tqp, tqn, tw, ty, a, stream)
-                : launch_codes<BN, false, MULTI, SINGLE, EPW, false, 1, W4>(tqp, tqn, tw, ty, a, stream);
+  return y_bf16 ? launch_codes<BN, true, MULTI, SINGLE, EPW, false, 1, WM>(tqp, tqn, tw, ty, a, stream)
+                : launch_codes<BN, false, MULTI, SINGLE, EPW, false, 1, WM>(tqp, tqn, tw, ty, a, stream);
 }
 
 // Whether int4 weights run through the GEMM from codes (unpack warps, one
@@ -506,7 +506,7 @@ int choose_bn(int64_t M, int64_t N, bool multi, bool f32x, bool codes_ring) {
 sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
                          const sq_segments* kseg, const float* s_pos, const float* s_neg,
                          int8_t* q_pos, int8_t* q_neg, int64_t ldq, int mode, cudaStream_t s) {
-  const bool combined = (mode != sq::CODES_DUAL);
+  const bool combined = (mode == sq::CODES_COMBINED || mode == sq::CODES_SINGLE);
   if (!dtype_ok(xt) || M < 0 || K <= 0 || ldx < K || ldq < K) return SQ_ERR_INVALID_ARG;
   if (K > SQ_MAX_K) return SQ_ERR_RANGE;
   SegBounds sb;
@@ -545,6 +545,15 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
     else
       sq::quantize_activations_combined_kernel<float, sq::CODES_SINGLE><<<grid, block, 0, s>>>(
           static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+  } else if (mode == sq::CODES_HADAMARD) {
+    if (xt == SQ_BF16)
+      sq::quantize_activations_hadamard_kernel<bf><<<grid, block, 0, s>>>(
+          static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, q_neg,
+          ldq);
+    else
+      sq::quantize_activations_hadamard_kernel<float><<<grid, block, 0, s>>>(
+          static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, q_neg,
+          ldq);
   } else {
     if (xt == SQ_BF16)
       sq::quantize_activations_kernel<bf><<<grid, block, 0, s>>>(
@@ -558,13 +567,17 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
   return cuda_status(cudaGetLastError());
 }
 
-enum class ASource { X, Codes, Combined, Single };
+// Hadamard: q+/q- codes of the block-Hadamard-transformed activations, against
+// the rotated int4 weight codes (int8 [N][ldr]) with the int4 group scales.
+enum class ASource { X, Codes, Combined, Single, Hadamard };
 
 sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_pos,
                       const int8_t* q_neg, int64_t ldq, int64_t M, int64_t K, int64_t ldx,
                       const sq_qweight* w, const float* s_pos, const float* s_neg,
                       const float* bias, void* y, sq_dtype yt, int64_t ldy, int32_t* acc,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const int8_t* w_rot = nullptr, int64_t ldr = 0) {
+  const bool had = (src == ASource::Hadamard);
+  const bool dual_codes = (src == ASource::Codes) || had;   // q+ and q- tensors
   if (src == ASource::X && !dtype_ok(xt)) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && !dtype_ok(yt)) return SQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
@@ -575,16 +588,19 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   if (src == ASource::X && ldx < K) return SQ_ERR_INVALID_ARG;
   if (src != ASource::X && ldq < K) return SQ_ERR_INVALID_ARG;
   if ((src == ASource::Combined || src == ASource::Single) && w->bits != 8) return SQ_ERR_UNSUPPORTED;
+  if (had && (w->bits != 4 || acc != nullptr)) return SQ_ERR_UNSUPPORTED;
+  if (had && (w_rot == nullptr || ldr < K)) return SQ_ERR_INVALID_ARG;
+  if (had && (!aligned16(w_rot) || ldr % 16 != 0)) return SQ_ERR_ALIGNMENT;
   if (acc == nullptr && ldy < N) return SQ_ERR_INVALID_ARG;
   if (M > (int64_t)INT32_MAX - 2 * sq::BM) return SQ_ERR_RANGE;
   if (M == 0) return SQ_OK;
   if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::X && x == nullptr) return SQ_ERR_INVALID_ARG;
-  if (src == ASource::Codes && (q_pos == nullptr || q_neg == nullptr)) return SQ_ERR_INVALID_ARG;
+  if (dual_codes && (q_pos == nullptr || q_neg == nullptr)) return SQ_ERR_INVALID_ARG;
   if ((src == ASource::Combined || src == ASource::Single) && q_pos == nullptr) return SQ_ERR_INVALID_ARG;
   if (acc == nullptr && y == nullptr) return SQ_ERR_INVALID_ARG;
   if (src == ASource::X && (!aligned16(x) || (ldx * elt_size(xt)) % 16 != 0)) return SQ_ERR_ALIGNMENT;
-  if (src == ASource::Codes && (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0))
+  if (dual_codes && (!aligned16(q_pos) || !aligned16(q_neg) || ldq % 16 != 0))
     return SQ_ERR_ALIGNMENT;
   if ((src == ASource::Combined || src == ASource::Single) && (!aligned16(q_pos) || ldq % 16 != 0))
     return SQ_ERR_ALIGNMENT;
@@ -612,7 +628,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   // One row tile of fewer than BM rows, read by the GEMM from codes: code boxes
   // of M rows rounded up to 16 instead of mostly out-of-bounds 128-row boxes.
   const bool codes_w4 = (src == ASource::Codes) && w4 && !pair && acc == nullptr && use_codes_w4();
-  const bool codes_kernel = (src == ASource::Single) || codes_ring || codes_w4;
+  const bool codes_kernel = (src == ASource::Single) || codes_ring || codes_w4 || had;
   const int a_rows = (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
   CUtensorMap ta, ta2, tw;
   if (src == ASource::X) {
@@ -625,7 +641,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
                    (uint64_t)ldq, 128, (uint32_t)a_rows);
     if (st != SQ_OK) return st;
-    if (src == ASource::Codes) {
+    if (dual_codes) {
       st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
                      (uint64_t)ldq, 128, (uint32_t)a_rows);
       if (st != SQ_OK) return st;
@@ -633,7 +649,10 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       ta2 = ta;
     }
   }
-  if (w4)
+  if (had)   // rotated codes, int8 rows of ldr bytes
+    st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_rot, (uint64_t)K, (uint64_t)N,
+                   (uint64_t)ldr, 128, (uint32_t)BN);
+  else if (w4)
     st = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)(K / 2), (uint64_t)N,
                    (uint64_t)(K / 2), 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   else
@@ -667,6 +686,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
   const bool yb = (yt == SQ_BF16);
   const bool ac = (acc != nullptr);
+  if (had) {
+    CUtensorMap ty;
+    st = make_tmap_y(&ty, y, yt, M, N, ldy);
+    if (st != SQ_OK) return st;
+    return launch_codes_out<128, true, false, sq::epi_warps(true), 2>(yb, ta, ta2, tw, ty, a, stream);
+  }
   if (src == ASource::Single) {
     CUtensorMap ty;
     st = make_tmap_y(&ty, y, yt, M, N, ldy);
@@ -693,7 +718,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       CUtensorMap ty;
       st = make_tmap_y(&ty, y, yt, M, N, ldy);
       if (st != SQ_OK) return st;
-      return launch_codes_out<128, true, false, sq::epi_warps(true), true>(yb, ta, ta2, tw, ty, a, stream);
+      return launch_codes_out<128, true, false, sq::epi_warps(true), 1>(yb, ta, ta2, tw, ty, a, stream);
     }
     if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
     if (!ac && use_codes_ring()) {
@@ -906,6 +931,83 @@ sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int6
                                    sq_stream_t stream) {
   return gemm_common(ASource::Single, nullptr, SQ_BF16, c, nullptr, ldc, M, K, 0, w, s_pos, s_neg,
                      bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_calibrate_hadamard(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
+                                const sq_segments* kseg, float* s_pos, float* s_neg,
+                                sq_stream_t stream) {
+  if (!dtype_ok(xt) || rows < 0 || K <= 0 || ldx < K) return SQ_ERR_INVALID_ARG;
+  if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
+  if (K > SQ_MAX_K) return SQ_ERR_RANGE;
+  SegBounds sb;
+  sq_status st = check_segments(kseg, K, SQ_MAX_SEGMENTS, 128, &sb);
+  if (st != SQ_OK) return st;
+  if (K % 16 != 0) return SQ_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(s_pos) & 3u) || (reinterpret_cast<uintptr_t>(s_neg) & 3u))
+    return SQ_ERR_ALIGNMENT;
+  const int xe = elt_size(xt);
+  if (rows > 0) {
+    if (x == nullptr) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || (ldx * xe) % 16 != 0) return SQ_ERR_ALIGNMENT;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(float) * (size_t)sb.count;
+  sq_status ms = cuda_status(cudaMemsetAsync(s_pos, 0, bytes, s));
+  if (ms != SQ_OK) return ms;
+  ms = cuda_status(cudaMemsetAsync(s_neg, 0, bytes, s));
+  if (ms != SQ_OK) return ms;
+  if (rows == 0) return SQ_OK;
+  const int64_t groups = K / 16;
+  const int gx = (int)((groups + 31) / 32);
+  int64_t gy = (rows + 7) / 8;
+  const int64_t cap = ((int64_t)num_sms() * 8 + gx - 1) / gx;
+  if (gy > cap) gy = cap;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  dim3 grid(gx, (unsigned)gy), block(32, 8);
+  if (xt == SQ_BF16)
+    sq::calibrate_hadamard_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), rows, (int32_t)K, ldx, sb, s_pos, s_neg);
+  else
+    sq::calibrate_hadamard_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(x), rows,
+                                                                (int32_t)K, ldx, sb, s_pos, s_neg);
+  return cuda_status(cudaGetLastError());
+}
+
+sq_status sq_quantize_activations_hadamard(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                           int64_t ldx, const sq_segments* kseg,
+                                           const float* s_pos, const float* s_neg, int8_t* q_pos,
+                                           int8_t* q_neg, int64_t ldq, sq_stream_t stream) {
+  return quantize_codes(x, xt, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq,
+                        sq::CODES_HADAMARD, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_rotate_weights_hadamard(const sq_qweight* w, int8_t* w_rot, int64_t ldr,
+                                     sq_stream_t stream) {
+  if (w == nullptr || w_rot == nullptr) return SQ_ERR_INVALID_ARG;
+  SegBounds kseg;
+  sq_status st = check_qweight(w, w->K, &kseg);
+  if (st != SQ_OK) return st;
+  if (w->bits != 4) return SQ_ERR_UNSUPPORTED;
+  if (ldr < w->K) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(w_rot) || ldr % 16 != 0) return SQ_ERR_ALIGNMENT;
+  const int64_t tasks = w->N * (w->K / 16);
+  const int64_t blocks = (tasks + 255) / 256;
+  if (blocks > INT32_MAX) return SQ_ERR_RANGE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  sq::rotate_weights_hadamard_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      static_cast<const uint8_t*>(w->codes), w->N, w->K, w_rot, ldr);
+  return cuda_status(cudaGetLastError());
+}
+
+sq_status sq_linear_forward_codes_hadamard(const int8_t* q_pos, const int8_t* q_neg, int64_t ldq,
+                                           int64_t M, int64_t K, const sq_qweight* w,
+                                           const int8_t* w_rot, int64_t ldr, const float* s_pos,
+                                           const float* s_neg, const float* bias, void* y,
+                                           sq_dtype yt, int64_t ldy, sq_stream_t stream) {
+  return gemm_common(ASource::Hadamard, nullptr, SQ_BF16, q_pos, q_neg, ldq, M, K, 0, w, s_pos,
+                     s_neg, bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream),
+                     w_rot, ldr);
 }
 
 sq_status sq_splitk_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {

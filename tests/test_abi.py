@@ -193,6 +193,42 @@ def test_splitk_entry_points_validate_before_launch():
     assert call(M=0) == L.SQ_OK
 
 
+def test_hadamard_entry_points_validate_before_launch():
+    lib = _lib.load()
+    L = _lib
+    seg, keep = _lib.segments((0, 512))
+    ca = lib.sq_calibrate_hadamard
+    assert ca(FAKE, 1, 16, 512, 512, ctypes.byref(seg), None, FAKE, None) == L.SQ_ERR_INVALID_ARG
+    assert ca(FAKE, 1, -1, 512, 512, ctypes.byref(seg), FAKE, FAKE, None) == L.SQ_ERR_INVALID_ARG
+    assert ca(FAKE + 8, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, None) == L.SQ_ERR_ALIGNMENT
+    odd, keep2 = _lib.segments((0, 520))
+    assert ca(FAKE, 0, 16, 520, 520, ctypes.byref(odd), FAKE, FAKE, None) == L.SQ_ERR_UNSUPPORTED
+    qa = lib.sq_quantize_activations_hadamard
+    assert qa(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, FAKE, 520, None) == L.SQ_ERR_ALIGNMENT
+    assert qa(FAKE, 1, 16, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, None, 512, None) == L.SQ_ERR_INVALID_ARG
+    assert qa(FAKE, 1, 0, 512, 512, ctypes.byref(seg), FAKE, FAKE, FAKE, FAKE, 512, None) == L.SQ_OK
+    qw4, k4 = _qw(bits=4, K=512)
+    qw8, k8 = _qw(bits=8, K=512)
+    ro = lib.sq_rotate_weights_hadamard
+    assert ro(ctypes.byref(qw8), FAKE, 512, None) == L.SQ_ERR_UNSUPPORTED
+    assert ro(ctypes.byref(qw4), None, 512, None) == L.SQ_ERR_INVALID_ARG
+    assert ro(ctypes.byref(qw4), FAKE, 256, None) == L.SQ_ERR_INVALID_ARG
+    assert ro(ctypes.byref(qw4), FAKE, 520, None) == L.SQ_ERR_ALIGNMENT
+    assert ro(ctypes.byref(qw4), FAKE + 8, 512, None) == L.SQ_ERR_ALIGNMENT
+    fh = lib.sq_linear_forward_codes_hadamard
+
+    def fwd(qw=qw4, wr=FAKE, ldr=512, M=256, q=FAKE):
+        return fh(q, q, 512, M, 512, ctypes.byref(qw), wr, ldr, FAKE, FAKE, None, FAKE, L.SQ_BF16,
+                  256, None)
+    assert fwd(qw=qw8) == L.SQ_ERR_UNSUPPORTED
+    assert fwd(wr=None) == L.SQ_ERR_INVALID_ARG
+    assert fwd(ldr=256) == L.SQ_ERR_INVALID_ARG
+    assert fwd(ldr=520) == L.SQ_ERR_ALIGNMENT
+    assert fwd(wr=FAKE + 8) == L.SQ_ERR_ALIGNMENT
+    assert fwd(q=None) == L.SQ_ERR_INVALID_ARG
+    assert fwd(M=0) == L.SQ_OK
+
+
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
