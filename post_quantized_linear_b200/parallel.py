@@ -40,6 +40,18 @@ def calibrate_sharded(x_local: torch.Tensor, kseg: Sequence[int], group=None,
     return s_pos, s_neg
 
 
+def calibrate_hadamard_sharded(x_local: torch.Tensor, kseg: Sequence[int], group=None,
+                               stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The same for the block-Hadamard variant: the transform acts within each
+    row (blocks of 16 along K), so each rank's scales of its own rows of XH
+    all-reduce with MAX to the scales of all rows of XH."""
+    from . import calibrate_hadamard
+    s_pos, s_neg = calibrate_hadamard(x_local, kseg, stream=stream)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        allreduce_scales_(s_pos, s_neg, group)
+    return s_pos, s_neg
+
+
 def shard_rows(M: int, rank: int, world: int) -> Tuple[int, int]:
     """Contiguous row range [r0, r1) of X owned by `rank` (balanced to one row)."""
     base, extra = divmod(M, world)

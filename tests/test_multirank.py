@@ -2,7 +2,8 @@
 
 Each rank calibrates its own rows (with the oracle, on the CPU), the scales are
 all-reduced with MAX by the product helper, and the result must equal the
-oracle's calibration over all rows bit for bit (fp32 rounding is monotone)."""
+oracle's calibration over all rows bit for bit (fp32 rounding is monotone);
+the same for the scales of the block-Hadamard-transformed rows."""
 import os
 import socket
 
@@ -38,6 +39,11 @@ def _worker(rank, world, port, result_dir):
         tp, tn = torch.from_numpy(sp.copy()), torch.from_numpy(sn.copy())
         allreduce_scales_(tp, tn)
         np.save(os.path.join(result_dir, f"r{rank}.npy"), np.stack([tp.numpy(), tn.numpy()]))
+        # the block-Hadamard variant: scales of this rank's rows of XH
+        hp, hn = O.calibrate_hadamard(np.ascontiguousarray(xn[r0:r1]), wl.kseg)
+        tp, tn = torch.from_numpy(hp.copy()), torch.from_numpy(hn.copy())
+        allreduce_scales_(tp, tn)
+        np.save(os.path.join(result_dir, f"h{rank}.npy"), np.stack([tp.numpy(), tn.numpy()]))
     finally:
         dist.destroy_process_group()
 
@@ -53,10 +59,14 @@ def test_sharded_calibration_equals_full_calibration(tmp_path):
                       x_dtype="bf16")
     x, _, _ = W.generate(wl)
     sp, sn = O.calibrate(W.to_numpy_x(x), wl.kseg)
+    hp, hn = O.calibrate_hadamard(W.to_numpy_x(x), wl.kseg)
     for r in range(world):
         got = np.load(tmp_path / f"r{r}.npy")
         np.testing.assert_array_equal(got[0], sp)
         np.testing.assert_array_equal(got[1], sn)
+        goth = np.load(tmp_path / f"h{r}.npy")
+        np.testing.assert_array_equal(goth[0], hp)
+        np.testing.assert_array_equal(goth[1], hn)
 
 
 @pytest.mark.parametrize("M,world", [(10, 3), (8192, 8), (5, 8), (1, 2)])
