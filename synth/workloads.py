@@ -7,8 +7,13 @@ the quantization arithmetic, so both the CUDA path and the CPU oracle can take
 their inputs from it.
 
 Readings of the workload text (stated once, used everywhere):
-  * N(mu, v): the second parameter is a standard deviation (torch.normal
-    convention).  "N(0,25)" therefore means sigma = 5 and "N(0,400)" sigma = 20.
+  * N(mu, v): for the unit-normal pre-activations and the weight and bias
+    draws (N(0,1), N(0,0.02), N(0,0.05), N(0,0.01)) the second parameter is
+    the standard deviation (the usual initialization convention); the two
+    perfect squares -- the timestep-feature segment N(0,25) and the outliers
+    N(0,400) -- are read as variances, sigma = 5 and sigma = 20.  A literal
+    standard-deviation reading of those two (sigma = 25, 400) would change the
+    value spread only, not the work or the parity checks.
   * GELU is the exact (erf) GELU.
   * Activations are produced in fp32 by the activation function and then
     rounded once to the storage dtype (bf16 where the workload says bf16).
