@@ -302,28 +302,6 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t a0, uint32_t a1, uint32_
   return __byte_perm(__byte_perm(a0, a1, 0x0040), __byte_perm(a2, a3, 0x0040), 0x5410);
 }
 
-// DualScale rounding: the fma adds the exact product to 1.5*2^23, whose fp32
-// spacing is 1, so it rounds half to even to an integer (the offset is even,
-// so ties still go to even); fmin/fmax clamp to [0,127] / [-127,0] in the
-// float domain (monotone, so clamping commutes with the rounding).
-__device__ __forceinline__ void quantize16(const float (&v)[16], float rp, float rn, uint4& qp,
-                                           uint4& qn) {
-  uint32_t p[16], n[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    p[i] = __float_as_uint(fminf(fmaf(fmaxf(v[i], 0.0f), rp, kMagic), kMagic + 127.0f));
-    n[i] = __float_as_uint(fmaxf(fmaf(fminf(v[i], 0.0f), rn, kMagic), kMagic - 127.0f));
-  }
-  qp.x = low_bytes4(p[0], p[1], p[2], p[3]);
-  qp.y = low_bytes4(p[4], p[5], p[6], p[7]);
-  qp.z = low_bytes4(p[8], p[9], p[10], p[11]);
-  qp.w = low_bytes4(p[12], p[13], p[14], p[15]);
-  qn.x = low_bytes4(n[0], n[1], n[2], n[3]);
-  qn.y = low_bytes4(n[4], n[5], n[6], n[7]);
-  qn.z = low_bytes4(n[8], n[9], n[10], n[11]);
-  qn.w = low_bytes4(n[12], n[13], n[14], n[15]);
-}
-
 // Eight int4 codes (two per byte, low nibble = even k) -> eight int8 codes.
 // A nibble n in 0..15 sign-extends to n | 0xF0 when bit 3 is set: the bit,
 // multiplied by 30 (8 * 30 = 0xF0), lands in the high nibble of its own byte.
