@@ -2,14 +2,21 @@
 """Benchmark of the DualScale / SegLinear quantized linear layer on B200.
 
 One step = one pass of the whole path over one batch: static calibration on
-the workload's calibration rows, weight quantization, and the fused forward
-(in-kernel DualScale quantization, two int8 tensor-core GEMMs, fused
-epilogue).  The metric counts the executed int8 work of the forward, 4*M*N*K
-ops (two GEMMs, one per polarity), per second of step time.
+the workload's calibration rows, weight quantization, and the forward.  With
+the default `--path codes` the forward writes the DualScale codes q+/q- once
+and runs the GEMM from codes (two int8 tensor-core products per k step, fused
+epilogue); `--path fused` quantizes inside the GEMM, `--path combined` goes
+through the combined code.  The metric counts the executed int8 work of the
+forward, 4*M*N*K ops (two products, one per polarity), per second of step
+time.  The same line reports the dominant kernel against its roofline, the
+fused, single-scale and (int4 weights) block-Hadamard forwards beside it, the
+small-M forwards, the end-to-end rate through the API with host buffers, and
+the CPU oracle on the host cores.
 
-Timing: W warm-up steps, then K timed steps on the device with CUDA events on
-the launching stream; a 256 MiB buffer is written between timed steps (outside
-the events) so that every step starts from a cold L2.  Under torchrun each rank
+Timing: W warm-up steps, then K timed steps (each one CUDA-graph replay) on
+the device with CUDA events on the launching stream; before every timed
+launch the L2 is flushed (a 256 MiB write, then a 256 MiB read, outside the
+events) so that every step starts from a cold L2.  Under torchrun each rank
 runs its own batch (independent problems, no collective on the data path), the
 per-rank time is the max over ranks, and the value is the whole-job rate.
 
@@ -47,11 +54,11 @@ NCU_TRAFFIC_BYTES = {
 
 
 def gemm_kernel_name(path: str, bits: int, x_dtype: str) -> str:
-    """The GEMM kernel a forward of this path launches."""
+    """The GEMM kernel a forward of this path launches (default switches)."""
+    if path == "codes":          # int8 and int4 weights alike
+        return "dualscale_gemm_codes_kernel"
     if bits == 4:
         return "dualscale_gemm_kernel"
-    if path == "codes":
-        return "dualscale_gemm_codes_kernel"
     if path == "combined":
         return "dualscale_gemm_combined_kernel"
     return "dualscale_gemm_inplace_kernel" if x_dtype == "bf16" else "dualscale_gemm_kernel"
