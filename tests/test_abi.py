@@ -27,6 +27,20 @@ def test_library_exports_every_declared_entry_point():
         assert n in _lib.SIGNATURES, n
 
 
+def test_binding_arity_matches_every_declaration():
+    """Each prototype in include/segquant.h takes as many parameters as the
+    ctypes signature the binding gives it (guards the two against drift)."""
+    src = open(os.path.join(ROOT, "include", "segquant.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    protos = re.findall(r"\b(?:sq_status|const char\s*\*|void)\s+(sq_[a-z_0-9]+)\s*\(([^)]*)\)\s*;",
+                        src)
+    assert len(protos) == len(declared_functions())
+    for name, params in protos:
+        params = params.strip()
+        n = 0 if params in ("", "void") else len([p for p in params.split(",") if p.strip()])
+        assert len(_lib.SIGNATURES[name][1]) == n, name
+
+
 def test_status_strings():
     assert _lib.status_string(0) == "SQ_OK"
     assert _lib.status_string(6) == "SQ_ERR_TIMEOUT"
