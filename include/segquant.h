@@ -309,7 +309,9 @@ sq_status sq_splitk_workspace_size(int64_t M, int64_t N, int64_t K, size_t* byte
  * cudaMalloc, cudaFree or allocating library routine).
  * Set-up: the first call on each device, with that device current, looks up
  * the array's address (cudaGetSymbolAddress); make that first call before any
- * stream capture.
+ * stream capture.  The look-up runs again on the first call after the
+ * device's context has been re-created (cudaDeviceReset), since the array
+ * then lives at a new address.
  * Zeroing: every call clears the array's arrival counters itself
  * (cudaMemsetAsync on `stream`) before its kernel; the partial sums need no
  * clearing.

@@ -405,18 +405,50 @@ bool plan_splitk_capped(int64_t M, int64_t N, int64_t K, size_t cap, SplitPlan* 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
+// Id of the calling thread's current CUDA context, 0 when there is none (or
+// it cannot be read).  Context ids are unique for the life of the process, so
+// a context re-created on the same device (after cudaDeviceReset) has a new id.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_splitk_scratch in the current device's context: looked
+// up with cudaGetSymbolAddress on the first call per device and again whenever
+// the device's context has changed since (the array lives in the context's
+// copy of the module).
 sq_status static_scratch(void** out) {
   int dev = 0;
   sq_status st = cuda_status(cudaGetDevice(&dev));
   if (st != SQ_OK) return st;
   if (dev < 0 || dev >= kMaxDevices) return SQ_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     st = cuda_status(cudaGetSymbolAddress(&p, g_splitk_scratch));
     if (st != SQ_OK) return st;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();   // the lookup made the context current
   }
   *out = g_scratch_ptr[dev];
   return SQ_OK;

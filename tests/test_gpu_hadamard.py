@@ -13,7 +13,7 @@ import oracle as O
 from synth import workloads as W
 
 from parity_util import (Case, assert_bf16_within_1ulp, assert_f32_within, bf16_bits,
-                         magnitude_sum, sample_rows)
+                         magnitude_sum)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +72,9 @@ CASES = [
     dict(M=257, K=1152, N=128, kseg=[0, 128, 640, 1152], x_sigmas=[1.0, 3.0, 0.5],
          x_dtype="bf16", out="f32"),
     dict(M=16, K=3072, N=1024, kseg=[0, 3072], x_dtype="bf16", out="bf16"),
+    # several row tiles and output tiles (ragged both ways), fp32 out: bit-exact
+    dict(M=300, K=1024, N=400, kseg=[0, 512, 1024], x_sigmas=[1.0, 4.0], x_dtype="bf16",
+         out="f32"),
 ]
 
 
@@ -105,10 +108,10 @@ def test_hadamard_forward_matches_oracle(i):
     h.compare_rows(y, np.arange(h.wl.M))
 
 
-def test_hadamard_full_size_sampled_rows():
+def test_hadamard_full_size_every_row():
     """The W4A8 workload (M = 16384, K = N = 3072) in the bench's launch
-    configuration: bit-exact scales, codes and rotated weights, sampled rows
-    against the oracle."""
+    configuration: bit-exact scales, every XH code and the rotated weights;
+    every output row against the oracle (in chunks of rows)."""
     import post_quantized_linear_b200 as pq
     h = HCase(W.WORKLOADS["w4a8"])
     y = h.forward()
@@ -116,13 +119,14 @@ def test_hadamard_full_size_sampled_rows():
     assert pq.stream_status() == 0
     np.testing.assert_array_equal(h.sp.cpu().numpy(), h.o_sp)
     np.testing.assert_array_equal(h.sn.cpu().numpy(), h.o_sn)
-    rows = sample_rows(h.wl.M, 64)
-    op, on = O.quantize_activations_hadamard(np.ascontiguousarray(h.c.x_np[rows]), h.wl.kseg,
-                                             h.o_sp, h.o_sn)
-    idx = torch.as_tensor(rows, device="cuda")
-    np.testing.assert_array_equal(h.qp[idx].cpu().numpy(), op)
-    np.testing.assert_array_equal(h.qn[idx].cpu().numpy(), on)
-    h.compare_rows(y, rows)
+    chunk = 2048
+    for r0 in range(0, h.wl.M, chunk):
+        rows = np.arange(r0, min(h.wl.M, r0 + chunk))
+        op, on = O.quantize_activations_hadamard(np.ascontiguousarray(h.c.x_np[rows]), h.wl.kseg,
+                                                 h.o_sp, h.o_sn)
+        np.testing.assert_array_equal(h.qp[r0:r0 + len(rows)].cpu().numpy(), op)
+        np.testing.assert_array_equal(h.qn[r0:r0 + len(rows)].cpu().numpy(), on)
+        h.compare_rows(y, rows)
 
 
 def test_hadamard_starved_pipeline_times_out_and_context_recovers():

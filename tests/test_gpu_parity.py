@@ -278,6 +278,24 @@ def test_forward_exact_in_fp32():
     np.testing.assert_array_equal(y, y_ref)
 
 
+@pytest.mark.parametrize("i", [7, 8])
+def test_int4_forward_exact_in_fp32(i):
+    """int4 weights (one unit per 128-wide group, seeded accumulators) with
+    fp32 outputs on several row and output tiles: the fused forward and the
+    GEMM from codes reproduce the oracle bit for bit (the fixed fp32 order)."""
+    import post_quantized_linear_b200 as pq
+    c = Case(_small(i))
+    assert c.wl.bits == 4 and c.wl.out == "f32"
+    y = c.forward()
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    y2 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    y_ref, _ = c.oracle_rows(np.arange(c.wl.M))
+    np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+    np.testing.assert_array_equal(y2.cpu().numpy(), y_ref)
+
+
 def test_nonnegative_input_and_zero_rows():
     import post_quantized_linear_b200 as pq
     wl = W.small_case(200, 256, 128, seed=3, act="none", bias=True, out="f32")
@@ -334,23 +352,29 @@ def test_strided_activations_and_outputs():
 
 @pytest.mark.parametrize("name", ["tiny_w8a8", "dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up",
                                   "w4a8"])
-def test_workloads_full_size_sampled_rows(name):
-    """Full-size workloads in the bench's launch configuration: bit-exact scales
-    and weights everywhere; outputs of sampled rows against the oracle."""
+def test_workloads_full_size_every_row(name):
+    """Full-size workloads in the bench's launch configuration: bit-exact
+    scales, weights and every DualScale code; every output row of the fused
+    forward against the oracle (rows in chunks, so host memory stays bounded);
+    the two-pass path (codes, then the GEMM from codes) bit-identical to it."""
+    import post_quantized_linear_b200 as pq
     wl = W.WORKLOADS[name]
     c = Case(wl)
     c.check_scales_and_weights()
     y = c.forward()
-    torch.cuda.synchronize()
-    rows = np.arange(wl.M) if wl.M <= 256 else sample_rows(wl.M, 96 if wl.N > 4096 else 160)
-    c.compare_rows(y, rows)
-    import post_quantized_linear_b200 as pq
-    assert pq.stream_status() == 0
-    # the two-pass path (codes, then the GEMM from codes) gives the same bits
     qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
     y2 = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
-    assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32),
-                       y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2.view(torch.int32))
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    iv = torch.int16 if y.dtype == torch.bfloat16 else torch.int32
+    assert torch.equal(y.view(iv), y2.view(iv))
+    chunk = 2048
+    for r0 in range(0, wl.M, chunk):
+        rows = np.arange(r0, min(wl.M, r0 + chunk))
+        op, on = O.quantize_activations(np.ascontiguousarray(c.x_np[rows]), wl.kseg, c.o_sp, c.o_sn)
+        np.testing.assert_array_equal(qp[r0:r0 + len(rows)].cpu().numpy(), op)
+        np.testing.assert_array_equal(qn[r0:r0 + len(rows)].cpu().numpy(), on)
+        c.compare_rows(y, rows)
 
 
 # ------------------------------------------------------------- status word

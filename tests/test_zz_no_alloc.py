@@ -1,6 +1,12 @@
 """The allocation-free split-K entry point (library-owned static scratch),
-called through the C ABI: the same bits as the split-K entry point with a
-caller workspace and as the one-pass GEMM from codes, on two calls in a row.
+called through the C ABI.  It serves callers that cannot allocate device
+memory while they run: an inference loop that forbids allocation after
+start-up, or a process whose device memory is held by another allocator.
+
+Checks, on two calls in a row: the same bits as the split-K entry point with a
+caller workspace and as the one-pass GEMM from codes; the oracle's result
+(fp32 bit-exact, bf16 within one ulp); and no device memory allocated by the
+call (torch's allocator and the device's free memory unchanged across it).
 Collected last; passes alone in a fresh process and after the other tests."""
 import ctypes
 
@@ -8,7 +14,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from synth import workloads as W
+
+from parity_util import assert_bf16_within_1ulp, bf16_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -52,13 +61,28 @@ def test_static_scratch_splitk_matches_existing_entry_points(M, K, N, out):
     ws = pq.splitk_workspace(M, N, K, device=dev)
     ref_ws = pq.linear_from_codes_splitk(qp, qn, qw, sp, sn, ws, bd, out_dtype=odt)
     ref = pq.linear_from_codes(qp, qn, qw, sp, sn, bd, out_dtype=odt)
-    for _ in range(2):                      # two calls in a row share the scratch
+    O.build()
+    xn = W.to_numpy_x(x)
+    o_sp, o_sn = O.calibrate(xn, wl.kseg)
+    o_wc, o_ws = O.quantize_weights_w8(w.numpy(), wl.kseg)
+    y_ref = O.linear_forward(xn, wl.kseg, o_sp, o_sn, 8, o_wc, o_ws, b.numpy(), out=out)
+    for call in range(2):                   # two calls in a row share the scratch
         y = torch.full((M, N), 3.0, dtype=odt, device=dev)
+        torch.cuda.synchronize()
+        torch_before = torch.cuda.memory_allocated(dev)
+        free_before = torch.cuda.mem_get_info(dev)[0]
         assert _static_call(qp, qn, qw, sp, sn, bd, y) == _lib.SQ_OK
         torch.cuda.synchronize()
+        if call == 1:                       # the first call may load the library's module
+            assert torch.cuda.memory_allocated(dev) == torch_before
+            assert torch.cuda.mem_get_info(dev)[0] == free_before
         assert pq.stream_status() == _lib.SQ_OK
         assert torch.equal(_bits(y), _bits(ref_ws))
         assert torch.equal(_bits(y), _bits(ref))
+        if out == "f32":
+            np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+        else:
+            assert_bf16_within_1ulp(bf16_bits(y), y_ref)
 
 
 def test_static_scratch_rejects_sizes_beyond_the_maximum():
