@@ -2,26 +2,34 @@
 """Benchmark of the DualScale / SegLinear quantized linear layer on B200.
 
 One step = one pass of the whole path over one batch: static calibration on
-the workload's calibration rows, weight quantization, and the forward.  With
-the default `--path codes` the forward writes the DualScale codes q+/q- once
-and runs the GEMM from codes (two int8 tensor-core products per k step, fused
-epilogue); `--path fused` quantizes inside the GEMM, `--path combined` goes
-through the combined code.  The metric counts the executed int8 work of the
-forward, 4*M*N*K ops (two products, one per polarity), per second of step
-time.  The same line reports the dominant kernel against its roofline, the
-fused, single-scale and (int4 weights) block-Hadamard forwards beside it, the
-small-M forwards, the end-to-end rate through the API with host buffers, and
-the CPU oracle on the host cores.
+the workload's calibration rows (token-sharded across ranks: each rank
+calibrates its own rows and the 2*J scales are all-reduced with MAX), weight
+quantization, and the forward.  With the default `--path codes` the forward
+writes the DualScale codes q+/q- once and runs the GEMM from codes (two int8
+tensor-core products per k step, fused epilogue); `--path fused` quantizes
+inside the GEMM, `--path combined` goes through the combined code.  The metric
+counts the executed int8 work of the forward, 4*M*N*K ops (two products, one
+per polarity), per second of step time.
 
-Timing: W warm-up steps, then K timed steps (each one CUDA-graph replay) on
-the device with CUDA events on the launching stream; before every timed
-launch the L2 is flushed (a 256 MiB write, then a 256 MiB read, outside the
-events) so that every step starts from a cold L2.  Under torchrun each rank
-runs its own batch (independent problems, no collective on the data path), the
-per-rank time is the max over ranks, and the value is the whole-job rate.
+The default workload is the largest one that fits one GPU, the MMDiT MLP
+up-projection (M = 16384, K = 3072, N = 12288).  The same JSON line reports the
+dominant kernel against its roofline, the fused, single-scale and (int4
+weights) block-Hadamard forwards beside it, every workload configuration
+(`configs`: GEMM, forward and step times with their roofline fractions), the
+small-M forwards, the host latency of one call, the end-to-end rate through
+the API with host buffers, and the CPU oracle on the host cores.
+
+Timing: W warm-up steps, then K timed steps on the device with CUDA events on
+the launching stream; before every timed step the L2 is flushed (a 256 MiB
+write, then a 256 MiB read, outside the events) so that every step starts from
+a cold L2.  `--gpus N` runs N ranks (one process per GPU, launched through
+torch.distributed.run when WORLD_SIZE is not set); each rank runs its own batch
+(independent problems), the step time is the max over ranks, and the value is
+the whole-job rate.
 
 `--impl reference` times the CPU oracle (the plain C implementation in
-oracle/) on the host cores, on a bounded row sample of the same workload.
+oracle/) on the host cores, each step on a bounded sample of the workload's
+rows.
 """
 from __future__ import annotations
 
@@ -29,6 +37,7 @@ import argparse
 import datetime
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -40,16 +49,21 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "quantized-linear int8 TOPS and % of B200 int8 tensor peak (GB/s at small M)"
+DEFAULT_WORKLOAD = "mmdit_mlp_up"
+CONFIG_ORDER = ("tiny_w8a8", "dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up", "w4a8")
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
+# tcgen05.mma.kind::i8 with M = 128 and N >= 128 completes 8192 int8 MACs per
+# clock per SM (measured with an issue-rate probe on this machine's B200s):
+# 16384 int8 ops per clock per SM.
+MMA_I8_OPS_PER_CLK_SM = 16384
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
     ("dit_xl2_fc2_cfg", "codes"): 93068032 + 11148288,   # dualscale_gemm_codes_kernel
-    ("w4a8", "codes"): 105879296 + 71072768,             # dualscale_gemm_codes_kernel (W4)
 }
 
 
@@ -64,13 +78,13 @@ def gemm_kernel_name(path: str, bits: int, x_dtype: str) -> str:
     return "dualscale_gemm_inplace_kernel" if x_dtype == "bf16" else "dualscale_gemm_kernel"
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="dit_xl2_fc2_cfg")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--path", choices=["fused", "codes", "combined"], default="codes",
                     help="fused: quantize X inside the GEMM; codes: quantize X once into "
                          "q+/q- code tensors, then the GEMM loads the codes; combined: quantize "
@@ -79,15 +93,20 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration table (every workload's GEMM/forward/step)")
     ap.add_argument("--no-small-m", action="store_true",
                     help="skip the small-M (M <= 128, HBM-bound) measurements")
     ap.add_argument("--small-m-only", action="store_true",
                     help="run only the small-M measurements (one GPU) and print them as one "
                          "JSON line; not a bench line")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
+    """(int8 TOPS denominator, HBM GB/s, source): the measured bf16 burst
+    figure times the nominal int8/bf16 ratio and the measured copy bandwidth,
+    else the recipe's fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
@@ -95,6 +114,62 @@ def peaks():
         return float(p["bf16_tflops"]) * INT8_PER_BF16, float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_BF16_TFLOPS * INT8_PER_BF16, FALLBACK_HBM_GBS, "fallback"
+
+
+def mma_rate_tops(sms: int, sm_mhz: float) -> float:
+    """The tcgen05 int8 MMA issue rate of `sms` SMs at `sm_mhz` (TOPS)."""
+    return MMA_I8_OPS_PER_CLK_SM * sms * sm_mhz * 1e6 / 1e12
+
+
+# ------------------------------------------------------------ rank launch
+def free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def rank_env():
+    """(world, rank, local rank) from the torch.distributed launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def relaunch_command(argv, gpus: int, port: int):
+    """The torch.distributed.run command that starts `gpus` ranks of this script."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def check_world(gpus: int):
+    """None when the launch matches --gpus; else the reason it does not."""
+    if "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) != gpus:
+        return f"WORLD_SIZE={os.environ['WORLD_SIZE']} but --gpus {gpus}"
+    return None
+
+
+def max_over_ranks(vals, world: int, device):
+    """Element-wise max of a list of floats over the ranks (identity at world 1)."""
+    if world == 1:
+        return list(vals)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def rank_workload(wl, rank: int):
+    """The batch of rank r: the workload drawn with seed + r (independent problems)."""
+    import dataclasses
+    return dataclasses.replace(wl, seed=wl.seed + rank)
+
+
+def whole_job_tops(world: int, steps: int, ops: int, total_ms: float) -> float:
+    """Executed int8 TOPS of the whole job: every rank's steps over the slowest rank's time."""
+    return world * steps * ops / (total_ms * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------ L2 flush
@@ -113,6 +188,36 @@ class L2Flush:
     def __call__(self, i: int):
         self.a.fill_(i & 0xFF)
         self.b.max()
+
+
+def timed_graph(graph, n: int, salt: int, flush, stream):
+    """Device times (ms) of n replays, each after an L2 flush, CUDA events on `stream`."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for i in range(n):
+        flush(i + salt)
+        evs[i][0].record(stream)
+        graph.replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def capture(fn):
+    """fn captured once into a CUDA graph (after one run on a side stream)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    torch.cuda.synchronize()
+    return graph
 
 
 # ------------------------------------------------------------------ small M
@@ -136,6 +241,7 @@ def small_m_measure(dev, flush, steps: int, hbm_peak: float):
     import torch
     import post_quantized_linear_b200 as pq
     from synth import workloads as W
+    stream = torch.cuda.current_stream()
     out = []
     for (K, N) in SMALL_M_SHAPES:
         for M in SMALL_M_ROWS:
@@ -148,24 +254,11 @@ def small_m_measure(dev, flush, steps: int, hbm_peak: float):
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = pq.splitk_workspace(M, N, K, device=dev)
             res = {"M": M, "K": K, "N": N}
+            byts = N * K + 4 * N + 2 * M * K + 2 * M * N
             for name, fn in (("splitk", lambda: pq.linear_from_codes_splitk(qp, qn, qw, sp, sn, ws, out=y)),
                              ("one_pass", lambda: pq.linear_from_codes(qp, qn, qw, sp, sn, out=y))):
-                fn()
-                torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    fn()
-                ts = []
-                for i in range(max(steps, 5)):
-                    flush(i)
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record()
-                    g.replay()
-                    e1.record()
-                    torch.cuda.synchronize()
-                    ts.append(e0.elapsed_time(e1))
-                us = statistics.median(ts) * 1e3
-                byts = N * K + 4 * N + 2 * M * K + 2 * M * N
+                g = capture(fn)
+                us = statistics.median(timed_graph(g, max(steps, 5), 0, flush, stream)) * 1e3
                 res[name] = {"us": us, "gbs": byts / (us * 1e-6) / 1e9,
                              "frac_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
                 del g
@@ -176,27 +269,49 @@ def small_m_measure(dev, flush, steps: int, hbm_peak: float):
             def layers():
                 for q_l, y_l in zip(qws, ys):
                     pq.linear_from_codes(qp, qn, q_l, sp, sn, out=y_l)
-            layers()
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                layers()
-            ts = []
-            for i in range(max(steps, 5)):
-                flush(i)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                g.replay()
-                e1.record()
-                torch.cuda.synchronize()
-                ts.append(e0.elapsed_time(e1))
-            us = statistics.median(ts) * 1e3 / len(qws)
+            g = capture(layers)
+            us = statistics.median(timed_graph(g, max(steps, 5), 0, flush, stream)) * 1e3 / len(qws)
             res["one_pass_layers"] = {"layers": len(qws), "us_per_layer": us,
                                       "gbs": byts / (us * 1e-6) / 1e9,
                                       "frac_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
             del g, qws, ys
             out.append(res)
     return out
+
+
+def per_call_measure(dev, calls: int = 200):
+    """Host cost of one forward call outside a CUDA graph, the cost a small-M
+    caller pays: the GEMM from codes at M = 16, (K, N) = (3072, 12288), called
+    `calls` times back to back.  host_us: time for the API call to return
+    (argument marshalling, validation, tensor-map encoding, launch); eager_us:
+    device time per call of the back-to-back eager launches."""
+    import torch
+    import post_quantized_linear_b200 as pq
+    from synth import workloads as W
+    M, K, N = 16, 3072, 12288
+    wl = W.small_case(M, K, N, seed=7, act="silu", bias=False, out="bf16")
+    x, w, _ = W.generate(wl)
+    xd, wd = x.to(dev), w.to(dev)
+    sp, sn = pq.calibrate(xd, wl.kseg)
+    qw = pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=8)
+    qp, qn = pq.quantize_activations(xd, wl.kseg, sp, sn)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for _ in range(10):
+        pq.linear_from_codes(qp, qn, qw, sp, sn, out=y)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        pq.linear_from_codes(qp, qn, qw, sp, sn, out=y)
+    t1 = time.perf_counter()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"M": M, "K": K, "N": N, "calls": calls,
+            "host_us": (t1 - t0) / calls * 1e6,
+            "eager_us": e0.elapsed_time(e1) / calls * 1e3,
+            "note": "sq_linear_forward_codes through the Python binding, outside a CUDA graph"}
 
 
 # ------------------------------------------------------------------ clocks
@@ -263,52 +378,60 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle
-def cpu_oracle_step(wl, xn, wn, bn, rows):
-    """One oracle step on a row sample; returns (seconds, seconds scaled to the full batch)."""
+def oracle_step(wl, xn, wn, bn, rows: int):
+    """One oracle step on a sample: calibration on the workload's calibration
+    rows, quantization of the whole weight, forward of the first `rows` rows.
+    Returns (seconds, executed int8 ops of the sampled forward)."""
     import numpy as np
     import oracle as O
     t0 = time.perf_counter()
     calib = xn if wl.calib_rows is None else xn[: wl.calib_rows]
     sp, sn = O.calibrate(calib, wl.kseg)
-    t1 = time.perf_counter()
     if wl.bits == 8:
         wc, ws = O.quantize_weights_w8(wn, wl.kseg)
     else:
         wc, ws = O.quantize_weights_w4(wn)
-    t2 = time.perf_counter()
     O.linear_forward(np.ascontiguousarray(xn[:rows]), wl.kseg, sp, sn, wl.bits, wc, ws, bn,
                      out="f32" if wl.out == "f32" else "bf16")
-    t3 = time.perf_counter()
-    return t3 - t0, (t2 - t0) + (t3 - t2) * (wl.M / rows)
+    return time.perf_counter() - t0, 4 * rows * wl.N * wl.K
+
+
+def oracle_sample_rows(wl, xn, wn, bn, step_budget_s: float) -> int:
+    """Rows of the sampled forward that keep one oracle step near the budget."""
+    t8, _ = oracle_step(wl, xn, wn, bn, 8)
+    t16, _ = oracle_step(wl, xn, wn, bn, 16)
+    per_row = max((t16 - t8) / 8, 1e-7)
+    fixed = max(t8 - 8 * per_row, 0.0)
+    return int(max(8, min(wl.M, (step_budget_s - fixed) / per_row)))
+
+
+def host_threads() -> int:
+    cores = len(os.sched_getaffinity(0))
+    return int(os.environ.get("OMP_NUM_THREADS", cores))
 
 
 def cpu_baseline(wl, x, w, b, target_s=12.0):
-    import numpy as np
+    """The oracle, as it stands, timed on the host cores on a bounded sample."""
     import oracle as O
     from synth import workloads as W
     O.build()
     xn, wn = W.to_numpy_x(x), w.numpy()
     bn = None if b is None else b.numpy()
-    probe_rows = 8
-    t_probe, _ = cpu_oracle_step(wl, xn, wn, bn, probe_rows)
-    per_row = max(t_probe / probe_rows, 1e-6)
-    rows = int(max(8, min(wl.M, target_s / per_row)))
-    t, t_full = cpu_oracle_step(wl, xn, wn, bn, rows)
-    cores = len(os.sched_getaffinity(0))
-    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    rows = oracle_sample_rows(wl, xn, wn, bn, target_s)
+    t, ops = oracle_step(wl, xn, wn, bn, rows)
     return {
-        "value": wl.exec_ops / t_full / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
-        "sample": (f"calibration on the full calibration rows, weight quantization of the full "
-                   f"[{wl.N},{wl.K}] weight, forward of {rows}/{wl.M} rows ({t:.1f} s); "
-                   "forward time scaled by M/rows"),
+        "value": ops / t / 1e12, "unit": "TOPS", "cores": host_threads(), "kind": "oracle",
+        "sample": (f"one step: calibration on the workload's calibration rows, quantization of "
+                   f"the whole [{wl.N},{wl.K}] weight, forward of {rows}/{wl.M} rows; "
+                   f"{t:.2f} s measured; value = executed ops of the sampled forward / step time"),
     }
 
 
 def run_reference(args):
-    """The reference arm: the CPU oracle, as it stands, on the host cores."""
-    import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    """The reference arm: the CPU oracle, as it stands, on the host cores; each
+    step a bounded sample of the workload's rows, sized so that the whole run
+    stays within a few minutes.  Every number is measured (no scaling)."""
+    world, rank, _ = rank_env()
     if rank != 0:
         return 0
     from synth import workloads as W
@@ -320,30 +443,26 @@ def run_reference(args):
     bn = None if b is None else b.numpy()
     steps, warm = args.steps, args.warmup
     budget_s = 150.0
-    t_probe, _ = cpu_oracle_step(wl, xn, wn, bn, 8)
-    per_row = max(t_probe / 8, 1e-6)
-    rows = int(max(8, min(wl.M, budget_s / (steps + warm) / per_row)))
+    rows = oracle_sample_rows(wl, xn, wn, bn, budget_s / max(1, steps + warm))
     for _ in range(warm):
-        cpu_oracle_step(wl, xn, wn, bn, rows)
-    full = []
-    raw = []
+        oracle_step(wl, xn, wn, bn, rows)
+    ts = []
+    ops = 0
     for _ in range(steps):
-        t, tf = cpu_oracle_step(wl, xn, wn, bn, rows)
-        raw.append(t)
-        full.append(tf)
-    t_step = sum(full) / len(full)
-    value = wl.exec_ops / t_step / 1e12
-    cores = len(os.sched_getaffinity(0))
-    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
-    sample = (f"each step: calibration on the calibration rows, full weight quantization, "
-              f"forward of {rows}/{wl.M} rows (mean {sum(raw)/len(raw):.2f} s); forward time "
-              "scaled by M/rows")
+        t, ops = oracle_step(wl, xn, wn, bn, rows)
+        ts.append(t)
+    total = sum(ts)
+    value = steps * ops / total / 1e12 if steps else 0.0
+    sample = (f"each step: calibration on the workload's calibration rows, quantization of the "
+              f"whole [{wl.N},{wl.K}] weight, forward of {rows}/{wl.M} rows; value = executed "
+              "ops of the sampled forwards / measured step time")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
-        "steps": steps, "warmup": warm, "ms_per_step": t_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": config_of(wl, "host cores, no L2 flush", "oracle"),
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
+        "steps": steps, "warmup": warm, "ms_per_step": total / max(1, steps) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": config_of(wl, "host cores, no L2 flush", "oracle", world, sample_rows=rows),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": host_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -351,157 +470,222 @@ def run_reference(args):
     return 0
 
 
-def config_of(wl, l2, path="fused"):
-    return {"workload": wl.name, "path": path, "M": wl.M, "K": wl.K, "N": wl.N, "bits": wl.bits,
-            "x_dtype": wl.x_dtype, "out_dtype": wl.out, "k_segments": list(wl.kseg),
-            "n_segments": list(wl.nseg), "calib_rows": wl.calib_rows or wl.M,
-            "global_batch": wl.M, "l2": l2}
+def config_of(wl, l2, path="codes", world=1, sample_rows=None):
+    c = {"workload": wl.name, "path": path, "M": wl.M, "K": wl.K, "N": wl.N, "bits": wl.bits,
+         "x_dtype": wl.x_dtype, "out_dtype": wl.out, "k_segments": list(wl.kseg),
+         "n_segments": list(wl.nseg), "calib_rows": wl.calib_rows or wl.M,
+         "global_batch": wl.M * world, "l2": l2, "parallelism": f"dp{world}"}
+    if sample_rows is not None:
+        c["sample_rows"] = sample_rows
+    return c
 
 
 # ------------------------------------------------------------- GPU arm
+class Layer:
+    """One workload's device state and its captured CUDA graphs.
+
+    step():      calibration (token-sharded: local calibration, then the MAX
+                 all-reduce of the scales when several ranks run) followed by
+                 `rest`, one graph replay of weight quantization + forward;
+    fwd_graph:   activation codes + the GEMM (the forward alone);
+    gemm_graph:  the GEMM alone (the dominant kernel)."""
+
+    def __init__(self, wl, dev, path: str, rank: int = 0, extras: bool = True):
+        import torch
+        import post_quantized_linear_b200 as pq
+        from synth import workloads as W
+        self.wl, self.dev, self.path = wl, dev, path
+        x, w, b = W.generate(rank_workload(wl, rank))
+        self.x_host, self.w_host = x, w
+        self.xd, self.wd = x.to(dev), w.to(dev)
+        self.bd = None if b is None else b.to(dev)
+        self.out_dtype = torch.float32 if wl.out == "f32" else torch.bfloat16
+        J = len(wl.kseg) - 1
+        self.sp = torch.empty(J, dtype=torch.float32, device=dev)
+        self.sn = torch.empty(J, dtype=torch.float32, device=dev)
+        self.qw = pq.quantize_weights(self.wd, wl.kseg, wl.nseg, bits=wl.bits)
+        self.y = torch.empty((wl.M, wl.N), dtype=self.out_dtype, device=dev)
+        self.calib = self.xd if wl.calib_rows is None else self.xd[: wl.calib_rows]
+        self.codes = path in ("codes", "combined")
+        self.combined = path == "combined"
+        ldq = (wl.K + 15) // 16 * 16
+        if self.codes:
+            self.qp = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
+            self.qn = (None if self.combined else
+                       torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K])
+        self.launches_per_step = 4 if self.codes else 3
+        self.calibrate()
+        torch.cuda.synchronize()
+        self.rest_graph = capture(self.rest)
+        self.fwd_graph = capture(lambda: self.forward(self.xd, self.y))
+        self.gemm_graph = capture(lambda: self.gemm(self.xd, self.y))
+        self.fused_graph = self.single_graph = self.had_graph = None
+        if not extras:
+            return
+        if self.codes:
+            self.fused_graph = capture(lambda: pq.linear(self.xd, self.qw, self.sp, self.sn,
+                                                         self.bd, out=self.y))
+        # the single-scale baseline (one symmetric scale per K segment): its
+        # codes, then one int8 product per unit
+        if wl.bits == 8:
+            self.c1 = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
+
+            def single_forward():
+                pq.quantize_activations_single(self.xd, wl.kseg, self.sp, self.sn, out=self.c1)
+                pq.linear_from_single(self.c1, self.qw, self.sp, self.sn, self.bd, out=self.y)
+            self.single_graph = capture(single_forward)
+        # int4 weights: the block-Hadamard variant (HQ-DM) of the same forward:
+        # codes of XH, then the product with the rotated int4 codes (its scales
+        # and the weight rotation are offline steps, made once here)
+        if wl.bits == 4:
+            self.hsp = torch.empty(J, dtype=torch.float32, device=dev)
+            self.hsn = torch.empty(J, dtype=torch.float32, device=dev)
+            pq.calibrate_hadamard(self.calib, wl.kseg, self.hsp, self.hsn)
+            self.w_rot = pq.rotate_weights_hadamard(self.qw)
+            self.hq_p = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
+            self.hq_n = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
+
+            def hadamard_forward():
+                pq.quantize_activations_hadamard(self.xd, wl.kseg, self.hsp, self.hsn,
+                                                 out=(self.hq_p, self.hq_n))
+                pq.linear_from_codes_hadamard(self.hq_p, self.hq_n, self.qw, self.w_rot, self.hsp,
+                                              self.hsn, self.bd, out=self.y)
+            self.had_graph = capture(hadamard_forward)
+
+    def calibrate(self, calib=None):
+        from post_quantized_linear_b200 import parallel
+        parallel.calibrate_sharded(self.calib if calib is None else calib, self.wl.kseg,
+                                   s_pos=self.sp, s_neg=self.sn)
+
+    def gemm(self, xs, ys):
+        import post_quantized_linear_b200 as pq
+        if self.combined:
+            pq.linear_from_combined(self.qp, self.qw, self.sp, self.sn, self.bd, out=ys)
+        elif self.codes:
+            pq.linear_from_codes(self.qp, self.qn, self.qw, self.sp, self.sn, self.bd, out=ys)
+        else:
+            pq.linear(xs, self.qw, self.sp, self.sn, self.bd, out=ys)
+
+    def forward(self, xs, ys):
+        import post_quantized_linear_b200 as pq
+        if self.combined:
+            pq.quantize_activations_combined(xs, self.wl.kseg, self.sp, self.sn, out=self.qp)
+        elif self.codes:
+            pq.quantize_activations(xs, self.wl.kseg, self.sp, self.sn, out=(self.qp, self.qn))
+        self.gemm(xs, ys)
+
+    def rest(self, xs=None, ws=None, ys=None):
+        import post_quantized_linear_b200 as pq
+        pq.quantize_weights(self.wd if ws is None else ws, self.wl.kseg, self.wl.nseg,
+                            bits=self.wl.bits, out=self.qw)
+        self.forward(self.xd if xs is None else xs, self.y if ys is None else ys)
+
+    def step(self):
+        self.calibrate()
+        self.rest_graph.replay()
+
+    def timed_steps(self, n: int, salt: int, flush, stream, world: int):
+        """Device times (ms) of n steps, each after an L2 flush; ranks enter each
+        step together."""
+        import torch
+        import torch.distributed as dist
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for i in range(n):
+            flush(i + salt)
+            evs[i][0].record(stream)
+            self.step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    def release(self):
+        self.rest_graph = self.fwd_graph = self.gemm_graph = None
+        self.fused_graph = self.single_graph = self.had_graph = None
+
+
+def measure_config(wl, dev, flush, steps: int, warmup: int, int8_peak: float, mma_peak: float,
+                   hbm_peak: float, path: str = "codes"):
+    """GEMM, forward and step times of one workload configuration (one GPU)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    L = Layer(wl, dev, path, extras=False)
+    for _ in range(warmup):
+        L.step()
+    torch.cuda.synchronize()
+    step_ms = statistics.mean(L.timed_steps(steps, 1, flush, stream, 1))
+    gemm_ms = statistics.mean(timed_graph(L.gemm_graph, steps, 3, flush, stream))
+    fwd_ms = statistics.mean(timed_graph(L.fwd_graph, steps, 5, flush, stream))
+    L.release()
+    ops, byts = wl.exec_ops, codes_gemm_bytes(wl)
+    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    # a problem of a few MB and tens of MFLOP is launch-latency bound, not tensor bound
+    bound = "latency" if byts < 16 * 2 ** 20 and ops < 10 ** 10 else "tensor"
+    return {
+        "M": wl.M, "K": wl.K, "N": wl.N, "bits": wl.bits, "k_segments": list(wl.kseg),
+        "gemm_us": gemm_ms * 1e3, "forward_us": fwd_ms * 1e3, "step_us": step_ms * 1e3,
+        "gemm_tops": gemm_tops, "step_tops": ops / (step_ms * 1e-3) / 1e12,
+        "roofline": {
+            "bound": bound, "kernel": gemm_kernel_name(path, wl.bits, wl.x_dtype),
+            "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+            "frac": gemm_tops / int8_peak, "frac_mma_rate": gemm_tops / mma_peak,
+            "traffic": NCU_TRAFFIC_BYTES.get((wl.name, path)),
+            "algorithmic_bytes_per_launch": byts,
+            "achieved_gbs": byts / (gemm_ms * 1e-3) / 1e9,
+            "frac_hbm": byts / (gemm_ms * 1e-3) / 1e9 / hbm_peak,
+        },
+    }
+
+
+def codes_gemm_bytes(wl) -> int:
+    """Algorithmic bytes of one launch of the GEMM from codes: q+ and q- codes,
+    weight codes and scales, activation scales, bias, Y."""
+    J = len(wl.kseg) - 1
+    ye = 4 if wl.out == "f32" else 2
+    if wl.bits == 8:
+        wb = wl.N * wl.K + 4 * J * wl.N
+    else:
+        wb = wl.N * wl.K // 2 + 2 * wl.N * (wl.K // 128)
+    bb = 4 * wl.N if wl.bias_sigma is not None else 0
+    return 2 * wl.M * wl.K + wb + 8 * J + bb + wl.M * wl.N * ye
+
+
+def num_sms(dev) -> int:
+    import torch
+    return torch.cuda.get_device_properties(dev).multi_processor_count
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
 
     import post_quantized_linear_b200 as pq
     from synth import workloads as W
 
+    int8_peak, hbm_peak, peak_kind = peaks()
     if args.small_m_only:
-        dev = torch.device("cuda", local)
-        hbm_peak = peaks()[1]
         print(json.dumps({"small_m": {"peak_gbs": hbm_peak, "cases": small_m_measure(
             dev, L2Flush(dev), args.steps, hbm_peak)}}), flush=True)
         return 0
 
     wl = W.WORKLOADS[args.workload]
-    import dataclasses
-    wl_rank = dataclasses.replace(wl, seed=wl.seed + rank)
-    x, w, b = W.generate(wl_rank)
-    dev = torch.device("cuda", local)
-    xd, wd = x.to(dev), w.to(dev)
-    bd = None if b is None else b.to(dev)
-    out_dtype = torch.float32 if wl.out == "f32" else torch.bfloat16
-    J = len(wl.kseg) - 1
-    sp = torch.empty(J, dtype=torch.float32, device=dev)
-    sn = torch.empty(J, dtype=torch.float32, device=dev)
-    qw = pq.quantize_weights(wd, wl.kseg, wl.nseg, bits=wl.bits)
-    y = torch.empty((wl.M, wl.N), dtype=out_dtype, device=dev)
-    calib = xd if wl.calib_rows is None else xd[: wl.calib_rows]
-    use_codes = args.path in ("codes", "combined")
-    combined = args.path == "combined"
-    if use_codes:
-        ldq = (wl.K + 15) // 16 * 16
-        qp_buf = torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
-        qn_buf = None if combined else torch.empty((wl.M, ldq), dtype=torch.int8, device=dev)[:, : wl.K]
     stream = torch.cuda.current_stream()
     flush = L2Flush(dev)
-
-    def step(xs=xd, ws=wd, ys=y, gemm_events=None):
-        pq.calibrate(calib if xs is xd else (xs if wl.calib_rows is None else xs[: wl.calib_rows]),
-                     wl.kseg, sp, sn)
-        pq.quantize_weights(ws, wl.kseg, wl.nseg, bits=wl.bits, out=qw)
-        forward(xs, ys, gemm_events)
-
-    def gemm(xs, ys):
-        if combined:
-            pq.linear_from_combined(qp_buf, qw, sp, sn, bd, out=ys)
-        elif use_codes:
-            pq.linear_from_codes(qp_buf, qn_buf, qw, sp, sn, bd, out=ys)
-        else:
-            pq.linear(xs, qw, sp, sn, bd, out=ys)
-
-    def forward(xs, ys, gemm_events=None):
-        if combined:
-            pq.quantize_activations_combined(xs, wl.kseg, sp, sn, out=qp_buf)
-        elif use_codes:
-            pq.quantize_activations(xs, wl.kseg, sp, sn, out=(qp_buf, qn_buf))
-        if gemm_events:
-            gemm_events[0].record(stream)
-        gemm(xs, ys)
-        if gemm_events:
-            gemm_events[1].record(stream)
-
-    def events(n):
-        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(n)]
-
-    launches_per_step = 4 if use_codes else 3
+    L = Layer(wl, dev, args.path, rank=rank)
     for _ in range(args.warmup):
-        step()
+        L.step()
     torch.cuda.synchronize()
     if pq.stream_status() != 0:
         raise RuntimeError("device status word set during warm-up")
+    L.timed_steps(2, 0, flush, stream, world)
 
-    # The step, the forward and the GEMM alone are each captured once into a
-    # CUDA graph and replayed: one launch per step, no host gaps between the
-    # step's kernels.
-    def capture(fn):
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            fn()
-        torch.cuda.current_stream().wait_stream(side)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            fn()
-        torch.cuda.synchronize()
-        return graph
-
-    def gemm_only():
-        gemm(xd, y)
-
-    step_graph = capture(step)
-    fwd_graph = capture(lambda: forward(xd, y))
-    gemm_graph = capture(gemm_only)
-    fused_graph = capture(lambda: pq.linear(xd, qw, sp, sn, bd, out=y)) if use_codes else None
-    # The single-scale baseline (one symmetric scale per K segment) of the same
-    # forward: its codes, then one int8 product per unit.
-    single_graph = None
-    if wl.bits == 8:
-        ldc = (wl.K + 15) // 16 * 16
-        c1_buf = torch.empty((wl.M, ldc), dtype=torch.int8, device=dev)[:, : wl.K]
-
-        def single_forward():
-            pq.quantize_activations_single(xd, wl.kseg, sp, sn, out=c1_buf)
-            pq.linear_from_single(c1_buf, qw, sp, sn, bd, out=y)
-        single_graph = capture(single_forward)
-    # int4 weights: the block-Hadamard variant (HQ-DM) of the same forward --
-    # codes of XH, then the product with the rotated int4 codes.  Its scales
-    # and the weight rotation are offline steps, made once here.
-    had_graph = None
-    if wl.bits == 4:
-        hsp = torch.empty(J, dtype=torch.float32, device=dev)
-        hsn = torch.empty(J, dtype=torch.float32, device=dev)
-        pq.calibrate_hadamard(calib, wl.kseg, hsp, hsn)
-        w_rot = pq.rotate_weights_hadamard(qw)
-        ldh = (wl.K + 15) // 16 * 16
-        hq_p = torch.empty((wl.M, ldh), dtype=torch.int8, device=dev)[:, : wl.K]
-        hq_n = torch.empty((wl.M, ldh), dtype=torch.int8, device=dev)[:, : wl.K]
-
-        def hadamard_forward():
-            pq.quantize_activations_hadamard(xd, wl.kseg, hsp, hsn, out=(hq_p, hq_n))
-            pq.linear_from_codes_hadamard(hq_p, hq_n, qw, w_rot, hsp, hsn, bd, out=y)
-        had_graph = capture(hadamard_forward)
-
-    def timed(graph, n, salt):
-        evs = events(n)
-        for i in range(n):
-            flush(i + salt)
-            evs[i][0].record(stream)
-            graph.replay()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        return [a.elapsed_time(b) for a, b in evs]
-
-    timed(step_graph, 2, 0)
     sampler = None if args.no_clocks else ClockSampler(local)
     if sampler:
         sampler.start()
@@ -509,98 +693,101 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = timed(step_graph, args.steps, 1)
+    step_ms = L.timed_steps(args.steps, 1, flush, stream, world)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     total_ms = sum(step_ms)
-    gemm_ms = timed(gemm_graph, args.steps, 3)
-    fwd_ms = timed(fwd_graph, args.steps, 5)
-    fused_ms = timed(fused_graph, args.steps, 7) if fused_graph is not None else None
-    single_ms = timed(single_graph, args.steps, 9) if single_graph is not None else None
-    had_ms = timed(had_graph, args.steps, 11) if had_graph is not None else None
+    gemm_ms = timed_graph(L.gemm_graph, args.steps, 3, flush, stream)
+    fwd_ms = timed_graph(L.fwd_graph, args.steps, 5, flush, stream)
+    fused_ms = timed_graph(L.fused_graph, args.steps, 7, flush, stream) if L.fused_graph else None
+    single_ms = timed_graph(L.single_graph, args.steps, 9, flush, stream) if L.single_graph else None
+    had_ms = timed_graph(L.had_graph, args.steps, 11, flush, stream) if L.had_graph else None
     if pq.stream_status() != 0:
         raise RuntimeError("device status word set during the timed region")
-    del step_graph, fwd_graph, gemm_graph, fused_graph, single_graph, had_graph
+    L.release()
 
-    # end to end through the API: host inputs in, host result out, every step
+    # end to end through the API: host inputs in (pinned), host result out, every step
     e2e = None
     if not args.no_e2e:
-        xh = x.pin_memory()
-        wh = w.pin_memory()
-        yh = torch.empty((wl.M, wl.N), dtype=out_dtype).pin_memory()
-        xdd = torch.empty_like(xd)
-        wdd = torch.empty_like(wd)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        xh = L.x_host.pin_memory()
+        wh = L.w_host.pin_memory()
+        yh = torch.empty((wl.M, wl.N), dtype=L.out_dtype).pin_memory()
+        xdd = torch.empty_like(L.xd)
+        wdd = torch.empty_like(L.wd)
+        calib_d = xdd if wl.calib_rows is None else xdd[: wl.calib_rows]
 
         def e2e_step():
             xdd.copy_(xh, non_blocking=True)
             wdd.copy_(wh, non_blocking=True)
-            step(xs=xdd, ws=wdd)
-            yh.copy_(y, non_blocking=True)
+            L.calibrate(calib_d)
+            L.rest(xs=xdd, ws=wdd)
+            yh.copy_(L.y, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_total = e0.elapsed_time(e1)
-        bi = xh.numel() * xh.element_size() + wh.numel() * wh.element_size()
-        bo = yh.numel() * yh.element_size()
-        e2e = {"ms": e2e_total, "bi": bi, "bo": bo}
+        e2e = {"ms": e0.elapsed_time(e1),
+               "bi": xh.numel() * xh.element_size() + wh.numel() * wh.element_size(),
+               "bo": yh.numel() * yh.element_size()}
 
-    # max over ranks
-    vals = [total_ms, statistics.mean(gemm_ms), statistics.mean(fwd_ms),
-            e2e["ms"] if e2e else 0.0, statistics.mean(fused_ms) if fused_ms else 0.0,
-            statistics.mean(single_ms) if single_ms else 0.0,
-            statistics.mean(had_ms) if had_ms else 0.0]
-    if world > 1:
-        t = torch.tensor(vals, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        vals = t.tolist()
+    mean = lambda v: statistics.mean(v) if v else 0.0   # noqa: E731
+    vals = max_over_ranks([total_ms, mean(gemm_ms), mean(fwd_ms), e2e["ms"] if e2e else 0.0,
+                           mean(fused_ms), mean(single_ms), mean(had_ms)], world, dev)
     total_ms, gemm_avg_ms, fwd_avg_ms, e2e_ms, fused_avg_ms, single_avg_ms, had_avg_ms = vals
 
+    line = None
     if rank == 0:
-        int8_peak_tops, hbm_peak, peak_kind = peaks()
+        sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+        mma_peak = mma_rate_tops(num_sms(dev), sm_mhz)
         ops = wl.exec_ops
-        value = world * args.steps * ops / (total_ms * 1e-3) / 1e12
         gemm_tops = ops / (gemm_avg_ms * 1e-3) / 1e12
+        byts = codes_gemm_bytes(wl) if L.codes else wl.alg_bytes()
         line = {
-            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-            "data": "synthetic",
-            "config": config_of(wl, "flushed (256 MiB write + 256 MiB read between steps)", args.path),
+            "metric": METRIC, "value": whole_job_tops(world, args.steps, ops, total_ms),
+            "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": config_of(wl, "flushed (256 MiB write + 256 MiB read between steps)",
+                                args.path, world),
             "roofline": {
                 "bound": "tensor", "kernel": gemm_kernel_name(args.path, wl.bits, wl.x_dtype),
-                "achieved": gemm_tops, "peak": int8_peak_tops, "unit": "TOPS",
-                "frac": gemm_tops / int8_peak_tops,
+                "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+                "frac": gemm_tops / int8_peak,
                 "traffic": NCU_TRAFFIC_BYTES.get((wl.name, args.path)),
                 "peak_source": f"{peak_kind} bf16 burst x {INT8_PER_BF16:g} (nominal int8/bf16)",
+                "mma_rate_tops": mma_peak, "frac_mma_rate": gemm_tops / mma_peak,
+                "mma_rate_source": (f"{MMA_I8_OPS_PER_CLK_SM} int8 ops/clk/SM (measured "
+                                    f"tcgen05 kind::i8 issue rate) x {num_sms(dev)} SMs x "
+                                    f"{sm_mhz:g} MHz"),
                 "algorithmic_ops_per_launch": ops,
-                "algorithmic_bytes_per_launch": wl.alg_bytes(),
-                "achieved_gbs": wl.alg_bytes() / (gemm_avg_ms * 1e-3) / 1e9,
+                "algorithmic_bytes_per_launch": byts,
+                "achieved_gbs": byts / (gemm_avg_ms * 1e-3) / 1e9,
                 "avg_launch_us": gemm_avg_ms * 1e3,
             },
             "forward_only": {
                 "us": fwd_avg_ms * 1e3, "exec_tops": ops / (fwd_avg_ms * 1e-3) / 1e12,
                 "linear_equiv_tops": ops / 2 / (fwd_avg_ms * 1e-3) / 1e12,
-                "frac_int8_peak": ops / (fwd_avg_ms * 1e-3) / 1e12 / int8_peak_tops,
+                "frac_int8_peak": ops / (fwd_avg_ms * 1e-3) / 1e12 / int8_peak,
             },
-            "gpu_launches": launches_per_step * args.steps,
-            "timing": "each step one CUDA-graph replay, CUDA events on the launching stream",
+            "gpu_launches": L.launches_per_step * args.steps,
+            "timing": ("each step: the calibration launch (+ the MAX all-reduce of the scales "
+                       "over ranks), then one CUDA-graph replay of weight quantization and the "
+                       "forward; CUDA events on the launching stream"),
             "clocks": clocks,
         }
         if had_ms:
             line["hadamard_forward"] = {
-                "us": had_avg_ms * 1e3,
-                "exec_tops": ops / (had_avg_ms * 1e-3) / 1e12,
+                "us": had_avg_ms * 1e3, "exec_tops": ops / (had_avg_ms * 1e-3) / 1e12,
                 "over_dualscale_forward": had_avg_ms / fwd_avg_ms,
                 "note": "block-Hadamard activations (blocks of 16): codes of XH, then the product "
                         "with the Hadamard-rotated int4 codes (rotation and its scales offline)"}
@@ -610,18 +797,30 @@ def run_ours(args):
                 "exec_tops": ops / 2 / (single_avg_ms * 1e-3) / 1e12,
                 "dualscale_over_single": fwd_avg_ms / single_avg_ms,
                 "note": "naive baseline: one symmetric scale per K segment, its codes, then one "
-                        "int8 product (half the MMA work of DualScale)",
-            }
+                        "int8 product (half the MMA work of DualScale)"}
         if fused_ms:
             line["fused_forward"] = {
                 "us": fused_avg_ms * 1e3, "exec_tops": ops / (fused_avg_ms * 1e-3) / 1e12,
-                "frac_int8_peak": ops / (fused_avg_ms * 1e-3) / 1e12 / int8_peak_tops,
+                "frac_int8_peak": ops / (fused_avg_ms * 1e-3) / 1e12 / int8_peak,
                 "note": "sq_linear_forward: activations quantized inside the GEMM"}
         if e2e:
-            line["e2e"] = {"value": world * args.steps * ops / (e2e_ms * 1e-3) / 1e12,
+            line["e2e"] = {"value": whole_job_tops(world, args.steps, ops, e2e_ms),
                            "unit": "TOPS", "h2d_bytes_per_step": e2e["bi"],
-                           "d2h_bytes_per_step": e2e["bo"]}
-        if world == 1 and not args.no_small_m:
+                           "d2h_bytes_per_step": e2e["bo"],
+                           "note": "inputs copied from pinned host memory and Y copied back "
+                                   "every step, around the library's calls (device pointers)"}
+    del L
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1:
+        if not args.no_configs:
+            table = {}
+            mma_peak = line["roofline"]["mma_rate_tops"]
+            for name in CONFIG_ORDER:
+                table[name] = measure_config(W.WORKLOADS[name], dev, flush, args.steps,
+                                             args.warmup, int8_peak, mma_peak, hbm_peak)
+                torch.cuda.empty_cache()
+            line["configs"] = table
+        if not args.no_small_m:
             line["small_m"] = {
                 "note": "HBM-bound forwards at M <= 128 (median of L2-flushed graph replays; "
                         "one_pass_layers: per layer of 8 back-to-back layers with distinct "
@@ -629,8 +828,12 @@ def run_ours(args):
                         "measured HBM copy",
                 "peak_gbs": hbm_peak,
                 "cases": small_m_measure(dev, flush, args.steps, hbm_peak)}
-        if world == 1 and not args.no_cpu_baseline:
+            line["per_call_us"] = per_call_measure(dev)
+        if not args.no_cpu_baseline:
+            from synth import workloads as W2
+            x, w, b = W2.generate(wl)
             line["cpu_baseline"] = cpu_baseline(wl, x, w, b)
+    if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -638,8 +841,17 @@ def run_ours(args):
     return 0
 
 
-def main():
-    args = parse_args()
+def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
+    args = parse_args(argv)
+    bad = check_world(args.gpus)
+    if bad is not None:
+        print(f"bench.py: {bad}", file=sys.stderr)
+        return 2
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks and wait for them
+        cmd = relaunch_command(argv, args.gpus, free_port())
+        return subprocess.run(cmd, timeout=3600).returncode
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

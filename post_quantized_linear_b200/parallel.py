@@ -28,13 +28,15 @@ def allreduce_scales_(s_pos: torch.Tensor, s_neg: torch.Tensor, group=None) -> N
 
 
 def calibrate_sharded(x_local: torch.Tensor, kseg: Sequence[int], group=None,
-                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                      stream=None, s_pos: Optional[torch.Tensor] = None,
+                      s_neg: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Static DualScale scales of the union of every rank's calibration rows.
 
     Each rank calibrates its own rows on its GPU, then the 2*J scales are
-    all-reduced with MAX (NCCL over NVLink for CUDA tensors)."""
+    all-reduced with MAX (NCCL over NVLink for CUDA tensors).  ``s_pos`` /
+    ``s_neg`` (fp32 [J]) receive the scales when given."""
     from . import calibrate
-    s_pos, s_neg = calibrate(x_local, kseg, stream=stream)
+    s_pos, s_neg = calibrate(x_local, kseg, s_pos, s_neg, stream=stream)
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
         allreduce_scales_(s_pos, s_neg, group)
     return s_pos, s_neg
