@@ -279,6 +279,50 @@ def small_m_measure(dev, flush, steps: int, hbm_peak: float):
     return out
 
 
+FUSED_ACT_CASES = (("dit_xl2_fc2_cfg", "gelu"), ("w4a8", "silu"))
+
+
+def fused_act_measure(dev, flush, steps: int, hbm_peak: float):
+    """The activation fused into the combined-code producer on the DiT fc2 input
+    (GELU) and the W4A8 input (SiLU), against the unfused pair (the framework's
+    activation kernel writing X in bf16, then the combined-code quantizer).
+    Bytes: fused = Z read (bf16) + codes written; unfused = Z read + X written
+    + X read + codes written.  Each a CUDA-graph replay after an L2 flush."""
+    import torch
+    import post_quantized_linear_b200 as pq
+    from synth import workloads as W
+    stream = torch.cuda.current_stream()
+    out = []
+    for name, act in FUSED_ACT_CASES:
+        wl = W.WORKLOADS[name]
+        g = torch.Generator().manual_seed(wl.seed)
+        z = torch.randn((wl.M, wl.K), generator=g).to(torch.bfloat16).to(dev)
+        x = torch.empty_like(z)
+        ldc = (wl.K + 15) // 16 * 16
+        c = torch.empty((wl.M, ldc), dtype=torch.int8, device=dev)[:, : wl.K]
+        sp, sn = pq.calibrate_act(z, act, wl.kseg)
+        fn = torch.nn.functional.silu if act == "silu" else torch.nn.functional.gelu
+
+        def fused():
+            pq.quantize_activations_combined_act(z, act, wl.kseg, sp, sn, out=c)
+
+        def unfused():
+            x.copy_(fn(z))
+            pq.quantize_activations_combined(x, wl.kseg, sp, sn, out=c)
+        res = {"workload": name, "act": act, "M": wl.M, "K": wl.K}
+        for key, f, byts in (("fused", fused, 3 * wl.M * wl.K), ("unfused", unfused, 7 * wl.M * wl.K)):
+            gph = capture(f)
+            us = statistics.median(timed_graph(gph, max(steps, 5), 0, flush, stream)) * 1e3
+            res[key] = {"us": us, "gbs": byts / (us * 1e-6) / 1e9,
+                        "frac_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak,
+                        "bytes": byts}
+            del gph
+        res["fused_over_unfused"] = res["fused"]["us"] / res["unfused"]["us"]
+        out.append(res)
+        del z, x, c
+    return out
+
+
 def per_call_measure(dev, calls: int = 200):
     """Host cost of one forward call outside a CUDA graph, the cost a small-M
     caller pays: the GEMM from codes at M = 16, (K, N) = (3072, 12288), called
@@ -829,6 +873,11 @@ def run_ours(args):
                 "peak_gbs": hbm_peak,
                 "cases": small_m_measure(dev, flush, args.steps, hbm_peak)}
             line["per_call_us"] = per_call_measure(dev)
+            line["fused_activation"] = {
+                "note": "SiLU / GELU fused into the combined-code producer (x = bf16_RN(act(z)) "
+                        "never stored) against the framework's activation kernel + the "
+                        "combined-code quantizer; bytes are the algorithmic traffic of each",
+                "peak_gbs": hbm_peak, "cases": fused_act_measure(dev, flush, args.steps, hbm_peak)}
         if not args.no_cpu_baseline:
             from synth import workloads as W2
             x, w, b = W2.generate(wl)

@@ -180,6 +180,38 @@ sq_status sq_quantize_activations_combined(const void* x, sq_dtype xt, int64_t M
                                            const float* s_pos, const float* s_neg, int8_t* c,
                                            int64_t ldc, sq_stream_t stream);
 
+/* Activation fused into the combined-code producer.  SegQuant (Spanish
+ * technical summary 1 and 2.B; Korean technical summary section 2,
+ * "DualScale"): the negative tail DualScale preserves is produced by the SiLU /
+ * GELU in front of the layer, so the producer reads the pre-activation Z and
+ * writes the codes of X = act(Z) without storing X.
+ *   SQ_ACT_SILU: act(z) = z / (1 + exp(-z));
+ *   SQ_ACT_GELU: act(z) = z/2 * erfc(-z / sqrt(2)) (the exact, erf-based GELU).
+ * Reading: x is the exact act(z) rounded once, to nearest even, to bf16 (the
+ * storage type of the activations this replaces); the kernels evaluate it in
+ * fp32 and fall back to fp64 wherever the fp32 error bound does not decide the
+ * bf16 rounding, so x equals the correctly rounded value (up to fp64 ties). */
+typedef enum { SQ_ACT_SILU = 1, SQ_ACT_GELU = 2 } sq_act;
+
+/* Static DualScale scales of X = act(Z) over the calibration rows of Z (rows x
+ * K, dtype zt, row stride ldz): sq_calibrate's rule applied to X.  Arguments,
+ * requirements and errors as for sq_calibrate (K a multiple of 16); an
+ * unknown `act` returns SQ_ERR_INVALID_ARG.  Z must be finite. */
+sq_status sq_calibrate_act(const void* z, sq_dtype zt, sq_act act, int64_t rows, int64_t K,
+                           int64_t ldz, const sq_segments* kseg, float* s_pos, float* s_neg,
+                           sq_stream_t stream);
+
+/* Combined DualScale codes c = q+ + q- of X = act(Z), read from the
+ * pre-activation Z [M, K] (dtype zt, row stride ldz): one pass over Z, X never
+ * written.  Codes, layout and requirements as for
+ * sq_quantize_activations_combined; an unknown `act` returns
+ * SQ_ERR_INVALID_ARG.  Z must be finite.  The codes feed
+ * sq_linear_forward_combined. */
+sq_status sq_quantize_activations_combined_act(const void* z, sq_dtype zt, sq_act act, int64_t M,
+                                               int64_t K, int64_t ldz, const sq_segments* kseg,
+                                               const float* s_pos, const float* s_neg, int8_t* c,
+                                               int64_t ldc, sq_stream_t stream);
+
 /* The forward pass from combined codes (written by
  * sq_quantize_activations_combined with the same scales): the kernel loads one
  * int8 code tile per k block by TMA, splits it into q+ and q- in shared memory

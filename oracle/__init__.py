@@ -71,9 +71,11 @@ def _load():
         lib.sqo_f32_to_f16.restype = ctypes.c_uint16
         lib.sqo_f16_to_f32.argtypes = [ctypes.c_uint16]
         lib.sqo_f16_to_f32.restype = ctypes.c_float
+        lib.sqo_activation_bf16.argtypes = [P, INT, I64, INT, P, P]
         for f in ("sqo_calibrate", "sqo_quantize_activations", "sqo_quantize_weights_w8",
                   "sqo_quantize_weights_w4", "sqo_accumulate", "sqo_epilogue",
-                  "sqo_quantize_activations_single", "sqo_epilogue_single"):
+                  "sqo_quantize_activations_single", "sqo_epilogue_single",
+                  "sqo_activation_bf16"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -421,3 +423,37 @@ def linear_forward_hadamard(x, kbounds, s_pos, s_neg, packed, scales, bias=None,
     if return_acc:
         return y, acc, (qp, qn), rot
     return y
+
+
+# ----------------------------------------------------------------------------
+# The activation in front of the layer, for the fused producer (SegQuant,
+# Spanish technical summary 1 and 2.B, Korean technical summary section 2: the
+# negative tail DualScale keeps comes from SiLU / GELU).  Reading: the layer
+# input is x = act(z) rounded once to bf16; act is evaluated in double by the
+# C library, and elements whose double lies within a relative 2^-40 of a bf16
+# rounding midpoint are flagged (their rounding is not decided by a double).
+ACTIVATIONS = {"silu": 1, "gelu": 2}
+
+
+def activation_bf16(z: np.ndarray, act: str):
+    """x = bf16_RN(act(z)) as bf16 bit patterns (uint16, z's shape) and a bool
+    mask of the elements flagged as undecided by the double evaluation.
+    z: fp32 values or bf16 bit patterns (uint16); act: 'silu' or 'gelu'."""
+    z = np.ascontiguousarray(z)
+    x = np.zeros(z.shape, np.uint16)
+    flags = np.zeros(z.shape, np.uint8)
+    _check("sqo_activation_bf16", _load().sqo_activation_bf16(
+        _ptr(z), _x_dtype(z), z.size, ACTIVATIONS[act], _ptr(x), _ptr(flags)))
+    return x, flags.astype(bool)
+
+
+def calibrate_act(z: np.ndarray, act: str, kbounds):
+    """Static DualScale scales of x = act(z) (calibrate applied to the bf16 x)."""
+    x, _ = activation_bf16(z, act)
+    return calibrate(x, kbounds)
+
+
+def quantize_activations_combined_act(z: np.ndarray, act: str, kbounds, s_pos, s_neg):
+    """Combined codes of x = act(z) and the flags of undecided elements."""
+    x, flags = activation_bf16(z, act)
+    return quantize_activations_combined(x, kbounds, s_pos, s_neg), flags

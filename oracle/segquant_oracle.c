@@ -368,3 +368,56 @@ int sqo_epilogue_f32(const int32_t* acc, int64_t M, int64_t N, int32_t U,
                      const float* sw, const float* bias, float* y) {
   return sqo_epilogue(acc, M, N, U, unit_seg, s_pos, s_neg, sw, bias, y, 0, N);
 }
+
+/* ---- Activation in front of the layer (the fused producer) -----------------
+ * [ES 1], [ES 2.B], [KO 2.2]: the small negative tail DualScale keeps comes
+ * from the SiLU / GELU that produces the layer input.  The fused producer
+ * quantizes x = act(z) straight from the pre-activation z.
+ *   act 1: SiLU(z) = z / (1 + exp(-z));
+ *   act 2: GELU(z) = z/2 * erfc(-z / sqrt(2))  (the exact, erf-based GELU).
+ * Reading: x is the exact act(z) rounded once, to nearest with ties to even,
+ * to bf16.  Here act(z) is evaluated in double with the C library (relative
+ * error far below 2^-40 for finite z); flags[i] = 1 when that double lies
+ * within a relative 2^-40 of a bf16 rounding midpoint, where a library's error
+ * could decide the rounding -- such elements are exempt from exact comparison.
+ * z: fp32 or bf16 patterns (dtype as load_elem); x: bf16 patterns. */
+static const double kBf16Max = 3.3895313892515355e38;   /* (2 - 2^-7) * 2^127 */
+
+/* bf16 round-half-even of a double, from the format: 8 significant bits,
+ * exponents down to -126, subnormal spacing 2^-133. */
+static uint16_t bf16_from_double(double d, int* near_mid) {
+  *near_mid = 0;
+  const uint16_t sign = signbit(d) ? 0x8000u : 0u;
+  double a = fabs(d);
+  if (a == 0.0) return sign;
+  int e;
+  (void)frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+  int E = e - 1;
+  if (E < -126) E = -126;             /* subnormal range: fixed spacing */
+  const double ulp = ldexp(1.0, E - 7);
+  const double q = a / ulp;           /* exact: a power-of-two scaling */
+  const double fl = floor(q);
+  if (fabs(q - (fl + 0.5)) <= q * 0x1p-40) *near_mid = 1;
+  const double r = nearbyint(q) * ulp;
+  if (r > kBf16Max) return (uint16_t)(sign | 0x7f80u);   /* rounds to infinity */
+  const float rf = (float)r;          /* exact: r has at most 8 significant bits */
+  uint32_t u;
+  memcpy(&u, &rf, 4);
+  return (uint16_t)(sign | ((u >> 16) & 0x7fffu));
+}
+
+int sqo_activation_bf16(const void* z, int dtype, int64_t n, int act, uint16_t* x,
+                        uint8_t* flags) {
+  if (act != 1 && act != 2) return SQO_ERR_ARG;
+  int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+  for (int64_t i = 0; i < n; ++i) {
+    const double zd = (double)load_elem(z, dtype, i);
+    if (!isfinite(zd)) bad = 1;
+    const double v = (act == 1) ? zd / (1.0 + exp(-zd)) : 0.5 * zd * erfc(-zd / sqrt(2.0));
+    int near_mid = 0;
+    x[i] = bf16_from_double(v, &near_mid);
+    flags[i] = (uint8_t)near_mid;
+  }
+  return bad ? SQO_ERR_RANGE : SQO_OK;
+}

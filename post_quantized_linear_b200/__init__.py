@@ -28,7 +28,7 @@ __all__ = ["QuantizedWeight", "SegQuantError", "calibrate", "quantize_weights", 
            "splitk_workspace_size", "splitk_workspace", "linear_from_codes_splitk",
            "linear_accumulators", "stream_status", "qweight_sizes", "calibrate_hadamard",
            "quantize_activations_hadamard", "rotate_weights_hadamard",
-           "linear_from_codes_hadamard"]
+           "linear_from_codes_hadamard", "calibrate_act", "quantize_activations_combined_act"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -197,6 +197,52 @@ def quantize_activations_combined(x: torch.Tensor, kseg: Sequence[int], s_pos: t
     _lib.check("sq_quantize_activations_combined", _lib.load().sq_quantize_activations_combined(
         _ptr(x), _dtype_code(x.dtype), M, K, x.stride(0), ctypes.byref(seg), _ptr(s_pos),
         _ptr(s_neg), _ptr(out), out.stride(0), _stream(stream)))
+    return out
+
+
+def _act_code(act: str) -> int:
+    if act == "silu":
+        return _lib.SQ_ACT_SILU
+    if act == "gelu":
+        return _lib.SQ_ACT_GELU
+    raise ValueError(f"unknown activation {act!r}: 'silu' or 'gelu'")
+
+
+def calibrate_act(z: torch.Tensor, act: str, kseg: Sequence[int],
+                  s_pos: Optional[torch.Tensor] = None, s_neg: Optional[torch.Tensor] = None,
+                  stream=None):
+    """Static DualScale scales (s+, s-) fp32 [J] of X = act(z) over the
+    calibration rows of the pre-activation ``z`` [rows, K]; act: 'silu' or 'gelu'."""
+    _check_2d(z, "z")
+    J = len(kseg) - 1
+    if s_pos is None:
+        s_pos = torch.empty(J, dtype=torch.float32, device=z.device)
+    if s_neg is None:
+        s_neg = torch.empty(J, dtype=torch.float32, device=z.device)
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_calibrate_act", _lib.load().sq_calibrate_act(
+        _ptr(z), _dtype_code(z.dtype), _act_code(act), z.shape[0], z.shape[1], z.stride(0),
+        ctypes.byref(seg), _ptr(s_pos), _ptr(s_neg), _stream(stream)))
+    return s_pos, s_neg
+
+
+def quantize_activations_combined_act(z: torch.Tensor, act: str, kseg: Sequence[int],
+                                      s_pos: torch.Tensor, s_neg: torch.Tensor,
+                                      out: Optional[torch.Tensor] = None,
+                                      stream=None) -> torch.Tensor:
+    """Combined DualScale codes of X = act(z) (X rounded once to bf16, never
+    stored), int8 [M, K] with row stride a multiple of 16; act: 'silu' or 'gelu'."""
+    _check_2d(z, "z")
+    M, K = z.shape
+    if out is None:
+        ldc = (K + 15) // 16 * 16
+        out = torch.empty((M, ldc), dtype=torch.int8, device=z.device)[:, :K]
+    seg, keep = _lib.segments(kseg)
+    _lib.check("sq_quantize_activations_combined_act",
+               _lib.load().sq_quantize_activations_combined_act(
+                   _ptr(z), _dtype_code(z.dtype), _act_code(act), M, K, z.stride(0),
+                   ctypes.byref(seg), _ptr(s_pos), _ptr(s_neg), _ptr(out), out.stride(0),
+                   _stream(stream)))
     return out
 
 

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libsegquant.so")
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED = 0, 1, 2, 3
 SQ_ERR_RANGE, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 4, 5, 6
 SQ_F32, SQ_BF16 = 0, 1
+SQ_ACT_SILU, SQ_ACT_GELU = 1, 2
 SQ_MAX_SEGMENTS = 16
 SQ_MAX_K = 131072
 
@@ -47,6 +48,9 @@ SIGNATURES = {
                                         c_vp, c_i64, c_vp]),
     "sq_quantize_activations_combined": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp,
                                                  c_vp, c_vp, c_i64, c_vp]),
+    "sq_calibrate_act": (c_i32, [c_vp, c_i32, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp, c_vp, c_vp]),
+    "sq_quantize_activations_combined_act": (c_i32, [c_vp, c_i32, c_i32, c_i64, c_i64, c_i64, P_SEG,
+                                                     c_vp, c_vp, c_vp, c_i64, c_vp]),
     "sq_linear_forward_combined": (c_i32, [c_vp, c_i64, c_i64, c_i64, P_QW, c_vp, c_vp, c_vp, c_vp,
                                            c_i32, c_i64, c_vp]),
     "sq_quantize_activations_single": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, P_SEG, c_vp,

@@ -526,6 +526,25 @@ __device__ __forceinline__ void fold8_seeded(const uint32_t (&ap)[8], const uint
   }
 }
 
+// int32 accumulator -> fp32, round to nearest even (an int8 unit's sum:
+// |acc| <= 127 * 127 * K).
+__device__ __forceinline__ float acc_f32(uint32_t v) { return __int2float_rn((int)v); }
+
+// y (+)= sw * (s- F(acc-) + s+ F(acc+)) for eight columns, the fixed fp32
+// order of fold8 on fp32 pairs (two outputs per packed instruction).
+__device__ __forceinline__ void fold8_exact(const uint32_t (&ap)[8], const uint32_t (&an)[8],
+                                            const float (&sw)[8], float sp, float sn, float* y) {
+  const uint64_t sp2 = f2_pack(sp, sp), sn2 = f2_pack(sn, sn);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const uint64_t fp = f2_pack(acc_f32(ap[i]), acc_f32(ap[i + 1]));
+    const uint64_t fn = f2_pack(acc_f32(an[i]), acc_f32(an[i + 1]));
+    const uint64_t yy = f2_fma(f2_pack(sw[i], sw[i + 1]), f2_fma(sn2, fn, f2_mul(sp2, fp)),
+                               f2_pack(y[i], y[i + 1]));
+    f2_unpack(yy, y[i], y[i + 1]);
+  }
+}
+
 // Weight scales of 8 consecutive output channels for unit u, as four fp32 pairs.
 __device__ __forceinline__ void load_wscales8_pairs(const GemmArgs& a, int u, int j, int n,
                                                     uint64_t (&sw2)[4]) {
@@ -838,19 +857,14 @@ __device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float&
 // (tile rows) and columns [part*HALF, (part+1)*HALF).  NACC accumulators per
 // unit (2: DualScale (+)/(-) products at columns c and c + BN of the buffer;
 // 1: single scale).  MULTI: several units (K segments) per tile, folded into
-// registers (HALF == 32), stored once per tile; otherwise one unit per tile,
-// streamed out in 32-column passes with the accumulators released after the
-// warp's last TMEM load.
-// SEED (one unit per 128-wide group, the accumulators seeded): 1 -- int4
-// weights unpacked as 16 x the code, the accumulators hold the bits of
-// 1.5 * 2^19 + acc (kMagicW4Bits plus 16 * acc); 2 -- int8 weight codes (the
-// Hadamard-rotated int4 codes, |acc| < 2^22), the accumulators hold the bits
-// of 1.5 * 2^23 + acc, and the activation scales are multiplied by the block
-// normalization 1/4 (exact).  The warps seed their columns of both buffers
-// before the first unit and again right after reading them, so F(acc) is one
-// exact subtraction; the group's fp16 weight scales and its segment's s+/s-
-// enter the same fp32 order as the other units.
-template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, int SEED, class TileFn>
+// fp32 partial outputs in registers (HALF = 32 or 64 columns per thread),
+// stored once per tile; otherwise one unit per tile, streamed out in
+// 32-column passes.  Either way the accumulator buffer is released as soon as
+// the warp's last TMEM load of the unit has landed, before the arithmetic on
+// it, so the MMA of the next unit or tile waits only for the loads.
+// (Group units -- one per 128-wide K group -- go through
+// epilogue_groups_tma_store.)
+template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
@@ -860,155 +874,108 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
   constexpr int ROWB = Y_BF16 ? 64 : 128;
   constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
   static_assert(HALF % 32 == 0, "32-column store passes");
-  static_assert(!MULTI || HALF == 32, "several units: one 32-column pass per warp");
-  constexpr bool SEEDED = (SEED != 0);
-  static_assert(!SEEDED || (MULTI && NACC == 2), "seeded accumulators: int4 groups, DualScale");
-  constexpr uint32_t seed_bits = (SEED == 1) ? kMagicW4Bits : kMagicBits;
-  constexpr float seed_value = (SEED == 1) ? kMagicW4 : kMagic;
-  constexpr float act_mult = (SEED == 2) ? 0.25f : 1.0f;   // Hadamard block normalization
+  static_assert(!MULTI || HALF <= 64, "several units: at most 64 partial outputs per thread");
   uint8_t* srow = stage_y + lane * ROWB;
   const uint32_t sbase = smem_u32(stage_y);
-  const int units = SEEDED ? args.num_kb : args.kseg.count;
+  const int units = args.kseg.count;
   auto release = [&](int b) {
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
   };
-  // fold of 16 columns at tile column cc of buffer b, unit / segment j, into o
-  auto fold = [&](int b, int cc, int j, const Tile& t, float* o) {
+  // Eight columns of buffer b at tile column cc into registers (both
+  // polarities, or the single code's accumulator in ap).
+  auto load8 = [&](int b, int cc, uint32_t (&ap)[8], uint32_t (&an)[8]) {
     const uint32_t tcol = (uint32_t)b * BUF_COLS + (uint32_t)cc;
-    float sw[16];
-    float sp, sn;
-    unit_act_scales(args, j, sp, sn);
-    if constexpr (NACC == 2) {
-      uint32_t ap[16], an[16];
-      tmem_ld16(t_lane + tcol, ap);
-      tmem_ld16(t_lane + tcol + BN, an);
-      tmem_wait_ld();
-      load_wscales16(args, j, j, t.n0 + cc, sw);
-      fold16<false>(ap, an, sw, sp, sn, o);
-    } else {
-      uint32_t ac[16];
-      tmem_ld16(t_lane + tcol, ac);
-      tmem_wait_ld();
-      load_wscales16(args, j, j, t.n0 + cc, sw);
-      fold16_single(ac, sw, fmaxf(sp, sn), o);
-    }
+    tmem_ld8(t_lane + tcol, ap);
+    if constexpr (NACC == 2) tmem_ld8(t_lane + tcol + BN, an);
   };
-  // Seeded (int4) unit: 16 columns at tile column cc of buffer b folded into
-  // y (fp32 pairs per eight columns), the columns re-seeded as soon as they
-  // are read.
-  auto fold_seeded = [&](int b, int cc, int u, int j, const Tile& t, float* y) {
-    const uint32_t tcol = (uint32_t)b * BUF_COLS + (uint32_t)cc;
-    float sp, sn;
-    unit_act_scales(args, j, sp, sn);
-    sp = __fmul_rn(sp, act_mult);
-    sn = __fmul_rn(sn, act_mult);
-    uint32_t ap[16], an[16];
-    tmem_ld16(t_lane + tcol, ap);
-    tmem_ld16(t_lane + tcol + BN, an);
-    tmem_wait_ld();
+  // y[0..8) (+)= the fold of eight loaded columns of unit / segment j
+  auto fold8c = [&](const uint32_t (&ap)[8], const uint32_t (&an)[8], int j, int n, float sp,
+                    float sn, float* y) {
+    float sw[8];
+    load_wscales8(args, j, j, n, sw);
+    if constexpr (NACC == 2) {
+      fold8_exact(ap, an, sw, sp, sn, y);
+    } else {
+      const float s = fmaxf(sp, sn);
 #pragma unroll
-    for (int h = 0; h < 16; h += 8) {
-      tmem_st8(t_lane + tcol + h, seed_bits);
-      tmem_st8(t_lane + tcol + BN + h, seed_bits);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {   // scales eight columns at a time (registers)
-      float sw8[8];
-      load_wscales8(args, u, j, t.n0 + cc + 8 * h, sw8);
-      fold8_seeded(*reinterpret_cast<const uint32_t(*)[8]>(ap + 8 * h),
-                   *reinterpret_cast<const uint32_t(*)[8]>(an + 8 * h), sw8, sp, sn, y + 8 * h,
-                   seed_value);
+      for (int i = 0; i < 8; ++i) y[i] = __fmaf_rn(sw[i], __fmul_rn(s, acc_f32(ap[i])), y[i]);
     }
   };
   int ug = 0;
   bool ok = true, pending = false;
-  if constexpr (SEEDED) {
-    // Seed this warp's columns of both buffers, then hand the buffers to the MMA.
-#pragma unroll
-    for (int b = 0; b < NBUF; ++b) {
-#pragma unroll
-      for (int c = 0; c < HALF; c += 8) {
-        const uint32_t col = (uint32_t)b * BUF_COLS + (uint32_t)(part * HALF + c);
-        tmem_st8(t_lane + col, seed_bits);
-        tmem_st8(t_lane + col + BN, seed_bits);
-      }
-    }
-    tmem_wait_st();
-    for (int b = 0; b < NBUF; ++b) release(b);
-  }
   for (int it = 0; it < rounds && ok; ++it) {
     Tile t;
     if (!tile_fn(it, t)) continue;
     const int c_lo = part * HALF;
     const int cols = min(HALF, t.width - c_lo);   // may be <= 0 on a narrow tail tile
     if (cols > 0) {
-      if constexpr (SEEDED) {   // fp16 scales [G][N]: 64 bytes per group for 32 columns
-        for (int u = lane; u < units; u += 32)
-          prefetch_l1(static_cast<const __half*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo);
-      } else {
-        for (int u = 0; u < units; ++u) {
-          const float* sw_row = static_cast<const float*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo;
-          for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
-        }
+      for (int u = 0; u < (MULTI ? units : 1); ++u) {
+        const float* sw_row = static_cast<const float*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo;
+        for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
       }
       if (args.bias != nullptr)
         for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(args.bias + t.n0 + c_lo + c);
     }
     const int npass = cols > 0 ? (cols + 31) / 32 : 0;
+    // the number of eight-column chunks this warp folds (a multiple of 8 columns)
+    const int nchunk = cols > 0 ? (cols + 7) / 8 : 0;
     if constexpr (MULTI) {
-      float y[32];
+      float y[HALF];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = 0.0f;
-      if constexpr (SEEDED) {
-        for (int u = 0; u < units; ++u) {
-          const int b = ug % NBUF;
-          if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
-          tc_fence_after();
-          if (npass > 0) {
-            const int j = args.kseg.segment_of(u * BK);
-            fold_seeded(b, c_lo, u, j, t, y);
-            if (c_lo + 16 < t.width) fold_seeded(b, c_lo + 16, u, j, t, y + 16);
+      for (int i = 0; i < HALF; ++i) y[i] = 0.0f;
+      for (int u = 0; u < units; ++u) {
+        const int b = ug % NBUF;
+        if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+        tc_fence_after();
+        float sp, sn;
+        unit_act_scales(args, u, sp, sn);
+        bool released = false;
+#pragma unroll
+        for (int c = 0; c < HALF / 8; ++c) {
+          if (c < nchunk) {
+            uint32_t ap[8], an[8];
+            load8(b, c_lo + 8 * c, ap, an);
+            tmem_wait_ld();
+            if (c + 1 == nchunk) {   // every column of the unit is in registers
+              release(b);
+              released = true;
+            }
+            fold8c(ap, an, u, t.n0 + c_lo + 8 * c, sp, sn, y + 8 * c);
           }
-          tmem_wait_st();
-          release(b);
-          ++ug;
         }
-      } else {
-        for (int u = 0; u < units; ++u) {
-          const int b = ug % NBUF;
-          if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
-          tc_fence_after();
-          if (npass > 0) {
-            fold(b, c_lo, u, t, y);
-            if (c_lo + 16 < t.width) fold(b, c_lo + 16, u, t, y + 16);
-          }
-          release(b);
-          ++ug;
-        }
+        if (!released) release(b);
+        ++ug;
       }
       if (!ok) break;
-      if (npass > 0) {
-        if (pending) {
-          if (lane == 0) bulk_wait_read_all();
+#pragma unroll
+      for (int p = 0; p < HALF / 32; ++p) {
+        if (p < npass) {
+          if (pending) {   // the previous store has read the staging tile
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
+          const int col = c_lo + p * 32;
+          stage16<Y_BF16>(args, t.n0 + col, *reinterpret_cast<float(*)[16]>(y + 32 * p), srow, lane, 0);
+          if (col + 16 < t.width)
+            stage16<Y_BF16>(args, t.n0 + col + 16, *reinterpret_cast<float(*)[16]>(y + 32 * p + 16),
+                            srow, lane, 1);
+          fence_proxy_async_smem();
           __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+            bulk_commit_group();
+          }
+          pending = true;
         }
-        stage16<Y_BF16>(args, t.n0 + c_lo, *reinterpret_cast<float(*)[16]>(y), srow, lane, 0);
-        if (c_lo + 16 < t.width)
-          stage16<Y_BF16>(args, t.n0 + c_lo + 16, *reinterpret_cast<float(*)[16]>(y + 16), srow, lane, 1);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(tmap_y, sbase, t.n0 + c_lo, t.m0 + quad * 32);
-          bulk_commit_group();
-        }
-        pending = true;
       }
     } else {
       const int b = ug % NBUF;
       if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
       tc_fence_after();
+      float sp, sn;
+      unit_act_scales(args, 0, sp, sn);
       for (int p = 0; p < npass; ++p) {
         const int col = c_lo + p * 32;
         if (pending) {   // the previous store has read the staging tile
@@ -1019,14 +986,19 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
         for (int h = 0; h < 2; ++h) {
           const int cc = col + 16 * h;
           if (cc < t.width) {
+            uint32_t ap[8], an[8], bp[8], bn[8];
+            load8(b, cc, ap, an);
+            load8(b, cc + 8, bp, bn);
+            tmem_wait_ld();
+            if (p == npass - 1 && (h == 1 || cc + 16 >= t.width)) release(b);   // last loads
             float o[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) o[i] = 0.0f;
-            fold(b, cc, 0, t, o);
+            fold8c(ap, an, 0, t.n0 + cc, sp, sn, o);
+            fold8c(bp, bn, 0, t.n0 + cc + 8, sp, sn, o + 8);
             stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
           }
         }
-        if (p == npass - 1) release(b);   // this warp's accumulator columns are all read
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -1037,6 +1009,154 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       }
       if (npass == 0) release(b);
       ++ug;
+    }
+  }
+  // Every store has completed before the CTA (and its shared memory) exits.
+  if (lane == 0) bulk_wait_all();
+  __syncwarp();
+}
+
+// ------------------------------------------- group-unit epilogue (int4 groups)
+// One unit per 128-wide K group (int4 weights, SEED 1; the Hadamard-rotated
+// codes, SEED 2): every k block ends a unit, so the whole accumulator pair is
+// folded once per 512 tensor-core cycles and the fold's instruction count sets
+// the kernel's speed.  Warp (quad, part) owns TMEM lanes quad*32 .. +31 (tile
+// rows) and the 32 columns [part*32, part*32 + 32) of every group:
+//   * the group's fp16 weight scales of those columns are widened to fp32 once
+//     per lane (lane l: column l, fetched one group ahead) and staged in the
+//     warp's shared-memory slot `sw_stage` (two buffers of 32 floats,
+//     alternating by group), from which every lane reads them back with
+//     broadcast 16-byte loads;
+//   * the accumulators are read eight columns at a time per polarity and
+//     re-seeded at once, so F(acc) is one exact subtraction (the seed's bits
+//     plus the integer sum are the float seed + acc);
+//   * the fold runs on fp32 pairs, five packed instructions per two outputs,
+//     in the fixed order t = fma(s-, F-, s+ * F+), y = fma(sw, t, y), y from 0.
+// After the tile's last group: + bias, convert, TMA store of the warp's
+// 32 x 32 block from its staging tile.
+template <int EPW, bool Y_BF16, int SEED, class TileFn>
+__device__ __forceinline__ void epilogue_groups_tma_store(
+    const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, float* sw_stage, int quad,
+    int part, int lane, uint32_t t_lane, uint64_t* tmem_full, uint32_t empty_base, int rounds,
+    TileFn tile_fn, volatile int* abort_flag, long long budget) {
+  constexpr int BN = 128;
+  constexpr int NBUF = 2;
+  static_assert(EPW == 16, "four parts of 32 columns per lane quarter");
+  static_assert(SEED == 1 || SEED == 2, "seeded group units");
+  constexpr uint32_t BUF_COLS = 2u * BN;
+  constexpr uint32_t seed_bits = (SEED == 1) ? kMagicW4Bits : kMagicBits;
+  constexpr float seed_value = (SEED == 1) ? kMagicW4 : kMagic;
+  constexpr float act_mult = (SEED == 2) ? 0.25f : 1.0f;   // Hadamard block normalization
+  constexpr int ROWB = Y_BF16 ? 64 : 128;
+  uint8_t* srow = stage_y + lane * ROWB;
+  const uint32_t sbase = smem_u32(stage_y);
+  const int G = args.num_kb;
+  const int c_lo = part * 32;
+  const __half* wsc = static_cast<const __half*>(args.wscales);
+  const uint64_t mseed = f2_pack(-seed_value, -seed_value);
+  auto release = [&](int b) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
+  };
+  // Seed this warp's columns of both buffers, then hand the buffers to the MMA.
+#pragma unroll
+  for (int b = 0; b < NBUF; ++b) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t col = (uint32_t)b * BUF_COLS + (uint32_t)(c_lo + 16 * h);
+      tmem_st16(t_lane + col, seed_bits);
+      tmem_st16(t_lane + col + BN, seed_bits);
+    }
+  }
+  tmem_wait_st();
+  for (int b = 0; b < NBUF; ++b) release(b);
+  int ug = 0;
+  bool ok = true, pending = false;
+  for (int it = 0; it < rounds && ok; ++it) {
+    Tile t;
+    if (!tile_fn(it, t)) continue;
+    const bool active = c_lo < t.width;                 // warp-uniform
+    const bool n_ok = active && (c_lo + lane < t.width);
+    const __half* wcol = wsc + t.n0 + c_lo + lane;      // this lane's column, group 0
+    const __half hzero = __ushort_as_half((unsigned short)0);
+    // group 0's scales staged now, group 1's fetched
+    sw_stage[lane] = __half2float(n_ok ? __ldg(wcol) : hzero);
+    __half h_next = (n_ok && G > 1) ? __ldg(wcol + args.N) : hzero;
+    __syncwarp();
+    uint64_t y2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y2[i] = 0ull;
+    int j = 0;
+    int seg_end = args.kseg.b[1];
+    float sp = __fmul_rn(__ldg(args.s_pos), act_mult), sn = __fmul_rn(__ldg(args.s_neg), act_mult);
+    uint64_t sp2 = f2_pack(sp, sp), sn2 = f2_pack(sn, sn);
+    for (int u = 0; u < G; ++u) {
+      if (u * BK >= seg_end) {   // the group opens the next K segment
+        ++j;
+        seg_end = args.kseg.b[j + 1];
+        sp = __fmul_rn(__ldg(args.s_pos + j), act_mult);
+        sn = __fmul_rn(__ldg(args.s_neg + j), act_mult);
+        sp2 = f2_pack(sp, sp);
+        sn2 = f2_pack(sn, sn);
+      }
+      const int b = ug % NBUF;
+      if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+      tc_fence_after();
+      if (active) {
+        const float* sw = sw_stage + (u & 1) * 32;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {   // eight columns at a time (register budget)
+          const uint32_t col = (uint32_t)b * BUF_COLS + (uint32_t)(c_lo + 8 * h);
+          uint32_t ap[8], an[8];
+          tmem_ld8(t_lane + col, ap);
+          tmem_ld8(t_lane + col + BN, an);
+          tmem_wait_ld();
+          tmem_st8(t_lane + col, seed_bits);
+          tmem_st8(t_lane + col + BN, seed_bits);
+          const float4* s4 = reinterpret_cast<const float4*>(sw + 8 * h);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const float4 s = s4[q];
+            const uint64_t sw_lo = f2_pack(s.x, s.y), sw_hi = f2_pack(s.z, s.w);
+            const int i = 4 * q;
+            const uint64_t fp0 = f2_add(f2_pack(__uint_as_float(ap[i]), __uint_as_float(ap[i + 1])), mseed);
+            const uint64_t fn0 = f2_add(f2_pack(__uint_as_float(an[i]), __uint_as_float(an[i + 1])), mseed);
+            const uint64_t fp1 = f2_add(f2_pack(__uint_as_float(ap[i + 2]), __uint_as_float(ap[i + 3])), mseed);
+            const uint64_t fn1 = f2_add(f2_pack(__uint_as_float(an[i + 2]), __uint_as_float(an[i + 3])), mseed);
+            y2[4 * h + 2 * q] = f2_fma(sw_lo, f2_fma(sn2, fn0, f2_mul(sp2, fp0)), y2[4 * h + 2 * q]);
+            y2[4 * h + 2 * q + 1] = f2_fma(sw_hi, f2_fma(sn2, fn1, f2_mul(sp2, fp1)), y2[4 * h + 2 * q + 1]);
+          }
+        }
+        tmem_wait_st();
+      }
+      release(b);
+      ++ug;
+      if (u + 1 < G) {   // stage group u+1's scales (its buffer was last read in group u-1)
+        sw_stage[((u + 1) & 1) * 32 + lane] = __half2float(h_next);
+        h_next = (n_ok && u + 2 < G) ? __ldg(wcol + (int64_t)(u + 2) * args.N) : hzero;
+        __syncwarp();
+      }
+    }
+    if (!ok) break;
+    if (active) {
+      if (pending) {   // the previous store has read the staging tile
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
+      float o[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) f2_unpack(y2[i], o[2 * i], o[2 * i + 1]);
+      stage16<Y_BF16>(args, t.n0 + c_lo, *reinterpret_cast<float(*)[16]>(o), srow, lane, 0);
+      if (c_lo + 16 < t.width)
+        stage16<Y_BF16>(args, t.n0 + c_lo + 16, *reinterpret_cast<float(*)[16]>(o + 16), srow, lane, 1);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmap_y, sbase, t.n0 + c_lo, t.m0 + quad * 32);
+        bulk_commit_group();
+      }
+      pending = true;
     }
   }
   // Every store has completed before the CTA (and its shared memory) exits.

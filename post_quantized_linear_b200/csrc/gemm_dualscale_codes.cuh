@@ -100,13 +100,17 @@ struct CodesCfg {
   static constexpr bool TMA_Y = SINGLE || MULTI || EPW != epi_warps(MULTI) ||
                                 (kStageBudget - EPW * stage_y_bytes(Y_BF16)) / STAGE >= 2;
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
-  static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
+  // group units: each epilogue warp's two 32-float buffers of widened weight scales
+  static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : 0;
+  static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) < 8
+                               ? ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) : 8;
   static_assert(KPS == 1 || !LDA_, "two k blocks per stage: TMA loads");
   static_assert(WM_ == 0 || (MULTI && !SINGLE && !LDA_ && KPS_ == 1 && BN_ == 128),
                 "group units: DualScale, one k block per stage, BN = 128");
   static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
   static constexpr int OFF_Y = S * STAGE;
-  static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
+  static constexpr int OFF_SW = OFF_Y + Y_BYTES;
+  static constexpr int OFF_BAR = OFF_SW + SW_BYTES;
   // full, empty; tmem full/empty; drain; (W4) unpacked
   static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -131,7 +135,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   constexpr bool SEEDED = (WM != 0);    // one unit per k block, seeded accumulators
   constexpr int EPI0 = codes_epi_warp0(LDA, W4);
   static_assert(EPW % 4 == 0 && (BN / (EPW / 4)) % 32 == 0, "32-column store passes per warp");
-  static_assert(!MULTI || (BN == 128 && C::NBUF == 2), "several units per tile: BN = 128, two buffers");
+  static_assert(!MULTI || (BN == 128 && C::NBUF == 2) || (C::NBUF == 1 && BN / (EPW / 4) == 64),
+                "several units per tile: BN = 128 with two buffers, or 64 columns per warp");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -356,9 +361,15 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     const int quad = warp & 3;
     const int part = (warp - EPI0) >> 2;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    if constexpr (C::TMA_Y) {
+    if constexpr (SEEDED) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, WM>(
+      float* sw_stage = reinterpret_cast<float*>(smem + C::OFF_SW) + (warp - EPI0) * 64;
+      epilogue_groups_tma_store<C::EPW, Y_BF16, WM>(
+          args, &tmap_y, stage_y, sw_stage, quad, part, lane, t_lane, tmem_full,
+          smem_u32(tmem_empty), rounds, tiles, abort_flag, budget);
+    } else if constexpr (C::TMA_Y) {
+      uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
+      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
           args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
           tiles, abort_flag, budget);
     } else {

@@ -185,6 +185,14 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, uint32_t v) {
                "r"(v)
                : "memory");
 }
+// 32 lanes x 16 consecutive 32-bit columns, every column set to v.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -189,6 +189,76 @@ __device__ __forceinline__ void hadamard16(float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], kHadamardNorm);
 }
 
+// ------------------------------------------- activation fused into the codes
+// SegQuant (Spanish technical summary 1 and 2.B; Korean technical summary
+// section 2 "DualScale"): the small negative tail DualScale keeps comes from
+// the SiLU / GELU that produces the layer input.  The fused producer reads
+// the pre-activation z and quantizes x = act(z) without storing x:
+//   SiLU(z) = z / (1 + e^-z),  GELU(z) = z/2 * erfc(-z / sqrt 2) (the exact,
+//   erf-based GELU),
+// with x the exact value rounded once, to nearest even, to bf16 (the
+// activation storage type of the workloads this replaces).
+//
+// Evaluation: in fp32 with CUDA's expf / erfcf, whose documented maximum
+// errors (2 and 4 units in the last place) bound the fp32 result's relative
+// error by `rel` units of 2^-24 (SiLU: the exponential, the sum and the
+// quotient; GELU: erfcf, the rounded argument -- whose relative error 2^-23 is
+// amplified by |d ln erfc(a) / d ln a| <= 2a^2 + 1 -- and two products), with a
+// safety factor of about two.  When no bf16 rounding midpoint lies within that
+// bound of the fp32 result, rounding it to bf16 gives the rounding of the
+// exact value; otherwise (about one element in ten thousand) the activation
+// is recomputed in fp64 (CUDA's exp / erfc, a relative error below 2^-44
+// here) and rounded from there.
+constexpr int ACT_SILU = 1, ACT_GELU = 2;
+
+// bf16 round-to-nearest-even of a double, directly (no intermediate fp32
+// rounding): the two bf16 neighbours of d and their midpoint are exact in
+// double.
+__device__ __forceinline__ float bf16_rn_of_double(double d) {
+  const float f = __double2float_rz(d);                 // |f| <= |d|, same sign
+  const uint32_t t = __float_as_uint(f) & 0xFFFF0000u;  // bf16 toward zero
+  const float lo = __uint_as_float(t);
+  const float hi = __uint_as_float(t + 0x10000u);       // next bf16 away from zero
+  const double mid = 0.5 * ((double)lo + (double)hi);
+  const double a = fabs(d), am = fabs(mid);
+  if (a > am) return hi;
+  if (a < am) return lo;
+  return ((t >> 16) & 1u) ? hi : lo;                    // a tie goes to the even one
+}
+
+template <int ACT>
+__device__ __forceinline__ double act_f64(float z) {
+  const double zd = (double)z;
+  if constexpr (ACT == ACT_SILU) return zd / (1.0 + exp(-zd));
+  else return 0.5 * zd * erfc(-zd * 0.70710678118654752440);
+}
+
+template <int ACT>
+__device__ __forceinline__ float act_bf16(float z) {
+  float v, rel;
+  if constexpr (ACT == ACT_SILU) {
+    v = __fdiv_rn(z, __fadd_rn(1.0f, expf(-z)));
+    rel = 16.0f;
+  } else {
+    const float a = __fmul_rn(z, -0.70710678f);
+    v = __fmul_rn(__fmul_rn(0.5f, z), erfcf(a));
+    rel = fmaf(8.0f * a, a, 24.0f);
+  }
+  // the bf16 rounding midpoint between v's two bf16 neighbours (same binade
+  // as v, so v - mid is exact)
+  const float mid = __uint_as_float((__float_as_uint(v) & 0xFFFF0000u) | 0x8000u);
+  const float margin = fmaf(rel * 5.9604645e-8f, fabsf(v), 1.0e-42f);
+  if (fabsf(__fsub_rn(v, mid)) <= margin || !(fabsf(v) <= 3.4028234663852886e38f))
+    return bf16_rn_of_double(act_f64<ACT>(z));
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+template <int ACT>
+__device__ __forceinline__ void act16(float (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = act_bf16<ACT>(v[i]);
+}
+
 // blockDim = (32, 8): lane x owns the 16-element group blockIdx.x*32 + x of
 // every row it visits (rows blockIdx.y*8 + y, stepping by gridDim.y*8), so its
 // segment and reciprocal scales are fixed; a warp reads 1 KiB (bf16) and
@@ -196,7 +266,10 @@ __device__ __forceinline__ void hadamard16(float (&v)[16]) {
 // MODE: CODES_DUAL (q+ and q-), CODES_COMBINED (c = q+ + q-), CODES_SINGLE
 // (the single-scale code: both branches with s = max(s+, s-)), CODES_HADAMARD
 // (q+ and q- of the block-Hadamard-transformed activations).
-constexpr int CODES_DUAL = 0, CODES_COMBINED = 1, CODES_SINGLE = 2, CODES_HADAMARD = 3;
+// CODES_SILU / CODES_GELU: the combined code c of x = bf16_RN(act(z)) from the
+// pre-activation z (the activation fused into the producer).
+constexpr int CODES_DUAL = 0, CODES_COMBINED = 1, CODES_SINGLE = 2, CODES_HADAMARD = 3,
+              CODES_SILU = 4, CODES_GELU = 5;
 
 template <typename XT, int MODE>
 __device__ __forceinline__ void quantize_activations_body(
@@ -206,7 +279,8 @@ __device__ __forceinline__ void quantize_activations_body(
   const int32_t k = (blockIdx.x * 32 + threadIdx.x) * 16;
   if (k >= K) return;
   const int j = kseg.segment_of(k);
-  constexpr bool COMBINED = (MODE == CODES_COMBINED || MODE == CODES_SINGLE);
+  constexpr bool COMBINED = (MODE == CODES_COMBINED || MODE == CODES_SINGLE ||
+                            MODE == CODES_SILU || MODE == CODES_GELU);
   const float sj_p = (MODE == CODES_SINGLE) ? fmaxf(s_pos[j], s_neg[j]) : s_pos[j];
   const float sj_n = (MODE == CODES_SINGLE) ? sj_p : s_neg[j];
   const float rp = sj_p > 0.0f ? __frcp_rn(sj_p) : 0.0f;
@@ -216,6 +290,8 @@ __device__ __forceinline__ void quantize_activations_body(
     float v[16];
     load16<XT>(x + (int64_t)m * ldx + k, v);
     if constexpr (MODE == CODES_HADAMARD) hadamard16(v);
+    if constexpr (MODE == CODES_SILU) act16<ACT_SILU>(v);
+    if constexpr (MODE == CODES_GELU) act16<ACT_GELU>(v);
     uint32_t p[16], n[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) { p[i] = code_pos(v[i], rp); n[i] = code_neg(v[i], rn); }
@@ -252,15 +328,16 @@ __global__ void __launch_bounds__(256) quantize_activations_hadamard_kernel(
   quantize_activations_body<XT, CODES_HADAMARD>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
 }
 
-// Calibration of the transformed activations: per K segment max(XH+) / 127
-// and max(-XH-) / 127.  blockDim = (32, 8) with the quantizer's layout (lane x
-// owns the 16-element group blockIdx.x*32 + x of every row it visits); eight
-// lanes cover 128 columns, which never straddle a segment bound, so an
-// eight-lane shuffle reduction is exact; then shared and global atomicMax on
-// the fp32 bit patterns as in calibrate_kernel.  The outputs must be zeroed
-// before the launch.
-template <typename XT>
-__global__ void __launch_bounds__(256) calibrate_hadamard_kernel(const XT* __restrict__ x,
+// Calibration of transformed activations: per K segment max(T+) / 127 and
+// max(-T-) / 127 of T = XH (XF = CODES_HADAMARD) or T = bf16_RN(act(Z))
+// (XF = CODES_SILU / CODES_GELU, Z the pre-activation).  blockDim = (32, 8)
+// with the quantizer's layout (lane x owns the 16-element group
+// blockIdx.x*32 + x of every row it visits); eight lanes cover 128 columns,
+// which never straddle a segment bound, so an eight-lane shuffle reduction is
+// exact; then shared and global atomicMax on the fp32 bit patterns as in
+// calibrate_kernel.  The outputs must be zeroed before the launch.
+template <typename XT, int XF = CODES_HADAMARD>
+__global__ void __launch_bounds__(256) calibrate_transformed_kernel(const XT* __restrict__ x,
                                                                  int64_t rows, int32_t K,
                                                                  int64_t ldx, SegBounds kseg,
                                                                  float* __restrict__ s_pos,
@@ -281,7 +358,9 @@ __global__ void __launch_bounds__(256) calibrate_hadamard_kernel(const XT* __res
     for (int64_t m = (int64_t)blockIdx.y * 8 + threadIdx.y; m < rows; m += step) {
       float v[16];
       load16<XT>(x + m * ldx + k, v);
-      hadamard16(v);
+      if constexpr (XF == CODES_HADAMARD) hadamard16(v);
+      if constexpr (XF == CODES_SILU) act16<ACT_SILU>(v);
+      if constexpr (XF == CODES_GELU) act16<ACT_GELU>(v);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         bad |= (v[i] != v[i]) || (fabsf(v[i]) == __int_as_float(0x7f800000));

@@ -244,7 +244,7 @@ template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULT
           int KPS = 1, int WM = 0>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (!LDA && KPS == 1 && WM == 0) {
+  if constexpr (!LDA && KPS == 1 && WM == 0 && !(MULTI && BN > 128)) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
   if constexpr (!LDA && KPS == 1 && WM == 0 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
@@ -532,13 +532,48 @@ int choose_bn(int64_t M, int64_t N, bool multi, bool f32x, bool codes_ring) {
   return c192 <= c128 ? 192 : 128;
 }
 
+// Tile width of the GEMM from codes when a tile folds several units (K
+// segments, int8 weights): 128 (two TMEM buffers, 16 epilogue warps), 192
+// (one buffer, 12 warps of 64 columns) or 256 (one buffer, 16 warps of 64
+// columns).  Per k block a tile needs 32 KiB of codes plus BN x 128 bytes of
+// weights per 4 x BN tensor-core cycles, against about 51 bytes per clock that
+// an SM's TMA engine delivers, so wider tiles run closer to the MMA rate
+// (about 0.53, 0.70 and 0.80 of it) but leave more tiles unbalanced over the
+// SMs; the makespan of the snake schedule over those rates decides.
+// SEGQUANT_BN overrides.
+int choose_bn_multi(int64_t M, int64_t N) {
+  if (const char* e = std::getenv("SEGQUANT_BN")) {
+    const int v = std::atoi(e);
+    if (v == 128 || v == 192 || v == 256) return v;
+  }
+  const int sms = num_sms();
+  const int64_t m_tiles = (M + sq::BM - 1) / sq::BM;
+  std::vector<double> load(sms);
+  auto cost = [&](int64_t bn, double eff) {
+    std::fill(load.begin(), load.end(), 0.0);
+    const int64_t n_full = N / bn, tail = N % bn;
+    const int64_t full_tiles = m_tiles * n_full;
+    const int64_t tiles = full_tiles + (tail ? m_tiles : 0);
+    for (int64_t idx = 0; idx < tiles; ++idx) {
+      const int64_t it = idx / sms, pos = idx % sms;
+      const int64_t cta = (it & 1) ? sms - 1 - pos : pos;
+      load[cta] += (double)(idx < full_tiles ? bn : std::max<int64_t>(tail, bn / 2)) / eff;
+    }
+    return *std::max_element(load.begin(), load.end());
+  };
+  const double c128 = cost(128, 0.53), c192 = cost(192, 0.70), c256 = cost(256, 0.80);
+  if (c256 <= c192 && c256 <= c128) return 256;
+  return c192 <= c128 ? 192 : 128;
+}
+
 // Codes of X: q+ and q- (CODES_DUAL), the combined code c = q+ + q-
 // (CODES_COMBINED) or the single-scale code (CODES_SINGLE), the last two
 // written to q_pos.
 sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
                          const sq_segments* kseg, const float* s_pos, const float* s_neg,
                          int8_t* q_pos, int8_t* q_neg, int64_t ldq, int mode, cudaStream_t s) {
-  const bool combined = (mode == sq::CODES_COMBINED || mode == sq::CODES_SINGLE);
+  const bool combined = (mode == sq::CODES_COMBINED || mode == sq::CODES_SINGLE ||
+                         mode == sq::CODES_SILU || mode == sq::CODES_GELU);
   if (!dtype_ok(xt) || M < 0 || K <= 0 || ldx < K || ldq < K) return SQ_ERR_INVALID_ARG;
   if (K > SQ_MAX_K) return SQ_ERR_RANGE;
   SegBounds sb;
@@ -569,6 +604,20 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
           static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
     else
       sq::quantize_activations_combined_kernel<float, sq::CODES_COMBINED><<<grid, block, 0, s>>>(
+          static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+  } else if (mode == sq::CODES_SILU) {
+    if (xt == SQ_BF16)
+      sq::quantize_activations_combined_kernel<bf, sq::CODES_SILU><<<grid, block, 0, s>>>(
+          static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+    else
+      sq::quantize_activations_combined_kernel<float, sq::CODES_SILU><<<grid, block, 0, s>>>(
+          static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+  } else if (mode == sq::CODES_GELU) {
+    if (xt == SQ_BF16)
+      sq::quantize_activations_combined_kernel<bf, sq::CODES_GELU><<<grid, block, 0, s>>>(
+          static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+    else
+      sq::quantize_activations_combined_kernel<float, sq::CODES_GELU><<<grid, block, 0, s>>>(
           static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
   } else if (mode == sq::CODES_SINGLE) {
     if (xt == SQ_BF16)
@@ -648,6 +697,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const bool pair = (src == ASource::Codes) && use_pair(N, w4);
   const bool codes_ring = (src == ASource::Codes) && !w4 && !pair && acc == nullptr && use_codes_ring();
   int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x, codes_ring);
+  if (multi && codes_ring) BN = choose_bn_multi(M, N);   // several K segments, from codes
   // one row tile, one unit per tile, GEMM from codes: narrow tiles over all SMs
   const int bn_small = (!multi && acc == nullptr && (src == ASource::Codes || src == ASource::Single) &&
                         !(src == ASource::Codes && use_pair(N, w4)) && use_codes_ring())
@@ -757,7 +807,11 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       CUtensorMap ty;
       st = make_tmap_y(&ty, y, yt, M, N, ldy);
       if (st != SQ_OK) return st;
-      if (multi) return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
+      if (multi) {
+        if (BN == 256) return launch_codes_out<256, true, false, 16>(yb, ta, ta2, tw, ty, a, stream);
+        if (BN == 192) return launch_codes_out<192, true, false, 12>(yb, ta, ta2, tw, ty, a, stream);
+        return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
+      }
       if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256 && codes_wide_epilogue())
         return launch_codes_out<256, false, false, 16>(yb, ta, ta2, tw, ty, a, stream);
@@ -965,9 +1019,15 @@ sq_status sq_linear_forward_single(const int8_t* c, int64_t ldc, int64_t M, int6
                      bias, y, yt, ldy, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
-sq_status sq_calibrate_hadamard(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
-                                const sq_segments* kseg, float* s_pos, float* s_neg,
-                                sq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Calibration of transformed rows (XH, or the activation of a pre-activation):
+// xf is sq::CODES_HADAMARD, sq::CODES_SILU or sq::CODES_GELU.
+sq_status calibrate_transformed(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
+                                const sq_segments* kseg, float* s_pos, float* s_neg, int xf,
+                                cudaStream_t s) {
   if (!dtype_ok(xt) || rows < 0 || K <= 0 || ldx < K) return SQ_ERR_INVALID_ARG;
   if (s_pos == nullptr || s_neg == nullptr) return SQ_ERR_INVALID_ARG;
   if (K > SQ_MAX_K) return SQ_ERR_RANGE;
@@ -982,7 +1042,6 @@ sq_status sq_calibrate_hadamard(const void* x, sq_dtype xt, int64_t rows, int64_
     if (x == nullptr) return SQ_ERR_INVALID_ARG;
     if (!aligned16(x) || (ldx * xe) % 16 != 0) return SQ_ERR_ALIGNMENT;
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bytes = sizeof(float) * (size_t)sb.count;
   sq_status ms = cuda_status(cudaMemsetAsync(s_pos, 0, bytes, s));
   if (ms != SQ_OK) return ms;
@@ -997,13 +1056,61 @@ sq_status sq_calibrate_hadamard(const void* x, sq_dtype xt, int64_t rows, int64_
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;
   dim3 grid(gx, (unsigned)gy), block(32, 8);
-  if (xt == SQ_BF16)
-    sq::calibrate_hadamard_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), rows, (int32_t)K, ldx, sb, s_pos, s_neg);
-  else
-    sq::calibrate_hadamard_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(x), rows,
-                                                                (int32_t)K, ldx, sb, s_pos, s_neg);
+  using bf = __nv_bfloat16;
+  const bf* xb = static_cast<const bf*>(x);
+  const float* xf32 = static_cast<const float*>(x);
+  const int32_t k32 = (int32_t)K;
+  if (xf == sq::CODES_SILU) {
+    if (xt == SQ_BF16)
+      sq::calibrate_transformed_kernel<bf, sq::CODES_SILU><<<grid, block, 0, s>>>(xb, rows, k32, ldx, sb, s_pos, s_neg);
+    else
+      sq::calibrate_transformed_kernel<float, sq::CODES_SILU><<<grid, block, 0, s>>>(xf32, rows, k32, ldx, sb, s_pos, s_neg);
+  } else if (xf == sq::CODES_GELU) {
+    if (xt == SQ_BF16)
+      sq::calibrate_transformed_kernel<bf, sq::CODES_GELU><<<grid, block, 0, s>>>(xb, rows, k32, ldx, sb, s_pos, s_neg);
+    else
+      sq::calibrate_transformed_kernel<float, sq::CODES_GELU><<<grid, block, 0, s>>>(xf32, rows, k32, ldx, sb, s_pos, s_neg);
+  } else {
+    if (xt == SQ_BF16)
+      sq::calibrate_transformed_kernel<bf><<<grid, block, 0, s>>>(xb, rows, k32, ldx, sb, s_pos, s_neg);
+    else
+      sq::calibrate_transformed_kernel<float><<<grid, block, 0, s>>>(xf32, rows, k32, ldx, sb, s_pos, s_neg);
+  }
   return cuda_status(cudaGetLastError());
+}
+
+int act_mode(sq_act act) {
+  return act == SQ_ACT_SILU ? sq::CODES_SILU : (act == SQ_ACT_GELU ? sq::CODES_GELU : -1);
+}
+
+}  // namespace
+
+extern "C" {
+
+sq_status sq_calibrate_hadamard(const void* x, sq_dtype xt, int64_t rows, int64_t K, int64_t ldx,
+                                const sq_segments* kseg, float* s_pos, float* s_neg,
+                                sq_stream_t stream) {
+  return calibrate_transformed(x, xt, rows, K, ldx, kseg, s_pos, s_neg, sq::CODES_HADAMARD,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_calibrate_act(const void* z, sq_dtype zt, sq_act act, int64_t rows, int64_t K,
+                           int64_t ldz, const sq_segments* kseg, float* s_pos, float* s_neg,
+                           sq_stream_t stream) {
+  const int mode = act_mode(act);
+  if (mode < 0) return SQ_ERR_INVALID_ARG;
+  return calibrate_transformed(z, zt, rows, K, ldz, kseg, s_pos, s_neg, mode,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quantize_activations_combined_act(const void* z, sq_dtype zt, sq_act act, int64_t M,
+                                               int64_t K, int64_t ldz, const sq_segments* kseg,
+                                               const float* s_pos, const float* s_neg, int8_t* c,
+                                               int64_t ldc, sq_stream_t stream) {
+  const int mode = act_mode(act);
+  if (mode < 0) return SQ_ERR_INVALID_ARG;
+  return quantize_codes(z, zt, M, K, ldz, kseg, s_pos, s_neg, c, nullptr, ldc, mode,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_quantize_activations_hadamard(const void* x, sq_dtype xt, int64_t M, int64_t K,
