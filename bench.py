@@ -68,7 +68,7 @@ NCU_TRAFFIC_BYTES = {
 
 
 def gemm_kernel_name(path: str, bits: int, x_dtype: str) -> str:
-    """The GEMM kernel a forward of this path launches (default switches)."""
+    """The GEMM kernel a forward of this path launches (product library)."""
     if path == "codes":          # int8 and int4 weights alike
         return "dualscale_gemm_codes_kernel"
     if bits == 4:
@@ -661,7 +661,7 @@ def measure_config(wl, dev, flush, steps: int, warmup: int, int8_peak: float, mm
     gemm_ms = statistics.mean(timed_graph(L.gemm_graph, steps, 3, flush, stream))
     fwd_ms = statistics.mean(timed_graph(L.fwd_graph, steps, 5, flush, stream))
     L.release()
-    ops, byts = wl.exec_ops, codes_gemm_bytes(wl)
+    ops, byts = wl.exec_ops, codes_gemm_bytes(wl, path)
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
     # a problem of a few MB and tens of MFLOP is launch-latency bound, not tensor bound
     bound = "latency" if byts < 16 * 2 ** 20 and ops < 10 ** 10 else "tensor"
@@ -681,9 +681,10 @@ def measure_config(wl, dev, flush, steps: int, warmup: int, int8_peak: float, mm
     }
 
 
-def codes_gemm_bytes(wl) -> int:
-    """Algorithmic bytes of one launch of the GEMM from codes: q+ and q- codes,
-    weight codes and scales, activation scales, bias, Y."""
+def codes_gemm_bytes(wl, path: str = "codes") -> int:
+    """Algorithmic bytes of one launch of the GEMM from codes: q+ and q- codes
+    (or the one combined code), weight codes and scales, activation scales,
+    bias, Y."""
     J = len(wl.kseg) - 1
     ye = 4 if wl.out == "f32" else 2
     if wl.bits == 8:
@@ -691,7 +692,8 @@ def codes_gemm_bytes(wl) -> int:
     else:
         wb = wl.N * wl.K // 2 + 2 * wl.N * (wl.K // 128)
     bb = 4 * wl.N if wl.bias_sigma is not None else 0
-    return 2 * wl.M * wl.K + wb + 8 * J + bb + wl.M * wl.N * ye
+    codes = (1 if path == "combined" else 2) * wl.M * wl.K
+    return codes + wb + 8 * J + bb + wl.M * wl.N * ye
 
 
 def num_sms(dev) -> int:
@@ -795,7 +797,7 @@ def run_ours(args):
         mma_peak = mma_rate_tops(num_sms(dev), sm_mhz)
         ops = wl.exec_ops
         gemm_tops = ops / (gemm_avg_ms * 1e-3) / 1e12
-        byts = codes_gemm_bytes(wl) if L.codes else wl.alg_bytes()
+        byts = codes_gemm_bytes(wl, args.path) if L.codes else wl.alg_bytes()
         line = {
             "metric": METRIC, "value": whole_job_tops(world, args.steps, ops, total_ms),
             "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

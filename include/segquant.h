@@ -381,14 +381,18 @@ const char* sq_status_string(sq_status status);
  * SQ_ERR_CUDA ("no CUDA error" if none).  Static string; host only. */
 const char* sq_last_cuda_error(void);
 
-/* Test hook: the device-side wait budget in clock cycles (default about one
- * second).  0 restores the default.  Host only; affects later launches. */
-void sq_set_wait_budget(int64_t cycles);
+/* Development library only (libsegquant_dev.so, built with SQ_DEV_BUILD; the
+ * product library libsegquant.so returns SQ_ERR_UNSUPPORTED and changes
+ * nothing).  Test hook: the device-side wait budget in clock cycles (default
+ * about one second); 0 restores the default.  Host only; affects later
+ * launches of the process. */
+sq_status sq_set_wait_budget(int64_t cycles);
 
-/* Test hook: while enabled, the GEMM kernels' TMA producer issues no copy, so
- * every consumer's bounded wait expires; the launch still returns SQ_OK and
- * sq_stream_status() then reports SQ_ERR_TIMEOUT.  Host only. */
-void sq_debug_starve_pipeline(int32_t enable);
+/* Development library only (as above).  Test hook: while enabled, the GEMM
+ * kernels' TMA producer issues no copy, so every consumer's bounded wait
+ * expires; the launch still returns SQ_OK and sq_stream_status() then reports
+ * SQ_ERR_TIMEOUT.  Host only. */
+sq_status sq_debug_starve_pipeline(int32_t enable);
 
 #ifdef __cplusplus
 }

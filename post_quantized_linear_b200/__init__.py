@@ -357,13 +357,15 @@ def stream_status(stream=None) -> int:
 
 
 def set_wait_budget(cycles: int) -> None:
-    """Device-side pipeline wait budget in SM clock cycles (0 = default, ~1 s)."""
-    _lib.load().sq_set_wait_budget(int(cycles))
+    """Test hook of the development library (inside ``_lib.dev_library()``):
+    device-side pipeline wait budget in SM clock cycles (0 = default, ~1 s)."""
+    _lib.check("sq_set_wait_budget", _lib.load().sq_set_wait_budget(int(cycles)))
 
 
 def debug_starve_pipeline(enable: bool) -> None:
-    """Test hook: GEMM launches issue no TMA copies, so their waits expire."""
-    _lib.load().sq_debug_starve_pipeline(1 if enable else 0)
+    """Test hook of the development library: GEMM launches issue no TMA
+    copies, so their waits expire."""
+    _lib.check("sq_debug_starve_pipeline", _lib.load().sq_debug_starve_pipeline(1 if enable else 0))
 
 
 # ------------------------------------------------- block-Hadamard activations

@@ -5,11 +5,15 @@ fails loudly when the compiled library is missing; there is no fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libsegquant.so")
+# The development build of the same sources: environment switches for the
+# measured alternative kernels and the two test hooks (tests only).
+DEV_LIB_PATH = os.path.join(PKG_DIR, "libsegquant_dev.so")
 
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED = 0, 1, 2, 3
 SQ_ERR_RANGE, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 4, 5, 6
@@ -75,28 +79,52 @@ SIGNATURES = {
     "sq_stream_status": (c_i32, [c_vp]),
     "sq_status_string": (ctypes.c_char_p, [c_i32]),
     "sq_last_cuda_error": (ctypes.c_char_p, []),
-    "sq_set_wait_budget": (None, [c_i64]),
-    "sq_debug_starve_pipeline": (None, [c_i32]),
+    "sq_set_wait_budget": (c_i32, [c_i64]),
+    "sq_debug_starve_pipeline": (c_i32, [c_i32]),
 }
 
-_lib = None
+_libs = {}
+_active = None   # the development library while dev_library() is open
 
 
-def load():
-    """Load ``libsegquant.so`` (built by ``post_quantized_linear_b200.build``)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
+def _open(path: str):
+    if path not in _libs:
+        if not os.path.exists(path):
             raise ImportError(
-                f"{LIB_PATH} is missing: build it with `python -m post_quantized_linear_b200.build`"
+                f"{path} is missing: build it with `python -m post_quantized_linear_b200.build`"
                 " (there is no CPU fallback)")
-        lib = ctypes.CDLL(LIB_PATH)
+        lib = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
-        _lib = lib
-    return _lib
+        _libs[path] = lib
+    return _libs[path]
+
+
+def load():
+    """The library the binding calls: ``libsegquant.so`` (built by
+    ``post_quantized_linear_b200.build``), or the development build inside
+    ``dev_library()``."""
+    return _active if _active is not None else _open(LIB_PATH)
+
+
+def load_dev():
+    """The development build ``libsegquant_dev.so``."""
+    return _open(DEV_LIB_PATH)
+
+
+@contextlib.contextmanager
+def dev_library():
+    """Route the binding's calls to the development build for the duration
+    (tests of the alternative kernels and of the wait hooks)."""
+    global _active
+    prev = _active
+    _active = load_dev()
+    try:
+        yield _active
+    finally:
+        _active = prev
 
 
 def status_string(code: int) -> str:

@@ -190,8 +190,12 @@ __device__ __forceinline__ bool wait1s(uint32_t bar, uint32_t parity, volatile i
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           long long budget) {
+  if (__all_sync(0xffffffffu, try_wait_scoped<CLUSTER>(bar, parity))) return true;
   const long long t0 = clock64();
   while (true) {
+    // a waiting warp sleeps between polls instead of taking issue slots from
+    // the warps that are computing
+    __nanosleep(64);
     const bool ok = try_wait_scoped<CLUSTER>(bar, parity);
     if (__all_sync(0xffffffffu, ok)) return true;
     int stop = 0;
@@ -1120,10 +1124,25 @@ __device__ __forceinline__ void epilogue_groups_tma_store(
             const float4 s = s4[q];
             const uint64_t sw_lo = f2_pack(s.x, s.y), sw_hi = f2_pack(s.z, s.w);
             const int i = 4 * q;
-            const uint64_t fp0 = f2_add(f2_pack(__uint_as_float(ap[i]), __uint_as_float(ap[i + 1])), mseed);
-            const uint64_t fn0 = f2_add(f2_pack(__uint_as_float(an[i]), __uint_as_float(an[i + 1])), mseed);
-            const uint64_t fp1 = f2_add(f2_pack(__uint_as_float(ap[i + 2]), __uint_as_float(ap[i + 3])), mseed);
-            const uint64_t fn1 = f2_add(f2_pack(__uint_as_float(an[i + 2]), __uint_as_float(an[i + 3])), mseed);
+            // F(acc): one exact subtraction per accumulator, packed for int4
+            // weights, scalar for the Hadamard-rotated codes (each measured
+            // faster for its kernel)
+            uint64_t fp0, fn0, fp1, fn1;
+            if constexpr (SEED == 1) {
+              fp0 = f2_add(f2_pack(__uint_as_float(ap[i]), __uint_as_float(ap[i + 1])), mseed);
+              fn0 = f2_add(f2_pack(__uint_as_float(an[i]), __uint_as_float(an[i + 1])), mseed);
+              fp1 = f2_add(f2_pack(__uint_as_float(ap[i + 2]), __uint_as_float(ap[i + 3])), mseed);
+              fn1 = f2_add(f2_pack(__uint_as_float(an[i + 2]), __uint_as_float(an[i + 3])), mseed);
+            } else {
+              fp0 = f2_pack(__fadd_rn(__uint_as_float(ap[i]), -seed_value),
+                            __fadd_rn(__uint_as_float(ap[i + 1]), -seed_value));
+              fn0 = f2_pack(__fadd_rn(__uint_as_float(an[i]), -seed_value),
+                            __fadd_rn(__uint_as_float(an[i + 1]), -seed_value));
+              fp1 = f2_pack(__fadd_rn(__uint_as_float(ap[i + 2]), -seed_value),
+                            __fadd_rn(__uint_as_float(ap[i + 3]), -seed_value));
+              fn1 = f2_pack(__fadd_rn(__uint_as_float(an[i + 2]), -seed_value),
+                            __fadd_rn(__uint_as_float(an[i + 3]), -seed_value));
+            }
             y2[4 * h + 2 * q] = f2_fma(sw_lo, f2_fma(sn2, fn0, f2_mul(sp2, fp0)), y2[4 * h + 2 * q]);
             y2[4 * h + 2 * q + 1] = f2_fma(sw_hi, f2_fma(sn2, fn1, f2_mul(sp2, fp1)), y2[4 * h + 2 * q + 1]);
           }

@@ -208,7 +208,8 @@ __device__ __forceinline__ void hadamard16(float (&v)[16]) {
 // bound of the fp32 result, rounding it to bf16 gives the rounding of the
 // exact value; otherwise (about one element in ten thousand) the activation
 // is recomputed in fp64 (CUDA's exp / erfc, a relative error below 2^-44
-// here) and rounded from there.
+// here) and rounded from there; so are results below 2^-110, where the fp32
+// intermediates overflow or lose precision.
 constexpr int ACT_SILU = 1, ACT_GELU = 2;
 
 // bf16 round-to-nearest-even of a double, directly (no intermediate fp32
@@ -247,8 +248,13 @@ __device__ __forceinline__ float act_bf16(float z) {
   // the bf16 rounding midpoint between v's two bf16 neighbours (same binade
   // as v, so v - mid is exact)
   const float mid = __uint_as_float((__float_as_uint(v) & 0xFFFF0000u) | 0x8000u);
-  const float margin = fmaf(rel * 5.9604645e-8f, fabsf(v), 1.0e-42f);
-  if (fabsf(__fsub_rn(v, mid)) <= margin || !(fabsf(v) <= 3.4028234663852886e38f))
+  const float margin = rel * 5.9604645e-8f * fabsf(v);
+  // Results below 2^-110 come from an exponential that overflowed (SiLU,
+  // z < -87) or an erfc near or in the fp32 subnormal range (GELU, z < -12),
+  // where the relative bound does not hold: those, like non-finite results,
+  // take the fp64 path too.
+  if (fabsf(__fsub_rn(v, mid)) <= margin || !(fabsf(v) >= 0x1p-110f) ||
+      !(fabsf(v) <= 3.4028234663852886e38f))
     return bf16_rn_of_double(act_f64<ACT>(z));
   return __bfloat162float(__float2bfloat16_rn(v));
 }
@@ -326,6 +332,96 @@ __global__ void __launch_bounds__(256) quantize_activations_hadamard_kernel(
     const float* __restrict__ s_pos, const float* __restrict__ s_neg, int8_t* __restrict__ q_pos,
     int8_t* __restrict__ q_neg, int64_t ldq) {
   quantize_activations_body<XT, CODES_HADAMARD>(x, M, K, ldx, kseg, s_pos, s_neg, q_pos, q_neg, ldq);
+}
+
+// ------------------------------------------ table-driven activation (bf16 Z)
+// A bf16 pre-activation has 65536 possible bit patterns, so x = act(z) for bf16
+// z is a table: lut[b] = bits of bf16_RN(act(z_b)), filled by act_table_kernel
+// with act_bf16 itself (the same values the direct path computes); non-finite
+// patterns map to a quiet NaN (inputs must be finite).
+constexpr int kActTableSize = 65536;
+
+template <int ACT>
+__global__ void __launch_bounds__(256) act_table_kernel(uint16_t* __restrict__ lut) {
+  const int b = blockIdx.x * 256 + threadIdx.x;
+  const float z = __uint_as_float((uint32_t)b << 16);
+  uint16_t r = 0x7FC0u;
+  if (fabsf(z) <= 3.4028234663852886e38f) r = (uint16_t)(__float_as_uint(act_bf16<ACT>(z)) >> 16);
+  lut[b] = r;
+}
+
+// Combined codes of x = act(z) for bf16 z through the table, staged in shared
+// memory (128 KiB, one block of 1024 threads per SM).  blockDim = (32, 32):
+// lane x owns the 16-element group blockIdx.x*32 + x of every row it visits
+// (rows blockIdx.y*32 + y, stepping by gridDim.y*32, two rows per iteration
+// so that four 16-byte loads are in flight per thread); the reciprocal scales
+// of every segment sit in shared memory.
+constexpr int kActRowsPerIter = 2;
+
+__global__ void __launch_bounds__(1024, 1) quantize_combined_act_table_kernel(
+    const __nv_bfloat16* __restrict__ z, int32_t M, int32_t K, int64_t ldz, SegBounds kseg,
+    const float* __restrict__ s_pos, const float* __restrict__ s_neg,
+    const uint16_t* __restrict__ lut, int8_t* __restrict__ c, int64_t ldc) {
+  extern __shared__ __align__(16) uint16_t tab[];     // kActTableSize entries
+  __shared__ float sh_rp[SQ_MAX_SEG], sh_rn[SQ_MAX_SEG];
+  const int tid = threadIdx.y * 32 + threadIdx.x;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(lut);
+    uint4* dst = reinterpret_cast<uint4*>(tab);
+    for (int i = tid; i < kActTableSize * 2 / 16; i += 1024) dst[i] = __ldg(src + i);
+  }
+  if (tid < kseg.count) {
+    const float sp = s_pos[tid], sn = s_neg[tid];
+    sh_rp[tid] = sp > 0.0f ? __frcp_rn(sp) : 0.0f;
+    sh_rn[tid] = sn > 0.0f ? __frcp_rn(sn) : 0.0f;
+  }
+  __syncthreads();
+  const int32_t k = (blockIdx.x * 32 + threadIdx.x) * 16;
+  if (k >= K) return;
+  const int j = kseg.segment_of(k);
+  const float rp = sh_rp[j], rn = sh_rn[j];
+  const int32_t step = gridDim.y * 32;
+  auto codes16 = [&](const uint4 (&u)[2], uint4& out) {
+    uint32_t p[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t w[4] = {u[h].x, u[h].y, u[h].z, u[h].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float x0 = __uint_as_float((uint32_t)tab[w[i] & 0xFFFFu] << 16);
+        const float x1 = __uint_as_float((uint32_t)tab[w[i] >> 16] << 16);
+        p[8 * h + 2 * i] = code_pos(x0, rp) + code_neg(x0, rn);
+        p[8 * h + 2 * i + 1] = code_pos(x1, rp) + code_neg(x1, rn);
+      }
+    }
+    out.x = pack4_low(p[0], p[1], p[2], p[3]);   out.y = pack4_low(p[4], p[5], p[6], p[7]);
+    out.z = pack4_low(p[8], p[9], p[10], p[11]); out.w = pack4_low(p[12], p[13], p[14], p[15]);
+  };
+  int32_t m = blockIdx.y * 32 + threadIdx.y;
+  for (; m + step < M; m += kActRowsPerIter * step) {
+    uint4 u[kActRowsPerIter][2];
+#pragma unroll
+    for (int r = 0; r < kActRowsPerIter; ++r) {
+      const uint4* src = reinterpret_cast<const uint4*>(z + (int64_t)(m + r * step) * ldz + k);
+      u[r][0] = __ldg(src);
+      u[r][1] = __ldg(src + 1);
+    }
+#pragma unroll
+    for (int r = 0; r < kActRowsPerIter; ++r) {
+      uint4 o;
+      codes16(u[r], o);
+      *reinterpret_cast<uint4*>(c + (int64_t)(m + r * step) * ldc + k) = o;
+    }
+  }
+  if (m < M) {
+    uint4 u[2];
+    const uint4* src = reinterpret_cast<const uint4*>(z + (int64_t)m * ldz + k);
+    u[0] = __ldg(src);
+    u[1] = __ldg(src + 1);
+    uint4 o;
+    codes16(u, o);
+    *reinterpret_cast<uint4*>(c + (int64_t)m * ldc + k) = o;
+  }
 }
 
 // Calibration of transformed activations: per K segment max(T+) / 127 and

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -29,13 +30,41 @@
 // once per device on the first call with that device current.
 static __device__ __align__(256) uint8_t g_splitk_scratch[SQ_SPLITK_STATIC_SCRATCH_BYTES];
 
+// Activation tables of the fused producer for bf16 pre-activations: entry b of
+// table a (0: SiLU, 1: GELU) is the bf16 pattern of act(z) for the bf16
+// pattern b of z.  Filled once per device context by act_table_kernel.
+static __device__ __align__(16) uint16_t g_act_table[2][sq::kActTableSize];
+
 namespace {
 
 using sq::SegBounds;
 
+// Development build (-DSQ_DEV_BUILD, libsegquant_dev.so): the environment
+// switches below select measured alternatives of the default kernels (kept so
+// that tests can prove them bit-identical to the defaults) and the two test
+// hooks (wait budget, starved pipeline) are live.  The product build
+// (libsegquant.so) reads no environment, compiles only the default kernels
+// and runs with the fixed wait budget.
+#ifdef SQ_DEV_BUILD
+constexpr bool kDev = true;
+#else
+constexpr bool kDev = false;
+#endif
+
 constexpr long long kDefaultWaitBudget = 2000000000LL;  // ~1 s of SM clock
-long long g_wait_budget = kDefaultWaitBudget;
+long long g_wait_budget = kDefaultWaitBudget;            // written by the development hooks only
 int g_debug_starve = 0;
+
+// An integer development switch: the environment's value in the development
+// build, `dflt` when unset and always in the product build.
+int dev_switch(const char* name, int dflt) {
+#ifdef SQ_DEV_BUILD
+  if (const char* e = std::getenv(name)) return std::atoi(e);
+#else
+  (void)name;
+#endif
+  return dflt;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int elt_size(sq_dtype t) { return t == SQ_F32 ? 4 : 2; }
@@ -128,21 +157,68 @@ sq_status check_qweight(const sq_qweight* w, int64_t K, SegBounds* kseg) {
   return SQ_OK;
 }
 
+constexpr int kMaxDevices = 64;
+
+// SM count of the current device, looked up once per device.
 int num_sms() {
+  static std::atomic<int> cached[kMaxDevices] = {};
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDevices && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return 148;
+  if (dev >= 0 && dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
   return n;
+}
+
+// Id of the calling thread's current CUDA context, 0 when there is none (or
+// it cannot be read).  Context ids are unique for the life of the process, so
+// a context re-created on the same device (after cudaDeviceReset) has a new id.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Raises kernel KERN's dynamic shared memory limit to `bytes`, once per
+// context (the attribute lasts as long as the context): later launches skip
+// the call.
+template <auto KERN>
+cudaError_t smem_limit(int bytes) {
+  static std::atomic<unsigned long long> done_ctx[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  const unsigned long long ctx = current_context_id();
+  if (cacheable && ctx != 0 && done_ctx[dev].load(std::memory_order_acquire) == ctx) return cudaSuccess;
+  e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cacheable && ctx != 0) done_ctx[dev].store(ctx, std::memory_order_release);
+  return e;
 }
 
 template <int BN, int ASRC, typename XT, bool W4, bool ACC, bool YB, bool MULTI>
 sq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tw,
                       sq::GemmArgs a, cudaStream_t stream) {
   using C = sq::GemmCfg<BN, ASRC, XT, W4>;
-  auto kern = sq::dualscale_gemm_kernel<BN, ASRC, XT, W4, ACC, YB, MULTI>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  constexpr auto kern = sq::dualscale_gemm_kernel<BN, ASRC, XT, W4, ACC, YB, MULTI>;
+  cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
   a.tail = a.N % BN;
@@ -170,9 +246,8 @@ template <int BN, bool ACC, bool YB, bool MULTI>
 sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tw,
                       sq::GemmArgs a, cudaStream_t stream) {
   using C = sq::PairCfg<BN>;
-  auto kern = sq::dualscale_gemm_pair_kernel<BN, ACC, YB, MULTI>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  constexpr auto kern = sq::dualscale_gemm_pair_kernel<BN, ACC, YB, MULTI>;
+  cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
   a.tail = a.N % BN;
@@ -199,9 +274,8 @@ template <int BN, bool ACC, bool YB, bool MULTI>
 sq_status launch_inplace(const CUtensorMap& tx, const CUtensorMap& tw, sq::GemmArgs a,
                          cudaStream_t stream) {
   using C = sq::InplaceCfg<BN>;
-  auto kern = sq::dualscale_gemm_inplace_kernel<BN, ACC, YB, MULTI>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  constexpr auto kern = sq::dualscale_gemm_inplace_kernel<BN, ACC, YB, MULTI>;
+  cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
   a.tail = a.N % BN;
@@ -227,33 +301,27 @@ sq_status launch_inplace_out(bool acc, bool y_bf16, const CUtensorMap& tx, const
 // Whether the GEMM from codes copies the code tiles with cp.async loader warps
 // (TMA then carries only the weight tile); off unless SEGQUANT_CODES_LDA=1
 // (measured slower than all-TMA loads on the DiT, MMDiT and SegLinear shapes).
-bool use_codes_lda() {
-  if (const char* e = std::getenv("SEGQUANT_CODES_LDA")) return std::atoi(e) != 0;
-  return false;
-}
+bool use_codes_lda() { return dev_switch("SEGQUANT_CODES_LDA", 0) != 0; }
 
 
 // k blocks per pipeline stage of the GEMM from codes (2 for TMA loads at
 // BN <= 192, where two such stages fit; 1 otherwise); SEGQUANT_KPS=1 forces one.
-int codes_kps() {
-  if (const char* e = std::getenv("SEGQUANT_KPS")) return std::atoi(e) == 2 ? 2 : 1;
-  return 2;
-}
+int codes_kps() { return dev_switch("SEGQUANT_KPS", 2) == 2 ? 2 : 1; }
 
 template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false,
           int KPS = 1, int WM = 0>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (!LDA && KPS == 1 && WM == 0 && !(MULTI && BN > 128)) {
+  if constexpr (kDev && !LDA && KPS == 1 && WM == 0 && !(MULTI && BN > 128)) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
   if constexpr (!LDA && KPS == 1 && WM == 0 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
-    if (codes_kps() == 2) return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
+    if (codes_kps() == 2)
+      return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
   }
   using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, WM>;
-  auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  constexpr auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM>;
+  cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
   a.tail = a.N % BN;
@@ -276,18 +344,12 @@ sq_status launch_codes_out(bool y_bf16, const CUtensorMap& tqp, const CUtensorMa
 // Whether int4 weights run through the GEMM from codes (unpack warps, one
 // ring of stages, seeded accumulators); SEGQUANT_W4_CODES=0 selects the
 // operand-ring kernel with producer warps.
-bool use_codes_w4() {
-  if (const char* e = std::getenv("SEGQUANT_W4_CODES")) return std::atoi(e) != 0;
-  return true;
-}
+bool use_codes_w4() { return dev_switch("SEGQUANT_W4_CODES", 1) != 0; }
 
 // Whether 256-wide tiles of the GEMM from codes drain TMEM with 16 epilogue
 // warps instead of 8 (one TMEM buffer at that width: the MMA waits for the
 // drain); SEGQUANT_EPW16=0|1 overrides the default.
-bool codes_wide_epilogue() {
-  if (const char* e = std::getenv("SEGQUANT_EPW16")) return std::atoi(e) != 0;
-  return true;
-}
+bool codes_wide_epilogue() { return dev_switch("SEGQUANT_EPW16", 1) != 0; }
 
 // Small M (one row tile): the work is streaming the weight codes, so the tile
 // width spreads N over as many SMs as possible.  Candidates 32..256 (multiples
@@ -296,8 +358,8 @@ bool codes_wide_epilogue() {
 // ties go to the narrower tile (more SMs share the stream).  0 = not small.
 int choose_bn_small(int64_t M, int64_t N) {
   if (M > sq::BM) return 0;
-  if (const char* e = std::getenv("SEGQUANT_BN_SMALL")) {
-    const int v = std::atoi(e);
+  {
+    const int v = dev_switch("SEGQUANT_BN_SMALL", 0);
     if (v == 32 || v == 64 || v == 96 || v == 128) return v;
     if (v == -1) return 0;   // the regular tile choice
   }
@@ -342,9 +404,8 @@ template <int BN, bool YB, bool MULTI>
 sq_status launch_combined(const CUtensorMap& tc, const CUtensorMap& tw, sq::GemmArgs a,
                           cudaStream_t stream) {
   using C = sq::CombinedCfg<BN>;
-  auto kern = sq::dualscale_gemm_combined_kernel<BN, YB, MULTI>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  constexpr auto kern = sq::dualscale_gemm_combined_kernel<BN, YB, MULTI>;
+  cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
   a.tail = a.N % BN;
@@ -402,34 +463,41 @@ bool plan_splitk_capped(int64_t M, int64_t N, int64_t K, size_t cap, SplitPlan* 
   return false;
 }
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
-// Id of the calling thread's current CUDA context, 0 when there is none (or
-// it cannot be read).  Context ids are unique for the life of the process, so
-// a context re-created on the same device (after cudaDeviceReset) has a new id.
-unsigned long long current_context_id() {
-  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
-  static PFN_cuCtxGetId_v12000 get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
+std::mutex g_table_mu;
+const uint16_t* g_table_ptr[kMaxDevices] = {};
+unsigned long long g_table_ctx[kMaxDevices] = {};
+
+// Device address of the filled activation tables in the current context.  The
+// first call per device (and per re-created context) launches the two table
+// kernels on `s` and waits for them, so that calls on any stream find the
+// tables complete.
+sq_status act_tables(cudaStream_t s, const uint16_t** out) {
+  int dev = 0;
+  sq_status st = cuda_status(cudaGetDevice(&dev));
+  if (st != SQ_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return SQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_table_mu);
+  const unsigned long long ctx = current_context_id();
+  if (g_table_ptr[dev] == nullptr || ctx == 0 || ctx != g_table_ctx[dev]) {
     void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-  });
-  if (get_current == nullptr || get_id == nullptr) return 0;
-  CUcontext c = nullptr;
-  unsigned long long id = 0;
-  if (get_current(&c) != CUDA_SUCCESS || c == nullptr || get_id(c, &id) != CUDA_SUCCESS) return 0;
-  return id;
+    st = cuda_status(cudaGetSymbolAddress(&p, g_act_table));
+    if (st != SQ_OK) return st;
+    uint16_t* t = static_cast<uint16_t*>(p);
+    sq::act_table_kernel<sq::ACT_SILU><<<sq::kActTableSize / 256, 256, 0, s>>>(t);
+    sq::act_table_kernel<sq::ACT_GELU><<<sq::kActTableSize / 256, 256, 0, s>>>(t + sq::kActTableSize);
+    st = cuda_status(cudaGetLastError());
+    if (st != SQ_OK) return st;
+    st = cuda_status(cudaStreamSynchronize(s));
+    if (st != SQ_OK) return st;
+    g_table_ptr[dev] = t;
+    g_table_ctx[dev] = current_context_id();
+  }
+  *out = g_table_ptr[dev];
+  return SQ_OK;
 }
 
 // Device address of g_splitk_scratch in the current device's context: looked
@@ -458,9 +526,8 @@ template <int BN, bool YB>
 sq_status launch_splitk(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                         sq::GemmArgs a, cudaStream_t stream) {
   using C = sq::SplitKCfg<BN>;
-  auto kern = sq::dualscale_gemm_splitk_kernel<BN, YB>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  constexpr auto kern = sq::dualscale_gemm_splitk_kernel<BN, YB>;
+  cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   int grid = num_sms();
   const int units = a.num_tiles * a.splits;
@@ -472,26 +539,21 @@ sq_status launch_splitk(const CUtensorMap& tqp, const CUtensorMap& tqn, const CU
 // Whether the GEMM from int8 codes runs the one-ring kernel (codes and weight
 // tile in one stage); SEGQUANT_CODES_RING=0 selects the kernel with separate
 // operand rings.
-bool use_codes_ring() {
-  if (const char* e = std::getenv("SEGQUANT_CODES_RING")) return std::atoi(e) != 0;
-  return true;
-}
+bool use_codes_ring() { return dev_switch("SEGQUANT_CODES_RING", 1) != 0; }
 
 // Whether the fused path quantizes bf16 activations in place (one ring of
 // stages): int8 weights; SEGQUANT_INPLACE=0 selects the separate-ring kernel.
 bool use_inplace(bool w4) {
   if (w4) return false;
-  if (const char* e = std::getenv("SEGQUANT_INPLACE")) return std::atoi(e) != 0;
-  return true;
+  return dev_switch("SEGQUANT_INPLACE", 1) != 0;
 }
 
 // Whether the GEMM from codes runs on CTA pairs (2-SM UMMA): int8 weights and a
 // last tile width that is a multiple of 32 (pair MMA N granularity).
 // SEGQUANT_PAIR=0|1 overrides the default.
 bool use_pair(int64_t N, bool w4) {
-  if (w4 || N % 32 != 0) return false;
-  if (const char* e = std::getenv("SEGQUANT_PAIR")) return std::atoi(e) != 0;
-  return false;
+  if (!kDev || w4 || N % 32 != 0) return false;
+  return dev_switch("SEGQUANT_PAIR", 0) != 0;
 }
 
 // Output-tile width.  Several units per tile need double-buffered TMEM, which
@@ -506,8 +568,8 @@ bool use_pair(int64_t N, bool w4) {
 // SEGQUANT_BN=128|192|256 overrides the choice (a tuning knob).
 int choose_bn(int64_t M, int64_t N, bool multi, bool f32x, bool codes_ring) {
   if (multi || f32x) return 128;
-  if (const char* e = std::getenv("SEGQUANT_BN")) {
-    const int v = std::atoi(e);
+  {
+    const int v = dev_switch("SEGQUANT_BN", 0);
     if (v == 128 || v == 192 || v == 256) return v;
   }
   const int sms = num_sms();
@@ -542,8 +604,8 @@ int choose_bn(int64_t M, int64_t N, bool multi, bool f32x, bool codes_ring) {
 // SMs; the makespan of the snake schedule over those rates decides.
 // SEGQUANT_BN overrides.
 int choose_bn_multi(int64_t M, int64_t N) {
-  if (const char* e = std::getenv("SEGQUANT_BN")) {
-    const int v = std::atoi(e);
+  {
+    const int v = dev_switch("SEGQUANT_BN", 0);
     if (v == 128 || v == 192 || v == 256) return v;
   }
   const int sms = num_sms();
@@ -605,6 +667,21 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
     else
       sq::quantize_activations_combined_kernel<float, sq::CODES_COMBINED><<<grid, block, 0, s>>>(
           static_cast<const float*>(x), (int32_t)M, (int32_t)K, ldx, sb, s_pos, s_neg, q_pos, ldq);
+  } else if ((mode == sq::CODES_SILU || mode == sq::CODES_GELU) && xt == SQ_BF16) {
+    // bf16 pre-activations: through the activation table in shared memory
+    const uint16_t* tables = nullptr;
+    st = act_tables(s, &tables);
+    if (st != SQ_OK) return st;
+    const uint16_t* lut = tables + (mode == sq::CODES_GELU ? sq::kActTableSize : 0);
+    constexpr int kTableSmem = sq::kActTableSize * 2;
+    constexpr auto kern = sq::quantize_combined_act_table_kernel;
+    st = cuda_status(smem_limit<kern>(kTableSmem));
+    if (st != SQ_OK) return st;
+    const int64_t ty = std::min<int64_t>((M + 31) / 32,
+                                         std::max<int64_t>(1, (num_sms() + gx - 1) / gx));
+    dim3 tgrid(gx, (unsigned)std::min<int64_t>(ty, 65535)), tblock(32, 32);
+    kern<<<tgrid, tblock, kTableSmem, s>>>(static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx,
+                                           sb, s_pos, s_neg, lut, q_pos, ldq);
   } else if (mode == sq::CODES_SILU) {
     if (xt == SQ_BF16)
       sq::quantize_activations_combined_kernel<bf, sq::CODES_SILU><<<grid, block, 0, s>>>(
@@ -705,7 +782,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   if (bn_small) BN = bn_small;
   if (pair && !multi && acc == nullptr) {
     BN = 256;
-    if (const char* e = std::getenv("SEGQUANT_BN")) BN = std::atoi(e) == 128 ? 128 : 256;
+    BN = dev_switch("SEGQUANT_BN", 256) == 128 ? 128 : 256;
   }
   // One row tile of fewer than BM rows, read by the GEMM from codes: code boxes
   // of M rows rounded up to 16 instead of mostly out-of-bounds 128-row boxes.
@@ -757,8 +834,8 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   a.y = y;
   a.ldy = ldy;
   a.acc_out = acc;
-  a.wait_budget = g_wait_budget;
-  a.starve = g_debug_starve;
+  a.wait_budget = kDev ? g_wait_budget : kDefaultWaitBudget;
+  a.starve = kDev ? g_debug_starve : 0;
   a.a_pos = q_pos;
   a.a_neg = q_neg;
   a.lda = ldq;
@@ -790,10 +867,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     if (BN == 192) return launch_combined_out<192, false>(yb, ta, tw, a, stream);
     return launch_combined_out<128, false>(yb, ta, tw, a, stream);
   }
-  if (pair) {
-    if (multi || ac) return launch_pair_out<128, true>(ac, yb, ta, ta2, tw, a, stream);
-    if (BN == 256) return launch_pair_out<256, false>(ac, yb, ta, ta2, tw, a, stream);
-    return launch_pair_out<128, false>(ac, yb, ta, ta2, tw, a, stream);
+  if constexpr (kDev) {   // 2-SM pair tiles: a measured alternative
+    if (pair) {
+      if (multi || ac) return launch_pair_out<128, true>(ac, yb, ta, ta2, tw, a, stream);
+      if (BN == 256) return launch_pair_out<256, false>(ac, yb, ta, ta2, tw, a, stream);
+      return launch_pair_out<128, false>(ac, yb, ta, ta2, tw, a, stream);
+    }
   }
   if (src == ASource::Codes) {
     if (codes_w4) {
@@ -802,7 +881,9 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       if (st != SQ_OK) return st;
       return launch_codes_out<128, true, false, sq::epi_warps(true), 1>(yb, ta, ta2, tw, ty, a, stream);
     }
-    if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
+    if constexpr (kDev) {   // int4 through the operand-ring kernel
+      if (w4) return launch_out<128, AC, bf, true, true>(ac, yb, ta, ta2, tw, a, stream);
+    }
     if (!ac && use_codes_ring()) {
       CUtensorMap ty;
       st = make_tmap_y(&ty, y, yt, M, N, ldy);
@@ -815,14 +896,19 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256 && codes_wide_epilogue())
         return launch_codes_out<256, false, false, 16>(yb, ta, ta2, tw, ty, a, stream);
-      if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, ty, a, stream);
+      if constexpr (kDev) {   // eight epilogue warps at BN = 256
+        if (BN == 256) return launch_codes_out<256, false>(yb, ta, ta2, tw, ty, a, stream);
+      }
       if (BN == 192) return launch_codes_out<192, false>(yb, ta, ta2, tw, ty, a, stream);
       return launch_codes_out<128, false>(yb, ta, ta2, tw, ty, a, stream);
     }
-    if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
-    if (BN == 256) return launch_out<256, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
-    if (BN == 192) return launch_out<192, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
-    return launch_out<128, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+    if constexpr (kDev) {   // separate operand rings
+      if (multi || ac) return launch_out<128, AC, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
+      if (BN == 256) return launch_out<256, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+      if (BN == 192) return launch_out<192, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+      return launch_out<128, AC, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+    }
+    return SQ_ERR_UNSUPPORTED;   // not reached in the product build
   }
   if (f32x) {
     if (w4) return launch_out<128, AX, float, true, true>(ac, yb, ta, ta2, tw, a, stream);
@@ -836,10 +922,13 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     if (BN == 192) return launch_inplace_out<192, false>(ac, yb, ta, tw, a, stream);
     return launch_inplace_out<128, false>(ac, yb, ta, tw, a, stream);
   }
-  if (multi || ac) return launch_out<128, AX, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
-  if (BN == 256) return launch_out<256, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
-  if (BN == 192) return launch_out<192, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
-  return launch_out<128, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+  if constexpr (kDev) {   // bf16 activations quantized by producer warps into separate tiles
+    if (multi || ac) return launch_out<128, AX, bf, false, true>(ac, yb, ta, ta2, tw, a, stream);
+    if (BN == 256) return launch_out<256, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+    if (BN == 192) return launch_out<192, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+    return launch_out<128, AX, bf, false, false>(ac, yb, ta, ta2, tw, a, stream);
+  }
+  return SQ_ERR_UNSUPPORTED;   // not reached in the product build
 }
 
 }  // namespace
@@ -863,9 +952,17 @@ const char* sq_status_string(sq_status s) {
   return "SQ_UNKNOWN_STATUS";
 }
 
-void sq_set_wait_budget(int64_t cycles) { g_wait_budget = cycles > 0 ? cycles : kDefaultWaitBudget; }
+sq_status sq_set_wait_budget(int64_t cycles) {
+  if constexpr (!kDev) return SQ_ERR_UNSUPPORTED;
+  g_wait_budget = cycles > 0 ? cycles : kDefaultWaitBudget;
+  return SQ_OK;
+}
 
-void sq_debug_starve_pipeline(int32_t enable) { g_debug_starve = enable != 0; }
+sq_status sq_debug_starve_pipeline(int32_t enable) {
+  if constexpr (!kDev) return SQ_ERR_UNSUPPORTED;
+  g_debug_starve = enable != 0;
+  return SQ_OK;
+}
 
 sq_status sq_qweight_sizes(int32_t bits, int64_t N, int64_t K, int32_t J, int32_t group,
                            size_t* code_bytes, size_t* scale_bytes) {
@@ -1208,8 +1305,8 @@ sq_status sq_linear_forward_codes_splitk(const int8_t* q_pos, const int8_t* q_ne
   a.bias = bias;
   a.y = y;
   a.ldy = ldy;
-  a.wait_budget = g_wait_budget;
-  a.starve = g_debug_starve;
+  a.wait_budget = kDev ? g_wait_budget : kDefaultWaitBudget;
+  a.starve = kDev ? g_debug_starve : 0;
   a.splits = p.splits;
   a.kb_per_split = p.kb_per_split;
   a.ws_count = static_cast<int32_t*>(workspace);
@@ -1276,8 +1373,8 @@ sq_status sq_linear_forward_codes_splitk_static(const int8_t* q_pos, const int8_
   a.bias = bias;
   a.y = y;
   a.ldy = ldy;
-  a.wait_budget = g_wait_budget;
-  a.starve = g_debug_starve;
+  a.wait_budget = kDev ? g_wait_budget : kDefaultWaitBudget;
+  a.starve = kDev ? g_debug_starve : 0;
   a.splits = p.splits;
   a.kb_per_split = p.kb_per_split;
   a.ws_count = static_cast<int32_t*>(scratch);

@@ -25,3 +25,13 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture
+def dev_lib():
+    """The binding routed to the development build (libsegquant_dev.so: the
+    environment switches of the measured alternative kernels and the wait
+    hooks) for one test."""
+    from post_quantized_linear_b200 import _lib
+    with _lib.dev_library() as lib:
+        yield lib

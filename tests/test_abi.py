@@ -19,12 +19,33 @@ def declared_functions():
 
 
 def test_library_exports_every_declared_entry_point():
-    lib = _lib.load()
     names = declared_functions()
     assert len(names) >= 9
-    for n in names:
-        assert hasattr(lib, n), n
-        assert n in _lib.SIGNATURES, n
+    for lib in (_lib.load(), _lib.load_dev()):
+        for n in names:
+            assert hasattr(lib, n), n
+            assert n in _lib.SIGNATURES, n
+
+
+def test_test_hooks_live_only_in_the_development_library():
+    """The product library refuses the wait hooks (fixed budget, no starvation
+    switch); the development build accepts them."""
+    prod, dev = _lib.load(), _lib.load_dev()
+    assert prod.sq_set_wait_budget(1000) == _lib.SQ_ERR_UNSUPPORTED
+    assert prod.sq_debug_starve_pipeline(1) == _lib.SQ_ERR_UNSUPPORTED
+    assert dev.sq_set_wait_budget(0) == _lib.SQ_OK
+    assert dev.sq_debug_starve_pipeline(0) == _lib.SQ_OK
+
+
+def test_product_library_reads_no_environment():
+    """No switch of the product build reads the environment: the variable names
+    the development build's switches look up are absent from the product
+    library's binary, present in the development library's."""
+    def has_switch_names(path):
+        data = open(path, "rb").read()
+        return b"SEGQUANT_BN" in data or b"SEGQUANT_PAIR" in data or b"SEGQUANT_KPS" in data
+    assert not has_switch_names(_lib.LIB_PATH)
+    assert has_switch_names(_lib.DEV_LIB_PATH)
 
 
 def test_binding_arity_matches_every_declaration():
@@ -244,7 +265,8 @@ def test_hadamard_entry_points_validate_before_launch():
 
 
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
-    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "_libs", {})
+    monkeypatch.setattr(_lib, "_active", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         _lib.load()

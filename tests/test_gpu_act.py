@@ -154,3 +154,33 @@ def test_fused_activation_full_size_every_element(name, act):
         np.testing.assert_array_equal(part[~flags], oc[~flags])
     print(f"{name} {act}: {flagged} elements flagged as undecided in double")
     assert flagged <= 4
+
+
+@pytest.mark.parametrize("act", ["silu", "gelu"])
+def test_table_and_direct_paths_agree_on_every_bf16_input(act):
+    """bf16 pre-activations go through the activation table, fp32 ones through
+    the direct evaluation: on all 65536 bf16 patterns (non-finite ones replaced
+    by zero) both give the oracle's codes."""
+    import post_quantized_linear_b200 as pq
+    bits = np.arange(65536, dtype=np.uint32)
+    finite = ((bits >> 7) & 0xFF) != 0xFF
+    bits = np.where(finite, bits, 0).astype(np.uint16).reshape(64, 1024)
+    z32 = (bits.astype(np.uint32) << 16).view(np.float32)
+    kseg = [0, 512, 1024]
+    osp = np.float32([2.0 ** -3, 0.0371])
+    osn = np.float32([2.0 ** -5, 0.0113])
+    sp, sn = torch.from_numpy(osp).cuda(), torch.from_numpy(osn).cuda()
+    zb = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    c_tab = pq.quantize_activations_combined_act(zb, act, kseg, sp, sn)
+    c_dir = pq.quantize_activations_combined_act(torch.from_numpy(z32).cuda(), act, kseg, sp, sn)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    oc, flags = O.quantize_activations_combined_act(bits, act, kseg, osp, osn)
+    # Only |z| < 2^-125 can be undecided: act(z) = z/2 + O(z^2) there, z/2 falls
+    # in bf16's subnormal range where it is a rounding midpoint for half of
+    # them, and the O(z^2) term lies far below double precision; every flagged
+    # element must be one of those.
+    tiny = np.abs(z32) < 2.0 ** -125
+    assert not flags[~tiny].any()
+    np.testing.assert_array_equal(c_tab.cpu().numpy()[~flags], oc[~flags])
+    np.testing.assert_array_equal(c_dir.cpu().numpy()[~flags], oc[~flags])

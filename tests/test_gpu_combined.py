@@ -56,7 +56,7 @@ def test_combined_codes_bit_exact(i):
 
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("i", range(len(CASES)))
-def test_forward_from_combined_matches_oracle_and_fused(i, bn, monkeypatch):
+def test_forward_from_combined_matches_oracle_and_fused(i, bn, monkeypatch, dev_lib):
     import post_quantized_linear_b200 as pq
     monkeypatch.setenv("SEGQUANT_BN", bn)
     c = Case(_case(i))
@@ -101,7 +101,7 @@ def test_combined_rejects_int4_weights():
         pq.linear_from_combined(code, c.qw, c.sp, c.sn, c.b)
 
 
-def test_combined_starved_pipeline_times_out_and_context_recovers():
+def test_combined_starved_pipeline_times_out_and_context_recovers(dev_lib):
     import post_quantized_linear_b200 as pq
     from post_quantized_linear_b200 import _lib
     c = Case(_case(0))

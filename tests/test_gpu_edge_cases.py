@@ -135,16 +135,21 @@ FUSED = [("bf16", 8, "1"), ("bf16", 8, "0"), ("bf16", 4, "1"), ("f32", 8, "1"), 
 
 @pytest.mark.parametrize("dtype,bits,inplace", FUSED)
 def test_fused_quantizers_edge_accumulators_and_fp32_outputs(dtype, bits, inplace, monkeypatch):
+    """The in-place option off is a measured alternative: it runs in the
+    development build; every other case runs in the product library."""
+    import contextlib
     import post_quantized_linear_b200 as pq
+    from post_quantized_linear_b200 import _lib
     monkeypatch.setenv("SEGQUANT_INPLACE", inplace)
     xd, xo, sp, sn, osp, osn = _inputs(dtype, 5 + bits)
     K = E.EDGE_KSEG[-1]
     w = _identity_plus_random_weight(K, 48, seed=bits)           # N = 560: ragged N tail
     bias = torch.randn(w.shape[0], generator=torch.Generator().manual_seed(9)) * 0.01
-    qw = pq.quantize_weights(w.cuda(), E.EDGE_KSEG, bits=bits)
-    acc = pq.linear_accumulators(xd, qw, sp, sn)
-    y = pq.linear(xd, qw, sp, sn, bias.cuda(), out_dtype=torch.float32)
-    _status_ok()
+    with (_lib.dev_library() if inplace == "0" else contextlib.nullcontext()):
+        qw = pq.quantize_weights(w.cuda(), E.EDGE_KSEG, bits=bits)
+        acc = pq.linear_accumulators(xd, qw, sp, sn)
+        y = pq.linear(xd, qw, sp, sn, bias.cuda(), out_dtype=torch.float32)
+        _status_ok()
     if bits == 8:
         wc, ws = O.quantize_weights_w8(w.numpy(), E.EDGE_KSEG)
     else:

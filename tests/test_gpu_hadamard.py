@@ -129,7 +129,7 @@ def test_hadamard_full_size_every_row():
         h.compare_rows(y, rows)
 
 
-def test_hadamard_starved_pipeline_times_out_and_context_recovers():
+def test_hadamard_starved_pipeline_times_out_and_context_recovers(dev_lib):
     import post_quantized_linear_b200 as pq
     from post_quantized_linear_b200 import _lib
     h = HCase(_case(0))

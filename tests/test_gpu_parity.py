@@ -96,7 +96,7 @@ def test_forward_from_codes_equals_fused(i):
 
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("codes", [False, True])
-def test_tile_width_variants_match_oracle(bn, codes, monkeypatch):
+def test_tile_width_variants_match_oracle(bn, codes, monkeypatch, dev_lib):
     """Both output-tile widths (BN = 128 double-buffered TMEM, BN = 256 single
     buffer with the streaming epilogue), fused and from codes, on ragged shapes."""
     import post_quantized_linear_b200 as pq
@@ -114,7 +114,7 @@ def test_tile_width_variants_match_oracle(bn, codes, monkeypatch):
 
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("i", [0, 1, 2, 5])
-def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch):
+def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch, dev_lib):
     """The GEMM from codes with one ring of stages (codes and weights in one
     stage) and with separate operand rings: the oracle's result, bit-identical
     to each other, on one and several K segments, bf16 and fp32 outputs."""
@@ -136,7 +136,7 @@ def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch):
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("MKN", [(390, 768, 656), (300, 640, 272), (64, 1024, 512), (1, 256, 96),
                                  (300, 640, 272, (0, 256, 640))])
-def test_code_tiles_by_cp_async_or_tma_agree(MKN, bn, monkeypatch):
+def test_code_tiles_by_cp_async_or_tma_agree(MKN, bn, monkeypatch, dev_lib):
     """The GEMM from codes with the code tiles copied by cp.async loader warps
     and with every operand loaded by TMA: the oracle's result, identical bits,
     DualScale and single-scale, ragged M, N and K tails, one and two K segments."""
@@ -166,7 +166,7 @@ def test_code_tiles_by_cp_async_or_tma_agree(MKN, bn, monkeypatch):
 @pytest.mark.parametrize("MKN", [(390, 640, 656), (300, 1040, 272), (129, 768, 400), (64, 3072, 1024),
                                  (300, 640, 272, (0, 256, 640)),
                                  (257, 1040, 256, (0, 128, 512, 1040))])
-def test_two_k_blocks_per_stage_agree(MKN, bn, monkeypatch):
+def test_two_k_blocks_per_stage_agree(MKN, bn, monkeypatch, dev_lib):
     """The GEMM from codes with two k blocks per pipeline stage (one commit per
     stage; odd k-block counts end in a half stage; K tails; K segments that
     begin or end inside a stage) against the oracle and bit-identical to one k
@@ -194,7 +194,7 @@ def test_two_k_blocks_per_stage_agree(MKN, bn, monkeypatch):
 
 
 @pytest.mark.parametrize("out", ["bf16", "f32"])
-def test_wide_tiles_with_sixteen_epilogue_warps_agree(out, monkeypatch):
+def test_wide_tiles_with_sixteen_epilogue_warps_agree(out, monkeypatch, dev_lib):
     """256-wide tiles drained by 16 epilogue warps: the oracle's result and the
     same bits as with 8 warps (ragged M, N tail)."""
     import post_quantized_linear_b200 as pq
@@ -216,7 +216,7 @@ def test_wide_tiles_with_sixteen_epilogue_warps_agree(out, monkeypatch):
 @pytest.mark.parametrize("MKN", [(300, 640, 272, (0, 256, 640)), (129, 384, 144), (200, 1024, 400),
                                  (64, 3072, 1024), (1, 256, 96), (16, 1024, 272, (0, 512, 1024)),
                                  (257, 1152, 128, (0, 128, 640, 1152))])
-def test_int4_codes_kernel_and_operand_ring_kernel_agree(MKN, out, monkeypatch):
+def test_int4_codes_kernel_and_operand_ring_kernel_agree(MKN, out, monkeypatch, dev_lib):
     """int4 weights (group 128) through the GEMM from codes (unpack warps, one
     ring of stages, seeded accumulators) and through the operand-ring kernel:
     the oracle's result on every row and identical bits; ragged M and N tails,
@@ -240,7 +240,7 @@ def test_int4_codes_kernel_and_operand_ring_kernel_agree(MKN, out, monkeypatch):
 
 @pytest.mark.parametrize("kseg", [None, (0, 256, 640)])
 @pytest.mark.parametrize("M", [1, 17, 48, 100, 127])
-def test_code_boxes_sized_to_a_short_row_tile(M, kseg, monkeypatch):
+def test_code_boxes_sized_to_a_short_row_tile(M, kseg, monkeypatch, dev_lib):
     """Fewer than 128 rows: the GEMM from codes loads code boxes of M rows
     rounded up to 16 and the MMA's other rows read stale shared memory.  Every
     row against the oracle (DualScale and single-scale, one and two K
@@ -407,7 +407,7 @@ def test_weight_quantization_range_status():
 
 
 @pytest.mark.parametrize("codes,i", [(False, 0), (True, 0), (True, 6)])
-def test_starved_pipeline_times_out_and_context_recovers(codes, i):
+def test_starved_pipeline_times_out_and_context_recovers(codes, i, dev_lib):
     """Bounded waits: with the producer starved every wait expires; the kernel
     records SQ_ERR_TIMEOUT, frees its TMEM and exits, and the next launch on the
     same context is correct again (int8 and int4 weights)."""
@@ -445,7 +445,7 @@ PAIR_CASES = [
 
 @pytest.mark.parametrize("bn", ["128", "256"])
 @pytest.mark.parametrize("i", range(len(PAIR_CASES)))
-def test_pair_gemm_matches_oracle(i, bn, monkeypatch):
+def test_pair_gemm_matches_oracle(i, bn, monkeypatch, dev_lib):
     """The GEMM from codes on CTA pairs (tcgen05.mma.cta_group::2) gives the
     oracle's result; several K segments use the double-buffered BN = 128 path."""
     import post_quantized_linear_b200 as pq
@@ -465,7 +465,7 @@ def test_pair_gemm_matches_oracle(i, bn, monkeypatch):
     assert torch.equal(y.view(torch.int16), y1.view(torch.int16))
 
 
-def test_pair_gemm_fp32_bit_exact(monkeypatch):
+def test_pair_gemm_fp32_bit_exact(monkeypatch, dev_lib):
     import post_quantized_linear_b200 as pq
     monkeypatch.setenv("SEGQUANT_PAIR", "1")
     wl = W.small_case(300, 640, 288, seed=50, kseg=[0, 256, 640], x_sigmas=[1.0, 3.0], out="bf16")
@@ -484,7 +484,7 @@ def _epi_args(c, wl):
 
 
 @pytest.mark.parametrize("name", ["dit_xl2_fc2_cfg", "seglinear_qkv", "mmdit_mlp_up"])
-def test_pair_gemm_full_size_sampled_rows(name, monkeypatch):
+def test_pair_gemm_full_size_sampled_rows(name, monkeypatch, dev_lib):
     import post_quantized_linear_b200 as pq
     monkeypatch.setenv("SEGQUANT_PAIR", "1")
     wl = W.WORKLOADS[name]

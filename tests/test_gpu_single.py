@@ -48,7 +48,7 @@ def test_single_codes_bit_exact(i):
 
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("i", range(len(CASES)))
-def test_single_forward_matches_oracle(i, bn, monkeypatch):
+def test_single_forward_matches_oracle(i, bn, monkeypatch, dev_lib):
     import post_quantized_linear_b200 as pq
     monkeypatch.setenv("SEGQUANT_BN", bn)
     c = Case(_case(i))
@@ -70,7 +70,7 @@ def test_single_forward_fp32_bit_exact():
     np.testing.assert_array_equal(y.cpu().numpy(), ref)
 
 
-def test_single_starved_pipeline_times_out_and_context_recovers():
+def test_single_starved_pipeline_times_out_and_context_recovers(dev_lib):
     import post_quantized_linear_b200 as pq
     from post_quantized_linear_b200 import _lib
     c = Case(_case(0))

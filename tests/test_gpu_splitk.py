@@ -94,7 +94,7 @@ def test_splitk_rejects_large_m_and_segments():
         pq.linear_from_codes_splitk(qp2, qn2, c2.qw, c2.sp, c2.sn, ws)
 
 
-def test_splitk_starved_pipeline_times_out_and_recovers():
+def test_splitk_starved_pipeline_times_out_and_recovers(dev_lib):
     import post_quantized_linear_b200 as pq
     from post_quantized_linear_b200 import _lib
     wl = W.small_case(64, 1024, 512, seed=133, out="bf16")
@@ -138,7 +138,7 @@ def test_splitk_small_m_configs(M, KN):
 
 @pytest.mark.parametrize("bn", ["32", "64", "96", "128", "-1"])
 @pytest.mark.parametrize("MKN", [(100, 640, 272), (1, 384, 96), (128, 1024, 1024), (64, 3072, 12288)])
-def test_small_m_narrow_tiles_match_oracle(MKN, bn, monkeypatch):
+def test_small_m_narrow_tiles_match_oracle(MKN, bn, monkeypatch, dev_lib):
     """One row tile: the GEMM from codes with narrow tiles and four epilogue
     warps (forced widths, and -1 for the regular choice) against the oracle,
     and bit-identical to the fused forward; also the single-scale kernel."""
