@@ -63,7 +63,9 @@ MMA_I8_OPS_PER_CLK_SM = 16384
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
-    ("dit_xl2_fc2_cfg", "codes"): 93068032 + 11148288,   # dualscale_gemm_codes_kernel
+    ("mmdit_mlp_up", "codes"): 161525248 + 378640896,     # dualscale_gemm_codes_kernel
+    ("dit_xl2_fc2_cfg", "codes"): 92216576 + 9675264,     # dualscale_gemm_codes_kernel
+    ("seglinear_qkv", "codes"): 56912128 + 31624448,      # dualscale_gemm_codes_kernel
 }
 
 
@@ -100,6 +102,9 @@ def parse_args(argv=None):
     ap.add_argument("--small-m-only", action="store_true",
                     help="run only the small-M measurements (one GPU) and print them as one "
                          "JSON line; not a bench line")
+    ap.add_argument("--fused-act-only", action="store_true",
+                    help="run only the fused-activation measurements (one GPU) and print them "
+                         "as one JSON line; not a bench line")
     return ap.parse_args(argv)
 
 
@@ -718,6 +723,10 @@ def run_ours(args):
     int8_peak, hbm_peak, peak_kind = peaks()
     if args.small_m_only:
         print(json.dumps({"small_m": {"peak_gbs": hbm_peak, "cases": small_m_measure(
+            dev, L2Flush(dev), args.steps, hbm_peak)}}), flush=True)
+        return 0
+    if args.fused_act_only:
+        print(json.dumps({"fused_activation": {"peak_gbs": hbm_peak, "cases": fused_act_measure(
             dev, L2Flush(dev), args.steps, hbm_peak)}}), flush=True)
         return 0
 

@@ -868,12 +868,18 @@ __device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float&
 // it, so the MMA of the next unit or tile waits only for the loads.
 // (Group units -- one per 128-wide K group -- go through
 // epilogue_groups_tma_store.)
-template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn>
+// PAIR: a CTA of a 2-SM pair: its TMEM lanes are tile rows row_shift + 0..127,
+// the full barriers are signalled by the leader's commits (cluster-scope
+// acquire), and `empty_base` may be a cluster address of the leader's
+// barriers (empty_remote).
+template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn,
+          bool PAIR = false>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
                                                    uint32_t empty_base, int rounds, TileFn tile_fn,
-                                                   volatile int* abort_flag, long long budget) {
+                                                   volatile int* abort_flag, long long budget,
+                                                   int row_shift = 0, bool empty_remote = false) {
   constexpr int HALF = BN / (EPW / 4);
   constexpr int ROWB = Y_BF16 ? 64 : 128;
   constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
@@ -885,7 +891,10 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
   auto release = [&](int b) {
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
+    if (lane == 0) {
+      if (PAIR && empty_remote) mbar_arrive_remote(empty_base + 8u * (uint32_t)b);
+      else mbar_arrive(empty_base + 8u * (uint32_t)b);
+    }
   };
   // Eight columns of buffer b at tile column cc into registers (both
   // polarities, or the single code's accumulator in ap).
@@ -931,7 +940,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       for (int i = 0; i < HALF; ++i) y[i] = 0.0f;
       for (int u = 0; u < units; ++u) {
         const int b = ug % NBUF;
-        if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+        if (!(ok = wait_warp<PAIR>(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
         tc_fence_after();
         float sp, sn;
         unit_act_scales(args, u, sp, sn);
@@ -968,7 +977,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+            tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + row_shift + quad * 32);
             bulk_commit_group();
           }
           pending = true;
@@ -976,7 +985,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       }
     } else {
       const int b = ug % NBUF;
-      if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+      if (!(ok = wait_warp<PAIR>(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
       tc_fence_after();
       float sp, sn;
       unit_act_scales(args, 0, sp, sn);
@@ -1006,7 +1015,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+          tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + row_shift + quad * 32);
           bulk_commit_group();
         }
         pending = true;

@@ -15,8 +15,13 @@
 //     leader's teardown drain of `full` covers every copy either CTA issued;
 //   * warp 1: TMEM allocation for the pair; in the leader (rank 0) the single
 //     MMA-issuing thread;
-//   * epilogue warps: read this CTA's 128 TMEM lanes, fold, store its rows, and
-//     arrive on the leader's `tmem_empty` barrier.
+//   * warps 2..: epilogue (epilogue_tma_store): read this CTA's 128 TMEM lanes,
+//     fold, stage and store its rows with TMA stores, and arrive on the
+//     leader's `tmem_empty` barrier as soon as the last TMEM loads landed.
+// Per SM and k block the pair moves 32 KiB of codes and BN/2 x 128 bytes of
+// weights, and its tensor core reads only its own half of the weight tile:
+// at BN = 256 that is 48 KiB and half the shared-memory operand traffic of
+// the one-CTA 256-wide tile.
 // The leader commits each stage's MMAs to its `empty` barrier and each unit to
 // both CTAs' `tmem_full` barriers (cluster addresses from mapa).
 #pragma once
@@ -27,16 +32,22 @@ namespace sq {
 
 constexpr int BM_PAIR = 2 * BM;  // token rows per pair tile
 
-template <int BN_>
+constexpr int kPairEpiWarp0 = 2;
+__host__ __device__ constexpr int pair_threads(int epw) { return (kPairEpiWarp0 + epw) * 32; }
+
+template <int BN_, int EPW_, bool Y_BF16>
 struct PairCfg {
   static constexpr int BN = BN_;
+  static constexpr int EPW = EPW_;
   static constexpr int HB = BN / 2;                 // weight rows loaded per CTA
   static constexpr int Q_TILE = BM * BK;
   static constexpr int W_HALF = HB * BK;
   static constexpr int STAGE = 2 * Q_TILE + W_HALF;
-  static constexpr int S = (kStageBudget / STAGE) < 8 ? (kStageBudget / STAGE) : 8;
+  static constexpr int Y_BYTES = EPW * stage_y_bytes(Y_BF16);
+  static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
   static constexpr int NBUF = (BN <= 128) ? 2 : 1;
-  static constexpr int OFF_BAR = S * STAGE;
+  static constexpr int OFF_Y = S * STAGE;
+  static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
   static constexpr int NUM_BARS = 3 * 8 + 2 * 2 + 1;  // full, empty, armed; tmem full/empty; drain
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -44,6 +55,7 @@ struct PairCfg {
   static constexpr int TMEM_ALLOC = TMEM_COLS <= 256 ? 256 : 512;
   static_assert(BN % 32 == 0 && BN <= 256, "pair UMMA N");
   static_assert(S >= 2 && TMEM_COLS <= 512 && SMEM_BYTES <= 232448, "budgets");
+  static_assert(OFF_Y % 1024 == 0, "staging alignment");
 };
 
 // Pair tiles in the same snake order as tile_of, over pairs of CTAs; m_tiles
@@ -66,13 +78,16 @@ __device__ __forceinline__ bool pair_tile_of(const GemmArgs& a, int it, int bn, 
   return true;
 }
 
-template <int BN, bool ACC_OUT, bool Y_BF16, bool MULTI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kernel_threads(MULTI), 1)
+template <int BN, bool Y_BF16, bool MULTI, int EPW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1)
     dualscale_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                const __grid_constant__ CUtensorMap tmap_qn,
                                const __grid_constant__ CUtensorMap tmap_w,
+                               const __grid_constant__ CUtensorMap tmap_y,
                                const __grid_constant__ GemmArgs args) {
-  using C = PairCfg<BN>;
+  using C = PairCfg<BN, EPW, Y_BF16>;
+  static_assert(EPW % 4 == 0 && (BN / (EPW / 4)) % 32 == 0, "32-column store passes per warp");
+  static_assert(!MULTI || BN / (EPW / 4) <= 64, "several units: at most 64 partials per thread");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -100,7 +115,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kernel_threads(MULTI
     }
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(smem_u32(tmem_full + i), 1);
-      mbar_init(smem_u32(tmem_empty + i), 2 * epi_warps(MULTI));
+      mbar_init(smem_u32(tmem_empty + i), 2 * EPW);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
@@ -126,6 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kernel_threads(MULTI
       tma_prefetch_desc(&tmap_qp);
       tma_prefetch_desc(&tmap_qn);
       tma_prefetch_desc(&tmap_w);
+      tma_prefetch_desc(&tmap_y);
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);   // leader's barriers
       const uint32_t armed1 = mapa_shared(smem_u32(armed), 1); // peer's barriers
       int c = 0;
@@ -206,15 +222,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kernel_threads(MULTI
       umma_commit_pair(smem_u32(drain_bar));
       wait_drain(smem_u32(drain_bar), 0, kDrainBudget);
     }
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= kPairEpiWarp0) {
     // --------------------------------------------------------- epilogue
     const int quad = warp & 3;
-    const int part = (warp - kEpiWarp0) >> 2;
+    const int part = (warp - kPairEpiWarp0) >> 2;
     const uint32_t empty0 = smem_u32(tmem_empty);
-    epilogue_role<BN, C::NBUF, MULTI, ACC_OUT, Y_BF16, false, decltype(tiles), true>(
-        args, quad, part, lane, tmem_base + ((uint32_t)(quad * 32) << 16), tmem_full,
-        leader ? empty0 : mapa_shared(empty0, 0), /*empty_remote=*/!leader, (int)rank * BM, rounds,
-        tiles, abort_flag, budget);
+    uint8_t* stage_y = smem + C::OFF_Y + (warp - kPairEpiWarp0) * stage_y_bytes(Y_BF16);
+    epilogue_tma_store<BN, C::NBUF, EPW, 2, MULTI, Y_BF16, decltype(tiles), true>(
+        args, &tmap_y, stage_y, quad, part, lane, tmem_base + ((uint32_t)(quad * 32) << 16),
+        tmem_full, leader ? empty0 : mapa_shared(empty0, 0), rounds, tiles, abort_flag, budget,
+        (int)rank * BM, /*empty_remote=*/!leader);
   }
 
   // ---------------------------------------------------------------- teardown

@@ -242,11 +242,11 @@ sq_status launch_out(bool acc, bool y_bf16, const CUtensorMap& ta, const CUtenso
                 : launch_gemm<BN, ASRC, XT, W4, false, false, MULTI>(ta, ta2, tw, a, stream);
 }
 
-template <int BN, bool ACC, bool YB, bool MULTI>
+template <int BN, bool YB, bool MULTI, int EPW>
 sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tw,
-                      sq::GemmArgs a, cudaStream_t stream) {
-  using C = sq::PairCfg<BN>;
-  constexpr auto kern = sq::dualscale_gemm_pair_kernel<BN, ACC, YB, MULTI>;
+                      const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
+  using C = sq::PairCfg<BN, EPW, YB>;
+  constexpr auto kern = sq::dualscale_gemm_pair_kernel<BN, YB, MULTI, EPW>;
   cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
@@ -255,19 +255,17 @@ sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& ta2, const CUten
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int pairs = num_sms() / 2;
   if (pairs > a.num_tiles) pairs = a.num_tiles;
-  kern<<<2 * pairs, sq::kernel_threads(MULTI), C::SMEM_BYTES, stream>>>(ta, ta2, tw, a);
+  kern<<<2 * pairs, sq::pair_threads(EPW), C::SMEM_BYTES, stream>>>(ta, ta2, tw, ty, a);
   return cuda_status(cudaGetLastError());
 }
 
+// 2-SM pair tiles with 16 epilogue warps per CTA (32 or 64 columns per warp).
 template <int BN, bool MULTI>
-sq_status launch_pair_out(bool acc, bool y_bf16, const CUtensorMap& ta, const CUtensorMap& ta2,
-                          const CUtensorMap& tw, const sq::GemmArgs& a, cudaStream_t stream) {
-  if constexpr (MULTI) {
-    if (acc) return launch_pair<BN, true, false, true>(ta, ta2, tw, a, stream);
-  }
-  if (acc) return SQ_ERR_UNSUPPORTED;
-  return y_bf16 ? launch_pair<BN, false, true, MULTI>(ta, ta2, tw, a, stream)
-                : launch_pair<BN, false, false, MULTI>(ta, ta2, tw, a, stream);
+sq_status launch_pair_out(bool y_bf16, const CUtensorMap& ta, const CUtensorMap& ta2,
+                          const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                          cudaStream_t stream) {
+  return y_bf16 ? launch_pair<BN, true, MULTI, 16>(ta, ta2, tw, ty, a, stream)
+                : launch_pair<BN, false, MULTI, 16>(ta, ta2, tw, ty, a, stream);
 }
 
 template <int BN, bool ACC, bool YB, bool MULTI>
@@ -677,8 +675,10 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
     constexpr auto kern = sq::quantize_combined_act_table_kernel;
     st = cuda_status(smem_limit<kern>(kTableSmem));
     if (st != SQ_OK) return st;
+    // One 1024-thread block per SM (the table fills its shared memory): at most
+    // one block per SM, so no SM runs a second one after the others finish.
     const int64_t ty = std::min<int64_t>((M + 31) / 32,
-                                         std::max<int64_t>(1, (num_sms() + gx - 1) / gx));
+                                         std::max<int64_t>(1, num_sms() / gx));
     dim3 tgrid(gx, (unsigned)std::min<int64_t>(ty, 65535)), tblock(32, 32);
     kern<<<tgrid, tblock, kTableSmem, s>>>(static_cast<const bf*>(x), (int32_t)M, (int32_t)K, ldx,
                                            sb, s_pos, s_neg, lut, q_pos, ldq);
@@ -780,10 +780,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
                         !(src == ASource::Codes && use_pair(N, w4)) && use_codes_ring())
                            ? choose_bn_small(M, N) : 0;
   if (bn_small) BN = bn_small;
-  if (pair && !multi && acc == nullptr) {
-    BN = 256;
-    BN = dev_switch("SEGQUANT_BN", 256) == 128 ? 128 : 256;
-  }
+  if (pair && acc == nullptr) BN = dev_switch("SEGQUANT_BN", 256) == 128 ? 128 : 256;
   // One row tile of fewer than BM rows, read by the GEMM from codes: code boxes
   // of M rows rounded up to 16 instead of mostly out-of-bounds 128-row boxes.
   const bool codes_w4 = (src == ASource::Codes) && w4 && !pair && acc == nullptr && use_codes_w4();
@@ -869,9 +866,15 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   }
   if constexpr (kDev) {   // 2-SM pair tiles: a measured alternative
     if (pair) {
-      if (multi || ac) return launch_pair_out<128, true>(ac, yb, ta, ta2, tw, a, stream);
-      if (BN == 256) return launch_pair_out<256, false>(ac, yb, ta, ta2, tw, a, stream);
-      return launch_pair_out<128, false>(ac, yb, ta, ta2, tw, a, stream);
+      CUtensorMap ty;
+      st = make_tmap_y(&ty, y, yt, M, N, ldy);
+      if (st != SQ_OK) return st;
+      if (multi) {
+        if (BN == 256) return launch_pair_out<256, true>(yb, ta, ta2, tw, ty, a, stream);
+        return launch_pair_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
+      }
+      if (BN == 256) return launch_pair_out<256, false>(yb, ta, ta2, tw, ty, a, stream);
+      return launch_pair_out<128, false>(yb, ta, ta2, tw, ty, a, stream);
     }
   }
   if (src == ASource::Codes) {
