@@ -66,6 +66,7 @@ NCU_TRAFFIC_BYTES = {
     ("mmdit_mlp_up", "codes"): 161525248 + 378640896,     # dualscale_gemm_codes_kernel
     ("dit_xl2_fc2_cfg", "codes"): 92216576 + 9675264,     # dualscale_gemm_codes_kernel
     ("seglinear_qkv", "codes"): 56912128 + 31624448,      # dualscale_gemm_codes_kernel
+    ("w4a8", "codes"): 106261760 + 69462784,              # dualscale_gemm_codes_kernel (int4)
 }
 
 

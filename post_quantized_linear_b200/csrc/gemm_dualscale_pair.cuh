@@ -9,10 +9,12 @@
 //
 // Per CTA of the pair:
 //   * warp 0: TMA of its 128 rows of q+ / q- and its BN/2 weight rows into one
-//     stage.  All copies of a stage complete on the leader's `full` barrier: the
-//     leader arms it with both CTAs' bytes, then signals the peer's `armed`
-//     barrier, and the peer issues its copies only for armed stages, so the
-//     leader's teardown drain of `full` covers every copy either CTA issued;
+//     stage, once its own `empty` barrier says the pair's MMAs are done with
+//     the stage.  All copies of a stage complete on the leader's `full`
+//     barrier, which the leader arms with both CTAs' bytes; a peer copy that
+//     lands before the leader armed the barrier only takes its transaction
+//     count below zero for a while (the phase still needs the leader's
+//     arrival);
 //   * warp 1: TMEM allocation for the pair; in the leader (rank 0) the single
 //     MMA-issuing thread;
 //   * warps 2..: epilogue (epilogue_tma_store): read this CTA's 128 TMEM lanes,
@@ -22,8 +24,11 @@
 // weights, and its tensor core reads only its own half of the weight tile:
 // at BN = 256 that is 48 KiB and half the shared-memory operand traffic of
 // the one-CTA 256-wide tile.
-// The leader commits each stage's MMAs to its `empty` barrier and each unit to
-// both CTAs' `tmem_full` barriers (cluster addresses from mapa).
+// The leader commits the MMAs of every KP consecutive stages (two where the
+// ring has an even number of stages: one commit per k block stalls the issue
+// of the next MMAs) to both CTAs' `empty` barrier of that stage group, and
+// each unit to both CTAs' `tmem_full` barriers, each with one multicast
+// commit.
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -45,10 +50,11 @@ struct PairCfg {
   static constexpr int STAGE = 2 * Q_TILE + W_HALF;
   static constexpr int Y_BYTES = EPW * stage_y_bytes(Y_BF16);
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
+  static constexpr int KP = (S % 2 == 0) ? 2 : 1;   // stages per release of the ring
   static constexpr int NBUF = (BN <= 128) ? 2 : 1;
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
-  static constexpr int NUM_BARS = 3 * 8 + 2 * 2 + 1;  // full, empty, armed; tmem full/empty; drain
+  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1;  // full, empty; tmem full/empty; drain
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 2 * BN * NBUF;
@@ -93,9 +99,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;              // [8] (leader) both CTAs' copies landed
-  uint64_t* empty = full + 8;         // [8] (leader) the pair's MMAs are done with the stage
-  uint64_t* armed = empty + 8;        // [8] (peer) the leader armed `full` for this use
-  uint64_t* tmem_full = armed + 8;    // [2]
+  uint64_t* empty = full + 8;         // [8 / KP] (both) the pair's MMAs are done with the stages
+  uint64_t* tmem_full = empty + 8;    // [2]
   uint64_t* tmem_empty = tmem_full + 2;  // [2] (leader) both CTAs drained the buffer
   uint64_t* drain_bar = tmem_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -108,11 +113,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1
   const long long budget = args.wait_budget;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::S; ++i) {
-      mbar_init(smem_u32(full + i), 1);
-      mbar_init(smem_u32(empty + i), 1);
-      mbar_init(smem_u32(armed + i), 1);
-    }
+    for (int i = 0; i < C::S; ++i) mbar_init(smem_u32(full + i), 1);
+    for (int i = 0; i < C::S / C::KP; ++i) mbar_init(smem_u32(empty + i), 1);
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(smem_u32(tmem_full + i), 1);
       mbar_init(smem_u32(tmem_empty + i), 2 * EPW);
@@ -143,7 +145,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_y);
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);   // leader's barriers
-      const uint32_t armed1 = mapa_shared(smem_u32(armed), 1); // peer's barriers
       int c = 0;
       bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
@@ -153,14 +154,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1
         const int n_cta = t.n0 + (int)rank * (t.width / 2);
         for (int kb = 0; kb < num_kb; ++kb) {
           const int s = c % C::S;
-          const uint32_t par = ((c / C::S) & 1) ^ 1;
-          if (leader) {
-            if (!(ok = wait1s<false>(smem_u32(empty + s), par, abort_flag, budget))) break;
-            mbar_arrive_expect_tx(smem_u32(full + s), 2 * C::STAGE);
-            mbar_arrive_remote(armed1 + 8u * (uint32_t)s);
-          } else {
-            if (!(ok = wait1s<true>(smem_u32(armed + s), (c / C::S) & 1, abort_flag, budget))) break;
-          }
+          if (s % C::KP == 0 &&
+              !(ok = wait1s<true>(smem_u32(empty + s / C::KP), ((c / C::S) & 1) ^ 1, abort_flag,
+                                  budget)))
+            break;
+          if (leader) mbar_arrive_expect_tx(smem_u32(full + s), 2 * C::STAGE);
           uint8_t* st = smem + s * C::STAGE;
           const uint32_t bar = full0 + 8u * (uint32_t)s;
           tma_load_2d_pair(smem_u32(st), &tmap_qp, bar, kb * BK, m_cta);
@@ -170,13 +168,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1
         }
       }
       // The leader's `full` phases count both CTAs' copies: draining them lets
-      // every issued copy land before the pair tears down.
+      // every issued copy land before the pair tears down (the cluster barrier
+      // of the teardown holds the peer until then).
       if (leader) drain_ring(full, C::S, c, kDrainBudget);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------- MMA issuer (pair)
-      const uint32_t peer = 1;
       int c = 0, ug = 0;
       bool ok = true;
       for (int it = 0; it < rounds && ok; ++it) {
@@ -208,12 +206,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(EPW), 1
             umma_i8_pair(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
           }
           unit_open = true;
-          umma_commit_pair(smem_u32(empty + s));
+          if (s % C::KP == C::KP - 1) umma_commit_pair_to(smem_u32(empty + s / C::KP), 0x3);
           ++c;
           if (kb_closes_unit(args, kb)) {
-            const int b = ug % C::NBUF;
-            umma_commit_pair(smem_u32(tmem_full + b));
-            umma_commit_pair(mapa_shared(smem_u32(tmem_full + b), peer));
+            umma_commit_pair_to(smem_u32(tmem_full + ug % C::NBUF), 0x3);
             ++ug;
             unit_open = false;
           }
