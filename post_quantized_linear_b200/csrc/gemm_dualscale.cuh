@@ -1029,6 +1029,120 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
   __syncwarp();
 }
 
+// ------------------------------------- stacked-polarity epilogue (small M)
+// One row tile whose q+ and q- code rows were stacked in one A tile: the
+// accumulator of tile row r sits in TMEM lane r (q+ product) and lane P + r
+// (q- product), P = args.a_rows in {16, 32, 64}, one buffer of BN columns per
+// tile.  The warps that own lanes [0, P) fold and store rows [0, P); the q-
+// values reach them by a shuffle (P = 16: both halves in the first lane
+// quarter) or, XCH, through shared memory (P = 32, 64: from lane quarter
+// q + P/32 to quarter q), 32 columns at a time, with bounded mbarrier
+// handshakes (xfull: the q- warps wrote; xempty: the q+ warps have read).  The
+// fold is fold8_exact's and the store epilogue_tma_store's, so the outputs are
+// those of the two-tile form.
+template <int BN, int NBUF, bool Y_BF16, bool XCH, class TileFn>
+__device__ __forceinline__ void epilogue_stacked(
+    const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, uint32_t* xch, int quad,
+    int lane, uint32_t t_lane, uint64_t* tmem_full, uint32_t empty_base, uint32_t xfull,
+    uint32_t xempty, int rounds, TileFn tile_fn, volatile int* abort_flag, long long budget) {
+  constexpr int ROWB = Y_BF16 ? 64 : 128;
+  uint8_t* srow = stage_y + lane * ROWB;
+  const uint32_t sbase = smem_u32(stage_y);
+  const int qparts = args.a_rows / 32;                          // 0 when P = 16
+  const bool pos_warp = XCH ? (quad < qparts) : (quad == 0);    // folds and stores
+  const bool neg_warp = XCH && quad >= qparts && quad < 2 * qparts;   // hands q- over
+  auto release = [&](int b) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
+  };
+  float sp, sn;
+  unit_act_scales(args, 0, sp, sn);
+  int ug = 0, xu = 0;
+  bool ok = true, pending = false;
+  for (int it = 0; it < rounds && ok; ++it) {
+    Tile t;
+    if (!tile_fn(it, t)) continue;
+    const int b = ug % NBUF;
+    if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
+    tc_fence_after();
+    ++ug;
+    if (!pos_warp && !neg_warp) {   // lanes past 2P: nothing to read
+      release(b);
+      continue;
+    }
+    const int npass = (t.width + 31) / 32;
+    for (int p = 0; p < npass; ++p) {
+      const int col = 32 * p;
+      const uint32_t tcol = (uint32_t)b * BN + (uint32_t)col;
+      uint32_t v[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld8(t_lane + tcol + 8 * i, v[i]);
+      tmem_wait_ld();
+      if (p == npass - 1) release(b);   // every column of the tile is in registers
+      uint32_t vn[4][8];
+      if constexpr (!XCH) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) vn[i][k] = __shfl_down_sync(0xffffffffu, v[i][k], 16);
+      } else {
+        const int xrow = (neg_warp ? quad - qparts : quad) * 32 + lane;
+        uint32_t* xr = xch + xrow * 32;
+        if (neg_warp) {
+          if (!(ok = wait_warp(xempty, (xu & 1) ^ 1, abort_flag, budget))) break;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) xr[(8 * i + k) ^ lane] = v[i][k];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xfull);
+          ++xu;
+          continue;
+        }
+        if (!(ok = wait_warp(xfull, xu & 1, abort_flag, budget))) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) vn[i][k] = xr[(8 * i + k) ^ lane];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xempty);
+        ++xu;
+      }
+      // q+ warps: fold, stage and store rows quad*32 .. +31, columns col .. +31
+      if (pending) {   // the previous store has read the staging tile
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cc = col + 16 * h;
+        if (cc < t.width) {
+          float o[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+          float sw[8];
+          load_wscales8(args, 0, 0, t.n0 + cc, sw);
+          fold8_exact(v[2 * h], vn[2 * h], sw, sp, sn, o);
+          load_wscales8(args, 0, 0, t.n0 + cc + 8, sw);
+          fold8_exact(v[2 * h + 1], vn[2 * h + 1], sw, sp, sn, o + 8);
+          stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+        bulk_commit_group();
+      }
+      pending = true;
+    }
+  }
+  // Every store has completed before the CTA (and its shared memory) exits.
+  if (lane == 0) bulk_wait_all();
+  __syncwarp();
+}
+
 // ------------------------------------------- group-unit epilogue (int4 groups)
 // One unit per 128-wide K group (int4 weights, SEED 1; the Hadamard-rotated
 // codes, SEED 2): every k block ends a unit, so the whole accumulator pair is

@@ -80,8 +80,15 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
   return (kStageBudget - y_bytes) / stage >= 2 || (!tma_y_forced && kStageBudget / stage >= 2);
 }
 
+// STK_ (stacked polarities, one row tile of M <= STK_ rows, one unit per
+// tile): the q+ box lands in rows [0, P) of one A tile and the q- box in rows
+// [P, 2P), P = M rounded up to 16, so a single MMA per k step yields both
+// products (accumulator lanes r and P + r) and half the MMAs of the two-tile
+// form are issued.  The A area of a k block is 2 * STK_ rows; the MMA still
+// reads 128 rows from its start (the rows past 2P belong to the weight tile or
+// the next k block and land in accumulator lanes nobody reads).
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
-          bool LDA_ = false, int KPS_ = 1, int WM_ = 0>
+          bool LDA_ = false, int KPS_ = 1, int WM_ = 0, int STK_ = 0>
 struct CodesCfg {
   static constexpr bool W4_ = (WM_ == 1);
   static constexpr bool LDA = LDA_;
@@ -89,8 +96,11 @@ struct CodesCfg {
   // full barrier: the TMA thread's arrival (+ bytes), plus one per loader thread
   static constexpr int FULL_COUNT = 1 + (LDA_ ? kLoaderWarps * 32 : 0);
   static constexpr int BN = BN_;
-  static constexpr int NACC = SINGLE ? 1 : 2;          // accumulators (code tiles) per unit
-  static constexpr int A_BYTES = NACC * BM * BK;      // q+ and q- tiles, or the single code tile
+  static constexpr int STK = STK_;
+  static constexpr int CODE_TILES = SINGLE ? 1 : 2;    // code boxes per k block
+  static constexpr int NACC = (SINGLE || STK_) ? 1 : 2;   // accumulators per unit
+  // q+ and q- tiles, or the single code tile, or the stacked rows
+  static constexpr int A_BYTES = STK_ ? 2 * STK_ * BK : CODE_TILES * BM * BK;
   static constexpr int W_BYTES = BN * BK;
   static constexpr int WP_BYTES = W4_ ? BN * (BK / 2) : 0;   // packed int4 rows of 64 bytes
   static constexpr int KB_BYTES = A_BYTES + W_BYTES + WP_BYTES;  // one k block of operands
@@ -100,10 +110,14 @@ struct CodesCfg {
   static constexpr bool TMA_Y = SINGLE || MULTI || EPW != epi_warps(MULTI) ||
                                 (kStageBudget - EPW * stage_y_bytes(Y_BF16)) / STAGE >= 2;
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
-  // group units: each epilogue warp's two 32-float buffers of widened weight scales
-  static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : 0;
+  // group units: each epilogue warp's two 32-float buffers of widened weight scales;
+  // stacked polarities: the q- accumulators of 32 columns, handed between warps
+  static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : (STK_ > 16 ? STK_ * 32 * 4 : 0);
   static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) < 8
                                ? ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) : 8;
+  static_assert(STK_ == 0 || ((STK_ == 16 || STK_ == 32 || STK_ == 64) && !MULTI && !SINGLE &&
+                              !LDA_ && WM_ == 0 && EPW_ == 4),
+                "stacked polarities: DualScale, one unit, four epilogue warps");
   static_assert(KPS == 1 || !LDA_, "two k blocks per stage: TMA loads");
   static_assert(WM_ == 0 || (MULTI && !SINGLE && !LDA_ && KPS_ == 1 && BN_ == 128),
                 "group units: DualScale, one k block per stage, BN = 128");
@@ -111,8 +125,8 @@ struct CodesCfg {
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
   static constexpr int OFF_BAR = OFF_SW + SW_BYTES;
-  // full, empty; tmem full/empty; drain; (W4) unpacked
-  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0);
+  // full, empty; tmem full/empty; drain; (W4) unpacked; (stacked) exchange full/empty
+  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0) + (STK_ > 16 ? 2 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = NACC * BN * NBUF;
@@ -120,17 +134,19 @@ struct CodesCfg {
   static_assert(S >= 2 && TMEM_COLS <= 512 && SMEM_BYTES <= 232448, "budgets");
   static_assert(BN % 16 == 0 && BN <= 256, "UMMA N for M = 128");
   static_assert(OFF_Y % 1024 == 0 && stage_y_bytes(Y_BF16) % 1024 == 0, "staging alignment");
+  // the MMA's 128-row read from the last k block's A start stays in the allocation
+  static_assert(STK_ == 0 || S * STAGE - KB_BYTES + BM * BK <= OFF_MISC, "stacked A read");
 };
 
 template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false, int EPW = epi_warps(MULTI),
-          bool LDA = false, int KPS = 1, int WM = 0>
+          bool LDA = false, int KPS = 1, int WM = 0, int STK = 0>
 __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, WM>;
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, WM, STK>;
   constexpr bool W4 = (WM == 1);        // packed int4 tiles, unpack warps
   constexpr bool SEEDED = (WM != 0);    // one unit per k block, seeded accumulators
   constexpr int EPI0 = codes_epi_warp0(LDA, W4);
@@ -147,6 +163,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   uint64_t* tmem_empty = tmem_full + 2;   // [2]
   uint64_t* drain_bar = tmem_empty + 2;
   uint64_t* ready = drain_bar + 1;        // [8] (W4) int4 tile unpacked
+  uint64_t* xfull = ready + (W4 ? 8 : 0);  // (stacked, P > 16) q- accumulators handed over
+  uint64_t* xempty = xfull + 1;            // (stacked, P > 16) q+ warps done reading them
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -166,6 +184,10 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     mbar_init(smem_u32(drain_bar), 1);
     if constexpr (W4)
       for (int i = 0; i < C::S; ++i) mbar_init(smem_u32(ready + i), kUnpackWarps);
+    if constexpr (STK > 16) {   // one arrival per 32-row quarter of q- (q+) rows
+      mbar_init(smem_u32(xfull), (uint32_t)((args.a_rows + 31) / 32));
+      mbar_init(smem_u32(xempty), (uint32_t)((args.a_rows + 31) / 32));
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -189,8 +211,10 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_y);
       // bytes one k block brings: the code boxes (a_rows rows each) + the weight box
-      const uint32_t kb_tx = (uint32_t)(C::NACC * (args.a_rows > 0 ? args.a_rows : BM) * BK +
+      const uint32_t kb_tx = (uint32_t)(C::CODE_TILES * (args.a_rows > 0 ? args.a_rows : BM) * BK +
                                         (W4 ? C::WP_BYTES : C::W_BYTES));
+      // the q- box: right below the q+ rows (stacked) or its own 128-row tile
+      const int qn_off = STK ? args.a_rows * BK : BM * BK;
       int c = 0;
       bool ok = (args.starve == 0);
       for (int it = 0; it < rounds && ok; ++it) {
@@ -211,7 +235,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
             if constexpr (!LDA) {
               tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
               if constexpr (!SINGLE)
-                tma_load_2d(smem_u32(st + BM * BK), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
+                tma_load_2d(smem_u32(st + qn_off), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
             }
             if constexpr (W4)   // packed rows land after the unpacked tile's place
               tma_load_2d(smem_u32(st + C::A_BYTES + C::W_BYTES), &tmap_w, smem_u32(full + s),
@@ -263,7 +287,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
               const uint32_t acc = (SEEDED || unit_open || ks > 0) ? 1u : 0u;
               const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
               umma_i8(d_pos, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, acc);
-              if constexpr (!SINGLE)
+              if constexpr (!SINGLE && !STK)
                 umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
             }
             unit_open = true;
@@ -361,7 +385,13 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     const int quad = warp & 3;
     const int part = (warp - EPI0) >> 2;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-    if constexpr (SEEDED) {
+    if constexpr (STK != 0) {
+      uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
+      epilogue_stacked<BN, C::NBUF, Y_BF16, (STK > 16)>(
+          args, &tmap_y, stage_y, reinterpret_cast<uint32_t*>(smem + C::OFF_SW), quad, lane, t_lane,
+          tmem_full, smem_u32(tmem_empty), smem_u32(xfull), smem_u32(xempty), rounds, tiles,
+          abort_flag, budget);
+    } else if constexpr (SEEDED) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
       float* sw_stage = reinterpret_cast<float*>(smem + C::OFF_SW) + (warp - EPI0) * 64;
       epilogue_groups_tma_store<C::EPW, Y_BF16, WM>(

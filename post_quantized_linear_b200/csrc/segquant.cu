@@ -306,19 +306,24 @@ bool use_codes_lda() { return dev_switch("SEGQUANT_CODES_LDA", 0) != 0; }
 // BN <= 192, where two such stages fit; 1 otherwise); SEGQUANT_KPS=1 forces one.
 int codes_kps() { return dev_switch("SEGQUANT_KPS", 2) == 2 ? 2 : 1; }
 
+// Whether a single row tile of M <= 64 stacks its q+ and q- rows in one A
+// tile (one MMA per k step); SEGQUANT_STACK=0 selects two 128-row code tiles.
+bool use_stacked() { return dev_switch("SEGQUANT_STACK", 1) != 0; }
+
 template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false,
-          int KPS = 1, int WM = 0>
+          int KPS = 1, int WM = 0, int STK = 0>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (kDev && !LDA && KPS == 1 && WM == 0 && !(MULTI && BN > 128)) {
+  if constexpr (kDev && !LDA && KPS == 1 && WM == 0 && STK == 0 && !(MULTI && BN > 128)) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
-  if constexpr (!LDA && KPS == 1 && WM == 0 && BN <= 192 && sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
+  if constexpr (!LDA && KPS == 1 && WM == 0 && STK == 0 && BN <= 192 &&
+                sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
     if (codes_kps() == 2)
       return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
   }
-  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, WM>;
-  constexpr auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM>;
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, WM, STK>;
+  constexpr auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM, STK>;
   cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
@@ -374,6 +379,32 @@ int choose_bn_small(int64_t M, int64_t N) {
     }
   }
   return best;
+}
+
+// Small M with stacked polarities (one MMA per k step for both products):
+// stk = 16 for M <= 16, 64 for 16 < M <= 64 (args.a_rows = 32 or 64); two k
+// blocks per stage.
+template <int BN>
+sq_status launch_codes_stacked(int stk, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+                               const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                               cudaStream_t stream) {
+  if (stk == 16)
+    return y_bf16 ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16>(tqp, tqn, tw, ty, a, stream)
+                  : launch_codes<BN, false, false, false, 4, false, 2, 0, 16>(tqp, tqn, tw, ty, a, stream);
+  return y_bf16 ? launch_codes<BN, true, false, false, 4, false, 2, 0, 64>(tqp, tqn, tw, ty, a, stream)
+                : launch_codes<BN, false, false, false, 4, false, 2, 0, 64>(tqp, tqn, tw, ty, a, stream);
+}
+
+sq_status launch_codes_small_stacked(int bn, int stk, bool y_bf16, const CUtensorMap& tqp,
+                                     const CUtensorMap& tqn, const CUtensorMap& tw,
+                                     const CUtensorMap& ty, const sq::GemmArgs& a,
+                                     cudaStream_t stream) {
+  switch (bn) {
+    case 32: return launch_codes_stacked<32>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 64: return launch_codes_stacked<64>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 96: return launch_codes_stacked<96>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+    default: return launch_codes_stacked<128>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+  }
 }
 
 template <bool SINGLE>
@@ -785,7 +816,10 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   // of M rows rounded up to 16 instead of mostly out-of-bounds 128-row boxes.
   const bool codes_w4 = (src == ASource::Codes) && w4 && !pair && acc == nullptr && use_codes_w4();
   const bool codes_kernel = (src == ASource::Single) || codes_ring || codes_w4 || had;
-  const int a_rows = (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
+  // M <= 64 rows of q+ and q- stacked in one A tile (P = 16, 32 or 64 rows each)
+  const bool stacked = bn_small && src == ASource::Codes && M <= 64 && use_stacked();
+  const int a_rows = stacked ? (M <= 16 ? 16 : M <= 32 ? 32 : 64)
+                     : (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
   CUtensorMap ta, ta2, tw;
   if (src == ASource::X) {
     const int xe = elt_size(xt);
@@ -896,6 +930,9 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
         if (BN == 192) return launch_codes_out<192, true, false, 12>(yb, ta, ta2, tw, ty, a, stream);
         return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
       }
+      if (stacked)
+        return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
+                                          stream);
       if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256 && codes_wide_epilogue())
         return launch_codes_out<256, false, false, 16>(yb, ta, ta2, tw, ty, a, stream);

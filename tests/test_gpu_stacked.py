@@ -1,0 +1,70 @@
+"""Small M with stacked polarities: one row tile of M <= 64 rows puts its q+
+code rows in rows [0, P) and its q- rows in rows [P, 2P) of one A tile
+(P = 16, 32 or 64), so one tcgen05 MMA per k step yields both DualScale
+products (SegQuant DualScale, Spanish technical summary 2.B: two int8
+products per unit, folded in the epilogue).  The q- accumulators reach the
+folding warps by a shuffle (P = 16) or through shared memory (P = 32, 64).
+
+Checked against the oracle (fp32 outputs bit-exact, bf16 within one ulp,
+every row), and bit for bit against the two-tile form (the development
+build's SEGQUANT_STACK=0) at every narrow tile width, including a ragged
+last tile column."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from synth import workloads as W
+
+from parity_util import Case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import post_quantized_linear_b200 as pq  # noqa: F401  (fails loudly without the library)
+    O.build()
+    yield
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("M", [1, 15, 16, 17, 32, 33, 63, 64])
+def test_stacked_rows_against_oracle_and_two_tile_form(M, out, monkeypatch, dev_lib):
+    import post_quantized_linear_b200 as pq
+    K, N = 1152, 400                      # nine k blocks, N = 400: ragged at every width
+    c = Case(W.small_case(M, K, N, seed=300 + M, out=out))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    res = {}
+    for stack in ("1", "0"):
+        monkeypatch.setenv("SEGQUANT_STACK", stack)
+        for bn in ("32", "64", "96", "128"):
+            monkeypatch.setenv("SEGQUANT_BN_SMALL", bn)
+            res[(stack, bn)] = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b,
+                                                    out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(res[("1", "96")], np.arange(M))
+    if out == "f32":
+        y_ref, _ = c.oracle_rows(np.arange(M))
+        np.testing.assert_array_equal(res[("1", "96")].cpu().numpy(), y_ref)
+    iv = torch.int32 if out == "f32" else torch.int16
+    ref = res[("0", "96")].view(iv)
+    for key, y in res.items():
+        assert torch.equal(y.view(iv), ref), key
+
+
+@pytest.mark.parametrize("M", [16, 64])
+def test_stacked_product_library_full_weight(M):
+    """The product library's default path (stacked at M <= 64) on the
+    (K, N) = (3072, 12288) weight the bench streams: every row against the
+    oracle."""
+    import post_quantized_linear_b200 as pq
+    c = Case(W.small_case(M, 3072, 12288, seed=7, act="silu", bias=False, out="bf16"))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, None)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(y, np.arange(M))
