@@ -200,6 +200,11 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = args.num_kb;
+  // Setup above overlaps the previous kernel in the stream; everything below
+  // reads what earlier kernels wrote (codes, scales) or writes Y.  The next
+  // GEMM may start its own setup on SMs this grid leaves free.
+  grid_dep_launch();
+  grid_dep_wait();
   const int rounds = num_rounds(args);
   auto tiles = [&](int it, Tile& t) { return tile_of(args, it, BN, t); };
 

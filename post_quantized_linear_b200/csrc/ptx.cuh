@@ -57,6 +57,18 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
+// ------------------------------------------------- programmatic launches
+// Under a programmatic (dependent) launch the grid may start before the
+// kernels ahead of it in the stream have finished: grid_dep_wait() returns
+// once they have completed and their memory is visible (immediately for an
+// ordinary launch); grid_dep_launch() lets the next such grid start early.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -332,8 +332,20 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int grid = num_sms();
   if (grid > a.num_tiles) grid = a.num_tiles;
-  kern<<<grid, sq::codes_threads(EPW, LDA, WM == 1), C::SMEM_BYTES, stream>>>(tqp, tqn, tw, ty, a);
-  return cuda_status(cudaGetLastError());
+  // Programmatic launch: the kernel's setup (barriers, TMEM, descriptor
+  // prefetch) overlaps the tail of the kernel before it in the stream; the
+  // kernel waits for that kernel before touching its inputs.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)sq::codes_threads(EPW, LDA, WM == 1));
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tqp, tqn, tw, ty, a));
 }
 
 template <int BN, bool MULTI, bool SINGLE = false, int EPW = sq::epi_warps(MULTI), int WM = 0>
