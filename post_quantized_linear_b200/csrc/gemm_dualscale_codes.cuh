@@ -113,8 +113,12 @@ struct CodesCfg {
   // group units: each epilogue warp's two 32-float buffers of widened weight scales;
   // stacked polarities: the q- accumulators of 32 columns, handed between warps
   static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : (STK_ > 16 ? STK_ * 32 * 4 : 0);
-  static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) < 8
-                               ? ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) : 8;
+  // stacked (small M): three stages at most, so that about 105 KiB of shared
+  // memory and 256 TMEM columns let a CTA of the next GEMM in the stream share
+  // the SM and prefetch its weights while this one finishes
+  static constexpr int S_CAP = STK_ ? 3 : 8;
+  static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) < S_CAP
+                               ? ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) : S_CAP;
   static_assert(STK_ == 0 || ((STK_ == 16 || STK_ == 32 || STK_ == 64) && !MULTI && !SINGLE &&
                               !LDA_ && WM_ == 0 && EPW_ == 4),
                 "stacked polarities: DualScale, one unit, four epilogue warps");
@@ -200,11 +204,12 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = args.num_kb;
-  // Setup above overlaps the previous kernel in the stream; everything below
-  // reads what earlier kernels wrote (codes, scales) or writes Y.  The next
-  // GEMM may start its own setup on SMs this grid leaves free.
+  // Setup above overlaps the previous kernel in the stream; what follows the
+  // wait reads what earlier kernels wrote (codes, scales) or writes Y.  The
+  // next GEMM may start its own setup on SMs this grid leaves free.  (The TMA
+  // thread waits after its weight prefetch.)
   grid_dep_launch();
-  grid_dep_wait();
+  if (warp != 0) grid_dep_wait();
   const int rounds = num_rounds(args);
   auto tiles = [&](int it, Tile& t) { return tile_of(args, it, BN, t); };
 
@@ -222,17 +227,39 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       const int qn_off = STK ? args.a_rows * BK : BM * BK;
       int c = 0;
       bool ok = (args.starve == 0);
+      // Stacked (small M): the weight boxes of the first stages are requested
+      // before the wait -- no kernel writes the weights -- and their stages'
+      // full barriers armed with the whole stage's bytes; the code boxes
+      // follow after the wait.
+      int pre = 0;
+      if constexpr (STK != 0) {
+        Tile t0;
+        if (ok && tiles(0, t0)) {
+          pre = min(C::S, (num_kb + KPS - 1) / KPS);
+          for (int q = 0; q < pre; ++q) {
+            const int nk = min(KPS, num_kb - q * KPS);
+            mbar_arrive_expect_tx(smem_u32(full + q), (uint32_t)nk * kb_tx);
+            for (int j = 0; j < nk; ++j)
+              tma_load_2d(smem_u32(smem + q * C::STAGE + j * C::KB_BYTES + C::A_BYTES), &tmap_w,
+                          smem_u32(full + q), (q * KPS + j) * BK, t0.n0);
+          }
+        }
+      }
+      grid_dep_wait();
       for (int it = 0; it < rounds && ok; ++it) {
         Tile t;
         if (!tiles(it, t)) continue;
         for (int kb0 = 0; kb0 < num_kb; kb0 += KPS) {
           const int s = c % C::S;
-          if (!(ok = wait1(smem_u32(empty + s), ((c / C::S) & 1) ^ 1, abort_flag, budget))) break;
           const int nk = min(KPS, num_kb - kb0);           // k blocks in this stage
-          if constexpr (LDA) {
-            mbar_arrive_expect_tx(smem_u32(full + s), C::W_BYTES);
-          } else {
-            mbar_arrive_expect_tx(smem_u32(full + s), (uint32_t)nk * kb_tx);
+          const bool prefetched = c < pre;                 // weights already requested
+          if (!prefetched) {
+            if (!(ok = wait1(smem_u32(empty + s), ((c / C::S) & 1) ^ 1, abort_flag, budget))) break;
+            if constexpr (LDA) {
+              mbar_arrive_expect_tx(smem_u32(full + s), C::W_BYTES);
+            } else {
+              mbar_arrive_expect_tx(smem_u32(full + s), (uint32_t)nk * kb_tx);
+            }
           }
           for (int j = 0; j < nk; ++j) {
             const int kb = kb0 + j;
@@ -242,6 +269,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
               if constexpr (!SINGLE)
                 tma_load_2d(smem_u32(st + qn_off), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
             }
+            if (prefetched) continue;
             if constexpr (W4)   // packed rows land after the unpacked tile's place
               tma_load_2d(smem_u32(st + C::A_BYTES + C::W_BYTES), &tmap_w, smem_u32(full + s),
                           kb * (BK / 2), t.n0);
