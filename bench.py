@@ -447,12 +447,16 @@ def oracle_step(wl, xn, wn, bn, rows: int):
 
 
 def oracle_sample_rows(wl, xn, wn, bn, step_budget_s: float) -> int:
-    """Rows of the sampled forward that keep one oracle step near the budget."""
-    t8, _ = oracle_step(wl, xn, wn, bn, 8)
-    t16, _ = oracle_step(wl, xn, wn, bn, 16)
-    per_row = max((t16 - t8) / 8, 1e-7)
-    fixed = max(t8 - 8 * per_row, 0.0)
-    return int(max(8, min(wl.M, (step_budget_s - fixed) / per_row)))
+    """Rows of the sampled forward that keep one oracle step near the budget.
+    The oracle runs the rows in parallel on the host threads, so the cost per
+    row is taken between one and four rows per thread."""
+    r1 = min(wl.M, host_threads())
+    r2 = min(wl.M, 4 * r1)
+    t1, _ = oracle_step(wl, xn, wn, bn, r1)
+    t2, _ = oracle_step(wl, xn, wn, bn, r2)
+    per_row = max((t2 - t1) / max(r2 - r1, 1), 1e-7)
+    fixed = max(t1 - r1 * per_row, 0.0)
+    return int(max(r1, min(wl.M, (step_budget_s - fixed) / per_row)))
 
 
 def host_threads() -> int:
