@@ -372,15 +372,51 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs:
+    NVML polled every 2 ms (the GPU this process uses, matched by PCI bus id),
+    else nvidia-smi every 200 ms."""
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
         self.gpu = gpu_index
+        self.period = period_s
         self.rows = []
         self.proc = None
         self.thread = None
+        self.halt = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, pynvml, h):
+        reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.halt.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = reasons(h)
+                self.rows.append([str(sm), str(mx), "", f"{r:x}"])
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
+        try:
+            pynvml, h = self._nvml_handle()
+            self.proc = "nvml"
+            self.thread = threading.Thread(target=self._poll, args=(pynvml, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         cmd = ["nvidia-smi", "-i", str(self.gpu),
                "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
                "--format=csv,noheader,nounits", "-lms", "200"]
@@ -402,12 +438,16 @@ class ClockSampler:
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+        if self.proc == "nvml":
+            self.halt.set()
+            self.thread.join(timeout=5)
+        else:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
         sm, mx, reasons = [], None, set()
         for p in self.rows:
             try:

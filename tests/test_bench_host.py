@@ -50,3 +50,33 @@ def test_timed_kernel_of_each_path():
     assert bench.gemm_kernel_name("combined", 8, "bf16") == "dualscale_gemm_combined_kernel"
     assert bench.gemm_kernel_name("fused", 8, "bf16") == "dualscale_gemm_inplace_kernel"
     assert bench.gemm_kernel_name("fused", 8, "f32") == "dualscale_gemm_kernel"
+
+
+def test_clock_sampler_reads_nvml(monkeypatch):
+    """The sampler polls NVML (a fake module here): idle samples are dropped,
+    the SM clock is the median of the busy samples, and the reasons are the
+    names of the bits seen while busy."""
+    import types
+    fake = types.ModuleType("pynvml")
+    fake.NVML_CLOCK_SM = 1
+    seq = iter([(1965, 0x0), (1965, 0x4), (1800, 0x4), (300, 0x1)] * 1000)
+    state = {"v": (1965, 0)}
+
+    def clock(h, kind):
+        state["v"] = next(seq)
+        return state["v"][0]
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByIndex = lambda i: "h%d" % i
+    fake.nvmlDeviceGetHandleByPciBusId_v2 = lambda bus: "bus"
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: state["v"][1]
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0, period_s=0.0005)
+    s.start()
+    import time
+    time.sleep(0.05)
+    out = s.stop()
+    assert out["samples"] > 10 and out["sm_max_mhz"] == 1965
+    assert out["sm_mhz"] in (1800, 1965)
+    assert out["reasons"] == ["sw_power_cap"]
