@@ -39,7 +39,10 @@
  *     Leading dimensions are in elements.
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream).  Arguments are validated on the host before any
- *     launch; a rejected call enqueues nothing.
+ *     launch; a rejected call enqueues nothing.  The GEMMs from codes are
+ *     programmatic dependent launches: their setup may overlap the kernel
+ *     before them in the stream, but they read their inputs and write Y only
+ *     after that kernel has completed, so stream order holds as usual.
  *   - Device-side conditions (a non-finite calibration maximum, an fp16 group
  *     scale overflow, a bounded pipeline wait that expired) are recorded in a
  *     per-device status word and returned by sq_stream_status().

@@ -554,16 +554,37 @@ __global__ void __launch_bounds__(128) quantize_weights_w8_kernel(
   const WT* row = w + n * ldw;
   const int tid = threadIdx.x, lane = tid & 31;
   if (tid == 0) sh_bad = 0;
+  // A segment row of up to 128 x 16 x 2 values stays in registers between the
+  // two passes (both loads in flight at once, one read of the row).
+  constexpr int kRegIters = 2;
+  const bool in_regs = (k1 - k0) <= 128 * 16 * kRegIters;
+  float vr[kRegIters][16];
   float amax = 0.0f;
   bool bad = false;
-  for (int32_t k = k0 + tid * 16; k < k1; k += 128 * 16) {
-    float v[16];
-    load16<WT>(row + k, v);
+  if (in_regs) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float a = fabsf(v[i]);
-      bad |= !(a <= 3.4028234663852886e38f);
-      amax = fmaxf(amax, a);
+    for (int it = 0; it < kRegIters; ++it)
+      if (k0 + tid * 16 + it * 128 * 16 < k1) load16<WT>(row + k0 + tid * 16 + it * 128 * 16, vr[it]);
+#pragma unroll
+    for (int it = 0; it < kRegIters; ++it)
+      if (k0 + tid * 16 + it * 128 * 16 < k1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = fabsf(vr[it][i]);
+          bad |= !(a <= 3.4028234663852886e38f);
+          amax = fmaxf(amax, a);
+        }
+      }
+  } else {
+    for (int32_t k = k0 + tid * 16; k < k1; k += 128 * 16) {
+      float v[16];
+      load16<WT>(row + k, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float a = fabsf(v[i]);
+        bad |= !(a <= 3.4028234663852886e38f);
+        amax = fmaxf(amax, a);
+      }
     }
   }
 #pragma unroll
@@ -580,9 +601,7 @@ __global__ void __launch_bounds__(128) quantize_weights_w8_kernel(
   const float s = amax / 127.0f;
   const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
   if (tid == 0) scales[(int64_t)j * N + n] = s;
-  for (int32_t k = k0 + tid * 16; k < k1; k += 128 * 16) {
-    float v[16];
-    load16<WT>(row + k, v);
+  auto store16 = [&](const float (&v)[16], int32_t k) {
     uint32_t c[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i)
@@ -591,6 +610,19 @@ __global__ void __launch_bounds__(128) quantize_weights_w8_kernel(
     out.x = pack4_low(c[0], c[1], c[2], c[3]);   out.y = pack4_low(c[4], c[5], c[6], c[7]);
     out.z = pack4_low(c[8], c[9], c[10], c[11]); out.w = pack4_low(c[12], c[13], c[14], c[15]);
     *reinterpret_cast<uint4*>(codes + n * K + k) = out;
+  };
+  if (in_regs) {
+#pragma unroll
+    for (int it = 0; it < kRegIters; ++it) {
+      const int32_t k = k0 + tid * 16 + it * 128 * 16;
+      if (k < k1) store16(vr[it], k);
+    }
+    return;
+  }
+  for (int32_t k = k0 + tid * 16; k < k1; k += 128 * 16) {
+    float v[16];
+    load16<WT>(row + k, v);
+    store16(v, k);
   }
 }
 
@@ -608,13 +640,20 @@ __global__ void __launch_bounds__(256) quantize_weights_w4_kernel(
   if (warp >= N * G) return;
   const int64_t n = warp / G;
   const int64_t g = warp - n * G;
-  const WT* src = w + n * ldw + g * 128 + lane * 4;
+  const WT* src = w + n * ldw + g * 128 + lane * 4;   // 16-byte (fp32) / 8-byte (bf16) aligned
   float v[4];
+  if constexpr (sizeof(WT) == 4) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(src));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+    const uint2 t = __ldg(reinterpret_cast<const uint2*>(src));
+    v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xFFFF0000u);
+  }
   float amax = 0.0f;
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    v[i] = to_f32(src[i]);
     const float a = fabsf(v[i]);
     bad |= !(a <= 3.4028234663852886e38f);
     amax = fmaxf(amax, a);
