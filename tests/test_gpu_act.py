@@ -184,3 +184,25 @@ def test_table_and_direct_paths_agree_on_every_bf16_input(act):
     assert not flags[~tiny].any()
     np.testing.assert_array_equal(c_tab.cpu().numpy()[~flags], oc[~flags])
     np.testing.assert_array_equal(c_dir.cpu().numpy()[~flags], oc[~flags])
+
+
+@pytest.mark.parametrize("act", ["silu", "gelu"])
+def test_fused_activation_k_not_a_multiple_of_128(act):
+    """K = 208 (a multiple of 16 only): the last block of 128 columns is
+    partial; bf16 pre-activations through the code table, every code against
+    the oracle, and nothing written past K."""
+    import post_quantized_linear_b200 as pq
+    M, K = 37, 208
+    z = _z_matrix(act, M, K, "bf16", seed=21)
+    zd, zo = _to_device(z, "bf16")
+    kseg = [0, K]
+    sp, sn = pq.calibrate_act(zd, act, kseg)
+    out = torch.full((M, 224), 55, dtype=torch.int8, device="cuda")
+    c = pq.quantize_activations_combined_act(zd, act, kseg, sp, sn, out=out[:, :K])
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    osp, osn = O.calibrate_act(zo, act, kseg)
+    oc, flags = O.quantize_activations_combined_act(zo, act, kseg, osp, osn)
+    assert not flags.any()
+    np.testing.assert_array_equal(c.cpu().numpy(), oc)
+    assert (out[:, K:].cpu().numpy() == 55).all()
