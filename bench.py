@@ -504,7 +504,7 @@ def host_threads() -> int:
     return int(os.environ.get("OMP_NUM_THREADS", cores))
 
 
-def cpu_baseline(wl, x, w, b, target_s=12.0):
+def cpu_baseline(wl, x, w, b, target_s=20.0):
     """The oracle, as it stands, timed on the host cores on a bounded sample."""
     import oracle as O
     from synth import workloads as W

@@ -23,7 +23,9 @@ template <typename XT> struct Vec;
 template <> struct Vec<__nv_bfloat16> {
   static constexpr int n = 8;
   __device__ __forceinline__ static void load(const void* p, float (&v)[8]) {
-    uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    load_raw(__ldg(reinterpret_cast<const uint4*>(p)), v);
+  }
+  __device__ __forceinline__ static void load_raw(const uint4& u, float (&v)[8]) {
     uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -37,6 +39,10 @@ template <> struct Vec<float> {
   __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
     float4 u = __ldg(reinterpret_cast<const float4*>(p));
     v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+  __device__ __forceinline__ static void load_raw(const uint4& u, float (&v)[4]) {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
   }
 };
 
@@ -74,6 +80,25 @@ __global__ void __launch_bounds__(256) calibrate_kernel(const XT* __restrict__ x
     const XT* col = x + v * VN;
     int64_t m = (int64_t)blockIdx.y * 8 + threadIdx.y;
     const int64_t step = (int64_t)gridDim.y * 8;
+    // eight rows in flight per thread, kept as raw 16-byte vectors
+    for (; m + 7 * step < rows; m += 8 * step) {
+      uint4 raw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(col + (m + u * step) * ldx));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float a[VN];
+        Vec<XT>::load_raw(raw[u], a);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) {
+          const float t = a[i];
+          bad |= (t != t) || (fabsf(t) == __int_as_float(0x7f800000));
+          P = fmaxf(P, t);
+          Q = fmaxf(Q, -t);
+        }
+      }
+    }
     for (; m + 3 * step < rows; m += 4 * step) {
       float a[4][VN];
 #pragma unroll

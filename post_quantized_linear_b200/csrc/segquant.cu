@@ -695,7 +695,9 @@ sq_status quantize_codes(const void* x, sq_dtype xt, int64_t M, int64_t K, int64
   const int64_t groups = K / 16;
   const int gx = (int)((groups + 31) / 32);
   int64_t gy = (M + 7) / 8;
-  const int64_t cap = ((int64_t)num_sms() * 16 + gx - 1) / gx;  // ~16 blocks of 256 per SM
+  // sixteen 256-thread blocks per SM: two full waves of eight resident blocks
+  // (a grid just past that would leave a few blocks for a third)
+  const int64_t cap = (int64_t)num_sms() * 16 / gx;
   if (gy > cap) gy = cap;
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;
@@ -1061,8 +1063,10 @@ sq_status sq_calibrate(const void* x, sq_dtype xt, int64_t rows, int64_t K, int6
   const int64_t nvec = K / (16 / xe);
   const int gx = (int)((nvec + 31) / 32);
   int64_t gy = (rows + 7) / 8;
-  const int64_t target = (int64_t)148 * 8;
-  int64_t cap = (target + gx - 1) / gx;
+  // eight resident 256-thread blocks per SM; every block streams an equal
+  // share of the rows, so the grid fills the SMs once and no block runs in a
+  // second wave after the others
+  int64_t cap = (int64_t)num_sms() * 8 / gx;
   if (cap < 1) cap = 1;
   if (gy > cap) gy = cap;
   if (gy > 65535) gy = 65535;
@@ -1200,7 +1204,7 @@ sq_status calibrate_transformed(const void* x, sq_dtype xt, int64_t rows, int64_
   const int64_t groups = K / 16;
   const int gx = (int)((groups + 31) / 32);
   int64_t gy = (rows + 7) / 8;
-  const int64_t cap = ((int64_t)num_sms() * 8 + gx - 1) / gx;
+  const int64_t cap = std::max<int64_t>(1, (int64_t)num_sms() * 8 / gx);   // one wave
   if (gy > cap) gy = cap;
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;

@@ -179,3 +179,35 @@ def test_gemm_from_codes_edge_fp32_outputs(dtype, bits):
         wc, ws = O.quantize_weights_w4(w.numpy())
     y_ref = O.linear_forward(xo, E.EDGE_KSEG, osp, osn, bits, wc, ws, None, out="f32")
     np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_calibration_of_subnormals_and_signed_zeros(dtype):
+    """Calibration (a7) on columns whose values are all subnormal, signed zeros
+    or a mix: the maxima are taken without flushing subnormals, so the scales
+    equal the oracle's bit for bit (bf16 maxima are taken on packed pairs)."""
+    import post_quantized_linear_b200 as pq
+    rng = np.random.default_rng(31)
+    M, K = 300, 512
+    kseg = [0, 128, 256, 384, 512]
+    if dtype == "bf16":
+        mant = rng.integers(1, 128, size=(M, K)).astype(np.uint16)        # subnormal bf16
+        sign = (rng.random((M, K)) < 0.5).astype(np.uint16) << 15
+        bits = mant | sign
+        bits[:, 128:256] = np.where(rng.random((M, 128)) < 0.5, 0x0000, 0x8000)   # +-0 only
+        bits[:, 256:384] &= 0x807F                                          # subnormal, both signs
+        bits[:, 384:448] |= 0x8000                                          # negatives only
+        xo = bits
+        xd = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    else:
+        v = (rng.integers(1, 1 << 23, size=(M, K)).astype(np.uint32)).view(np.float32).copy()
+        v[rng.random((M, K)) < 0.5] *= -1
+        v[:, 128:256] = np.where(rng.random((M, 128)) < 0.5, 0.0, -0.0)
+        v[:, 384:448] = -np.abs(v[:, 384:448])
+        xo = np.ascontiguousarray(v)
+        xd = torch.from_numpy(xo).cuda()
+    sp, sn = pq.calibrate(xd, kseg)
+    _status_ok()
+    osp, osn = O.calibrate(xo, kseg)
+    np.testing.assert_array_equal(sp.cpu().numpy(), osp)
+    np.testing.assert_array_equal(sn.cpu().numpy(), osn)
