@@ -63,10 +63,10 @@ MMA_I8_OPS_PER_CLK_SM = 16384
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
-    ("mmdit_mlp_up", "codes"): 161525248 + 378640896,     # dualscale_gemm_codes_kernel
-    ("dit_xl2_fc2_cfg", "codes"): 92216576 + 9675264,     # dualscale_gemm_codes_kernel
-    ("seglinear_qkv", "codes"): 56912128 + 31624448,      # dualscale_gemm_codes_kernel
-    ("w4a8", "codes"): 106261760 + 69462784,              # dualscale_gemm_codes_kernel (int4)
+    ("mmdit_mlp_up", "codes"): 163565568 + 380856832,     # dualscale_gemm_codes_kernel
+    ("dit_xl2_fc2_cfg", "codes"): 86029056 + 9071872,     # dualscale_gemm_codes_kernel
+    ("seglinear_qkv", "codes"): 56157696 + 30311936,      # dualscale_gemm_codes_kernel
+    ("w4a8", "codes"): 106174720 + 69751296,              # dualscale_gemm_codes_kernel (int4)
 }
 
 
@@ -808,37 +808,61 @@ def run_ours(args):
         raise RuntimeError("device status word set during the timed region")
     L.release()
 
-    # end to end through the API: host inputs in (pinned), host result out, every step
+    # end to end through the API: host inputs in (pinned), host result out, every
+    # step.  Steps are pipelined over two sets of device buffers: step i's
+    # inputs are copied in (copy-in stream) while step i-1 computes and step
+    # i-2's result is copied out (copy-out stream); PCIe carries both
+    # directions at once.  Every step's copies lie inside the timed region.
     e2e = None
     if not args.no_e2e:
         xh = L.x_host.pin_memory()
         wh = L.w_host.pin_memory()
-        yh = torch.empty((wl.M, wl.N), dtype=L.out_dtype).pin_memory()
-        xdd = torch.empty_like(L.xd)
-        wdd = torch.empty_like(L.wd)
-        calib_d = xdd if wl.calib_rows is None else xdd[: wl.calib_rows]
+        yh = [torch.empty((wl.M, wl.N), dtype=L.out_dtype).pin_memory() for _ in range(2)]
+        xdd = [torch.empty_like(L.xd) for _ in range(2)]
+        wdd = [torch.empty_like(L.wd) for _ in range(2)]
+        ydd = [L.y, torch.empty_like(L.y)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_step():
-            xdd.copy_(xh, non_blocking=True)
-            wdd.copy_(wh, non_blocking=True)
-            L.calibrate(calib_d)
-            L.rest(xs=xdd, ws=wdd)
-            yh.copy_(L.y, non_blocking=True)
+        def e2e_run(n: int):
+            start = torch.cuda.Event()
+            start.record(stream)
+            done_in = [torch.cuda.Event() for _ in range(n)]
+            done_comp = [torch.cuda.Event() for _ in range(n)]
+            done_out = [torch.cuda.Event() for _ in range(n)]
+            s_in.wait_event(start)
+            for i in range(n):
+                b = i % 2
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(done_comp[i - 2])   # the compute read buffer b
+                    xdd[b].copy_(xh, non_blocking=True)
+                    wdd[b].copy_(wh, non_blocking=True)
+                    done_in[i].record(s_in)
+                stream.wait_event(done_in[i])
+                if i >= 2:
+                    stream.wait_event(done_out[i - 2])      # ydd[b] was copied out
+                L.calibrate(xdd[b] if wl.calib_rows is None else xdd[b][: wl.calib_rows])
+                L.rest(xs=xdd[b], ws=wdd[b], ys=ydd[b])
+                done_comp[i].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(done_comp[i])
+                    yh[b].copy_(ydd[b], non_blocking=True)
+                    done_out[i].record(s_out)
+            stream.wait_event(done_out[n - 1])
+            stream.wait_event(done_in[n - 1])
 
-        for _ in range(2):
-            e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_run(args.steps)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e = {"ms": e0.elapsed_time(e1),
                "bi": xh.numel() * xh.element_size() + wh.numel() * wh.element_size(),
-               "bo": yh.numel() * yh.element_size()}
+               "bo": yh[0].numel() * yh[0].element_size()}
 
     mean = lambda v: statistics.mean(v) if v else 0.0   # noqa: E731
     vals = max_over_ranks([total_ms, mean(gemm_ms), mean(fwd_ms), e2e["ms"] if e2e else 0.0,
@@ -908,7 +932,9 @@ def run_ours(args):
                            "unit": "TOPS", "h2d_bytes_per_step": e2e["bi"],
                            "d2h_bytes_per_step": e2e["bo"],
                            "note": "inputs copied from pinned host memory and Y copied back "
-                                   "every step, around the library's calls (device pointers)"}
+                                   "every step, around the library's calls (device pointers); "
+                                   "steps pipelined over two buffer sets, copies in and out on "
+                                   "their own streams"}
     del L
     torch.cuda.empty_cache()
     if rank == 0 and world == 1:
