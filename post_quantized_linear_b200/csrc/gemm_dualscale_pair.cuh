@@ -24,11 +24,9 @@
 // weights, and its tensor core reads only its own half of the weight tile:
 // at BN = 256 that is 48 KiB and half the shared-memory operand traffic of
 // the one-CTA 256-wide tile.
-// The leader commits the MMAs of every KP consecutive stages (two where the
-// ring has an even number of stages: one commit per k block stalls the issue
-// of the next MMAs) to both CTAs' `empty` barrier of that stage group, and
-// each unit to both CTAs' `tmem_full` barriers, each with one multicast
-// commit.
+// The leader commits the MMAs of every KP consecutive stages to both CTAs'
+// `empty` barrier of that stage group, and each unit to both CTAs'
+// `tmem_full` barriers, each with one multicast commit.
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -50,7 +48,9 @@ struct PairCfg {
   static constexpr int STAGE = 2 * Q_TILE + W_HALF;
   static constexpr int Y_BYTES = EPW * stage_y_bytes(Y_BF16);
   static constexpr int S = ((kStageBudget - Y_BYTES) / STAGE) < 8 ? ((kStageBudget - Y_BYTES) / STAGE) : 8;
-  static constexpr int KP = (S % 2 == 0) ? 2 : 1;   // stages per release of the ring
+  // stages per release of the ring: one (releasing two at a time measured
+  // slower with the four stages that fit: 705 against 693 us on the MMDiT shape)
+  static constexpr int KP = 1;
   static constexpr int NBUF = (BN <= 128) ? 2 : 1;
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_BAR = OFF_Y + Y_BYTES;
