@@ -1040,11 +1040,23 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // handshakes (xfull: the q- warps wrote; xempty: the q+ warps have read).  The
 // fold is fold8_exact's and the store epilogue_tma_store's, so the outputs are
 // those of the two-tile form.
-template <int BN, int NBUF, bool Y_BF16, bool XCH, class TileFn>
+// CSPLIT (P = 16, the tile's K range split over the CTAs of a cluster): a CTA
+// of rank r > 0 adds its raw accumulators (lanes 0..31, the tile's columns)
+// into the [32][BN] int32 buffer of the rank-0 CTA (`part`, zeroed before the
+// cluster started; lane l's column c at l*BN + c with the low five bits of c
+// XOR l), then arrives on that CTA's `parts` barrier; rank 0 waits for the
+// others (bounded), adds the buffer to its own accumulators -- integer sums,
+// exact in any order -- and folds and stores as above.
+template <int BN, int NBUF, bool Y_BF16, bool XCH, bool CSPLIT = false, class TileFn>
 __device__ __forceinline__ void epilogue_stacked(
     const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, uint32_t* xch, int quad,
     int lane, uint32_t t_lane, uint64_t* tmem_full, uint32_t empty_base, uint32_t xfull,
-    uint32_t xempty, int rounds, TileFn tile_fn, volatile int* abort_flag, long long budget) {
+    uint32_t xempty, int rounds, TileFn tile_fn, volatile int* abort_flag, long long budget,
+    uint32_t crank = 0, uint32_t part = 0, uint32_t parts_bar = 0) {
+  static_assert(!CSPLIT || !XCH, "K split: P = 16");
+  auto pidx = [&](int c) { return (uint32_t)(lane * BN + ((c & ~31) | ((c & 31) ^ lane))); };
+  const uint32_t part0 = CSPLIT ? mapa_shared(part, 0) : 0u;   // rank 0's buffer
+  bool parts_in = false;
   constexpr int ROWB = Y_BF16 ? 64 : 128;
   uint8_t* srow = stage_y + lane * ROWB;
   const uint32_t sbase = smem_u32(stage_y);
@@ -1080,6 +1092,29 @@ __device__ __forceinline__ void epilogue_stacked(
       for (int i = 0; i < 4; ++i) tmem_ld8(t_lane + tcol + 8 * i, v[i]);
       tmem_wait_ld();
       if (p == npass - 1) release(b);   // every column of the tile is in registers
+      if constexpr (CSPLIT) {
+        if (crank != 0) {   // add into rank 0's buffer; it folds and stores
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) red_add_cluster(part0 + 4u * pidx(col + 8 * i + k), v[i][k]);
+          if (p == npass - 1) {
+            fence_cluster();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(mapa_shared(parts_bar, 0));
+          }
+          continue;
+        }
+        if (!parts_in) {   // the other CTAs' partial sums have landed
+          if (!(ok = wait_warp<true>(parts_bar, 0, abort_flag, budget))) break;
+          parts_in = true;
+        }
+        const uint32_t* pb = reinterpret_cast<const uint32_t*>(__cvta_shared_to_generic(part));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[i][k] += pb[pidx(col + 8 * i + k)];
+      }
       uint32_t vn[4][8];
       if constexpr (!XCH) {
 #pragma unroll

@@ -87,8 +87,11 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 // form are issued.  The A area of a k block is 2 * STK_ rows; the MMA still
 // reads 128 rows from its start (the rows past 2P belong to the weight tile or
 // the next k block and land in accumulator lanes nobody reads).
+// CSPLIT_ (stacked rows, P = 16): the K range of an N tile is split over the
+// CTAs of a cluster; the first CTA keeps a [32][BN] int32 buffer in shared
+// memory into which the others add their accumulators.
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
-          bool LDA_ = false, int KPS_ = 1, int WM_ = 0, int STK_ = 0>
+          bool LDA_ = false, int KPS_ = 1, int WM_ = 0, int STK_ = 0, bool CSPLIT_ = false>
 struct CodesCfg {
   static constexpr bool W4_ = (WM_ == 1);
   static constexpr bool LDA = LDA_;
@@ -117,8 +120,10 @@ struct CodesCfg {
   // memory and 256 TMEM columns let a CTA of the next GEMM in the stream share
   // the SM and prefetch its weights while this one finishes
   static constexpr int S_CAP = STK_ ? 3 : 8;
-  static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) < S_CAP
-                               ? ((kStageBudget - Y_BYTES - SW_BYTES) / STAGE) : S_CAP;
+  static constexpr int PART_BYTES = CSPLIT_ ? 32 * BN_ * 4 : 0;
+  static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) < S_CAP
+                               ? ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) : S_CAP;
+  static_assert(!CSPLIT_ || STK_ == 16, "K split over a cluster: stacked rows with P = 16");
   static_assert(STK_ == 0 || ((STK_ == 16 || STK_ == 32 || STK_ == 64) && !MULTI && !SINGLE &&
                               !LDA_ && WM_ == 0 && EPW_ == 4),
                 "stacked polarities: DualScale, one unit, four epilogue warps");
@@ -128,9 +133,12 @@ struct CodesCfg {
   static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
-  static constexpr int OFF_BAR = OFF_SW + SW_BYTES;
+  static constexpr int OFF_PART = OFF_SW + SW_BYTES;
+  static constexpr int OFF_BAR = OFF_PART + PART_BYTES;
   // full, empty; tmem full/empty; drain; (W4) unpacked; (stacked) exchange full/empty
-  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0) + (STK_ > 16 ? 2 : 0);
+  // (+ K split: the partial sums of the other CTAs have landed)
+  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0) + (STK_ > 16 ? 2 : 0) +
+                                  (CSPLIT_ ? 1 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = NACC * BN * NBUF;
@@ -143,14 +151,14 @@ struct CodesCfg {
 };
 
 template <int BN, bool Y_BF16, bool MULTI, bool SINGLE = false, int EPW = epi_warps(MULTI),
-          bool LDA = false, int KPS = 1, int WM = 0, int STK = 0>
+          bool LDA = false, int KPS = 1, int WM = 0, int STK = 0, bool CSPLIT = false>
 __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     dualscale_gemm_codes_kernel(const __grid_constant__ CUtensorMap tmap_qp,
                                 const __grid_constant__ CUtensorMap tmap_qn,
                                 const __grid_constant__ CUtensorMap tmap_w,
                                 const __grid_constant__ CUtensorMap tmap_y,
                                 const __grid_constant__ GemmArgs args) {
-  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, WM, STK>;
+  using C = CodesCfg<BN, MULTI, Y_BF16, SINGLE, EPW, LDA, KPS, WM, STK, CSPLIT>;
   constexpr bool W4 = (WM == 1);        // packed int4 tiles, unpack warps
   constexpr bool SEEDED = (WM != 0);    // one unit per k block, seeded accumulators
   constexpr int EPI0 = codes_epi_warp0(LDA, W4);
@@ -169,6 +177,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   uint64_t* ready = drain_bar + 1;        // [8] (W4) int4 tile unpacked
   uint64_t* xfull = ready + (W4 ? 8 : 0);  // (stacked, P > 16) q- accumulators handed over
   uint64_t* xempty = xfull + 1;            // (stacked, P > 16) q+ warps done reading them
+  uint64_t* parts = xfull + (STK > 16 ? 2 : 0);   // (K split, first CTA) partial sums added
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -192,6 +201,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       mbar_init(smem_u32(xfull), (uint32_t)((args.a_rows + 31) / 32));
       mbar_init(smem_u32(xempty), (uint32_t)((args.a_rows + 31) / 32));
     }
+    if constexpr (CSPLIT) mbar_init(smem_u32(parts), (uint32_t)(args.splits - 1));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -199,19 +209,40 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
     tmem_relinquish();
   }
+  if constexpr (CSPLIT) {   // the partial-sum buffer starts at zero
+    uint4* pb = reinterpret_cast<uint4*>(smem + C::OFF_PART);
+    for (int i = threadIdx.x; i < C::PART_BYTES / 16; i += blockDim.x) pb[i] = make_uint4(0, 0, 0, 0);
+  }
   tc_fence_before();
   __syncthreads();
+  // K split: every CTA of the cluster has its barriers and a zeroed buffer
+  // before any of them signals or adds into another's
+  if constexpr (CSPLIT) cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = args.num_kb;
+  // K split over the cluster: this CTA's k blocks of its cluster's N tile
+  const uint32_t crank = CSPLIT ? cluster_ctarank() : 0u;
+  // (k blocks shared evenly: every range is nonempty while num_kb >= splits)
+  const int kb_lo = CSPLIT ? (int)crank * num_kb / args.splits : 0;
+  const int kb_hi = CSPLIT ? ((int)crank + 1) * num_kb / args.splits : num_kb;
   // Setup above overlaps the previous kernel in the stream; what follows the
   // wait reads what earlier kernels wrote (codes, scales) or writes Y.  The
   // next GEMM may start its own setup on SMs this grid leaves free.  (The TMA
   // thread waits after its weight prefetch.)
   grid_dep_launch();
   if (warp != 0) grid_dep_wait();
-  const int rounds = num_rounds(args);
-  auto tiles = [&](int it, Tile& t) { return tile_of(args, it, BN, t); };
+  const int rounds = CSPLIT ? 1 : num_rounds(args);
+  auto tiles = [&](int it, Tile& t) {
+    if constexpr (CSPLIT) {   // one N tile per cluster, one row tile
+      if (it != 0) return false;
+      t.m0 = 0;
+      t.n0 = (int)(blockIdx.x / (unsigned)args.splits) * BN;
+      t.width = min(BN, args.N - t.n0);
+      return true;
+    }
+    return tile_of(args, it, BN, t);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -235,13 +266,13 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       if constexpr (STK != 0) {
         Tile t0;
         if (ok && tiles(0, t0)) {
-          pre = min(C::S, (num_kb + KPS - 1) / KPS);
+          pre = min(C::S, (kb_hi - kb_lo + KPS - 1) / KPS);
           for (int q = 0; q < pre; ++q) {
-            const int nk = min(KPS, num_kb - q * KPS);
+            const int nk = min(KPS, kb_hi - kb_lo - q * KPS);
             mbar_arrive_expect_tx(smem_u32(full + q), (uint32_t)nk * kb_tx);
             for (int j = 0; j < nk; ++j)
               tma_load_2d(smem_u32(smem + q * C::STAGE + j * C::KB_BYTES + C::A_BYTES), &tmap_w,
-                          smem_u32(full + q), (q * KPS + j) * BK, t0.n0);
+                          smem_u32(full + q), (kb_lo + q * KPS + j) * BK, t0.n0);
           }
         }
       }
@@ -249,9 +280,9 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       for (int it = 0; it < rounds && ok; ++it) {
         Tile t;
         if (!tiles(it, t)) continue;
-        for (int kb0 = 0; kb0 < num_kb; kb0 += KPS) {
+        for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += KPS) {
           const int s = c % C::S;
-          const int nk = min(KPS, num_kb - kb0);           // k blocks in this stage
+          const int nk = min(KPS, kb_hi - kb0);            // k blocks in this stage
           const bool prefetched = c < pre;                 // weights already requested
           if (!prefetched) {
             if (!(ok = wait1(smem_u32(empty + s), ((c / C::S) & 1) ^ 1, abort_flag, budget))) break;
@@ -293,14 +324,14 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
         const uint32_t idesc = idesc_i8(BM, t.width);
         bool unit_open = false;
         uint32_t d_pos = 0;
-        for (int kb0 = 0; kb0 < num_kb && ok; kb0 += KPS) {
+        for (int kb0 = kb_lo; kb0 < kb_hi && ok; kb0 += KPS) {
           const int s = c % C::S;
           // W4: the unpack warps' ready barrier (it follows the stage's full barrier)
           if (!(ok = wait1(smem_u32((W4 ? ready : full) + s), (c / C::S) & 1, abort_flag, budget))) break;
           // tiles written by cp.async or by the unpack warps (generic proxy)
           // before the tensor core reads them
           if constexpr (LDA || W4) fence_proxy_async_smem();
-          const int nk = min(KPS, num_kb - kb0);
+          const int nk = min(KPS, kb_hi - kb0);
           for (int j = 0; j < nk; ++j) {
             const int kb = kb0 + j;
             if (!unit_open) {   // a unit (K segment) may start inside a stage
@@ -324,7 +355,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
                 umma_i8(d_pos + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, acc);
             }
             unit_open = true;
-            if (kb_closes_unit(args, kb)) {
+            // (K split: the CTA's range is one unit)
+            if (CSPLIT ? kb + 1 == kb_hi : kb_closes_unit(args, kb)) {
               umma_commit(smem_u32(tmem_full + (ug % C::NBUF)));
               ++ug;
               unit_open = false;
@@ -420,10 +452,10 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
     if constexpr (STK != 0) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-      epilogue_stacked<BN, C::NBUF, Y_BF16, (STK > 16)>(
+      epilogue_stacked<BN, C::NBUF, Y_BF16, (STK > 16), CSPLIT>(
           args, &tmap_y, stage_y, reinterpret_cast<uint32_t*>(smem + C::OFF_SW), quad, lane, t_lane,
           tmem_full, smem_u32(tmem_empty), smem_u32(xfull), smem_u32(xempty), rounds, tiles,
-          abort_flag, budget);
+          abort_flag, budget, crank, smem_u32(smem + C::OFF_PART), smem_u32(parts));
     } else if constexpr (SEEDED) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
       float* sw_stage = reinterpret_cast<float*>(smem + C::OFF_SW) + (warp - EPI0) * 64;
@@ -446,6 +478,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  // K split: the first CTA's buffer outlives every add into it
+  if constexpr (CSPLIT) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_ALLOC);

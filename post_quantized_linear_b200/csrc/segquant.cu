@@ -310,8 +310,12 @@ int codes_kps() { return dev_switch("SEGQUANT_KPS", 2) == 2 ? 2 : 1; }
 // tile (one MMA per k step); SEGQUANT_STACK=0 selects two 128-row code tiles.
 bool use_stacked() { return dev_switch("SEGQUANT_STACK", 1) != 0; }
 
+// Whether a stacked row tile of M <= 16 with few N tiles splits the K range of
+// each tile over a cluster of CTAs; SEGQUANT_CSPLIT=0 keeps one CTA per tile.
+bool use_cluster_split() { return dev_switch("SEGQUANT_CSPLIT", 1) != 0; }
+
 template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULTI), bool LDA = false,
-          int KPS = 1, int WM = 0, int STK = 0>
+          int KPS = 1, int WM = 0, int STK = 0, bool CSPLIT = false>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
   if constexpr (kDev && !LDA && KPS == 1 && WM == 0 && STK == 0 && !(MULTI && BN > 128)) {
@@ -322,8 +326,9 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
     if (codes_kps() == 2)
       return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
   }
-  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, WM, STK>;
-  constexpr auto kern = sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM, STK>;
+  using C = sq::CodesCfg<BN, MULTI, YB, SINGLE, EPW, LDA, KPS, WM, STK, CSPLIT>;
+  constexpr auto kern =
+      sq::dualscale_gemm_codes_kernel<BN, YB, MULTI, SINGLE, EPW, LDA, KPS, WM, STK, CSPLIT>;
   cudaError_t e = smem_limit<kern>(C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_status(e);
   a.n_full = a.N / BN;
@@ -332,6 +337,7 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   a.num_tiles = a.m_tiles * (a.n_full + (a.tail ? 1 : 0));
   int grid = num_sms();
   if (grid > a.num_tiles) grid = a.num_tiles;
+  if constexpr (CSPLIT) grid = a.num_tiles * a.splits;   // one cluster of `splits` CTAs per tile
   // Programmatic launch: the kernel's setup (barriers, TMEM, descriptor
   // prefetch) overlaps the tail of the kernel before it in the stream; the
   // kernel waits for that kernel before touching its inputs.
@@ -340,11 +346,15 @@ sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUt
   cfg.blockDim = dim3((unsigned)sq::codes_threads(EPW, LDA, WM == 1));
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CSPLIT ? (unsigned)a.splits : 1u;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = CSPLIT ? 2 : 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, tqp, tqn, tw, ty, a));
 }
 
@@ -400,6 +410,10 @@ template <int BN>
 sq_status launch_codes_stacked(int stk, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                                const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                                cudaStream_t stream) {
+  if (stk == 16 && a.splits > 1)   // the K range split over a cluster
+    return y_bf16
+               ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream)
+               : launch_codes<BN, false, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream);
   if (stk == 16)
     return y_bf16 ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16>(tqp, tqn, tw, ty, a, stream)
                   : launch_codes<BN, false, false, false, 4, false, 2, 0, 16>(tqp, tqn, tw, ty, a, stream);
@@ -944,9 +958,17 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
         if (BN == 192) return launch_codes_out<192, true, false, 12>(yb, ta, ta2, tw, ty, a, stream);
         return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
       }
-      if (stacked)
+      if (stacked) {
+        // M <= 16 with few N tiles: split each tile's K range over a cluster of
+        // up to four CTAs, so that more SMs stream the weight
+        const int64_t ntiles = (N + bn_small - 1) / bn_small;
+        int cs = 1;
+        if (a_rows <= 16 && use_cluster_split())
+          while (cs < 4 && ntiles * cs * 2 <= num_sms() && a.num_kb >= cs * 2 * 2) cs *= 2;
+        if (cs > 1) a.splits = cs;   // the kernel gives CTA r k blocks [r*kb/cs, (r+1)*kb/cs)
         return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
                                           stream);
+      }
       if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256 && codes_wide_epilogue())
         return launch_codes_out<256, false, false, 16>(yb, ta, ta2, tw, ty, a, stream);

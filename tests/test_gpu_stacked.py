@@ -8,7 +8,8 @@ folding warps by a shuffle (P = 16) or through shared memory (P = 32, 64).
 Checked against the oracle (fp32 outputs bit-exact, bf16 within one ulp,
 every row), and bit for bit against the two-tile form (the development
 build's SEGQUANT_STACK=0) at every narrow tile width, including a ragged
-last tile column."""
+last tile column.  At M <= 16 with few N tiles the K range of a tile is
+split over a cluster of CTAs; that form is checked the same way."""
 import numpy as np
 import pytest
 import torch
@@ -68,3 +69,35 @@ def test_stacked_product_library_full_weight(M):
     torch.cuda.synchronize()
     assert pq.stream_status() == 0
     c.compare_rows(y, np.arange(M))
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("M", [1, 16])
+@pytest.mark.parametrize("K,N", [(1152, 1152), (4608, 1152), (1152, 400), (3072, 2048)])
+def test_k_split_over_a_cluster(K, N, M, out, monkeypatch, dev_lib):
+    """M <= 16 with few N tiles: each N tile's k blocks are shared evenly by
+    the CTAs of a cluster (2 or 4; 9 k blocks over 4 CTAs gives 2, 2, 2, 3),
+    which add their int32 accumulators into the first CTA's shared memory
+    before it folds.  Integer sums, so the result is bit-identical to one CTA
+    per tile (the development build's SEGQUANT_CSPLIT=0) at every tile width,
+    and fp32 outputs equal the oracle's."""
+    import post_quantized_linear_b200 as pq
+    c = Case(W.small_case(M, K, N, seed=900 + M + K // 128, out=out))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    res = {}
+    for split in ("1", "0"):
+        monkeypatch.setenv("SEGQUANT_CSPLIT", split)
+        for bn in ("32", "64", "128"):
+            monkeypatch.setenv("SEGQUANT_BN_SMALL", bn)
+            res[(split, bn)] = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b,
+                                                    out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(res[("1", "32")], np.arange(M))
+    if out == "f32":
+        y_ref, _ = c.oracle_rows(np.arange(M))
+        np.testing.assert_array_equal(res[("1", "32")].cpu().numpy(), y_ref)
+    iv = torch.int32 if out == "f32" else torch.int16
+    ref = res[("0", "32")].view(iv)
+    for key, y in res.items():
+        assert torch.equal(y.view(iv), ref), key
