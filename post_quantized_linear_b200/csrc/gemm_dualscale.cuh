@@ -1041,12 +1041,14 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // fold is fold8_exact's and the store epilogue_tma_store's, so the outputs are
 // those of the two-tile form.
 // CSPLIT (P = 16, the tile's K range split over the CTAs of a cluster): a CTA
-// of rank r > 0 adds its raw accumulators (lanes 0..31, the tile's columns)
-// into the [32][BN] int32 buffer of the rank-0 CTA (`part`, zeroed before the
-// cluster started; lane l's column c at l*BN + c with the low five bits of c
-// XOR l), then arrives on that CTA's `parts` barrier; rank 0 waits for the
-// others (bounded), adds the buffer to its own accumulators -- integer sums,
-// exact in any order -- and folds and stores as above.
+// of rank r > 0 writes its raw accumulators (lanes 0..31, the tile's columns)
+// into its own [32][BN] int32 buffer (`part`, zeroed at setup; lane l's column
+// c at l*BN + c with the low five bits of c XOR l), then one bulk reduction adds
+// that buffer into the rank-0 CTA's, counted as bytes on rank 0's `parts`
+// barrier; rank 0 waits for every byte (bounded), adds the buffer to its own
+// accumulators -- integer sums, exact in any order -- and folds and stores as
+// above.  (The buffers stay alive until rank 0 has seen every byte: the CTAs
+// leave through a cluster barrier after the epilogue.)
 template <int BN, int NBUF, bool Y_BF16, bool XCH, bool CSPLIT = false, class TileFn>
 __device__ __forceinline__ void epilogue_stacked(
     const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, uint32_t* xch, int quad,
@@ -1093,15 +1095,17 @@ __device__ __forceinline__ void epilogue_stacked(
       tmem_wait_ld();
       if (p == npass - 1) release(b);   // every column of the tile is in registers
       if constexpr (CSPLIT) {
-        if (crank != 0) {   // add into rank 0's buffer; it folds and stores
+        if (crank != 0) {   // into this CTA's buffer, then added into rank 0's
+          uint32_t* own = reinterpret_cast<uint32_t*>(__cvta_shared_to_generic(part));
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) red_add_cluster(part0 + 4u * pidx(col + 8 * i + k), v[i][k]);
+            for (int k = 0; k < 8; ++k) own[pidx(col + 8 * i + k)] = v[i][k];
           if (p == npass - 1) {
-            fence_cluster();
+            fence_proxy_async_smem();   // the bulk copy reads through the async proxy
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(mapa_shared(parts_bar, 0));
+            if (lane == 0)
+              bulk_reduce_add_u32_cluster(part0, part, 32u * BN * 4u, mapa_shared(parts_bar, 0));
           }
           continue;
         }

@@ -89,7 +89,8 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 // the next k block and land in accumulator lanes nobody reads).
 // CSPLIT_ (stacked rows, P = 16): the K range of an N tile is split over the
 // CTAs of a cluster; the first CTA keeps a [32][BN] int32 buffer in shared
-// memory into which the others add their accumulators.
+// memory into which the others add their accumulators (one bulk reduction
+// each).  One tile per CTA: one TMEM buffer.
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
           bool LDA_ = false, int KPS_ = 1, int WM_ = 0, int STK_ = 0, bool CSPLIT_ = false>
 struct CodesCfg {
@@ -130,7 +131,8 @@ struct CodesCfg {
   static_assert(KPS == 1 || !LDA_, "two k blocks per stage: TMA loads");
   static_assert(WM_ == 0 || (MULTI && !SINGLE && !LDA_ && KPS_ == 1 && BN_ == 128),
                 "group units: DualScale, one k block per stage, BN = 128");
-  static constexpr int NBUF = (2 * NACC * BN <= 512) ? 2 : 1;   // TMEM accumulator buffers
+  // TMEM accumulator buffers (K split: one tile per CTA, one buffer)
+  static constexpr int NBUF = CSPLIT_ ? 1 : ((2 * NACC * BN <= 512) ? 2 : 1);
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
   static constexpr int OFF_PART = OFF_SW + SW_BYTES;
@@ -201,9 +203,13 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       mbar_init(smem_u32(xfull), (uint32_t)((args.a_rows + 31) / 32));
       mbar_init(smem_u32(xempty), (uint32_t)((args.a_rows + 31) / 32));
     }
-    if constexpr (CSPLIT) mbar_init(smem_u32(parts), (uint32_t)(args.splits - 1));
+    if constexpr (CSPLIT) mbar_init(smem_u32(parts), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // K split, first CTA: the others' partial sums arrive as bytes on `parts`
+    if constexpr (CSPLIT)
+      if (cluster_ctarank() == 0)
+        mbar_arrive_expect_tx(smem_u32(parts), (uint32_t)((args.splits - 1) * C::PART_BYTES));
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);

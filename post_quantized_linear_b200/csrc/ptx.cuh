@@ -253,13 +253,17 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
                    "memory");
 }
-// Integer add into another CTA's shared memory (cluster address), no return.
-__device__ __forceinline__ void red_add_cluster(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v)
-               : "memory");
-}
-__device__ __forceinline__ void fence_cluster() {
-  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+// Adds `bytes` of u32 words from this CTA's shared memory into another CTA's
+// (cluster address `dst`), elementwise, by the bulk copy engine; the bytes
+// count toward the transaction count of the mbarrier `bar` (a cluster address
+// in the destination CTA).  Addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_reduce_add_u32_cluster(uint32_t dst, uint32_t src, uint32_t bytes,
+                                                            uint32_t bar) {
+  asm volatile(
+      "cp.reduce.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes.add.u32 "
+      "[%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 // Wait with cluster-scope acquire (for barriers that receive remote arrivals).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {

@@ -381,6 +381,12 @@ bool codes_wide_epilogue() { return dev_switch("SEGQUANT_EPW16", 1) != 0; }
 // of 32, four epilogue warps); cost = waves x cycles per MMA, where an M = 128
 // MMA takes about BN/2 cycles but no less than 48 (narrow products lose rate);
 // ties go to the narrower tile (more SMs share the stream).  0 = not small.
+// Whether the development switch SEGQUANT_BN_SMALL fixes the small-M tile width.
+bool bn_small_forced() {
+  const int v = dev_switch("SEGQUANT_BN_SMALL", 0);
+  return v == 32 || v == 64 || v == 96 || v == 128;
+}
+
 int choose_bn_small(int64_t M, int64_t N) {
   if (M > sq::BM) return 0;
   {
@@ -410,15 +416,98 @@ template <int BN>
 sq_status launch_codes_stacked(int stk, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                                const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                                cudaStream_t stream) {
-  if (stk == 16 && a.splits > 1)   // the K range split over a cluster
-    return y_bf16
-               ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream)
-               : launch_codes<BN, false, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream);
   if (stk == 16)
     return y_bf16 ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16>(tqp, tqn, tw, ty, a, stream)
                   : launch_codes<BN, false, false, false, 4, false, 2, 0, 16>(tqp, tqn, tw, ty, a, stream);
   return y_bf16 ? launch_codes<BN, true, false, false, 4, false, 2, 0, 64>(tqp, tqn, tw, ty, a, stream)
                 : launch_codes<BN, false, false, false, 4, false, 2, 0, 64>(tqp, tqn, tw, ty, a, stream);
+}
+
+// Stacked rows (M <= 16) with each N tile's k blocks shared by the a.splits
+// CTAs of a cluster.
+template <int BN>
+sq_status launch_codes_split(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+                             const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                             cudaStream_t stream) {
+  return y_bf16
+             ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream)
+             : launch_codes<BN, false, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream);
+}
+
+sq_status launch_codes_small_split(int bn, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+                                   const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                                   cudaStream_t stream) {
+  switch (bn) {
+    case 32: return launch_codes_split<32>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 64: return launch_codes_split<64>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 96: return launch_codes_split<96>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    default: return launch_codes_split<128>(y_bf16, tqp, tqn, tw, ty, a, stream);
+  }
+}
+
+// How many clusters of `cs` CTAs (one CTA per SM, with the widest split
+// kernel's shared memory) the current device runs at once.  A cluster stays inside one
+// group of SMs, so this is below num_sms() / cs when the groups' sizes are not
+// multiples of cs.  0 when the query fails.
+int max_clusters(int cs) {
+  static std::atomic<int> cached[kMaxDevices][9] = {};
+  int dev = 0;
+  if (cs < 1 || cs > 8 || cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  if (cacheable) {
+    const int v = cached[dev][cs].load(std::memory_order_relaxed);
+    if (v != 0) return v > 0 ? v : 0;
+  }
+  constexpr auto kern = sq::dualscale_gemm_codes_kernel<128, true, false, false, 4, false, 2, 0, 16, true>;
+  // most of an SM's shared memory: one CTA per SM whatever the tile width (the
+  // attribute is an upper bound, so raising it leaves every launch valid)
+  constexpr int kQuerySmem = 200 * 1024;
+  int n = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuerySmem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs);
+    cfg.blockDim = dim3((unsigned)sq::codes_threads(4, false, false));
+    cfg.dynamicSmemBytes = kQuerySmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+  }
+  if (cacheable) cached[dev][cs].store(n > 0 ? n : -1, std::memory_order_relaxed);
+  return n;
+}
+
+// M <= 16 rows (stacked): the tile width and the cluster size that shares each
+// N tile's k blocks.  The time of such a layer follows the number of k blocks
+// a CTA streams (the stages in flight cover a fixed HBM latency each), not
+// the tile width: the narrow tile `bn0` split over as many CTAs (2..8, at least
+// two k blocks apiece, clusters the device runs at once) as the SMs hold;
+// when bn0 cannot be split and its tiles leave a fifth of the SMs idle, the
+// tile of twice its width split in two or more.  `forced`: keep bn0.
+void choose_small_split(int64_t N, int num_kb, int bn0, bool forced, int& bn, int& cs) {
+  const int sms = num_sms();
+  auto split_of = [&](int b) {
+    const int64_t tiles = (N + b - 1) / b;
+    int c = 1;
+    for (int k = 2; k <= 8; ++k)
+      if (tiles * k <= sms && num_kb >= 2 * k && tiles <= max_clusters(k)) c = k;
+    return c;
+  };
+  bn = bn0;
+  cs = split_of(bn0);
+  if (forced || cs > 1 || bn0 * 2 > 128 || ((N + bn0 - 1) / bn0) * 5 >= (int64_t)sms * 4) return;
+  const int c2 = split_of(bn0 * 2);
+  if (c2 > 1) {
+    bn = bn0 * 2;
+    cs = c2;
+  }
 }
 
 sq_status launch_codes_small_stacked(int bn, int stk, bool y_bf16, const CUtensorMap& tqp,
@@ -835,7 +924,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   int BN = (acc != nullptr || multi) ? 128 : choose_bn(M, N, multi, f32x, codes_ring);
   if (multi && codes_ring) BN = choose_bn_multi(M, N);   // several K segments, from codes
   // one row tile, one unit per tile, GEMM from codes: narrow tiles over all SMs
-  const int bn_small = (!multi && acc == nullptr && (src == ASource::Codes || src == ASource::Single) &&
+  int bn_small = (!multi && acc == nullptr && (src == ASource::Codes || src == ASource::Single) &&
                         !(src == ASource::Codes && use_pair(N, w4)) && use_codes_ring())
                            ? choose_bn_small(M, N) : 0;
   if (bn_small) BN = bn_small;
@@ -846,6 +935,17 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const bool codes_kernel = (src == ASource::Single) || codes_ring || codes_w4 || had;
   // M <= 64 rows of q+ and q- stacked in one A tile (P = 16, 32 or 64 rows each)
   const bool stacked = bn_small && src == ASource::Codes && M <= 64 && use_stacked();
+  // M <= 16: each N tile's k blocks shared by a cluster of split_cs CTAs,
+  // on a tile width chosen for it
+  int split_cs = 1;
+  if (stacked && M <= 16 && use_cluster_split()) {
+    int sbn = bn_small;
+    choose_small_split(N, (int)((K + sq::BK - 1) / sq::BK), bn_small, bn_small_forced(), sbn, split_cs);
+    if (split_cs > 1) {
+      bn_small = sbn;
+      BN = sbn;
+    }
+  }
   const int a_rows = stacked ? (M <= 16 ? 16 : M <= 32 ? 32 : 64)
                      : (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
   CUtensorMap ta, ta2, tw;
@@ -959,13 +1059,10 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
         return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
       }
       if (stacked) {
-        // M <= 16 with few N tiles: split each tile's K range over a cluster of
-        // up to four CTAs, so that more SMs stream the weight
-        const int64_t ntiles = (N + bn_small - 1) / bn_small;
-        int cs = 1;
-        if (a_rows <= 16 && use_cluster_split())
-          while (cs < 4 && ntiles * cs * 2 <= num_sms() && a.num_kb >= cs * 2 * 2) cs *= 2;
-        if (cs > 1) a.splits = cs;   // the kernel gives CTA r k blocks [r*kb/cs, (r+1)*kb/cs)
+        if (split_cs > 1) {   // CTA r of a cluster: k blocks [r*kb/cs, (r+1)*kb/cs)
+          a.splits = split_cs;
+          return launch_codes_small_split(bn_small, yb, ta, ta2, tw, ty, a, stream);
+        }
         return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
                                           stream);
       }

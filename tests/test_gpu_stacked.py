@@ -73,21 +73,23 @@ def test_stacked_product_library_full_weight(M):
 
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 @pytest.mark.parametrize("M", [1, 16])
-@pytest.mark.parametrize("K,N", [(1152, 1152), (4608, 1152), (1152, 400), (3072, 2048)])
+@pytest.mark.parametrize("K,N", [(1152, 1152), (4608, 1152), (1152, 400), (3072, 2048),
+                                 (3072, 12288)])
 def test_k_split_over_a_cluster(K, N, M, out, monkeypatch, dev_lib):
-    """M <= 16 with few N tiles: each N tile's k blocks are shared evenly by
-    the CTAs of a cluster (2 or 4; 9 k blocks over 4 CTAs gives 2, 2, 2, 3),
-    which add their int32 accumulators into the first CTA's shared memory
-    before it folds.  Integer sums, so the result is bit-identical to one CTA
-    per tile (the development build's SEGQUANT_CSPLIT=0) at every tile width,
-    and fp32 outputs equal the oracle's."""
+    """M <= 16: each N tile's k blocks are shared evenly by the CTAs of a
+    cluster (2 to 8; 9 k blocks over 4 CTAs gives 2, 2, 2, 3), which add their
+    int32 accumulators into the first CTA's shared memory before it folds.
+    Integer sums, so the result is bit-identical to one CTA per tile (the
+    development build's SEGQUANT_CSPLIT=0) at every tile width -- the widths
+    fixed here and the library's own choice ("0": up to 256 columns) -- and
+    fp32 outputs equal the oracle's."""
     import post_quantized_linear_b200 as pq
     c = Case(W.small_case(M, K, N, seed=900 + M + K // 128, out=out))
     qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
     res = {}
     for split in ("1", "0"):
         monkeypatch.setenv("SEGQUANT_CSPLIT", split)
-        for bn in ("32", "64", "128"):
+        for bn in ("32", "64", "128", "0"):
             monkeypatch.setenv("SEGQUANT_BN_SMALL", bn)
             res[(split, bn)] = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b,
                                                     out_dtype=c.out_dtype)
