@@ -1040,23 +1040,26 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // handshakes (xfull: the q- warps wrote; xempty: the q+ warps have read).  The
 // fold is fold8_exact's and the store epilogue_tma_store's, so the outputs are
 // those of the two-tile form.
-// CSPLIT (P = 16, the tile's K range split over the CTAs of a cluster): a CTA
-// of rank r > 0 writes its raw accumulators (lanes 0..31, the tile's columns)
-// into its own [32][BN] int32 buffer (`part`, zeroed at setup; lane l's column
-// c at l*BN + c with the low five bits of c XOR l), then one bulk reduction adds
-// that buffer into the rank-0 CTA's, counted as bytes on rank 0's `parts`
-// barrier; rank 0 waits for every byte (bounded), adds the buffer to its own
-// accumulators -- integer sums, exact in any order -- and folds and stores as
-// above.  (The buffers stay alive until rank 0 has seen every byte: the CTAs
-// leave through a cluster barrier after the epilogue.)
+// CSPLIT (the tile's K range split over the CTAs of a cluster): in a CTA of
+// rank r > 0 every warp holding accumulator lanes (TMEM lanes 0 .. 2P) writes
+// its raw accumulators into its 32-lane slice of this CTA's [2P][BN] int32
+// buffer (`part`, zeroed at setup; lane l of lane quarter q, column c, at
+// (32q + l)*BN + c with the low five bits of c XOR l), then adds the slice into
+// the rank-0 CTA's by one bulk reduction, counted as bytes on rank 0's `parts`
+// barrier; rank 0's warps wait for every byte (bounded), add their slices to
+// their own accumulators -- integer sums, exact in any order -- and exchange,
+// fold and store as above.  (The buffers stay alive until rank 0 has seen every
+// byte: the CTAs leave through a cluster barrier after the epilogue.)
 template <int BN, int NBUF, bool Y_BF16, bool XCH, bool CSPLIT = false, class TileFn>
 __device__ __forceinline__ void epilogue_stacked(
     const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, uint32_t* xch, int quad,
     int lane, uint32_t t_lane, uint64_t* tmem_full, uint32_t empty_base, uint32_t xfull,
     uint32_t xempty, int rounds, TileFn tile_fn, volatile int* abort_flag, long long budget,
     uint32_t crank = 0, uint32_t part = 0, uint32_t parts_bar = 0) {
-  static_assert(!CSPLIT || !XCH, "K split: P = 16");
-  auto pidx = [&](int c) { return (uint32_t)(lane * BN + ((c & ~31) | ((c & 31) ^ lane))); };
+  // K split: this warp's 32 lanes of the [2P][BN] partial-sum buffer
+  auto pidx = [&](int c) {
+    return (uint32_t)((quad * 32 + lane) * BN + ((c & ~31) | ((c & 31) ^ lane)));
+  };
   const uint32_t part0 = CSPLIT ? mapa_shared(part, 0) : 0u;   // rank 0's buffer
   bool parts_in = false;
   constexpr int ROWB = Y_BF16 ? 64 : 128;
@@ -1104,8 +1107,11 @@ __device__ __forceinline__ void epilogue_stacked(
           if (p == npass - 1) {
             fence_proxy_async_smem();   // the bulk copy reads through the async proxy
             __syncwarp();
-            if (lane == 0)
-              bulk_reduce_add_u32_cluster(part0, part, 32u * BN * 4u, mapa_shared(parts_bar, 0));
+            if (lane == 0) {
+              const uint32_t slice = (uint32_t)quad * 32u * BN * 4u;
+              bulk_reduce_add_u32_cluster(part0 + slice, part + slice, 32u * BN * 4u,
+                                          mapa_shared(parts_bar, 0));
+            }
           }
           continue;
         }

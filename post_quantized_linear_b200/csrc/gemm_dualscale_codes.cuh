@@ -87,10 +87,10 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 // form are issued.  The A area of a k block is 2 * STK_ rows; the MMA still
 // reads 128 rows from its start (the rows past 2P belong to the weight tile or
 // the next k block and land in accumulator lanes nobody reads).
-// CSPLIT_ (stacked rows, P = 16): the K range of an N tile is split over the
-// CTAs of a cluster; the first CTA keeps a [32][BN] int32 buffer in shared
-// memory into which the others add their accumulators (one bulk reduction
-// each).  One tile per CTA: one TMEM buffer.
+// CSPLIT_ (stacked rows): the K range of an N tile is split over the CTAs of
+// a cluster; the first CTA keeps a [2P][BN] int32 buffer in shared memory into
+// which the others add their accumulators (one bulk reduction per warp holding
+// accumulator lanes).  One tile per CTA: one TMEM buffer.
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
           bool LDA_ = false, int KPS_ = 1, int WM_ = 0, int STK_ = 0, bool CSPLIT_ = false>
 struct CodesCfg {
@@ -121,10 +121,10 @@ struct CodesCfg {
   // memory and 256 TMEM columns let a CTA of the next GEMM in the stream share
   // the SM and prefetch its weights while this one finishes
   static constexpr int S_CAP = STK_ ? 3 : 8;
-  static constexpr int PART_BYTES = CSPLIT_ ? 32 * BN_ * 4 : 0;
+  static constexpr int PART_BYTES = CSPLIT_ ? 2 * STK_ * BN_ * 4 : 0;   // [2P][BN] int32
   static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) < S_CAP
                                ? ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) : S_CAP;
-  static_assert(!CSPLIT_ || STK_ == 16, "K split over a cluster: stacked rows with P = 16");
+  static_assert(!CSPLIT_ || STK_ != 0, "K split over a cluster: stacked rows");
   static_assert(STK_ == 0 || ((STK_ == 16 || STK_ == 32 || STK_ == 64) && !MULTI && !SINGLE &&
                               !LDA_ && WM_ == 0 && EPW_ == 4),
                 "stacked polarities: DualScale, one unit, four epilogue warps");
@@ -209,7 +209,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     // K split, first CTA: the others' partial sums arrive as bytes on `parts`
     if constexpr (CSPLIT)
       if (cluster_ctarank() == 0)
-        mbar_arrive_expect_tx(smem_u32(parts), (uint32_t)((args.splits - 1) * C::PART_BYTES));
+        mbar_arrive_expect_tx(smem_u32(parts),
+                              (uint32_t)((args.splits - 1) * 2 * args.a_rows * BN * 4));
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);

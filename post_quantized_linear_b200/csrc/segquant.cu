@@ -310,7 +310,7 @@ int codes_kps() { return dev_switch("SEGQUANT_KPS", 2) == 2 ? 2 : 1; }
 // tile (one MMA per k step); SEGQUANT_STACK=0 selects two 128-row code tiles.
 bool use_stacked() { return dev_switch("SEGQUANT_STACK", 1) != 0; }
 
-// Whether a stacked row tile of M <= 16 with few N tiles splits the K range of
+// Whether a stacked row tile (M <= 64) with few N tiles splits the K range of
 // each tile over a cluster of CTAs; SEGQUANT_CSPLIT=0 keeps one CTA per tile.
 bool use_cluster_split() { return dev_switch("SEGQUANT_CSPLIT", 1) != 0; }
 
@@ -423,25 +423,29 @@ sq_status launch_codes_stacked(int stk, bool y_bf16, const CUtensorMap& tqp, con
                 : launch_codes<BN, false, false, false, 4, false, 2, 0, 64>(tqp, tqn, tw, ty, a, stream);
 }
 
-// Stacked rows (M <= 16) with each N tile's k blocks shared by the a.splits
-// CTAs of a cluster.
+// Stacked rows (stk = 16: M <= 16; 64: 16 < M <= 64) with each N tile's k
+// blocks shared by the a.splits CTAs of a cluster.
 template <int BN>
-sq_status launch_codes_split(bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+sq_status launch_codes_split(int stk, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
                              const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
                              cudaStream_t stream) {
+  if (stk == 16)
+    return y_bf16
+               ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream)
+               : launch_codes<BN, false, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream);
   return y_bf16
-             ? launch_codes<BN, true, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream)
-             : launch_codes<BN, false, false, false, 4, false, 2, 0, 16, true>(tqp, tqn, tw, ty, a, stream);
+             ? launch_codes<BN, true, false, false, 4, false, 2, 0, 64, true>(tqp, tqn, tw, ty, a, stream)
+             : launch_codes<BN, false, false, false, 4, false, 2, 0, 64, true>(tqp, tqn, tw, ty, a, stream);
 }
 
-sq_status launch_codes_small_split(int bn, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
-                                   const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
-                                   cudaStream_t stream) {
+sq_status launch_codes_small_split(int bn, int stk, bool y_bf16, const CUtensorMap& tqp,
+                                   const CUtensorMap& tqn, const CUtensorMap& tw,
+                                   const CUtensorMap& ty, const sq::GemmArgs& a, cudaStream_t stream) {
   switch (bn) {
-    case 32: return launch_codes_split<32>(y_bf16, tqp, tqn, tw, ty, a, stream);
-    case 64: return launch_codes_split<64>(y_bf16, tqp, tqn, tw, ty, a, stream);
-    case 96: return launch_codes_split<96>(y_bf16, tqp, tqn, tw, ty, a, stream);
-    default: return launch_codes_split<128>(y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 32: return launch_codes_split<32>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 64: return launch_codes_split<64>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+    case 96: return launch_codes_split<96>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
+    default: return launch_codes_split<128>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
   }
 }
 
@@ -484,7 +488,7 @@ int max_clusters(int cs) {
   return n;
 }
 
-// M <= 16 rows (stacked): the tile width and the cluster size that shares each
+// Stacked rows (M <= 64): the tile width and the cluster size that shares each
 // N tile's k blocks.  The time of such a layer follows the number of k blocks
 // a CTA streams (the stages in flight cover a fixed HBM latency each), not
 // the tile width: the narrow tile `bn0` split over as many CTAs (2..8, at least
@@ -935,10 +939,10 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   const bool codes_kernel = (src == ASource::Single) || codes_ring || codes_w4 || had;
   // M <= 64 rows of q+ and q- stacked in one A tile (P = 16, 32 or 64 rows each)
   const bool stacked = bn_small && src == ASource::Codes && M <= 64 && use_stacked();
-  // M <= 16: each N tile's k blocks shared by a cluster of split_cs CTAs,
-  // on a tile width chosen for it
+  // each N tile's k blocks shared by a cluster of split_cs CTAs, on a tile
+  // width chosen for it
   int split_cs = 1;
-  if (stacked && M <= 16 && use_cluster_split()) {
+  if (stacked && use_cluster_split()) {
     int sbn = bn_small;
     choose_small_split(N, (int)((K + sq::BK - 1) / sq::BK), bn_small, bn_small_forced(), sbn, split_cs);
     if (split_cs > 1) {
@@ -1061,7 +1065,8 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       if (stacked) {
         if (split_cs > 1) {   // CTA r of a cluster: k blocks [r*kb/cs, (r+1)*kb/cs)
           a.splits = split_cs;
-          return launch_codes_small_split(bn_small, yb, ta, ta2, tw, ty, a, stream);
+          return launch_codes_small_split(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
+                                          stream);
         }
         return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
                                           stream);
