@@ -39,9 +39,19 @@ def _dtype_code(t: torch.dtype) -> int:
     raise TypeError(f"unsupported dtype {t}: float32 or bfloat16")
 
 
+# the current stream's raw handle without building a Stream object (a few
+# microseconds per call at small M); the public call where it is missing
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream: Optional[torch.cuda.Stream]):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    """The given stream, else the current stream of the current device (the
+    device the library launches on)."""
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(torch.cuda.current_device()))
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -71,11 +81,19 @@ class QuantizedWeight:
         return 0 if self.bits == 8 else 128
 
     def c_struct(self):
+        """The C view (sq_qweight) of this weight, rebuilt only when a field
+        it is made of has changed."""
+        key = (self.bits, self.N, self.K, tuple(self.kseg), tuple(self.nseg),
+               self.codes.data_ptr(), self.scales.data_ptr())
+        cached = self.__dict__.get("_c_struct")
+        if cached is not None and cached[0] == key:
+            return cached[1], cached[2]
         ks, ka = _lib.segments(self.kseg)
         ns, na = _lib.segments(self.nseg)
         qw = _lib.SqQWeight(self.bits, self.group, self.N, self.K, ks, ns,
                             ctypes.c_void_p(self.codes.data_ptr()),
                             ctypes.c_void_p(self.scales.data_ptr()))
+        self.__dict__["_c_struct"] = (key, qw, (ka, na))
         return qw, (ka, na)
 
 
