@@ -1039,7 +1039,8 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // q + P/32 to quarter q), 32 columns at a time, with bounded mbarrier
 // handshakes (xfull: the q- warps wrote; xempty: the q+ warps have read).  The
 // fold is fold8_exact's and the store epilogue_tma_store's, so the outputs are
-// those of the two-tile form.
+// those of the two-tile form.  `stage_y`: the four epilogue warps' staging
+// tiles, which the storing warps share out among themselves.
 // CSPLIT (the tile's K range split over the CTAs of a cluster): in a CTA of
 // rank r > 0 every warp holding accumulator lanes (TMEM lanes 0 .. 2P) writes
 // its raw accumulators into its 32-lane slice of this CTA's [2P][BN] int32
@@ -1063,9 +1064,14 @@ __device__ __forceinline__ void epilogue_stacked(
   const uint32_t part0 = CSPLIT ? mapa_shared(part, 0) : 0u;   // rank 0's buffer
   bool parts_in = false;
   constexpr int ROWB = Y_BF16 ? 64 : 128;
-  uint8_t* srow = stage_y + lane * ROWB;
-  const uint32_t sbase = smem_u32(stage_y);
+  constexpr int SYB = stage_y_bytes(Y_BF16);                    // one 32 x 32 staging tile
   const int qparts = args.a_rows / 32;                          // 0 when P = 16
+  // The warps that fold and store (lane quarters 0 .. nstore-1) take turns
+  // over all four epilogue warps' staging tiles, nb each, so a pass seldom
+  // waits for an earlier store to have read its tile.
+  const int nstore = (XCH && qparts > 1) ? qparts : 1;
+  const int nb = 4 / nstore;
+  int sp_count = 0;                                             // stores issued
   const bool pos_warp = XCH ? (quad < qparts) : (quad == 0);    // folds and stores
   const bool neg_warp = XCH && quad >= qparts && quad < 2 * qparts;   // hands q- over
   auto release = [&](int b) {
@@ -1076,10 +1082,16 @@ __device__ __forceinline__ void epilogue_stacked(
   float sp, sn;
   unit_act_scales(args, 0, sp, sn);
   int ug = 0, xu = 0;
-  bool ok = true, pending = false;
+  bool ok = true;
   for (int it = 0; it < rounds && ok; ++it) {
     Tile t;
     if (!tile_fn(it, t)) continue;
+    // the tile's weight scales and bias into L1 while its MMAs run (a pass
+    // would otherwise wait for them from HBM after the last MMA)
+    if (pos_warp && lane * 32 < t.width) {
+      prefetch_l1(static_cast<const float*>(args.wscales) + t.n0 + lane * 32);
+      if (args.bias != nullptr) prefetch_l1(args.bias + t.n0 + lane * 32);
+    }
     const int b = ug % NBUF;
     if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
     tc_fence_after();
@@ -1126,11 +1138,21 @@ __device__ __forceinline__ void epilogue_stacked(
           for (int k = 0; k < 8; ++k) v[i][k] += pb[pidx(col + 8 * i + k)];
       }
       uint32_t vn[4][8];
+      // P = 16: lane l folds row l & 15, columns 16 * (l >> 4) .. +16 of the
+      // pass: the q- values of the first 16 columns go down to lanes 0-15 and
+      // the q+ values of the last 16 up to lanes 16-31 (one exchange), and
+      // each lane's (q+, q-) pair is picked without branching
+      const bool hi = lane >= 16;
+      uint32_t fp[2][8], fn[2][8];
       if constexpr (!XCH) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 2; ++i)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) vn[i][k] = __shfl_down_sync(0xffffffffu, v[i][k], 16);
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t x = __shfl_xor_sync(0xffffffffu, hi ? v[i][k] : v[2 + i][k], 16);
+            fp[i][k] = hi ? x : v[i][k];
+            fn[i][k] = hi ? v[2 + i][k] : x;
+          }
       } else {
         const int xrow = (neg_warp ? quad - qparts : quad) * 32 + lane;
         uint32_t* xr = xch + xrow * 32;
@@ -1155,12 +1177,19 @@ __device__ __forceinline__ void epilogue_stacked(
         ++xu;
       }
       // q+ warps: fold, stage and store rows quad*32 .. +31, columns col .. +31
-      if (pending) {   // the previous store has read the staging tile
-        if (lane == 0) bulk_wait_read_all();
+      // into staging tile (quad * nb + sp_count % nb), once the store that last
+      // used it has read it
+      uint8_t* stile = stage_y + (quad * nb + sp_count % nb) * SYB;
+      const uint32_t sbase = smem_u32(stile);
+      if (sp_count >= nb) {
+        if (lane == 0) {
+          if (nb == 4) bulk_wait_read<3>();
+          else bulk_wait_read<1>();
+        }
         __syncwarp();
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      if constexpr (!XCH) {
+        const int h = hi ? 1 : 0, r = lane & 15;
         const int cc = col + 16 * h;
         if (cc < t.width) {
           float o[16];
@@ -1168,10 +1197,27 @@ __device__ __forceinline__ void epilogue_stacked(
           for (int i = 0; i < 16; ++i) o[i] = 0.0f;
           float sw[8];
           load_wscales8(args, 0, 0, t.n0 + cc, sw);
-          fold8_exact(v[2 * h], vn[2 * h], sw, sp, sn, o);
+          fold8_exact(fp[0], fn[0], sw, sp, sn, o);
           load_wscales8(args, 0, 0, t.n0 + cc + 8, sw);
-          fold8_exact(v[2 * h + 1], vn[2 * h + 1], sw, sp, sn, o + 8);
-          stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+          fold8_exact(fp[1], fn[1], sw, sp, sn, o + 8);
+          stage16<Y_BF16>(args, t.n0 + cc, o, stile + r * ROWB, r, h);
+        }
+      } else {
+        uint8_t* srow = stile + lane * ROWB;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int cc = col + 16 * h;
+          if (cc < t.width) {
+            float o[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+            float sw[8];
+            load_wscales8(args, 0, 0, t.n0 + cc, sw);
+            fold8_exact(v[2 * h], vn[2 * h], sw, sp, sn, o);
+            load_wscales8(args, 0, 0, t.n0 + cc + 8, sw);
+            fold8_exact(v[2 * h + 1], vn[2 * h + 1], sw, sp, sn, o + 8);
+            stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -1180,7 +1226,7 @@ __device__ __forceinline__ void epilogue_stacked(
         tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
         bulk_commit_group();
       }
-      pending = true;
+      ++sp_count;
     }
   }
   // Every store has completed before the CTA (and its shared memory) exits.

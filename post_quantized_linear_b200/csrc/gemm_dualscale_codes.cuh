@@ -458,9 +458,9 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     const int part = (warp - EPI0) >> 2;
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
     if constexpr (STK != 0) {
-      uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
+      static_assert(!STK || C::Y_BYTES == 4 * stage_y_bytes(Y_BF16), "four staging tiles");
       epilogue_stacked<BN, C::NBUF, Y_BF16, (STK > 16), CSPLIT>(
-          args, &tmap_y, stage_y, reinterpret_cast<uint32_t*>(smem + C::OFF_SW), quad, lane, t_lane,
+          args, &tmap_y, smem + C::OFF_Y, reinterpret_cast<uint32_t*>(smem + C::OFF_SW), quad, lane, t_lane,
           tmem_full, smem_u32(tmem_empty), smem_u32(xfull), smem_u32(xempty), rounds, tiles,
           abort_flag, budget, crank, smem_u32(smem + C::OFF_PART), smem_u32(parts));
     } else if constexpr (SEEDED) {
