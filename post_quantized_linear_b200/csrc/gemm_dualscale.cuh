@@ -1101,14 +1101,38 @@ __device__ __forceinline__ void epilogue_stacked(
       continue;
     }
     const int npass = (t.width + 31) / 32;
-    for (int p = 0; p < npass; ++p) {
-      const int col = 32 * p;
-      const uint32_t tcol = (uint32_t)b * BN + (uint32_t)col;
-      uint32_t v[4][8];
+    static_assert(BN % 32 == 0, "32-column passes");
+    constexpr int NPM = BN / 32;
+    // P = 16: every column of the tile into registers at once (one TMEM round
+    // trip instead of one per pass), and the buffer released before the passes
+    uint32_t va[XCH ? 1 : NPM][4][8];
+    if constexpr (!XCH) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld8(t_lane + tcol + 8 * i, v[i]);
+      for (int p = 0; p < NPM; ++p)
+        if (p < npass)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            tmem_ld8(t_lane + (uint32_t)b * BN + (uint32_t)(32 * p + 8 * i), va[p][i]);
       tmem_wait_ld();
-      if (p == npass - 1) release(b);   // every column of the tile is in registers
+      release(b);
+    }
+#pragma unroll
+    for (int p = 0; p < NPM; ++p) {
+      if (p >= npass) break;
+      const int col = 32 * p;
+      uint32_t v[4][8];
+      if constexpr (!XCH) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[i][k] = va[p][i][k];
+      } else {
+        const uint32_t tcol = (uint32_t)b * BN + (uint32_t)col;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_ld8(t_lane + tcol + 8 * i, v[i]);
+        tmem_wait_ld();
+        if (p == npass - 1) release(b);   // every column of the tile is in registers
+      }
       if constexpr (CSPLIT) {
         if (crank != 0) {   // into this CTA's buffer, then added into rank 0's
           uint32_t* own = reinterpret_cast<uint32_t*>(__cvta_shared_to_generic(part));
