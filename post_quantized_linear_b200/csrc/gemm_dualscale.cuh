@@ -1115,6 +1115,12 @@ __device__ __forceinline__ void epilogue_stacked(
             tmem_ld8(t_lane + (uint32_t)b * BN + (uint32_t)(32 * p + 8 * i), va[p][i]);
       tmem_wait_ld();
       release(b);
+      // P = 16: pass p stages into tile p (at most four passes, four tiles),
+      // all stored together after the last pass
+      if (sp_count > 0) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
     }
 #pragma unroll
     for (int p = 0; p < NPM; ++p) {
@@ -1203,9 +1209,9 @@ __device__ __forceinline__ void epilogue_stacked(
       // q+ warps: fold, stage and store rows quad*32 .. +31, columns col .. +31
       // into staging tile (quad * nb + sp_count % nb), once the store that last
       // used it has read it
-      uint8_t* stile = stage_y + (quad * nb + sp_count % nb) * SYB;
+      uint8_t* stile = stage_y + (XCH ? (quad * nb + sp_count % nb) : p) * SYB;
       const uint32_t sbase = smem_u32(stile);
-      if (sp_count >= nb) {
+      if (XCH && sp_count >= nb) {
         if (lane == 0) {
           if (nb == 4) bulk_wait_read<3>();
           else bulk_wait_read<1>();
@@ -1244,13 +1250,27 @@ __device__ __forceinline__ void epilogue_stacked(
           }
         }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
-        bulk_commit_group();
+      if constexpr (XCH) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+          bulk_commit_group();
+        }
+        ++sp_count;
       }
-      ++sp_count;
+    }
+    if constexpr (!XCH) {   // the tile's passes, stored together
+      if (ok && (CSPLIT ? crank == 0 : true)) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int p = 0; p < npass; ++p)
+            tma_store_2d(tmap_y, smem_u32(stage_y + p * SYB), t.n0 + 32 * p, t.m0 + quad * 32);
+          bulk_commit_group();
+        }
+        sp_count += npass;
+      }
     }
   }
   // Every store has completed before the CTA (and its shared memory) exits.
