@@ -872,14 +872,29 @@ __device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float&
 // the full barriers are signalled by the leader's commits (cluster-scope
 // acquire), and `empty_base` may be a cluster address of the leader's
 // barriers (empty_remote).
+// CSPLIT (one unit, two accumulators, four warps: the small-M two-tile form
+// with the tile's k blocks split over the CTAs of a cluster): a CTA of rank
+// r > 0 writes its raw accumulators into its own [2][128][BN] int32 buffer
+// (`part`; accumulator a, lane quarter q, lane l, column c at
+// ((128a + 32q + l) * BN + c) with the low five bits of c XOR l) and adds each
+// warp's two 32-lane slices into the rank-0 CTA's buffer by bulk reductions
+// counted on its `parts` barrier; rank 0 adds the buffer to its accumulators
+// (integer sums, any order) before folding.
 template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn,
-          bool PAIR = false>
+          bool PAIR = false, bool CSPLIT = false>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
                                                    uint32_t empty_base, int rounds, TileFn tile_fn,
                                                    volatile int* abort_flag, long long budget,
-                                                   int row_shift = 0, bool empty_remote = false) {
+                                                   int row_shift = 0, bool empty_remote = false,
+                                                   uint32_t crank = 0, uint32_t part_buf = 0,
+                                                   uint32_t parts_bar = 0) {
+  static_assert(!CSPLIT || (!MULTI && NACC == 2 && EPW == 4 && !PAIR), "K split: two-tile form");
+  auto pidx = [&](int a, int c) {
+    return (uint32_t)(((128 * a + quad * 32 + lane) * BN) + ((c & ~31) | ((c & 31) ^ lane)));
+  };
+  bool parts_in = false;
   constexpr int HALF = BN / (EPW / 4);
   constexpr int ROWB = Y_BF16 ? 64 : 128;
   constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
@@ -1004,12 +1019,54 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
             load8(b, cc + 8, bp, bn);
             tmem_wait_ld();
             if (p == npass - 1 && (h == 1 || cc + 16 >= t.width)) release(b);   // last loads
+            if constexpr (CSPLIT) {
+              uint32_t* pb = reinterpret_cast<uint32_t*>(__cvta_shared_to_generic(part_buf));
+              if (crank != 0) {   // into this CTA's buffer; rank 0 folds
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  pb[pidx(0, cc + k)] = ap[k];
+                  pb[pidx(1, cc + k)] = an[k];
+                  pb[pidx(0, cc + 8 + k)] = bp[k];
+                  pb[pidx(1, cc + 8 + k)] = bn[k];
+                }
+                continue;
+              }
+              if (!parts_in) {   // the other CTAs' partial sums have landed
+                if (!(ok = wait_warp<true>(parts_bar, 0, abort_flag, budget))) break;
+                parts_in = true;
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                ap[k] += pb[pidx(0, cc + k)];
+                an[k] += pb[pidx(1, cc + k)];
+                bp[k] += pb[pidx(0, cc + 8 + k)];
+                bn[k] += pb[pidx(1, cc + 8 + k)];
+              }
+            }
             float o[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) o[i] = 0.0f;
             fold8c(ap, an, 0, t.n0 + cc, sp, sn, o);
             fold8c(bp, bn, 0, t.n0 + cc + 8, sp, sn, o + 8);
             stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
+          }
+        }
+        if (!ok) break;
+        if constexpr (CSPLIT) {
+          if (crank != 0) {   // after the last pass: this warp's two slices into rank 0's buffer
+            if (p == npass - 1) {
+              fence_proxy_async_smem();   // the bulk copy reads through the async proxy
+              __syncwarp();
+              if (lane == 0) {
+                const uint32_t part0 = mapa_shared(part_buf, 0), bar0 = mapa_shared(parts_bar, 0);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                  const uint32_t off = (uint32_t)((128 * a + quad * 32) * BN * 4);
+                  bulk_reduce_add_u32_cluster(part0 + off, part_buf + off, 32u * BN * 4u, bar0);
+                }
+              }
+            }
+            continue;
           }
         }
         fence_proxy_async_smem();

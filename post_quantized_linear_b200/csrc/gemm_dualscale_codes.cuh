@@ -121,10 +121,12 @@ struct CodesCfg {
   // memory and 256 TMEM columns let a CTA of the next GEMM in the stream share
   // the SM and prefetch its weights while this one finishes
   static constexpr int S_CAP = STK_ ? 3 : 8;
-  static constexpr int PART_BYTES = CSPLIT_ ? 2 * STK_ * BN_ * 4 : 0;   // [2P][BN] int32
+  // K split: [2P][BN] int32 (stacked) or [2][128][BN] (two-tile form)
+  static constexpr int PART_BYTES = CSPLIT_ ? (STK_ ? 2 * STK_ : 2 * BM) * BN_ * 4 : 0;
   static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) < S_CAP
                                ? ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) : S_CAP;
-  static_assert(!CSPLIT_ || STK_ != 0, "K split over a cluster: stacked rows");
+  static_assert(!CSPLIT_ || STK_ != 0 || (!MULTI && !SINGLE && !LDA_ && WM_ == 0 && EPW_ == 4),
+                "K split over a cluster: stacked rows, or the two-tile form with four warps");
   static_assert(STK_ == 0 || ((STK_ == 16 || STK_ == 32 || STK_ == 64) && !MULTI && !SINGLE &&
                               !LDA_ && WM_ == 0 && EPW_ == 4),
                 "stacked polarities: DualScale, one unit, four epilogue warps");
@@ -209,8 +211,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     // K split, first CTA: the others' partial sums arrive as bytes on `parts`
     if constexpr (CSPLIT)
       if (cluster_ctarank() == 0)
-        mbar_arrive_expect_tx(smem_u32(parts),
-                              (uint32_t)((args.splits - 1) * 2 * args.a_rows * BN * 4));
+        mbar_arrive_expect_tx(smem_u32(parts), (uint32_t)((args.splits - 1) *
+                                                          (STK ? 2 * args.a_rows : 2 * BM) * BN * 4));
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
@@ -471,9 +473,9 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
           smem_u32(tmem_empty), rounds, tiles, abort_flag, budget);
     } else if constexpr (C::TMA_Y) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16>(
+      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, decltype(tiles), false, CSPLIT>(
           args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
-          tiles, abort_flag, budget);
+          tiles, abort_flag, budget, 0, false, crank, smem_u32(smem + C::OFF_PART), smem_u32(parts));
     } else {
       // no room for staging tiles: 16-byte stores straight from registers (DualScale, one unit)
       epilogue_role<BN, C::NBUF, false, false, Y_BF16, false>(

@@ -310,7 +310,7 @@ int codes_kps() { return dev_switch("SEGQUANT_KPS", 2) == 2 ? 2 : 1; }
 // tile (one MMA per k step); SEGQUANT_STACK=0 selects two 128-row code tiles.
 bool use_stacked() { return dev_switch("SEGQUANT_STACK", 1) != 0; }
 
-// Whether a stacked row tile (M <= 64) with few N tiles splits the K range of
+// Whether a small-M row tile with few N tiles splits the K range of
 // each tile over a cluster of CTAs; SEGQUANT_CSPLIT=0 keeps one CTA per tile.
 bool use_cluster_split() { return dev_switch("SEGQUANT_CSPLIT", 1) != 0; }
 
@@ -318,10 +318,11 @@ template <int BN, bool YB, bool MULTI, bool SINGLE, int EPW = sq::epi_warps(MULT
           int KPS = 1, int WM = 0, int STK = 0, bool CSPLIT = false>
 sq_status launch_codes(const CUtensorMap& tqp, const CUtensorMap& tqn, const CUtensorMap& tw,
                        const CUtensorMap& ty, sq::GemmArgs a, cudaStream_t stream) {
-  if constexpr (kDev && !LDA && KPS == 1 && WM == 0 && STK == 0 && !(MULTI && BN > 128)) {
+  if constexpr (kDev && !LDA && KPS == 1 && WM == 0 && STK == 0 && !CSPLIT && !(MULTI && BN > 128)) {
     if (use_codes_lda()) return launch_codes<BN, YB, MULTI, SINGLE, EPW, true>(tqp, tqn, tw, ty, a, stream);
   }
-  if constexpr (!LDA && KPS == 1 && WM == 0 && STK == 0 && BN <= 192 &&
+  // (not for a K split: its partial sums take the room of the second k block)
+  if constexpr (!LDA && KPS == 1 && WM == 0 && STK == 0 && !CSPLIT && BN <= 192 &&
                 sq::codes_kps2_fits(BN, MULTI, YB, SINGLE, EPW)) {
     if (codes_kps() == 2)
       return launch_codes<BN, YB, MULTI, SINGLE, EPW, false, 2>(tqp, tqn, tw, ty, a, stream);
@@ -488,25 +489,29 @@ int max_clusters(int cs) {
   return n;
 }
 
-// Stacked rows (M <= 64): the tile width and the cluster size that shares each
+// Small M (one row tile): the tile width and the cluster size that shares each
 // N tile's k blocks.  The time of such a layer follows the number of k blocks
 // a CTA streams (the stages in flight cover a fixed HBM latency each), not
 // the tile width: the narrow tile `bn0` split over as many CTAs (2..8, at least
-// two k blocks apiece, clusters the device runs at once) as the SMs hold;
+// min_kb k blocks apiece, clusters the device runs at once) as the SMs hold;
 // when bn0 cannot be split and its tiles leave a fifth of the SMs idle, the
-// tile of twice its width split in two or more.  `forced`: keep bn0.
-void choose_small_split(int64_t N, int num_kb, int bn0, bool forced, int& bn, int& cs) {
+// tile of twice its width split in two or more (up to max_bn: the two-tile
+// form's partial sums fit beside two stages up to 96 columns).  `forced`: keep bn0.
+void choose_small_split(int64_t N, int num_kb, int bn0, bool forced, int max_bn, int min_kb, int& bn,
+                        int& cs) {
   const int sms = num_sms();
+  bn = bn0;
+  cs = 1;
+  if (bn0 > max_bn) return;
   auto split_of = [&](int b) {
     const int64_t tiles = (N + b - 1) / b;
     int c = 1;
     for (int k = 2; k <= 8; ++k)
-      if (tiles * k <= sms && num_kb >= 2 * k && tiles <= max_clusters(k)) c = k;
+      if (tiles * k <= sms && num_kb >= min_kb * k && tiles <= max_clusters(k)) c = k;
     return c;
   };
-  bn = bn0;
   cs = split_of(bn0);
-  if (forced || cs > 1 || bn0 * 2 > 128 || ((N + bn0 - 1) / bn0) * 5 >= (int64_t)sms * 4) return;
+  if (forced || cs > 1 || bn0 * 2 > max_bn || ((N + bn0 - 1) / bn0) * 5 >= (int64_t)sms * 4) return;
   const int c2 = split_of(bn0 * 2);
   if (c2 > 1) {
     bn = bn0 * 2;
@@ -524,6 +529,23 @@ sq_status launch_codes_small_stacked(int bn, int stk, bool y_bf16, const CUtenso
     case 96: return launch_codes_stacked<96>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
     default: return launch_codes_stacked<128>(stk, y_bf16, tqp, tqn, tw, ty, a, stream);
   }
+}
+
+// The two-tile form (16 < M <= 128, or M <= 64 without stacking) with each N
+// tile's k blocks shared by the a.splits CTAs of a cluster.
+sq_status launch_codes_small_split2(int bn, bool y_bf16, const CUtensorMap& tqp, const CUtensorMap& tqn,
+                                    const CUtensorMap& tw, const CUtensorMap& ty, const sq::GemmArgs& a,
+                                    cudaStream_t stream) {
+#define SQ_SPLIT2(B)                                                                                  \
+  return y_bf16 ? launch_codes<B, true, false, false, 4, false, 1, 0, 0, true>(tqp, tqn, tw, ty, a, stream) \
+                : launch_codes<B, false, false, false, 4, false, 1, 0, 0, true>(tqp, tqn, tw, ty, a, stream)
+  switch (bn) {   // (the [2][128][BN] partial sums leave room for two stages up to BN = 96)
+    case 32: SQ_SPLIT2(32);
+    case 64: SQ_SPLIT2(64);
+    case 96: SQ_SPLIT2(96);
+    default: return SQ_ERR_UNSUPPORTED;
+  }
+#undef SQ_SPLIT2
 }
 
 template <bool SINGLE>
@@ -942,9 +964,12 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   // each N tile's k blocks shared by a cluster of split_cs CTAs, on a tile
   // width chosen for it
   int split_cs = 1;
-  if (stacked && use_cluster_split()) {
+  if (bn_small && src == ASource::Codes && !pair && use_cluster_split()) {
     int sbn = bn_small;
-    choose_small_split(N, (int)((K + sq::BK - 1) / sq::BK), bn_small, bn_small_forced(), sbn, split_cs);
+    // (k blocks per CTA: at least 2 with 16 stacked rows, 5 otherwise -- below
+    // that the exchange of partial sums costs more than the split saves)
+    choose_small_split(N, (int)((K + sq::BK - 1) / sq::BK), bn_small, bn_small_forced(),
+                       stacked ? 128 : 96, (stacked && M <= 16) ? 2 : 5, sbn, split_cs);
     if (split_cs > 1) {
       bn_small = sbn;
       BN = sbn;
@@ -1070,6 +1095,10 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
         }
         return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
                                           stream);
+      }
+      if (bn_small && split_cs > 1) {   // two-tile form, k blocks shared by a cluster
+        a.splits = split_cs;
+        return launch_codes_small_split2(bn_small, yb, ta, ta2, tw, ty, a, stream);
       }
       if (bn_small) return launch_codes_small<false>(bn_small, yb, ta, ta2, tw, ty, a, stream);
       if (BN == 256 && codes_wide_epilogue())

@@ -72,14 +72,15 @@ def test_stacked_product_library_full_weight(M):
 
 
 @pytest.mark.parametrize("out", ["f32", "bf16"])
-@pytest.mark.parametrize("M", [1, 16, 17, 33, 64])
+@pytest.mark.parametrize("M", [1, 16, 17, 33, 64, 65, 100, 128])
 @pytest.mark.parametrize("K,N", [(1152, 1152), (4608, 1152), (1152, 400), (3072, 2048),
                                  (3072, 12288)])
 def test_k_split_over_a_cluster(K, N, M, out, monkeypatch, dev_lib):
-    """M <= 64: each N tile's k blocks are shared evenly by the CTAs of a
-    cluster (2 to 8; 9 k blocks over 4 CTAs gives 2, 2, 2, 3), which add their
-    int32 accumulators (every warp its lanes of q+ and q- rows) into the first
-    CTA's shared memory before it exchanges and folds.
+    """One row tile (M <= 128): each N tile's k blocks are shared evenly by the
+    CTAs of a cluster (2 to 8; 9 k blocks over 4 CTAs gives 2, 2, 2, 3), which
+    add their int32 accumulators (every warp its lanes: of the stacked q+ and
+    q- rows at M <= 64, of both accumulators of the two-tile form above) into
+    the first CTA's shared memory before it folds.
     Integer sums, so the result is bit-identical to one CTA per tile (the
     development build's SEGQUANT_CSPLIT=0) at every tile width -- the widths
     fixed here and the library's own choice ("0": up to 256 columns) -- and
