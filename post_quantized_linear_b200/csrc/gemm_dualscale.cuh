@@ -1090,14 +1090,19 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // One row tile whose q+ and q- code rows were stacked in one A tile: the
 // accumulator of tile row r sits in TMEM lane r (q+ product) and lane P + r
 // (q- product), P = args.a_rows in {16, 32, 64}, one buffer of BN columns per
-// tile.  The warps that own lanes [0, P) fold and store rows [0, P); the q-
-// values reach them by a shuffle (P = 16: both halves in the first lane
-// quarter) or, XCH, through shared memory (P = 32, 64: from lane quarter
-// q + P/32 to quarter q), 32 columns at a time, with bounded mbarrier
-// handshakes (xfull: the q- warps wrote; xempty: the q+ warps have read).  The
-// fold is fold8_exact's and the store epilogue_tma_store's, so the outputs are
-// those of the two-tile form.  `stage_y`: the four epilogue warps' staging
-// tiles, which the storing warps share out among themselves.
+// tile.  The tile's weight scales and bias are prefetched into L1 while its
+// MMAs run.  P = 16 (both halves in the first lane quarter): that warp reads
+// the whole tile from TMEM at once; per 32-column pass one exchange of 16
+// values gives lane l the (q+, q-) pair of row l & 15, columns 16 * (l >> 4)
+// .. +16, so all 32 lanes fold; pass p stages into staging tile p and the
+// passes are stored together.  XCH (P = 32, 64): the warps owning lanes
+// [0, P) fold and store rows [0, P), the q- values reaching them through
+// shared memory (from lane quarter q + P/32 to quarter q), 32 columns at a
+// time, with bounded mbarrier handshakes (xfull: the q- warps wrote; xempty:
+// the q+ warps have read), each pass stored on its own, the storing warps
+// taking turns over the staging tiles.  The fold is fold8_exact's, so the
+// outputs are those of the two-tile form.  `stage_y`: the four epilogue
+// warps' staging tiles (32 x 32 outputs each).
 // CSPLIT (the tile's K range split over the CTAs of a cluster): in a CTA of
 // rank r > 0 every warp holding accumulator lanes (TMEM lanes 0 .. 2P) writes
 // its raw accumulators into its 32-lane slice of this CTA's [2P][BN] int32
@@ -1123,9 +1128,9 @@ __device__ __forceinline__ void epilogue_stacked(
   constexpr int ROWB = Y_BF16 ? 64 : 128;
   constexpr int SYB = stage_y_bytes(Y_BF16);                    // one 32 x 32 staging tile
   const int qparts = args.a_rows / 32;                          // 0 when P = 16
-  // The warps that fold and store (lane quarters 0 .. nstore-1) take turns
-  // over all four epilogue warps' staging tiles, nb each, so a pass seldom
-  // waits for an earlier store to have read its tile.
+  // XCH: the warps that fold and store (lane quarters 0 .. nstore-1) take
+  // turns over the four staging tiles, nb each, so a pass seldom waits for an
+  // earlier store to have read its tile.
   const int nstore = (XCH && qparts > 1) ? qparts : 1;
   const int nb = 4 / nstore;
   int sp_count = 0;                                             // stores issued
@@ -1263,9 +1268,9 @@ __device__ __forceinline__ void epilogue_stacked(
         if (lane == 0) mbar_arrive(xempty);
         ++xu;
       }
-      // q+ warps: fold, stage and store rows quad*32 .. +31, columns col .. +31
-      // into staging tile (quad * nb + sp_count % nb), once the store that last
-      // used it has read it
+      // q+ warps: fold and stage rows quad*32 .. +31, columns col .. +31 into
+      // staging tile p (P = 16) or (quad * nb + sp_count % nb) once the store
+      // that last used it has read it (XCH)
       uint8_t* stile = stage_y + (XCH ? (quad * nb + sp_count % nb) : p) * SYB;
       const uint32_t sbase = smem_u32(stile);
       if (XCH && sp_count >= nb) {
