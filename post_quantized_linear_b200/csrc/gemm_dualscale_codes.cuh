@@ -87,10 +87,12 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 // form are issued.  The A area of a k block is 2 * STK_ rows; the MMA still
 // reads 128 rows from its start (the rows past 2P belong to the weight tile or
 // the next k block and land in accumulator lanes nobody reads).
-// CSPLIT_ (stacked rows): the K range of an N tile is split over the CTAs of
-// a cluster; the first CTA keeps a [2P][BN] int32 buffer in shared memory into
-// which the others add their accumulators (one bulk reduction per warp holding
-// accumulator lanes).  One tile per CTA: one TMEM buffer.
+// CSPLIT_ (one row tile: stacked rows, or the two-tile form with four
+// epilogue warps): the K range of an N tile is split over the CTAs of a
+// cluster; the first CTA keeps an int32 buffer in shared memory -- [2P][BN]
+// stacked, [2][128][BN] two-tile -- into which the others add their
+// accumulators (bulk reductions by every warp holding accumulator lanes).
+// One tile per CTA: one TMEM buffer.
 template <int BN_, bool MULTI, bool Y_BF16, bool SINGLE, int EPW_ = epi_warps(MULTI),
           bool LDA_ = false, int KPS_ = 1, int WM_ = 0, int STK_ = 0, bool CSPLIT_ = false>
 struct CodesCfg {
