@@ -4,7 +4,8 @@ stream, but they must read their codes and scales, and write Y, only after
 that kernel has finished.  A chain of dependent calls issued back to back
 (eagerly and from one CUDA graph) gives the same bits as the same calls with
 a synchronisation between each; small-M layers (stacked rows, whose CTAs may
-share SMs with the previous GEMM's) and a large-M layer."""
+share SMs with the previous GEMM's, and layers whose k blocks are split over
+clusters) and a large-M layer."""
 import numpy as np
 import pytest
 import torch
@@ -52,10 +53,16 @@ def _chain(x, qws, sync: bool):
     return outs
 
 
-@pytest.mark.parametrize("M", [16, 48, 300])
-def test_dependent_layers_back_to_back(M):
+@pytest.mark.parametrize("M,dims", [(16, [1024, 1536, 512, 768]), (48, [1024, 1536, 512, 768]),
+                                    (300, [1024, 1536, 512, 768]),
+                                    # DiT-like widths: the 4608-deep layers split their
+                                    # k blocks over clusters at M = 16 (stacked rows),
+                                    # 40 (stacked, P = 64) and 100 (two-tile form)
+                                    (16, [4608, 1152, 4608, 1152]), (40, [4608, 1152, 4608, 1152]),
+                                    (100, [4608, 1152, 4608, 1152])])
+def test_dependent_layers_back_to_back(M, dims):
     import post_quantized_linear_b200 as pq
-    x, qws = _layers(M, [1024, 1536, 512, 768], seed=M)
+    x, qws = _layers(M, dims, seed=M)
     ref = [y.clone() for y in _chain(x, qws, sync=True)]
     for _ in range(3):
         got = _chain(x, qws, sync=False)
