@@ -97,6 +97,12 @@ struct GemmArgs {
   // past the box keep stale shared memory; their accumulator lanes are never
   // stored.
   int32_t a_rows;
+  // Stacked rows, M a multiple of 16: tmap_qp is a 4-D map (K bytes x 16 rows x
+  // {q+, q-} x groups of 16 rows) whose one box per k block lands every group's
+  // q+ and q- rows in the stacked order (1), or each group and polarity comes
+  // as its own 16-row box (0).
+  int32_t code_box4;
+  int32_t code_neg_first;   // (code_box4) the map starts at q-: each group's q- rows come first
 };
 
 // Teardown waits (copies and MMAs that were issued always complete) get a
@@ -1087,22 +1093,21 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 }
 
 // ------------------------------------- stacked-polarity epilogue (small M)
-// One row tile whose q+ and q- code rows were stacked in one A tile: the
-// accumulator of tile row r sits in TMEM lane r (q+ product) and lane P + r
-// (q- product), P = args.a_rows in {16, 32, 64}, one buffer of BN columns per
-// tile.  The tile's weight scales and bias are prefetched into L1 while its
-// MMAs run.  P = 16 (both halves in the first lane quarter): that warp reads
-// the whole tile from TMEM at once; per 32-column pass one exchange of 16
-// values gives lane l the (q+, q-) pair of row l & 15, columns 16 * (l >> 4)
-// .. +16, so all 32 lanes fold; pass p stages into staging tile p and the
-// passes are stored together.  XCH (P = 32, 64): the warps owning lanes
-// [0, P) fold and store rows [0, P), the q- values reaching them through
-// shared memory (from lane quarter q + P/32 to quarter q), 32 columns at a
-// time, with bounded mbarrier handshakes (xfull: the q- warps wrote; xempty:
-// the q+ warps have read), each pass stored on its own, the storing warps
-// taking turns over the staging tiles.  The fold is fold8_exact's, so the
-// outputs are those of the two-tile form.  `stage_y`: the four epilogue
-// warps' staging tiles (32 x 32 outputs each).
+// One row tile of P = args.a_rows rows (16, 32 or 64) whose codes were stacked
+// in one A tile in groups of 16 rows: group g's q+ rows in A rows 32g .. +15,
+// its q- rows in 32g + 16 .. +31.  The MMA therefore leaves the q+ product of
+// tile row 16g + r in TMEM lane 32g + r and the q- product in lane 32g + 16 + r:
+// epilogue warp g (lane quarter g, g < P/16) holds both halves of its 16 rows
+// (the q- rows first, lanes 32g .. +15, when the codes map starts at q-).
+// Each such warp prefetches the tile's weight scales and bias into L1 while
+// the MMAs run, reads the whole tile from TMEM at once (BN/32 passes of 32
+// columns in registers, one round trip) and releases it; per pass one exchange
+// of 16 values gives lane l the (q+, q-) pair of row 16g + (l & 15), columns
+// 16 * (l >> 4) .. +16, so all 32 lanes fold (fold8_exact: the outputs are
+// those of the two-tile form); the passes stage into the warp's share of the
+// eight 16-row staging tiles (`stage_y`: the four epilogue warps' 32 x 32
+// tiles, halved) and leave by TMA stores of 16-row boxes (`tmap_y`), a batch
+// at a time.
 // CSPLIT (the tile's K range split over the CTAs of a cluster): in a CTA of
 // rank r > 0 every warp holding accumulator lanes (TMEM lanes 0 .. 2P) writes
 // its raw accumulators into its 32-lane slice of this CTA's [2P][BN] int32
@@ -1110,32 +1115,33 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // (32q + l)*BN + c with the low five bits of c XOR l), then adds the slice into
 // the rank-0 CTA's by one bulk reduction, counted as bytes on rank 0's `parts`
 // barrier; rank 0's warps wait for every byte (bounded), add their slices to
-// their own accumulators -- integer sums, exact in any order -- and exchange,
-// fold and store as above.  (The buffers stay alive until rank 0 has seen every
-// byte: the CTAs leave through a cluster barrier after the epilogue.)
-template <int BN, int NBUF, bool Y_BF16, bool XCH, bool CSPLIT = false, class TileFn>
+// their own accumulators -- integer sums, exact in any order -- and fold and
+// store as above.  (The buffers stay alive until rank 0 has seen every byte:
+// the CTAs leave through a cluster barrier after the epilogue.)
+template <int BN, int NBUF, bool Y_BF16, bool CSPLIT = false, class TileFn>
 __device__ __forceinline__ void epilogue_stacked(
-    const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, uint32_t* xch, int quad,
-    int lane, uint32_t t_lane, uint64_t* tmem_full, uint32_t empty_base, uint32_t xfull,
-    uint32_t xempty, int rounds, TileFn tile_fn, volatile int* abort_flag, long long budget,
-    uint32_t crank = 0, uint32_t part = 0, uint32_t parts_bar = 0) {
+    const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, int quad, int lane,
+    uint32_t t_lane, uint64_t* tmem_full, uint32_t empty_base, int rounds, TileFn tile_fn,
+    volatile int* abort_flag, long long budget, uint32_t crank = 0, uint32_t part = 0,
+    uint32_t parts_bar = 0) {
+  static_assert(BN % 32 == 0 && BN <= 128, "32-column passes, at most four");
+  constexpr int NPM = BN / 32;
+  constexpr int ROWB = Y_BF16 ? 64 : 128;
+  constexpr int SUB = 16 * ROWB;                                // one 16-row staging tile
+  constexpr int NSUB = 4 * stage_y_bytes(Y_BF16) / SUB;         // eight
   // K split: this warp's 32 lanes of the [2P][BN] partial-sum buffer
   auto pidx = [&](int c) {
     return (uint32_t)((quad * 32 + lane) * BN + ((c & ~31) | ((c & 31) ^ lane)));
   };
   const uint32_t part0 = CSPLIT ? mapa_shared(part, 0) : 0u;   // rank 0's buffer
   bool parts_in = false;
-  constexpr int ROWB = Y_BF16 ? 64 : 128;
-  constexpr int SYB = stage_y_bytes(Y_BF16);                    // one 32 x 32 staging tile
-  const int qparts = args.a_rows / 32;                          // 0 when P = 16
-  // XCH: the warps that fold and store (lane quarters 0 .. nstore-1) take
-  // turns over the four staging tiles, nb each, so a pass seldom waits for an
-  // earlier store to have read its tile.
-  const int nstore = (XCH && qparts > 1) ? qparts : 1;
-  const int nb = 4 / nstore;
-  int sp_count = 0;                                             // stores issued
-  const bool pos_warp = XCH ? (quad < qparts) : (quad == 0);    // folds and stores
-  const bool neg_warp = XCH && quad >= qparts && quad < 2 * qparts;   // hands q- over
+  const int groups = args.a_rows / 16;                          // warps holding rows
+  const bool data_warp = quad < groups;
+  const int ns = NSUB / groups;                                 // staging tiles per warp
+  uint8_t* my_sub = stage_y + quad * ns * SUB;
+  const bool hi = lane >= 16;
+  const int r = lane & 15;                                      // row within the group
+  const bool neg_first = args.code_box4 && args.code_neg_first;
   auto release = [&](int b) {
     tc_fence_before();
     __syncwarp();
@@ -1143,14 +1149,14 @@ __device__ __forceinline__ void epilogue_stacked(
   };
   float sp, sn;
   unit_act_scales(args, 0, sp, sn);
-  int ug = 0, xu = 0;
-  bool ok = true;
+  int ug = 0;
+  bool ok = true, stored = false;
   for (int it = 0; it < rounds && ok; ++it) {
     Tile t;
     if (!tile_fn(it, t)) continue;
     // the tile's weight scales and bias into L1 while its MMAs run (a pass
     // would otherwise wait for them from HBM after the last MMA)
-    if (pos_warp && lane * 32 < t.width) {
+    if (data_warp && lane * 32 < t.width) {
       prefetch_l1(static_cast<const float*>(args.wscales) + t.n0 + lane * 32);
       if (args.bias != nullptr) prefetch_l1(args.bias + t.n0 + lane * 32);
     }
@@ -1158,49 +1164,31 @@ __device__ __forceinline__ void epilogue_stacked(
     if (!(ok = wait_warp(smem_u32(tmem_full + b), (ug / NBUF) & 1, abort_flag, budget))) break;
     tc_fence_after();
     ++ug;
-    if (!pos_warp && !neg_warp) {   // lanes past 2P: nothing to read
+    if (!data_warp) {   // lanes past 2P: nothing to read
       release(b);
       continue;
     }
     const int npass = (t.width + 31) / 32;
-    static_assert(BN % 32 == 0, "32-column passes");
-    constexpr int NPM = BN / 32;
-    // P = 16: every column of the tile into registers at once (one TMEM round
-    // trip instead of one per pass), and the buffer released before the passes
-    uint32_t va[XCH ? 1 : NPM][4][8];
-    if constexpr (!XCH) {
+    // every column of the tile into registers at once, then the buffer released
+    uint32_t va[NPM][4][8];
 #pragma unroll
-      for (int p = 0; p < NPM; ++p)
-        if (p < npass)
+    for (int p = 0; p < NPM; ++p)
+      if (p < npass)
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tmem_ld8(t_lane + (uint32_t)b * BN + (uint32_t)(32 * p + 8 * i), va[p][i]);
-      tmem_wait_ld();
-      release(b);
-      // P = 16: pass p stages into tile p (at most four passes, four tiles),
-      // all stored together after the last pass
-      if (sp_count > 0) {
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
-    }
+        for (int i = 0; i < 4; ++i)
+          tmem_ld8(t_lane + (uint32_t)b * BN + (uint32_t)(32 * p + 8 * i), va[p][i]);
+    tmem_wait_ld();
+    release(b);
+    int first = 0;   // first pass of the batch being staged
 #pragma unroll
     for (int p = 0; p < NPM; ++p) {
       if (p >= npass) break;
       const int col = 32 * p;
       uint32_t v[4][8];
-      if constexpr (!XCH) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[i][k] = va[p][i][k];
-      } else {
-        const uint32_t tcol = (uint32_t)b * BN + (uint32_t)col;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_ld8(t_lane + tcol + 8 * i, v[i]);
-        tmem_wait_ld();
-        if (p == npass - 1) release(b);   // every column of the tile is in registers
-      }
+        for (int k = 0; k < 8; ++k) v[i][k] = va[p][i][k];
       if constexpr (CSPLIT) {
         if (crank != 0) {   // into this CTA's buffer, then added into rank 0's
           uint32_t* own = reinterpret_cast<uint32_t*>(__cvta_shared_to_generic(part));
@@ -1229,109 +1217,51 @@ __device__ __forceinline__ void epilogue_stacked(
 #pragma unroll
           for (int k = 0; k < 8; ++k) v[i][k] += pb[pidx(col + 8 * i + k)];
       }
-      uint32_t vn[4][8];
-      // P = 16: lane l folds row l & 15, columns 16 * (l >> 4) .. +16 of the
-      // pass: the q- values of the first 16 columns go down to lanes 0-15 and
-      // the q+ values of the last 16 up to lanes 16-31 (one exchange), and
-      // each lane's (q+, q-) pair is picked without branching
-      const bool hi = lane >= 16;
+      // lane l: the (q+, q-) pair of row r, columns col + 16 * hi .. +16 --
+      // the q- values of the first 16 columns go down to lanes 0-15, the q+
+      // values of the last 16 up to lanes 16-31, picked without branching
+      // (q- rows first in each group: the two halves swap roles)
       uint32_t fp[2][8], fn[2][8];
-      if constexpr (!XCH) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t x = __shfl_xor_sync(0xffffffffu, hi ? v[i][k] : v[2 + i][k], 16);
-            fp[i][k] = hi ? x : v[i][k];
-            fn[i][k] = hi ? v[2 + i][k] : x;
-          }
-      } else {
-        const int xrow = (neg_warp ? quad - qparts : quad) * 32 + lane;
-        uint32_t* xr = xch + xrow * 32;
-        if (neg_warp) {
-          if (!(ok = wait_warp(xempty, (xu & 1) ^ 1, abort_flag, budget))) break;
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) xr[(8 * i + k) ^ lane] = v[i][k];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xfull);
-          ++xu;
-          continue;
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t x = __shfl_xor_sync(0xffffffffu, hi ? v[i][k] : v[2 + i][k], 16);
+          const uint32_t lo_half = hi ? x : v[i][k], hi_half = hi ? v[2 + i][k] : x;
+          fp[i][k] = neg_first ? hi_half : lo_half;
+          fn[i][k] = neg_first ? lo_half : hi_half;
         }
-        if (!(ok = wait_warp(xfull, xu & 1, abort_flag, budget))) break;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) vn[i][k] = xr[(8 * i + k) ^ lane];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(xempty);
-        ++xu;
-      }
-      // q+ warps: fold and stage rows quad*32 .. +31, columns col .. +31 into
-      // staging tile p (P = 16) or (quad * nb + sp_count % nb) once the store
-      // that last used it has read it (XCH)
-      uint8_t* stile = stage_y + (XCH ? (quad * nb + sp_count % nb) : p) * SYB;
-      const uint32_t sbase = smem_u32(stile);
-      if (XCH && sp_count >= nb) {
-        if (lane == 0) {
-          if (nb == 4) bulk_wait_read<3>();
-          else bulk_wait_read<1>();
-        }
+      // a new batch: the stores of the previous one have read their tiles
+      if (p == first && stored) {
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
       }
-      if constexpr (!XCH) {
-        const int h = hi ? 1 : 0, r = lane & 15;
-        const int cc = col + 16 * h;
-        if (cc < t.width) {
-          float o[16];
+      uint8_t* sub = my_sub + (p - first) * SUB;
+      const int h = hi ? 1 : 0;
+      const int cc = col + 16 * h;
+      if (cc < t.width) {
+        float o[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = 0.0f;
-          float sw[8];
-          load_wscales8(args, 0, 0, t.n0 + cc, sw);
-          fold8_exact(fp[0], fn[0], sw, sp, sn, o);
-          load_wscales8(args, 0, 0, t.n0 + cc + 8, sw);
-          fold8_exact(fp[1], fn[1], sw, sp, sn, o + 8);
-          stage16<Y_BF16>(args, t.n0 + cc, o, stile + r * ROWB, r, h);
-        }
-      } else {
-        uint8_t* srow = stile + lane * ROWB;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int cc = col + 16 * h;
-          if (cc < t.width) {
-            float o[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = 0.0f;
-            float sw[8];
-            load_wscales8(args, 0, 0, t.n0 + cc, sw);
-            fold8_exact(v[2 * h], vn[2 * h], sw, sp, sn, o);
-            load_wscales8(args, 0, 0, t.n0 + cc + 8, sw);
-            fold8_exact(v[2 * h + 1], vn[2 * h + 1], sw, sp, sn, o + 8);
-            stage16<Y_BF16>(args, t.n0 + cc, o, srow, lane, h);
-          }
-        }
+        for (int i = 0; i < 16; ++i) o[i] = 0.0f;
+        float sw[8];
+        load_wscales8(args, 0, 0, t.n0 + cc, sw);
+        fold8_exact(fp[0], fn[0], sw, sp, sn, o);
+        load_wscales8(args, 0, 0, t.n0 + cc + 8, sw);
+        fold8_exact(fp[1], fn[1], sw, sp, sn, o + 8);
+        stage16<Y_BF16>(args, t.n0 + cc, o, sub + r * ROWB, r, h);
       }
-      if constexpr (XCH) {
+      // the batch leaves when the warp's tiles are full or the tile is done
+      if (p - first == ns - 1 || p == npass - 1) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(tmap_y, sbase, t.n0 + col, t.m0 + quad * 32);
+          for (int q = first; q <= p; ++q)
+            tma_store_2d(tmap_y, smem_u32(my_sub + (q - first) * SUB), t.n0 + 32 * q,
+                         t.m0 + 16 * quad);
           bulk_commit_group();
         }
-        ++sp_count;
-      }
-    }
-    if constexpr (!XCH) {   // the tile's passes, stored together
-      if (ok && (CSPLIT ? crank == 0 : true)) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          for (int p = 0; p < npass; ++p)
-            tma_store_2d(tmap_y, smem_u32(stage_y + p * SYB), t.n0 + 32 * p, t.m0 + quad * 32);
-          bulk_commit_group();
-        }
-        sp_count += npass;
+        stored = true;
+        first = p + 1;
       }
     }
   }

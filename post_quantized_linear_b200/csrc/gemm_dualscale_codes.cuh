@@ -81,12 +81,13 @@ __host__ __device__ constexpr bool codes_kps2_fits(int bn, bool multi, bool y_bf
 }
 
 // STK_ (stacked polarities, one row tile of M <= STK_ rows, one unit per
-// tile): the q+ box lands in rows [0, P) of one A tile and the q- box in rows
-// [P, 2P), P = M rounded up to 16, so a single MMA per k step yields both
-// products (accumulator lanes r and P + r) and half the MMAs of the two-tile
-// form are issued.  The A area of a k block is 2 * STK_ rows; the MMA still
-// reads 128 rows from its start (the rows past 2P belong to the weight tile or
-// the next k block and land in accumulator lanes nobody reads).
+// tile): the P rows (M rounded up to 16, 32 or 64) are stacked in groups of
+// 16 -- group g's q+ box in A rows 32g .. +15, its q- box in rows 32g + 16 ..
+// +31 -- so a single MMA per k step yields both products (accumulator lanes
+// 32g + r and 32g + 16 + r, both in lane quarter g) and half the MMAs of the
+// two-tile form are issued.  The A area of a k block is 2 * STK_ rows; the MMA
+// still reads 128 rows from its start (the rows past 2P belong to the weight
+// tile or the next k block and land in accumulator lanes nobody reads).
 // CSPLIT_ (one row tile: stacked rows, or the two-tile form with four
 // epilogue warps): the K range of an N tile is split over the CTAs of a
 // cluster; the first CTA keeps an int32 buffer in shared memory -- [2P][BN]
@@ -116,9 +117,8 @@ struct CodesCfg {
   static constexpr bool TMA_Y = SINGLE || MULTI || EPW != epi_warps(MULTI) ||
                                 (kStageBudget - EPW * stage_y_bytes(Y_BF16)) / STAGE >= 2;
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
-  // group units: each epilogue warp's two 32-float buffers of widened weight scales;
-  // stacked polarities: the q- accumulators of 32 columns, handed between warps
-  static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : (STK_ > 16 ? STK_ * 32 * 4 : 0);
+  // group units: each epilogue warp's two 32-float buffers of widened weight scales
+  static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : 0;
   // stacked (small M): three stages at most, so that about 105 KiB of shared
   // memory and 256 TMEM columns let a CTA of the next GEMM in the stream share
   // the SM and prefetch its weights while this one finishes
@@ -141,10 +141,9 @@ struct CodesCfg {
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
   static constexpr int OFF_PART = OFF_SW + SW_BYTES;
   static constexpr int OFF_BAR = OFF_PART + PART_BYTES;
-  // full, empty; tmem full/empty; drain; (W4) unpacked; (stacked) exchange full/empty
+  // full, empty; tmem full/empty; drain; (W4) unpacked
   // (+ K split: the partial sums of the other CTAs have landed)
-  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0) + (STK_ > 16 ? 2 : 0) +
-                                  (CSPLIT_ ? 1 : 0);
+  static constexpr int NUM_BARS = 2 * 8 + 2 * 2 + 1 + (W4_ ? 8 : 0) + (CSPLIT_ ? 1 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = NACC * BN * NBUF;
@@ -181,9 +180,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   uint64_t* tmem_empty = tmem_full + 2;   // [2]
   uint64_t* drain_bar = tmem_empty + 2;
   uint64_t* ready = drain_bar + 1;        // [8] (W4) int4 tile unpacked
-  uint64_t* xfull = ready + (W4 ? 8 : 0);  // (stacked, P > 16) q- accumulators handed over
-  uint64_t* xempty = xfull + 1;            // (stacked, P > 16) q+ warps done reading them
-  uint64_t* parts = xfull + (STK > 16 ? 2 : 0);   // (K split, first CTA) partial sums added
+  uint64_t* parts = ready + (W4 ? 8 : 0);  // (K split, first CTA) partial sums added
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -203,10 +200,6 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     mbar_init(smem_u32(drain_bar), 1);
     if constexpr (W4)
       for (int i = 0; i < C::S; ++i) mbar_init(smem_u32(ready + i), kUnpackWarps);
-    if constexpr (STK > 16) {   // one arrival per 32-row quarter of q- (q+) rows
-      mbar_init(smem_u32(xfull), (uint32_t)((args.a_rows + 31) / 32));
-      mbar_init(smem_u32(xempty), (uint32_t)((args.a_rows + 31) / 32));
-    }
     if constexpr (CSPLIT) mbar_init(smem_u32(parts), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -266,7 +259,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       const uint32_t kb_tx = (uint32_t)(C::CODE_TILES * (args.a_rows > 0 ? args.a_rows : BM) * BK +
                                         (W4 ? C::WP_BYTES : C::W_BYTES));
       // the q- box: right below the q+ rows (stacked) or its own 128-row tile
-      const int qn_off = STK ? args.a_rows * BK : BM * BK;
+      const int qn_off = BM * BK;
       int c = 0;
       bool ok = (args.starve == 0);
       // Stacked (small M): the weight boxes of the first stages are requested
@@ -306,7 +299,17 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
           for (int j = 0; j < nk; ++j) {
             const int kb = kb0 + j;
             uint8_t* st = smem + s * C::STAGE + j * C::KB_BYTES;
-            if constexpr (!LDA) {
+            if constexpr (STK != 0) {   // groups of 16 rows: q+ rows, then q- rows
+              if (args.code_box4)
+                tma_load_4d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, 0, 0, t.m0 / 16);
+              else
+              for (int g = 0; g < args.a_rows / 16; ++g) {
+                tma_load_2d(smem_u32(st + 32 * g * BK), &tmap_qp, smem_u32(full + s), kb * BK,
+                            t.m0 + 16 * g);
+                tma_load_2d(smem_u32(st + (32 * g + 16) * BK), &tmap_qn, smem_u32(full + s), kb * BK,
+                            t.m0 + 16 * g);
+              }
+            } else if constexpr (!LDA) {
               tma_load_2d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, t.m0);
               if constexpr (!SINGLE)
                 tma_load_2d(smem_u32(st + qn_off), &tmap_qn, smem_u32(full + s), kb * BK, t.m0);
@@ -463,10 +466,9 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
     if constexpr (STK != 0) {
       static_assert(!STK || C::Y_BYTES == 4 * stage_y_bytes(Y_BF16), "four staging tiles");
-      epilogue_stacked<BN, C::NBUF, Y_BF16, (STK > 16), CSPLIT>(
-          args, &tmap_y, smem + C::OFF_Y, reinterpret_cast<uint32_t*>(smem + C::OFF_SW), quad, lane, t_lane,
-          tmem_full, smem_u32(tmem_empty), smem_u32(xfull), smem_u32(xempty), rounds, tiles,
-          abort_flag, budget, crank, smem_u32(smem + C::OFF_PART), smem_u32(parts));
+      epilogue_stacked<BN, C::NBUF, Y_BF16, CSPLIT>(
+          args, &tmap_y, smem + C::OFF_Y, quad, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
+          tiles, abort_flag, budget, crank, smem_u32(smem + C::OFF_PART), smem_u32(parts));
     } else if constexpr (SEEDED) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
       float* sw_stage = reinterpret_cast<float*>(smem + C::OFF_SW) + (warp - EPI0) * 64;

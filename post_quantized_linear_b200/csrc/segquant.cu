@@ -139,6 +139,25 @@ sq_status make_tmap(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
   return r == CUDA_SUCCESS ? SQ_OK : SQ_ERR_CUDA;
 }
 
+// A tiled map of rank 3 or 4 over int8 data (128-byte inner boxes, 128-byte
+// swizzle); strides in bytes for dimensions 1.. .
+sq_status make_tmap_nd(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return SQ_ERR_CUDA;
+  cuuint64_t d[4], st[3];
+  cuuint32_t bx[4], estr[4] = {1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), d, st,
+                  bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SQ_OK : SQ_ERR_CUDA;
+}
+
 sq_status check_qweight(const sq_qweight* w, int64_t K, SegBounds* kseg) {
   if (w == nullptr) return SQ_ERR_INVALID_ARG;
   if (w->N <= 0 || w->K <= 0 || w->K != K) return SQ_ERR_INVALID_ARG;
@@ -563,10 +582,13 @@ sq_status launch_codes_small(int bn, bool y_bf16, const CUtensorMap& tqp, const 
 // Tensor map of Y for the TMA-store epilogue: boxes of 32 rows x 32 columns,
 // bf16 rows of 64 bytes in the 64-byte swizzle, fp32 rows of 128 bytes in the
 // 128-byte swizzle (the staging layout of epilogue_tma_store).
-sq_status make_tmap_y(CUtensorMap* map, void* y, sq_dtype yt, int64_t M, int64_t N, int64_t ldy) {
+// Y for TMA stores of 32 columns x box_rows rows (32; 16 for stacked rows,
+// whose warps store groups of 16 rows).
+sq_status make_tmap_y(CUtensorMap* map, void* y, sq_dtype yt, int64_t M, int64_t N, int64_t ldy,
+                      uint32_t box_rows = 32) {
   const bool bf = (yt == SQ_BF16);
   return make_tmap(map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y,
-                   (uint64_t)N, (uint64_t)M, (uint64_t)(ldy * (bf ? 2 : 4)), 32, 32,
+                   (uint64_t)N, (uint64_t)M, (uint64_t)(ldy * (bf ? 2 : 4)), 32, box_rows,
                    bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -975,7 +997,7 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
       BN = sbn;
     }
   }
-  const int a_rows = stacked ? (M <= 16 ? 16 : M <= 32 ? 32 : 64)
+  const int a_rows = stacked ? (int)((M + 15) / 16 * 16)   // groups of 16 rows
                      : (codes_kernel && M < sq::BM) ? (int)((M + 15) / 16 * 16) : sq::BM;
   CUtensorMap ta, ta2, tw;
   if (src == ASource::X) {
@@ -985,12 +1007,14 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
     if (st != SQ_OK) return st;
     ta2 = ta;
   } else {
+    // (stacked rows: boxes of 16 rows, one per group and polarity)
+    const uint32_t box_rows = stacked ? 16u : (uint32_t)a_rows;
     st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_pos, (uint64_t)K, (uint64_t)M,
-                   (uint64_t)ldq, 128, (uint32_t)a_rows);
+                   (uint64_t)ldq, 128, box_rows);
     if (st != SQ_OK) return st;
     if (dual_codes) {
       st = make_tmap(&ta2, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_neg, (uint64_t)K, (uint64_t)M,
-                     (uint64_t)ldq, 128, (uint32_t)a_rows);
+                     (uint64_t)ldq, 128, box_rows);
       if (st != SQ_OK) return st;
     } else {
       ta2 = ta;
@@ -1028,6 +1052,24 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   a.a_neg = q_neg;
   a.lda = ldq;
   a.a_rows = a_rows;
+  // stacked rows: every group of 16 rows of both polarities in one box when M
+  // is whole groups (no row past M is addressed); the map starts at the lower
+  // of the two code tensors (its planes: q+, q- or q-, q+), whose distance
+  // must be a multiple of 16 bytes
+  if (stacked && M % 16 == 0) {
+    const uintptr_t pp = reinterpret_cast<uintptr_t>(q_pos), pn = reinterpret_cast<uintptr_t>(q_neg);
+    const bool neg_first = pn < pp;
+    const uintptr_t gap = neg_first ? pp - pn : pn - pp;
+    if (gap > 0 && gap % 16 == 0 && gap < (1ull << 40)) {
+      const uint64_t cd[4] = {(uint64_t)K, 16, 2, (uint64_t)(M / 16)};
+      const uint64_t cs[3] = {(uint64_t)ldq, (uint64_t)gap, (uint64_t)(16 * ldq)};
+      const uint32_t cb[4] = {(uint32_t)sq::BK, 16, 2, (uint32_t)(a_rows / 16)};
+      st = make_tmap_nd(&ta, neg_first ? q_neg : q_pos, 4, cd, cs, cb);
+      if (st != SQ_OK) return st;
+      a.code_box4 = 1;
+      a.code_neg_first = neg_first ? 1 : 0;
+    }
+  }
 
   using bf = __nv_bfloat16;
   constexpr int AX = sq::ASRC_X, AC = sq::ASRC_CODES;
@@ -1088,12 +1130,15 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
         return launch_codes_out<128, true>(yb, ta, ta2, tw, ty, a, stream);
       }
       if (stacked) {
+        CUtensorMap ty16;   // the warps store groups of 16 rows
+        st = make_tmap_y(&ty16, y, yt, M, N, ldy, 16);
+        if (st != SQ_OK) return st;
         if (split_cs > 1) {   // CTA r of a cluster: k blocks [r*kb/cs, (r+1)*kb/cs)
           a.splits = split_cs;
-          return launch_codes_small_split(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
+          return launch_codes_small_split(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty16, a,
                                           stream);
         }
-        return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty, a,
+        return launch_codes_small_stacked(bn_small, a_rows <= 16 ? 16 : 64, yb, ta, ta2, tw, ty16, a,
                                           stream);
       }
       if (bn_small && split_cs > 1) {   // two-tile form, k blocks shared by a cluster

@@ -105,3 +105,32 @@ def test_k_split_over_a_cluster(K, N, M, out, monkeypatch, dev_lib):
     ref = res[("0", "32")].view(iv)
     for key, y in res.items():
         assert torch.equal(y.view(iv), ref), key
+
+
+@pytest.mark.parametrize("layout", ["neg_below", "neg_far_above"])
+@pytest.mark.parametrize("M,K", [(16, 1152), (40, 1152), (16, 1040), (48, 1152), (64, 3072)])
+def test_code_boxes_follow_the_buffers(M, K, layout):
+    """Stacked rows come in groups of 16 (each group's q+ rows, then its q-
+    rows).  When M is whole groups one box of a 4-D map brings every group of
+    both polarities for a k block; the map starts at the lower of the two code
+    tensors, so with q- below q+ each group's q- rows come first and the fold
+    swaps the halves.  Otherwise (M = 40) each group and polarity comes as its
+    own 16-row box.  Codes written into one buffer with q- in its first half
+    (below q+), or far above q+, K = 1040 (a partial last k block): every row
+    against the oracle (fp32 out, bit-exact)."""
+    import post_quantized_linear_b200 as pq
+    N = 400
+    c = Case(W.small_case(M, K, N, seed=77 + M + K, out="f32"))
+    ldq = (K + 15) // 16 * 16
+    gap = 1 if layout == "neg_below" else 4096
+    buf = torch.zeros(((1 + gap) * M, ldq), dtype=torch.int8, device="cuda")
+    if layout == "neg_below":
+        qn, qp = buf[:M, :K], buf[M:, :K]
+    else:
+        qp, qn = buf[:M, :K], buf[gap * M:, :K]
+    pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn, out=(qp, qn))
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    y_ref, _ = c.oracle_rows(np.arange(M))
+    np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
