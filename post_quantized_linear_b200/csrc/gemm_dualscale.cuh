@@ -97,10 +97,12 @@ struct GemmArgs {
   // past the box keep stale shared memory; their accumulator lanes are never
   // stored.
   int32_t a_rows;
-  // Stacked rows, M a multiple of 16: tmap_qp is a 4-D map (K bytes x 16 rows x
-  // {q+, q-} x groups of 16 rows) whose one box per k block lands every group's
-  // q+ and q- rows in the stacked order (1), or each group and polarity comes
-  // as its own 16-row box (0).
+  // Stacked rows: tmap_qp is a 4-D map (K bytes x 16 rows x {q+, q-} x groups
+  // of 16 rows) whose one box per k block lands every whole group's q+ and q-
+  // rows in the stacked order (1); when M is not whole groups, tmap_qn is a
+  // 3-D map (K bytes x M rows x {q+, q-}) that brings the last, partial group
+  // in two 16-row boxes (2); or each group and polarity comes as its own
+  // 16-row box of the 2-D maps (0).
   int32_t code_box4;
   int32_t code_neg_first;   // (code_box4) the map starts at q-: each group's q- rows come first
 };

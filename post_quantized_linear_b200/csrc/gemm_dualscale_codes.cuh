@@ -300,9 +300,17 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
             const int kb = kb0 + j;
             uint8_t* st = smem + s * C::STAGE + j * C::KB_BYTES;
             if constexpr (STK != 0) {   // groups of 16 rows: q+ rows, then q- rows
-              if (args.code_box4)
-                tma_load_4d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, 0, 0, t.m0 / 16);
-              else
+              if (args.code_box4) {
+                const int whole = args.M / 16;   // whole groups: one 4-D box
+                if (whole > 0)
+                  tma_load_4d(smem_u32(st), &tmap_qp, smem_u32(full + s), kb * BK, 0, 0, t.m0 / 16);
+                if (args.code_box4 == 2) {       // the partial group: both planes of its 16 rows
+                  tma_load_3d(smem_u32(st + 32 * whole * BK), &tmap_qn, smem_u32(full + s), kb * BK,
+                              t.m0 + 16 * whole, 0);
+                  tma_load_3d(smem_u32(st + (32 * whole + 16) * BK), &tmap_qn, smem_u32(full + s),
+                              kb * BK, t.m0 + 16 * whole, 1);
+                }
+              } else
               for (int g = 0; g < args.a_rows / 16; ++g) {
                 tma_load_2d(smem_u32(st + 32 * g * BK), &tmap_qp, smem_u32(full + s), kb * BK,
                             t.m0 + 16 * g);

@@ -1052,21 +1052,33 @@ sq_status gemm_common(ASource src, const void* x, sq_dtype xt, const int8_t* q_p
   a.a_neg = q_neg;
   a.lda = ldq;
   a.a_rows = a_rows;
-  // stacked rows: every group of 16 rows of both polarities in one box when M
-  // is whole groups (no row past M is addressed); the map starts at the lower
-  // of the two code tensors (its planes: q+, q- or q-, q+), whose distance
-  // must be a multiple of 16 bytes
-  if (stacked && M % 16 == 0) {
+  // stacked rows: the whole groups of 16 rows of both polarities in one box
+  // of a 4-D map (no row past the whole groups is addressed), and a partial
+  // last group in two boxes of a 3-D map over all M rows (rows past M read as
+  // zeros).  Both maps start at the lower of the two code tensors (planes q+,
+  // q- or q-, q+), whose distance must be a multiple of 16 bytes.
+  if (stacked) {
     const uintptr_t pp = reinterpret_cast<uintptr_t>(q_pos), pn = reinterpret_cast<uintptr_t>(q_neg);
     const bool neg_first = pn < pp;
     const uintptr_t gap = neg_first ? pp - pn : pn - pp;
+    const void* low = neg_first ? static_cast<const void*>(q_neg) : static_cast<const void*>(q_pos);
     if (gap > 0 && gap % 16 == 0 && gap < (1ull << 40)) {
-      const uint64_t cd[4] = {(uint64_t)K, 16, 2, (uint64_t)(M / 16)};
-      const uint64_t cs[3] = {(uint64_t)ldq, (uint64_t)gap, (uint64_t)(16 * ldq)};
-      const uint32_t cb[4] = {(uint32_t)sq::BK, 16, 2, (uint32_t)(a_rows / 16)};
-      st = make_tmap_nd(&ta, neg_first ? q_neg : q_pos, 4, cd, cs, cb);
-      if (st != SQ_OK) return st;
-      a.code_box4 = 1;
+      const int64_t whole = M / 16;
+      if (whole > 0) {
+        const uint64_t cd[4] = {(uint64_t)K, 16, 2, (uint64_t)whole};
+        const uint64_t cs[3] = {(uint64_t)ldq, (uint64_t)gap, (uint64_t)(16 * ldq)};
+        const uint32_t cb[4] = {(uint32_t)sq::BK, 16, 2, (uint32_t)whole};
+        st = make_tmap_nd(&ta, low, 4, cd, cs, cb);
+        if (st != SQ_OK) return st;
+      }
+      if (M % 16 != 0) {
+        const uint64_t cd[3] = {(uint64_t)K, (uint64_t)M, 2};
+        const uint64_t cs[2] = {(uint64_t)ldq, (uint64_t)gap};
+        const uint32_t cb[3] = {(uint32_t)sq::BK, 16, 1};
+        st = make_tmap_nd(&ta2, low, 3, cd, cs, cb);
+        if (st != SQ_OK) return st;
+      }
+      a.code_box4 = (M % 16 != 0) ? 2 : 1;
       a.code_neg_first = neg_first ? 1 : 0;
     }
   }
