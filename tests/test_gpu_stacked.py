@@ -111,13 +111,13 @@ def test_k_split_over_a_cluster(K, N, M, out, monkeypatch, dev_lib):
 @pytest.mark.parametrize("M,K", [(16, 1152), (40, 1152), (16, 1040), (48, 1152), (64, 3072)])
 def test_code_boxes_follow_the_buffers(M, K, layout):
     """Stacked rows come in groups of 16 (each group's q+ rows, then its q-
-    rows).  When M is whole groups one box of a 4-D map brings every group of
-    both polarities for a k block; the map starts at the lower of the two code
-    tensors, so with q- below q+ each group's q- rows come first and the fold
-    swaps the halves.  Otherwise (M = 40) each group and polarity comes as its
-    own 16-row box.  Codes written into one buffer with q- in its first half
-    (below q+), or far above q+, K = 1040 (a partial last k block): every row
-    against the oracle (fp32 out, bit-exact)."""
+    rows).  One box of a 4-D map brings the whole groups of both polarities
+    for a k block and a 3-D map over all M rows the partial last group (M =
+    40: two whole groups and 8 rows); both maps start at the lower of the two
+    code tensors, so with q- below q+ each group's q- rows come first and the
+    fold swaps the halves.  Codes written into one buffer with q- in its first
+    half (below q+), or far above q+, K = 1040 (a partial last k block): every
+    row against the oracle (fp32 out, bit-exact)."""
     import post_quantized_linear_b200 as pq
     N = 400
     c = Case(W.small_case(M, K, N, seed=77 + M + K, out="f32"))
