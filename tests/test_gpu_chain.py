@@ -113,3 +113,41 @@ def test_two_gemms_write_the_same_output_in_turn():
     assert pq.stream_status() == 0
     assert torch.equal(y.view(torch.int16), y_ref2.view(torch.int16))
     assert s.item() == y_ref2.float().sum().item()
+
+
+def test_first_call_of_the_process_inside_graph_capture(tmp_path):
+    """A process whose first forward (small M, so the cluster-split choice and
+    its one-time device queries run) happens while a CUDA graph is being
+    captured: the graph replays to the same bits as an eager call."""
+    import subprocess
+    import sys
+    import os
+    script = tmp_path / "first_in_graph.py"
+    script.write_text(r'''
+import sys, torch
+import post_quantized_linear_b200 as pq
+M, K, N = 16, 4608, 1152
+g = torch.Generator().manual_seed(3)
+x = torch.nn.functional.silu(torch.randn((M, K), generator=g)).to(torch.bfloat16).cuda()
+w = (torch.randn((N, K), generator=g) * 0.02).cuda()
+sp = torch.tensor([0.05], device="cuda"); sn = torch.tensor([0.01], device="cuda")
+qw = pq.quantize_weights(w, [0, K], bits=8)
+qp, qn = pq.quantize_activations(x, [0, K], sp, sn)
+y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+torch.cuda.synchronize()
+graph = torch.cuda.CUDAGraph()
+with torch.cuda.graph(graph):
+    pq.linear_from_codes(qp, qn, qw, sp, sn, out=y)   # the process's first forward
+y.zero_()
+graph.replay()
+torch.cuda.synchronize()
+ref = pq.linear_from_codes(qp, qn, qw, sp, sn)
+torch.cuda.synchronize()
+assert pq.stream_status() == 0
+sys.exit(0 if torch.equal(y.view(torch.int16), ref.view(torch.int16)) else 3)
+''')
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PYTHONPATH=root + os.pathsep + os.environ.get("PYTHONPATH", ""))
+    res = subprocess.run([sys.executable, str(script)], capture_output=True, text=True, timeout=600,
+                         cwd=root, env=env)
+    assert res.returncode == 0, res.stdout[-2000:] + res.stderr[-2000:]
