@@ -469,10 +469,10 @@ sq_status launch_codes_small_split(int bn, int stk, bool y_bf16, const CUtensorM
   }
 }
 
-// How many clusters of `cs` CTAs (one CTA per SM, with the widest split
-// kernel's shared memory) the current device runs at once.  A cluster stays inside one
-// group of SMs, so this is below num_sms() / cs when the groups' sizes are not
-// multiples of cs.  0 when the query fails.
+// How many clusters of `cs` CTAs, one CTA per SM, the current device runs at
+// once.  A cluster stays inside one group of SMs, so this is below
+// num_sms() / cs when the groups' sizes are not multiples of cs.  0 when the
+// query fails.
 int max_clusters(int cs) {
   static std::atomic<int> cached[kMaxDevices][9] = {};
   int dev = 0;
