@@ -948,10 +948,15 @@ def run_ours(args):
             line["configs"] = table
         if not args.no_small_m:
             line["small_m"] = {
-                "note": "HBM-bound forwards at M <= 128 (median of L2-flushed graph replays; "
+                "note": "forwards at M <= 128 (median of L2-flushed graph replays; "
                         "one_pass_layers: per layer of 8 back-to-back layers with distinct "
-                        "weights); bytes = weight codes + scales + q+/q- codes + Y; peak = "
-                        "measured HBM copy",
+                        "weights, which hides part of each launch); bytes = weight codes + "
+                        "scales + q+/q- codes + Y; peak = the HBM copy bandwidth (measured "
+                        "figure, else the fallback). (3072, 12288) streams its weight at "
+                        "~4.6 TB/s in steady state, the rest of a layer being launch, "
+                        "first-load latency and epilogue; (4608, 1152) is a 5.3 MB weight "
+                        "whose time follows the k blocks each CTA streams, cut by sharing "
+                        "each N tile's k blocks over a cluster of CTAs",
                 "peak_gbs": hbm_peak,
                 "cases": small_m_measure(dev, flush, args.steps, hbm_peak)}
             line["per_call_us"] = per_call_measure(dev)
