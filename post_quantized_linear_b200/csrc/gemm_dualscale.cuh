@@ -903,6 +903,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
     return (uint32_t)(((128 * a + quad * 32 + lane) * BN) + ((c & ~31) | ((c & 31) ^ lane)));
   };
   bool parts_in = false;
+  bool sent = false;   // K split, rank > 0: this warp's slices have gone to rank 0
   constexpr int HALF = BN / (EPW / 4);
   constexpr int ROWB = Y_BF16 ? 64 : 128;
   constexpr uint32_t BUF_COLS = (uint32_t)(NACC * BN);
@@ -1073,6 +1074,7 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
                   bulk_reduce_add_u32_cluster(part0 + off, part_buf + off, 32u * BN * 4u, bar0);
                 }
               }
+              sent = true;
             }
             continue;
           }
@@ -1087,6 +1089,22 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       }
       if (npass == 0) release(b);
       ++ug;
+    }
+  }
+  if constexpr (CSPLIT) {
+    // After an abort the slices still go (their contents no longer count):
+    // rank 0's barrier then completes, and rank 0 holds the cluster until
+    // every add into its buffer has landed.
+    if (crank != 0 && !sent) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t part0 = mapa_shared(part_buf, 0), bar0 = mapa_shared(parts_bar, 0);
+        for (int a = 0; a < 2; ++a) {
+          const uint32_t off = (uint32_t)((128 * a + quad * 32) * BN * 4);
+          bulk_reduce_add_u32_cluster(part0 + off, part_buf + off, 32u * BN * 4u, bar0);
+        }
+      }
     }
   }
   // Every store has completed before the CTA (and its shared memory) exits.
@@ -1119,7 +1137,10 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
 // barrier; rank 0's warps wait for every byte (bounded), add their slices to
 // their own accumulators -- integer sums, exact in any order -- and fold and
 // store as above.  (The buffers stay alive until rank 0 has seen every byte:
-// the CTAs leave through a cluster barrier after the epilogue.)
+// the CTAs leave through a cluster barrier after the epilogue.  A warp that
+// gave up on a wait still sends its slice, and rank 0, after giving up
+// itself, waits for the bytes before that barrier, so no add lands in a CTA
+// that has left.)
 template <int BN, int NBUF, bool Y_BF16, bool CSPLIT = false, class TileFn>
 __device__ __forceinline__ void epilogue_stacked(
     const GemmArgs& args, const CUtensorMap* tmap_y, uint8_t* stage_y, int quad, int lane,
@@ -1137,6 +1158,7 @@ __device__ __forceinline__ void epilogue_stacked(
   };
   const uint32_t part0 = CSPLIT ? mapa_shared(part, 0) : 0u;   // rank 0's buffer
   bool parts_in = false;
+  bool sent = false;   // rank > 0: this warp's slice has gone to rank 0
   const int groups = args.a_rows / 16;                          // warps holding rows
   const bool data_warp = quad < groups;
   const int ns = NSUB / groups;                                 // staging tiles per warp
@@ -1206,6 +1228,7 @@ __device__ __forceinline__ void epilogue_stacked(
               bulk_reduce_add_u32_cluster(part0 + slice, part + slice, 32u * BN * 4u,
                                           mapa_shared(parts_bar, 0));
             }
+            sent = true;
           }
           continue;
         }
@@ -1264,6 +1287,20 @@ __device__ __forceinline__ void epilogue_stacked(
         }
         stored = true;
         first = p + 1;
+      }
+    }
+  }
+  if constexpr (CSPLIT) {
+    // After an abort the slice still goes (its contents no longer count):
+    // rank 0's barrier then completes, and rank 0 holds the cluster until
+    // every add into its buffer has landed.
+    if (crank != 0 && data_warp && !sent) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t slice = (uint32_t)quad * 32u * BN * 4u;
+        bulk_reduce_add_u32_cluster(part0 + slice, part + slice, 32u * BN * 4u,
+                                    mapa_shared(parts_bar, 0));
       }
     }
   }

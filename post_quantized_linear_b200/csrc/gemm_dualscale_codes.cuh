@@ -499,8 +499,14 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  // K split: the first CTA's buffer outlives every add into it
-  if constexpr (CSPLIT) cluster_sync();
+  // K split: the first CTA's buffer outlives every add into it.  Without an
+  // abort its epilogue has already seen every byte on `parts`; after one, the
+  // other CTAs still send their slices, so it waits for them here (bounded)
+  // while the others wait at the cluster barrier.
+  if constexpr (CSPLIT) {
+    if (threadIdx.x == 0 && crank == 0 && *abort_flag) wait_drain(smem_u32(parts), 0, 2 * budget);
+    cluster_sync();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_ALLOC);

@@ -134,3 +134,32 @@ def test_code_boxes_follow_the_buffers(M, K, layout):
     assert pq.stream_status() == 0
     y_ref, _ = c.oracle_rows(np.arange(M))
     np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("M", [16, 100])
+def test_k_split_starved_pipeline_times_out_and_context_recovers(M, dev_lib):
+    """(K, N) = (4608, 1152) splits each N tile's k blocks over a cluster (M =
+    16: stacked rows; M = 100: the two-tile form).  With the producer starved
+    (development build) every CTA gives up on a bounded wait; the CTAs of rank
+    > 0 still send their slices and rank 0 waits for them before the cluster
+    leaves, so the call ends with a timeout status, and the next call on the
+    same context gives the oracle's rows."""
+    import post_quantized_linear_b200 as pq
+    from post_quantized_linear_b200 import _lib
+    c = Case(W.small_case(M, 4608, 1152, seed=40 + M, out="f32"))
+    qp, qn = pq.quantize_activations(c.x, c.wl.kseg, c.sp, c.sn)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == _lib.SQ_OK
+    pq.set_wait_budget(2_000_000)
+    pq.debug_starve_pipeline(True)
+    try:
+        pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+        assert pq.stream_status() == _lib.SQ_ERR_TIMEOUT
+    finally:
+        pq.debug_starve_pipeline(False)
+        pq.set_wait_budget(0)
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b, out_dtype=c.out_dtype)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == _lib.SQ_OK
+    y_ref, _ = c.oracle_rows(np.arange(M))
+    np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
