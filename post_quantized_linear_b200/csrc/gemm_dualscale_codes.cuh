@@ -119,9 +119,10 @@ struct CodesCfg {
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
   // group units: each epilogue warp's two 32-float buffers of widened weight scales
   static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : 0;
-  // stacked (small M): three stages at most, so that about 105 KiB of shared
-  // memory and 256 TMEM columns let a CTA of the next GEMM in the stream share
-  // the SM and prefetch its weights while this one finishes
+  // stacked (small M): three stages at most (deeper rings stream no faster);
+  // at tiles of up to 64 columns a CTA of the next GEMM in the stream fits on
+  // the SM beside this one (shared memory, TMEM and registers) and requests
+  // its first weight stages while this one finishes
   static constexpr int S_CAP = STK_ ? 3 : 8;
   // K split: [2P][BN] int32 (stacked) or [2][128][BN] (two-tile form)
   static constexpr int PART_BYTES = CSPLIT_ ? (STK_ ? 2 * STK_ : 2 * BM) * BN_ * 4 : 0;
