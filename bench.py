@@ -127,6 +127,27 @@ def mma_rate_tops(sms: int, sm_mhz: float) -> float:
     return MMA_I8_OPS_PER_CLK_SM * sms * sm_mhz * 1e6 / 1e12
 
 
+# fp32 lanes per SM (four sub-partitions of 32).  A packed f32x2 instruction
+# holds its pipe for two cycles (instruction-mix counters of the int4 GEMM), so
+# pairs do not raise this rate.
+FP32_LANES_SM = 128
+# int4 groups: per output element and 128-wide group the fold takes two exact
+# seed subtractions, one product and two fused multiply-adds.
+FOLD_OPS_PER_OUTPUT_GROUP = 5
+
+
+def fold_roofline(wl, gemm_us: float, mma_peak: float) -> dict:
+    """The per-group fold of an int4 GEMM against the SMs' fp32 lane rate (an
+    FMA counted as one operation), at the clock the MMA rate was taken at."""
+    ops = wl.M * wl.N * (wl.K // 128) * FOLD_OPS_PER_OUTPUT_GROUP
+    peak = mma_peak * FP32_LANES_SM / MMA_I8_OPS_PER_CLK_SM      # T fp32 ops/s
+    achieved = ops / (gemm_us * 1e-6) / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "T fp32 ops/s",
+            "frac": achieved / peak, "ops_per_launch": ops,
+            "floor_us": ops / (peak * 1e12) * 1e6,
+            "peak_source": f"{FP32_LANES_SM} fp32 lanes/clk/SM x SMs x the MMA rate's clock"}
+
+
 # ------------------------------------------------------------ rank launch
 def free_port() -> int:
     s = socket.socket()
@@ -727,6 +748,7 @@ def measure_config(wl, dev, flush, steps: int, warmup: int, int8_peak: float, mm
             "algorithmic_bytes_per_launch": byts,
             "achieved_gbs": byts / (gemm_ms * 1e-3) / 1e9,
             "frac_hbm": byts / (gemm_ms * 1e-3) / 1e9 / hbm_peak,
+            **({"fold": fold_roofline(wl, gemm_ms * 1e3, mma_peak)} if wl.bits == 4 else {}),
         },
     }
 
@@ -897,6 +919,7 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": byts,
                 "achieved_gbs": byts / (gemm_avg_ms * 1e-3) / 1e9,
                 "avg_launch_us": gemm_avg_ms * 1e3,
+                **({"fold": fold_roofline(wl, gemm_avg_ms * 1e3, mma_peak)} if wl.bits == 4 else {}),
             },
             "forward_only": {
                 "us": fwd_avg_ms * 1e3, "exec_tops": ops / (fwd_avg_ms * 1e-3) / 1e12,

@@ -80,3 +80,16 @@ def test_clock_sampler_reads_nvml(monkeypatch):
     assert out["samples"] > 10 and out["sm_max_mhz"] == 1965
     assert out["sm_mhz"] in (1800, 1965)
     assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_fold_roofline_of_int4_groups():
+    """w4a8: 16384 x 3072 outputs, 24 groups, five fp32 operations each; the
+    fp32 lane rate of 148 SMs at 1965 MHz is 128 x 148 x 1.965e9 /s."""
+    from synth import workloads as W
+    wl = W.WORKLOADS["w4a8"]
+    r = bench.fold_roofline(wl, 550.0, bench.mma_rate_tops(148, 1965.0))
+    assert r["ops_per_launch"] == 16384 * 3072 * 24 * 5
+    assert r["peak"] == pytest.approx(128 * 148 * 1.965e9 / 1e12)
+    assert r["floor_us"] == pytest.approx(6039797760 / (128 * 148 * 1.965e9) * 1e6)
+    assert r["frac"] == pytest.approx(6039797760 / 550e-6 / 1e12 / r["peak"])
+    assert r["bound"] == "alu"
