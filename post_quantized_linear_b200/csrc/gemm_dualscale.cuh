@@ -1320,9 +1320,11 @@ __device__ __forceinline__ void epilogue_stacked(
 //     warp's shared-memory slot `sw_stage` (two buffers of 32 floats,
 //     alternating by group), from which every lane reads them back with
 //     broadcast 16-byte loads;
-//   * the accumulators are read eight columns at a time per polarity and
-//     re-seeded at once, so F(acc) is one exact subtraction (the seed's bits
-//     plus the integer sum are the float seed + acc);
+//   * the accumulators (seeded by the unit's first MMA) are read eight
+//     columns at a time per polarity, and the buffer goes back to the MMA as
+//     soon as its last columns are in registers; F(acc) is one exact
+//     subtraction (the seed's bits plus the integer sum are the float seed +
+//     acc);
 //   * the fold runs on fp32 pairs, five packed instructions per two outputs,
 //     in the fixed order t = fma(s-, F-, s+ * F+), y = fma(sw, t, y), y from 0.
 // After the tile's last group: + bias, convert, TMA store of the warp's
@@ -1337,7 +1339,6 @@ __device__ __forceinline__ void epilogue_groups_tma_store(
   static_assert(EPW == 16, "four parts of 32 columns per lane quarter");
   static_assert(SEED == 1 || SEED == 2, "seeded group units");
   constexpr uint32_t BUF_COLS = 2u * BN;
-  constexpr uint32_t seed_bits = (SEED == 1) ? kMagicW4Bits : kMagicBits;
   constexpr float seed_value = (SEED == 1) ? kMagicW4 : kMagic;
   constexpr float act_mult = (SEED == 2) ? 0.25f : 1.0f;   // Hadamard block normalization
   constexpr int ROWB = Y_BF16 ? 64 : 128;
@@ -1352,18 +1353,6 @@ __device__ __forceinline__ void epilogue_groups_tma_store(
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_base + 8u * (uint32_t)b);
   };
-  // Seed this warp's columns of both buffers, then hand the buffers to the MMA.
-#pragma unroll
-  for (int b = 0; b < NBUF; ++b) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t col = (uint32_t)b * BUF_COLS + (uint32_t)(c_lo + 16 * h);
-      tmem_st16(t_lane + col, seed_bits);
-      tmem_st16(t_lane + col + BN, seed_bits);
-    }
-  }
-  tmem_wait_st();
-  for (int b = 0; b < NBUF; ++b) release(b);
   int ug = 0;
   bool ok = true, pending = false;
   for (int it = 0; it < rounds && ok; ++it) {
@@ -1405,8 +1394,7 @@ __device__ __forceinline__ void epilogue_groups_tma_store(
           tmem_ld8(t_lane + col, ap);
           tmem_ld8(t_lane + col + BN, an);
           tmem_wait_ld();
-          tmem_st8(t_lane + col, seed_bits);
-          tmem_st8(t_lane + col + BN, seed_bits);
+          if (h == 3) release(b);   // the group's last columns are in registers
           const float4* s4 = reinterpret_cast<const float4*>(sw + 8 * h);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
@@ -1436,9 +1424,9 @@ __device__ __forceinline__ void epilogue_groups_tma_store(
             y2[4 * h + 2 * q + 1] = f2_fma(sw_hi, f2_fma(sn2, fn1, f2_mul(sp2, fp1)), y2[4 * h + 2 * q + 1]);
           }
         }
-        tmem_wait_st();
+      } else {
+        release(b);
       }
-      release(b);
       ++ug;
       if (u + 1 < G) {   // stage group u+1's scales (its buffer was last read in group u-1)
         sw_stage[((u + 1) & 1) * 32 + lane] = __half2float(h_next);

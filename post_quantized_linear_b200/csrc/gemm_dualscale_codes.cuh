@@ -26,12 +26,16 @@
 // the stage, two unpack warps widen it to int8 in the 128-byte-swizzled
 // layout beside it and signal a per-stage ready barrier that the MMA waits
 // on; every k block is its own unit, folded by the epilogue from seeded
-// accumulators (epilogue_tma_store, SEED 1).
+// accumulators (epilogue_groups_tma_store, SEED 1).  The seed is written by
+// the tensor core: each unit opens with one bf16 MMA, without the old
+// accumulator, of a ones column by a seed column (one 8-row swizzle atom
+// each, read for every row), which leaves the seed's fp32 bits in every
+// accumulator; the int8 MMAs add their int32 sums to those bits.
 // WM 2: int8 weight tiles with the units and fp16 scales of int4 groups -- the
 // int4 codes rotated by the block Hadamard matrix (HQ-DM, "Single Hadamard
 // Transformation", Spanish technical summary 2.1) -- folded from seeded
-// accumulators with the activation scales times the block normalization 1/4
-// (epilogue_tma_store, SEED 2).
+// accumulators the same way, with the activation scales times the block
+// normalization 1/4 (epilogue_groups_tma_store, SEED 2).
 #pragma once
 
 #include "gemm_dualscale.cuh"
@@ -119,6 +123,8 @@ struct CodesCfg {
   static constexpr int Y_BYTES = TMA_Y ? EPW * stage_y_bytes(Y_BF16) : 0;
   // group units: each epilogue warp's two 32-float buffers of widened weight scales
   static constexpr int SW_BYTES = (WM_ != 0) ? EPW * 2 * 32 * 4 : 0;
+  // group units: the seed MMA's operands, one 1024-byte swizzle atom each
+  static constexpr int SEED_BYTES = (WM_ != 0) ? 2048 : 0;
   // stacked (small M): three stages at most (deeper rings stream no faster);
   // at tiles of up to 64 columns a CTA of the next GEMM in the stream fits on
   // the SM beside this one (shared memory, TMEM and registers) and requests
@@ -126,8 +132,9 @@ struct CodesCfg {
   static constexpr int S_CAP = STK_ ? 3 : 8;
   // K split: [2P][BN] int32 (stacked) or [2][128][BN] (two-tile form)
   static constexpr int PART_BYTES = CSPLIT_ ? (STK_ ? 2 * STK_ : 2 * BM) * BN_ * 4 : 0;
-  static constexpr int S = ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) < S_CAP
-                               ? ((kStageBudget - Y_BYTES - SW_BYTES - PART_BYTES) / STAGE) : S_CAP;
+  static constexpr int S =
+      ((kStageBudget - Y_BYTES - SW_BYTES - SEED_BYTES - PART_BYTES) / STAGE) < S_CAP
+          ? ((kStageBudget - Y_BYTES - SW_BYTES - SEED_BYTES - PART_BYTES) / STAGE) : S_CAP;
   static_assert(!CSPLIT_ || STK_ != 0 || (!MULTI && !SINGLE && !LDA_ && WM_ == 0 && EPW_ == 4),
                 "K split over a cluster: stacked rows, or the two-tile form with four warps");
   static_assert(STK_ == 0 || ((STK_ == 16 || STK_ == 32 || STK_ == 64) && !MULTI && !SINGLE &&
@@ -140,7 +147,8 @@ struct CodesCfg {
   static constexpr int NBUF = CSPLIT_ ? 1 : ((2 * NACC * BN <= 512) ? 2 : 1);
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
-  static constexpr int OFF_PART = OFF_SW + SW_BYTES;
+  static constexpr int OFF_SEED = OFF_SW + SW_BYTES;
+  static constexpr int OFF_PART = OFF_SEED + SEED_BYTES;
   static constexpr int OFF_BAR = OFF_PART + PART_BYTES;
   // full, empty; tmem full/empty; drain; (W4) unpacked
   // (+ K split: the partial sums of the other CTAs have landed)
@@ -152,6 +160,7 @@ struct CodesCfg {
   static_assert(S >= 2 && TMEM_COLS <= 512 && SMEM_BYTES <= 232448, "budgets");
   static_assert(BN % 16 == 0 && BN <= 256, "UMMA N for M = 128");
   static_assert(OFF_Y % 1024 == 0 && stage_y_bytes(Y_BF16) % 1024 == 0, "staging alignment");
+  static_assert(OFF_SEED % 1024 == 0, "seed atoms: 128-byte swizzle alignment");
   // the MMA's 128-row read from the last k block's A start stays in the allocation
   static_assert(STK_ == 0 || S * STAGE - KB_BYTES + BM * BK <= OFF_MISC, "stacked A read");
 };
@@ -217,6 +226,20 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
   if constexpr (CSPLIT) {   // the partial-sum buffer starts at zero
     uint4* pb = reinterpret_cast<uint4*>(smem + C::OFF_PART);
     for (int i = threadIdx.x; i < C::PART_BYTES / 16; i += blockDim.x) pb[i] = make_uint4(0, 0, 0, 0);
+  }
+  if constexpr (SEEDED) {
+    // The seed MMA's operands, K-major in the 128-byte swizzle: A (first atom)
+    // holds bf16 1.0 and B (second atom) the seed in element 0 of each of its
+    // 8 rows -- row r's 16-byte chunk 0 sits at chunk r -- and zeros elsewhere.
+    // The seeds are exact in bf16 (their low 16 fp32 bits are zero).
+    constexpr uint32_t seed_bits = (WM == 1) ? kMagicW4Bits : kMagicBits;
+    static_assert((seed_bits & 0xFFFFu) == 0, "seed exact in bf16");
+    uint32_t* sw = reinterpret_cast<uint32_t*>(smem + C::OFF_SEED);
+    for (int i = threadIdx.x; i < 512; i += blockDim.x) {
+      const int byte = (i & 255) * 4, r = byte >> 7;
+      sw[i] = ((byte & 127) == r * 16) ? (i < 256 ? 0x3F80u : (seed_bits >> 16)) : 0u;
+    }
+    fence_proxy_async_smem();   // read by the tensor core (async proxy)
   }
   tc_fence_before();
   __syncthreads();
@@ -359,12 +382,15 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
             const int kb = kb0 + j;
             if (!unit_open) {   // a unit (K segment) may start inside a stage
               const int b = ug % C::NBUF;
-              // seeded buffers: the epilogue's first release (after seeding)
-              // completes phase 0, so every use waits one phase later
-              const uint32_t par = SEEDED ? ((ug / C::NBUF) & 1) : (((ug / C::NBUF) & 1) ^ 1);
+              const uint32_t par = ((ug / C::NBUF) & 1) ^ 1;
               if (!(ok = wait1(smem_u32(tmem_empty + b), par, abort_flag, budget))) break;
               tc_fence_after();
               d_pos = tmem_base + (uint32_t)(b * C::NACC * BN);
+              // group units: both accumulators set to the seed's bits (1 x seed, fp32)
+              if constexpr (SEEDED)
+                umma_bf16(d_pos, smem_desc_k_sw128_atom(smem_u32(smem + C::OFF_SEED)),
+                          smem_desc_k_sw128_atom(smem_u32(smem + C::OFF_SEED + 1024)),
+                          idesc_bf16(BM, C::NACC * BN), 0u);
             }
             const uint32_t a_p = smem_u32(smem + s * C::STAGE + j * C::KB_BYTES);
             const uint32_t a_n = a_p + BM * BK;
