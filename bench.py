@@ -66,7 +66,7 @@ NCU_TRAFFIC_BYTES = {
     ("mmdit_mlp_up", "codes"): 163565568 + 380856832,     # dualscale_gemm_codes_kernel
     ("dit_xl2_fc2_cfg", "codes"): 86029056 + 9071872,     # dualscale_gemm_codes_kernel
     ("seglinear_qkv", "codes"): 56157696 + 30311936,      # dualscale_gemm_codes_kernel
-    # ("w4a8", "codes"): recaptured after the seed moved into the tensor core
+    ("w4a8", "codes"): 105579776 + 67246080,              # dualscale_gemm_codes_kernel (int4)
 }
 
 
