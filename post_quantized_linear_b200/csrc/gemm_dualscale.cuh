@@ -889,7 +889,7 @@ __device__ __forceinline__ void unit_act_scales(const GemmArgs& a, int j, float&
 // counted on its `parts` barrier; rank 0 adds the buffer to its accumulators
 // (integer sums, any order) before folding.
 template <int BN, int NBUF, int EPW, int NACC, bool MULTI, bool Y_BF16, class TileFn,
-          bool PAIR = false, bool CSPLIT = false>
+          bool PAIR = false, bool CSPLIT = false, bool SPLIT = false>
 __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const CUtensorMap* tmap_y,
                                                    uint8_t* stage_y, int quad, int part, int lane,
                                                    uint32_t t_lane, uint64_t* tmem_full,
@@ -899,6 +899,8 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
                                                    uint32_t crank = 0, uint32_t part_buf = 0,
                                                    uint32_t parts_bar = 0) {
   static_assert(!CSPLIT || (!MULTI && NACC == 2 && EPW == 4 && !PAIR), "K split: two-tile form");
+  static_assert(!SPLIT || (BN == 256 && NBUF == 1 && EPW == 16 && NACC == 2 && !MULTI && !PAIR &&
+                           !CSPLIT), "buffer released in halves: one 256-wide DualScale buffer");
   auto pidx = [&](int a, int c) {
     return (uint32_t)(((128 * a + quad * 32 + lane) * BN) + ((c & ~31) | ((c & 31) ^ lane)));
   };
@@ -947,7 +949,13 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
     if (!tile_fn(it, t)) continue;
     const int c_lo = part * HALF;
     const int cols = min(HALF, t.width - c_lo);   // may be <= 0 on a narrow tail tile
-    if (cols > 0) {
+    if (SPLIT) {   // this warp's columns 32*part .. +32 and 128 + 32*part .. +32
+      const int c0 = 128 * lane + 32 * part;
+      if (lane < 2 && c0 < t.width) {
+        prefetch_l1(static_cast<const float*>(args.wscales) + t.n0 + c0);
+        if (args.bias != nullptr) prefetch_l1(args.bias + t.n0 + c0);
+      }
+    } else if (cols > 0) {
       for (int u = 0; u < (MULTI ? units : 1); ++u) {
         const float* sw_row = static_cast<const float*>(args.wscales) + (int64_t)u * args.N + t.n0 + c_lo;
         for (int c = lane * 32; c < cols; c += 32 * 32) prefetch_l1(sw_row + c);
@@ -1013,8 +1021,14 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
       tc_fence_after();
       float sp, sn;
       unit_act_scales(args, 0, sp, sn);
-      for (int p = 0; p < npass; ++p) {
-        const int col = c_lo + p * 32;
+      // SPLIT: pass p covers tile columns 128p + 32*part .. +32, so every warp
+      // reads the buffer's first half (both accumulators' columns 0 .. 127)
+      // before the second, and hands each half back to the MMA on its own
+      // barrier (tmem_empty[1]: first half; tmem_empty[0]: the whole buffer).
+      const int np = SPLIT ? (32 * part < t.width ? 1 : 0) + (128 + 32 * part < t.width ? 1 : 0)
+                           : npass;
+      for (int p = 0; p < np; ++p) {
+        const int col = SPLIT ? 128 * p + 32 * part : c_lo + p * 32;
         if (pending) {   // the previous store has read the staging tile
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
@@ -1027,7 +1041,14 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
             load8(b, cc, ap, an);
             load8(b, cc + 8, bp, bn);
             tmem_wait_ld();
-            if (p == npass - 1 && (h == 1 || cc + 16 >= t.width)) release(b);   // last loads
+            if (h == 1 || cc + 16 >= t.width) {   // the pass's last loads
+              if constexpr (SPLIT) {
+                if (p == 0) release(1);
+                if (p == np - 1) release(0);
+              } else if (p == npass - 1) {
+                release(b);
+              }
+            }
             if constexpr (CSPLIT) {
               uint32_t* pb = reinterpret_cast<uint32_t*>(__cvta_shared_to_generic(part_buf));
               if (crank != 0) {   // into this CTA's buffer; rank 0 folds
@@ -1087,7 +1108,14 @@ __device__ __forceinline__ void epilogue_tma_store(const GemmArgs& args, const C
         }
         pending = true;
       }
-      if (npass == 0) release(b);
+      if constexpr (SPLIT) {
+        if (np == 0) {
+          release(1);
+          release(0);
+        }
+      } else if (npass == 0) {
+        release(b);
+      }
       ++ug;
     }
   }

@@ -145,6 +145,16 @@ struct CodesCfg {
                 "group units: DualScale, one k block per stage, BN = 128");
   // TMEM accumulator buffers (K split: one tile per CTA, one buffer)
   static constexpr int NBUF = CSPLIT_ ? 1 : ((2 * NACC * BN <= 512) ? 2 : 1);
+  // One 256-wide DualScale buffer (both accumulators fill TMEM): the epilogue
+  // hands it back in halves, and each tile's first SPLIT_KB k blocks are multiplied
+  // into the first half (the first 128 columns of both accumulators) while
+  // the previous tile's second half drains, then into the second.
+  static constexpr bool SPLIT_DRAIN = BN_ == 256 && NBUF == 1 && NACC == 2 && !MULTI && !SINGLE &&
+                                      !LDA_ && KPS_ == 1 && WM_ == 0 && STK_ == 0 && !CSPLIT_ &&
+                                      EPW_ == 16 && TMA_Y;   // (the epilogue that releases halves)
+  // k blocks multiplied half by half at a tile's start (the rest of the ring
+  // keeps loading meanwhile)
+  static constexpr int SPLIT_KB = 1;
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
   static constexpr int OFF_SEED = OFF_SW + SW_BYTES;
@@ -203,7 +213,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
       mbar_init(smem_u32(full + i), C::FULL_COUNT);
       mbar_init(smem_u32(empty + i), 1);
     }
-    for (int i = 0; i < C::NBUF; ++i) {
+    // (SPLIT_DRAIN: tmem_empty[1] is the first half of the one buffer)
+    for (int i = 0; i < (C::SPLIT_DRAIN ? 2 : C::NBUF); ++i) {
       mbar_init(smem_u32(tmem_full + i), 1);
       mbar_init(smem_u32(tmem_empty + i), C::EPW);
     }
@@ -368,6 +379,63 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
         Tile t;
         if (!tiles(it, t)) continue;
         const uint32_t idesc = idesc_i8(BM, t.width);
+        if constexpr (C::SPLIT_DRAIN) {
+          // k blocks [kb_lo, kb_lo + P) into the first half as soon as it is
+          // free, then into the second half once the whole buffer is; the
+          // rest at full width.  Their stages are released after both halves.
+          const int P = min(min(C::SPLIT_KB, C::S), kb_hi - kb_lo);
+          const uint32_t par = (ug & 1) ^ 1;
+          const uint32_t d = tmem_base;
+          const int w1 = t.width - 128;                      // second half's columns
+          auto half = [&](int q, int col, uint32_t hdesc) {
+            const int s = (c + q) % C::S;
+            const uint32_t a_p = smem_u32(smem + s * C::STAGE);
+            const uint32_t a_n = a_p + BM * BK;
+            const uint32_t b_w = a_p + C::A_BYTES + (uint32_t)col * BK;   // weight rows col ..
+#pragma unroll
+            for (int ks = 0; ks < BK / 32; ++ks) {
+              const uint32_t acc = (q > 0 || ks > 0) ? 1u : 0u;
+              const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
+              umma_i8(d + (uint32_t)col, smem_desc_k_sw128(a_p + ks * 32), bd, hdesc, acc);
+              umma_i8(d + BN + (uint32_t)col, smem_desc_k_sw128(a_n + ks * 32), bd, hdesc, acc);
+            }
+          };
+          if (!(ok = wait1(smem_u32(tmem_empty + 1), par, abort_flag, budget))) break;
+          tc_fence_after();
+          for (int q = 0; q < P; ++q) {
+            if (!(ok = wait1(smem_u32(full + (c + q) % C::S), ((c + q) / C::S) & 1, abort_flag,
+                             budget)))
+              break;
+            half(q, 0, idesc_i8(BM, min(t.width, 128)));
+          }
+          if (!ok) break;
+          if (!(ok = wait1(smem_u32(tmem_empty), par, abort_flag, budget))) break;
+          tc_fence_after();
+          for (int q = 0; q < P; ++q) {
+            if (w1 > 0) half(q, 128, idesc_i8(BM, w1));
+            umma_commit(smem_u32(empty + (c + q) % C::S));
+          }
+          c += P;
+          for (int kb = kb_lo + P; kb < kb_hi; ++kb) {
+            const int s = c % C::S;
+            if (!(ok = wait1(smem_u32(full + s), (c / C::S) & 1, abort_flag, budget))) break;
+            const uint32_t a_p = smem_u32(smem + s * C::STAGE);
+            const uint32_t a_n = a_p + BM * BK;
+            const uint32_t b_w = a_p + C::A_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < BK / 32; ++ks) {
+              const uint64_t bd = smem_desc_k_sw128(b_w + ks * 32);
+              umma_i8(d, smem_desc_k_sw128(a_p + ks * 32), bd, idesc, 1u);
+              umma_i8(d + BN, smem_desc_k_sw128(a_n + ks * 32), bd, idesc, 1u);
+            }
+            umma_commit(smem_u32(empty + s));
+            ++c;
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(tmem_full));
+          ++ug;
+          continue;
+        }
         bool unit_open = false;
         uint32_t d_pos = 0;
         for (int kb0 = kb_lo; kb0 < kb_hi && ok; kb0 += KPS) {
@@ -512,7 +580,8 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
           smem_u32(tmem_empty), rounds, tiles, abort_flag, budget);
     } else if constexpr (C::TMA_Y) {
       uint8_t* stage_y = smem + C::OFF_Y + (warp - EPI0) * stage_y_bytes(Y_BF16);
-      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, decltype(tiles), false, CSPLIT>(
+      epilogue_tma_store<BN, C::NBUF, C::EPW, C::NACC, MULTI, Y_BF16, decltype(tiles), false, CSPLIT,
+                         C::SPLIT_DRAIN>(
           args, &tmap_y, stage_y, quad, part, lane, t_lane, tmem_full, smem_u32(tmem_empty), rounds,
           tiles, abort_flag, budget, 0, false, crank, smem_u32(smem + C::OFF_PART), smem_u32(parts));
     } else {
