@@ -63,8 +63,8 @@ MMA_I8_OPS_PER_CLK_SM = 16384
 # capture of the current kernel build (profiles/*.md); keyed by (workload,
 # path).  Absent: no capture of the current build.
 NCU_TRAFFIC_BYTES = {
-    ("mmdit_mlp_up", "codes"): 163565568 + 380856832,     # dualscale_gemm_codes_kernel
-    ("dit_xl2_fc2_cfg", "codes"): 86029056 + 9071872,     # dualscale_gemm_codes_kernel
+    ("mmdit_mlp_up", "codes"): 161485056 + 381627392,     # dualscale_gemm_codes_kernel
+    ("dit_xl2_fc2_cfg", "codes"): 91399680 + 11276032,    # dualscale_gemm_codes_kernel
     ("seglinear_qkv", "codes"): 56157696 + 30311936,      # dualscale_gemm_codes_kernel
     ("w4a8", "codes"): 105579776 + 67246080,              # dualscale_gemm_codes_kernel (int4)
 }
