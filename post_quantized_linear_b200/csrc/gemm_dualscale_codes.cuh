@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(codes_threads(EPW, LDA, WM == 1), 1)
         Tile t;
         if (!tiles(it, t)) continue;
         const uint32_t idesc = idesc_i8(BM, t.width);
-        if constexpr (C::SPLIT_DRAIN) {
+        if constexpr (C::SPLIT_DRAIN && C::SPLIT_KB > 0) {
           // k blocks [kb_lo, kb_lo + P) into the first half as soon as it is
           // free, then into the second half once the whole buffer is; the
           // rest at full width.  Their stages are released after both halves.
