@@ -112,6 +112,23 @@ def test_tile_width_variants_match_oracle(bn, codes, monkeypatch, dev_lib):
     c.compare_rows(y, np.arange(wl.M))
 
 
+@pytest.mark.parametrize("N", [304, 336])
+def test_narrow_tail_of_the_halved_buffer(N, monkeypatch, dev_lib):
+    """BN = 256 from codes, where the one TMEM buffer goes back to the MMA in
+    halves: a last tile column of 48 or 80 columns leaves some epilogue warps
+    without columns (they hand both halves back at once) and the MMA fills
+    only the first half; every row against the oracle."""
+    import post_quantized_linear_b200 as pq
+    monkeypatch.setenv("SEGQUANT_BN", "256")
+    wl = W.small_case(390, 768, N, seed=23, out="bf16")
+    c = Case(wl)
+    qp, qn = pq.quantize_activations(c.x, wl.kseg, c.sp, c.sn)
+    y = pq.linear_from_codes(qp, qn, c.qw, c.sp, c.sn, c.b)
+    torch.cuda.synchronize()
+    assert pq.stream_status() == 0
+    c.compare_rows(y, np.arange(wl.M))
+
+
 @pytest.mark.parametrize("bn", ["128", "192", "256"])
 @pytest.mark.parametrize("i", [0, 1, 2, 5])
 def test_codes_kernels_one_ring_and_two_rings_agree(i, bn, monkeypatch, dev_lib):
