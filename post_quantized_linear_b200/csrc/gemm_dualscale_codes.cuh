@@ -146,14 +146,16 @@ struct CodesCfg {
   // TMEM accumulator buffers (K split: one tile per CTA, one buffer)
   static constexpr int NBUF = CSPLIT_ ? 1 : ((2 * NACC * BN <= 512) ? 2 : 1);
   // One 256-wide DualScale buffer (both accumulators fill TMEM): the epilogue
-  // hands it back in halves, and each tile's first SPLIT_KB k blocks are multiplied
-  // into the first half (the first 128 columns of both accumulators) while
-  // the previous tile's second half drains, then into the second.
+  // hands it back in halves, and each tile's first SPLIT_KB k blocks are
+  // multiplied into the first half (the first 128 columns of both
+  // accumulators) while the previous tile's second half drains, then into
+  // the second.
   static constexpr bool SPLIT_DRAIN = BN_ == 256 && NBUF == 1 && NACC == 2 && !MULTI && !SINGLE &&
                                       !LDA_ && KPS_ == 1 && WM_ == 0 && STK_ == 0 && !CSPLIT_ &&
                                       EPW_ == 16 && TMA_Y;   // (the epilogue that releases halves)
   // k blocks multiplied half by half at a tile's start (the rest of the ring
-  // keeps loading meanwhile)
+  // keeps loading meanwhile; two or three held their stages through the
+  // drain and measured slower)
   static constexpr int SPLIT_KB = 1;
   static constexpr int OFF_Y = S * STAGE;
   static constexpr int OFF_SW = OFF_Y + Y_BYTES;
